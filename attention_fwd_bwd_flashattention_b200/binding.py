@@ -1,0 +1,213 @@
+"""Thin ctypes binding of the C ABI in include/relpos_attn.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory and the current stream.  If the
+compiled library is missing this module raises; there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+T5, SHAW, TXL, DEBERTA = 0, 1, 2, 3
+F32, BF16 = 0, 1
+PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "librelpos_attn.so")
+_lib = None
+
+
+class RelposError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+        self.code = code
+
+
+class relpos_params_t(ctypes.Structure):
+    _fields_ = [
+        ("mech", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("kernel_path", ctypes.c_int32),
+        ("B", ctypes.c_int64),
+        ("H", ctypes.c_int64),
+        ("L", ctypes.c_int64),
+        ("d", ctypes.c_int64),
+        ("scale", ctypes.c_float),
+        ("t5_num_buckets", ctypes.c_int32),
+        ("t5_max_distance", ctypes.c_int32),
+        ("t5_bidirectional", ctypes.c_int32),
+        ("shaw_clip", ctypes.c_int32),
+        ("deberta_span", ctypes.c_int32),
+    ]
+
+
+EXPORTS = ("relpos_attn_workspace_size", "relpos_attn_fwd", "relpos_attn_bwd", "relpos_attn_resolved_path",
+           "relpos_strerror", "relpos_attn_version")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load the compiled library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {_LIB_PATH} (run python -m attention_fwd_bwd_flashattention_b200.build)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.POINTER(relpos_params_t)
+    vp = ctypes.c_void_p
+    lib.relpos_attn_workspace_size.argtypes = [P, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+    lib.relpos_attn_workspace_size.restype = ctypes.c_int
+    lib.relpos_attn_fwd.argtypes = [P, vp, vp, vp, ctypes.POINTER(vp), vp, vp, vp, ctypes.c_size_t, vp, vp]
+    lib.relpos_attn_fwd.restype = ctypes.c_int
+    lib.relpos_attn_bwd.argtypes = [P, vp, vp, vp, ctypes.POINTER(vp), vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp), vp,
+                                    ctypes.c_size_t, vp, vp]
+    lib.relpos_attn_bwd.restype = ctypes.c_int
+    lib.relpos_attn_resolved_path.argtypes = [P]
+    lib.relpos_attn_resolved_path.restype = ctypes.c_int
+    lib.relpos_strerror.argtypes = [ctypes.c_int]
+    lib.relpos_strerror.restype = ctypes.c_char_p
+    lib.relpos_attn_version.argtypes = []
+    lib.relpos_attn_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load().relpos_strerror(int(code)).decode()
+
+
+@dataclass
+class Params:
+    mech: int
+    B: int
+    H: int
+    L: int
+    d: int = 64
+    dtype: int = BF16
+    causal: bool = False
+    scale: Optional[float] = None
+    kernel_path: int = PATH_AUTO
+    t5_num_buckets: int = 32
+    t5_max_distance: int = 128
+    t5_bidirectional: bool = True
+    shaw_clip: int = 64
+    deberta_span: int = 256
+
+    def c(self) -> relpos_params_t:
+        scale = self.scale
+        if scale is None:
+            scale = 1.0 / math.sqrt(3 * self.d) if self.mech == DEBERTA else 1.0 / math.sqrt(self.d)
+        return relpos_params_t(self.mech, self.dtype, int(self.causal), self.kernel_path, self.B, self.H, self.L, self.d,
+                               float(scale), self.t5_num_buckets, self.t5_max_distance, int(self.t5_bidirectional),
+                               self.shaw_clip, self.deberta_span)
+
+    def n_rel(self) -> int:
+        return {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2}[self.mech]
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
+    arr = (ctypes.c_void_p * 3)()
+    for i in range(3):
+        arr[i] = _ptr(ts[i]) if i < len(ts) else None
+    return arr
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# one-to-one wrappers of the C entry points
+# ---------------------------------------------------------------------------
+def relpos_attn_workspace_size(params: Params, pass_: int) -> int:
+    n = ctypes.c_size_t(0)
+    cp = params.c()
+    rc = load().relpos_attn_workspace_size(ctypes.byref(cp), int(pass_), ctypes.byref(n))
+    if rc != 0:
+        raise RelposError(rc, "relpos_attn_workspace_size")
+    return int(n.value)
+
+
+def relpos_attn_resolved_path(params: Params) -> int:
+    cp = params.c()
+    rc = load().relpos_attn_resolved_path(ctypes.byref(cp))
+    if rc < 0:
+        raise RelposError(rc, "relpos_attn_resolved_path")
+    return rc
+
+
+def tc_available(params: Params) -> bool:
+    """True when these params run on the tensor-core (tcgen05) kernels."""
+    return relpos_attn_resolved_path(params) == PATH_TC
+
+
+def relpos_attn_fwd(params: Params, q, k, v, rel, o, lse, workspace, dev_status=None, stream=None) -> None:
+    cp = params.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().relpos_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o), _ptr(lse),
+                                _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    if rc != 0:
+        raise RelposError(rc, "relpos_attn_fwd")
+
+
+def relpos_attn_bwd(params: Params, q, k, v, rel, o, lse, dout, dq, dk, dv, drel, workspace, dev_status=None,
+                    stream=None) -> None:
+    cp = params.c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().relpos_attn_bwd(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o), _ptr(lse),
+                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr_array(drel), _ptr(workspace), ws_bytes,
+                                _ptr(dev_status), _stream(stream))
+    if rc != 0:
+        raise RelposError(rc, "relpos_attn_bwd")
+
+
+# ---------------------------------------------------------------------------
+# convenience: allocate outputs / workspace with torch and call the C entry points
+# ---------------------------------------------------------------------------
+def params_for(mech, q: torch.Tensor, causal: bool, scale=None, kernel_path=PATH_AUTO, **cfg) -> Params:
+    B, H, L, d = q.shape
+    dt = BF16 if q.dtype == torch.bfloat16 else F32
+    return Params(mech=mech, B=B, H=H, L=L, d=d, dtype=dt, causal=causal, scale=scale, kernel_path=kernel_path, **cfg)
+
+
+def workspace(params: Params, pass_: int, device) -> Optional[torch.Tensor]:
+    n = relpos_attn_workspace_size(params, pass_)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def forward(params: Params, q, k, v, rel, ws=None, stream=None):
+    """Returns (O, LSE)."""
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(params, 0, q.device)
+    relpos_attn_fwd(params, q, k, v, rel, o, lse, ws, stream=stream)
+    return o, lse
+
+
+def backward(params: Params, q, k, v, rel, o, lse, dout, ws=None, stream=None):
+    """Returns (dQ, dK, dV, [drel...]) with drel float32, shaped like rel."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    drel = [torch.empty(r.shape, dtype=torch.float32, device=q.device) for r in rel[: params.n_rel()]]
+    if ws is None:
+        ws = workspace(params, 1, q.device)
+    relpos_attn_bwd(params, q, k, v, rel, o, lse, dout, dq, dk, dv, drel, ws, stream=stream)
+    return dq, dk, dv, drel

@@ -1,0 +1,292 @@
+// C ABI of the relative-position attention library: argument validation,
+// workspace layout and dispatch to the kernels.  Declared in relpos_attn.h.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "relpos_attn.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+using rp::Prm;
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
+constexpr int kMaxL = 1 << 20;
+
+// ---- exact T5 thresholds -------------------------------------------------
+// Little-endian base-2^32 big integers, just enough for a^x * b^y comparisons.
+typedef std::vector<uint32_t> Big;
+static void big_mul(Big &x, uint32_t m) {
+  uint64_t carry = 0;
+  for (auto &d : x) {
+    uint64_t t = (uint64_t)d * m + carry;
+    d = (uint32_t)t;
+    carry = t >> 32;
+  }
+  if (carry) x.push_back((uint32_t)carry);
+}
+static Big big_powmul(uint32_t a, int ea, uint32_t b, int eb) {
+  Big x(1, 1u);
+  for (int i = 0; i < ea; ++i) big_mul(x, a);
+  for (int i = 0; i < eb; ++i) big_mul(x, b);
+  while (x.size() > 1 && x.back() == 0) x.pop_back();
+  return x;
+}
+static int big_cmp(const Big &x, const Big &y) {
+  if (x.size() != y.size()) return x.size() < y.size() ? -1 : 1;
+  for (size_t i = x.size(); i-- > 0;)
+    if (x[i] != y[i]) return x[i] < y[i] ? -1 : 1;
+  return 0;
+}
+// Is bucket offset t reached at distance a?  (a/me)^span >= (md/me)^t
+static bool t5_reached(uint32_t a, int t, uint32_t me, uint32_t md, int span) {
+  return big_cmp(big_powmul(a, span, me, t), big_powmul(me, span, md, t)) >= 0;
+}
+
+static int fill_t5(const relpos_params_t *P, Prm &p) {
+  const int nb = P->t5_num_buckets, md = P->t5_max_distance;
+  const int bidir = P->t5_bidirectional ? 1 : 0;
+  if (nb < 2 || nb > 64 || (bidir && nb < 4)) return RELPOS_ERR_INVALID_ARG;
+  p.nb = nb;
+  p.bidir = bidir;
+  p.half = bidir ? nb / 2 : nb;
+  p.me = p.half / 2;
+  if (p.me < 1 || md <= p.me) return RELPOS_ERR_INVALID_ARG;
+  const int span = p.half - p.me;
+  p.nthr = span - 1;
+  if (p.nthr > 32) return RELPOS_ERR_INVALID_ARG;
+  for (int t = 1; t <= p.nthr; ++t) {
+    // smallest a in [me, md] with bucket offset >= t (monotone in a)
+    uint32_t lo = (uint32_t)p.me, hi = (uint32_t)md;
+    while (lo < hi) {
+      uint32_t mid = lo + (hi - lo) / 2;
+      if (t5_reached(mid, t, (uint32_t)p.me, (uint32_t)md, span))
+        hi = mid;
+      else
+        lo = mid + 1;
+    }
+    p.thr[t - 1] = (int)lo;
+  }
+  return RELPOS_OK;
+}
+
+static int validate_and_fill(const relpos_params_t *P, Prm &p) {
+  if (!P) return RELPOS_ERR_INVALID_ARG;
+  memset(&p, 0, sizeof(p));
+  if (P->mech < RELPOS_T5 || P->mech > RELPOS_DEBERTA) return RELPOS_ERR_INVALID_ARG;
+  if (P->dtype != RELPOS_F32 && P->dtype != RELPOS_BF16) return RELPOS_ERR_INVALID_ARG;
+  if (P->causal != 0 && P->causal != 1) return RELPOS_ERR_INVALID_ARG;
+  if (P->kernel_path < RELPOS_PATH_AUTO || P->kernel_path > RELPOS_PATH_TC) return RELPOS_ERR_INVALID_ARG;
+  if (P->d != rp::HD) return RELPOS_ERR_INVALID_ARG;
+  if (P->B < 1 || P->H < 1 || P->L < 1 || P->L > kMaxL || P->B * P->H > 65535) return RELPOS_ERR_INVALID_ARG;
+  if (!isfinite(P->scale)) return RELPOS_ERR_INVALID_ARG;
+  p.mech = P->mech;
+  p.causal = P->causal;
+  p.B = (int)P->B;
+  p.H = (int)P->H;
+  p.L = (int)P->L;
+  p.scale = P->scale;
+  p.nT = (p.L + kTile - 1) / kTile;
+  switch (P->mech) {
+    case RELPOS_T5: {
+      int e = fill_t5(P, p);
+      if (e) return e;
+      p.nrows = p.nb;
+      break;
+    }
+    case RELPOS_SHAW:
+      if (P->shaw_clip < 0 || P->shaw_clip > 4096) return RELPOS_ERR_INVALID_ARG;
+      p.clip = P->shaw_clip;
+      p.nrows = 2 * p.clip + 1;
+      break;
+    case RELPOS_TXL:
+      p.nrows = p.causal ? p.L : 2 * p.L - 1;
+      p.off = p.causal ? 0 : p.L - 1;
+      break;
+    default:
+      if (P->deberta_span < 1 || P->deberta_span > 4096) return RELPOS_ERR_INVALID_ARG;
+      p.span = P->deberta_span;
+      p.nrows = 2 * p.span;
+      break;
+  }
+  if (p.mech == rp::M_TXL) {
+    p.nbands = p.causal ? p.nT : 2 * p.nT - 1;
+    long long cap = 4000 / ((long long)p.B * p.H * p.nbands);
+    int nch = (int)((p.nT + 7) / 8);
+    if (cap < nch) nch = (int)(cap < 1 ? 1 : cap);
+    p.diag_ch = (p.nT + nch - 1) / nch;
+    p.diag_nchunk = (p.nT + p.diag_ch - 1) / p.diag_ch;
+  }
+  return RELPOS_OK;
+}
+
+static bool use_tc(const relpos_params_t *P) {
+  (void)P;
+  return false;
+}
+
+// ---- workspace layout ------------------------------------------------------
+struct Layout {
+  size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot, total;
+};
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static Layout layout_of(const Prm &p, int pass) {
+  Layout l;
+  memset(&l, 0, sizeof(l));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  const size_t BH = (size_t)p.B * p.H;
+  if (p.mech == rp::M_T5) {
+    l.t5_bias = take(sizeof(float) * (size_t)p.H * (2 * (size_t)p.L - 1));
+    l.t5_bkt = take(sizeof(int) * (2 * (size_t)p.L - 1));
+  }
+  if (pass == 1) {
+    l.dvec = take(sizeof(float) * BH * p.L);
+    const size_t tab = (size_t)p.nrows * rp::HD;
+    switch (p.mech) {
+      case rp::M_T5: l.part_small = take(sizeof(float) * BH * p.nT * p.nb); break;
+      case rp::M_SHAW: l.part_row = take(sizeof(float) * BH * p.nT * tab); break;
+      case rp::M_DEB:
+        l.part_row = take(sizeof(float) * BH * p.nT * tab);
+        l.part_col = take(sizeof(float) * BH * p.nT * tab);
+        break;
+      default:
+        l.part_small = take(sizeof(float) * BH * p.nT * rp::HD);
+        l.part_diag = take(sizeof(float) * BH * p.nbands * p.diag_nchunk * 128 * (rp::HD + 1));
+        l.gtot = take(sizeof(float) * (size_t)p.H * p.nrows);
+        break;
+    }
+  }
+  l.total = off;
+  return l;
+}
+
+static void bind_workspace(Prm &p, const Layout &l, void *ws) {
+  char *b = (char *)ws;
+  if (p.mech == rp::M_T5) {
+    p.t5_bias = (float *)(b + l.t5_bias);
+    p.t5_bkt = (int *)(b + l.t5_bkt);
+  }
+  p.Dvec = (float *)(b + l.dvec);
+  p.part_row = (float *)(b + l.part_row);
+  p.part_col = (float *)(b + l.part_col);
+  p.part_small = (float *)(b + l.part_small);
+  p.part_diag = (float *)(b + l.part_diag);
+  p.gtot = (float *)(b + l.gtot);
+}
+
+static int rel_count(int mech) { return mech == rp::M_TXL ? 3 : (mech == rp::M_DEB ? 2 : 1); }
+
+static int to_status(cudaError_t e) {
+  if (e == cudaSuccess) return RELPOS_OK;
+  cudaGetLastError();  // clear a sticky launch-configuration error
+  return RELPOS_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" int relpos_attn_workspace_size(const relpos_params_t *params, int pass, size_t *bytes) {
+  Prm p;
+  if (!bytes || (pass != 0 && pass != 1)) return RELPOS_ERR_INVALID_ARG;
+  int e = validate_and_fill(params, p);
+  if (e) return e;
+  *bytes = layout_of(p, pass).total;
+  return RELPOS_OK;
+}
+
+extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, const void *k, const void *v,
+                               const void *const rel[3], void *o, float *lse, void *workspace,
+                               size_t workspace_bytes, int32_t *dev_status, void *stream) {
+  Prm p;
+  int e = validate_and_fill(params, p);
+  if (e) return e;
+  if (!q || !k || !v || !rel || !o || !lse) return RELPOS_ERR_INVALID_ARG;
+  for (int i = 0; i < rel_count(p.mech); ++i)
+    if (!rel[i]) return RELPOS_ERR_INVALID_ARG;
+  if (params->kernel_path == RELPOS_PATH_TC && !use_tc(params)) return RELPOS_ERR_UNSUPPORTED;
+  const Layout l = layout_of(p, 0);
+  if (l.total > 0 && (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255))) return RELPOS_ERR_WORKSPACE;
+  bind_workspace(p, l, workspace);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.rel0 = rel[0];
+  p.rel1 = rel_count(p.mech) > 1 ? rel[1] : nullptr;
+  p.rel2 = rel_count(p.mech) > 2 ? rel[2] : nullptr;
+  p.out = o;
+  p.lse = lse;
+  p.status = dev_status;
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool bf16 = params->dtype == RELPOS_BF16;
+  if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
+  return to_status(rp::simt_fwd(p, bf16, st));
+}
+
+extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, const void *k, const void *v,
+                               const void *const rel[3], const void *o, const float *lse, const void *dout,
+                               void *dq, void *dk, void *dv, float *const drel[3], void *workspace,
+                               size_t workspace_bytes, int32_t *dev_status, void *stream) {
+  Prm p;
+  int e = validate_and_fill(params, p);
+  if (e) return e;
+  if (!q || !k || !v || !rel || !o || !lse || !dout || !dq || !dk || !dv || !drel) return RELPOS_ERR_INVALID_ARG;
+  for (int i = 0; i < rel_count(p.mech); ++i)
+    if (!rel[i] || !drel[i]) return RELPOS_ERR_INVALID_ARG;
+  if (params->kernel_path == RELPOS_PATH_TC && !use_tc(params)) return RELPOS_ERR_UNSUPPORTED;
+  const Layout l = layout_of(p, 1);
+  if (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255)) return RELPOS_ERR_WORKSPACE;
+  bind_workspace(p, l, workspace);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.rel0 = rel[0];
+  p.rel1 = rel_count(p.mech) > 1 ? rel[1] : nullptr;
+  p.rel2 = rel_count(p.mech) > 2 ? rel[2] : nullptr;
+  p.lse = (float *)lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.drel0 = drel[0];
+  p.drel1 = rel_count(p.mech) > 1 ? drel[1] : nullptr;
+  p.drel2 = rel_count(p.mech) > 2 ? drel[2] : nullptr;
+  p.status = dev_status;
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool bf16 = params->dtype == RELPOS_BF16;
+  if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
+  return to_status(rp::simt_bwd(p, bf16, st));
+}
+
+extern "C" int relpos_attn_resolved_path(const relpos_params_t *params) {
+  Prm p;
+  int e = validate_and_fill(params, p);
+  if (e) return e;
+  if (params->kernel_path == RELPOS_PATH_TC && !use_tc(params)) return RELPOS_ERR_UNSUPPORTED;
+  return use_tc(params) ? RELPOS_PATH_TC : RELPOS_PATH_SIMT;
+}
+
+extern "C" const char *relpos_strerror(int status) {
+  switch (status) {
+    case RELPOS_OK: return "ok";
+    case RELPOS_ERR_INVALID_ARG: return "invalid argument";
+    case RELPOS_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case RELPOS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RELPOS_ERR_LAUNCH: return "kernel launch failed";
+    case RELPOS_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case RELPOS_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int relpos_attn_version(void) { return kVersion; }

@@ -38,6 +38,7 @@ class Workload:
     d: int = 64
     t5_num_buckets: int = 32
     t5_max_distance: int = 128
+    t5_bidirectional: bool = True
     shaw_clip: int = 64
     deberta_span: int = 256
 

@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of relative-position attention, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = relpos_attn_fwd + relpos_attn_bwd of the whole workload (default:
+Transformer-XL, causal, B=1, H=8, L=8192, d=64, bf16) on inputs already resident
+in HBM.  The L2 cache (126 MB) is flushed by writing a 256 MB buffer before every
+timed step (outside the timed interval); each step is timed with CUDA events on
+the launching stream, and the reported time is the max over ranks.  With N > 1
+(torchrun) every rank runs its own batch of the workload (weak scaling) and the
+relative-table gradients, shared by all ranks, are summed with one NCCL
+all-reduce, as in data-parallel training.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
+(test infrastructure, the only reference there is) on a bounded sample of the
+same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from attention_fwd_bwd_flashattention_b200 import binding as bd  # noqa: E402
+from attention_fwd_bwd_flashattention_b200 import dist as rdist  # noqa: E402
+from attention_fwd_bwd_flashattention_b200.inputs import DEBERTA, SHAW, T5, TXL, WORKLOADS, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "txl_causal_L8192_bf16"
+METRIC = "fwd+bwd TFLOP/s and tokens/s at L=8192, % of B200 BF16 tensor peak"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic FLOPs (distinct products the method must compute; recompute and
+# window duplication are not credited)
+# ----------------------------------------------------------------------------
+def algo_flops(wl):
+    pairs = wl.L * (wl.L + 1) // 2 if wl.causal else wl.L * wl.L
+    U = 2.0 * wl.B * wl.H * wl.d * pairs
+
+    def R(rows):
+        return 2.0 * wl.B * wl.H * wl.L * rows * wl.d
+
+    if wl.mech == T5:
+        return 2 * U, 5 * U
+    if wl.mech == SHAW:
+        r = R(2 * wl.shaw_clip + 1)
+        return 2 * U + r, 5 * U + 3 * r
+    if wl.mech == TXL:
+        return 3 * U, 8 * U
+    r = R(2 * wl.deberta_span)
+    return 2 * U + 2 * r, 5 * U + 6 * r
+
+
+def fa_flops(wl):
+    pairs = wl.L * (wl.L + 1) // 2 if wl.causal else wl.L * wl.L
+    return 4.0 * pairs * wl.d * wl.B * wl.H, 10.0 * pairs * wl.d * wl.B * wl.H
+
+
+def kernel_launches(wl, path):
+    """Kernels this library launches per forward and per backward call."""
+    t5 = 1 if wl.mech == T5 else 0
+    if path == "simt":
+        fwd = 1 + t5
+        bwd = {T5: 5, SHAW: 4, TXL: 6, DEBERTA: 5}[wl.mech] + t5
+        return fwd, bwd
+    return 1 + t5, {T5: 5, SHAW: 4, TXL: 6, DEBERTA: 5}[wl.mech] + t5
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (baseline only)
+# ----------------------------------------------------------------------------
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(wl, rows_fraction=None):
+    """Time the fp64 oracle on one (batch 0, head 0) slice of the workload.
+    rows_fraction: only that fraction of query rows (forward rows + their dQ),
+    else the whole head forward + backward.  Returns (seconds, flops, sample)."""
+    import numpy as np
+
+    import oracle as orc
+    from attention_fwd_bwd_flashattention_b200.inputs import to_f64
+
+    one = wl.with_(B=1, H=1)
+    inp = make_inputs(one, 0)
+    q, k, v, do = (to_f64(inp[n]) for n in ("q", "k", "v", "do"))
+    rel = [to_f64(r) for r in inp["rel"]]
+    cfg = orc.RelCfg(t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance, shaw_clip=wl.shaw_clip,
+                     deberta_span=wl.deberta_span)
+    f_fwd, f_bwd = algo_flops(one)
+    t0 = time.perf_counter()
+    if rows_fraction is None:
+        orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg)
+        orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg)
+        flops = f_fwd + f_bwd
+        sample = f"1 of {wl.B * wl.H} (batch, head) slices at full L={wl.L}, forward + backward"
+    else:
+        step = max(1, int(round(1 / rows_fraction)))
+        rows = np.arange(0, wl.L, step)
+        orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, rows=rows)
+        orc.backward_rows(wl.mech, q, k, v, rel, wl.causal, do, rows, wl.scale, cfg)
+        flops = (f_fwd + f_bwd) * len(rows) / wl.L
+        sample = f"{len(rows)} of {wl.L} query rows of 1 of {wl.B * wl.H} (batch, head) slices: O, LSE and dQ"
+    return time.perf_counter() - t0, flops, sample
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(wl, rows_fraction=1 / 64)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        s, f, sample = oracle_sample(wl, rows_fraction=1 / 64)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "mech": wl.name.split("_")[0], "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d,
+                   "causal": wl.causal, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, wl):
+    rank, world, local = rdist.init_from_env(backend="nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    path_name = "simt" if args.path == "simt" else "auto"
+    path = bd.PATH_SIMT if args.path == "simt" else bd.PATH_AUTO
+    P = bd.Params(mech=wl.mech, B=wl.B, H=wl.H, L=wl.L, d=wl.d,
+                  dtype=bd.BF16 if wl.dtype == torch.bfloat16 else bd.F32, causal=wl.causal, scale=wl.scale,
+                  kernel_path=path, t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance,
+                  shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+    inp = make_inputs(wl, seed=rank)
+    if rank != 0:  # the relative tables are shared by all ranks (one model)
+        inp["rel"] = make_inputs(wl, seed=0)["rel"]
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    rel = [r.to(dev) for r in inp["rel"]]
+    ws_f = bd.workspace(P, 0, dev)
+    ws_b = bd.workspace(P, 1, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    drel = [torch.empty(r.shape, dtype=torch.float32, device=dev) for r in rel[: P.n_rel()]]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bd.relpos_attn_fwd(P, q, k, v, rel, o, lse, ws_f, stream=stream)
+        bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, ws_b, stream=stream)
+        if world > 1:
+            rdist.allreduce_table_grads(drel)
+
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_mem = torch.cuda.memory_allocated(dev)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    rdist.barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.fill_(float(s))
+        ev[s][0].record(stream)
+        bd.relpos_attn_fwd(P, q, k, v, rel, o, lse, ws_f, stream=stream)
+        ev[s][1].record(stream)
+        bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, ws_b, stream=stream)
+        if world > 1:
+            rdist.allreduce_table_grads(drel)
+        ev[s][2].record(stream)
+    torch.cuda.synchronize()
+    rdist.barrier()
+    clk = clocks.stop()
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    tot_ms = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
+    tot_ms = rdist.max_over_ranks(tot_ms)
+    peak_mem = torch.cuda.max_memory_allocated(dev) - base_mem
+
+    f_fwd, f_bwd = algo_flops(wl)
+    fa_f, fa_b = fa_flops(wl)
+    ms_step = tot_ms / args.steps
+    value = world * (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
+    tokens = world * wl.B * wl.L / (ms_step * 1e-3)
+    peaks, peak_src = load_peaks()
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_avg = statistics.mean(bwd_ms)
+    tensor_path = path_name == "auto" and wl.dtype == torch.bfloat16 and bd.tc_available(P)
+    # roofline of the dominant pass, timed as one unit on its stream
+    if bwd_avg >= fwd_avg:
+        dom, dom_flops, dom_ms = "relpos_attn_bwd", f_bwd, bwd_avg
+    else:
+        dom, dom_flops, dom_ms = "relpos_attn_fwd", f_fwd, fwd_avg
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    if tensor_path:
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": dom, "peak_kind": f"bf16 sustained ({peak_src})"}
+    else:
+        # CUDA-core path: fp32 FFMA bound, peak = 148 SMs x 128 lanes x 2 flop x max SM clock
+        peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": dom, "peak_kind": "fp32 FFMA, 148 SM x 128 lanes x 2 x max clock"}
+
+    # ---- end to end through the public API: pinned host in, host out ----
+    e2e = run_e2e(args, wl, P, inp, dev, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, flops, sample = oracle_sample(wl)
+        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": sample, "seconds": secs}
+
+    fl, bl = kernel_launches(wl, path_name if not tensor_path else "tc")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d, "causal": wl.causal,
+                   "kernel_path": "tcgen05" if tensor_path else "cuda-core fp32",
+                   "l2": "flushed before every timed step (256 MB write, untimed)",
+                   "parallelism": f"dp{world} (weak; table grads all-reduced)" if world > 1 else "single GPU"},
+        "tokens_per_s": tokens,
+        "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
+        "fwd_tflops": f_fwd / (fwd_avg * 1e-3) / 1e12, "bwd_tflops": f_bwd / (bwd_avg * 1e-3) / 1e12,
+        "fa_convention_tflops": world * (fa_f + fa_b) / (ms_step * 1e-3) / 1e12,
+        "frac_of_dense_bf16_datasheet": value / world / 2250.0,
+        "frac_of_measured_bf16": value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+        "peak_mem_bytes": int(peak_mem),
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": (fl + bl) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    rdist.shutdown()
+    return 0
+
+
+def run_e2e(args, wl, P, inp, dev, stream, world):
+    """Same metric through the public entry points, with the step's inputs copied
+    from pinned host memory and its results (dQ, dK, dV, drel) copied back."""
+    host_in = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
+    host_rel = [r.pin_memory() for r in inp["rel"]]
+    q, k, v, do = (torch.empty_like(host_in[n], device=dev) for n in ("q", "k", "v", "do"))
+    rel = [torch.empty_like(r, device=dev) for r in host_rel]
+    ws_f = bd.workspace(P, 0, dev)
+    ws_b = bd.workspace(P, 1, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    drel = [torch.empty(r.shape, dtype=torch.float32, device=dev) for r in rel[: P.n_rel()]]
+    out_host = [torch.empty_like(t, device="cpu").pin_memory() for t in [dq, dk, dv] + drel]
+    h2d = sum(t.numel() * t.element_size() for t in list(host_in.values()) + host_rel)
+    d2h = sum(t.numel() * t.element_size() for t in out_host)
+
+    def step():
+        for dst, src in zip([q, k, v, do], [host_in[n] for n in ("q", "k", "v", "do")]):
+            dst.copy_(src, non_blocking=True)
+        for dst, src in zip(rel, host_rel):
+            dst.copy_(src, non_blocking=True)
+        bd.relpos_attn_fwd(P, q, k, v, rel, o, lse, ws_f, stream=stream)
+        bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, ws_b, stream=stream)
+        if world > 1:
+            rdist.allreduce_table_grads(drel)
+        for dst, src in zip(out_host, [dq, dk, dv] + drel):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    rdist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = rdist.max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    f_fwd, f_bwd = algo_flops(wl)
+    return {"value": world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

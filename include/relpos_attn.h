@@ -1,0 +1,156 @@
+/*
+ * relpos_attn.h -- C ABI of the relative-position attention library (B200, sm_100a).
+ *
+ * Exact softmax attention with an additive relative-position term,
+ *
+ *     S_ij = scale * Q_i . K_j + R_ij        (masked to -inf when causal and j > i)
+ *     O    = softmax_j(S) V,   LSE_i = ln sum_j exp S_ij,
+ *
+ * forward and backward, as described by "Fast and Exact Relative-Position
+ * Attention via Structure-Aware Kernels" (Abstract: exact FlashAttention-style
+ * tiled computation with offset-aware tiling, reuse of the needed key/query
+ * relation products, and offset-sharded, atomic-free gradient aggregation) and by
+ * the article "结构感知内核让相对位置注意力加速21倍" (section
+ * "为什么相对位置注意力难做快": S = Q K^T / sqrt(d) + B, with B never
+ * materialised).  The four mechanisms are the ones the paper's Hugging Face page
+ * names (Community comment); their formulas follow their original papers:
+ *
+ *   RELPOS_T5       R_ij = t[h, bucket(j - i)]                      (added unscaled)
+ *   RELPOS_SHAW     R_ij = scale * q_i . a[h, clip(j - i, -c, c) + c]
+ *   RELPOS_TXL      R_ij = scale * (u[h] . k_j + (q_i + v[h]) . r[h, row(i - j)])
+ *                   row(x) = x when causal (table rows L), x + L - 1 otherwise (2L - 1)
+ *   RELPOS_DEBERTA  R_ij = scale * (q_i . Kr[h, clip(i - j + k, 0, 2k - 1)]
+ *                                 + k_j . Qr[h, clip(j - i + k, 0, 2k - 1)])
+ *
+ * T5 buckets: bidirectional (upper half for j > i) or unidirectional, exact
+ * distances below max_exact = (buckets per side) / 2, then
+ * max_exact + floor(log(a / max_exact) / log(max_distance / max_exact) *
+ * (per side - max_exact)) capped to the last bucket, evaluated in exact integer
+ * arithmetic.
+ *
+ * Memory and ownership
+ *   - Every pointer is a DEVICE pointer allocated by the caller; the library
+ *     allocates nothing, never synchronises the host, keeps no global state and
+ *     is safe to call from several host threads on different streams.
+ *   - Q, K, V, O, dO, dQ, dK, dV: contiguous [B, H, L, d] in the params' dtype
+ *     (float32 or bfloat16).  d must be 64.
+ *   - Relative parameters rel[0..2] (contiguous, params' dtype unless noted):
+ *       T5       rel[0] = t  [H, num_buckets]            float32 always
+ *       Shaw     rel[0] = a  [H, 2c + 1, d]
+ *       TXL      rel[0] = r  [H, n_off, d]  (n_off = L causal, 2L - 1 otherwise),
+ *                rel[1] = u  [H, d], rel[2] = v [H, d]
+ *       DeBERTa  rel[0] = Kr [H, 2k, d], rel[1] = Qr [H, 2k, d]
+ *     Unused entries may be NULL.
+ *   - LSE: float32 [B, H, L], natural log.
+ *   - drel[0..2]: float32 gradients with the shapes of rel[0..2], summed over the
+ *     batch; they are overwritten (not accumulated into).
+ *   - workspace: device scratch of at least relpos_attn_workspace_size() bytes,
+ *     256-byte aligned; its contents on entry do not matter.
+ *   - dev_status: optional device int32; kernels that wait on hardware barriers
+ *     write a RELPOS_ERR_* code there when a wait runs out (the caller clears it
+ *     to 0 and reads it back after synchronising).  NULL disables it.
+ *   - stream: a cudaStream_t (NULL = the legacy default stream).  All work is
+ *     enqueued on it asynchronously.
+ *
+ * Errors: every call returns RELPOS_OK (0) or a negative RELPOS_ERR_* code and
+ * enqueues nothing on error.  Launch failures are reported as RELPOS_ERR_LAUNCH.
+ * Nothing aborts, traps or throws across this boundary.
+ *
+ * Determinism: the backward pass uses no atomic operations; the relative-table
+ * gradients are reduced from per-shard partials in a fixed order, so repeated
+ * calls give bitwise identical results.
+ */
+#ifndef RELPOS_ATTN_H_
+#define RELPOS_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RELPOS_API __attribute__((visibility("default")))
+#else
+#define RELPOS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum relpos_mech { RELPOS_T5 = 0, RELPOS_SHAW = 1, RELPOS_TXL = 2, RELPOS_DEBERTA = 3 };
+enum relpos_dtype { RELPOS_F32 = 0, RELPOS_BF16 = 1 };
+
+/* kernel_path: which kernel family runs the call.  RELPOS_PATH_AUTO picks the
+ * tensor-core (tcgen05) kernels for bfloat16 and the fp32 CUDA-core kernels for
+ * float32.  RELPOS_PATH_SIMT forces the CUDA-core kernels (fp32 arithmetic on
+ * any dtype).  Both are GPU paths; there is no CPU path. */
+enum relpos_path { RELPOS_PATH_AUTO = 0, RELPOS_PATH_SIMT = 1, RELPOS_PATH_TC = 2 };
+
+enum relpos_status {
+  RELPOS_OK = 0,
+  RELPOS_ERR_INVALID_ARG = -1,      /* null pointer, bad enum, d != 64, bad sizes */
+  RELPOS_ERR_WORKSPACE = -2,        /* workspace NULL or smaller than required     */
+  RELPOS_ERR_UNSUPPORTED = -3,      /* valid but not implemented (e.g. path/dtype)  */
+  RELPOS_ERR_LAUNCH = -4,           /* a kernel launch was rejected by the driver  */
+  RELPOS_ERR_TIMEOUT = -5,          /* (device status only) a bounded wait ran out  */
+  RELPOS_ERR_CUDA = -6              /* a CUDA runtime call failed                    */
+};
+
+typedef struct relpos_params {
+  int32_t mech;              /* enum relpos_mech                                  */
+  int32_t dtype;             /* enum relpos_dtype                                 */
+  int32_t causal;            /* 1: mask keys j > i                                */
+  int32_t kernel_path;       /* enum relpos_path                                  */
+  int64_t B, H, L, d;        /* batch, heads, sequence length, head dim (64)      */
+  float scale;               /* multiplies q.k (and the terms listed above)       */
+  int32_t t5_num_buckets;    /* T5: number of buckets (e.g. 32), 2..64            */
+  int32_t t5_max_distance;   /* T5: distance of the last bucket (e.g. 128)        */
+  int32_t t5_bidirectional;  /* T5: 1 bidirectional, 0 unidirectional             */
+  int32_t shaw_clip;         /* Shaw: clip distance c (table rows 2c + 1)         */
+  int32_t deberta_span;      /* DeBERTa: relative span k (table rows 2k)          */
+} relpos_params_t;
+
+/* Bytes of device workspace a call needs.  pass: 0 forward, 1 backward.
+ * Returns RELPOS_OK and sets *bytes, or RELPOS_ERR_INVALID_ARG. */
+RELPOS_API int relpos_attn_workspace_size(const relpos_params_t *params, int pass, size_t *bytes);
+
+/* Forward pass: writes O [B,H,L,d] (params dtype) and LSE [B,H,L] (float32).
+ * The step of the method: exact tiled attention with the relative term folded
+ * into the online softmax ("Fast and Exact Relative-Position Attention via
+ * Structure-Aware Kernels", Abstract; article "结构感知内核让相对位置注意力加速21倍",
+ * section "结构感知分块如何保持精确性"). */
+RELPOS_API int relpos_attn_fwd(const relpos_params_t *params,
+                    const void *q, const void *k, const void *v,
+                    const void *const rel[3],
+                    void *o, float *lse,
+                    void *workspace, size_t workspace_bytes,
+                    int32_t *dev_status, void *stream);
+
+/* Backward pass: given O and LSE from relpos_attn_fwd and the output gradient
+ * dO, writes dQ, dK, dV (params dtype) and drel[0..2] (float32, see above).
+ * Gradients of the relative parameters are sharded by offset into partials and
+ * merged by a fixed-order second pass with no atomics (same Abstract, technique
+ * (3); article section "3. 基于偏移的梯度分片"). */
+RELPOS_API int relpos_attn_bwd(const relpos_params_t *params,
+                    const void *q, const void *k, const void *v,
+                    const void *const rel[3],
+                    const void *o, const float *lse, const void *dout,
+                    void *dq, void *dk, void *dv, float *const drel[3],
+                    void *workspace, size_t workspace_bytes,
+                    int32_t *dev_status, void *stream);
+
+/* Kernel family a call with these params runs: RELPOS_PATH_SIMT or
+ * RELPOS_PATH_TC (RELPOS_PATH_AUTO resolved), or a negative RELPOS_ERR_* code
+ * (RELPOS_ERR_UNSUPPORTED when RELPOS_PATH_TC is forced where it does not apply). */
+RELPOS_API int relpos_attn_resolved_path(const relpos_params_t *params);
+
+/* Static, NUL-terminated description of a status code. */
+RELPOS_API const char *relpos_strerror(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+RELPOS_API int relpos_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RELPOS_ATTN_H_ */

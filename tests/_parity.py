@@ -1,0 +1,73 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI
+binding and the fp64 oracle on the same seeded inputs, and compare."""
+import numpy as np
+import torch
+
+import oracle as orc
+from attention_fwd_bwd_flashattention_b200 import binding as bd
+from attention_fwd_bwd_flashattention_b200.inputs import to_f64
+
+# tolerances: max-abs on O (and LSE), relative L2 on every gradient
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+
+def oracle_cfg(wl):
+    return orc.RelCfg(t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance, t5_bidirectional=wl.t5_bidirectional,
+                      shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+
+
+def params_of(wl, path):
+    return bd.Params(mech=wl.mech, B=wl.B, H=wl.H, L=wl.L, d=wl.d, dtype=bd.BF16 if wl.dtype == torch.bfloat16 else bd.F32,
+                     causal=wl.causal, scale=wl.scale, kernel_path=path, t5_num_buckets=wl.t5_num_buckets,
+                     t5_max_distance=wl.t5_max_distance, t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+
+
+def run_gpu(wl, inp, path, dev="cuda"):
+    P = params_of(wl, path)
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    rel = [r.to(dev) for r in inp["rel"]]
+    o, lse = bd.forward(P, q, k, v, rel)
+    dq, dk, dv, drel = bd.backward(P, q, k, v, rel, o, lse, do)
+    torch.cuda.synchronize()
+    return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, drel=drel)
+
+
+def maxabs(got, want):
+    return float(np.max(np.abs(got - want))) if want.size else 0.0
+
+
+def rel_l2(got, want):
+    den = float(np.linalg.norm(want))
+    num = float(np.linalg.norm(got - want))
+    return num / den if den > 1e-30 else num
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def compare_full(wl, inp, out, heads=None):
+    """Compare every output with the oracle (optionally only some heads; table
+    gradients then cover those heads, which is exact when B == 1)."""
+    tol = TOL[wl.dtype]
+    cfg = oracle_cfg(wl)
+    q, k, v, do = (to_f64(inp[n]) for n in ("q", "k", "v", "do"))
+    rel = [to_f64(r) for r in inp["rel"]]
+    hs = slice(None) if heads is None else heads
+    if heads is not None:
+        q, k, v, do = q[:, hs], k[:, hs], v[:, hs], do[:, hs]
+        rel = [r[hs] for r in rel]
+    O, LSE = orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg)
+    dq, dk, dv, drel = orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg)
+    errs = {
+        "o": maxabs(f64(out["o"][:, hs]), O),
+        "lse": maxabs(f64(out["lse"][:, hs]), LSE),
+        "dq": rel_l2(f64(out["dq"][:, hs]), dq),
+        "dk": rel_l2(f64(out["dk"][:, hs]), dk),
+        "dv": rel_l2(f64(out["dv"][:, hs]), dv),
+    }
+    for n, g in enumerate(drel):
+        errs[f"drel{n}"] = rel_l2(f64(out["drel"][n][hs]), g)
+    bad = {n: e for n, e in errs.items() if not e <= tol}
+    assert not bad, f"{wl.name}: over tolerance {tol}: {bad} (all: {errs})"
+    return errs

@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol include/relpos_attn.h declares, the ctypes struct matches the C layout,
+and argument validation returns the documented codes without touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from attention_fwd_bwd_flashattention_b200 import binding as bd
+from attention_fwd_bwd_flashattention_b200 import build as bld
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "relpos_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    bld.build()
+    return bd.load()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"RELPOS_API\s+[\w\s\*]*?\b(relpos_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_symbols() == sorted(bd.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", bd.lib_path()], capture_output=True, text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for sym in declared_symbols():
+        assert sym in exported, sym
+        assert hasattr(lib, sym)
+    # nothing else of ours leaks out of the library
+    assert {s for s in exported if s.startswith("relpos")} == set(declared_symbols())
+
+
+def test_struct_layout_matches_c(tmp_path):
+    prog = tmp_path / "layout.c"
+    prog.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "relpos_attn.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
+        " offsetof(relpos_params_t,scale), offsetof(relpos_params_t,t5_num_buckets), offsetof(relpos_params_t,deberta_span));return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(prog), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    S = bd.relpos_params_t
+    assert got == [ctypes.sizeof(S), S.B.offset, S.scale.offset, S.t5_num_buckets.offset, S.deberta_span.offset]
+
+
+def test_version_and_strerror(lib):
+    assert lib.relpos_attn_version() == 10000
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert bd.strerror(code) and bd.strerror(code) != "unknown status"
+    assert bd.strerror(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("bad", [dict(d=32), dict(mech=7), dict(L=0), dict(B=0), dict(dtype=5), dict(scale=float("nan")),
+                                 dict(kernel_path=9), dict(mech=0, t5_num_buckets=1), dict(mech=0, t5_max_distance=4),
+                                 dict(mech=3, deberta_span=0), dict(mech=1, shaw_clip=-1)])
+def test_invalid_params_rejected(lib, bad):
+    kw = dict(mech=1, B=1, H=2, L=64)
+    kw.update(bad)
+    with pytest.raises(bd.RelposError) as e:
+        bd.relpos_attn_workspace_size(bd.Params(**kw), 0)
+    assert e.value.code == -1
+
+
+def test_workspace_sizes(lib):
+    for mech in range(4):
+        for causal in (False, True):
+            P = bd.Params(mech=mech, B=2, H=3, L=1000, causal=causal)
+            f = bd.relpos_attn_workspace_size(P, 0)
+            b = bd.relpos_attn_workspace_size(P, 1)
+            assert b >= 2 * 3 * 1000 * 4  # at least D
+            assert f % 256 == 0 and b % 256 == 0
+            assert (f > 0) == (mech == 0)
+    with pytest.raises(bd.RelposError):
+        bd.relpos_attn_workspace_size(bd.Params(mech=1, B=1, H=1, L=8), 2)
+
+
+def test_null_pointers_rejected_before_any_device_work(lib):
+    P = bd.Params(mech=1, B=1, H=1, L=64).c()
+    null3 = (ctypes.c_void_p * 3)()
+    rc = lib.relpos_attn_fwd(ctypes.byref(P), None, None, None, null3, None, None, None, 0, None, None)
+    assert rc == -1
+    rc = lib.relpos_attn_bwd(ctypes.byref(P), None, None, None, null3, None, None, None, None, None, None, null3, None, 0,
+                             None, None)
+    assert rc == -1
+    # a fake non-null pointer set with a missing table is still an argument error
+    fake = ctypes.c_void_p(0x1000)
+    rc = lib.relpos_attn_fwd(ctypes.byref(P), fake, fake, fake, null3, fake, fake, None, 0, None, None)
+    assert rc == -1
+
+
+def test_workspace_checked_before_launch(lib):
+    P = bd.Params(mech=0, B=1, H=1, L=64).c()  # T5 forward needs workspace
+    fake = ctypes.c_void_p(0x1000)
+    rel = (ctypes.c_void_p * 3)(0x1000, None, None)
+    assert lib.relpos_attn_fwd(ctypes.byref(P), fake, fake, fake, rel, fake, fake, None, 0, None, None) == -2
+    assert lib.relpos_attn_fwd(ctypes.byref(P), fake, fake, fake, rel, fake, fake, ctypes.c_void_p(0x1010), 1 << 20, None,
+                               None) == -2  # misaligned
+
+
+def test_t5_thresholds_match_oracle_buckets(lib):
+    """The library's exact integer bucket thresholds (host side) against the
+    oracle's bucket function, through the resolved-path query (validation only):
+    checked indirectly on the GPU; here only that odd settings are accepted."""
+    for nb, md, bidir in ((32, 128, True), (10, 40, True), (7, 20, False), (64, 1000, True)):
+        bd.relpos_attn_workspace_size(bd.Params(mech=0, B=1, H=1, L=100, t5_num_buckets=nb, t5_max_distance=md,
+                                                t5_bidirectional=bidir), 0)

@@ -1,0 +1,150 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element.
+
+Tolerances are the workloads': max-abs 1e-4 on O for float32 inputs and 2e-2
+for bfloat16, relative L2 1e-4 / 2e-2 on every gradient (dQ, dK, dV and each
+relative-parameter gradient).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from attention_fwd_bwd_flashattention_b200 import binding as bd
+from attention_fwd_bwd_flashattention_b200.inputs import DEBERTA, SHAW, T5, TXL, WORKLOADS, Workload, make_inputs, to_f64
+
+from _parity import TOL, compare_full, f64, maxabs, oracle_cfg, rel_l2, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+MECHS = {"t5": T5, "shaw": SHAW, "txl": TXL, "deberta": DEBERTA}
+
+
+def small_wl(mech, dtype, causal, L, B=2, H=2, **kw):
+    kw.setdefault("shaw_clip", 64)
+    kw.setdefault("deberta_span", 24)
+    return Workload(f"small_{mech}_{L}", MECHS[mech], dtype, causal, B, H, L, **kw)
+
+
+# --------------------------------------------------------------------------
+# small shapes: several tiles and a ragged tail, every mechanism, both dtypes,
+# causal and not, on both kernel families
+# --------------------------------------------------------------------------
+SMALL_L = [1, 17, 64, 130, 257]
+
+
+@pytest.mark.parametrize("path", [bd.PATH_SIMT])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("mech", list(MECHS))
+@pytest.mark.parametrize("L", SMALL_L)
+def test_parity_small(mech, causal, dtype, L, path):
+    wl = small_wl(mech, dtype, causal, L)
+    inp = make_inputs(wl, seed=L)
+    out = run_gpu(wl, inp, path)
+    compare_full(wl, inp, out)
+
+
+@pytest.mark.parametrize("path", [bd.PATH_SIMT])
+def test_parity_deberta_span256(path):
+    wl = Workload("deb600", DEBERTA, torch.bfloat16, False, 1, 2, 600)
+    inp = make_inputs(wl, 3)
+    compare_full(wl, inp, run_gpu(wl, inp, path))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_parity_t5_unidirectional_and_odd_buckets(causal):
+    for nb, md, bidir in ((32, 128, False), (10, 40, True), (7, 20, False)):
+        wl = Workload("t5x", T5, torch.float32, causal, 1, 2, 300, t5_num_buckets=nb, t5_max_distance=md,
+                      t5_bidirectional=bidir)
+        inp = make_inputs(wl, nb)
+        compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+def test_t5_small_buckets_and_fp32_config():
+    # the fp32 T5 workload itself (one batch, two heads, L = 128) on its own path
+    wl = WORKLOADS["t5_L128_fp32"]
+    inp = make_inputs(wl, 0)
+    errs = compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+    assert errs["o"] <= 1e-4
+
+
+def test_determinism():
+    for name in ("shaw_L2048_bf16",):
+        wl = WORKLOADS[name].with_(L=300, B=1, H=2)
+        inp = make_inputs(wl, 1)
+        a = run_gpu(wl, inp, bd.PATH_AUTO)
+        b = run_gpu(wl, inp, bd.PATH_AUTO)
+        for key in ("o", "lse", "dq", "dk", "dv"):
+            assert torch.equal(a[key], b[key]), key
+        for x, y in zip(a["drel"], b["drel"]):
+            assert torch.equal(x, y)
+    for mech in ("txl", "deberta", "t5"):
+        wl = small_wl(mech, torch.bfloat16, mech == "txl", 200)
+        inp = make_inputs(wl, 2)
+        a = run_gpu(wl, inp, bd.PATH_AUTO)
+        b = run_gpu(wl, inp, bd.PATH_AUTO)
+        for x, y in zip(a["drel"] + [a["dq"], a["dk"]], b["drel"] + [b["dq"], b["dk"]]):
+            assert torch.equal(x, y), mech
+
+
+def test_errors_are_reported_not_raised_on_device():
+    wl = small_wl("shaw", torch.bfloat16, False, 64)
+    P = bd.Params(mech=SHAW, B=2, H=2, L=64, d=32)
+    with pytest.raises(bd.RelposError) as e:
+        bd.relpos_attn_workspace_size(P, 0)
+    assert e.value.code == -1
+    inp = make_inputs(wl, 0)
+    P = bd.Params(mech=SHAW, B=2, H=2, L=64)
+    q = inp["q"].cuda()
+    o = torch.empty_like(q)
+    lse = torch.empty(2, 2, 64, device="cuda")
+    with pytest.raises(bd.RelposError) as e:
+        bd.relpos_attn_fwd(P, q, q, q, [None], o, lse, None)
+    assert e.value.code == -1
+
+
+# --------------------------------------------------------------------------
+# the workloads at full size
+# --------------------------------------------------------------------------
+def test_parity_shaw_L2048_full():
+    wl = WORKLOADS["shaw_L2048_bf16"]
+    inp = make_inputs(wl, 0)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+@pytest.mark.parametrize("name", ["txl_causal_L8192_bf16", "deberta_L8192_bf16", "txl_L8192_bf16"])
+def test_parity_L8192_one_head(name):
+    """Every output of head 0 (table gradients included, B = 1) at L = 8192."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, 0)
+    out = run_gpu(wl, inp, bd.PATH_AUTO)
+    compare_full(wl, inp, out, heads=slice(0, 1))
+
+
+@pytest.mark.parametrize("name", ["txl_L16384_bf16", "txl_L32768_bf16"])
+def test_parity_long_sampled(name):
+    """Sampled query rows of O, LSE and dQ (each a function of its own row), plus
+    properties that hold at any size: sum_j dV_j = sum_i dO_i, sum_j dK_j = 0 and
+    sum_rho dr_rho = 0 for Transformer-XL (each row of dS sums to zero)."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, 0)
+    out = run_gpu(wl, inp, bd.PATH_AUTO)
+    tol = TOL[wl.dtype]
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, 128], np.random.default_rng(0).integers(0, wl.L, 10), [wl.L - 1]]))
+    h = slice(0, 1)
+    q, k, v, do = (to_f64(inp[n])[:, h] for n in ("q", "k", "v", "do"))
+    rel = [to_f64(r)[h] for r in inp["rel"]]
+    cfg = oracle_cfg(wl)
+    O, LSE = orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, rows=rows)
+    assert maxabs(f64(out["o"][:, h][:, :, rows]), O) <= tol
+    assert maxabs(f64(out["lse"][:, h][:, :, rows]), LSE) <= tol
+    dq = orc.backward_rows(wl.mech, q, k, v, rel, wl.causal, do, rows, wl.scale, cfg)
+    assert rel_l2(f64(out["dq"][:, h][:, :, rows]), dq) <= tol
+    dv_sum = f64(out["dv"].float().sum(dim=2))
+    do_sum = to_f64(inp["do"]).sum(axis=2)
+    assert rel_l2(dv_sum, do_sum) <= tol
+    dk_sum = f64(out["dk"].float().sum(dim=2))
+    assert np.max(np.abs(dk_sum)) <= tol * np.linalg.norm(f64(out["dk"][0, 0])) + 1e-3
+    dr_sum = f64(out["drel"][0].sum(dim=1))
+    assert np.max(np.abs(dr_sum)) <= tol * float(torch.linalg.norm(out["drel"][0][0])) + 1e-4
