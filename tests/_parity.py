@@ -37,9 +37,14 @@ def maxabs(got, want):
 
 
 def rel_l2(got, want):
+    """||got - want|| / ||want||.  Where the exact gradient is zero (e.g. dQ at
+    L = 1) the ratio is meaningless, so the largest absolute entry of got is
+    returned instead (checked against the same tolerance)."""
     den = float(np.linalg.norm(want))
     num = float(np.linalg.norm(got - want))
-    return num / den if den > 1e-30 else num
+    if den <= 1e-6 * np.sqrt(max(want.size, 1)):
+        return float(np.max(np.abs(got))) if got.size else 0.0
+    return num / den
 
 
 def f64(t):
