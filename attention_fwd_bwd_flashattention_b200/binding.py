@@ -72,7 +72,7 @@ def load() -> ctypes.CDLL:
     lib.relpos_attn_bwd.argtypes = [P, vp, vp, vp, ctypes.POINTER(vp), vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp), vp,
                                     ctypes.c_size_t, vp, vp]
     lib.relpos_attn_bwd.restype = ctypes.c_int
-    lib.relpos_attn_resolved_path.argtypes = [P]
+    lib.relpos_attn_resolved_path.argtypes = [P, ctypes.c_int]
     lib.relpos_attn_resolved_path.restype = ctypes.c_int
     lib.relpos_strerror.argtypes = [ctypes.c_int]
     lib.relpos_strerror.restype = ctypes.c_char_p
@@ -144,17 +144,17 @@ def relpos_attn_workspace_size(params: Params, pass_: int) -> int:
     return int(n.value)
 
 
-def relpos_attn_resolved_path(params: Params) -> int:
+def relpos_attn_resolved_path(params: Params, pass_: int = 0) -> int:
     cp = params.c()
-    rc = load().relpos_attn_resolved_path(ctypes.byref(cp))
+    rc = load().relpos_attn_resolved_path(ctypes.byref(cp), int(pass_))
     if rc < 0:
         raise RelposError(rc, "relpos_attn_resolved_path")
     return rc
 
 
-def tc_available(params: Params) -> bool:
-    """True when these params run on the tensor-core (tcgen05) kernels."""
-    return relpos_attn_resolved_path(params) == PATH_TC
+def tc_available(params: Params, pass_: int = 0) -> bool:
+    """True when pass `pass_` (0 forward, 1 backward) runs on the tensor-core (tcgen05) kernels."""
+    return relpos_attn_resolved_path(params, pass_) == PATH_TC
 
 
 def relpos_attn_fwd(params: Params, q, k, v, rel, o, lse, workspace, dev_status=None, stream=None) -> None:

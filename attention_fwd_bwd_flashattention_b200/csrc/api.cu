@@ -125,18 +125,22 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   return RELPOS_OK;
 }
 
-static bool use_tc(const relpos_params_t *P) {
-  (void)P;
-  return false;
+// Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
+static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
+  if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
+  if (pass == 1) return false;  // the backward pass runs on the CUDA-core kernels
+  return rp::tc_supported(p);
 }
 
 // ---- workspace layout ------------------------------------------------------
 struct Layout {
-  size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot, total;
+  size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot;
+  size_t uk, vr, c2pE, p2cE;  // tensor-core forward products
+  size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-static Layout layout_of(const Prm &p, int pass) {
+static Layout layout_of(const Prm &p, int pass, bool tc) {
   Layout l;
   memset(&l, 0, sizeof(l));
   size_t off = 0;
@@ -149,6 +153,16 @@ static Layout layout_of(const Prm &p, int pass) {
   if (p.mech == rp::M_T5) {
     l.t5_bias = take(sizeof(float) * (size_t)p.H * (2 * (size_t)p.L - 1));
     l.t5_bkt = take(sizeof(int) * (2 * (size_t)p.L - 1));
+  }
+  if (pass == 0 && tc) {
+    if (p.mech == rp::M_TXL) {
+      l.uk = take(sizeof(float) * BH * p.L);
+      l.vr = take(sizeof(float) * (size_t)p.H * p.nrows);
+    }
+    if (p.mech == rp::M_DEB) {
+      l.c2pE = take(sizeof(float) * BH * p.L * 2);
+      l.p2cE = take(sizeof(float) * BH * p.L * 2);
+    }
   }
   if (pass == 1) {
     l.dvec = take(sizeof(float) * BH * p.L);
@@ -185,6 +199,18 @@ static void bind_workspace(Prm &p, const Layout &l, void *ws) {
   p.gtot = (float *)(b + l.gtot);
 }
 
+static rp::TcWork tc_work(const Layout &l, void *ws) {
+  char *b = (char *)ws;
+  rp::TcWork w;
+  w.uk = (float *)(b + l.uk);
+  w.vr = (float *)(b + l.vr);
+  w.c2pE = (float *)(b + l.c2pE);
+  w.p2cE = (float *)(b + l.p2cE);
+  return w;
+}
+
+static bool aligned16(const void *x) { return ((uintptr_t)x & 15) == 0; }
+
 static int rel_count(int mech) { return mech == rp::M_TXL ? 3 : (mech == rp::M_DEB ? 2 : 1); }
 
 static int to_status(cudaError_t e) {
@@ -200,7 +226,7 @@ extern "C" int relpos_attn_workspace_size(const relpos_params_t *params, int pas
   if (!bytes || (pass != 0 && pass != 1)) return RELPOS_ERR_INVALID_ARG;
   int e = validate_and_fill(params, p);
   if (e) return e;
-  *bytes = layout_of(p, pass).total;
+  *bytes = layout_of(p, pass, use_tc(params, p, pass)).total;
   return RELPOS_OK;
 }
 
@@ -213,8 +239,14 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   if (!q || !k || !v || !rel || !o || !lse) return RELPOS_ERR_INVALID_ARG;
   for (int i = 0; i < rel_count(p.mech); ++i)
     if (!rel[i]) return RELPOS_ERR_INVALID_ARG;
-  if (params->kernel_path == RELPOS_PATH_TC && !use_tc(params)) return RELPOS_ERR_UNSUPPORTED;
-  const Layout l = layout_of(p, 0);
+  const bool tc = use_tc(params, p, 0);
+  if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
+  if (tc) {  // TMA needs 16-byte aligned tensors
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(rel[0]) ||
+        (p.mech == rp::M_DEB && !aligned16(rel[1])))
+      return RELPOS_ERR_INVALID_ARG;
+  }
+  const Layout l = layout_of(p, 0, tc);
   if (l.total > 0 && (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255))) return RELPOS_ERR_WORKSPACE;
   bind_workspace(p, l, workspace);
   p.q = q;
@@ -229,6 +261,7 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   cudaStream_t st = (cudaStream_t)stream;
   const bool bf16 = params->dtype == RELPOS_BF16;
   if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
+  if (tc) return to_status(rp::tc_fwd(p, tc_work(l, workspace), st));
   return to_status(rp::simt_fwd(p, bf16, st));
 }
 
@@ -242,8 +275,9 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   if (!q || !k || !v || !rel || !o || !lse || !dout || !dq || !dk || !dv || !drel) return RELPOS_ERR_INVALID_ARG;
   for (int i = 0; i < rel_count(p.mech); ++i)
     if (!rel[i] || !drel[i]) return RELPOS_ERR_INVALID_ARG;
-  if (params->kernel_path == RELPOS_PATH_TC && !use_tc(params)) return RELPOS_ERR_UNSUPPORTED;
-  const Layout l = layout_of(p, 1);
+  const bool tc = use_tc(params, p, 1);
+  if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
+  const Layout l = layout_of(p, 1, tc);
   if (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255)) return RELPOS_ERR_WORKSPACE;
   bind_workspace(p, l, workspace);
   p.q = q;
@@ -268,12 +302,14 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   return to_status(rp::simt_bwd(p, bf16, st));
 }
 
-extern "C" int relpos_attn_resolved_path(const relpos_params_t *params) {
+extern "C" int relpos_attn_resolved_path(const relpos_params_t *params, int pass) {
   Prm p;
+  if (pass != 0 && pass != 1) return RELPOS_ERR_INVALID_ARG;
   int e = validate_and_fill(params, p);
   if (e) return e;
-  if (params->kernel_path == RELPOS_PATH_TC && !use_tc(params)) return RELPOS_ERR_UNSUPPORTED;
-  return use_tc(params) ? RELPOS_PATH_TC : RELPOS_PATH_SIMT;
+  const bool tc = use_tc(params, p, pass);
+  if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
+  return tc ? RELPOS_PATH_TC : RELPOS_PATH_SIMT;
 }
 
 extern "C" const char *relpos_strerror(int status) {

@@ -18,6 +18,7 @@
 namespace rp {
 
 constexpr int HD = 64;  // head dimension supported by every kernel
+constexpr int RELPOS_ERR_TIMEOUT_DEV = -5;  // value of RELPOS_ERR_TIMEOUT written to the device status word
 
 enum { M_T5 = 0, M_SHAW = 1, M_TXL = 2, M_DEB = 3 };
 

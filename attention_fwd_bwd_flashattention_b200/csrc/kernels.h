@@ -7,4 +7,11 @@ namespace rp {
 cudaError_t launch_t5_prep(const Prm &p, cudaStream_t st);
 cudaError_t simt_fwd(const Prm &p, bool bf16, cudaStream_t st);
 cudaError_t simt_bwd(const Prm &p, bool bf16, cudaStream_t st);
+
+// tensor-core (bf16) path
+struct TcWork {
+  float *uk, *vr, *c2pE, *p2cE;  // per-call products (Transformer-XL, DeBERTa)
+};
+bool tc_supported(const Prm &p);
+cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st);
 }  // namespace rp

@@ -1,0 +1,667 @@
+// Tensor-core (tcgen05 / TMEM / TMA) forward kernel of relative-position
+// attention for bf16 inputs, d = 64, on sm_100a.
+//
+// One CTA per 128-row query tile (heaviest causal tiles launched first), five
+// warps:
+//   warps 0-3  "softmax": thread t owns query row t (TMEM lane t).  It reads its
+//              row of S = Q K^T and of the relation products from TMEM, adds the
+//              relative term gathered by offset, runs the online softmax (lazy
+//              rescale of O only when the running max grows by more than 2^8),
+//              and writes P (bf16) into shared memory in the 128-byte-swizzled
+//              layout the tensor core reads.
+//   warp 4     lane 0 issues every TMA load (Q, K, V, relation-table windows,
+//              2-stage K/V ring) and every tcgen05.mma, and signals through
+//              mbarriers and tcgen05.commit.
+// TMEM (512 columns): S [0,128), relation products [128,384), O [384,448).
+//
+// Relation stage per mechanism ("Fast and Exact Relative-Position Attention via
+// Structure-Aware Kernels", Abstract, techniques (1) and (2)):
+//   T5       per-tile window of the per-offset bias vector (255 values) in smem.
+//   Shaw     QA = Q a^T (129 products per row) computed once per query tile by one
+//            MMA and kept in smem; each pair reads its clipped column.
+//   TXL      the offsets of tile (m, n) are 128 (m - n) + [-127, 127]: two
+//            128-offset blocks of r.  Block b's products Q r_b^T are computed by
+//            one 128x128x64 MMA and reused by the two consecutive key tiles that
+//            need it, so each key tile adds exactly one new block.  Each row's
+//            values are rotated into key order through a padded smem row.
+//   DeBERTa  tiles within the span: c2p = Q Kr_win^T (255 offsets) rotated per row,
+//            p2c = K Qr_win^T computed with keys as rows and transposed through
+//            smem; tiles outside the span use per-row / per-key end products.
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace rp {
+namespace tc {
+
+constexpr int BM = 128, BN = 128;
+constexpr int NTHREADS = 160;
+constexpr int ROT_LD = 132;  // fp32 stride of the per-row skew buffer (conflict-free rotations)
+
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + 16384;    // 2 stages
+constexpr int OFF_V = OFF_K + 32768;    // 2 stages
+constexpr int OFF_P = OFF_V + 32768;    // two 64-key halves of P
+constexpr int OFF_R = OFF_P + 32768;    // relation-table staging (2 x 16 KB or one 32 KB window)
+constexpr int OFF_ROT = OFF_R + 32768;  // 128 x ROT_LD fp32
+constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;  // 2 x 512 fp32 per-tile vectors
+constexpr int OFF_BAR = OFF_VEC + 2 * 512 * 4;
+constexpr int SMEM_USED = OFF_BAR + 256;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+
+enum {
+  B_Q = 0, B_KV0 = 1, B_KV1 = 2, B_SFULL = 3, B_SFREE = 4, B_PFULL = 5, B_PV = 6, B_PLOAD = 7, B_PFULLPRO = 8,
+  B_PFREEPRO = 9, B_RLOAD = 10, B_RFREE = 11, B_GFULL = 12, B_DRAIN = 13, NBARS = 14
+};
+
+constexpr uint32_t TM_S = 0, TM_REL = 128, TM_O = 384, TM_COLS = 512;
+
+struct FwdArgs {
+  CUtensorMap mq, mk, mv, mt0, mt1;
+  Prm p;
+  const float *uk, *vr, *c2pE, *p2cE;
+  int shaw_n;  // N of the Shaw QA MMA (2c + 1 rounded up to 16)
+};
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// A wait whose result is the same on all 32 lanes (tcgen05.ld/st are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *ab, int32_t *st) {
+  const bool ok = mbar_wait(bar, parity, ab, st, RELPOS_ERR_TIMEOUT_DEV);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int MECH>
+__global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ FwdArgs A) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Prm &p = A.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m = p.nT - 1 - (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int L = p.L, i0 = m * BM;
+  const int nTiles = p.causal ? m + 1 : p.nT;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NBARS + 4);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NBARS);
+  float *rot = (float *)(smem + OFF_ROT);
+  float *vec = (float *)(smem + OFF_VEC);
+
+  if (tid == 0) {
+    mbar_init(BAR(B_Q), 1);
+    mbar_init(BAR(B_KV0), 1);
+    mbar_init(BAR(B_KV1), 1);
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_SFREE), 128);
+    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_PV), 1);
+    mbar_init(BAR(B_PLOAD), 1);
+    mbar_init(BAR(B_PFULLPRO), 1);
+    mbar_init(BAR(B_PFREEPRO), 128);
+    mbar_init(BAR(B_RLOAD), 1);
+    mbar_init(BAR(B_RFREE), 128);
+    mbar_init(BAR(B_GFULL), 1);
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), TM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  int32_t *status = p.status;
+  const float c1 = p.scale * 1.4426950408889634f;  // scale * log2(e)
+
+  if (warp == 4) {
+    // ======================= TMA + MMA issuer ==========================
+    if (lane == 0) {
+      prefetch_tmap(&A.mq);
+      prefetch_tmap(&A.mk);
+      prefetch_tmap(&A.mv);
+      if (MECH != M_T5) prefetch_tmap(&A.mt0);
+      if (MECH == M_DEB) prefetch_tmap(&A.mt1);
+      const uint32_t idS = idesc_bf16(128, 128, false);
+      const uint32_t idPV = idesc_bf16(128, 64, true);
+      const uint32_t idW = idesc_bf16(128, 256, false);
+      // TMA loads issued but not yet waited for, drained before exit on abort
+      uint32_t pend_bar[8];
+      uint32_t pend_par[8];
+      int npend = 0;
+      auto expect = [&](int bi, uint32_t par, uint32_t bytes) {
+        mbar_expect_tx(BAR(bi), bytes);
+        pend_bar[npend] = BAR(bi);
+        pend_par[npend] = par;
+        ++npend;
+      };
+      auto waited = [&](uint32_t bar) {  // drop one pending entry of this barrier
+        for (int e = 0; e < npend; ++e)
+          if (pend_bar[e] == bar) {
+            pend_bar[e] = pend_bar[npend - 1];
+            pend_par[e] = pend_par[npend - 1];
+            --npend;
+            return;
+          }
+      };
+      auto wait_load = [&](int bi, uint32_t par) {
+        const bool r = mbar_wait(BAR(bi), par, abort_flag, status, RELPOS_ERR_TIMEOUT_DEV);
+        if (r) waited(BAR(bi));
+        return r;
+      };
+      auto wait_bar = [&](int bi, uint32_t par) { return mbar_wait(BAR(bi), par, abort_flag, status, RELPOS_ERR_TIMEOUT_DEV); };
+
+      expect(B_Q, 0, 16384);
+      tma_load_3d(sbase + OFF_Q, &A.mq, BAR(B_Q), 0, i0, bh);
+      int rl_phase = 0, band_cnt = 0;
+      bool ok = true;
+      if (MECH == M_SHAW) {
+        expect(B_PLOAD, 0, (uint32_t)A.shaw_n * 128u);
+        tma_load_3d(sbase + OFF_R, &A.mt0, BAR(B_PLOAD), 0, 0, h);
+        ok = wait_load(B_Q, 0) && wait_load(B_PLOAD, 0);
+        if (ok) {
+          tc_fence_after();
+          umma_k64(tbase + TM_REL, sbase + OFF_Q, sbase + OFF_R, idesc_bf16(128, A.shaw_n, false), false);
+          umma_commit(BAR(B_PFULLPRO));
+          ok = wait_bar(B_PFREEPRO, 0);
+        }
+      }
+      if (MECH == M_TXL) {  // first relation block: offsets 128 m + [0, 128)
+        expect(B_PLOAD, 0, 16384);
+        tma_load_3d(sbase + OFF_P, &A.mt0, BAR(B_PLOAD), 0, 128 * m + p.off, h);
+      }
+      auto needs_new_block = [&](int n) {  // TXL: block (m - n - 1), unless it is entirely masked
+        return !(p.causal && m - n - 1 < 0);
+      };
+      auto issue_kv = [&](int n) {
+        const int st = n & 1;
+        uint32_t bytes = 32768;
+        if (MECH == M_TXL && needs_new_block(n)) bytes += 16384;
+        expect(B_KV0 + st, (uint32_t)((n >> 1) & 1), bytes);
+        tma_load_3d(sbase + OFF_K + 16384 * st, &A.mk, BAR(B_KV0 + st), 0, n * BN, bh);
+        tma_load_3d(sbase + OFF_V + 16384 * st, &A.mv, BAR(B_KV0 + st), 0, n * BN, bh);
+        if (MECH == M_TXL && needs_new_block(n))
+          tma_load_3d(sbase + OFF_R + 16384 * st, &A.mt0, BAR(B_KV0 + st), 0, 128 * (m - n - 1) + p.off, h);
+      };
+      auto issue_pv = [&](int n) {  // O (+)= P(n) V(n)
+        const int ps = n & 1;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
+                    sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024), idPV, (n > 0 || k > 0) ? 1u : 0u);
+        umma_commit(BAR(B_PV));
+      };
+      if (ok) {
+        issue_kv(0);
+        if (nTiles > 1) issue_kv(1);
+      }
+      for (int n = 0; ok && n < nTiles; ++n) {
+        const int st = n & 1;
+        const int Delta = m - n;
+        if (!wait_load(B_KV0 + st, (n >> 1) & 1)) break;
+        if (n == 0) {
+          if (MECH != M_SHAW && !wait_load(B_Q, 0)) break;
+          if (MECH == M_TXL && !wait_load(B_PLOAD, 0)) break;
+        } else if (!wait_bar(B_SFREE, (n - 1) & 1)) {
+          break;
+        }
+        tc_fence_after();
+        umma_k64(tbase + TM_S, sbase + OFF_Q, sbase + OFF_K + 16384 * st, idS, false);
+        if (MECH == M_TXL) {
+          if (n == 0) umma_k64(tbase + TM_REL + 128 * (m & 1), sbase + OFF_Q, sbase + OFF_P, idS, false);
+          if (needs_new_block(n))
+            umma_k64(tbase + TM_REL + 128 * ((Delta - 1) & 1), sbase + OFF_Q, sbase + OFF_R + 16384 * st, idS, false);
+        }
+        const bool band = (MECH == M_DEB) && (128 * (Delta < 0 ? -Delta : Delta) - 127 < p.span);
+        if (band) {
+          expect(B_RLOAD, (uint32_t)rl_phase, 32768);
+          tma_load_3d(sbase + OFF_R, &A.mt0, BAR(B_RLOAD), 0, p.span + 128 * Delta - 127, h);
+          if (!wait_load(B_RLOAD, rl_phase)) break;
+          rl_phase ^= 1;
+          umma_k64(tbase + TM_REL, sbase + OFF_Q, sbase + OFF_R, idW, false);
+        }
+        umma_commit(BAR(B_SFULL));
+        if (band) {
+          if (!wait_bar(B_RFREE, band_cnt & 1)) break;
+          tc_fence_after();
+          expect(B_RLOAD, (uint32_t)rl_phase, 32768);
+          tma_load_3d(sbase + OFF_R, &A.mt1, BAR(B_RLOAD), 0, p.span - 128 * Delta - 127, h);
+          if (!wait_load(B_RLOAD, rl_phase)) break;
+          rl_phase ^= 1;
+          umma_k64(tbase + TM_REL, sbase + OFF_K + 16384 * st, sbase + OFF_R, idW, false);
+          umma_commit(BAR(B_GFULL));
+          ++band_cnt;
+        }
+        if (n >= 1) {
+          if (!wait_bar(B_PFULL, (n - 1) & 1)) break;
+          tc_fence_after();
+          issue_pv(n - 1);
+          if (n + 1 < nTiles) {  // refill the stage tile n-1 used
+            if (!wait_bar(B_PV, (n - 1) & 1)) break;
+            issue_kv(n + 1);
+          }
+        }
+      }
+      if (ok && !*abort_flag && wait_bar(B_PFULL, (nTiles - 1) & 1)) {
+        tc_fence_after();
+        issue_pv(nTiles - 1);
+      }
+      // drain: every MMA issued by this thread, then every TMA load still in flight
+      umma_commit(BAR(B_DRAIN));
+      volatile int no_abort = 0;
+      mbar_wait(BAR(B_DRAIN), 0, &no_abort, status, RELPOS_ERR_TIMEOUT_DEV);
+      for (int e = 0; e < npend; ++e) mbar_wait(pend_bar[e], pend_par[e], &no_abort, status, RELPOS_ERR_TIMEOUT_DEV);
+    }
+    __syncwarp();
+  } else {
+    // ========================== softmax warps ===========================
+    const int il = tid, i = i0 + il;
+    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+    float *rrow = rot + il * ROT_LD;
+    float m2 = -INFINITY, lsum = 0.f;
+    float cE0 = 0.f, cE1 = 0.f;
+    bool good = true;  // warp-uniform: false once any wait of the CTA ran out
+    if (MECH == M_DEB && i < L) {
+      cE0 = A.c2pE[((size_t)bh * L + i) * 2 + 0];
+      cE1 = A.c2pE[((size_t)bh * L + i) * 2 + 1];
+    }
+    if (MECH == M_SHAW) {  // QA row -> smem (kept for the whole CTA)
+      good = warp_wait(BAR(B_PFULLPRO), 0, abort_flag, status);
+      if (good) {
+        tc_fence_after();
+        const int nq = (2 * p.clip + 1 + 31) / 32;
+        for (int q = 0; q < nq; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tl + TM_REL + 32 * q, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (32 * q + t < ROT_LD) rrow[32 * q + t] = u2f(r[t]);
+        }
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFREEPRO));
+      }
+    }
+    int band_cnt = 0;
+    for (int n = 0; n < nTiles; ++n) {
+      const int j0 = n * BN, Delta = m - n;
+      float *tv = vec + 512 * (n & 1);
+      // ---- per-tile vectors (shared by the four softmax warps) ----
+      if (MECH == M_TXL) {
+        const int j = j0 + il;
+        tv[il] = (j < L) ? A.uk[(size_t)bh * L + j] : 0.f;
+        const int ra = 128 * Delta + il + p.off, rb = 128 * (Delta - 1) + il + p.off;
+        tv[128 + il] = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
+        tv[256 + il] = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
+      } else if (MECH == M_T5) {
+        const int dmin = j0 - i0 - 127;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int w = il + 128 * k;
+          const int idx = dmin + w + L - 1;
+          if (w < 255) tv[w] = (idx >= 0 && idx < 2 * L - 1) ? p.t5_bias[(size_t)h * (2 * L - 1) + idx] : 0.f;
+        }
+      } else if (MECH == M_DEB) {
+        const int j = j0 + il;
+        tv[2 * il] = (j < L) ? A.p2cE[((size_t)bh * L + j) * 2] : 0.f;
+        tv[2 * il + 1] = (j < L) ? A.p2cE[((size_t)bh * L + j) * 2 + 1] : 0.f;
+      }
+      named_bar_sync(1, 128);
+      good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
+      float x[128];
+      if (good) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tl + TM_S + 32 * q, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) x[32 * q + t] = u2f(r[t]);
+        }
+      } else {
+#pragma unroll
+        for (int jl = 0; jl < 128; ++jl) x[jl] = 0.f;
+      }
+      // ---- relative term, gathered by offset ----
+      if (MECH == M_TXL) {
+        if (good) {
+          const bool hasB = !(p.causal && Delta == 0);
+          const uint32_t colA = TM_REL + 128 * (Delta & 1), colB = TM_REL + 128 * ((Delta - 1) & 1);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(tl + colA + 32 * q, ra);
+            if (hasB) tmem_ld32(tl + colB + 32 * q, rb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              const int c = 32 * q + t;
+              float val;
+              if (c <= il)
+                val = u2f(ra[t]) + tv[128 + c];
+              else
+                val = hasB ? u2f(rb[t]) + tv[256 + c] : 0.f;
+              rrow[(il - c) & 127] = val;
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(BAR(B_SFREE));
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const float4 rr = *reinterpret_cast<const float4 *>(rrow + 4 * c4);
+          x[4 * c4 + 0] = (x[4 * c4 + 0] + rr.x + tv[4 * c4 + 0]) * c1;
+          x[4 * c4 + 1] = (x[4 * c4 + 1] + rr.y + tv[4 * c4 + 1]) * c1;
+          x[4 * c4 + 2] = (x[4 * c4 + 2] + rr.z + tv[4 * c4 + 2]) * c1;
+          x[4 * c4 + 3] = (x[4 * c4 + 3] + rr.w + tv[4 * c4 + 3]) * c1;
+        }
+      } else if (MECH == M_T5) {
+        if (good) {
+          tc_fence_before();
+          mbar_arrive(BAR(B_SFREE));
+        }
+        const float lg = 1.4426950408889634f;
+#pragma unroll
+        for (int jl = 0; jl < 128; ++jl) x[jl] = x[jl] * c1 + tv[jl - il + 127] * lg;
+      } else if (MECH == M_SHAW) {
+        if (good) {
+          tc_fence_before();
+          mbar_arrive(BAR(B_SFREE));
+        }
+        const int d0 = j0 - i;
+#pragma unroll
+        for (int jl = 0; jl < 128; ++jl) x[jl] = (x[jl] + rrow[iclamp(d0 + jl, -p.clip, p.clip) + p.clip]) * c1;
+      } else {  // DeBERTa
+        const bool band = 128 * (Delta < 0 ? -Delta : Delta) - 127 < p.span;
+        if (band) {
+          if (good) {
+            const int lo = p.span + 128 * Delta - 127;  // unclipped Kr row of window column 0
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              uint32_t r[32];
+              tmem_ld32(tl + TM_REL + 32 * q, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int t = 0; t < 32; ++t) {
+                const int w = 32 * q + t;  // pair (il, jl) with jl = il + 127 - w
+                if (w >= il && w <= il + 127) {
+                  const int rho = lo + w;
+                  rrow[il + 127 - w] = (rho < 0) ? cE0 : (rho > 2 * p.span - 1 ? cE1 : u2f(r[t]));
+                }
+              }
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(B_RFREE));
+#pragma unroll
+            for (int jl = 0; jl < 128; ++jl) x[jl] += rrow[jl];
+          }
+          named_bar_sync(1, 128);
+          good = good && warp_wait(BAR(B_GFULL), band_cnt & 1, abort_flag, status);
+          ++band_cnt;
+          if (good) {
+            tc_fence_after();
+            // this thread is key jl = il of the tile: TMEM lane il holds K_j . Qr_win
+            const int lo2 = p.span - 128 * Delta - 127;  // unclipped Qr row of window column 0
+            const float e0 = tv[2 * il], e1 = tv[2 * il + 1];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              uint32_t r[32];
+              tmem_ld32(tl + TM_REL + 32 * q, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int t = 0; t < 32; ++t) {
+                const int w = 32 * q + t;  // pair (query il + 127 - w, key il)
+                if (w >= il && w <= il + 127) {
+                  const int rho = lo2 + w;
+                  rot[(il + 127 - w) * ROT_LD + il] = (rho < 0) ? e0 : (rho > 2 * p.span - 1 ? e1 : u2f(r[t]));
+                }
+              }
+            }
+            tc_fence_before();
+            mbar_arrive(BAR(B_SFREE));
+          }
+          named_bar_sync(1, 128);
+#pragma unroll
+          for (int jl = 0; jl < 128; ++jl) x[jl] = (x[jl] + rrow[jl]) * c1;
+        } else {
+          if (good) {
+            tc_fence_before();
+            mbar_arrive(BAR(B_SFREE));
+          }
+          const float c2p = Delta > 0 ? cE1 : cE0;
+          const int sel = Delta < 0 ? 1 : 0;
+#pragma unroll
+          for (int jl = 0; jl < 128; ++jl) x[jl] = (x[jl] + c2p + tv[2 * jl + sel]) * c1;
+        }
+      }
+      // ---- mask, online softmax (base 2, lazy rescale) ----
+      float mt = -INFINITY;
+#pragma unroll
+      for (int jl = 0; jl < 128; ++jl) {
+        const int j = j0 + jl;
+        if (j >= L || (p.causal && j > i)) x[jl] = -INFINITY;
+        mt = fmaxf(mt, x[jl]);
+      }
+      if (n == 0) {
+        m2 = mt;
+      } else {
+        const bool need = mt > m2 + 8.f;
+        if (__any_sync(0xffffffffu, need)) {
+          good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
+          if (good) {
+            tc_fence_after();
+            const float alpha = need ? ex2(m2 - mt) : 1.f;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              uint32_t r[32];
+              tmem_ld32(tl + TM_O + 32 * q, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(u2f(r[t]) * alpha);
+              tmem_st32(tl + TM_O + 32 * q, r);
+            }
+            tmem_wait_st();
+          }
+          if (need) {
+            lsum *= ex2(m2 - mt);
+            m2 = mt;
+          }
+        }
+      }
+      const float msub = (m2 == -INFINITY) ? 0.f : m2;
+#pragma unroll
+      for (int jl = 0; jl < 128; ++jl) {
+        x[jl] = ex2(x[jl] - msub);
+        lsum += x[jl];
+      }
+      if (n >= 1) good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
+      if (good) {
+        // P row -> smem, K-major 128B swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int j8 = 64 * kb + 8 * ch;
+            uint4 v;
+            v.x = pack_bf16x2(x[j8 + 0], x[j8 + 1]);
+            v.y = pack_bf16x2(x[j8 + 2], x[j8 + 3]);
+            v.z = pack_bf16x2(x[j8 + 4], x[j8 + 5]);
+            v.w = pack_bf16x2(x[j8 + 6], x[j8 + 7]);
+            *reinterpret_cast<uint4 *>(smem + OFF_P + 16384 * kb + 128 * il + ((ch ^ (il & 7)) << 4)) = v;
+          }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFULL));
+      }
+    }
+    // ---- epilogue: O / l, LSE ----
+    good = good && warp_wait(BAR(B_PV), (nTiles - 1) & 1, abort_flag, status);
+    if (good) {
+      tc_fence_after();
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      __nv_bfloat16 *orow = (__nv_bfloat16 *)p.out + ((size_t)bh * L + i) * HD;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t r[32];
+        tmem_ld32(tl + TM_O + 32 * q, r);
+        tmem_wait_ld();
+        if (i < L) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 v;
+            v.x = pack_bf16x2(u2f(r[8 * c8 + 0]) * inv, u2f(r[8 * c8 + 1]) * inv);
+            v.y = pack_bf16x2(u2f(r[8 * c8 + 2]) * inv, u2f(r[8 * c8 + 3]) * inv);
+            v.z = pack_bf16x2(u2f(r[8 * c8 + 4]) * inv, u2f(r[8 * c8 + 5]) * inv);
+            v.w = pack_bf16x2(u2f(r[8 * c8 + 6]) * inv, u2f(r[8 * c8 + 7]) * inv);
+            *reinterpret_cast<uint4 *>(orow + 32 * q + 8 * c8) = v;
+          }
+        }
+      }
+      if (i < L) p.lse[(size_t)bh * L + i] = lsum > 0.f ? (m2 + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TM_COLS);
+  }
+}
+
+// Per-call products for the tensor-core forward: Transformer-XL u.k_j and v.r_rho,
+// DeBERTa end-row products q_i.Kr[0], q_i.Kr[2k-1], k_j.Qr[0], k_j.Qr[2k-1].
+__global__ void tc_prep_kernel(Prm p, float *uk, float *vr, float *c2pE, float *p2cE) {
+  const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t rows = (size_t)p.B * p.H * p.L;
+  typedef __nv_bfloat16 bf;
+  if (p.mech == M_TXL) {
+    if (x < rows) {
+      const int h = (int)((x / p.L) % p.H);
+      const bf *k = (const bf *)p.k + x * HD, *u = (const bf *)p.rel1 + (size_t)h * HD;
+      float a = 0.f;
+      for (int c = 0; c < HD; ++c) a = fmaf(ldf(u, c), ldf(k, c), a);
+      uk[x] = a;
+    }
+    if (x < (size_t)p.H * p.nrows) {
+      const int h = (int)(x / p.nrows);
+      const bf *r = (const bf *)p.rel0 + x * HD, *v = (const bf *)p.rel2 + (size_t)h * HD;
+      float a = 0.f;
+      for (int c = 0; c < HD; ++c) a = fmaf(ldf(v, c), ldf(r, c), a);
+      vr[x] = a;
+    }
+  } else if (p.mech == M_DEB) {
+    if (x < rows) {
+      const int h = (int)((x / p.L) % p.H);
+      const bf *q = (const bf *)p.q + x * HD, *k = (const bf *)p.k + x * HD;
+      const bf *Kr = (const bf *)p.rel0 + (size_t)h * p.nrows * HD, *Qr = (const bf *)p.rel1 + (size_t)h * p.nrows * HD;
+      const size_t last = (size_t)(p.nrows - 1) * HD;
+      float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+      for (int c = 0; c < HD; ++c) {
+        const float qc = ldf(q, c), kc = ldf(k, c);
+        a0 = fmaf(qc, ldf(Kr, c), a0);
+        a1 = fmaf(qc, ldf(Kr, last + c), a1);
+        b0 = fmaf(kc, ldf(Qr, c), b0);
+        b1 = fmaf(kc, ldf(Qr, last + c), b1);
+      }
+      c2pE[2 * x] = a0;
+      c2pE[2 * x + 1] = a1;
+      p2cE[2 * x] = b0;
+      p2cE[2 * x + 1] = b1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)f;
+  }
+  return fn;
+}
+
+// [planes][rows][64] bf16 viewed as a 3D tensor; box = 64 x box_rows x 1, 128B swizzle,
+// rows outside [0, rows) read as zeros.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {64, rows, planes};
+  cuuint64_t strides[2] = {64 * 2, rows * 64 * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MECH>
+static cudaError_t launch_fwd_t(const FwdArgs &a, cudaStream_t st) {
+  auto k = tc_fwd_kernel<MECH>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.p.nT, a.p.H, a.p.B);
+  k<<<grid, NTHREADS, SMEM_BYTES, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+bool tc_supported(const Prm &p) {
+  if (p.mech == M_SHAW && 2 * p.clip + 1 > 131) return false;  // QA row must fit the 132-float smem row
+  return true;
+}
+
+cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st) {
+  using namespace tc;
+  FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.p = p;
+  a.p.nT = (p.L + BM - 1) / BM;  // 128-row tiles
+  a.uk = w.uk;
+  a.vr = w.vr;
+  a.c2pE = w.c2pE;
+  a.p2cE = w.p2cE;
+  const uint64_t BH = (uint64_t)p.B * p.H;
+  bool ok = make_map(&a.mq, p.q, p.L, BH, 128) && make_map(&a.mk, p.k, p.L, BH, 128) && make_map(&a.mv, p.v, p.L, BH, 128);
+  if (p.mech == M_TXL) ok = ok && make_map(&a.mt0, p.rel0, p.nrows, p.H, 128);
+  if (p.mech == M_SHAW) {
+    a.shaw_n = ((2 * p.clip + 1) + 15) / 16 * 16;
+    ok = ok && make_map(&a.mt0, p.rel0, p.nrows, p.H, a.shaw_n);
+  }
+  if (p.mech == M_DEB) ok = ok && make_map(&a.mt0, p.rel0, p.nrows, p.H, 256) && make_map(&a.mt1, p.rel1, p.nrows, p.H, 256);
+  if (!ok) return cudaErrorInvalidValue;
+  if (p.mech == M_TXL || p.mech == M_DEB) {
+    const size_t n = std::max((size_t)p.B * p.H * p.L, (size_t)p.H * p.nrows);
+    tc_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  switch (p.mech) {
+    case M_T5: return launch_fwd_t<M_T5>(a, st);
+    case M_SHAW: return launch_fwd_t<M_SHAW>(a, st);
+    case M_TXL: return launch_fwd_t<M_TXL>(a, st);
+    default: return launch_fwd_t<M_DEB>(a, st);
+  }
+}
+
+}  // namespace rp

@@ -138,10 +138,11 @@ RELPOS_API int relpos_attn_bwd(const relpos_params_t *params,
                     void *workspace, size_t workspace_bytes,
                     int32_t *dev_status, void *stream);
 
-/* Kernel family a call with these params runs: RELPOS_PATH_SIMT or
- * RELPOS_PATH_TC (RELPOS_PATH_AUTO resolved), or a negative RELPOS_ERR_* code
- * (RELPOS_ERR_UNSUPPORTED when RELPOS_PATH_TC is forced where it does not apply). */
-RELPOS_API int relpos_attn_resolved_path(const relpos_params_t *params);
+/* Kernel family that pass `pass` (0 forward, 1 backward) of a call with these
+ * params runs: RELPOS_PATH_SIMT or RELPOS_PATH_TC (RELPOS_PATH_AUTO resolved),
+ * or a negative RELPOS_ERR_* code (RELPOS_ERR_UNSUPPORTED when RELPOS_PATH_TC is
+ * forced where it does not apply). */
+RELPOS_API int relpos_attn_resolved_path(const relpos_params_t *params, int pass);
 
 /* Static, NUL-terminated description of a status code. */
 RELPOS_API const char *relpos_strerror(int status);

@@ -79,7 +79,11 @@ def test_workspace_sizes(lib):
             b = bd.relpos_attn_workspace_size(P, 1)
             assert b >= 2 * 3 * 1000 * 4  # at least D
             assert f % 256 == 0 and b % 256 == 0
-            assert (f > 0) == (mech == 0)
+            # forward scratch: T5's per-offset bias vector; on the bf16 tensor-core
+            # path also Transformer-XL's u.k / v.r and DeBERTa's end-row products
+            assert (f > 0) == (mech in (0, 2, 3))
+            f32 = bd.relpos_attn_workspace_size(bd.Params(mech=mech, B=2, H=3, L=1000, causal=causal, dtype=bd.F32), 0)
+            assert (f32 > 0) == (mech == 0)
     with pytest.raises(bd.RelposError):
         bd.relpos_attn_workspace_size(bd.Params(mech=1, B=1, H=1, L=8), 2)
 

@@ -30,22 +30,24 @@ def small_wl(mech, dtype, causal, L, B=2, H=2, **kw):
 # small shapes: several tiles and a ragged tail, every mechanism, both dtypes,
 # causal and not, on both kernel families
 # --------------------------------------------------------------------------
-SMALL_L = [1, 17, 64, 130, 257]
+SMALL_L = [1, 17, 64, 130, 257, 300, 700]
 
 
-@pytest.mark.parametrize("path", [bd.PATH_SIMT])
+@pytest.mark.parametrize("path", [bd.PATH_SIMT, bd.PATH_AUTO], ids=["simt", "auto"])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
 @pytest.mark.parametrize("mech", list(MECHS))
 @pytest.mark.parametrize("L", SMALL_L)
 def test_parity_small(mech, causal, dtype, L, path):
+    if path == bd.PATH_AUTO and dtype == torch.float32:
+        pytest.skip("float32 always runs the CUDA-core kernels")
     wl = small_wl(mech, dtype, causal, L)
     inp = make_inputs(wl, seed=L)
     out = run_gpu(wl, inp, path)
     compare_full(wl, inp, out)
 
 
-@pytest.mark.parametrize("path", [bd.PATH_SIMT])
+@pytest.mark.parametrize("path", [bd.PATH_SIMT, bd.PATH_AUTO], ids=["simt", "auto"])
 def test_parity_deberta_span256(path):
     wl = Workload("deb600", DEBERTA, torch.bfloat16, False, 1, 2, 600)
     inp = make_inputs(wl, 3)
