@@ -1,15 +1,16 @@
 // Tensor-core (tcgen05 / TMEM / TMA) forward kernel of relative-position
 // attention for bf16 inputs, d = 64, on sm_100a.
 //
-// One CTA per 128-row query tile (heaviest causal tiles launched first), five
+// One CTA per 128-row query tile (heaviest causal tiles launched first), nine
 // warps:
-//   warps 0-3  "softmax": thread t owns query row t (TMEM lane t).  It reads its
-//              row of S = Q K^T and of the relation products from TMEM, adds the
-//              relative term gathered by offset, runs the online softmax (lazy
-//              rescale of O only when the running max grows by more than 2^8),
-//              and writes P (bf16) into shared memory in the 128-byte-swizzled
-//              layout the tensor core reads.
-//   warp 4     lane 0 issues every TMA load (Q, K, V, relation-table windows,
+//   warps 0-7  "softmax": two threads per query row (warps w and w + 4 share TMEM
+//              lanes 32 (w & 3)..+31 and take key columns [0, 64) and [64, 128)).
+//              They read S = Q K^T and the relation products from TMEM, add the
+//              relative term gathered by offset, run the online softmax (row max
+//              exchanged through smem; lazy rescale of O only when the running max
+//              grows by more than 2^8), and write P (bf16) into shared memory in the
+//              128-byte-swizzled layout the tensor core reads.
+//   warp 8     lane 0 issues every TMA load (Q, K, V, relation-table windows,
 //              2-stage K/V ring) and every tcgen05.mma, and signals through
 //              mbarriers and tcgen05.commit.
 // TMEM (512 columns): S [0,128), relation products [128,384), O [384,448).
@@ -38,7 +39,8 @@ namespace rp {
 namespace tc {
 
 constexpr int BM = 128, BN = 128;
-constexpr int NTHREADS = 160;
+constexpr int NSOFT = 256;    // softmax threads: two per query row
+constexpr int NTHREADS = NSOFT + 32;
 constexpr int ROT_LD = 132;  // fp32 stride of the per-row skew buffer (conflict-free rotations)
 
 constexpr int OFF_Q = 0;
@@ -48,7 +50,8 @@ constexpr int OFF_P = OFF_V + 32768;    // two 64-key halves of P
 constexpr int OFF_R = OFF_P + 32768;    // relation-table staging (2 x 16 KB or one 32 KB window)
 constexpr int OFF_ROT = OFF_R + 32768;  // 128 x ROT_LD fp32
 constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;  // 2 x 512 fp32 per-tile vectors
-constexpr int OFF_BAR = OFF_VEC + 2 * 512 * 4;
+constexpr int OFF_RED = OFF_VEC + 2 * 512 * 4;  // 2 x 256 fp32 row-max exchange
+constexpr int OFF_BAR = OFF_RED + 2 * 256 * 4;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 
@@ -102,14 +105,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     mbar_init(BAR(B_KV0), 1);
     mbar_init(BAR(B_KV1), 1);
     mbar_init(BAR(B_SFULL), 1);
-    mbar_init(BAR(B_SFREE), 128);
-    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_SFREE), NSOFT);
+    mbar_init(BAR(B_PFULL), NSOFT);
     mbar_init(BAR(B_PV), 1);
     mbar_init(BAR(B_PLOAD), 1);
     mbar_init(BAR(B_PFULLPRO), 1);
-    mbar_init(BAR(B_PFREEPRO), 128);
+    mbar_init(BAR(B_PFREEPRO), NSOFT);
     mbar_init(BAR(B_RLOAD), 1);
-    mbar_init(BAR(B_RFREE), 128);
+    mbar_init(BAR(B_RFREE), NSOFT);
     mbar_init(BAR(B_GFULL), 1);
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   int32_t *status = p.status;
   const float c1 = p.scale * 1.4426950408889634f;  // scale * log2(e)
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ======================= TMA + MMA issuer ==========================
     if (lane == 0) {
       prefetch_tmap(&A.mq);
@@ -264,9 +267,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     __syncwarp();
   } else {
     // ========================== softmax warps ===========================
-    const int il = tid, i = i0 + il;
-    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+    // warp w: TMEM lanes 32 (w & 3) .. +31 (query rows), key columns [64 hf, 64 hf + 64), hf = w >> 2
+    const int g = warp & 3, hf = warp >> 2;
+    const int il = 32 * g + lane, i = i0 + il;
+    const int cb = 64 * hf;  // first key column of this thread
+    const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
+    float *red = (float *)(smem + OFF_RED);
     float m2 = -INFINITY, lsum = 0.f;
     float cE0 = 0.f, cE1 = 0.f;
     bool good = true;  // warp-uniform: false once any wait of the CTA ran out
@@ -274,12 +281,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       cE0 = A.c2pE[((size_t)bh * L + i) * 2 + 0];
       cE1 = A.c2pE[((size_t)bh * L + i) * 2 + 1];
     }
-    if (MECH == M_SHAW) {  // QA row -> smem (kept for the whole CTA)
+    if (MECH == M_SHAW) {  // QA row -> smem (kept for the whole CTA); 32-column chunks split by parity
       good = warp_wait(BAR(B_PFULLPRO), 0, abort_flag, status);
       if (good) {
         tc_fence_after();
         const int nq = (2 * p.clip + 1 + 31) / 32;
-        for (int q = 0; q < nq; ++q) {
+        for (int q = hf; q < nq; q += 2) {
           uint32_t r[32];
           tmem_ld32(tl + TM_REL + 32 * q, r);
           tmem_wait_ld();
@@ -290,80 +297,81 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         tc_fence_before();
         mbar_arrive(BAR(B_PFREEPRO));
       }
+      named_bar_sync(1, NSOFT);
     }
     int band_cnt = 0;
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * BN, Delta = m - n;
       float *tv = vec + 512 * (n & 1);
-      // ---- per-tile vectors (shared by the four softmax warps) ----
+      // ---- per-tile vectors (one element per softmax thread) ----
       if (MECH == M_TXL) {
-        const int j = j0 + il;
-        tv[il] = (j < L) ? A.uk[(size_t)bh * L + j] : 0.f;
-        const int ra = 128 * Delta + il + p.off, rb = 128 * (Delta - 1) + il + p.off;
-        tv[128 + il] = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
-        tv[256 + il] = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
-      } else if (MECH == M_T5) {
-        const int dmin = j0 - i0 - 127;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int w = il + 128 * k;
-          const int idx = dmin + w + L - 1;
-          if (w < 255) tv[w] = (idx >= 0 && idx < 2 * L - 1) ? p.t5_bias[(size_t)h * (2 * L - 1) + idx] : 0.f;
+        if (tid < 128) {
+          const int j = j0 + tid;
+          tv[tid] = (j < L) ? A.uk[(size_t)bh * L + j] : 0.f;
         }
+        const int rr = 128 * (tid < 128 ? Delta : Delta - 1) + (tid & 127) + p.off;
+        tv[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+      } else if (MECH == M_T5) {
+        const int idx = j0 - i0 - 127 + tid + L - 1;
+        if (tid < 255) tv[tid] = (idx >= 0 && idx < 2 * L - 1) ? p.t5_bias[(size_t)h * (2 * L - 1) + idx] : 0.f;
       } else if (MECH == M_DEB) {
-        const int j = j0 + il;
-        tv[2 * il] = (j < L) ? A.p2cE[((size_t)bh * L + j) * 2] : 0.f;
-        tv[2 * il + 1] = (j < L) ? A.p2cE[((size_t)bh * L + j) * 2 + 1] : 0.f;
+        const int j = j0 + (tid >> 1);
+        tv[tid] = (j < L) ? A.p2cE[((size_t)bh * L + j) * 2 + (tid & 1)] : 0.f;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
-      float x[128];
+      float x[64];
       if (good) {
         tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           uint32_t r[32];
-          tmem_ld32(tl + TM_S + 32 * q, r);
+          tmem_ld32(tl + TM_S + cb + 32 * q, r);
           tmem_wait_ld();
 #pragma unroll
           for (int t = 0; t < 32; ++t) x[32 * q + t] = u2f(r[t]);
         }
       } else {
 #pragma unroll
-        for (int jl = 0; jl < 128; ++jl) x[jl] = 0.f;
+        for (int t = 0; t < 64; ++t) x[t] = 0.f;
       }
       // ---- relative term, gathered by offset ----
       if (MECH == M_TXL) {
         if (good) {
+          // this thread rotates offsets c in [cb, cb + 64) of its row into key order
           const bool hasB = !(p.causal && Delta == 0);
           const uint32_t colA = TM_REL + 128 * (Delta & 1), colB = TM_REL + 128 * ((Delta - 1) & 1);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             uint32_t ra[32], rb[32];
-            tmem_ld32(tl + colA + 32 * q, ra);
-            if (hasB) tmem_ld32(tl + colB + 32 * q, rb);
+            tmem_ld32(tl + colA + cb + 32 * q, ra);
+            if (hasB) {
+              tmem_ld32(tl + colB + cb + 32 * q, rb);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) rb[t] = 0u;
+            }
             tmem_wait_ld();
 #pragma unroll
             for (int t = 0; t < 32; ++t) {
-              const int c = 32 * q + t;
-              float val;
-              if (c <= il)
-                val = u2f(ra[t]) + tv[128 + c];
-              else
-                val = hasB ? u2f(rb[t]) + tv[256 + c] : 0.f;
-              rrow[(il - c) & 127] = val;
+              const int c = cb + 32 * q + t;
+              const float va = u2f(ra[t]) + tv[128 + c];
+              const float vb = hasB ? u2f(rb[t]) + tv[256 + c] : 0.f;
+              rrow[(il - c) & 127] = (c <= il) ? va : vb;
             }
           }
           tc_fence_before();
           mbar_arrive(BAR(B_SFREE));
         }
+        named_bar_sync(1, NSOFT);
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
-          const float4 rr = *reinterpret_cast<const float4 *>(rrow + 4 * c4);
-          x[4 * c4 + 0] = (x[4 * c4 + 0] + rr.x + tv[4 * c4 + 0]) * c1;
-          x[4 * c4 + 1] = (x[4 * c4 + 1] + rr.y + tv[4 * c4 + 1]) * c1;
-          x[4 * c4 + 2] = (x[4 * c4 + 2] + rr.z + tv[4 * c4 + 2]) * c1;
-          x[4 * c4 + 3] = (x[4 * c4 + 3] + rr.w + tv[4 * c4 + 3]) * c1;
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
+          const float4 uk = *reinterpret_cast<const float4 *>(tv + cb + 4 * c4);
+          x[4 * c4 + 0] = (x[4 * c4 + 0] + rr.x + uk.x) * c1;
+          x[4 * c4 + 1] = (x[4 * c4 + 1] + rr.y + uk.y) * c1;
+          x[4 * c4 + 2] = (x[4 * c4 + 2] + rr.z + uk.z) * c1;
+          x[4 * c4 + 3] = (x[4 * c4 + 3] + rr.w + uk.w) * c1;
         }
       } else if (MECH == M_T5) {
         if (good) {
@@ -371,29 +379,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           mbar_arrive(BAR(B_SFREE));
         }
         const float lg = 1.4426950408889634f;
+        const float *bw = tv + cb - il + 127;
 #pragma unroll
-        for (int jl = 0; jl < 128; ++jl) x[jl] = x[jl] * c1 + tv[jl - il + 127] * lg;
+        for (int t = 0; t < 64; ++t) x[t] = x[t] * c1 + bw[t] * lg;
       } else if (MECH == M_SHAW) {
         if (good) {
           tc_fence_before();
           mbar_arrive(BAR(B_SFREE));
         }
-        const int d0 = j0 - i;
+        const int d0 = j0 + cb - i;
 #pragma unroll
-        for (int jl = 0; jl < 128; ++jl) x[jl] = (x[jl] + rrow[iclamp(d0 + jl, -p.clip, p.clip) + p.clip]) * c1;
+        for (int t = 0; t < 64; ++t) x[t] = (x[t] + rrow[iclamp(d0 + t, -p.clip, p.clip) + p.clip]) * c1;
       } else {  // DeBERTa
         const bool band = 128 * (Delta < 0 ? -Delta : Delta) - 127 < p.span;
         if (band) {
+          // c2p: window column w (Kr row lo + w) belongs to key il + 127 - w; this
+          // thread handles w in [128 hf, 128 hf + 128)
           if (good) {
-            const int lo = p.span + 128 * Delta - 127;  // unclipped Kr row of window column 0
+            const int lo = p.span + 128 * Delta - 127;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
               uint32_t r[32];
-              tmem_ld32(tl + TM_REL + 32 * q, r);
+              tmem_ld32(tl + TM_REL + 128 * hf + 32 * q, r);
               tmem_wait_ld();
 #pragma unroll
               for (int t = 0; t < 32; ++t) {
-                const int w = 32 * q + t;  // pair (il, jl) with jl = il + 127 - w
+                const int w = 128 * hf + 32 * q + t;
                 if (w >= il && w <= il + 127) {
                   const int rho = lo + w;
                   rrow[il + 127 - w] = (rho < 0) ? cE0 : (rho > 2 * p.span - 1 ? cE1 : u2f(r[t]));
@@ -402,25 +413,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             }
             tc_fence_before();
             mbar_arrive(BAR(B_RFREE));
-#pragma unroll
-            for (int jl = 0; jl < 128; ++jl) x[jl] += rrow[jl];
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1, NSOFT);
+#pragma unroll
+          for (int t = 0; t < 64; ++t) x[t] += rrow[cb + t];
+          named_bar_sync(1, NSOFT);
           good = good && warp_wait(BAR(B_GFULL), band_cnt & 1, abort_flag, status);
           ++band_cnt;
           if (good) {
             tc_fence_after();
-            // this thread is key jl = il of the tile: TMEM lane il holds K_j . Qr_win
-            const int lo2 = p.span - 128 * Delta - 127;  // unclipped Qr row of window column 0
+            // TMEM lane il now holds key il of the tile: K_j . Qr_win; window column w
+            // belongs to query il + 127 - w
+            const int lo2 = p.span - 128 * Delta - 127;
             const float e0 = tv[2 * il], e1 = tv[2 * il + 1];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
               uint32_t r[32];
-              tmem_ld32(tl + TM_REL + 32 * q, r);
+              tmem_ld32(tl + TM_REL + 128 * hf + 32 * q, r);
               tmem_wait_ld();
 #pragma unroll
               for (int t = 0; t < 32; ++t) {
-                const int w = 32 * q + t;  // pair (query il + 127 - w, key il)
+                const int w = 128 * hf + 32 * q + t;
                 if (w >= il && w <= il + 127) {
                   const int rho = lo2 + w;
                   rot[(il + 127 - w) * ROT_LD + il] = (rho < 0) ? e0 : (rho > 2 * p.span - 1 ? e1 : u2f(r[t]));
@@ -430,9 +443,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             tc_fence_before();
             mbar_arrive(BAR(B_SFREE));
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1, NSOFT);
 #pragma unroll
-          for (int jl = 0; jl < 128; ++jl) x[jl] = (x[jl] + rrow[jl]) * c1;
+          for (int t = 0; t < 64; ++t) x[t] = (x[t] + rrow[cb + t]) * c1;
         } else {
           if (good) {
             tc_fence_before();
@@ -441,93 +454,97 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           const float c2p = Delta > 0 ? cE1 : cE0;
           const int sel = Delta < 0 ? 1 : 0;
 #pragma unroll
-          for (int jl = 0; jl < 128; ++jl) x[jl] = (x[jl] + c2p + tv[2 * jl + sel]) * c1;
+          for (int t = 0; t < 64; ++t) x[t] = (x[t] + c2p + tv[2 * (cb + t) + sel]) * c1;
         }
       }
-      // ---- mask, online softmax (base 2, lazy rescale) ----
+      // ---- mask (diagonal / ragged tiles only), row max over both halves ----
+      const bool need_mask = (p.causal && n == m) || (j0 + BN > L);
       float mt = -INFINITY;
+      if (need_mask) {
 #pragma unroll
-      for (int jl = 0; jl < 128; ++jl) {
-        const int j = j0 + jl;
-        if (j >= L || (p.causal && j > i)) x[jl] = -INFINITY;
-        mt = fmaxf(mt, x[jl]);
+        for (int t = 0; t < 64; ++t) {
+          const int j = j0 + cb + t;
+          if (j >= L || (p.causal && j > i)) x[t] = -INFINITY;
+          mt = fmaxf(mt, x[t]);
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < 64; ++t) mt = fmaxf(mt, x[t]);
       }
+      float *rd = red + 256 * (n & 1);
+      rd[128 * hf + il] = mt;
+      named_bar_sync(1, NSOFT);
+      mt = fmaxf(rd[il], rd[128 + il]);
       if (n == 0) {
         m2 = mt;
       } else {
-        const bool need = mt > m2 + 8.f;
+        const bool need = mt > m2 + 8.f;  // identical in both threads of the row
         if (__any_sync(0xffffffffu, need)) {
           good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
+          const float alpha = need ? ex2(m2 - mt) : 1.f;
           if (good) {
             tc_fence_after();
-            const float alpha = need ? ex2(m2 - mt) : 1.f;
+            uint32_t r[32];
+            tmem_ld32(tl + TM_O + 32 * hf, r);
+            tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              uint32_t r[32];
-              tmem_ld32(tl + TM_O + 32 * q, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(u2f(r[t]) * alpha);
-              tmem_st32(tl + TM_O + 32 * q, r);
-            }
+            for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(u2f(r[t]) * alpha);
+            tmem_st32(tl + TM_O + 32 * hf, r);
             tmem_wait_st();
           }
           if (need) {
-            lsum *= ex2(m2 - mt);
+            lsum *= alpha;
             m2 = mt;
           }
         }
       }
       const float msub = (m2 == -INFINITY) ? 0.f : m2;
 #pragma unroll
-      for (int jl = 0; jl < 128; ++jl) {
-        x[jl] = ex2(x[jl] - msub);
-        lsum += x[jl];
+      for (int t = 0; t < 64; ++t) {
+        x[t] = ex2(x[t] - msub);
+        lsum += x[t];
       }
       if (n >= 1) good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
       if (good) {
-        // P row -> smem, K-major 128B swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
+        // P half-row -> smem sub-tile hf, K-major 128B swizzle: chunk c of row r at chunk c ^ (r & 7)
 #pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int j8 = 64 * kb + 8 * ch;
-            uint4 v;
-            v.x = pack_bf16x2(x[j8 + 0], x[j8 + 1]);
-            v.y = pack_bf16x2(x[j8 + 2], x[j8 + 3]);
-            v.z = pack_bf16x2(x[j8 + 4], x[j8 + 5]);
-            v.w = pack_bf16x2(x[j8 + 6], x[j8 + 7]);
-            *reinterpret_cast<uint4 *>(smem + OFF_P + 16384 * kb + 128 * il + ((ch ^ (il & 7)) << 4)) = v;
-          }
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 v;
+          v.x = pack_bf16x2(x[8 * ch + 0], x[8 * ch + 1]);
+          v.y = pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]);
+          v.z = pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]);
+          v.w = pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]);
+          *reinterpret_cast<uint4 *>(smem + OFF_P + 16384 * hf + 128 * il + ((ch ^ (il & 7)) << 4)) = v;
+        }
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PFULL));
       }
     }
-    // ---- epilogue: O / l, LSE ----
+    // ---- epilogue: O / l (l summed over the two halves), LSE ----
+    red[256 * (nTiles & 1) + 128 * hf + il] = lsum;
+    named_bar_sync(1, NSOFT);
+    const float ltot = red[256 * (nTiles & 1) + il] + red[256 * (nTiles & 1) + 128 + il];
     good = good && warp_wait(BAR(B_PV), (nTiles - 1) & 1, abort_flag, status);
     if (good) {
       tc_fence_after();
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      __nv_bfloat16 *orow = (__nv_bfloat16 *)p.out + ((size_t)bh * L + i) * HD;
+      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+      __nv_bfloat16 *orow = (__nv_bfloat16 *)p.out + ((size_t)bh * L + i) * HD + 32 * hf;
+      uint32_t r[32];
+      tmem_ld32(tl + TM_O + 32 * hf, r);
+      tmem_wait_ld();
+      if (i < L) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t r[32];
-        tmem_ld32(tl + TM_O + 32 * q, r);
-        tmem_wait_ld();
-        if (i < L) {
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint4 v;
-            v.x = pack_bf16x2(u2f(r[8 * c8 + 0]) * inv, u2f(r[8 * c8 + 1]) * inv);
-            v.y = pack_bf16x2(u2f(r[8 * c8 + 2]) * inv, u2f(r[8 * c8 + 3]) * inv);
-            v.z = pack_bf16x2(u2f(r[8 * c8 + 4]) * inv, u2f(r[8 * c8 + 5]) * inv);
-            v.w = pack_bf16x2(u2f(r[8 * c8 + 6]) * inv, u2f(r[8 * c8 + 7]) * inv);
-            *reinterpret_cast<uint4 *>(orow + 32 * q + 8 * c8) = v;
-          }
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint4 v;
+          v.x = pack_bf16x2(u2f(r[8 * c8 + 0]) * inv, u2f(r[8 * c8 + 1]) * inv);
+          v.y = pack_bf16x2(u2f(r[8 * c8 + 2]) * inv, u2f(r[8 * c8 + 3]) * inv);
+          v.z = pack_bf16x2(u2f(r[8 * c8 + 4]) * inv, u2f(r[8 * c8 + 5]) * inv);
+          v.w = pack_bf16x2(u2f(r[8 * c8 + 6]) * inv, u2f(r[8 * c8 + 7]) * inv);
+          *reinterpret_cast<uint4 *>(orow + 8 * c8) = v;
         }
+        if (hf == 0) p.lse[(size_t)bh * L + i] = ltot > 0.f ? (m2 + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
       }
-      if (i < L) p.lse[(size_t)bh * L + i] = lsum > 0.f ? (m2 + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
     }
     tc_fence_before();
   }
