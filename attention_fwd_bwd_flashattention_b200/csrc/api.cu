@@ -128,14 +128,15 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
-  if (pass == 1) return false;  // the backward pass runs on the CUDA-core kernels
+  if (pass == 1) return p.mech == rp::M_TXL;  // other mechanisms: CUDA-core backward
   return rp::tc_supported(p);
 }
 
 // ---- workspace layout ------------------------------------------------------
 struct Layout {
   size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot;
-  size_t uk, vr, c2pE, p2cE;  // tensor-core forward products
+  size_t uk, vr, c2pE, p2cE;  // tensor-core products
+  size_t part_kv, part_dg;    // tensor-core backward partials
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -164,7 +165,16 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
       l.p2cE = take(sizeof(float) * BH * p.L * 2);
     }
   }
-  if (pass == 1) {
+  if (pass == 1 && tc) {  // tensor-core backward (Transformer-XL)
+    size_t kvf = 0;
+    const size_t dgf = rp::tc_bwd_part_floats(p, kvf);
+    l.dvec = take(sizeof(float) * BH * p.L);
+    l.uk = take(sizeof(float) * BH * p.L);
+    l.vr = take(sizeof(float) * (size_t)p.H * p.nrows);
+    l.part_kv = take(sizeof(float) * kvf);
+    l.part_dg = take(sizeof(float) * dgf);
+    l.gtot = take(sizeof(float) * (size_t)p.H * p.nrows);
+  } else if (pass == 1) {
     l.dvec = take(sizeof(float) * BH * p.L);
     const size_t tab = (size_t)p.nrows * rp::HD;
     switch (p.mech) {
@@ -206,6 +216,8 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.vr = (float *)(b + l.vr);
   w.c2pE = (float *)(b + l.c2pE);
   w.p2cE = (float *)(b + l.p2cE);
+  w.part_kv = (float *)(b + l.part_kv);
+  w.part_dg = (float *)(b + l.part_dg);
   return w;
 }
 
@@ -298,6 +310,12 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   p.status = dev_status;
   cudaStream_t st = (cudaStream_t)stream;
   const bool bf16 = params->dtype == RELPOS_BF16;
+  if (tc) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(rel[0]))
+      return RELPOS_ERR_INVALID_ARG;
+    if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;
+    return to_status(rp::tc_bwd(p, tc_work(l, workspace), st));
+  }
   if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
   return to_status(rp::simt_bwd(p, bf16, st));
 }

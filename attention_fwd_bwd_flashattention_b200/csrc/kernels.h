@@ -11,7 +11,12 @@ cudaError_t simt_bwd(const Prm &p, bool bf16, cudaStream_t st);
 // tensor-core (bf16) path
 struct TcWork {
   float *uk, *vr, *c2pE, *p2cE;  // per-call products (Transformer-XL, DeBERTa)
+  float *part_kv, *part_dg;      // backward partials (Transformer-XL)
 };
 bool tc_supported(const Prm &p);
+cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st);
 cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st);
+cudaError_t tc_bwd(const Prm &p, const TcWork &w, cudaStream_t st);
+size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats);
+cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st);
 }  // namespace rp

@@ -864,6 +864,15 @@ __global__ void t5_prep_kernel(Prm p) {
   for (int h = 0; h < p.H; ++h) p.t5_bias[(size_t)h * n + x] = t[h * p.nb + bk];
 }
 
+cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st) {
+  const size_t rows = (size_t)p.B * p.H * p.L;
+  if (bf16)
+    simt::dvec_kernel<__nv_bfloat16><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+  else
+    simt::dvec_kernel<float><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_t5_prep(const Prm &p, cudaStream_t st) {
   const int n = 2 * p.L - 1;
   t5_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(p);

@@ -1,0 +1,1036 @@
+// Tensor-core (tcgen05 / TMEM / TMA) backward pass of Transformer-XL relative
+// attention, bf16, d = 64, sm_100a.  No atomics anywhere.
+//
+// Three kernels share one per-tile engine: two threads per query row (warps w and
+// w + 4 share TMEM lanes 32 (w & 3)..+31 and take key columns [0,64) / [64,128));
+// warp 8 lane 0 issues every TMA load and tcgen05.mma.  For a 128 x 128 tile
+// (query tile m, key tile n, Delta = m - n) the offsets are i - j = 128 Delta +
+// [-127, 127], i.e. the two 128-offset blocks Delta and Delta - 1 of r; the rows
+// recompute S = s((q + u).k + (q + v).r) exactly as the forward does (relation
+// products by MMA, rotated into key order through a padded smem row), then
+// P = exp(S - LSE), dP = dO V^T, dS = P (dP - D) with D = rowsum(dO o O).
+//
+//   key-tile kernel   (one CTA per key tile n, query tiles streamed):
+//                     dV += P^T dO, dK += dS^T Q, c += dS^T 1 (column sums of dS),
+//                     all with P / dS from smem as MN-major A operands; at the end
+//                     dK += c u^T and a du partial sum_j c_j k_j.
+//   query-tile kernel (one CTA per query tile m, key tiles streamed; the relation
+//                     blocks are reused across key tiles as in the forward):
+//                     dQ += dS K_n (dS as the TMEM A operand) + E_lo r_Delta +
+//                     E_hi r_{Delta-1}, where E is dS moved into offset
+//                     coordinates (E[i][c] = dS[i][i - c] by block).
+//   diagonal kernel   (one CTA per chunk of a diagonal band Delta): every tile of
+//                     the band reads the same two offset blocks, so the CTA keeps
+//                     G += E^T Q and g += E^T 1 for both blocks in TMEM and writes one
+//                     partial per chunk ("offset-based gradient sharding",
+//                     "Fast and Exact Relative-Position Attention via Structure-Aware
+//                     Kernels", Abstract, technique (3)).
+// A fixed-order reduction turns the partials into dr = s (G + g v), dv = s sum g r
+// and du = s sum_j c_j k_j.
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace rp {
+namespace tcb {
+
+using namespace tc;
+
+constexpr int NSOFT = 256;
+constexpr int NTHREADS = NSOFT + 32;
+constexpr int ROT_LD = 132;
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct BwdArgs {
+  CUtensorMap mq, mk, mv, mdo, mr;
+  Prm p;                 // nT counts 128-row tiles
+  const float *uk, *vr;  // u.k_j [B,H,L], v.r_rho [H,rows]
+  float *part_kv;        // [B,H,nT][64]  du partial per key tile
+  float *part_dg;        // [B,H,nbands,nchunk][2][128][65] diagonal partials (G then g)
+  int dg_ch, dg_nchunk, nbands;
+};
+
+constexpr int DG_STRIDE = 2 * 128 * 65;
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *ab, int32_t *st) {
+  const bool ok = mbar_wait(bar, parity, ab, st, RELPOS_ERR_TIMEOUT_DEV);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Control-thread bookkeeping: TMA loads issued but not waited for are drained on exit.
+struct Ctl {
+  uint32_t pb[8], pp[8];
+  int np;
+  volatile int *ab;
+  int32_t *st;
+  __device__ void expect(uint32_t bar, uint32_t par, uint32_t bytes) {
+    mbar_expect_tx(bar, bytes);
+    pb[np] = bar;
+    pp[np] = par;
+    ++np;
+  }
+  __device__ bool wait(uint32_t bar, uint32_t par) { return mbar_wait(bar, par, ab, st, RELPOS_ERR_TIMEOUT_DEV); }
+  __device__ bool wait_load(uint32_t bar, uint32_t par) {
+    if (!wait(bar, par)) return false;
+    for (int e = 0; e < np; ++e)
+      if (pb[e] == bar && pp[e] == par) {
+        pb[e] = pb[np - 1];
+        pp[e] = pp[np - 1];
+        --np;
+        break;
+      }
+    return true;
+  }
+  __device__ void drain(uint32_t drain_bar) {
+    umma_commit(drain_bar);
+    volatile int none = 0;
+    mbar_wait(drain_bar, 0, &none, st, RELPOS_ERR_TIMEOUT_DEV);
+    for (int e = 0; e < np; ++e) mbar_wait(pb[e], pp[e], &none, st, RELPOS_ERR_TIMEOUT_DEV);
+  }
+};
+
+// 64 values of row il, columns [64 hf, 64 hf + 64) of a 128 x 128 bf16 tile kept as
+// two 128B-swizzled 64-column sub-tiles.
+__device__ __forceinline__ void store_half_row(uint8_t *tile, int il, int hf, const float (&v)[64]) {
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]);
+    w.y = pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]);
+    w.z = pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]);
+    w.w = pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]);
+    *reinterpret_cast<uint4 *>(tile + 16384 * hf + 128 * il + ((ch ^ (il & 7)) << 4)) = w;
+  }
+}
+__device__ __forceinline__ void store_elem(uint8_t *tile, int r, int c, float x) {
+  *reinterpret_cast<__nv_bfloat16 *>(tile + 16384 * (c >> 6) + 128 * r + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1)) =
+      __float2bfloat16_rn(x);
+}
+
+// Rotate offsets c in [cb, cb + 64) of the two relation blocks (TMEM columns colA,
+// colB of this warp's lanes) into key order: rrow[(il - c) & 127] gets block Delta
+// for c <= il, block Delta - 1 otherwise, plus the per-offset v.r term.
+__device__ __forceinline__ void txl_rotate(uint32_t tl, uint32_t colA, uint32_t colB, bool hasB, int il, int cb,
+                                           const float *vA, const float *vB, float *rrow) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    uint32_t ra[32], rb[32];
+    tmem_ld32(tl + colA + cb + 32 * q, ra);
+    if (hasB) {
+      tmem_ld32(tl + colB + cb + 32 * q, rb);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) rb[t] = 0u;
+    }
+    tmem_wait_ld();
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const int c = cb + 32 * q + t;
+      const float va = u2f(ra[t]) + vA[c];
+      const float vb = hasB ? u2f(rb[t]) + vB[c] : 0.f;
+      rrow[(il - c) & 127] = (c <= il) ? va : vb;
+    }
+  }
+}
+
+// Offset block b of r (rows 128 b + off .. +127) exists unless causal and b < 0.
+__device__ __forceinline__ bool block_valid(const Prm &p, int b) { return !(p.causal && b < 0); }
+__device__ __forceinline__ int slot3(int b) { return ((b % 3) + 3) % 3; }
+
+// ============================================================================
+// key-tile kernel: dK, dV, column sums of dS
+// ============================================================================
+namespace kv {
+constexpr int OFF_K = 0, OFF_V = 16384, OFF_Q = 32768, OFF_DO = OFF_Q + 32768, OFF_R = OFF_DO + 32768;
+constexpr int OFF_ROT = OFF_R + 3 * 16384;            // rot rows; P tile at +0, dS tile at +32768
+constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;  // [16][128] bf16 ones, K-major (2 x 2 KB)
+constexpr int OFF_VEC = OFF_ONES + 4096;              // uk[128] + vr[2][256]
+constexpr int OFF_BAR = OFF_VEC + 4096;
+constexpr int SMEM = OFF_BAR + 256 + 1024;
+enum { B_KV = 0, B_ST0, B_ST1, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
+constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320, T_CS = 384;
+}  // namespace kv
+
+__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_constant__ BwdArgs A) {
+  using namespace kv;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Prm &p = A.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, bh = b * p.H + h;
+  const int L = p.L, j0 = n * 128;
+  const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
+  const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NB);
+  float *rot = (float *)(smem + OFF_ROT);
+  float *vec = (float *)(smem + OFF_VEC);
+  int32_t *status = p.status;
+  const float c1 = p.scale * LOG2E;
+
+  if (tid == 0) {
+    mbar_init(BAR(B_KV), 1);
+    mbar_init(BAR(B_ST0), 1);
+    mbar_init(BAR(B_ST1), 1);
+    mbar_init(BAR(B_TFULL), 1);
+    mbar_init(BAR(B_TCONS), NSOFT);
+    mbar_init(BAR(B_SDP), 1);
+    mbar_init(BAR(B_PDS), NSOFT);
+    mbar_init(BAR(B_PDSFREE), 1);
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  // all-ones B operand for the column sums (any swizzle of all-ones is all-ones)
+  for (int x = tid; x < 4096 / 16; x += NTHREADS) {
+    const uint32_t one2 = 0x3F803F80u;
+    *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
+  }
+  if (tid < 128) vec[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+  fence_async_smem();
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      Ctl ctl;
+      ctl.np = 0;
+      ctl.ab = abort_flag;
+      ctl.st = status;
+      prefetch_tmap(&A.mq);
+      prefetch_tmap(&A.mk);
+      prefetch_tmap(&A.mv);
+      prefetch_tmap(&A.mdo);
+      prefetch_tmap(&A.mr);
+      const uint32_t idS = idesc_bf16(128, 128, false);
+      const uint32_t idAcc = idesc_bf16(128, 64, true, true);
+      const uint32_t idCs = idesc_bf16(128, 16, false, true);
+      ctl.expect(BAR(B_KV), 0, 32768);
+      tma_load_3d(sbase + OFF_K, &A.mk, BAR(B_KV), 0, j0, bh);
+      tma_load_3d(sbase + OFF_V, &A.mv, BAR(B_KV), 0, j0, bh);
+      auto issue_stage = [&](int t) {
+        const int m = mStart + t, D = m - n, st = t & 1;
+        const bool bA = block_valid(p, D), bB = (t == 0) && block_valid(p, D - 1);
+        ctl.expect(BAR(B_ST0 + st), (uint32_t)((t >> 1) & 1), 32768u + (bA ? 16384u : 0u) + (bB ? 16384u : 0u));
+        tma_load_3d(sbase + OFF_Q + 16384 * st, &A.mq, BAR(B_ST0 + st), 0, m * 128, bh);
+        tma_load_3d(sbase + OFF_DO + 16384 * st, &A.mdo, BAR(B_ST0 + st), 0, m * 128, bh);
+        if (bA) tma_load_3d(sbase + OFF_R + 16384 * slot3(D), &A.mr, BAR(B_ST0 + st), 0, 128 * D + p.off, h);
+        if (bB) tma_load_3d(sbase + OFF_R + 16384 * slot3(D - 1), &A.mr, BAR(B_ST0 + st), 0, 128 * (D - 1) + p.off, h);
+      };
+      auto accumulate = [&](int t) {  // dV, dK, column sums of tile t (P, dS in smem)
+        const int st = t & 1;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
+          umma_bf16(tbase + T_DV, sdesc_sw128(sbase + OFF_ROT + 2048 * k, 16384, 1024),
+                    sdesc_sw128(sbase + OFF_DO + 16384 * st + 2048 * k, 16, 1024), idAcc, acc);
+          umma_bf16(tbase + T_DK, sdesc_sw128(sbase + OFF_ROT + 32768 + 2048 * k, 16384, 1024),
+                    sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, 16, 1024), idAcc, acc);
+          umma_bf16(tbase + T_CS, sdesc_sw128(sbase + OFF_ROT + 32768 + 2048 * k, 16384, 1024),
+                    sdesc_sw128(sbase + OFF_ONES + 2048 * (k >> 2) + 32 * (k & 3), 16, 1024), idCs, acc);
+        }
+        umma_commit(BAR(B_PDSFREE));
+      };
+      issue_stage(0);
+      if (iters > 1) issue_stage(1);
+      bool ok = true;
+      for (int t = 0; ok && t < iters; ++t) {
+        const int m = mStart + t, D = m - n, st = t & 1;
+        if (!ctl.wait_load(BAR(B_ST0 + st), (t >> 1) & 1)) break;
+        if (t == 0 && !ctl.wait_load(BAR(B_KV), 0)) break;
+        if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
+        tc_fence_after();
+        if (block_valid(p, D)) umma_k64(tbase + 0, sbase + OFF_Q + 16384 * st, sbase + OFF_R + 16384 * slot3(D), idS, false);
+        if (block_valid(p, D - 1))
+          umma_k64(tbase + 128, sbase + OFF_Q + 16384 * st, sbase + OFF_R + 16384 * slot3(D - 1), idS, false);
+        umma_commit(BAR(B_TFULL));
+        if (t >= 1) accumulate(t - 1);
+        if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
+        tc_fence_after();
+        umma_k64(tbase + T_S, sbase + OFF_Q + 16384 * st, sbase + OFF_K, idS, false);
+        umma_k64(tbase + T_DP, sbase + OFF_DO + 16384 * st, sbase + OFF_V, idS, false);
+        umma_commit(BAR(B_SDP));
+        if (t >= 1 && t + 1 < iters) {
+          if (!ctl.wait(BAR(B_PDSFREE), (t - 1) & 1)) break;
+          issue_stage(t + 1);
+        }
+      }
+      if (!*abort_flag && ctl.wait(BAR(B_PDS), (iters - 1) & 1)) {
+        tc_fence_after();
+        accumulate(iters - 1);
+      }
+      ctl.drain(BAR(B_DRAIN));
+    }
+    __syncwarp();
+  } else {
+    const int g = warp & 3, hf = warp >> 2, il = 32 * g + lane, cb = 64 * hf;
+    const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
+    float *rrow = rot + il * ROT_LD;
+    bool good = true;
+    for (int t = 0; t < iters; ++t) {
+      const int m = mStart + t, D = m - n, i = m * 128 + il;
+      const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      float *tv = vec + 128 + 256 * (t & 1);  // v.r of blocks D (c < 128) and D - 1
+      {
+        const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
+        tv[tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+      }
+      named_bar_sync(1, NSOFT);
+      good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
+      if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
+      const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
+      if (good) {
+        tc_fence_after();
+        if (hasA) {
+          txl_rotate(tl, 0, 128, hasB, il, cb, tv, tv + 128, rrow);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) rrow[(il - cb - c) & 127] = 0.f;
+        }
+        tc_fence_before();
+        mbar_arrive(BAR(B_TCONS));
+      }
+      named_bar_sync(1, NSOFT);
+      good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
+      float pv[64], ds[64];
+      if (good) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t rs[32], rp[32];
+          tmem_ld32(tl + T_S + cb + 32 * q, rs);
+          tmem_ld32(tl + T_DP + cb + 32 * q, rp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            pv[32 * q + x] = u2f(rs[x]);
+            ds[32 * q + x] = u2f(rp[x]);
+          }
+        }
+        tc_fence_before();
+      } else {
+#pragma unroll
+        for (int x = 0; x < 64; ++x) pv[x] = ds[x] = 0.f;
+      }
+      const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
+        const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + 4 * c4);
+        const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int x = 4 * c4 + e;
+          float y = (pv[x] + rv[e]) * c1;
+          if (need_mask) {
+            const int j = j0 + cb + x;
+            if (j >= L || (p.causal && j > i)) y = -INFINITY;
+          }
+          const float pr = ex2(y - lse2);
+          pv[x] = pr;
+          ds[x] = pr * (ds[x] - Dv);
+        }
+      }
+      named_bar_sync(1, NSOFT);  // every rot row read; the P / dS tiles overwrite them
+      if (good) {
+        store_half_row(smem + OFF_ROT, il, hf, pv);
+        store_half_row(smem + OFF_ROT + 32768, il, hf, ds);
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PDS));
+      }
+    }
+    // ---- epilogue: lanes are keys now ----
+    good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
+    const int j = j0 + il;
+    float csum = 0.f;
+    if (good) {
+      tc_fence_after();
+      uint32_t rv[32], rk[32], rc[16];
+      tmem_ld32(tl + T_DV + 32 * hf, rv);
+      tmem_ld32(tl + T_DK + 32 * hf, rk);
+      tmem_ld16(tl + T_CS, rc);
+      tmem_wait_ld();
+      csum = u2f(rc[0]);
+      if (j < L) {
+        const __nv_bfloat16 *u = (const __nv_bfloat16 *)p.rel1 + (size_t)h * HD + 32 * hf;
+        __nv_bfloat16 *dvp = (__nv_bfloat16 *)p.dv + ((size_t)bh * L + j) * HD + 32 * hf;
+        __nv_bfloat16 *dkp = (__nv_bfloat16 *)p.dk + ((size_t)bh * L + j) * HD + 32 * hf;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float kv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[e] = p.scale * (u2f(rk[8 * c8 + e]) + csum * __bfloat162float(u[8 * c8 + e]));
+          uint4 wv, wk;
+          wv.x = pack_bf16x2(u2f(rv[8 * c8 + 0]), u2f(rv[8 * c8 + 1]));
+          wv.y = pack_bf16x2(u2f(rv[8 * c8 + 2]), u2f(rv[8 * c8 + 3]));
+          wv.z = pack_bf16x2(u2f(rv[8 * c8 + 4]), u2f(rv[8 * c8 + 5]));
+          wv.w = pack_bf16x2(u2f(rv[8 * c8 + 6]), u2f(rv[8 * c8 + 7]));
+          wk.x = pack_bf16x2(kv[0], kv[1]);
+          wk.y = pack_bf16x2(kv[2], kv[3]);
+          wk.z = pack_bf16x2(kv[4], kv[5]);
+          wk.w = pack_bf16x2(kv[6], kv[7]);
+          *reinterpret_cast<uint4 *>(dvp + 8 * c8) = wv;
+          *reinterpret_cast<uint4 *>(dkp + 8 * c8) = wk;
+        }
+      } else {
+        csum = 0.f;
+      }
+    }
+    // du partial: s * sum_j c_j k_j over this key tile (fixed order)
+    named_bar_sync(1, NSOFT);
+    if (hf == 0) vec[il] = csum;
+    named_bar_sync(1, NSOFT);
+    if (tid < HD) {
+      const __nv_bfloat16 *kp = (const __nv_bfloat16 *)p.k + (size_t)bh * L * HD;
+      float acc = 0.f;
+      for (int jj = 0; jj < 128 && j0 + jj < L; ++jj) acc = fmaf(vec[jj], __bfloat162float(kp[(size_t)(j0 + jj) * HD + tid]), acc);
+      A.part_kv[((size_t)bh * p.nT + n) * HD + tid] = p.scale * acc;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ============================================================================
+// query-tile kernel: dQ
+// ============================================================================
+namespace qk {
+constexpr int OFF_Q = 0, OFF_DO = 16384, OFF_K = 32768, OFF_V = OFF_K + 32768, OFF_R = OFF_V + 32768;
+constexpr int OFF_ROT = OFF_R + 3 * 16384;  // rot rows; E_lo at +0, E_hi at +32768
+constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;
+constexpr int OFF_BAR = OFF_VEC + 4096;
+constexpr int SMEM = OFF_BAR + 256 + 1024;
+enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_PDS, B_PDSFREE, B_DRAIN, NB };
+constexpr uint32_t T_S = 0, T_REL = 128, T_DQ = 384, T_DS = 448;
+}  // namespace qk
+
+__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_constant__ BwdArgs A) {
+  using namespace qk;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Prm &p = A.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m = p.nT - 1 - (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z, bh = b * p.H + h;
+  const int L = p.L, i0 = m * 128;
+  const int nTiles = p.causal ? m + 1 : p.nT;
+  const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NB);
+  float *rot = (float *)(smem + OFF_ROT);
+  float *vec = (float *)(smem + OFF_VEC);
+  int32_t *status = p.status;
+  const float c1 = p.scale * LOG2E;
+
+  if (tid == 0) {
+    mbar_init(BAR(B_QD), 1);
+    mbar_init(BAR(B_ST0), 1);
+    mbar_init(BAR(B_ST1), 1);
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_TCONS), NSOFT);
+    mbar_init(BAR(B_DPF), 1);
+    mbar_init(BAR(B_PDS), NSOFT);
+    mbar_init(BAR(B_PDSFREE), 1);
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      Ctl ctl;
+      ctl.np = 0;
+      ctl.ab = abort_flag;
+      ctl.st = status;
+      prefetch_tmap(&A.mq);
+      prefetch_tmap(&A.mk);
+      prefetch_tmap(&A.mv);
+      prefetch_tmap(&A.mdo);
+      prefetch_tmap(&A.mr);
+      const uint32_t idS = idesc_bf16(128, 128, false);
+      const uint32_t idDQ = idesc_bf16(128, 64, true);
+      ctl.expect(BAR(B_QD), 0, 32768);
+      tma_load_3d(sbase + OFF_Q, &A.mq, BAR(B_QD), 0, i0, bh);
+      tma_load_3d(sbase + OFF_DO, &A.mdo, BAR(B_QD), 0, i0, bh);
+      auto issue_stage = [&](int n) {  // K_n, V_n and the relation block tile n adds
+        const int st = n & 1, D = m - n;
+        const bool b0 = (n == 0) && block_valid(p, D), b1 = block_valid(p, D - 1);
+        ctl.expect(BAR(B_ST0 + st), (uint32_t)((n >> 1) & 1), 32768u + (b0 ? 16384u : 0u) + (b1 ? 16384u : 0u));
+        tma_load_3d(sbase + OFF_K + 16384 * st, &A.mk, BAR(B_ST0 + st), 0, n * 128, bh);
+        tma_load_3d(sbase + OFF_V + 16384 * st, &A.mv, BAR(B_ST0 + st), 0, n * 128, bh);
+        if (b0) tma_load_3d(sbase + OFF_R + 16384 * slot3(D), &A.mr, BAR(B_ST0 + st), 0, 128 * D + p.off, h);
+        if (b1) tma_load_3d(sbase + OFF_R + 16384 * slot3(D - 1), &A.mr, BAR(B_ST0 + st), 0, 128 * (D - 1) + p.off, h);
+      };
+      issue_stage(0);
+      if (nTiles > 1) issue_stage(1);
+      bool ok = ctl.wait_load(BAR(B_QD), 0) && ctl.wait_load(BAR(B_ST0), 0);
+      if (ok) {
+        tc_fence_after();
+        umma_k64(tbase + T_S, sbase + OFF_Q, sbase + OFF_K, idS, false);
+        if (block_valid(p, m)) umma_k64(tbase + T_REL + 128 * (m & 1), sbase + OFF_Q, sbase + OFF_R + 16384 * slot3(m), idS, false);
+        if (block_valid(p, m - 1))
+          umma_k64(tbase + T_REL + 128 * ((m - 1) & 1), sbase + OFF_Q, sbase + OFF_R + 16384 * slot3(m - 1), idS, false);
+        umma_commit(BAR(B_SFULL));
+      }
+      for (int n = 0; ok && n < nTiles; ++n) {
+        const int st = n & 1, D = m - n;
+        const uint32_t slotA = T_REL + 128 * (D & 1);  // block D's products; reused for dP(n)
+        if (!ctl.wait(BAR(B_TCONS), n & 1)) break;
+        tc_fence_after();
+        umma_k64(tbase + slotA, sbase + OFF_DO, sbase + OFF_V + 16384 * st, idS, false);  // dP(n)
+        umma_commit(BAR(B_DPF));
+        if (n + 1 < nTiles) {
+          if (!ctl.wait_load(BAR(B_ST0 + (st ^ 1)), ((n + 1) >> 1) & 1)) break;
+          umma_k64(tbase + T_S, sbase + OFF_Q, sbase + OFF_K + 16384 * (st ^ 1), idS, false);  // S(n+1)
+        }
+        if (!ctl.wait(BAR(B_PDS), n & 1)) break;
+        tc_fence_after();
+        // dQ += dS K_n (dS from TMEM) + E_lo r_D + E_hi r_{D-1}
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_bf16_ts(tbase + T_DQ, tbase + T_DS + 8 * k, sdesc_sw128(sbase + OFF_K + 16384 * st + 2048 * k, 16, 1024), idDQ,
+                       (n > 0 || k > 0) ? 1u : 0u);
+        if (block_valid(p, D)) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_bf16(tbase + T_DQ, sdesc_sw128(sbase + OFF_ROT + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
+                      sdesc_sw128(sbase + OFF_R + 16384 * slot3(D) + 2048 * k, 16, 1024), idDQ, 1u);
+        }
+        if (block_valid(p, D - 1)) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_bf16(tbase + T_DQ, sdesc_sw128(sbase + OFF_ROT + 32768 + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
+                      sdesc_sw128(sbase + OFF_R + 16384 * slot3(D - 1) + 2048 * k, 16, 1024), idDQ, 1u);
+        }
+        umma_commit(BAR(B_PDSFREE));
+        if (n + 1 < nTiles) {  // relation block D - 2 for tile n + 1, into the slot dP(n) used
+          if (block_valid(p, D - 2))
+            umma_k64(tbase + slotA, sbase + OFF_Q, sbase + OFF_R + 16384 * slot3(D - 2), idS, false);
+          umma_commit(BAR(B_SFULL));
+        }
+        if (n + 2 < nTiles) {
+          if (!ctl.wait(BAR(B_PDSFREE), n & 1)) break;
+          issue_stage(n + 2);
+        }
+      }
+      ctl.drain(BAR(B_DRAIN));
+    }
+    __syncwarp();
+  } else {
+    const int g = warp & 3, hf = warp >> 2, il = 32 * g + lane, cb = 64 * hf;
+    const int i = i0 + il;
+    const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
+    float *rrow = rot + il * ROT_LD;
+    const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+    const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+    bool good = true;
+    for (int n = 0; n < nTiles; ++n) {
+      const int j0 = n * 128, D = m - n;
+      float *tu = vec + 384 * (n & 1);  // uk[128] | v.r block D [128] | v.r block D - 1 [128]
+      if (tid < 128) tu[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      {
+        const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
+        tu[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+      }
+      named_bar_sync(1, NSOFT);
+      good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
+      if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
+      const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
+      float x[64];
+      if (good) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tl + T_S + cb + 32 * q, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[32 * q + e] = u2f(r[e]);
+        }
+        if (hasA) {
+          txl_rotate(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, il, cb, tu + 128, tu + 256, rrow);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) rrow[(il - cb - c) & 127] = 0.f;
+        }
+        tc_fence_before();
+        mbar_arrive(BAR(B_TCONS));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) x[e] = 0.f;
+      }
+      named_bar_sync(1, NSOFT);
+      const bool need_mask = (p.causal && n == m) || (j0 + 128 > L);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
+        const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
+        const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int xx = 4 * c4 + e;
+          float y = (x[xx] + rv[e]) * c1;
+          if (need_mask) {
+            const int j = j0 + cb + xx;
+            if (j >= L || (p.causal && j > i)) y = -INFINITY;
+          }
+          x[xx] = ex2(y - lse2);
+        }
+      }
+      good = good && warp_wait(BAR(B_DPF), n & 1, abort_flag, status);
+      if (good) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tl + T_REL + 128 * (D & 1) + cb + 32 * q, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[32 * q + e] = x[32 * q + e] * (u2f(r[e]) - Dv);
+        }
+        tc_fence_before();
+      }
+      named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
+      if (good) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        tmem_st32(tl + T_DS + 32 * hf, pk);
+        uint8_t *Elo = smem + OFF_ROT, *Ehi = smem + OFF_ROT + 32768;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const int jl = cb + e, c = (il - jl) & 127;
+          const bool lo = jl <= il;
+          store_elem(Elo, il, c, lo ? x[e] : 0.f);
+          store_elem(Ehi, il, c, lo ? 0.f : x[e]);
+        }
+        tmem_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PDS));
+      }
+    }
+    good = good && warp_wait(BAR(B_PDSFREE), (nTiles - 1) & 1, abort_flag, status);
+    if (good) {
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(tl + T_DQ + 32 * hf, r);
+      tmem_wait_ld();
+      if (i < L) {
+        __nv_bfloat16 *dqp = (__nv_bfloat16 *)p.dq + ((size_t)bh * L + i) * HD + 32 * hf;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint4 w;
+          w.x = pack_bf16x2(p.scale * u2f(r[8 * c8 + 0]), p.scale * u2f(r[8 * c8 + 1]));
+          w.y = pack_bf16x2(p.scale * u2f(r[8 * c8 + 2]), p.scale * u2f(r[8 * c8 + 3]));
+          w.z = pack_bf16x2(p.scale * u2f(r[8 * c8 + 4]), p.scale * u2f(r[8 * c8 + 5]));
+          w.w = pack_bf16x2(p.scale * u2f(r[8 * c8 + 6]), p.scale * u2f(r[8 * c8 + 7]));
+          *reinterpret_cast<uint4 *>(dqp + 8 * c8) = w;
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ============================================================================
+// diagonal kernel: per-offset sums G = sum dS q and g = sum dS for dr
+// ============================================================================
+namespace dg {
+constexpr int OFF_Q = 0, OFF_DO = 32768, OFF_K = 65536, OFF_V = OFF_K + 16384, OFF_R = OFF_V + 16384;
+constexpr int OFF_ROT = OFF_R + 32768;  // rot rows; E_lo at +0, E_hi at +32768
+constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;
+constexpr int OFF_VEC = OFF_ONES + 4096;
+constexpr int OFF_BAR = OFF_VEC + 4096;
+constexpr int SMEM = OFF_BAR + 256 + 1024;
+enum { B_R = 0, B_ST0, B_ST1, B_KV, B_KVFREE, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
+constexpr uint32_t T_S = 0, T_DP = 128, T_GLO = 256, T_GHI = 320, T_GL = 384, T_GH = 416;
+}  // namespace dg
+
+__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_constant__ BwdArgs A) {
+  using namespace dg;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Prm &p = A.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int band = blockIdx.x, chunk = blockIdx.y, bhi = blockIdx.z;
+  const int b = bhi / p.H, h = bhi % p.H, bh = bhi;
+  const int D = p.causal ? band : band - (p.nT - 1);
+  const int mlo = max(0, D), mhi = min(p.nT - 1, p.nT - 1 + D);
+  const int m0 = mlo + chunk * A.dg_ch, m1 = min(mhi, m0 + A.dg_ch - 1);
+  if (m0 > m1) return;  // whole CTA, before any barrier or TMEM allocation
+  const int iters = m1 - m0 + 1;
+  const int L = p.L;
+  const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NB);
+  float *rot = (float *)(smem + OFF_ROT);
+  float *vec = (float *)(smem + OFF_VEC);
+  int32_t *status = p.status;
+  const float c1 = p.scale * LOG2E;
+  const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
+  (void)b;
+
+  if (tid == 0) {
+    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), (k == B_TCONS || k == B_PDS) ? NSOFT : 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  for (int x = tid; x < 4096 / 16; x += NTHREADS) {
+    const uint32_t one2 = 0x3F803F80u;
+    *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
+  }
+  {  // v.r of the band's two blocks (fixed for the CTA)
+    const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
+    vec[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+  }
+  fence_async_smem();
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      Ctl ctl;
+      ctl.np = 0;
+      ctl.ab = abort_flag;
+      ctl.st = status;
+      prefetch_tmap(&A.mq);
+      prefetch_tmap(&A.mk);
+      prefetch_tmap(&A.mv);
+      prefetch_tmap(&A.mdo);
+      prefetch_tmap(&A.mr);
+      const uint32_t idS = idesc_bf16(128, 128, false);
+      const uint32_t idG = idesc_bf16(128, 64, true, true);
+      const uint32_t idg = idesc_bf16(128, 16, false, true);
+      ctl.expect(BAR(B_R), 0, (hasA ? 16384u : 0u) + (hasB ? 16384u : 0u));
+      if (hasA) tma_load_3d(sbase + OFF_R, &A.mr, BAR(B_R), 0, 128 * D + p.off, h);
+      if (hasB) tma_load_3d(sbase + OFF_R + 16384, &A.mr, BAR(B_R), 0, 128 * (D - 1) + p.off, h);
+      auto issue_qd = [&](int t) {
+        const int m = m0 + t, st = t & 1;
+        ctl.expect(BAR(B_ST0 + st), (uint32_t)((t >> 1) & 1), 32768);
+        tma_load_3d(sbase + OFF_Q + 16384 * st, &A.mq, BAR(B_ST0 + st), 0, m * 128, bh);
+        tma_load_3d(sbase + OFF_DO + 16384 * st, &A.mdo, BAR(B_ST0 + st), 0, m * 128, bh);
+      };
+      auto issue_kv = [&](int t) {
+        const int nn = m0 + t - D;
+        ctl.expect(BAR(B_KV), (uint32_t)(t & 1), 32768);
+        tma_load_3d(sbase + OFF_K, &A.mk, BAR(B_KV), 0, nn * 128, bh);
+        tma_load_3d(sbase + OFF_V, &A.mv, BAR(B_KV), 0, nn * 128, bh);
+      };
+      auto accumulate = [&](int t) {  // G_lo, G_hi += E^T Q_t ; g_lo, g_hi += E^T 1
+        const int st = t & 1;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
+          const uint64_t bq = sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, 16, 1024);
+          const uint64_t b1 = sdesc_sw128(sbase + OFF_ONES + 2048 * (k >> 2) + 32 * (k & 3), 16, 1024);
+          const uint64_t elo = sdesc_sw128(sbase + OFF_ROT + 2048 * k, 16384, 1024);
+          const uint64_t ehi = sdesc_sw128(sbase + OFF_ROT + 32768 + 2048 * k, 16384, 1024);
+          umma_bf16(tbase + T_GLO, elo, bq, idG, acc);
+          umma_bf16(tbase + T_GHI, ehi, bq, idG, acc);
+          umma_bf16(tbase + T_GL, elo, b1, idg, acc);
+          umma_bf16(tbase + T_GH, ehi, b1, idg, acc);
+        }
+        umma_commit(BAR(B_PDSFREE));
+      };
+      issue_qd(0);
+      issue_kv(0);
+      if (iters > 1) issue_qd(1);
+      bool ok = ctl.wait_load(BAR(B_R), 0);
+      for (int t = 0; ok && t < iters; ++t) {
+        const int st = t & 1;
+        if (!ctl.wait_load(BAR(B_ST0 + st), (t >> 1) & 1)) break;
+        if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
+        tc_fence_after();
+        if (hasA) umma_k64(tbase + 0, sbase + OFF_Q + 16384 * st, sbase + OFF_R, idS, false);
+        if (hasB) umma_k64(tbase + 128, sbase + OFF_Q + 16384 * st, sbase + OFF_R + 16384, idS, false);
+        umma_commit(BAR(B_TFULL));
+        if (t >= 1) accumulate(t - 1);
+        if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
+        if (!ctl.wait_load(BAR(B_KV), t & 1)) break;
+        tc_fence_after();
+        umma_k64(tbase + T_S, sbase + OFF_Q + 16384 * st, sbase + OFF_K, idS, false);
+        umma_k64(tbase + T_DP, sbase + OFF_DO + 16384 * st, sbase + OFF_V, idS, false);
+        umma_commit(BAR(B_SDP));
+        umma_commit(BAR(B_KVFREE));
+        if (t + 1 < iters) {
+          if (!ctl.wait(BAR(B_KVFREE), t & 1)) break;
+          issue_kv(t + 1);
+          if (t >= 1) {
+            if (!ctl.wait(BAR(B_PDSFREE), (t - 1) & 1)) break;
+            issue_qd(t + 1);
+          }
+        }
+      }
+      if (!*abort_flag && ctl.wait(BAR(B_PDS), (iters - 1) & 1)) {
+        tc_fence_after();
+        accumulate(iters - 1);
+      }
+      ctl.drain(BAR(B_DRAIN));
+    }
+    __syncwarp();
+  } else {
+    const int g = warp & 3, hf = warp >> 2, il = 32 * g + lane, cb = 64 * hf;
+    const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
+    float *rrow = rot + il * ROT_LD;
+    bool good = true;
+    for (int t = 0; t < iters; ++t) {
+      const int m = m0 + t, nn = m - D, i = m * 128 + il, j0 = nn * 128;
+      const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      float *tu = vec + 384 + 128 * (t & 1);
+      if (tid < 128) tu[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      named_bar_sync(1, NSOFT);
+      good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
+      if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
+      if (good) {
+        tc_fence_after();
+        if (hasA) {
+          txl_rotate(tl, 0, 128, hasB, il, cb, vec + 128, vec + 256, rrow);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) rrow[(il - cb - c) & 127] = 0.f;
+        }
+        tc_fence_before();
+        mbar_arrive(BAR(B_TCONS));
+      }
+      named_bar_sync(1, NSOFT);
+      good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
+      float pv[64], ds[64];
+      if (good) {
+        tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t rs[32], rp[32];
+          tmem_ld32(tl + T_S + cb + 32 * q, rs);
+          tmem_ld32(tl + T_DP + cb + 32 * q, rp);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            pv[32 * q + x] = u2f(rs[x]);
+            ds[32 * q + x] = u2f(rp[x]);
+          }
+        }
+        tc_fence_before();
+      } else {
+#pragma unroll
+        for (int x = 0; x < 64; ++x) pv[x] = ds[x] = 0.f;
+      }
+      const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
+        const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
+        const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int x = 4 * c4 + e;
+          float y = (pv[x] + rv[e]) * c1;
+          if (need_mask) {
+            const int j = j0 + cb + x;
+            if (j >= L || (p.causal && j > i)) y = -INFINITY;
+          }
+          const float pr = ex2(y - lse2);
+          ds[x] = pr * (ds[x] - Dv);
+        }
+      }
+      named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
+      if (good) {
+        uint8_t *Elo = smem + OFF_ROT, *Ehi = smem + OFF_ROT + 32768;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const int jl = cb + e, c = (il - jl) & 127;
+          const bool lo = jl <= il;
+          store_elem(Elo, il, c, lo ? ds[e] : 0.f);
+          store_elem(Ehi, il, c, lo ? 0.f : ds[e]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PDS));
+      }
+    }
+    // ---- epilogue: lane il now is offset c = il of both blocks ----
+    good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
+    if (good) {
+      tc_fence_after();
+      uint32_t rlo[32], rhi[32], glo[16], ghi[16];
+      tmem_ld32(tl + T_GLO + 32 * hf, rlo);
+      tmem_ld32(tl + T_GHI + 32 * hf, rhi);
+      tmem_ld16(tl + T_GL, glo);
+      tmem_ld16(tl + T_GH, ghi);
+      tmem_wait_ld();
+      float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        part[(size_t)il * 65 + 32 * hf + e] = u2f(rlo[e]);
+        part[(size_t)(128 + il) * 65 + 32 * hf + e] = u2f(rhi[e]);
+      }
+      if (hf == 0) {
+        part[(size_t)il * 65 + 64] = u2f(glo[0]);
+        part[(size_t)(128 + il) * 65 + 64] = u2f(ghi[0]);
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// dr[h][rho][e] = s (sum G + (sum g) v[e]) over the batch, the bands holding
+// offset delta = rho - off (as block D or D - 1) and their chunks; gtot gets sum g.
+__global__ void reduce_dr_kernel(BwdArgs A) {
+  const Prm &p = A.p;
+  const size_t per = (size_t)p.nrows * HD;
+  const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= (size_t)p.H * per) return;
+  const int h = (int)(x / per), rho = (int)((x % per) / HD), e = (int)(x % HD);
+  const int delta = rho - p.off;
+  const int blk = delta >= 0 ? delta / 128 : -((-delta + 127) / 128);
+  const int c = delta - 128 * blk;
+  float acc = 0.f, gs = 0.f;
+  for (int bb = 0; bb < p.B; ++bb) {
+    const size_t bh = (size_t)bb * p.H + h;
+    for (int w = 0; w < 2; ++w) {  // w = 0: band blk (block = D); w = 1: band blk + 1 (block = D - 1)
+      const int D = blk + w;
+      const int band = p.causal ? D : D + (p.nT - 1);
+      if (band < 0 || band >= A.nbands) continue;
+      const int len = p.nT - (D < 0 ? -D : D);
+      const int nch = (len + A.dg_ch - 1) / A.dg_ch;
+      for (int ch = 0; ch < nch; ++ch) {
+        const float *part = A.part_dg + ((bh * A.nbands + band) * A.dg_nchunk + ch) * DG_STRIDE + (size_t)(128 * w + c) * 65;
+        acc += part[e];
+        gs += part[64];
+      }
+    }
+  }
+  const float vv = __bfloat162float(((const __nv_bfloat16 *)p.rel2)[(size_t)h * HD + e]);
+  p.drel0[x] = p.scale * (acc + gs * vv);
+  if (e == 0) p.gtot[(size_t)h * p.nrows + rho] = gs;
+}
+
+// dv[h][e] = s sum_rho gtot r; du[h][e] = sum over key tiles of the du partials
+__global__ void reduce_uv_kernel(BwdArgs A) {
+  const Prm &p = A.p;
+  __shared__ float red[256];
+  const int h = blockIdx.x / HD, e = blockIdx.x % HD;
+  const __nv_bfloat16 *r = (const __nv_bfloat16 *)p.rel0 + (size_t)h * p.nrows * HD;
+  float acc = 0.f;
+  for (int rho = threadIdx.x; rho < p.nrows; rho += 256)
+    acc = fmaf(p.gtot[(size_t)h * p.nrows + rho], __bfloat162float(r[(size_t)rho * HD + e]), acc);
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    p.drel2[(size_t)h * HD + e] = p.scale * red[0];
+    float du = 0.f;
+    for (int bb = 0; bb < p.B; ++bb)
+      for (int n = 0; n < p.nT; ++n) du += A.part_kv[(((size_t)bb * p.H + h) * p.nT + n) * HD + e];
+    p.drel1[(size_t)h * HD + e] = du;
+  }
+}
+
+}  // namespace tcb
+
+// ---------------------------------------------------------------------------
+// host
+// ---------------------------------------------------------------------------
+void tc_bwd_shape(const Prm &p, int &nT, int &nbands, int &ch, int &nchunk) {
+  nT = (p.L + 127) / 128;
+  nbands = p.causal ? nT : 2 * nT - 1;
+  long long cap = 3000 / ((long long)p.B * p.H * nbands);
+  int nch = (nT + 3) / 4;
+  if (cap < nch) nch = (int)(cap < 1 ? 1 : cap);
+  ch = (nT + nch - 1) / nch;
+  nchunk = (nT + ch - 1) / ch;
+}
+
+size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats) {
+  int nT, nbands, ch, nchunk;
+  tc_bwd_shape(p, nT, nbands, ch, nchunk);
+  kv_floats = (size_t)p.B * p.H * nT * HD;
+  return (size_t)p.B * p.H * nbands * nchunk * tcb::DG_STRIDE;
+}
+
+bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows);
+
+cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
+  using namespace tcb;
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.p = p0;
+  int nT, nbands, ch, nchunk;
+  tc_bwd_shape(p0, nT, nbands, ch, nchunk);
+  a.p.nT = nT;
+  a.nbands = nbands;
+  a.dg_ch = ch;
+  a.dg_nchunk = nchunk;
+  a.uk = w.uk;
+  a.vr = w.vr;
+  a.part_kv = w.part_kv;
+  a.part_dg = w.part_dg;
+  a.p.part_small = w.part_kv;
+  const uint64_t BH = (uint64_t)p0.B * p0.H;
+  if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
+        tc_make_map(&a.mv, p0.v, p0.L, BH, 128) && tc_make_map(&a.mdo, p0.dout, p0.L, BH, 128) &&
+        tc_make_map(&a.mr, p0.rel0, p0.nrows, p0.H, 128)))
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  if ((e = tc_prep(a.p, w, st)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(tc_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::SMEM)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(tc_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qk::SMEM)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(tc_bwd_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dg::SMEM)) != cudaSuccess)
+    return e;
+  dim3 grid(nT, p0.H, p0.B);
+  tc_bwd_kv_kernel<<<grid, NTHREADS, kv::SMEM, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc_bwd_q_kernel<<<grid, NTHREADS, qk::SMEM, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc_bwd_diag_kernel<<<dim3(nbands, nchunk, p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t nr = (size_t)p0.H * p0.nrows * HD;
+  reduce_dr_kernel<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  reduce_uv_kernel<<<p0.H * HD, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace rp

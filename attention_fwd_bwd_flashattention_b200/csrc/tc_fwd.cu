@@ -619,7 +619,7 @@ static EncodeTiledFn encode_fn() {
 
 // [planes][rows][64] bf16 viewed as a 3D tensor; box = 64 x box_rows x 1, 128B swizzle,
 // rows outside [0, rows) read as zeros.
-static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows) {
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {64, rows, planes};
@@ -642,6 +642,17 @@ static cudaError_t launch_fwd_t(const FwdArgs &a, cudaStream_t st) {
 }
 
 }  // namespace tc
+
+bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows) {
+  return tc::make_map(m, base, rows, planes, box_rows);
+}
+
+cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st) {
+  if (p.mech != M_TXL && p.mech != M_DEB) return cudaSuccess;
+  const size_t n = std::max((size_t)p.B * p.H * p.L, (size_t)p.H * p.nrows);
+  tc::tc_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE);
+  return cudaGetLastError();
+}
 
 bool tc_supported(const Prm &p) {
   if (p.mech == M_SHAW && 2 * p.clip + 1 > 131) return false;  // QA row must fit the 132-float smem row
@@ -667,12 +678,8 @@ cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st) {
   }
   if (p.mech == M_DEB) ok = ok && make_map(&a.mt0, p.rel0, p.nrows, p.H, 256) && make_map(&a.mt1, p.rel1, p.nrows, p.H, 256);
   if (!ok) return cudaErrorInvalidValue;
-  if (p.mech == M_TXL || p.mech == M_DEB) {
-    const size_t n = std::max((size_t)p.B * p.H * p.L, (size_t)p.H * p.nrows);
-    tc_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = tc_prep(p, w, st);
+  if (e != cudaSuccess) return e;
   switch (p.mech) {
     case M_T5: return launch_fwd_t<M_T5>(a, st);
     case M_SHAW: return launch_fwd_t<M_SHAW>(a, st);
