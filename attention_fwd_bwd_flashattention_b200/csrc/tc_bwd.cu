@@ -116,6 +116,49 @@ __device__ __forceinline__ void store_elem(uint8_t *tile, int r, int c, float x)
       __float2bfloat16_rn(x);
 }
 
+__device__ __forceinline__ uint32_t E_addr(int r, int c) {  // byte offset of (row r, even col c)
+  return 16384 * (c >> 6) + 128 * r + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+
+// Move this thread's 64 dS values (keys jl = cb + e, e = 0..63) of row il into offset
+// coordinates: E_lo[il][c] (keys jl <= il) and E_hi[il][c] (keys jl > il) with
+// c = (il - jl) & 127, zero in the other tile.  The thread's offsets are s0 .. s0 + 63
+// (mod 128), s0 = (il - cb - 63) & 127, offset s0 + k holding x[63 - k]; they are
+// written as aligned bf16 pairs (4-byte stores).  When s0 is odd its first and last
+// offsets pair with the other half-row thread's values and are written alone.
+__device__ __forceinline__ void store_E(uint8_t *Elo, uint8_t *Ehi, int il, int cb, const float (&x)[64]) {
+  const int s0 = (il - cb - 63) & 127;
+  const bool odd = (s0 & 1) != 0;
+  const int c0 = s0 & ~1;
+  auto put = [&](int c, float va, int ja, float vb, int jb) {  // pair (c, c + 1), c even
+    const bool la = ja <= il, lb = jb <= il;
+    const uint32_t off = E_addr(il, c);
+    *reinterpret_cast<uint32_t *>(Elo + off) = pack2(la ? va : 0.f, lb ? vb : 0.f);
+    *reinterpret_cast<uint32_t *>(Ehi + off) = pack2(la ? 0.f : va, lb ? 0.f : vb);
+  };
+  auto put1 = [&](int c, float v, int jj) {  // single element
+    const uint32_t off = E_addr(il, c & ~1) + ((c & 1) << 1);
+    const bool l = jj <= il;
+    *reinterpret_cast<__nv_bfloat16 *>(Elo + off) = __float2bfloat16_rn(l ? v : 0.f);
+    *reinterpret_cast<__nv_bfloat16 *>(Ehi + off) = __float2bfloat16_rn(l ? 0.f : v);
+  };
+  // pair p >= 1 holds offsets c0 + 2p, c0 + 2p + 1: k = 2p - odd, 2p + 1 - odd
+#pragma unroll
+  for (int pp = 1; pp < 32; ++pp) {
+    const float va = odd ? x[64 - 2 * pp] : x[63 - 2 * pp];
+    const float vb = odd ? x[63 - 2 * pp] : x[62 - 2 * pp];
+    const int ea = odd ? 64 - 2 * pp : 63 - 2 * pp;
+    put((c0 + 2 * pp) & 127, va, cb + ea, vb, cb + ea - 1);
+  }
+  if (!odd) {
+    put(c0, x[63], cb + 63, x[62], cb + 62);
+  } else {
+    put1(s0, x[63], cb + 63);
+    put1((s0 + 63) & 127, x[0], cb);
+  }
+}
+
 // Rotate offsets c in [cb, cb + 64) of the two relation blocks (TMEM columns colA,
 // colB of this warp's lanes) into key order: rrow[(il - c) & 127] gets block Delta
 // for c <= il, block Delta - 1 otherwise, plus the per-offset v.r term.
@@ -166,7 +209,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, bh = b * p.H + h;
+  // 1-D grid: key tiles with the most causal query tiles first, over every head
+  const int BH = p.B * p.H;
+  const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, j0 = n * 128;
   const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
@@ -280,15 +325,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
+    // row statistics and v.r of the next query tile, fetched one iteration ahead
+    auto fetch = [&](int t, float &l2, float &dv, float &vrv) {
+      const int m = mStart + t, D = m - n, i = m * 128 + il;
+      l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
+      vrv = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+    };
+    float nl2, ndv, nvr;
+    fetch(0, nl2, ndv, nvr);
     for (int t = 0; t < iters; ++t) {
       const int m = mStart + t, D = m - n, i = m * 128 + il;
-      const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
-      const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      const float lse2 = nl2, Dv = ndv;
       float *tv = vec + 128 + 256 * (t & 1);  // v.r of blocks D (c < 128) and D - 1
-      {
-        const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
-        tv[tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
-      }
+      tv[tid] = nvr;
+      if (t + 1 < iters) fetch(t + 1, nl2, ndv, nvr);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
@@ -306,7 +358,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       }
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
-      float pv[64], ds[64];
+      // P and dS of this thread's 64 keys, packed to bf16 pairs as they are made
+      uint32_t pk[32], dk[32];
+      const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
 #pragma unroll
@@ -316,39 +370,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
           tmem_ld32(tl + T_DP + cb + 32 * q, rp);
           tmem_wait_ld();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            pv[32 * q + x] = u2f(rs[x]);
-            ds[32 * q + x] = u2f(rp[x]);
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const int x0 = 32 * q + 4 * c4;
+            const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
+            const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
+            const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+            float pr[4], dd[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float y = (u2f(rs[4 * c4 + e]) + rv[e]) * c1;
+              if (need_mask) {
+                const int j = j0 + cb + x0 + e;
+                if (j >= L || (p.causal && j > i)) y = -INFINITY;
+              }
+              pr[e] = ex2(y - lse2);
+              dd[e] = pr[e] * (u2f(rp[4 * c4 + e]) - Dv);
+            }
+            pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
+            pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+            dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
+            dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
           }
         }
         tc_fence_before();
-      } else {
-#pragma unroll
-        for (int x = 0; x < 64; ++x) pv[x] = ds[x] = 0.f;
-      }
-      const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
-#pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
-        const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + 4 * c4);
-        const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int x = 4 * c4 + e;
-          float y = (pv[x] + rv[e]) * c1;
-          if (need_mask) {
-            const int j = j0 + cb + x;
-            if (j >= L || (p.causal && j > i)) y = -INFINITY;
-          }
-          const float pr = ex2(y - lse2);
-          pv[x] = pr;
-          ds[x] = pr * (ds[x] - Dv);
-        }
       }
       named_bar_sync(1, NSOFT);  // every rot row read; the P / dS tiles overwrite them
       if (good) {
-        store_half_row(smem + OFF_ROT, il, hf, pv);
-        store_half_row(smem + OFF_ROT + 32768, il, hf, ds);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t off = 16384 * hf + 128 * il + ((ch ^ (il & 7)) << 4);
+          *reinterpret_cast<uint4 *>(smem + OFF_ROT + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          *reinterpret_cast<uint4 *>(smem + OFF_ROT + 32768 + off) =
+              make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+        }
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
@@ -429,7 +483,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m = p.nT - 1 - (int)blockIdx.x, h = blockIdx.y, b = blockIdx.z, bh = b * p.H + h;
+  const int BH = p.B * p.H;
+  const int bh = (int)blockIdx.x % BH, m = p.nT - 1 - (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, i0 = m * 128;
   const int nTiles = p.causal ? m + 1 : p.nT;
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
@@ -548,14 +603,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
     bool good = true;
+    auto fetch = [&](int n, float &ukv, float &vrv) {  // one key tile ahead
+      const int j0 = n * 128, D = m - n;
+      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
+      vrv = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+    };
+    float nuk, nvr;
+    fetch(0, nuk, nvr);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * 128, D = m - n;
       float *tu = vec + 384 * (n & 1);  // uk[128] | v.r block D [128] | v.r block D - 1 [128]
-      if (tid < 128) tu[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
-      {
-        const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
-        tu[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
-      }
+      if (tid < 128) tu[tid] = nuk;
+      tu[128 + tid] = nvr;
+      if (n + 1 < nTiles) fetch(n + 1, nuk, nvr);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
@@ -620,14 +681,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
         tmem_st32(tl + T_DS + 32 * hf, pk);
-        uint8_t *Elo = smem + OFF_ROT, *Ehi = smem + OFF_ROT + 32768;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const int jl = cb + e, c = (il - jl) & 127;
-          const bool lo = jl <= il;
-          store_elem(Elo, il, c, lo ? x[e] : 0.f);
-          store_elem(Ehi, il, c, lo ? 0.f : x[e]);
-        }
+        store_E(smem + OFF_ROT, smem + OFF_ROT + 32768, il, cb, x);
         tmem_wait_st();
         fence_async_smem();
         tc_fence_before();
@@ -682,9 +736,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int band = blockIdx.x, chunk = blockIdx.y, bhi = blockIdx.z;
-  const int b = bhi / p.H, h = bhi % p.H, bh = bhi;
-  const int D = p.causal ? band : band - (p.nT - 1);
+  // 1-D grid: longest bands first (causal: D = 0, 1, ...; otherwise 0, 1, -1, 2, -2, ...)
+  const int BH = p.B * p.H;
+  const int bh = (int)blockIdx.x % BH, rr0 = (int)blockIdx.x / BH;
+  const int chunk = rr0 % A.dg_nchunk, rank = rr0 / A.dg_nchunk;
+  const int D = p.causal ? rank : ((rank & 1) ? (rank + 1) / 2 : -(rank / 2));
+  const int band = p.causal ? D : D + (p.nT - 1);
+  const int b = bh / p.H, h = bh % p.H;
   const int mlo = max(0, D), mhi = min(p.nT - 1, p.nT - 1 + D);
   const int m0 = mlo + chunk * A.dg_ch, m1 = min(mhi, m0 + A.dg_ch - 1);
   if (m0 > m1) return;  // whole CTA, before any barrier or TMEM allocation
@@ -807,12 +865,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
+    auto fetch = [&](int t, float &l2, float &dv, float &ukv) {  // one tile ahead
+      const int m = m0 + t, i = m * 128 + il, j0 = (m - D) * 128;
+      l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+    };
+    float nl2, ndv, nuk;
+    fetch(0, nl2, ndv, nuk);
     for (int t = 0; t < iters; ++t) {
       const int m = m0 + t, nn = m - D, i = m * 128 + il, j0 = nn * 128;
-      const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
-      const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      const float lse2 = nl2, Dv = ndv;
       float *tu = vec + 384 + 128 * (t & 1);
-      if (tid < 128) tu[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      if (tid < 128) tu[tid] = nuk;
+      if (t + 1 < iters) fetch(t + 1, nl2, ndv, nuk);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
@@ -869,14 +935,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
-        uint8_t *Elo = smem + OFF_ROT, *Ehi = smem + OFF_ROT + 32768;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const int jl = cb + e, c = (il - jl) & 127;
-          const bool lo = jl <= il;
-          store_elem(Elo, il, c, lo ? ds[e] : 0.f);
-          store_elem(Ehi, il, c, lo ? 0.f : ds[e]);
-        }
+        store_E(smem + OFF_ROT, smem + OFF_ROT + 32768, il, cb, ds);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
@@ -1019,12 +1078,12 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qk::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(tc_bwd_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dg::SMEM)) != cudaSuccess)
     return e;
-  dim3 grid(nT, p0.H, p0.B);
-  tc_bwd_kv_kernel<<<grid, NTHREADS, kv::SMEM, st>>>(a);
+  const unsigned tiles = (unsigned)(nT * p0.H * p0.B);
+  tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_bwd_q_kernel<<<grid, NTHREADS, qk::SMEM, st>>>(a);
+  tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_bwd_diag_kernel<<<dim3(nbands, nchunk, p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a);
+  tc_bwd_diag_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t nr = (size_t)p0.H * p0.nrows * HD;
   reduce_dr_kernel<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(a);

@@ -87,9 +87,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m = p.nT - 1 - (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
+  // 1-D grid, heaviest (longest causal) query tiles of every head first
+  const int BH = p.B * p.H;
+  const int bh = (int)blockIdx.x % BH, m = p.nT - 1 - (int)blockIdx.x / BH;
+  const int h = bh % p.H;
   const int L = p.L, i0 = m * BM;
   const int nTiles = p.causal ? m + 1 : p.nT;
   const uint32_t sbase = smem_u32(smem);
@@ -300,24 +301,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       named_bar_sync(1, NSOFT);
     }
     int band_cnt = 0;
+    // per-tile vectors, fetched one key tile ahead (one or two elements per thread)
+    auto fetch_vec = [&](int n, float &va, float &vb) {
+      const int j0 = n * BN, Delta = m - n;
+      va = 0.f;
+      vb = 0.f;
+      if (MECH == M_TXL) {
+        const int j = j0 + tid;
+        if (tid < 128 && j < L) va = A.uk[(size_t)bh * L + j];
+        const int rr = 128 * (tid < 128 ? Delta : Delta - 1) + (tid & 127) + p.off;
+        if (rr >= 0 && rr < p.nrows) vb = A.vr[(size_t)h * p.nrows + rr];
+      } else if (MECH == M_T5) {
+        const int idx = j0 - i0 - 127 + tid + L - 1;
+        if (tid < 255 && idx >= 0 && idx < 2 * L - 1) va = p.t5_bias[(size_t)h * (2 * L - 1) + idx];
+      } else if (MECH == M_DEB) {
+        const int j = j0 + (tid >> 1);
+        if (j < L) va = A.p2cE[((size_t)bh * L + j) * 2 + (tid & 1)];
+      }
+    };
+    float nva, nvb;
+    fetch_vec(0, nva, nvb);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * BN, Delta = m - n;
       float *tv = vec + 512 * (n & 1);
-      // ---- per-tile vectors (one element per softmax thread) ----
       if (MECH == M_TXL) {
-        if (tid < 128) {
-          const int j = j0 + tid;
-          tv[tid] = (j < L) ? A.uk[(size_t)bh * L + j] : 0.f;
-        }
-        const int rr = 128 * (tid < 128 ? Delta : Delta - 1) + (tid & 127) + p.off;
-        tv[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+        if (tid < 128) tv[tid] = nva;
+        tv[128 + tid] = nvb;
       } else if (MECH == M_T5) {
-        const int idx = j0 - i0 - 127 + tid + L - 1;
-        if (tid < 255) tv[tid] = (idx >= 0 && idx < 2 * L - 1) ? p.t5_bias[(size_t)h * (2 * L - 1) + idx] : 0.f;
+        if (tid < 255) tv[tid] = nva;
       } else if (MECH == M_DEB) {
-        const int j = j0 + (tid >> 1);
-        tv[tid] = (j < L) ? A.p2cE[((size_t)bh * L + j) * 2 + (tid & 1)] : 0.f;
+        tv[tid] = nva;
       }
+      if (n + 1 < nTiles) fetch_vec(n + 1, nva, nvb);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       float x[64];
@@ -636,8 +651,7 @@ static cudaError_t launch_fwd_t(const FwdArgs &a, cudaStream_t st) {
   auto k = tc_fwd_kernel<MECH>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.p.nT, a.p.H, a.p.B);
-  k<<<grid, NTHREADS, SMEM_BYTES, st>>>(a);
+  k<<<(unsigned)(a.p.nT * a.p.H * a.p.B), NTHREADS, SMEM_BYTES, st>>>(a);
   return cudaGetLastError();
 }
 
