@@ -47,8 +47,9 @@ class relpos_params_t(ctypes.Structure):
     ]
 
 
-EXPORTS = ("relpos_attn_workspace_size", "relpos_attn_fwd", "relpos_attn_bwd", "relpos_attn_resolved_path",
-           "relpos_strerror", "relpos_attn_version")
+EXPORTS = ("relpos_attn_workspace_size", "relpos_attn_fwd", "relpos_attn_bwd", "relpos_attn_fwd_noalloc",
+           "relpos_attn_resolved_path", "relpos_strerror", "relpos_attn_version")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def lib_path() -> str:
@@ -72,6 +73,8 @@ def load() -> ctypes.CDLL:
     lib.relpos_attn_bwd.argtypes = [P, vp, vp, vp, ctypes.POINTER(vp), vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp), vp,
                                     ctypes.c_size_t, vp, vp]
     lib.relpos_attn_bwd.restype = ctypes.c_int
+    lib.relpos_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, ctypes.POINTER(vp), vp, vp, vp, vp]
+    lib.relpos_attn_fwd_noalloc.restype = ctypes.c_int
     lib.relpos_attn_resolved_path.argtypes = [P, ctypes.c_int]
     lib.relpos_attn_resolved_path.restype = ctypes.c_int
     lib.relpos_strerror.argtypes = [ctypes.c_int]
@@ -164,6 +167,16 @@ def relpos_attn_fwd(params: Params, q, k, v, rel, o, lse, workspace, dev_status=
                                 _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
     if rc != 0:
         raise RelposError(rc, "relpos_attn_fwd")
+
+
+def relpos_attn_fwd_noalloc(params: Params, q, k, v, rel, o, lse, dev_status=None, stream=None) -> None:
+    """Forward pass that allocates nothing: its scratch is the library's built-in
+    device array (see relpos_attn_fwd_noalloc in include/relpos_attn.h)."""
+    cp = params.c()
+    rc = load().relpos_attn_fwd_noalloc(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o),
+                                        _ptr(lse), _ptr(dev_status), _stream(stream))
+    if rc != 0:
+        raise RelposError(rc, "relpos_attn_fwd_noalloc")
 
 
 def relpos_attn_bwd(params: Params, q, k, v, rel, o, lse, dout, dq, dk, dv, drel, workspace, dev_status=None,

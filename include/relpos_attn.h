@@ -138,6 +138,27 @@ RELPOS_API int relpos_attn_bwd(const relpos_params_t *params,
                     void *workspace, size_t workspace_bytes,
                     int32_t *dev_status, void *stream);
 
+/* Size of the device scratch array built into the library for
+ * relpos_attn_fwd_noalloc (per GPU, held until the process exits). */
+#define RELPOS_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* relpos_attn_fwd for callers that cannot allocate device memory -- e.g. a plugin
+ * inside a framework that owns the whole device-memory budget, or a latency-critical
+ * loop where cudaMalloc / cudaFree would synchronise the device.  It has no
+ * counterpart in the paper; it is the same forward pass with its scratch taken from
+ * a static device array of RELPOS_NOALLOC_SCRATCH_BYTES instead of a caller
+ * workspace.  Arguments, outputs and errors are those of relpos_attn_fwd; a problem
+ * whose forward scratch (relpos_attn_workspace_size, pass 0) exceeds the array is
+ * rejected with RELPOS_ERR_WORKSPACE before anything is enqueued.  It allocates
+ * nothing.  All calls share the array: calls that may overlap on the GPU race and
+ * must be ordered by the caller.  The first call on a device looks up the array's
+ * device address (with that device current); make it before any stream capture. */
+RELPOS_API int relpos_attn_fwd_noalloc(const relpos_params_t *params,
+                                       const void *q, const void *k, const void *v,
+                                       const void *const rel[3],
+                                       void *o, float *lse,
+                                       int32_t *dev_status, void *stream);
+
 /* Kernel family that pass `pass` (0 forward, 1 backward) of a call with these
  * params runs: RELPOS_PATH_SIMT or RELPOS_PATH_TC (RELPOS_PATH_AUTO resolved),
  * or a negative RELPOS_ERR_* code (RELPOS_ERR_UNSUPPORTED when RELPOS_PATH_TC is
