@@ -3,14 +3,14 @@
 //
 // One CTA per 128-row query tile (heaviest causal tiles launched first), nine
 // warps:
-//   warps 0-7  "softmax": two threads per query row (warps w and w + 4 share TMEM
-//              lanes 32 (w & 3)..+31 and take key columns [0, 64) and [64, 128)).
+//   warps 0-15 "softmax": four threads per query row (warps w, w + 4, w + 8, w + 12
+//              share TMEM lanes 32 (w & 3)..+31 and take 32 key columns each).
 //              They read S = Q K^T and the relation products from TMEM, add the
 //              relative term gathered by offset, run the online softmax (row max
 //              exchanged through smem; lazy rescale of O only when the running max
 //              grows by more than 2^8), and write P (bf16) into shared memory in the
 //              128-byte-swizzled layout the tensor core reads.
-//   warp 8     lane 0 issues every TMA load (Q, K, V, relation-table windows,
+//   warp 16    lane 0 issues every TMA load (Q, K, V, relation-table windows,
 //              2-stage K/V ring) and every tcgen05.mma, and signals through
 //              mbarriers and tcgen05.commit.
 // TMEM (512 columns): S [0,128), relation products [128,384), O [384,448).
@@ -39,7 +39,10 @@ namespace rp {
 namespace tc {
 
 constexpr int BM = 128, BN = 128;
-constexpr int NSOFT = 256;    // softmax threads: two per query row
+constexpr int TPR = 4;             // softmax threads per query row
+constexpr int NC = 128 / TPR;      // key columns per softmax thread
+constexpr int NSOFT = 128 * TPR;   // softmax threads
+constexpr int CTRL_WARP = NSOFT / 32;
 constexpr int NTHREADS = NSOFT + 32;
 constexpr int ROT_LD = 132;  // fp32 stride of the per-row skew buffer (conflict-free rotations)
 
@@ -50,8 +53,8 @@ constexpr int OFF_P = OFF_V + 32768;    // two 64-key halves of P
 constexpr int OFF_R = OFF_P + 32768;    // relation-table staging (2 x 16 KB or one 32 KB window)
 constexpr int OFF_ROT = OFF_R + 32768;  // 128 x ROT_LD fp32
 constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;  // 2 x 512 fp32 per-tile vectors
-constexpr int OFF_RED = OFF_VEC + 2 * 512 * 4;  // 2 x 256 fp32 row-max exchange
-constexpr int OFF_BAR = OFF_RED + 2 * 256 * 4;
+constexpr int OFF_RED = OFF_VEC + 2 * 512 * 4;  // 2 x TPR x 128 fp32 row-max exchange
+constexpr int OFF_BAR = OFF_RED + 2 * TPR * 128 * 4;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   int32_t *status = p.status;
   const float c1 = p.scale * 1.4426950408889634f;  // scale * log2(e)
 
-  if (warp == 8) {
+  if (warp == CTRL_WARP) {
     // ======================= TMA + MMA issuer ==========================
     if (lane == 0) {
       prefetch_tmap(&A.mq);
@@ -268,10 +271,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     __syncwarp();
   } else {
     // ========================== softmax warps ===========================
-    // warp w: TMEM lanes 32 (w & 3) .. +31 (query rows), key columns [64 hf, 64 hf + 64), hf = w >> 2
-    const int g = warp & 3, hf = warp >> 2;
+    // warp w: TMEM lanes 32 (w & 3) .. +31 (query rows), key columns [NC qt, NC qt + NC), qt = w >> 2
+    const int g = warp & 3, qt = warp >> 2;
     const int il = 32 * g + lane, i = i0 + il;
-    const int cb = 64 * hf;  // first key column of this thread
+    const int cb = NC * qt;  // first key column of this thread
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     float *red = (float *)(smem + OFF_RED);
@@ -282,12 +285,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       cE0 = A.c2pE[((size_t)bh * L + i) * 2 + 0];
       cE1 = A.c2pE[((size_t)bh * L + i) * 2 + 1];
     }
-    if (MECH == M_SHAW) {  // QA row -> smem (kept for the whole CTA); 32-column chunks split by parity
+    if (MECH == M_SHAW) {  // QA row -> smem (kept for the whole CTA); 32-column chunks split by thread
       good = warp_wait(BAR(B_PFULLPRO), 0, abort_flag, status);
       if (good) {
         tc_fence_after();
         const int nq = (2 * p.clip + 1 + 31) / 32;
-        for (int q = hf; q < nq; q += 2) {
+        for (int q = qt; q < nq; q += TPR) {
           uint32_t r[32];
           tmem_ld32(tl + TM_REL + 32 * q, r);
           tmem_wait_ld();
@@ -301,75 +304,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       named_bar_sync(1, NSOFT);
     }
     int band_cnt = 0;
-    // per-tile vectors, fetched one key tile ahead (one or two elements per thread)
-    auto fetch_vec = [&](int n, float &va, float &vb) {
+    // per-tile vectors, fetched one key tile ahead (one element per thread)
+    auto fetch_vec = [&](int n) {
       const int j0 = n * BN, Delta = m - n;
-      va = 0.f;
-      vb = 0.f;
+      float va = 0.f;
       if (MECH == M_TXL) {
-        const int j = j0 + tid;
-        if (tid < 128 && j < L) va = A.uk[(size_t)bh * L + j];
-        const int rr = 128 * (tid < 128 ? Delta : Delta - 1) + (tid & 127) + p.off;
-        if (rr >= 0 && rr < p.nrows) vb = A.vr[(size_t)h * p.nrows + rr];
+        if (tid < 128) {
+          if (j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid];
+        } else if (tid < 384) {
+          const int rr = 128 * (tid < 256 ? Delta : Delta - 1) + ((tid - 128) & 127) + p.off;
+          if (rr >= 0 && rr < p.nrows) va = A.vr[(size_t)h * p.nrows + rr];
+        }
       } else if (MECH == M_T5) {
         const int idx = j0 - i0 - 127 + tid + L - 1;
         if (tid < 255 && idx >= 0 && idx < 2 * L - 1) va = p.t5_bias[(size_t)h * (2 * L - 1) + idx];
       } else if (MECH == M_DEB) {
         const int j = j0 + (tid >> 1);
-        if (j < L) va = A.p2cE[((size_t)bh * L + j) * 2 + (tid & 1)];
+        if (tid < 256 && j < L) va = A.p2cE[((size_t)bh * L + j) * 2 + (tid & 1)];
       }
+      return va;
     };
-    float nva, nvb;
-    fetch_vec(0, nva, nvb);
+    float nva = fetch_vec(0);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * BN, Delta = m - n;
       float *tv = vec + 512 * (n & 1);
-      if (MECH == M_TXL) {
-        if (tid < 128) tv[tid] = nva;
-        tv[128 + tid] = nvb;
-      } else if (MECH == M_T5) {
-        if (tid < 255) tv[tid] = nva;
-      } else if (MECH == M_DEB) {
-        tv[tid] = nva;
-      }
-      if (n + 1 < nTiles) fetch_vec(n + 1, nva, nvb);
+      if ((MECH == M_TXL && tid < 384) || (MECH == M_T5 && tid < 255) || (MECH == M_DEB && tid < 256)) tv[tid] = nva;
+      if (n + 1 < nTiles) nva = fetch_vec(n + 1);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
-      float x[64];
+      float x[NC];
       if (good) {
         tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(tl + TM_S + cb, r);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tl + TM_S + cb + 32 * q, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) x[32 * q + t] = u2f(r[t]);
-        }
+        for (int t = 0; t < NC; ++t) x[t] = u2f(r[t]);
       } else {
 #pragma unroll
-        for (int t = 0; t < 64; ++t) x[t] = 0.f;
+        for (int t = 0; t < NC; ++t) x[t] = 0.f;
       }
       // ---- relative term, gathered by offset ----
       if (MECH == M_TXL) {
         if (good) {
-          // this thread rotates offsets c in [cb, cb + 64) of its row into key order
+          // this thread rotates offsets c in [cb, cb + NC) of its row into key order
           const bool hasB = !(p.causal && Delta == 0);
           const uint32_t colA = TM_REL + 128 * (Delta & 1), colB = TM_REL + 128 * ((Delta - 1) & 1);
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t ra[32], rb[32];
-            tmem_ld32(tl + colA + cb + 32 * q, ra);
+          for (int hq = 0; hq < NC / 16; ++hq) {
+            uint32_t ra[16], rb[16];
+            tmem_ld16(tl + colA + cb + 16 * hq, ra);
             if (hasB) {
-              tmem_ld32(tl + colB + cb + 32 * q, rb);
+              tmem_ld16(tl + colB + cb + 16 * hq, rb);
             } else {
 #pragma unroll
-              for (int t = 0; t < 32; ++t) rb[t] = 0u;
+              for (int t = 0; t < 16; ++t) rb[t] = 0u;
             }
             tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              const int c = cb + 32 * q + t;
+            for (int t = 0; t < 16; ++t) {
+              const int c = cb + 16 * hq + t;
               const float va = u2f(ra[t]) + tv[128 + c];
               const float vb = hasB ? u2f(rb[t]) + tv[256 + c] : 0.f;
               rrow[(il - c) & 127] = (c <= il) ? va : vb;
@@ -380,7 +374,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
         named_bar_sync(1, NSOFT);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
           const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
           const float4 uk = *reinterpret_cast<const float4 *>(tv + cb + 4 * c4);
           x[4 * c4 + 0] = (x[4 * c4 + 0] + rr.x + uk.x) * c1;
@@ -396,7 +390,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         const float lg = 1.4426950408889634f;
         const float *bw = tv + cb - il + 127;
 #pragma unroll
-        for (int t = 0; t < 64; ++t) x[t] = x[t] * c1 + bw[t] * lg;
+        for (int t = 0; t < NC; ++t) x[t] = x[t] * c1 + bw[t] * lg;
       } else if (MECH == M_SHAW) {
         if (good) {
           tc_fence_before();
@@ -404,22 +398,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
         const int d0 = j0 + cb - i;
 #pragma unroll
-        for (int t = 0; t < 64; ++t) x[t] = (x[t] + rrow[iclamp(d0 + t, -p.clip, p.clip) + p.clip]) * c1;
+        for (int t = 0; t < NC; ++t) x[t] = (x[t] + rrow[iclamp(d0 + t, -p.clip, p.clip) + p.clip]) * c1;
       } else {  // DeBERTa
         const bool band = 128 * (Delta < 0 ? -Delta : Delta) - 127 < p.span;
         if (band) {
           // c2p: window column w (Kr row lo + w) belongs to key il + 127 - w; this
-          // thread handles w in [128 hf, 128 hf + 128)
+          // thread handles w in [64 qt, 64 qt + 64)
           if (good) {
             const int lo = p.span + 128 * Delta - 127;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
               uint32_t r[32];
-              tmem_ld32(tl + TM_REL + 128 * hf + 32 * q, r);
+              tmem_ld32(tl + TM_REL + 64 * qt + 32 * q, r);
               tmem_wait_ld();
 #pragma unroll
               for (int t = 0; t < 32; ++t) {
-                const int w = 128 * hf + 32 * q + t;
+                const int w = 64 * qt + 32 * q + t;
                 if (w >= il && w <= il + 127) {
                   const int rho = lo + w;
                   rrow[il + 127 - w] = (rho < 0) ? cE0 : (rho > 2 * p.span - 1 ? cE1 : u2f(r[t]));
@@ -431,7 +425,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           }
           named_bar_sync(1, NSOFT);
 #pragma unroll
-          for (int t = 0; t < 64; ++t) x[t] += rrow[cb + t];
+          for (int t = 0; t < NC; ++t) x[t] += rrow[cb + t];
           named_bar_sync(1, NSOFT);
           good = good && warp_wait(BAR(B_GFULL), band_cnt & 1, abort_flag, status);
           ++band_cnt;
@@ -442,13 +436,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             const int lo2 = p.span - 128 * Delta - 127;
             const float e0 = tv[2 * il], e1 = tv[2 * il + 1];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
               uint32_t r[32];
-              tmem_ld32(tl + TM_REL + 128 * hf + 32 * q, r);
+              tmem_ld32(tl + TM_REL + 64 * qt + 32 * q, r);
               tmem_wait_ld();
 #pragma unroll
               for (int t = 0; t < 32; ++t) {
-                const int w = 128 * hf + 32 * q + t;
+                const int w = 64 * qt + 32 * q + t;
                 if (w >= il && w <= il + 127) {
                   const int rho = lo2 + w;
                   rot[(il + 127 - w) * ROT_LD + il] = (rho < 0) ? e0 : (rho > 2 * p.span - 1 ? e1 : u2f(r[t]));
@@ -460,7 +454,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           }
           named_bar_sync(1, NSOFT);
 #pragma unroll
-          for (int t = 0; t < 64; ++t) x[t] = (x[t] + rrow[cb + t]) * c1;
+          for (int t = 0; t < NC; ++t) x[t] = (x[t] + rrow[cb + t]) * c1;
         } else {
           if (good) {
             tc_fence_before();
@@ -469,42 +463,44 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           const float c2p = Delta > 0 ? cE1 : cE0;
           const int sel = Delta < 0 ? 1 : 0;
 #pragma unroll
-          for (int t = 0; t < 64; ++t) x[t] = (x[t] + c2p + tv[2 * (cb + t) + sel]) * c1;
+          for (int t = 0; t < NC; ++t) x[t] = (x[t] + c2p + tv[2 * (cb + t) + sel]) * c1;
         }
       }
-      // ---- mask (diagonal / ragged tiles only), row max over both halves ----
+      // ---- mask (diagonal / ragged tiles only), row max over the row's threads ----
       const bool need_mask = (p.causal && n == m) || (j0 + BN > L);
       float mt = -INFINITY;
       if (need_mask) {
 #pragma unroll
-        for (int t = 0; t < 64; ++t) {
+        for (int t = 0; t < NC; ++t) {
           const int j = j0 + cb + t;
           if (j >= L || (p.causal && j > i)) x[t] = -INFINITY;
           mt = fmaxf(mt, x[t]);
         }
       } else {
 #pragma unroll
-        for (int t = 0; t < 64; ++t) mt = fmaxf(mt, x[t]);
+        for (int t = 0; t < NC; ++t) mt = fmaxf(mt, x[t]);
       }
-      float *rd = red + 256 * (n & 1);
-      rd[128 * hf + il] = mt;
+      float *rd = red + TPR * 128 * (n & 1);
+      rd[128 * qt + il] = mt;
       named_bar_sync(1, NSOFT);
-      mt = fmaxf(rd[il], rd[128 + il]);
+      mt = rd[il];
+#pragma unroll
+      for (int u = 1; u < TPR; ++u) mt = fmaxf(mt, rd[128 * u + il]);
       if (n == 0) {
         m2 = mt;
       } else {
-        const bool need = mt > m2 + 8.f;  // identical in both threads of the row
+        const bool need = mt > m2 + 8.f;  // identical in every thread of the row
         if (__any_sync(0xffffffffu, need)) {
           good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
           const float alpha = need ? ex2(m2 - mt) : 1.f;
           if (good) {
             tc_fence_after();
-            uint32_t r[32];
-            tmem_ld32(tl + TM_O + 32 * hf, r);
+            uint32_t r[16];
+            tmem_ld16(tl + TM_O + 16 * qt, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(u2f(r[t]) * alpha);
-            tmem_st32(tl + TM_O + 32 * hf, r);
+            for (int t = 0; t < 16; ++t) r[t] = __float_as_uint(u2f(r[t]) * alpha);
+            tmem_st16(tl + TM_O + 16 * qt, r);
             tmem_wait_st();
           }
           if (need) {
@@ -515,42 +511,46 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       }
       const float msub = (m2 == -INFINITY) ? 0.f : m2;
 #pragma unroll
-      for (int t = 0; t < 64; ++t) {
+      for (int t = 0; t < NC; ++t) {
         x[t] = ex2(x[t] - msub);
         lsum += x[t];
       }
       if (n >= 1) good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
       if (good) {
-        // P half-row -> smem sub-tile hf, K-major 128B swizzle: chunk c of row r at chunk c ^ (r & 7)
+        // P quarter-row -> smem sub-tile qt / 2, K-major 128B swizzle: chunk c of row r at chunk c ^ (r & 7)
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int cc = 0; cc < NC / 8; ++cc) {
+          const int ch = (NC / 8) * (qt & 1) + cc;
           uint4 v;
-          v.x = pack_bf16x2(x[8 * ch + 0], x[8 * ch + 1]);
-          v.y = pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]);
-          v.z = pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]);
-          v.w = pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]);
-          *reinterpret_cast<uint4 *>(smem + OFF_P + 16384 * hf + 128 * il + ((ch ^ (il & 7)) << 4)) = v;
+          v.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+          v.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+          v.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+          v.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+          *reinterpret_cast<uint4 *>(smem + OFF_P + 16384 * (qt >> 1) + 128 * il + ((ch ^ (il & 7)) << 4)) = v;
         }
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PFULL));
       }
     }
-    // ---- epilogue: O / l (l summed over the two halves), LSE ----
-    red[256 * (nTiles & 1) + 128 * hf + il] = lsum;
+    // ---- epilogue: O / l (l summed over the row's threads), LSE ----
+    float *rl = red + TPR * 128 * (nTiles & 1);
+    rl[128 * qt + il] = lsum;
     named_bar_sync(1, NSOFT);
-    const float ltot = red[256 * (nTiles & 1) + il] + red[256 * (nTiles & 1) + 128 + il];
+    float ltot = 0.f;
+#pragma unroll
+    for (int u = 0; u < TPR; ++u) ltot += rl[128 * u + il];
     good = good && warp_wait(BAR(B_PV), (nTiles - 1) & 1, abort_flag, status);
     if (good) {
       tc_fence_after();
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-      __nv_bfloat16 *orow = (__nv_bfloat16 *)p.out + ((size_t)bh * L + i) * HD + 32 * hf;
-      uint32_t r[32];
-      tmem_ld32(tl + TM_O + 32 * hf, r);
+      __nv_bfloat16 *orow = (__nv_bfloat16 *)p.out + ((size_t)bh * L + i) * HD + 16 * qt;
+      uint32_t r[16];
+      tmem_ld16(tl + TM_O + 16 * qt, r);
       tmem_wait_ld();
       if (i < L) {
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
+        for (int c8 = 0; c8 < 2; ++c8) {
           uint4 v;
           v.x = pack_bf16x2(u2f(r[8 * c8 + 0]) * inv, u2f(r[8 * c8 + 1]) * inv);
           v.y = pack_bf16x2(u2f(r[8 * c8 + 2]) * inv, u2f(r[8 * c8 + 3]) * inv);
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           v.w = pack_bf16x2(u2f(r[8 * c8 + 6]) * inv, u2f(r[8 * c8 + 7]) * inv);
           *reinterpret_cast<uint4 *>(orow + 8 * c8) = v;
         }
-        if (hf == 0) p.lse[(size_t)bh * L + i] = ltot > 0.f ? (m2 + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+        if (qt == 0) p.lse[(size_t)bh * L + i] = ltot > 0.f ? (m2 + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
       }
     }
     tc_fence_before();
