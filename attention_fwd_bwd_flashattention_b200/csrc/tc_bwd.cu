@@ -39,7 +39,10 @@ namespace tcb {
 
 using namespace tc;
 
-constexpr int NSOFT = 256;
+constexpr int TPR = 4;            // row threads per query row
+constexpr int NC = 128 / TPR;     // key columns per row thread
+constexpr int NSOFT = 128 * TPR;  // row threads
+constexpr int CTRL_WARP = NSOFT / 32;
 constexpr int NTHREADS = NSOFT + 32;
 constexpr int ROT_LD = 132;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -98,37 +101,19 @@ struct Ctl {
   }
 };
 
-// 64 values of row il, columns [64 hf, 64 hf + 64) of a 128 x 128 bf16 tile kept as
-// two 128B-swizzled 64-column sub-tiles.
-__device__ __forceinline__ void store_half_row(uint8_t *tile, int il, int hf, const float (&v)[64]) {
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * ch + 0], v[8 * ch + 1]);
-    w.y = pack_bf16x2(v[8 * ch + 2], v[8 * ch + 3]);
-    w.z = pack_bf16x2(v[8 * ch + 4], v[8 * ch + 5]);
-    w.w = pack_bf16x2(v[8 * ch + 6], v[8 * ch + 7]);
-    *reinterpret_cast<uint4 *>(tile + 16384 * hf + 128 * il + ((ch ^ (il & 7)) << 4)) = w;
-  }
-}
-__device__ __forceinline__ void store_elem(uint8_t *tile, int r, int c, float x) {
-  *reinterpret_cast<__nv_bfloat16 *>(tile + 16384 * (c >> 6) + 128 * r + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1)) =
-      __float2bfloat16_rn(x);
-}
-
 __device__ __forceinline__ uint32_t E_addr(int r, int c) {  // byte offset of (row r, even col c)
   return 16384 * (c >> 6) + 128 * r + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
 }
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
-// Move this thread's 64 dS values (keys jl = cb + e, e = 0..63) of row il into offset
-// coordinates: E_lo[il][c] (keys jl <= il) and E_hi[il][c] (keys jl > il) with
-// c = (il - jl) & 127, zero in the other tile.  The thread's offsets are s0 .. s0 + 63
-// (mod 128), s0 = (il - cb - 63) & 127, offset s0 + k holding x[63 - k]; they are
-// written as aligned bf16 pairs (4-byte stores).  When s0 is odd its first and last
-// offsets pair with the other half-row thread's values and are written alone.
-__device__ __forceinline__ void store_E(uint8_t *Elo, uint8_t *Ehi, int il, int cb, const float (&x)[64]) {
-  const int s0 = (il - cb - 63) & 127;
+// Move this thread's NC dS values (keys jl = cb + e, e = 0..NC-1) of row il into
+// offset coordinates: E_lo[il][c] (keys jl <= il) and E_hi[il][c] (keys jl > il) with
+// c = (il - jl) & 127, zero in the other tile.  The thread's offsets are s0 .. s0 + NC-1
+// (mod 128), s0 = (il - cb - NC + 1) & 127, offset s0 + k holding x[NC - 1 - k]; they
+// are written as aligned bf16 pairs (4-byte stores).  When s0 is odd the first and
+// last offsets pair with a neighbouring thread's values and are written alone.
+__device__ __forceinline__ void store_E(uint8_t *Elo, uint8_t *Ehi, int il, int cb, const float (&x)[NC]) {
+  const int s0 = (il - cb - NC + 1) & 127;
   const bool odd = (s0 & 1) != 0;
   const int c0 = s0 & ~1;
   auto put = [&](int c, float va, int ja, float vb, int jb) {  // pair (c, c + 1), c even
@@ -145,39 +130,39 @@ __device__ __forceinline__ void store_E(uint8_t *Elo, uint8_t *Ehi, int il, int 
   };
   // pair p >= 1 holds offsets c0 + 2p, c0 + 2p + 1: k = 2p - odd, 2p + 1 - odd
 #pragma unroll
-  for (int pp = 1; pp < 32; ++pp) {
-    const float va = odd ? x[64 - 2 * pp] : x[63 - 2 * pp];
-    const float vb = odd ? x[63 - 2 * pp] : x[62 - 2 * pp];
-    const int ea = odd ? 64 - 2 * pp : 63 - 2 * pp;
+  for (int pp = 1; pp < NC / 2; ++pp) {
+    const int ea = odd ? NC - 2 * pp : NC - 1 - 2 * pp;
+    const float va = odd ? x[NC - 2 * pp] : x[NC - 1 - 2 * pp];
+    const float vb = odd ? x[NC - 1 - 2 * pp] : x[NC - 2 - 2 * pp];
     put((c0 + 2 * pp) & 127, va, cb + ea, vb, cb + ea - 1);
   }
   if (!odd) {
-    put(c0, x[63], cb + 63, x[62], cb + 62);
+    put(c0, x[NC - 1], cb + NC - 1, x[NC - 2], cb + NC - 2);
   } else {
-    put1(s0, x[63], cb + 63);
-    put1((s0 + 63) & 127, x[0], cb);
+    put1(s0, x[NC - 1], cb + NC - 1);
+    put1((s0 + NC - 1) & 127, x[0], cb);
   }
 }
 
-// Rotate offsets c in [cb, cb + 64) of the two relation blocks (TMEM columns colA,
+// Rotate offsets c in [cb, cb + NC) of the two relation blocks (TMEM columns colA,
 // colB of this warp's lanes) into key order: rrow[(il - c) & 127] gets block Delta
 // for c <= il, block Delta - 1 otherwise, plus the per-offset v.r term.
 __device__ __forceinline__ void txl_rotate(uint32_t tl, uint32_t colA, uint32_t colB, bool hasB, int il, int cb,
                                            const float *vA, const float *vB, float *rrow) {
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    uint32_t ra[32], rb[32];
-    tmem_ld32(tl + colA + cb + 32 * q, ra);
+  for (int q = 0; q < NC / 16; ++q) {
+    uint32_t ra[16], rb[16];
+    tmem_ld16(tl + colA + cb + 16 * q, ra);
     if (hasB) {
-      tmem_ld32(tl + colB + cb + 32 * q, rb);
+      tmem_ld16(tl + colB + cb + 16 * q, rb);
     } else {
 #pragma unroll
-      for (int t = 0; t < 32; ++t) rb[t] = 0u;
+      for (int t = 0; t < 16; ++t) rb[t] = 0u;
     }
     tmem_wait_ld();
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      const int c = cb + 32 * q + t;
+    for (int t = 0; t < 16; ++t) {
+      const int c = cb + 16 * q + t;
       const float va = u2f(ra[t]) + vA[c];
       const float vb = hasB ? u2f(rb[t]) + vB[c] : 0.f;
       rrow[(il - c) & 127] = (c <= il) ? va : vb;
@@ -249,7 +234,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
       Ctl ctl;
       ctl.np = 0;
@@ -321,7 +306,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     }
     __syncwarp();
   } else {
-    const int g = warp & 3, hf = warp >> 2, il = 32 * g + lane, cb = 64 * hf;
+    const int g = warp & 3, qt = warp >> 2, il = 32 * g + lane, cb = NC * qt;
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
@@ -331,7 +316,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
       dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
       const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
-      vrv = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+      vrv = (tid < 256 && rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
     };
     float nl2, ndv, nvr;
     fetch(0, nl2, ndv, nvr);
@@ -339,7 +324,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       const int m = mStart + t, D = m - n, i = m * 128 + il;
       const float lse2 = nl2, Dv = ndv;
       float *tv = vec + 128 + 256 * (t & 1);  // v.r of blocks D (c < 128) and D - 1
-      tv[tid] = nvr;
+      if (tid < 256) tv[tid] = nvr;
       if (t + 1 < iters) fetch(t + 1, nl2, ndv, nvr);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
@@ -351,81 +336,79 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
           txl_rotate(tl, 0, 128, hasB, il, cb, tv, tv + 128, rrow);
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) rrow[(il - cb - c) & 127] = 0.f;
+          for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
         }
         tc_fence_before();
         mbar_arrive(BAR(B_TCONS));
       }
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
-      // P and dS of this thread's 64 keys, packed to bf16 pairs as they are made
-      uint32_t pk[32], dk[32];
+      // P and dS of this thread's NC keys, packed to bf16 pairs as they are made
+      uint32_t pk[NC / 2], dk[NC / 2];
       const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tl + T_S + cb, rs);
+        tmem_ld32(tl + T_DP + cb, rp);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t rs[32], rp[32];
-          tmem_ld32(tl + T_S + cb + 32 * q, rs);
-          tmem_ld32(tl + T_DP + cb + 32 * q, rp);
-          tmem_wait_ld();
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
+          const int x0 = 4 * c4;
+          const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
+          const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
+          const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+          float pr[4], dd[4];
 #pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const int x0 = 32 * q + 4 * c4;
-            const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
-            const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
-            const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
-            float pr[4], dd[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float y = (u2f(rs[4 * c4 + e]) + rv[e]) * c1;
-              if (need_mask) {
-                const int j = j0 + cb + x0 + e;
-                if (j >= L || (p.causal && j > i)) y = -INFINITY;
-              }
-              pr[e] = ex2(y - lse2);
-              dd[e] = pr[e] * (u2f(rp[4 * c4 + e]) - Dv);
+          for (int e = 0; e < 4; ++e) {
+            float y = (u2f(rs[x0 + e]) + rv[e]) * c1;
+            if (need_mask) {
+              const int j = j0 + cb + x0 + e;
+              if (j >= L || (p.causal && j > i)) y = -INFINITY;
             }
-            pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
-            pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-            dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
-            dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
+            pr[e] = ex2(y - lse2);
+            dd[e] = pr[e] * (u2f(rp[x0 + e]) - Dv);
           }
+          pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
+          pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+          dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
+          dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
         }
         tc_fence_before();
       }
       named_bar_sync(1, NSOFT);  // every rot row read; the P / dS tiles overwrite them
       if (good) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t off = 16384 * hf + 128 * il + ((ch ^ (il & 7)) << 4);
-          *reinterpret_cast<uint4 *>(smem + OFF_ROT + off) = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        for (int cc = 0; cc < NC / 8; ++cc) {
+          const int ch = (NC / 8) * (qt & 1) + cc;
+          const uint32_t off = 16384 * (qt >> 1) + 128 * il + ((ch ^ (il & 7)) << 4);
+          *reinterpret_cast<uint4 *>(smem + OFF_ROT + off) = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
           *reinterpret_cast<uint4 *>(smem + OFF_ROT + 32768 + off) =
-              make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+              make_uint4(dk[4 * cc], dk[4 * cc + 1], dk[4 * cc + 2], dk[4 * cc + 3]);
         }
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
     }
-    // ---- epilogue: lanes are keys now ----
+    // ---- epilogue: lanes are keys now; this thread takes 16 of the 64 columns ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
     const int j = j0 + il;
     float csum = 0.f;
     if (good) {
       tc_fence_after();
-      uint32_t rv[32], rk[32], rc[16];
-      tmem_ld32(tl + T_DV + 32 * hf, rv);
-      tmem_ld32(tl + T_DK + 32 * hf, rk);
+      uint32_t rv[16], rk[16], rc[16];
+      tmem_ld16(tl + T_DV + 16 * qt, rv);
+      tmem_ld16(tl + T_DK + 16 * qt, rk);
       tmem_ld16(tl + T_CS, rc);
       tmem_wait_ld();
       csum = u2f(rc[0]);
       if (j < L) {
-        const __nv_bfloat16 *u = (const __nv_bfloat16 *)p.rel1 + (size_t)h * HD + 32 * hf;
-        __nv_bfloat16 *dvp = (__nv_bfloat16 *)p.dv + ((size_t)bh * L + j) * HD + 32 * hf;
-        __nv_bfloat16 *dkp = (__nv_bfloat16 *)p.dk + ((size_t)bh * L + j) * HD + 32 * hf;
+        const __nv_bfloat16 *u = (const __nv_bfloat16 *)p.rel1 + (size_t)h * HD + 16 * qt;
+        __nv_bfloat16 *dvp = (__nv_bfloat16 *)p.dv + ((size_t)bh * L + j) * HD + 16 * qt;
+        __nv_bfloat16 *dkp = (__nv_bfloat16 *)p.dk + ((size_t)bh * L + j) * HD + 16 * qt;
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
+        for (int c8 = 0; c8 < 2; ++c8) {
           float kv[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) kv[e] = p.scale * (u2f(rk[8 * c8 + e]) + csum * __bfloat162float(u[8 * c8 + e]));
@@ -447,7 +430,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     }
     // du partial: s * sum_j c_j k_j over this key tile (fixed order)
     named_bar_sync(1, NSOFT);
-    if (hf == 0) vec[il] = csum;
+    if (qt == 0) vec[il] = csum;
     named_bar_sync(1, NSOFT);
     if (tid < HD) {
       const __nv_bfloat16 *kp = (const __nv_bfloat16 *)p.k + (size_t)bh * L * HD;
@@ -515,7 +498,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
       Ctl ctl;
       ctl.np = 0;
@@ -596,58 +579,58 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     }
     __syncwarp();
   } else {
-    const int g = warp & 3, hf = warp >> 2, il = 32 * g + lane, cb = 64 * hf;
+    const int g = warp & 3, qt = warp >> 2, il = 32 * g + lane, cb = NC * qt;
     const int i = i0 + il;
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
     bool good = true;
-    auto fetch = [&](int n, float &ukv, float &vrv) {  // one key tile ahead
+    auto fetch = [&](int n) {  // one key tile ahead: uk (tid < 128), v.r of blocks D, D - 1
       const int j0 = n * 128, D = m - n;
-      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
-      const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
-      vrv = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+      float v = 0.f;
+      if (tid < 128) {
+        if (j0 + tid < L) v = A.uk[(size_t)bh * L + j0 + tid];
+      } else if (tid < 384) {
+        const int rr = 128 * (tid < 256 ? D : D - 1) + ((tid - 128) & 127) + p.off;
+        if (rr >= 0 && rr < p.nrows) v = A.vr[(size_t)h * p.nrows + rr];
+      }
+      return v;
     };
-    float nuk, nvr;
-    fetch(0, nuk, nvr);
+    float nv = fetch(0);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * 128, D = m - n;
       float *tu = vec + 384 * (n & 1);  // uk[128] | v.r block D [128] | v.r block D - 1 [128]
-      if (tid < 128) tu[tid] = nuk;
-      tu[128 + tid] = nvr;
-      if (n + 1 < nTiles) fetch(n + 1, nuk, nvr);
+      if (tid < 384) tu[tid] = nv;
+      if (n + 1 < nTiles) nv = fetch(n + 1);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
       const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
-      float x[64];
+      float x[NC];
       if (good) {
         tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(tl + T_S + cb, r);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tl + T_S + cb + 32 * q, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[32 * q + e] = u2f(r[e]);
-        }
+        for (int e = 0; e < NC; ++e) x[e] = u2f(r[e]);
         if (hasA) {
           txl_rotate(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, il, cb, tu + 128, tu + 256, rrow);
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) rrow[(il - cb - c) & 127] = 0.f;
+          for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
         }
         tc_fence_before();
         mbar_arrive(BAR(B_TCONS));
       } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) x[e] = 0.f;
+        for (int e = 0; e < NC; ++e) x[e] = 0.f;
       }
       named_bar_sync(1, NSOFT);
       const bool need_mask = (p.causal && n == m) || (j0 + 128 > L);
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < NC / 4; ++c4) {
         const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
         const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
         const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
@@ -665,22 +648,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       good = good && warp_wait(BAR(B_DPF), n & 1, abort_flag, status);
       if (good) {
         tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(tl + T_REL + 128 * (D & 1) + cb, r);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tl + T_REL + 128 * (D & 1) + cb + 32 * q, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[32 * q + e] = x[32 * q + e] * (u2f(r[e]) - Dv);
-        }
+        for (int e = 0; e < NC; ++e) x[e] = x[e] * (u2f(r[e]) - Dv);
         tc_fence_before();
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-        tmem_st32(tl + T_DS + 32 * hf, pk);
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        tmem_st16(tl + T_DS + 16 * qt, pk);
         store_E(smem + OFF_ROT, smem + OFF_ROT + 32768, il, cb, x);
         tmem_wait_st();
         fence_async_smem();
@@ -691,13 +671,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     good = good && warp_wait(BAR(B_PDSFREE), (nTiles - 1) & 1, abort_flag, status);
     if (good) {
       tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tl + T_DQ + 32 * hf, r);
+      uint32_t r[16];
+      tmem_ld16(tl + T_DQ + 16 * qt, r);
       tmem_wait_ld();
       if (i < L) {
-        __nv_bfloat16 *dqp = (__nv_bfloat16 *)p.dq + ((size_t)bh * L + i) * HD + 32 * hf;
+        __nv_bfloat16 *dqp = (__nv_bfloat16 *)p.dq + ((size_t)bh * L + i) * HD + 16 * qt;
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
+        for (int c8 = 0; c8 < 2; ++c8) {
           uint4 w;
           w.x = pack_bf16x2(p.scale * u2f(r[8 * c8 + 0]), p.scale * u2f(r[8 * c8 + 1]));
           w.y = pack_bf16x2(p.scale * u2f(r[8 * c8 + 2]), p.scale * u2f(r[8 * c8 + 3]));
@@ -768,7 +748,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
-  {  // v.r of the band's two blocks (fixed for the CTA)
+  if (tid < 256) {  // v.r of the band's two blocks (fixed for the CTA)
     const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
     vec[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
   }
@@ -779,7 +759,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
       Ctl ctl;
       ctl.np = 0;
@@ -861,7 +841,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     }
     __syncwarp();
   } else {
-    const int g = warp & 3, hf = warp >> 2, il = 32 * g + lane, cb = 64 * hf;
+    const int g = warp & 3, qt = warp >> 2, il = 32 * g + lane, cb = NC * qt;
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
@@ -888,50 +868,41 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
           txl_rotate(tl, 0, 128, hasB, il, cb, vec + 128, vec + 256, rrow);
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) rrow[(il - cb - c) & 127] = 0.f;
+          for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
         }
         tc_fence_before();
         mbar_arrive(BAR(B_TCONS));
       }
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
-      float pv[64], ds[64];
+      float ds[NC];
+      const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tl + T_S + cb, rs);
+        tmem_ld32(tl + T_DP + cb, rp);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t rs[32], rp[32];
-          tmem_ld32(tl + T_S + cb + 32 * q, rs);
-          tmem_ld32(tl + T_DP + cb + 32 * q, rp);
-          tmem_wait_ld();
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
+          const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
+          const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
+          const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            pv[32 * q + x] = u2f(rs[x]);
-            ds[32 * q + x] = u2f(rp[x]);
+          for (int e = 0; e < 4; ++e) {
+            const int x = 4 * c4 + e;
+            float y = (u2f(rs[x]) + rv[e]) * c1;
+            if (need_mask) {
+              const int j = j0 + cb + x;
+              if (j >= L || (p.causal && j > i)) y = -INFINITY;
+            }
+            ds[x] = ex2(y - lse2) * (u2f(rp[x]) - Dv);
           }
         }
         tc_fence_before();
       } else {
 #pragma unroll
-        for (int x = 0; x < 64; ++x) pv[x] = ds[x] = 0.f;
-      }
-      const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
-#pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
-        const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
-        const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int x = 4 * c4 + e;
-          float y = (pv[x] + rv[e]) * c1;
-          if (need_mask) {
-            const int j = j0 + cb + x;
-            if (j >= L || (p.causal && j > i)) y = -INFINITY;
-          }
-          const float pr = ex2(y - lse2);
-          ds[x] = pr * (ds[x] - Dv);
-        }
+        for (int x = 0; x < NC; ++x) ds[x] = 0.f;
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
@@ -941,23 +912,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         mbar_arrive(BAR(B_PDS));
       }
     }
-    // ---- epilogue: lane il now is offset c = il of both blocks ----
+    // ---- epilogue: lane il now is offset c = il of both blocks; 16 columns per thread ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
     if (good) {
       tc_fence_after();
-      uint32_t rlo[32], rhi[32], glo[16], ghi[16];
-      tmem_ld32(tl + T_GLO + 32 * hf, rlo);
-      tmem_ld32(tl + T_GHI + 32 * hf, rhi);
+      uint32_t rlo[16], rhi[16], glo[16], ghi[16];
+      tmem_ld16(tl + T_GLO + 16 * qt, rlo);
+      tmem_ld16(tl + T_GHI + 16 * qt, rhi);
       tmem_ld16(tl + T_GL, glo);
       tmem_ld16(tl + T_GH, ghi);
       tmem_wait_ld();
       float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        part[(size_t)il * 65 + 32 * hf + e] = u2f(rlo[e]);
-        part[(size_t)(128 + il) * 65 + 32 * hf + e] = u2f(rhi[e]);
+      for (int e = 0; e < 16; ++e) {
+        part[(size_t)il * 65 + 16 * qt + e] = u2f(rlo[e]);
+        part[(size_t)(128 + il) * 65 + 16 * qt + e] = u2f(rhi[e]);
       }
-      if (hf == 0) {
+      if (qt == 0) {
         part[(size_t)il * 65 + 64] = u2f(glo[0]);
         part[(size_t)(128 + il) * 65 + 64] = u2f(ghi[0]);
       }
