@@ -52,7 +52,7 @@ struct BwdArgs {
   Prm p;                 // nT counts 128-row tiles
   const float *uk, *vr;  // u.k_j [B,H,L], v.r_rho [H,rows]
   float *part_kv;        // [B,H,nT][64]  du partial per key tile
-  float *part_dg;        // [B,H,nbands,nchunk][2][128][65] diagonal partials (G then g)
+  float *part_dg;        // [B,H,nbands,nchunk][2][65][128] diagonal partials (G then g)
   int dg_ch, dg_nchunk, nbands;
 };
 
@@ -348,31 +348,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
-        uint32_t rs[32], rp[32];
-        tmem_ld32(tl + T_S + cb, rs);
-        tmem_ld32(tl + T_DP + cb, rp);
-        tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < NC / 4; ++c4) {
-          const int x0 = 4 * c4;
-          const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
-          const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
-          const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
-          float pr[4], dd[4];
+        for (int hq = 0; hq < NC / 16; ++hq) {
+          uint32_t rs[16], rp[16];
+          tmem_ld16(tl + T_S + cb + 16 * hq, rs);
+          tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float y = (u2f(rs[x0 + e]) + rv[e]) * c1;
-            if (need_mask) {
-              const int j = j0 + cb + x0 + e;
-              if (j >= L || (p.causal && j > i)) y = -INFINITY;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int x0 = 16 * hq + 4 * c4;
+            const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
+            const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
+            const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+            float pr[4], dd[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float y = (u2f(rs[4 * c4 + e]) + rv[e]) * c1;
+              if (need_mask) {
+                const int j = j0 + cb + x0 + e;
+                if (j >= L || (p.causal && j > i)) y = -INFINITY;
+              }
+              pr[e] = ex2(y - lse2);
+              dd[e] = pr[e] * (u2f(rp[4 * c4 + e]) - Dv);
             }
-            pr[e] = ex2(y - lse2);
-            dd[e] = pr[e] * (u2f(rp[x0 + e]) - Dv);
+            pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
+            pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+            dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
+            dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
           }
-          pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
-          pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-          dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
-          dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
         }
         tc_fence_before();
       }
@@ -879,24 +882,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
-        uint32_t rs[32], rp[32];
-        tmem_ld32(tl + T_S + cb, rs);
-        tmem_ld32(tl + T_DP + cb, rp);
-        tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < NC / 4; ++c4) {
-          const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
-          const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
-          const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+        for (int hq = 0; hq < NC / 16; ++hq) {
+          uint32_t rs[16], rp[16];
+          tmem_ld16(tl + T_S + cb + 16 * hq, rs);
+          tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int x = 4 * c4 + e;
-            float y = (u2f(rs[x]) + rv[e]) * c1;
-            if (need_mask) {
-              const int j = j0 + cb + x;
-              if (j >= L || (p.causal && j > i)) y = -INFINITY;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int x0 = 16 * hq + 4 * c4;
+            const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
+            const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + x0);
+            const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float y = (u2f(rs[4 * c4 + e]) + rv[e]) * c1;
+              if (need_mask) {
+                const int j = j0 + cb + x0 + e;
+                if (j >= L || (p.causal && j > i)) y = -INFINITY;
+              }
+              ds[x0 + e] = ex2(y - lse2) * (u2f(rp[4 * c4 + e]) - Dv);
             }
-            ds[x] = ex2(y - lse2) * (u2f(rp[x]) - Dv);
           }
         }
         tc_fence_before();
@@ -922,15 +928,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       tmem_ld16(tl + T_GL, glo);
       tmem_ld16(tl + T_GH, ghi);
       tmem_wait_ld();
+      // partial layout [block lo / hi][65][128 offsets]: G columns 0..63, then g
       float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        part[(size_t)il * 65 + 16 * qt + e] = u2f(rlo[e]);
-        part[(size_t)(128 + il) * 65 + 16 * qt + e] = u2f(rhi[e]);
+        part[(size_t)(16 * qt + e) * 128 + il] = u2f(rlo[e]);
+        part[(size_t)(65 + 16 * qt + e) * 128 + il] = u2f(rhi[e]);
       }
       if (qt == 0) {
-        part[(size_t)il * 65 + 64] = u2f(glo[0]);
-        part[(size_t)(128 + il) * 65 + 64] = u2f(ghi[0]);
+        part[(size_t)64 * 128 + il] = u2f(glo[0]);
+        part[(size_t)(65 + 64) * 128 + il] = u2f(ghi[0]);
       }
     }
     tc_fence_before();
@@ -949,7 +956,8 @@ __global__ void reduce_dr_kernel(BwdArgs A) {
   const size_t per = (size_t)p.nrows * HD;
   const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (x >= (size_t)p.H * per) return;
-  const int h = (int)(x / per), rho = (int)((x % per) / HD), e = (int)(x % HD);
+  // consecutive threads take consecutive offsets (the partials are offset-contiguous)
+  const int h = (int)(x / per), e = (int)((x % per) / p.nrows), rho = (int)(x % p.nrows);
   const int delta = rho - p.off;
   const int blk = delta >= 0 ? delta / 128 : -((-delta + 127) / 128);
   const int c = delta - 128 * blk;
@@ -963,14 +971,14 @@ __global__ void reduce_dr_kernel(BwdArgs A) {
       const int len = p.nT - (D < 0 ? -D : D);
       const int nch = (len + A.dg_ch - 1) / A.dg_ch;
       for (int ch = 0; ch < nch; ++ch) {
-        const float *part = A.part_dg + ((bh * A.nbands + band) * A.dg_nchunk + ch) * DG_STRIDE + (size_t)(128 * w + c) * 65;
-        acc += part[e];
-        gs += part[64];
+        const float *part = A.part_dg + ((bh * A.nbands + band) * A.dg_nchunk + ch) * DG_STRIDE + (size_t)(65 * w) * 128 + c;
+        acc += part[(size_t)e * 128];
+        gs += part[(size_t)64 * 128];
       }
     }
   }
   const float vv = __bfloat162float(((const __nv_bfloat16 *)p.rel2)[(size_t)h * HD + e]);
-  p.drel0[x] = p.scale * (acc + gs * vv);
+  p.drel0[((size_t)h * p.nrows + rho) * HD + e] = p.scale * (acc + gs * vv);
   if (e == 0) p.gtot[(size_t)h * p.nrows + rho] = gs;
 }
 
