@@ -161,11 +161,18 @@ __device__ __forceinline__ void txl_rotate(uint32_t tl, uint32_t colA, uint32_t 
     }
     tmem_wait_ld();
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const int c = cb + 16 * q + t;
-      const float va = u2f(ra[t]) + vA[c];
-      const float vb = hasB ? u2f(rb[t]) + vB[c] : 0.f;
-      rrow[(il - c) & 127] = (c <= il) ? va : vb;
+    for (int c4 = 0; c4 < 4; ++c4) {
+      // the per-offset terms are the same for every lane: one broadcast 16-byte load
+      const float4 a4 = *reinterpret_cast<const float4 *>(vA + cb + 16 * q + 4 * c4);
+      const float4 b4 = *reinterpret_cast<const float4 *>(vB + cb + 16 * q + 4 * c4);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 4 * c4 + e, c = cb + 16 * q + t;
+        const float va = u2f(ra[t]) + av[e];
+        const float vb = hasB ? u2f(rb[t]) + bv[e] : 0.f;
+        rrow[(il - c) & 127] = (c <= il) ? va : vb;
+      }
     }
   }
 }

@@ -362,11 +362,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             }
             tmem_wait_ld();
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              const int c = cb + 16 * hq + t;
-              const float va = u2f(ra[t]) + tv[128 + c];
-              const float vb = hasB ? u2f(rb[t]) + tv[256 + c] : 0.f;
-              rrow[(il - c) & 127] = (c <= il) ? va : vb;
+            for (int c4 = 0; c4 < 4; ++c4) {
+              // per-offset v.r, the same for every lane: one broadcast 16-byte load
+              const float4 a4 = *reinterpret_cast<const float4 *>(tv + 128 + cb + 16 * hq + 4 * c4);
+              const float4 b4 = *reinterpret_cast<const float4 *>(tv + 256 + cb + 16 * hq + 4 * c4);
+              const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int t = 4 * c4 + e, c = cb + 16 * hq + t;
+                const float va = u2f(ra[t]) + av[e];
+                const float vb = hasB ? u2f(rb[t]) + bv[e] : 0.f;
+                rrow[(il - c) & 127] = (c <= il) ? va : vb;
+              }
             }
           }
           tc_fence_before();
