@@ -33,6 +33,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
+#include "tc_skew.cuh"
 
 namespace rp {
 namespace tcb {
@@ -144,39 +145,6 @@ __device__ __forceinline__ void store_E(uint8_t *Elo, uint8_t *Ehi, int il, int 
   }
 }
 
-// Rotate offsets c in [cb, cb + NC) of the two relation blocks (TMEM columns colA,
-// colB of this warp's lanes) into key order: rrow[(il - c) & 127] gets block Delta
-// for c <= il, block Delta - 1 otherwise, plus the per-offset v.r term.
-__device__ __forceinline__ void txl_rotate(uint32_t tl, uint32_t colA, uint32_t colB, bool hasB, int il, int cb,
-                                           const float *vA, const float *vB, float *rrow) {
-#pragma unroll
-  for (int q = 0; q < NC / 16; ++q) {
-    uint32_t ra[16], rb[16];
-    tmem_ld16(tl + colA + cb + 16 * q, ra);
-    if (hasB) {
-      tmem_ld16(tl + colB + cb + 16 * q, rb);
-    } else {
-#pragma unroll
-      for (int t = 0; t < 16; ++t) rb[t] = 0u;
-    }
-    tmem_wait_ld();
-#pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
-      // the per-offset terms are the same for every lane: one broadcast 16-byte load
-      const float4 a4 = *reinterpret_cast<const float4 *>(vA + cb + 16 * q + 4 * c4);
-      const float4 b4 = *reinterpret_cast<const float4 *>(vB + cb + 16 * q + 4 * c4);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = 4 * c4 + e, c = cb + 16 * q + t;
-        const float va = u2f(ra[t]) + av[e];
-        const float vb = hasB ? u2f(rb[t]) + bv[e] : 0.f;
-        rrow[(il - c) & 127] = (c <= il) ? va : vb;
-      }
-    }
-  }
-}
-
 // Offset block b of r (rows 128 b + off .. +127) exists unless causal and b < 0.
 __device__ __forceinline__ bool block_valid(const Prm &p, int b) { return !(p.causal && b < 0); }
 __device__ __forceinline__ int slot3(int b) { return ((b % 3) + 3) % 3; }
@@ -188,7 +156,7 @@ namespace kv {
 constexpr int OFF_K = 0, OFF_V = 16384, OFF_Q = 32768, OFF_DO = OFF_Q + 32768, OFF_R = OFF_DO + 32768;
 constexpr int OFF_ROT = OFF_R + 3 * 16384;            // rot rows; P tile at +0, dS tile at +32768
 constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;  // [16][128] bf16 ones, K-major (2 x 2 KB)
-constexpr int OFF_VEC = OFF_ONES + 4096;              // uk[128] + vr[2][256]
+constexpr int OFF_VEC = OFF_ONES + 4096;              // uk[128], then the du column sums
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 enum { B_KV = 0, B_ST0, B_ST1, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
@@ -290,9 +258,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         if (t == 0 && !ctl.wait_load(BAR(B_KV), 0)) break;
         if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
         tc_fence_after();
-        if (block_valid(p, D)) umma_k64(tbase + 0, sbase + OFF_Q + 16384 * st, sbase + OFF_R + 16384 * slot3(D), idS, false);
+        // relation products transposed (lane = offset, column = query row)
+        if (block_valid(p, D)) umma_k64(tbase + 0, sbase + OFF_R + 16384 * slot3(D), sbase + OFF_Q + 16384 * st, idS, false);
         if (block_valid(p, D - 1))
-          umma_k64(tbase + 128, sbase + OFF_Q + 16384 * st, sbase + OFF_R + 16384 * slot3(D - 1), idS, false);
+          umma_k64(tbase + 128, sbase + OFF_R + 16384 * slot3(D - 1), sbase + OFF_Q + 16384 * st, idS, false);
         umma_commit(BAR(B_TFULL));
         if (t >= 1) accumulate(t - 1);
         if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
@@ -317,22 +286,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
-    // row statistics and v.r of the next query tile, fetched one iteration ahead
-    auto fetch = [&](int t, float &l2, float &dv, float &vrv) {
+    // row statistics and this thread's v.r (offset 32 g + lane of blocks D, D - 1) of
+    // the next query tile, fetched one iteration ahead
+    auto fetch = [&](int t, float &l2, float &dv, float &va, float &vb) {
       const int m = mStart + t, D = m - n, i = m * 128 + il;
       l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
       dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
-      const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
-      vrv = (tid < 256 && rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
+      const int ra = 128 * D + il + p.off, rb = ra - 128;
+      va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
+      vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
     };
-    float nl2, ndv, nvr;
-    fetch(0, nl2, ndv, nvr);
+    float nl2, ndv, nva, nvb;
+    fetch(0, nl2, ndv, nva, nvb);
     for (int t = 0; t < iters; ++t) {
       const int m = mStart + t, D = m - n, i = m * 128 + il;
-      const float lse2 = nl2, Dv = ndv;
-      float *tv = vec + 128 + 256 * (t & 1);  // v.r of blocks D (c < 128) and D - 1
-      if (tid < 256) tv[tid] = nvr;
-      if (t + 1 < iters) fetch(t + 1, nl2, ndv, nvr);
+      const float lse2 = nl2, Dv = ndv, vrA = nva, vrB = nvb;
+      if (t + 1 < iters) fetch(t + 1, nl2, ndv, nva, nvb);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
@@ -340,7 +309,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_rotate(tl, 0, 128, hasB, il, cb, tv, tv + 128, rrow);
+          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, vrA, vrB, rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -539,9 +508,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       if (ok) {
         tc_fence_after();
         umma_k64(tbase + T_S, sbase + OFF_Q, sbase + OFF_K, idS, false);
-        if (block_valid(p, m)) umma_k64(tbase + T_REL + 128 * (m & 1), sbase + OFF_Q, sbase + OFF_R + 16384 * slot3(m), idS, false);
+        // relation products transposed (lane = offset, column = query row)
+        if (block_valid(p, m)) umma_k64(tbase + T_REL + 128 * (m & 1), sbase + OFF_R + 16384 * slot3(m), sbase + OFF_Q, idS, false);
         if (block_valid(p, m - 1))
-          umma_k64(tbase + T_REL + 128 * ((m - 1) & 1), sbase + OFF_Q, sbase + OFF_R + 16384 * slot3(m - 1), idS, false);
+          umma_k64(tbase + T_REL + 128 * ((m - 1) & 1), sbase + OFF_R + 16384 * slot3(m - 1), sbase + OFF_Q, idS, false);
         umma_commit(BAR(B_SFULL));
       }
       for (int n = 0; ok && n < nTiles; ++n) {
@@ -577,7 +547,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         umma_commit(BAR(B_PDSFREE));
         if (n + 1 < nTiles) {  // relation block D - 2 for tile n + 1, into the slot dP(n) used
           if (block_valid(p, D - 2))
-            umma_k64(tbase + slotA, sbase + OFF_Q, sbase + OFF_R + 16384 * slot3(D - 2), idS, false);
+            umma_k64(tbase + slotA, sbase + OFF_R + 16384 * slot3(D - 2), sbase + OFF_Q, idS, false);
           umma_commit(BAR(B_SFULL));
         }
         if (n + 2 < nTiles) {
@@ -596,23 +566,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
     bool good = true;
-    auto fetch = [&](int n) {  // one key tile ahead: uk (tid < 128), v.r of blocks D, D - 1
+    // one key tile ahead: uk (tid < 128) and this thread's v.r (offset il of blocks D, D - 1)
+    auto fetch = [&](int n, float &ukv, float &va, float &vb) {
       const int j0 = n * 128, D = m - n;
-      float v = 0.f;
-      if (tid < 128) {
-        if (j0 + tid < L) v = A.uk[(size_t)bh * L + j0 + tid];
-      } else if (tid < 384) {
-        const int rr = 128 * (tid < 256 ? D : D - 1) + ((tid - 128) & 127) + p.off;
-        if (rr >= 0 && rr < p.nrows) v = A.vr[(size_t)h * p.nrows + rr];
-      }
-      return v;
+      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      const int ra = 128 * D + il + p.off, rb = ra - 128;
+      va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
+      vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
     };
-    float nv = fetch(0);
+    float nuk, nva, nvb;
+    fetch(0, nuk, nva, nvb);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * 128, D = m - n;
-      float *tu = vec + 384 * (n & 1);  // uk[128] | v.r block D [128] | v.r block D - 1 [128]
-      if (tid < 384) tu[tid] = nv;
-      if (n + 1 < nTiles) nv = fetch(n + 1);
+      float *tu = vec + 128 * (n & 1);  // uk of key tile n
+      if (tid < 128) tu[tid] = nuk;
+      const float vrA = nva, vrB = nvb;
+      if (n + 1 < nTiles) fetch(n + 1, nuk, nva, nvb);
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
@@ -620,17 +589,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       float x[NC];
       if (good) {
         tc_fence_after();
+        if (hasA) {
+          txl_skew<ROT_LD>(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, g, qt, lane, vrA, vrB, rot);
+        } else {
+#pragma unroll
+          for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
+        }
         uint32_t r[32];
         tmem_ld32(tl + T_S + cb, r);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < NC; ++e) x[e] = u2f(r[e]);
-        if (hasA) {
-          txl_rotate(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, il, cb, tu + 128, tu + 256, rrow);
-        } else {
-#pragma unroll
-          for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
-        }
         tc_fence_before();
         mbar_arrive(BAR(B_TCONS));
       } else {
@@ -758,10 +727,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
-  if (tid < 256) {  // v.r of the band's two blocks (fixed for the CTA)
-    const int rr = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
-    vec[128 + tid] = (rr >= 0 && rr < p.nrows) ? A.vr[(size_t)h * p.nrows + rr] : 0.f;
-  }
   fence_async_smem();
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
   tc_fence_before();
@@ -823,8 +788,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         if (!ctl.wait_load(BAR(B_ST0 + st), (t >> 1) & 1)) break;
         if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
         tc_fence_after();
-        if (hasA) umma_k64(tbase + 0, sbase + OFF_Q + 16384 * st, sbase + OFF_R, idS, false);
-        if (hasB) umma_k64(tbase + 128, sbase + OFF_Q + 16384 * st, sbase + OFF_R + 16384, idS, false);
+        // relation products transposed (lane = offset, column = query row)
+        if (hasA) umma_k64(tbase + 0, sbase + OFF_R, sbase + OFF_Q + 16384 * st, idS, false);
+        if (hasB) umma_k64(tbase + 128, sbase + OFF_R + 16384, sbase + OFF_Q + 16384 * st, idS, false);
         umma_commit(BAR(B_TFULL));
         if (t >= 1) accumulate(t - 1);
         if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
@@ -855,6 +821,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
+    // v.r of offset il of the band's two blocks (fixed for the CTA)
+    const int ra = 128 * D + il + p.off, rb = ra - 128;
+    const float vrA = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
+    const float vrB = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
     auto fetch = [&](int t, float &l2, float &dv, float &ukv) {  // one tile ahead
       const int m = m0 + t, i = m * 128 + il, j0 = (m - D) * 128;
       l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
@@ -875,7 +845,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_rotate(tl, 0, 128, hasB, il, cb, vec + 128, vec + 256, rrow);
+          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, vrA, vrB, rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;

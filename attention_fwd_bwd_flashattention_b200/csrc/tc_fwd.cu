@@ -21,10 +21,11 @@
 //   Shaw     QA = Q a^T (129 products per row) computed once per query tile by one
 //            MMA and kept in smem; each pair reads its clipped column.
 //   TXL      the offsets of tile (m, n) are 128 (m - n) + [-127, 127]: two
-//            128-offset blocks of r.  Block b's products Q r_b^T are computed by
+//            128-offset blocks of r.  Block b's products r_b Q^T are computed by
 //            one 128x128x64 MMA and reused by the two consecutive key tiles that
 //            need it, so each key tile adds exactly one new block.  Each row's
-//            values are rotated into key order through a padded smem row.
+//            products are computed transposed (lane = offset) and written into
+//            key order through padded smem rows.
 //   DeBERTa  tiles within the span: c2p = Q Kr_win^T (255 offsets) rotated per row,
 //            p2c = K Qr_win^T computed with keys as rows and transposed through
 //            smem; tiles outside the span use per-row / per-key end products.
@@ -34,6 +35,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
+#include "tc_skew.cuh"
 
 namespace rp {
 namespace tc {
@@ -224,9 +226,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         tc_fence_after();
         umma_k64(tbase + TM_S, sbase + OFF_Q, sbase + OFF_K + 16384 * st, idS, false);
         if (MECH == M_TXL) {
-          if (n == 0) umma_k64(tbase + TM_REL + 128 * (m & 1), sbase + OFF_Q, sbase + OFF_P, idS, false);
+          // relation products transposed (lane = offset, column = query row)
+          if (n == 0) umma_k64(tbase + TM_REL + 128 * (m & 1), sbase + OFF_P, sbase + OFF_Q, idS, false);
           if (needs_new_block(n))
-            umma_k64(tbase + TM_REL + 128 * ((Delta - 1) & 1), sbase + OFF_Q, sbase + OFF_R + 16384 * st, idS, false);
+            umma_k64(tbase + TM_REL + 128 * ((Delta - 1) & 1), sbase + OFF_R + 16384 * st, sbase + OFF_Q, idS, false);
         }
         const bool band = (MECH == M_DEB) && (128 * (Delta < 0 ? -Delta : Delta) - 127 < p.span);
         if (band) {
@@ -306,15 +309,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     int band_cnt = 0;
     // per-tile vectors, fetched one key tile ahead (one element per thread)
     auto fetch_vec = [&](int n) {
-      const int j0 = n * BN, Delta = m - n;
+      const int j0 = n * BN;
       float va = 0.f;
       if (MECH == M_TXL) {
-        if (tid < 128) {
-          if (j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid];
-        } else if (tid < 384) {
-          const int rr = 128 * (tid < 256 ? Delta : Delta - 1) + ((tid - 128) & 127) + p.off;
-          if (rr >= 0 && rr < p.nrows) va = A.vr[(size_t)h * p.nrows + rr];
-        }
+        if (tid < 128 && j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid];
       } else if (MECH == M_T5) {
         const int idx = j0 - i0 - 127 + tid + L - 1;
         if (tid < 255 && idx >= 0 && idx < 2 * L - 1) va = p.t5_bias[(size_t)h * (2 * L - 1) + idx];
@@ -324,12 +322,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       }
       return va;
     };
-    float nva = fetch_vec(0);
+    // TXL: this thread's v.r, offset il of blocks Delta and Delta - 1, one key tile ahead
+    auto fetch_vr = [&](int n, float &va, float &vb) {
+      if (MECH == M_TXL) {
+        const int ra = 128 * (m - n) + il + p.off, rb = ra - 128;
+        va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
+        vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
+      }
+    };
+    float nva = fetch_vec(0), nvrA = 0.f, nvrB = 0.f;
+    fetch_vr(0, nvrA, nvrB);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * BN, Delta = m - n;
       float *tv = vec + 512 * (n & 1);
-      if ((MECH == M_TXL && tid < 384) || (MECH == M_T5 && tid < 255) || (MECH == M_DEB && tid < 256)) tv[tid] = nva;
-      if (n + 1 < nTiles) nva = fetch_vec(n + 1);
+      if ((MECH == M_TXL && tid < 128) || (MECH == M_T5 && tid < 255) || (MECH == M_DEB && tid < 256)) tv[tid] = nva;
+      const float vrA = nvrA, vrB = nvrB;
+      if (n + 1 < nTiles) {
+        nva = fetch_vec(n + 1);
+        fetch_vr(n + 1, nvrA, nvrB);
+      }
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       float x[NC];
@@ -347,35 +358,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       // ---- relative term, gathered by offset ----
       if (MECH == M_TXL) {
         if (good) {
-          // this thread rotates offsets c in [cb, cb + NC) of its row into key order
           const bool hasB = !(p.causal && Delta == 0);
-          const uint32_t colA = TM_REL + 128 * (Delta & 1), colB = TM_REL + 128 * ((Delta - 1) & 1);
-#pragma unroll
-          for (int hq = 0; hq < NC / 16; ++hq) {
-            uint32_t ra[16], rb[16];
-            tmem_ld16(tl + colA + cb + 16 * hq, ra);
-            if (hasB) {
-              tmem_ld16(tl + colB + cb + 16 * hq, rb);
-            } else {
-#pragma unroll
-              for (int t = 0; t < 16; ++t) rb[t] = 0u;
-            }
-            tmem_wait_ld();
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              // per-offset v.r, the same for every lane: one broadcast 16-byte load
-              const float4 a4 = *reinterpret_cast<const float4 *>(tv + 128 + cb + 16 * hq + 4 * c4);
-              const float4 b4 = *reinterpret_cast<const float4 *>(tv + 256 + cb + 16 * hq + 4 * c4);
-              const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int t = 4 * c4 + e, c = cb + 16 * hq + t;
-                const float va = u2f(ra[t]) + av[e];
-                const float vb = hasB ? u2f(rb[t]) + bv[e] : 0.f;
-                rrow[(il - c) & 127] = (c <= il) ? va : vb;
-              }
-            }
-          }
+          txl_skew<ROT_LD>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane, vrA, vrB, rot);
           tc_fence_before();
           mbar_arrive(BAR(B_SFREE));
         }
