@@ -29,6 +29,7 @@
 // and du = s sum_j c_j k_j.
 #include <algorithm>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -65,6 +66,19 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Four log2-domain scores y = s c1 + (r' + u') - lse2 of consecutive keys, from the
+// QK^T accumulator bits, the relative terms r' and u.k terms u' (both already
+// multiplied by c1 = scale log2 e) and nlse = (-lse2, -lse2); two f32x2 pairs.
+__device__ __forceinline__ void score_pairs(const uint32_t *s, float4 rr, float4 uk, uint64_t c12, uint64_t nlse, float (&y)[4]) {
+  f2_split(fma2(f2(u2f(s[0]), u2f(s[1])), c12, add2(add2(f2(rr.x, rr.y), f2(uk.x, uk.y)), nlse)), y[0], y[1]);
+  f2_split(fma2(f2(u2f(s[2]), u2f(s[3])), c12, add2(add2(f2(rr.z, rr.w), f2(uk.z, uk.w)), nlse)), y[2], y[3]);
+}
+// dS = P (dP - D) for four keys, nDv = (-D, -D).
+__device__ __forceinline__ void ds_pairs(const float (&pr)[4], const uint32_t *dp, uint64_t nDv, float (&dd)[4]) {
+  f2_split(mul2(f2(pr[0], pr[1]), add2(f2(u2f(dp[0]), u2f(dp[1])), nDv)), dd[0], dd[1]);
+  f2_split(mul2(f2(pr[2], pr[3]), add2(f2(u2f(dp[2]), u2f(dp[3])), nDv)), dd[2], dd[3]);
+}
+
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *ab, int32_t *st) {
   const bool ok = mbar_wait(bar, parity, ab, st, RELPOS_ERR_TIMEOUT_DEV);
   return __all_sync(0xffffffffu, ok);
@@ -201,7 +215,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
-  if (tid < 128) vec[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+  if (tid < 128) vec[tid] = (j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] * c1 : 0.f;  // u.k, pre-scaled
   fence_async_smem();
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
   tc_fence_before();
@@ -309,7 +323,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, vrA, vrB, rot);
+          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, c1, vrA * c1, vrB * c1, rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -324,35 +338,39 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
+        const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
+        auto pds = [&](auto masked) {
 #pragma unroll
-        for (int hq = 0; hq < NC / 16; ++hq) {
-          uint32_t rs[16], rp[16];
-          tmem_ld16(tl + T_S + cb + 16 * hq, rs);
-          tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
-          tmem_wait_ld();
+          for (int hq = 0; hq < NC / 16; ++hq) {
+            uint32_t rs[16], rp[16];
+            tmem_ld16(tl + T_S + cb + 16 * hq, rs);
+            tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int x0 = 16 * hq + 4 * c4;
-            const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
-            const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
-            const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
-            float pr[4], dd[4];
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const int x0 = 16 * hq + 4 * c4;
+              const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
+              const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
+              float y[4], pr[4], dd[4];
+              score_pairs(rs + 4 * c4, rr, uk, c12, nlse, y);
+              if constexpr (decltype(masked)::value) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float y = (u2f(rs[4 * c4 + e]) + rv[e]) * c1;
-              if (need_mask) {
-                const int j = j0 + cb + x0 + e;
-                if (j >= L || (p.causal && j > i)) y = -INFINITY;
+                for (int e = 0; e < 4; ++e) {
+                  const int j = j0 + cb + x0 + e;
+                  if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+                }
               }
-              pr[e] = ex2(y - lse2);
-              dd[e] = pr[e] * (u2f(rp[4 * c4 + e]) - Dv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) pr[e] = ex2(y[e]);
+              ds_pairs(pr, rp + 4 * c4, nDv, dd);
+              pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
+              pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
+              dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
+              dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
             }
-            pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
-            pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
-            dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
-            dk[x0 / 2 + 1] = pack_bf16x2(dd[2], dd[3]);
           }
-        }
+        };
+        if (need_mask) pds(std::true_type{}); else pds(std::false_type{});
         tc_fence_before();
       }
       named_bar_sync(1, NSOFT);  // every rot row read; the P / dS tiles overwrite them
@@ -565,11 +583,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     float *rrow = rot + il * ROT_LD;
     const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+    const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
     bool good = true;
     // one key tile ahead: uk (tid < 128) and this thread's v.r (offset il of blocks D, D - 1)
     auto fetch = [&](int n, float &ukv, float &va, float &vb) {
       const int j0 = n * 128, D = m - n;
-      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] * c1 : 0.f;  // pre-scaled
       const int ra = 128 * D + il + p.off, rb = ra - 128;
       va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
       vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
@@ -590,7 +609,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_skew<ROT_LD>(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, g, qt, lane, vrA, vrB, rot);
+          txl_skew<ROT_LD>(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, g, qt, lane, c1, vrA * c1, vrB * c1,
+                           rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -608,22 +628,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       }
       named_bar_sync(1, NSOFT);
       const bool need_mask = (p.causal && n == m) || (j0 + 128 > L);
+      auto probs = [&](auto masked) {  // x <- P = 2^(s c1 + r' + u' - lse2)
 #pragma unroll
-      for (int c4 = 0; c4 < NC / 4; ++c4) {
-        const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
-        const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
-        const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
+          const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
+          const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + 4 * c4);
+          const uint32_t sb[4] = {__float_as_uint(x[4 * c4]), __float_as_uint(x[4 * c4 + 1]), __float_as_uint(x[4 * c4 + 2]),
+                                  __float_as_uint(x[4 * c4 + 3])};
+          float y[4];
+          score_pairs(sb, rr, uk, c12, nlse, y);
+          if constexpr (decltype(masked)::value) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int xx = 4 * c4 + e;
-          float y = (x[xx] + rv[e]) * c1;
-          if (need_mask) {
-            const int j = j0 + cb + xx;
-            if (j >= L || (p.causal && j > i)) y = -INFINITY;
+            for (int e = 0; e < 4; ++e) {
+              const int j = j0 + cb + 4 * c4 + e;
+              if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+            }
           }
-          x[xx] = ex2(y - lse2);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[4 * c4 + e] = ex2(y[e]);
         }
-      }
+      };
+      if (need_mask) probs(std::true_type{}); else probs(std::false_type{});
       good = good && warp_wait(BAR(B_DPF), n & 1, abort_flag, status);
       if (good) {
         tc_fence_after();
@@ -631,7 +656,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         tmem_ld32(tl + T_REL + 128 * (D & 1) + cb, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < NC; ++e) x[e] = x[e] * (u2f(r[e]) - Dv);
+        for (int c4 = 0; c4 < NC / 4; ++c4) {
+          const float pr[4] = {x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]};
+          float dd[4];
+          ds_pairs(pr, r + 4 * c4, nDv, dd);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[4 * c4 + e] = dd[e];
+        }
         tc_fence_before();
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
@@ -829,7 +860,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       const int m = m0 + t, i = m * 128 + il, j0 = (m - D) * 128;
       l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
       dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
-      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] : 0.f;
+      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] * c1 : 0.f;  // pre-scaled
     };
     float nl2, ndv, nuk;
     fetch(0, nl2, ndv, nuk);
@@ -845,7 +876,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, vrA, vrB, rot);
+          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, c1, vrA * c1, vrB * c1, rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -859,29 +890,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
+        const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
+        auto pds = [&](auto masked) {
 #pragma unroll
-        for (int hq = 0; hq < NC / 16; ++hq) {
-          uint32_t rs[16], rp[16];
-          tmem_ld16(tl + T_S + cb + 16 * hq, rs);
-          tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
-          tmem_wait_ld();
+          for (int hq = 0; hq < NC / 16; ++hq) {
+            uint32_t rs[16], rp[16];
+            tmem_ld16(tl + T_S + cb + 16 * hq, rs);
+            tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int x0 = 16 * hq + 4 * c4;
-            const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
-            const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + x0);
-            const float rv[4] = {rr.x + uk.x, rr.y + uk.y, rr.z + uk.z, rr.w + uk.w};
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const int x0 = 16 * hq + 4 * c4;
+              const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
+              const float4 uk = *reinterpret_cast<const float4 *>(tu + cb + x0);
+              float y[4], pr[4], dd[4];
+              score_pairs(rs + 4 * c4, rr, uk, c12, nlse, y);
+              if constexpr (decltype(masked)::value) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float y = (u2f(rs[4 * c4 + e]) + rv[e]) * c1;
-              if (need_mask) {
-                const int j = j0 + cb + x0 + e;
-                if (j >= L || (p.causal && j > i)) y = -INFINITY;
+                for (int e = 0; e < 4; ++e) {
+                  const int j = j0 + cb + x0 + e;
+                  if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+                }
               }
-              ds[x0 + e] = ex2(y - lse2) * (u2f(rp[4 * c4 + e]) - Dv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) pr[e] = ex2(y[e]);
+              ds_pairs(pr, rp + 4 * c4, nDv, dd);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) ds[x0 + e] = dd[e];
             }
           }
-        }
+        };
+        if (need_mask) pds(std::true_type{}); else pds(std::false_type{});
         tc_fence_before();
       } else {
 #pragma unroll
