@@ -116,46 +116,51 @@ struct Ctl {
   }
 };
 
-__device__ __forceinline__ uint32_t E_addr(int r, int c) {  // byte offset of (row r, even col c)
-  return 16384 * (c >> 6) + 128 * r + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1);
+// dS of this thread's NC keys (jl = cb + e, e = 0..NC-1) of row il, written into
+// the two 128x128 bf16 operand tiles of the relation products in offset order
+// (128-byte-swizzled K-major, 64-column halves 16 KB apart; E_lo at E, E_hi at
+// E + 32768).  In the combined offset c' = il - jl + 128, c' >= 128 is E_lo column
+// c' - 128 (keys jl <= il) and c' < 128 is E_hi column c' (keys jl > il); the value's
+// partner c' ^ 128 in the other tile gets 0, so both tiles are fully rewritten.
+// x[e] sits at c' = C0 - e, C0 = il - cb + 128: values go out as aligned bf16 pairs;
+// when C0 is even the first and last value pair with a neighbouring thread's and
+// are written alone.
+__device__ __forceinline__ uint32_t E_off(uint32_t t, uint32_t rowb, uint32_t r7) {  // t = 2 c', c' even
+  return (((t << 7) & 0xC000u) ^ 0x8000u) + rowb + ((t & 126u) ^ r7);
 }
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
-
-// Move this thread's NC dS values (keys jl = cb + e, e = 0..NC-1) of row il into
-// offset coordinates: E_lo[il][c] (keys jl <= il) and E_hi[il][c] (keys jl > il) with
-// c = (il - jl) & 127, zero in the other tile.  The thread's offsets are s0 .. s0 + NC-1
-// (mod 128), s0 = (il - cb - NC + 1) & 127, offset s0 + k holding x[NC - 1 - k]; they
-// are written as aligned bf16 pairs (4-byte stores).  When s0 is odd the first and
-// last offsets pair with a neighbouring thread's values and are written alone.
-__device__ __forceinline__ void store_E(uint8_t *Elo, uint8_t *Ehi, int il, int cb, const float (&x)[NC]) {
-  const int s0 = (il - cb - NC + 1) & 127;
-  const bool odd = (s0 & 1) != 0;
-  const int c0 = s0 & ~1;
-  auto put = [&](int c, float va, int ja, float vb, int jb) {  // pair (c, c + 1), c even
-    const bool la = ja <= il, lb = jb <= il;
-    const uint32_t off = E_addr(il, c);
-    *reinterpret_cast<uint32_t *>(Elo + off) = pack2(la ? va : 0.f, lb ? vb : 0.f);
-    *reinterpret_cast<uint32_t *>(Ehi + off) = pack2(la ? 0.f : va, lb ? 0.f : vb);
-  };
-  auto put1 = [&](int c, float v, int jj) {  // single element
-    const uint32_t off = E_addr(il, c & ~1) + ((c & 1) << 1);
-    const bool l = jj <= il;
-    *reinterpret_cast<__nv_bfloat16 *>(Elo + off) = __float2bfloat16_rn(l ? v : 0.f);
-    *reinterpret_cast<__nv_bfloat16 *>(Ehi + off) = __float2bfloat16_rn(l ? 0.f : v);
-  };
-  // pair p >= 1 holds offsets c0 + 2p, c0 + 2p + 1: k = 2p - odd, 2p + 1 - odd
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const float (&x)[NC]) {
+  const uint32_t C0 = (uint32_t)(il - cb + 128);
+  const bool ev = (C0 & 1u) == 0;
+  const uint32_t rowb = 128u * (uint32_t)il, r7 = (uint32_t)(il & 7) << 4;
+  const uint32_t T0 = 2u * ((C0 - 1u) & ~1u);  // 2 c' of the first whole pair
+  // pk[k] = (x[2k+1], x[2k]) is the pair at c' = C0 - 2k - 1 when C0 is odd; when it
+  // is even the pair at c' = C0 - 2k - 2 is (x[2k+2], x[2k+1]): high half of pk[k+1],
+  // low half of pk[k], picked by one byte permute
+  uint32_t pk[NC / 2];
 #pragma unroll
-  for (int pp = 1; pp < NC / 2; ++pp) {
-    const int ea = odd ? NC - 2 * pp : NC - 1 - 2 * pp;
-    const float va = odd ? x[NC - 2 * pp] : x[NC - 1 - 2 * pp];
-    const float vb = odd ? x[NC - 1 - 2 * pp] : x[NC - 2 - 2 * pp];
-    put((c0 + 2 * pp) & 127, va, cb + ea, vb, cb + ea - 1);
+  for (int k = 0; k < NC / 2; ++k) pk[k] = pack_bf16x2(x[2 * k + 1], x[2 * k]);
+  const uint32_t sel = ev ? 0x1076u : 0x3210u;
+#pragma unroll
+  for (int k = 0; k < NC / 2 - 1; ++k) {
+    const uint32_t off = E_off(T0 - 4u * k, rowb, r7);
+    *reinterpret_cast<uint32_t *>(E + off) = prmt(pk[k], pk[k + 1], sel);
+    *reinterpret_cast<uint32_t *>(E + (off ^ 0x8000u)) = 0u;
   }
-  if (!odd) {
-    put(c0, x[NC - 1], cb + NC - 1, x[NC - 2], cb + NC - 2);
+  if (!ev) {
+    const uint32_t off = E_off(T0 - 4u * (NC / 2 - 1), rowb, r7);
+    *reinterpret_cast<uint32_t *>(E + off) = pk[NC / 2 - 1];
+    *reinterpret_cast<uint32_t *>(E + (off ^ 0x8000u)) = 0u;
   } else {
-    put1(s0, x[NC - 1], cb + NC - 1);
-    put1((s0 + NC - 1) & 127, x[0], cb);
+    const uint32_t o0 = E_off(2u * C0, rowb, r7), o1 = E_off(2u * (C0 - NC), rowb, r7) + 2u;
+    *reinterpret_cast<uint16_t *>(E + o0) = (uint16_t)(pk[0] >> 16);
+    *reinterpret_cast<uint16_t *>(E + (o0 ^ 0x8000u)) = 0;
+    *reinterpret_cast<uint16_t *>(E + o1) = (uint16_t)(pk[NC / 2 - 1] & 0xFFFFu);
+    *reinterpret_cast<uint16_t *>(E + (o1 ^ 0x8000u)) = 0;
   }
 }
 
@@ -671,7 +676,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
         tmem_st16(tl + T_DS + 16 * qt, pk);
-        store_E(smem + OFF_ROT, smem + OFF_ROT + 32768, il, cb, x);
+        store_E(smem + OFF_ROT, il, cb, x);
         tmem_wait_st();
         fence_async_smem();
         tc_fence_before();
@@ -928,7 +933,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
-        store_E(smem + OFF_ROT, smem + OFF_ROT + 32768, il, cb, ds);
+        store_E(smem + OFF_ROT, il, cb, ds);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
