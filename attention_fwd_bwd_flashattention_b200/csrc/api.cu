@@ -136,7 +136,7 @@ static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
 struct Layout {
   size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot;
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
-  size_t part_kv, part_dg;    // tensor-core backward partials
+  size_t part_kv, part_dg, part_uv;  // tensor-core backward partials
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -173,7 +173,7 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
     l.vr = take(sizeof(float) * (size_t)p.H * p.nrows);
     l.part_kv = take(sizeof(float) * kvf);
     l.part_dg = take(sizeof(float) * dgf);
-    l.gtot = take(sizeof(float) * (size_t)p.H * p.nrows);
+    l.part_uv = take(sizeof(float) * (size_t)p.H * ((p.nrows + 31) / 32) * rp::HD);
   } else if (pass == 1) {
     l.dvec = take(sizeof(float) * BH * p.L);
     const size_t tab = (size_t)p.nrows * rp::HD;
@@ -218,6 +218,7 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.p2cE = (float *)(b + l.p2cE);
   w.part_kv = (float *)(b + l.part_kv);
   w.part_dg = (float *)(b + l.part_dg);
+  w.part_uv = (float *)(b + l.part_uv);
   return w;
 }
 

@@ -12,6 +12,7 @@ cudaError_t simt_bwd(const Prm &p, bool bf16, cudaStream_t st);
 struct TcWork {
   float *uk, *vr, *c2pE, *p2cE;  // per-call products (Transformer-XL, DeBERTa)
   float *part_kv, *part_dg;      // backward partials (Transformer-XL)
+  float *part_uv;                // [H][ceil(rows / 32)][64] dv partials per 32-offset tile
 };
 bool tc_supported(const Prm &p);
 cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st);

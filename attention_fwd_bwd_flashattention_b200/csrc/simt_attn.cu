@@ -395,15 +395,22 @@ __device__ __forceinline__ void zero_W(float *W, int nw) {
 // ---------------------------------------------------------------------------
 // D_i = dO_i . O_i
 // ---------------------------------------------------------------------------
+// eight threads per 64-element row (a warp reads four whole rows), fixed shuffle tree
 template <class T>
-__global__ void dvec_kernel(Prm p) {
+__global__ void __launch_bounds__(256) dvec_kernel(Prm p) {
   const size_t n = (size_t)p.B * p.H * p.L;
-  const size_t row = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= n) return;
-  const T *o = (const T *)p.o + row * HD, *g = (const T *)p.dout + row * HD;
+  const size_t row = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int sub = threadIdx.x & 7;
   float acc = 0.f;
-  for (int c = 0; c < HD; ++c) acc = fmaf(ldf(o, c), ldf(g, c), acc);
-  p.Dvec[row] = acc;
+  if (row < n) {
+    const T *o = (const T *)p.o + row * HD + 8 * sub, *g = (const T *)p.dout + row * HD + 8 * sub;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc = fmaf(ldf(o, c), ldf(g, c), acc);
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  if (row < n && sub == 0) p.Dvec[row] = acc;
 }
 
 // ---------------------------------------------------------------------------
@@ -813,7 +820,7 @@ template <int MECH, class T>
 static cudaError_t run_bwd_t(const Prm &p, cudaStream_t st) {
   cudaError_t e;
   const size_t rows = (size_t)p.B * p.H * p.L;
-  dvec_kernel<T><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+  dvec_kernel<T><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   auto kq = bwd_q_kernel<MECH, T>;
   auto kkv = bwd_kv_kernel<MECH, T>;
@@ -867,9 +874,9 @@ __global__ void t5_prep_kernel(Prm p) {
 cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st) {
   const size_t rows = (size_t)p.B * p.H * p.L;
   if (bf16)
-    simt::dvec_kernel<__nv_bfloat16><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+    simt::dvec_kernel<__nv_bfloat16><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p);
   else
-    simt::dvec_kernel<float><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+    simt::dvec_kernel<float><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

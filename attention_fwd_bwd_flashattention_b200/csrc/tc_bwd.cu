@@ -55,6 +55,7 @@ struct BwdArgs {
   const float *uk, *vr;  // u.k_j [B,H,L], v.r_rho [H,rows]
   float *part_kv;        // [B,H,nT][64]  du partial per key tile
   float *part_dg;        // [B,H,nbands,nchunk][2][65][128] diagonal partials (G then g)
+  float *part_uv;        // [H][ceil(rows / 32)][64] dv partials per 32-offset tile
   int dg_ch, dg_nchunk, nbands;
 };
 
@@ -971,59 +972,88 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
 }
 
 // dr[h][rho][e] = s (sum G + (sum g) v[e]) over the batch, the bands holding
-// offset delta = rho - off (as block D or D - 1) and their chunks; gtot gets sum g.
-__global__ void reduce_dr_kernel(BwdArgs A) {
+// offset delta = rho - off (as block D or D - 1) and their chunks, in a fixed order.
+// One CTA per 32 consecutive offsets (the lanes; the partials are offset-contiguous,
+// so each warp load is one 128-byte run) and 8 warps of 8 columns e each.  The CTA
+// also writes the dv partial of its 32 offsets, sum_rho (sum g)_rho r_rho[e], reduced
+// over the lanes by a fixed shuffle tree.
+__global__ void __launch_bounds__(256) reduce_dr_kernel(BwdArgs A) {
   const Prm &p = A.p;
-  const size_t per = (size_t)p.nrows * HD;
-  const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (x >= (size_t)p.H * per) return;
-  // consecutive threads take consecutive offsets (the partials are offset-contiguous)
-  const int h = (int)(x / per), e = (int)((x % per) / p.nrows), rho = (int)(x % p.nrows);
-  const int delta = rho - p.off;
-  const int blk = delta >= 0 ? delta / 128 : -((-delta + 127) / 128);
-  const int c = delta - 128 * blk;
-  float acc = 0.f, gs = 0.f;
-  for (int bb = 0; bb < p.B; ++bb) {
-    const size_t bh = (size_t)bb * p.H + h;
-    for (int w = 0; w < 2; ++w) {  // w = 0: band blk (block = D); w = 1: band blk + 1 (block = D - 1)
-      const int D = blk + w;
-      const int band = p.causal ? D : D + (p.nT - 1);
-      if (band < 0 || band >= A.nbands) continue;
-      const int len = p.nT - (D < 0 ? -D : D);
-      const int nch = (len + A.dg_ch - 1) / A.dg_ch;
-      for (int ch = 0; ch < nch; ++ch) {
-        const float *part = A.part_dg + ((bh * A.nbands + band) * A.dg_nchunk + ch) * DG_STRIDE + (size_t)(65 * w) * 128 + c;
-        acc += part[(size_t)e * 128];
-        gs += part[(size_t)64 * 128];
+  const int ntile = (p.nrows + 31) / 32;
+  const int h = (int)blockIdx.x / ntile, tile = (int)blockIdx.x % ntile;
+  const int lane = threadIdx.x & 31, eg = threadIdx.x >> 5;
+  const int rho = 32 * tile + lane;
+  const bool ok = rho < p.nrows;
+  float acc[8], gs = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+  if (ok) {
+    const int delta = rho - p.off;
+    const int blk = delta >= 0 ? delta / 128 : -((-delta + 127) / 128);
+    const int c = delta - 128 * blk;
+    for (int bb = 0; bb < p.B; ++bb) {
+      const size_t bh = (size_t)bb * p.H + h;
+      for (int w = 0; w < 2; ++w) {  // w = 0: band blk (block = D); w = 1: band blk + 1 (block = D - 1)
+        const int D = blk + w;
+        const int band = p.causal ? D : D + (p.nT - 1);
+        if (band < 0 || band >= A.nbands) continue;
+        const int len = p.nT - (D < 0 ? -D : D);
+        const int nch = (len + A.dg_ch - 1) / A.dg_ch;
+        for (int ch = 0; ch < nch; ++ch) {
+          const float *part = A.part_dg + ((bh * A.nbands + band) * A.dg_nchunk + ch) * DG_STRIDE + (size_t)(65 * w) * 128 + c;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] += part[(size_t)(8 * eg + k) * 128];
+          gs += part[(size_t)64 * 128];
+        }
       }
     }
   }
-  const float vv = __bfloat162float(((const __nv_bfloat16 *)p.rel2)[(size_t)h * HD + e]);
-  p.drel0[((size_t)h * p.nrows + rho) * HD + e] = p.scale * (acc + gs * vv);
-  if (e == 0) p.gtot[(size_t)h * p.nrows + rho] = gs;
+  const __nv_bfloat16 *vv = (const __nv_bfloat16 *)p.rel2 + (size_t)h * HD + 8 * eg;
+  const __nv_bfloat16 *rr = (const __nv_bfloat16 *)p.rel0 + ((size_t)h * p.nrows + (ok ? rho : 0)) * HD + 8 * eg;
+  float pv[8];
+  if (ok) {
+    float *out = p.drel0 + ((size_t)h * p.nrows + rho) * HD + 8 * eg;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      out[k] = p.scale * (acc[k] + gs * __bfloat162float(vv[k]));
+      pv[k] = gs * __bfloat162float(rr[k]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) pv[k] = 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) pv[k] += __shfl_xor_sync(0xffffffffu, pv[k], sh);
+  }
+  if (lane == 0) {
+    float *dst = A.part_uv + ((size_t)h * ntile + tile) * HD + 8 * eg;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dst[k] = pv[k];
+  }
 }
 
-// dv[h][e] = s sum_rho gtot r; du[h][e] = sum over key tiles of the du partials
-__global__ void reduce_uv_kernel(BwdArgs A) {
+// dv[h][e] = s * sum over the 32-offset tiles of the dv partials; du[h][e] = sum over
+// (batch, key tile) of the du partials.  One CTA per head: 4 strided partial sums per
+// column, combined in a fixed order.
+__global__ void __launch_bounds__(256) reduce_uv_kernel(BwdArgs A) {
   const Prm &p = A.p;
-  __shared__ float red[256];
-  const int h = blockIdx.x / HD, e = blockIdx.x % HD;
-  const __nv_bfloat16 *r = (const __nv_bfloat16 *)p.rel0 + (size_t)h * p.nrows * HD;
-  float acc = 0.f;
-  for (int rho = threadIdx.x; rho < p.nrows; rho += 256)
-    acc = fmaf(p.gtot[(size_t)h * p.nrows + rho], __bfloat162float(r[(size_t)rho * HD + e]), acc);
-  red[threadIdx.x] = acc;
-  __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
-    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
-    __syncthreads();
+  __shared__ float red[2][4][HD];
+  const int h = blockIdx.x, e = threadIdx.x & (HD - 1), part = threadIdx.x >> 6;
+  const int ntile = (p.nrows + 31) / 32, nkv = p.B * p.nT;
+  float dv = 0.f, du = 0.f;
+  for (int t = part; t < ntile; t += 4) dv += A.part_uv[((size_t)h * ntile + t) * HD + e];
+  for (int x = part; x < nkv; x += 4) {
+    const int bb = x / p.nT, n = x % p.nT;
+    du += A.part_kv[(((size_t)bb * p.H + h) * p.nT + n) * HD + e];
   }
-  if (threadIdx.x == 0) {
-    p.drel2[(size_t)h * HD + e] = p.scale * red[0];
-    float du = 0.f;
-    for (int bb = 0; bb < p.B; ++bb)
-      for (int n = 0; n < p.nT; ++n) du += A.part_kv[(((size_t)bb * p.H + h) * p.nT + n) * HD + e];
-    p.drel1[(size_t)h * HD + e] = du;
+  red[0][part][e] = dv;
+  red[1][part][e] = du;
+  __syncthreads();
+  if (part == 0) {
+    p.drel2[(size_t)h * HD + e] = p.scale * (((red[0][0][e] + red[0][1][e]) + red[0][2][e]) + red[0][3][e]);
+    p.drel1[(size_t)h * HD + e] = ((red[1][0][e] + red[1][1][e]) + red[1][2][e]) + red[1][3][e];
   }
 }
 
@@ -1066,6 +1096,7 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   a.vr = w.vr;
   a.part_kv = w.part_kv;
   a.part_dg = w.part_dg;
+  a.part_uv = w.part_uv;
   a.p.part_small = w.part_kv;
   const uint64_t BH = (uint64_t)p0.B * p0.H;
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
@@ -1085,10 +1116,9 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   tc_bwd_diag_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t nr = (size_t)p0.H * p0.nrows * HD;
-  reduce_dr_kernel<<<(unsigned)((nr + 255) / 256), 256, 0, st>>>(a);
+  reduce_dr_kernel<<<(unsigned)(p0.H * ((p0.nrows + 31) / 32)), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reduce_uv_kernel<<<p0.H * HD, 256, 0, st>>>(a);
+  reduce_uv_kernel<<<p0.H, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -565,43 +565,66 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 
 // Per-call products for the tensor-core forward: Transformer-XL u.k_j and v.r_rho,
 // DeBERTa end-row products q_i.Kr[0], q_i.Kr[2k-1], k_j.Qr[0], k_j.Qr[2k-1].
-__global__ void tc_prep_kernel(Prm p, float *uk, float *vr, float *c2pE, float *p2cE) {
-  const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const size_t rows = (size_t)p.B * p.H * p.L;
+// Per-row / per-offset products of the relation stage.  Eight threads share one
+// 64-element row (eight consecutive elements each, so a warp reads four whole rows),
+// and the partial dot products are combined by a fixed shuffle tree.
+//   TXL      uk[b,h,j] = u_h . k_j  and  vr[h,rho] = v_h . r_rho
+//   DeBERTa  c2pE[b,h,i] = (q_i . Kr_0, q_i . Kr_last), p2cE[b,h,j] = (k_j . Qr_0, k_j . Qr_last)
+__device__ __forceinline__ float dot8(const __nv_bfloat16 *a, const __nv_bfloat16 *b) {
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) s = fmaf(__bfloat162float(a[c]), __bfloat162float(b[c]), s);
+  return s;
+}
+__device__ __forceinline__ float sum8(float x) {  // over the eight threads of a row
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  return x;
+}
+__global__ void __launch_bounds__(256) tc_prep_kernel(Prm p, float *uk, float *vr, float *c2pE, float *p2cE) {
   typedef __nv_bfloat16 bf;
+  const size_t row = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int sub = threadIdx.x & 7;
+  const size_t rows = (size_t)p.B * p.H * p.L;
   if (p.mech == M_TXL) {
-    if (x < rows) {
-      const int h = (int)((x / p.L) % p.H);
-      const bf *k = (const bf *)p.k + x * HD, *u = (const bf *)p.rel1 + (size_t)h * HD;
-      float a = 0.f;
-      for (int c = 0; c < HD; ++c) a = fmaf(ldf(u, c), ldf(k, c), a);
-      uk[x] = a;
+    const size_t nr = rows + (size_t)p.H * p.nrows;  // key rows, then table rows
+    float a = 0.f;
+    if (row < rows) {
+      const int h = (int)((row / p.L) % p.H);
+      a = dot8((const bf *)p.k + row * HD + 8 * sub, (const bf *)p.rel1 + (size_t)h * HD + 8 * sub);
+    } else if (row < nr) {
+      const size_t rr = row - rows;
+      const int h = (int)(rr / p.nrows);
+      a = dot8((const bf *)p.rel0 + rr * HD + 8 * sub, (const bf *)p.rel2 + (size_t)h * HD + 8 * sub);
     }
-    if (x < (size_t)p.H * p.nrows) {
-      const int h = (int)(x / p.nrows);
-      const bf *r = (const bf *)p.rel0 + x * HD, *v = (const bf *)p.rel2 + (size_t)h * HD;
-      float a = 0.f;
-      for (int c = 0; c < HD; ++c) a = fmaf(ldf(v, c), ldf(r, c), a);
-      vr[x] = a;
+    a = sum8(a);
+    if (sub == 0) {
+      if (row < rows) uk[row] = a;
+      else if (row < nr) vr[row - rows] = a;
     }
   } else if (p.mech == M_DEB) {
-    if (x < rows) {
-      const int h = (int)((x / p.L) % p.H);
-      const bf *q = (const bf *)p.q + x * HD, *k = (const bf *)p.k + x * HD;
-      const bf *Kr = (const bf *)p.rel0 + (size_t)h * p.nrows * HD, *Qr = (const bf *)p.rel1 + (size_t)h * p.nrows * HD;
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+    if (row < rows) {
+      const int h = (int)((row / p.L) % p.H);
+      const bf *q = (const bf *)p.q + row * HD + 8 * sub, *k = (const bf *)p.k + row * HD + 8 * sub;
+      const bf *Kr = (const bf *)p.rel0 + (size_t)h * p.nrows * HD + 8 * sub;
+      const bf *Qr = (const bf *)p.rel1 + (size_t)h * p.nrows * HD + 8 * sub;
       const size_t last = (size_t)(p.nrows - 1) * HD;
-      float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-      for (int c = 0; c < HD; ++c) {
-        const float qc = ldf(q, c), kc = ldf(k, c);
-        a0 = fmaf(qc, ldf(Kr, c), a0);
-        a1 = fmaf(qc, ldf(Kr, last + c), a1);
-        b0 = fmaf(kc, ldf(Qr, c), b0);
-        b1 = fmaf(kc, ldf(Qr, last + c), b1);
-      }
-      c2pE[2 * x] = a0;
-      c2pE[2 * x + 1] = a1;
-      p2cE[2 * x] = b0;
-      p2cE[2 * x + 1] = b1;
+      a0 = dot8(q, Kr);
+      a1 = dot8(q, Kr + last);
+      b0 = dot8(k, Qr);
+      b1 = dot8(k, Qr + last);
+    }
+    a0 = sum8(a0);
+    a1 = sum8(a1);
+    b0 = sum8(b0);
+    b1 = sum8(b1);
+    if (row < rows && sub == 0) {
+      c2pE[2 * row] = a0;
+      c2pE[2 * row + 1] = a1;
+      p2cE[2 * row] = b0;
+      p2cE[2 * row + 1] = b1;
     }
   }
 }
@@ -656,8 +679,8 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t plane
 
 cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st) {
   if (p.mech != M_TXL && p.mech != M_DEB) return cudaSuccess;
-  const size_t n = std::max((size_t)p.B * p.H * p.L, (size_t)p.H * p.nrows);
-  tc::tc_prep_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE);
+  const size_t rows = (size_t)p.B * p.H * p.L + (p.mech == M_TXL ? (size_t)p.H * p.nrows : 0);
+  tc::tc_prep_kernel<<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE);
   return cudaGetLastError();
 }
 
