@@ -718,12 +718,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
 namespace dg {
 constexpr int OFF_Q = 0, OFF_DO = 32768, OFF_K = 65536, OFF_V = OFF_K + 16384, OFF_R = OFF_V + 16384;
 constexpr int OFF_ROT = OFF_R + 32768;  // rot rows; E_lo at +0, E_hi at +32768
+// 128 x 64 bf16 ones in the MN-major 128-byte-swizzled layout: the second N atom
+// of the G MMAs' B operand [Q_m | 1], so that columns 64..79 of G give g = E^T 1
 constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;
-constexpr int OFF_VEC = OFF_ONES + 4096;
+constexpr int OFF_VEC = OFF_ONES + 16384;
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
+static_assert(OFF_ONES % 1024 == 0, "swizzled operand tiles are 1024-byte aligned");
 enum { B_R = 0, B_ST0, B_ST1, B_KV, B_KVFREE, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
-constexpr uint32_t T_S = 0, T_DP = 128, T_GLO = 256, T_GHI = 320, T_GL = 384, T_GH = 416;
+constexpr uint32_t T_S = 0, T_DP = 128, T_GLO = 256, T_GHI = 336;  // G | g: 80 columns each
 }  // namespace dg
 
 __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_constant__ BwdArgs A) {
@@ -760,7 +763,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int x = tid; x < 4096 / 16; x += NTHREADS) {
+  for (int x = tid; x < 16384 / 16; x += NTHREADS) {
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
@@ -783,8 +786,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       prefetch_tmap(&A.mdo);
       prefetch_tmap(&A.mr);
       const uint32_t idS = idesc_bf16(128, 128, false);
-      const uint32_t idG = idesc_bf16(128, 64, true, true);
-      const uint32_t idg = idesc_bf16(128, 16, false, true);
+      const uint32_t idG = idesc_bf16(128, 80, true, true);
       ctl.expect(BAR(B_R), 0, (hasA ? 16384u : 0u) + (hasB ? 16384u : 0u));
       if (hasA) tma_load_3d(sbase + OFF_R, &A.mr, BAR(B_R), 0, 128 * D + p.off, h);
       if (hasB) tma_load_3d(sbase + OFF_R + 16384, &A.mr, BAR(B_R), 0, 128 * (D - 1) + p.off, h);
@@ -800,19 +802,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         tma_load_3d(sbase + OFF_K, &A.mk, BAR(B_KV), 0, nn * 128, bh);
         tma_load_3d(sbase + OFF_V, &A.mv, BAR(B_KV), 0, nn * 128, bh);
       };
-      auto accumulate = [&](int t) {  // G_lo, G_hi += E^T Q_t ; g_lo, g_hi += E^T 1
+      auto accumulate = [&](int t) {  // [G | g]_lo, [G | g]_hi += E^T [Q_t | 1]
         const int st = t & 1;
+        const uint32_t lbo = (uint32_t)(OFF_ONES - OFF_Q - 16384 * st);  // Q atom -> ones atom
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
-          const uint64_t bq = sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, 16, 1024);
-          const uint64_t b1 = sdesc_sw128(sbase + OFF_ONES + 2048 * (k >> 2) + 32 * (k & 3), 16, 1024);
+          const uint64_t bq = sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, lbo, 1024);
           const uint64_t elo = sdesc_sw128(sbase + OFF_ROT + 2048 * k, 16384, 1024);
           const uint64_t ehi = sdesc_sw128(sbase + OFF_ROT + 32768 + 2048 * k, 16384, 1024);
           umma_bf16(tbase + T_GLO, elo, bq, idG, acc);
           umma_bf16(tbase + T_GHI, ehi, bq, idG, acc);
-          umma_bf16(tbase + T_GL, elo, b1, idg, acc);
-          umma_bf16(tbase + T_GH, ehi, b1, idg, acc);
         }
         umma_commit(BAR(B_PDSFREE));
       };
@@ -947,8 +947,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       uint32_t rlo[16], rhi[16], glo[16], ghi[16];
       tmem_ld16(tl + T_GLO + 16 * qt, rlo);
       tmem_ld16(tl + T_GHI + 16 * qt, rhi);
-      tmem_ld16(tl + T_GL, glo);
-      tmem_ld16(tl + T_GH, ghi);
+      tmem_ld16(tl + T_GLO + 64, glo);
+      tmem_ld16(tl + T_GHI + 64, ghi);
       tmem_wait_ld();
       // partial layout [block lo / hi][65][128 offsets]: G columns 0..63, then g
       float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
@@ -999,11 +999,28 @@ __global__ void __launch_bounds__(256) reduce_dr_kernel(BwdArgs A) {
         if (band < 0 || band >= A.nbands) continue;
         const int len = p.nT - (D < 0 ? -D : D);
         const int nch = (len + A.dg_ch - 1) / A.dg_ch;
-        for (int ch = 0; ch < nch; ++ch) {
-          const float *part = A.part_dg + ((bh * A.nbands + band) * A.dg_nchunk + ch) * DG_STRIDE + (size_t)(65 * w) * 128 + c;
+        const float *part = A.part_dg + (bh * A.nbands + band) * A.dg_nchunk * DG_STRIDE + (size_t)(65 * w) * 128 + c;
+        // two chunks' loads in flight before their (in-order) accumulation
+        int ch = 0;
+        for (; ch + 1 < nch; ch += 2) {
+          const float *p0 = part + (size_t)ch * DG_STRIDE, *p1 = p0 + DG_STRIDE;
+          float v0[9], v1[9];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] += part[(size_t)(8 * eg + k) * 128];
-          gs += part[(size_t)64 * 128];
+          for (int k = 0; k < 8; ++k) {
+            v0[k] = __ldg(p0 + (size_t)(8 * eg + k) * 128);
+            v1[k] = __ldg(p1 + (size_t)(8 * eg + k) * 128);
+          }
+          v0[8] = __ldg(p0 + (size_t)64 * 128);
+          v1[8] = __ldg(p1 + (size_t)64 * 128);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = (acc[k] + v0[k]) + v1[k];
+          gs = (gs + v0[8]) + v1[8];
+        }
+        if (ch < nch) {
+          const float *p0 = part + (size_t)ch * DG_STRIDE;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] += __ldg(p0 + (size_t)(8 * eg + k) * 128);
+          gs += __ldg(p0 + (size_t)64 * 128);
         }
       }
     }
