@@ -173,14 +173,19 @@ __device__ __forceinline__ int slot3(int b) { return ((b % 3) + 3) % 3; }
 // key-tile kernel: dK, dV, column sums of dS
 // ============================================================================
 namespace kv {
+// relation blocks in a 2-slot ring (block b in slot b & 1): the load of block D + 1
+// replaces block D - 1 only after T(t), its last reader, has been consumed
 constexpr int OFF_K = 0, OFF_V = 16384, OFF_Q = 32768, OFF_DO = OFF_Q + 32768, OFF_R = OFF_DO + 32768;
-constexpr int OFF_ROT = OFF_R + 3 * 16384;            // rot rows; P tile at +0, dS tile at +32768
-constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;  // [16][128] bf16 ones, K-major (2 x 2 KB)
-constexpr int OFF_VEC = OFF_ONES + 4096;              // uk[128], then the du column sums
+constexpr int OFF_ROT = OFF_R + 2 * 16384;            // rot rows; P tile at +0, dS tile at +32768
+// 128 x 64 bf16 ones in the MN-major 128-byte-swizzled layout: the second N atom of
+// the dK MMA's B operand [Q_m | 1], so that columns 64..79 of dK give c = dS^T 1
+constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;
+constexpr int OFF_VEC = OFF_ONES + 16384;             // uk[128], then the du column sums
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
+static_assert(OFF_ONES % 1024 == 0, "swizzled operand tiles are 1024-byte aligned");
 enum { B_KV = 0, B_ST0, B_ST1, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
-constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320, T_CS = 384;
+constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320;  // dK | c: 80 columns
 }  // namespace kv
 
 __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_constant__ BwdArgs A) {
@@ -217,7 +222,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     mbar_fence_init();
   }
   // all-ones B operand for the column sums (any swizzle of all-ones is all-ones)
-  for (int x = tid; x < 4096 / 16; x += NTHREADS) {
+  for (int x = tid; x < 16384 / 16; x += NTHREADS) {
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
@@ -242,7 +247,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       prefetch_tmap(&A.mr);
       const uint32_t idS = idesc_bf16(128, 128, false);
       const uint32_t idAcc = idesc_bf16(128, 64, true, true);
-      const uint32_t idCs = idesc_bf16(128, 16, false, true);
+      const uint32_t idK = idesc_bf16(128, 80, true, true);
       ctl.expect(BAR(B_KV), 0, 32768);
       tma_load_3d(sbase + OFF_K, &A.mk, BAR(B_KV), 0, j0, bh);
       tma_load_3d(sbase + OFF_V, &A.mv, BAR(B_KV), 0, j0, bh);
@@ -252,25 +257,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         ctl.expect(BAR(B_ST0 + st), (uint32_t)((t >> 1) & 1), 32768u + (bA ? 16384u : 0u) + (bB ? 16384u : 0u));
         tma_load_3d(sbase + OFF_Q + 16384 * st, &A.mq, BAR(B_ST0 + st), 0, m * 128, bh);
         tma_load_3d(sbase + OFF_DO + 16384 * st, &A.mdo, BAR(B_ST0 + st), 0, m * 128, bh);
-        if (bA) tma_load_3d(sbase + OFF_R + 16384 * slot3(D), &A.mr, BAR(B_ST0 + st), 0, 128 * D + p.off, h);
-        if (bB) tma_load_3d(sbase + OFF_R + 16384 * slot3(D - 1), &A.mr, BAR(B_ST0 + st), 0, 128 * (D - 1) + p.off, h);
+        if (bA) tma_load_3d(sbase + OFF_R + 16384 * (D & 1), &A.mr, BAR(B_ST0 + st), 0, 128 * D + p.off, h);
+        if (bB) tma_load_3d(sbase + OFF_R + 16384 * ((D - 1) & 1), &A.mr, BAR(B_ST0 + st), 0, 128 * (D - 1) + p.off, h);
       };
-      auto accumulate = [&](int t) {  // dV, dK, column sums of tile t (P, dS in smem)
+      auto accumulate = [&](int t) {  // dV += P^T dO, [dK | c] += dS^T [Q | 1] of tile t (P, dS in smem)
         const int st = t & 1;
+        const uint32_t lbo = (uint32_t)(OFF_ONES - OFF_Q - 16384 * st);  // Q atom -> ones atom
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
           umma_bf16(tbase + T_DV, sdesc_sw128(sbase + OFF_ROT + 2048 * k, 16384, 1024),
                     sdesc_sw128(sbase + OFF_DO + 16384 * st + 2048 * k, 16, 1024), idAcc, acc);
           umma_bf16(tbase + T_DK, sdesc_sw128(sbase + OFF_ROT + 32768 + 2048 * k, 16384, 1024),
-                    sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, 16, 1024), idAcc, acc);
-          umma_bf16(tbase + T_CS, sdesc_sw128(sbase + OFF_ROT + 32768 + 2048 * k, 16384, 1024),
-                    sdesc_sw128(sbase + OFF_ONES + 2048 * (k >> 2) + 32 * (k & 3), 16, 1024), idCs, acc);
+                    sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, lbo, 1024), idK, acc);
         }
         umma_commit(BAR(B_PDSFREE));
       };
       issue_stage(0);
-      if (iters > 1) issue_stage(1);
       bool ok = true;
       for (int t = 0; ok && t < iters; ++t) {
         const int m = mStart + t, D = m - n, st = t & 1;
@@ -279,9 +282,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
         tc_fence_after();
         // relation products transposed (lane = offset, column = query row)
-        if (block_valid(p, D)) umma_k64(tbase + 0, sbase + OFF_R + 16384 * slot3(D), sbase + OFF_Q + 16384 * st, idS, false);
+        if (block_valid(p, D)) umma_k64(tbase + 0, sbase + OFF_R + 16384 * (D & 1), sbase + OFF_Q + 16384 * st, idS, false);
         if (block_valid(p, D - 1))
-          umma_k64(tbase + 128, sbase + OFF_R + 16384 * slot3(D - 1), sbase + OFF_Q + 16384 * st, idS, false);
+          umma_k64(tbase + 128, sbase + OFF_R + 16384 * ((D - 1) & 1), sbase + OFF_Q + 16384 * st, idS, false);
         umma_commit(BAR(B_TFULL));
         if (t >= 1) accumulate(t - 1);
         if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
@@ -289,8 +292,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         umma_k64(tbase + T_S, sbase + OFF_Q + 16384 * st, sbase + OFF_K, idS, false);
         umma_k64(tbase + T_DP, sbase + OFF_DO + 16384 * st, sbase + OFF_V, idS, false);
         umma_commit(BAR(B_SDP));
-        if (t >= 1 && t + 1 < iters) {
-          if (!ctl.wait(BAR(B_PDSFREE), (t - 1) & 1)) break;
+        if (t + 1 < iters) {  // T(t) consumed: its block D - 1 slot takes block D + 1
+          if (t >= 1 && !ctl.wait(BAR(B_PDSFREE), (t - 1) & 1)) break;
           issue_stage(t + 1);
         }
       }
@@ -403,7 +406,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       uint32_t rv[16], rk[16], rc[16];
       tmem_ld16(tl + T_DV + 16 * qt, rv);
       tmem_ld16(tl + T_DK + 16 * qt, rk);
-      tmem_ld16(tl + T_CS, rc);
+      tmem_ld16(tl + T_DK + 64, rc);
       tmem_wait_ld();
       csum = u2f(rc[0]);
       if (j < L) {
