@@ -462,7 +462,7 @@ constexpr int OFF_ROT = OFF_R + 3 * 16384;  // rot rows; E_lo at +0, E_hi at +32
 constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
-enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_PDS, B_PDSFREE, B_DRAIN, NB };
+enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_PDS, B_PDSFREE, B_DSFREE, B_DRAIN, NB };
 constexpr uint32_t T_S = 0, T_REL = 128, T_DQ = 384, T_DS = 448;
 }  // namespace qk
 
@@ -494,6 +494,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     mbar_init(BAR(B_DPF), 1);
     mbar_init(BAR(B_PDS), NSOFT);
     mbar_init(BAR(B_PDSFREE), 1);
+    mbar_init(BAR(B_DSFREE), 1);
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -554,22 +555,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         }
         if (!ctl.wait(BAR(B_PDS), n & 1)) break;
         tc_fence_after();
-        // dQ += dS K_n (dS from TMEM) + E_lo r_D + E_hi r_{D-1}
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_bf16_ts(tbase + T_DQ, tbase + T_DS + 8 * k, sdesc_sw128(sbase + OFF_K + 16384 * st + 2048 * k, 16, 1024), idDQ,
-                       (n > 0 || k > 0) ? 1u : 0u);
+        // dQ += E_lo r_D + E_hi r_{D-1} (E in smem, freed first so the rows can skew the
+        // next tile), then the next tile's relation block, then dQ += dS K_n (dS in TMEM)
+        uint32_t acc = n > 0 ? 1u : 0u;
         if (block_valid(p, D)) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             umma_bf16(tbase + T_DQ, sdesc_sw128(sbase + OFF_ROT + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
-                      sdesc_sw128(sbase + OFF_R + 16384 * slot3(D) + 2048 * k, 16, 1024), idDQ, 1u);
+                      sdesc_sw128(sbase + OFF_R + 16384 * slot3(D) + 2048 * k, 16, 1024), idDQ, (acc || k > 0) ? 1u : 0u);
+          acc = 1u;
         }
         if (block_valid(p, D - 1)) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             umma_bf16(tbase + T_DQ, sdesc_sw128(sbase + OFF_ROT + 32768 + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
-                      sdesc_sw128(sbase + OFF_R + 16384 * slot3(D - 1) + 2048 * k, 16, 1024), idDQ, 1u);
+                      sdesc_sw128(sbase + OFF_R + 16384 * slot3(D - 1) + 2048 * k, 16, 1024), idDQ, (acc || k > 0) ? 1u : 0u);
+          acc = 1u;
         }
         umma_commit(BAR(B_PDSFREE));
         if (n + 1 < nTiles) {  // relation block D - 2 for tile n + 1, into the slot dP(n) used
@@ -577,8 +578,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
             umma_k64(tbase + slotA, sbase + OFF_R + 16384 * slot3(D - 2), sbase + OFF_Q, idS, false);
           umma_commit(BAR(B_SFULL));
         }
-        if (n + 2 < nTiles) {
-          if (!ctl.wait(BAR(B_PDSFREE), n & 1)) break;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_bf16_ts(tbase + T_DQ, tbase + T_DS + 8 * k, sdesc_sw128(sbase + OFF_K + 16384 * st + 2048 * k, 16, 1024), idDQ,
+                       (acc || k > 0) ? 1u : 0u);
+        umma_commit(BAR(B_DSFREE));
+        if (n + 2 < nTiles) {  // K_n, V_n and the tile's relation block slot are free once dS K_n is done
+          if (!ctl.wait(BAR(B_DSFREE), n & 1)) break;
           issue_stage(n + 2);
         }
       }
@@ -679,7 +685,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-        tmem_st16(tl + T_DS + 16 * qt, pk);
+        // the previous tile's dS K MMAs read T_DS: wait for them (long done in practice)
+        if (n >= 1 && !warp_wait(BAR(B_DSFREE), (n - 1) & 1, abort_flag, status)) good = false;
+        if (good) tmem_st16(tl + T_DS + 16 * qt, pk);
         store_E(smem + OFF_ROT, il, cb, x);
         tmem_wait_st();
         fence_async_smem();
@@ -687,7 +695,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         mbar_arrive(BAR(B_PDS));
       }
     }
-    good = good && warp_wait(BAR(B_PDSFREE), (nTiles - 1) & 1, abort_flag, status);
+    good = good && warp_wait(BAR(B_DSFREE), (nTiles - 1) & 1, abort_flag, status);  // last dQ MMAs done
     if (good) {
       tc_fence_after();
       uint32_t r[16];
