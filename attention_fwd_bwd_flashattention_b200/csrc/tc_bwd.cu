@@ -184,7 +184,7 @@ constexpr int OFF_VEC = OFF_ONES + 16384;             // uk[128], then the du co
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 static_assert(OFF_ONES % 1024 == 0, "swizzled operand tiles are 1024-byte aligned");
-enum { B_KV = 0, B_ST0, B_ST1, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
+enum { B_KV = 0, B_ST0, B_ST1, B_TFULL, B_TCONS, B_SDP, B_SDPCONS, B_PDS, B_PDSFREE, B_DRAIN, NB };
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320;  // dK | c: 80 columns
 }  // namespace kv
 
@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     mbar_init(BAR(B_TFULL), 1);
     mbar_init(BAR(B_TCONS), NSOFT);
     mbar_init(BAR(B_SDP), 1);
+    mbar_init(BAR(B_SDPCONS), NSOFT);
     mbar_init(BAR(B_PDS), NSOFT);
     mbar_init(BAR(B_PDSFREE), 1);
     mbar_init(BAR(B_DRAIN), 1);
@@ -273,33 +274,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         }
         umma_commit(BAR(B_PDSFREE));
       };
-      issue_stage(0);
-      bool ok = true;
-      for (int t = 0; ok && t < iters; ++t) {
-        const int m = mStart + t, D = m - n, st = t & 1;
-        if (!ctl.wait_load(BAR(B_ST0 + st), (t >> 1) & 1)) break;
-        if (t == 0 && !ctl.wait_load(BAR(B_KV), 0)) break;
-        if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
-        tc_fence_after();
-        // relation products transposed (lane = offset, column = query row)
+      // relation products of tile t, transposed (lane = offset, column = query row);
+      // they overwrite S / dP of tile t - 1, which the rows have read by then
+      auto issue_T = [&](int t) {
+        const int D = mStart + t - n, st = t & 1;
         if (block_valid(p, D)) umma_k64(tbase + 0, sbase + OFF_R + 16384 * (D & 1), sbase + OFF_Q + 16384 * st, idS, false);
         if (block_valid(p, D - 1))
           umma_k64(tbase + 128, sbase + OFF_R + 16384 * ((D - 1) & 1), sbase + OFF_Q + 16384 * st, idS, false);
         umma_commit(BAR(B_TFULL));
-        if (t >= 1) accumulate(t - 1);
+      };
+      issue_stage(0);
+      bool ok = ctl.wait_load(BAR(B_ST0), 0) && ctl.wait_load(BAR(B_KV), 0);
+      if (ok) {
+        tc_fence_after();
+        issue_T(0);
+      }
+      for (int t = 0; ok && t < iters; ++t) {
+        const int st = t & 1;
         if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
         tc_fence_after();
         umma_k64(tbase + T_S, sbase + OFF_Q + 16384 * st, sbase + OFF_K, idS, false);
         umma_k64(tbase + T_DP, sbase + OFF_DO + 16384 * st, sbase + OFF_V, idS, false);
         umma_commit(BAR(B_SDP));
-        if (t + 1 < iters) {  // T(t) consumed: its block D - 1 slot takes block D + 1
-          if (t >= 1 && !ctl.wait(BAR(B_PDSFREE), (t - 1) & 1)) break;
-          issue_stage(t + 1);
+        if (t == 0 && iters > 1) issue_stage(1);  // T(0) consumed: block D0 - 1's slot is free
+        if (t + 1 < iters) {  // S / dP(t) read by the rows: T(t + 1) overlaps their P / dS stores
+          if (!ctl.wait(BAR(B_SDPCONS), t & 1)) break;
+          if (!ctl.wait_load(BAR(B_ST0 + (st ^ 1)), ((t + 1) >> 1) & 1)) break;
+          tc_fence_after();
+          issue_T(t + 1);
         }
-      }
-      if (!*abort_flag && ctl.wait(BAR(B_PDS), (iters - 1) & 1)) {
+        if (!ctl.wait(BAR(B_PDS), t & 1)) break;
         tc_fence_after();
-        accumulate(iters - 1);
+        accumulate(t);
+        if (t + 2 < iters) {  // Q / dO of tile t and relation block D (last read by T(t + 1)) are free
+          if (!ctl.wait(BAR(B_PDSFREE), t & 1)) break;
+          issue_stage(t + 2);
+        }
       }
       ctl.drain(BAR(B_DRAIN));
     }
@@ -381,6 +391,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         };
         if (need_mask) pds(std::true_type{}); else pds(std::false_type{});
         tc_fence_before();
+        mbar_arrive(BAR(B_SDPCONS));  // S / dP read: T(t + 1) may overwrite them
       }
       named_bar_sync(1, NSOFT);  // every rot row read; the P / dS tiles overwrite them
       if (good) {
@@ -736,7 +747,7 @@ constexpr int OFF_VEC = OFF_ONES + 16384;
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 static_assert(OFF_ONES % 1024 == 0, "swizzled operand tiles are 1024-byte aligned");
-enum { B_R = 0, B_ST0, B_ST1, B_KV, B_KVFREE, B_TFULL, B_TCONS, B_SDP, B_PDS, B_PDSFREE, B_DRAIN, NB };
+enum { B_R = 0, B_ST0, B_ST1, B_KV, B_KVFREE, B_TFULL, B_TCONS, B_SDP, B_SDPCONS, B_PDS, B_PDSFREE, B_DRAIN, NB };
 constexpr uint32_t T_S = 0, T_DP = 128, T_GLO = 256, T_GHI = 336;  // G | g: 80 columns each
 }  // namespace dg
 
@@ -770,7 +781,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
   (void)b;
 
   if (tid == 0) {
-    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), (k == B_TCONS || k == B_PDS) ? NSOFT : 1);
+    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), (k == B_TCONS || k == B_SDPCONS || k == B_PDS) ? NSOFT : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -830,17 +841,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       issue_qd(0);
       issue_kv(0);
       if (iters > 1) issue_qd(1);
-      bool ok = ctl.wait_load(BAR(B_R), 0);
-      for (int t = 0; ok && t < iters; ++t) {
+      // relation products of tile t, transposed (lane = offset, column = query row);
+      // they overwrite S / dP of tile t - 1, which the rows have read by then
+      auto issue_T = [&](int t) {
         const int st = t & 1;
-        if (!ctl.wait_load(BAR(B_ST0 + st), (t >> 1) & 1)) break;
-        if (t >= 1 && !ctl.wait(BAR(B_PDS), (t - 1) & 1)) break;
-        tc_fence_after();
-        // relation products transposed (lane = offset, column = query row)
         if (hasA) umma_k64(tbase + 0, sbase + OFF_R, sbase + OFF_Q + 16384 * st, idS, false);
         if (hasB) umma_k64(tbase + 128, sbase + OFF_R + 16384, sbase + OFF_Q + 16384 * st, idS, false);
         umma_commit(BAR(B_TFULL));
-        if (t >= 1) accumulate(t - 1);
+      };
+      bool ok = ctl.wait_load(BAR(B_R), 0) && ctl.wait_load(BAR(B_ST0), 0);
+      if (ok) {
+        tc_fence_after();
+        issue_T(0);
+      }
+      for (int t = 0; ok && t < iters; ++t) {
+        const int st = t & 1;
         if (!ctl.wait(BAR(B_TCONS), t & 1)) break;
         if (!ctl.wait_load(BAR(B_KV), t & 1)) break;
         tc_fence_after();
@@ -851,15 +866,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         if (t + 1 < iters) {
           if (!ctl.wait(BAR(B_KVFREE), t & 1)) break;
           issue_kv(t + 1);
-          if (t >= 1) {
-            if (!ctl.wait(BAR(B_PDSFREE), (t - 1) & 1)) break;
-            issue_qd(t + 1);
-          }
+          // S / dP(t) read by the rows: T(t + 1) overlaps their dS / E stores
+          if (!ctl.wait(BAR(B_SDPCONS), t & 1)) break;
+          if (!ctl.wait_load(BAR(B_ST0 + (st ^ 1)), ((t + 1) >> 1) & 1)) break;
+          tc_fence_after();
+          issue_T(t + 1);
         }
-      }
-      if (!*abort_flag && ctl.wait(BAR(B_PDS), (iters - 1) & 1)) {
+        if (!ctl.wait(BAR(B_PDS), t & 1)) break;
         tc_fence_after();
-        accumulate(iters - 1);
+        accumulate(t);
+        if (t + 2 < iters) {  // Q / dO of tile t are free once G(t) is done
+          if (!ctl.wait(BAR(B_PDSFREE), t & 1)) break;
+          issue_qd(t + 2);
+        }
       }
       ctl.drain(BAR(B_DRAIN));
     }
@@ -939,6 +958,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         };
         if (need_mask) pds(std::true_type{}); else pds(std::false_type{});
         tc_fence_before();
+        mbar_arrive(BAR(B_SDPCONS));  // S / dP read: T(t + 1) may overwrite them
       } else {
 #pragma unroll
         for (int x = 0; x < NC; ++x) ds[x] = 0.f;

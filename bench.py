@@ -71,13 +71,18 @@ def fa_flops(wl):
 
 
 def kernel_launches(wl, path):
-    """Kernels this library launches per forward and per backward call."""
-    t5 = 1 if wl.mech == T5 else 0
-    if path == "simt":
+    """Kernels this library launches per forward and per backward call (the dispatch of csrc/api.cu)."""
+    t5 = 1 if wl.mech == T5 else 0  # per-call bucket/bias preparation
+    tc = path != "simt" and wl.dtype == torch.bfloat16
+    if tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
+        fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
+    else:
         fwd = 1 + t5
-        bwd = {T5: 5, SHAW: 4, TXL: 6, DEBERTA: 5}[wl.mech] + t5
-        return fwd, bwd
-    return 1 + t5, {T5: 5, SHAW: 4, TXL: 6, DEBERTA: 5}[wl.mech] + t5
+    if tc and wl.mech == TXL:  # D, relation prep, key-tile, query-tile, diagonal, dr and u/v reductions
+        bwd = 7
+    else:  # D, key-tile, query-tile, then the table-gradient reductions
+        bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2}[wl.mech]
+    return fwd, bwd
 
 
 def load_peaks():
