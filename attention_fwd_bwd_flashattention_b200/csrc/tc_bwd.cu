@@ -134,7 +134,8 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
   return d;
 }
-__device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const float (&x)[NC]) {
+// pk[k] = bf16 pair (x[2k+1] low, x[2k] high) of the thread's values
+__device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const uint32_t (&pk)[NC / 2]) {
   const uint32_t C0 = (uint32_t)(il - cb + 128);
   const bool ev = (C0 & 1u) == 0;
   const uint32_t rowb = 128u * (uint32_t)il, r7 = (uint32_t)(il & 7) << 4;
@@ -142,9 +143,6 @@ __device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const float 
   // pk[k] = (x[2k+1], x[2k]) is the pair at c' = C0 - 2k - 1 when C0 is odd; when it
   // is even the pair at c' = C0 - 2k - 2 is (x[2k+2], x[2k+1]): high half of pk[k+1],
   // low half of pk[k], picked by one byte permute
-  uint32_t pk[NC / 2];
-#pragma unroll
-  for (int k = 0; k < NC / 2; ++k) pk[k] = pack_bf16x2(x[2 * k + 1], x[2 * k]);
   const uint32_t sel = ev ? 0x1076u : 0x3210u;
 #pragma unroll
   for (int k = 0; k < NC / 2 - 1; ++k) {
@@ -180,8 +178,10 @@ constexpr int OFF_ROT = OFF_R + 2 * 16384;            // rot rows; P tile at +0,
 // 128 x 64 bf16 ones in the MN-major 128-byte-swizzled layout: the second N atom of
 // the dK MMA's B operand [Q_m | 1], so that columns 64..79 of dK give c = dS^T 1
 constexpr int OFF_ONES = OFF_ROT + 128 * ROT_LD * 4;
-constexpr int OFF_VEC = OFF_ONES + 16384;             // uk[128], then the du column sums
-constexpr int OFF_BAR = OFF_VEC + 4096;
+// uk[128] (then the du column sums), then per-tile row / offset terms, double-buffered:
+// [lse2 | D | v.r block D | v.r block D - 1] x 128
+constexpr int OFF_VEC = OFF_ONES + 16384;
+constexpr int OFF_BAR = OFF_VEC + 8192;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 static_assert(OFF_ONES % 1024 == 0, "swizzled operand tiles are 1024-byte aligned");
 enum { B_KV = 0, B_ST0, B_ST1, B_TFULL, B_TCONS, B_SDP, B_SDPCONS, B_PDS, B_PDSFREE, B_DRAIN, NB };
@@ -319,22 +319,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
-    // row statistics and this thread's v.r (offset 32 g + lane of blocks D, D - 1) of
-    // the next query tile, fetched one iteration ahead
-    auto fetch = [&](int t, float &l2, float &dv, float &va, float &vb) {
-      const int m = mStart + t, D = m - n, i = m * 128 + il;
-      l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
-      dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
-      const int ra = 128 * D + il + p.off, rb = ra - 128;
-      va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
-      vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
+    // per-tile terms staged through smem one tile ahead, one element per thread:
+    // [lse2 of the 128 rows | D of the rows | c1 v.r of block D's 128 offsets | same, block D - 1]
+    auto fetch1 = [&](int t) {
+      const int m = mStart + t, D = m - n, r = tid & 127, w = tid >> 7;
+      const int i = m * 128 + r, ro = 128 * (w == 2 ? D : D - 1) + r + p.off;
+      if (w == 0) return (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      if (w == 1) return (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      return (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
     };
-    float nl2, ndv, nva, nvb;
-    fetch(0, nl2, ndv, nva, nvb);
+    vec[128 + tid] = fetch1(0);
     for (int t = 0; t < iters; ++t) {
       const int m = mStart + t, D = m - n, i = m * 128 + il;
-      const float lse2 = nl2, Dv = ndv, vrA = nva, vrB = nvb;
-      if (t + 1 < iters) fetch(t + 1, nl2, ndv, nva, nvb);
+      const float *tv = vec + 128 + 512 * (t & 1);
+      const float nv = (t + 1 < iters) ? fetch1(t + 1) : 0.f;
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
@@ -342,7 +340,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, c1, vrA * c1, vrB * c1, rot);
+          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, c1, tv[256 + il], tv[384 + il], rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -357,6 +355,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
+        const float lse2 = tv[il], Dv = tv[128 + il];
         const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
         auto pds = [&](auto masked) {
 #pragma unroll
@@ -407,6 +406,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
+      vec[128 + 512 * ((t + 1) & 1) + tid] = nv;  // tile t - 1's terms were last read before this tile's first barrier
     }
     // ---- epilogue: lanes are keys now; this thread takes 16 of the 64 columns ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
@@ -611,22 +611,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
     const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
     bool good = true;
-    // one key tile ahead: uk (tid < 128) and this thread's v.r (offset il of blocks D, D - 1)
-    auto fetch = [&](int n, float &ukv, float &va, float &vb) {
-      const int j0 = n * 128, D = m - n;
-      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] * c1 : 0.f;  // pre-scaled
-      const int ra = 128 * D + il + p.off, rb = ra - 128;
-      va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
-      vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
+    // per key tile, staged through smem one tile ahead (one element per thread, double-
+    // buffered): [c1 u.k of the keys | c1 v.r of block D's offsets | same, block D - 1]
+    auto fetch1 = [&](int n) {
+      const int j0 = n * 128, D = m - n, r = tid & 127, w = tid >> 7;
+      if (w == 0) return (j0 + r < L) ? A.uk[(size_t)bh * L + j0 + r] * c1 : 0.f;
+      const int ro = 128 * (w == 1 ? D : D - 1) + r + p.off;
+      return (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
     };
-    float nuk, nva, nvb;
-    fetch(0, nuk, nva, nvb);
+    if (tid < 384) vec[tid] = fetch1(0);
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * 128, D = m - n;
-      float *tu = vec + 128 * (n & 1);  // uk of key tile n
-      if (tid < 128) tu[tid] = nuk;
-      const float vrA = nva, vrB = nvb;
-      if (n + 1 < nTiles) fetch(n + 1, nuk, nva, nvb);
+      const float *tu = vec + 384 * (n & 1);
+      const float nv = (tid < 384 && n + 1 < nTiles) ? fetch1(n + 1) : 0.f;
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
@@ -635,8 +632,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_skew<ROT_LD>(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, g, qt, lane, c1, vrA * c1, vrB * c1,
-                           rot);
+          txl_skew<ROT_LD>(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, g, qt, lane, c1, tu[128 + il],
+                           tu[256 + il], rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -699,12 +696,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         // the previous tile's dS K MMAs read T_DS: wait for them (long done in practice)
         if (n >= 1 && !warp_wait(BAR(B_DSFREE), (n - 1) & 1, abort_flag, status)) good = false;
         if (good) tmem_st16(tl + T_DS + 16 * qt, pk);
-        store_E(smem + OFF_ROT, il, cb, x);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = prmt(pk[e], pk[e], 0x1032u);  // swap halves: (x[2e+1], x[2e])
+        store_E(smem + OFF_ROT, il, cb, pk);
         tmem_wait_st();
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
+      if (tid < 384) vec[384 * ((n + 1) & 1) + tid] = nv;  // tile n - 1's terms were read before this tile's first barrier
     }
     good = good && warp_wait(BAR(B_DSFREE), (nTiles - 1) & 1, abort_flag, status);  // last dQ MMAs done
     if (good) {
@@ -888,31 +888,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
     bool good = true;
-    // v.r of offset il of the band's two blocks (fixed for the CTA)
-    const int ra = 128 * D + il + p.off, rb = ra - 128;
-    const float vrA = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
-    const float vrB = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
-    auto fetch = [&](int t, float &l2, float &dv, float &ukv) {  // one tile ahead
-      const int m = m0 + t, i = m * 128 + il, j0 = (m - D) * 128;
-      l2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
-      dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
-      ukv = (tid < 128 && j0 + tid < L) ? A.uk[(size_t)bh * L + j0 + tid] * c1 : 0.f;  // pre-scaled
+    // smem terms: c1 v.r of the band's two blocks (offset r: [r], [128 + r], fixed), then
+    // per tile, double-buffered and staged one tile ahead (one element per thread):
+    // [lse2 of the rows | D of the rows | c1 u.k of the keys]
+    if (tid < 256) {
+      const int ro = 128 * (tid < 128 ? D : D - 1) + (tid & 127) + p.off;
+      vec[tid] = (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
+    }
+    auto fetch1 = [&](int t) {
+      const int m = m0 + t, r = tid & 127, w = tid >> 7, i = m * 128 + r, j = (m - D) * 128 + r;
+      if (w == 0) return (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      if (w == 1) return (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
+      return (j < L) ? A.uk[(size_t)bh * L + j] * c1 : 0.f;
     };
-    float nl2, ndv, nuk;
-    fetch(0, nl2, ndv, nuk);
+    if (tid < 384) vec[256 + tid] = fetch1(0);
     for (int t = 0; t < iters; ++t) {
       const int m = m0 + t, nn = m - D, i = m * 128 + il, j0 = nn * 128;
-      const float lse2 = nl2, Dv = ndv;
-      float *tu = vec + 384 + 128 * (t & 1);
-      if (tid < 128) tu[tid] = nuk;
-      if (t + 1 < iters) fetch(t + 1, nl2, ndv, nuk);
+      const float *tv = vec + 256 + 384 * (t & 1), *tu = tv + 256;
+      const float nv = (tid < 384 && t + 1 < iters) ? fetch1(t + 1) : 0.f;
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
       if (good) {
         tc_fence_after();
         if (hasA) {
-          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, c1, vrA * c1, vrB * c1, rot);
+          txl_skew<ROT_LD>(tl, 0, 128, hasB, g, qt, lane, c1, vec[il], vec[128 + il], rot);
         } else {
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
@@ -922,10 +922,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       }
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
-      float ds[NC];
+      uint32_t ds[NC / 2];  // dS as bf16 pairs (x[2k+1] low, x[2k] high)
       const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
       if (good) {
         tc_fence_after();
+        const float lse2 = tv[il], Dv = tv[128 + il];
         const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
         auto pds = [&](auto masked) {
 #pragma unroll
@@ -951,8 +952,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
 #pragma unroll
               for (int e = 0; e < 4; ++e) pr[e] = ex2(y[e]);
               ds_pairs(pr, rp + 4 * c4, nDv, dd);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) ds[x0 + e] = dd[e];
+              ds[x0 / 2] = pack_bf16x2(dd[1], dd[0]);
+              ds[x0 / 2 + 1] = pack_bf16x2(dd[3], dd[2]);
             }
           }
         };
@@ -961,7 +962,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         mbar_arrive(BAR(B_SDPCONS));  // S / dP read: T(t + 1) may overwrite them
       } else {
 #pragma unroll
-        for (int x = 0; x < NC; ++x) ds[x] = 0.f;
+        for (int x = 0; x < NC / 2; ++x) ds[x] = 0u;
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
@@ -970,6 +971,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
+      if (tid < 384) vec[256 + 384 * ((t + 1) & 1) + tid] = nv;  // tile t - 1's terms were read before this tile's first barrier
     }
     // ---- epilogue: lane il now is offset c = il of both blocks; 16 columns per thread ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);

@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       const int j0 = n * BN;
       float va = 0.f;
       if (MECH == M_TXL) {
-        if (tid < 128 && j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid] * c1;  // pre-scaled
+        if (tid < 128 && j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid];
       } else if (MECH == M_T5) {
         const int idx = j0 - i0 - 127 + tid + L - 1;
         if (tid < 255 && idx >= 0 && idx < 2 * L - 1) va = p.t5_bias[(size_t)h * (2 * L - 1) + idx];
@@ -359,8 +359,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (MECH == M_TXL) {
         if (good) {
           const bool hasB = !(p.causal && Delta == 0);
-          txl_skew<ROT_LD, SK_PACKED>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane, c1,
-                                      vrA * c1, vrB * c1, rot);
+          txl_skew<ROT_LD, SK_ADD>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane, 1.f,
+                                   vrA, vrB, rot);
           tc_fence_before();
           mbar_arrive(BAR(B_SFREE));
         }
@@ -370,10 +370,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int c4 = 0; c4 < NC / 4; ++c4) {
           const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
           const float4 uk = *reinterpret_cast<const float4 *>(tv + cb + 4 * c4);
-          // log2-domain score s c1 + r' + u' (relative and u.k terms pre-scaled by c1)
-          f2_split(fma2(f2(x[4 * c4], x[4 * c4 + 1]), c12, add2(f2(rr.x, rr.y), f2(uk.x, uk.y))), x[4 * c4], x[4 * c4 + 1]);
-          f2_split(fma2(f2(x[4 * c4 + 2], x[4 * c4 + 3]), c12, add2(f2(rr.z, rr.w), f2(uk.z, uk.w))), x[4 * c4 + 2],
-                   x[4 * c4 + 3]);
+          x[4 * c4 + 0] = (x[4 * c4 + 0] + rr.x + uk.x) * c1;
+          x[4 * c4 + 1] = (x[4 * c4 + 1] + rr.y + uk.y) * c1;
+          x[4 * c4 + 2] = (x[4 * c4 + 2] + rr.z + uk.z) * c1;
+          x[4 * c4 + 3] = (x[4 * c4 + 3] + rr.w + uk.w) * c1;
         }
       } else if (MECH == M_T5) {
         if (good) {
