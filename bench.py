@@ -85,6 +85,17 @@ def kernel_launches(wl, path):
     return fwd, bwd
 
 
+# DRAM traffic per call (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture of the same build and workload, summed over the pass's captured kernels; set to
+# None whenever those kernels change.  Source: profiles/tc_kernels_txl_causal_L8192.md.
+DRAM_TRAFFIC = {
+    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (308.63e6, "tc_bwd_kv + tc_bwd_q + tc_bwd_diag + reduce_dr "
+                                                   "(the relation prep, D and u/v reduction kernels, about 35 MB "
+                                                   "of algorithmic traffic, were not captured)"),
+    ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.20e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
+}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -302,8 +313,11 @@ def run_ours(args, wl):
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     if tensor_path:
         peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        traffic, traffic_src = DRAM_TRAFFIC.get((wl.name, dom), (None, None))
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None, "kernel": dom, "peak_kind": f"bf16 sustained ({peak_src})"}
+                "traffic": traffic, "kernel": dom, "peak_kind": f"bf16 sustained ({peak_src})"}
+        if traffic is not None:
+            roof["traffic_kernels"] = traffic_src
     else:
         # CUDA-core path: fp32 FFMA bound, peak = 148 SMs x 128 lanes x 2 flop x max SM clock
         peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
