@@ -128,7 +128,7 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
-  if (pass == 1) return p.mech == rp::M_TXL;  // other mechanisms: CUDA-core backward
+  if (pass == 1) return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p));
   return rp::tc_supported(p);
 }
 
@@ -136,7 +136,7 @@ static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
 struct Layout {
   size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot;
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
-  size_t part_kv, part_dg, part_uv;  // tensor-core backward partials
+  size_t part_kv, part_dg, part_uv, qa;  // tensor-core backward partials / products
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -165,7 +165,11 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
       l.p2cE = take(sizeof(float) * BH * p.L * 2);
     }
   }
-  if (pass == 1 && tc) {  // tensor-core backward (Transformer-XL)
+  if (pass == 1 && tc && p.mech == rp::M_SHAW) {  // tensor-core backward (Shaw)
+    l.dvec = take(sizeof(float) * BH * p.L);
+    l.qa = take(sizeof(float) * rp::tc_bwd_shaw_qa_floats(p));
+    l.part_row = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nrows * rp::HD);
+  } else if (pass == 1 && tc) {  // tensor-core backward (Transformer-XL)
     size_t kvf = 0;
     const size_t dgf = rp::tc_bwd_part_floats(p, kvf);
     l.dvec = take(sizeof(float) * BH * p.L);
@@ -219,6 +223,7 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.part_kv = (float *)(b + l.part_kv);
   w.part_dg = (float *)(b + l.part_dg);
   w.part_uv = (float *)(b + l.part_uv);
+  w.qa = (float *)(b + l.qa);
   return w;
 }
 
@@ -315,6 +320,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(rel[0]))
       return RELPOS_ERR_INVALID_ARG;
     if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;
+    if (p.mech == rp::M_SHAW) return to_status(rp::tc_bwd_shaw(p, tc_work(l, workspace), st));
     return to_status(rp::tc_bwd(p, tc_work(l, workspace), st));
   }
   if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;

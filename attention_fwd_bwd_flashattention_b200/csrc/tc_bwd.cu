@@ -1,13 +1,13 @@
 // Tensor-core (tcgen05 / TMEM / TMA) backward pass of Transformer-XL relative
 // attention, bf16, d = 64, sm_100a.  No atomics anywhere.
 //
-// Three kernels share one per-tile engine: two threads per query row (warps w and
-// w + 4 share TMEM lanes 32 (w & 3)..+31 and take key columns [0,64) / [64,128));
-// warp 8 lane 0 issues every TMA load and tcgen05.mma.  For a 128 x 128 tile
+// Three kernels share one per-tile engine (tc_bwd_common.cuh): four threads per query
+// row in 16 row warps, and one control warp whose lane 0 issues every TMA load and
+// tcgen05.mma.  For a 128 x 128 tile
 // (query tile m, key tile n, Delta = m - n) the offsets are i - j = 128 Delta +
 // [-127, 127], i.e. the two 128-offset blocks Delta and Delta - 1 of r; the rows
 // recompute S = s((q + u).k + (q + v).r) exactly as the forward does (relation
-// products by MMA, rotated into key order through a padded smem row), then
+// products by MMA, skewed into key order through padded smem rows), then
 // P = exp(S - LSE), dP = dO V^T, dS = P (dP - D) with D = rowsum(dO o O).
 //
 //   key-tile kernel   (one CTA per key tile n, query tiles streamed):
@@ -35,19 +35,12 @@
 #include "kernels.h"
 #include "tc_ptx.cuh"
 #include "tc_skew.cuh"
+#include "tc_bwd_common.cuh"
 
 namespace rp {
 namespace tcb {
 
 using namespace tc;
-
-constexpr int TPR = 4;            // row threads per query row
-constexpr int NC = 128 / TPR;     // key columns per row thread
-constexpr int NSOFT = 128 * TPR;  // row threads
-constexpr int CTRL_WARP = NSOFT / 32;
-constexpr int NTHREADS = NSOFT + 32;
-constexpr int ROT_LD = 132;
-constexpr float LOG2E = 1.4426950408889634f;
 
 struct BwdArgs {
   CUtensorMap mq, mk, mv, mdo, mr;
@@ -61,62 +54,6 @@ struct BwdArgs {
 
 constexpr int DG_STRIDE = 2 * 128 * 65;
 
-__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-// Four log2-domain scores y = s c1 + (r' + u') - lse2 of consecutive keys, from the
-// QK^T accumulator bits, the relative terms r' and u.k terms u' (both already
-// multiplied by c1 = scale log2 e) and nlse = (-lse2, -lse2); two f32x2 pairs.
-__device__ __forceinline__ void score_pairs(const uint32_t *s, float4 rr, float4 uk, uint64_t c12, uint64_t nlse, float (&y)[4]) {
-  f2_split(fma2(f2(u2f(s[0]), u2f(s[1])), c12, add2(add2(f2(rr.x, rr.y), f2(uk.x, uk.y)), nlse)), y[0], y[1]);
-  f2_split(fma2(f2(u2f(s[2]), u2f(s[3])), c12, add2(add2(f2(rr.z, rr.w), f2(uk.z, uk.w)), nlse)), y[2], y[3]);
-}
-// dS = P (dP - D) for four keys, nDv = (-D, -D).
-__device__ __forceinline__ void ds_pairs(const float (&pr)[4], const uint32_t *dp, uint64_t nDv, float (&dd)[4]) {
-  f2_split(mul2(f2(pr[0], pr[1]), add2(f2(u2f(dp[0]), u2f(dp[1])), nDv)), dd[0], dd[1]);
-  f2_split(mul2(f2(pr[2], pr[3]), add2(f2(u2f(dp[2]), u2f(dp[3])), nDv)), dd[2], dd[3]);
-}
-
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *ab, int32_t *st) {
-  const bool ok = mbar_wait(bar, parity, ab, st, RELPOS_ERR_TIMEOUT_DEV);
-  return __all_sync(0xffffffffu, ok);
-}
-
-// Control-thread bookkeeping: TMA loads issued but not waited for are drained on exit.
-struct Ctl {
-  uint32_t pb[8], pp[8];
-  int np;
-  volatile int *ab;
-  int32_t *st;
-  __device__ void expect(uint32_t bar, uint32_t par, uint32_t bytes) {
-    mbar_expect_tx(bar, bytes);
-    pb[np] = bar;
-    pp[np] = par;
-    ++np;
-  }
-  __device__ bool wait(uint32_t bar, uint32_t par) { return mbar_wait(bar, par, ab, st, RELPOS_ERR_TIMEOUT_DEV); }
-  __device__ bool wait_load(uint32_t bar, uint32_t par) {
-    if (!wait(bar, par)) return false;
-    for (int e = 0; e < np; ++e)
-      if (pb[e] == bar && pp[e] == par) {
-        pb[e] = pb[np - 1];
-        pp[e] = pp[np - 1];
-        --np;
-        break;
-      }
-    return true;
-  }
-  __device__ void drain(uint32_t drain_bar) {
-    umma_commit(drain_bar);
-    volatile int none = 0;
-    mbar_wait(drain_bar, 0, &none, st, RELPOS_ERR_TIMEOUT_DEV);
-    for (int e = 0; e < np; ++e) mbar_wait(pb[e], pp[e], &none, st, RELPOS_ERR_TIMEOUT_DEV);
-  }
-};
-
 // dS of this thread's NC keys (jl = cb + e, e = 0..NC-1) of row il, written into
 // the two 128x128 bf16 operand tiles of the relation products in offset order
 // (128-byte-swizzled K-major, 64-column halves 16 KB apart; E_lo at E, E_hi at
@@ -128,11 +65,6 @@ struct Ctl {
 // are written alone.
 __device__ __forceinline__ uint32_t E_off(uint32_t t, uint32_t rowb, uint32_t r7) {  // t = 2 c', c' even
   return (((t << 7) & 0xC000u) ^ 0x8000u) + rowb + ((t & 126u) ^ r7);
-}
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
 }
 // pk[k] = bf16 pair (x[2k+1] low, x[2k] high) of the thread's values
 __device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const uint32_t (&pk)[NC / 2]) {

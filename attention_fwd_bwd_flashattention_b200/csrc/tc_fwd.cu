@@ -673,6 +673,22 @@ static cudaError_t launch_fwd_t(const FwdArgs &a, cudaStream_t st) {
 
 }  // namespace tc
 
+// [planes][rows][row_len] fp32 rows (row_len * 4 bytes a multiple of 16), no swizzle;
+// box = row_len x box_rows x 1 lands as contiguous padded rows; rows outside
+// [0, rows) read as zeros.
+bool tc_make_map_f32_rows(CUtensorMap *m, const void *base, uint32_t row_len, uint64_t rows, uint64_t planes,
+                          uint32_t box_rows) {
+  tc::EncodeTiledFn enc = tc::encode_fn();
+  if (!enc || (row_len * 4u) % 16u != 0 || row_len > 256) return false;
+  cuuint64_t dims[3] = {row_len, rows, planes};
+  cuuint64_t strides[2] = {(cuuint64_t)row_len * 4, (cuuint64_t)rows * row_len * 4};
+  cuuint32_t box[3] = {row_len, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows) {
   return tc::make_map(m, base, rows, planes, box_rows);
 }

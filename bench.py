@@ -80,6 +80,8 @@ def kernel_launches(wl, path):
         fwd = 1 + t5
     if tc and wl.mech == TXL:  # D, relation prep, key-tile, query-tile, diagonal, dr and u/v reductions
         bwd = 7
+    elif tc and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction
+        bwd = 5
     else:  # D, key-tile, query-tile, then the table-gradient reductions
         bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2}[wl.mech]
     return fwd, bwd

@@ -23,12 +23,20 @@ def params_of(wl, path):
 
 
 def run_gpu(wl, inp, path, dev="cuda"):
+    """Forward + backward through the C ABI; the device status word must stay 0 (a
+    bounded wait that ran out inside a kernel reports RELPOS_ERR_TIMEOUT there)."""
     P = params_of(wl, path)
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
     rel = [r.to(dev) for r in inp["rel"]]
-    o, lse = bd.forward(P, q, k, v, rel)
-    dq, dk, dv, drel = bd.backward(P, q, k, v, rel, o, lse, do)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    bd.relpos_attn_fwd(P, q, k, v, rel, o, lse, bd.workspace(P, 0, q.device), dev_status=status)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    drel = [torch.empty(r.shape, dtype=torch.float32, device=dev) for r in rel[: P.n_rel()]]
+    bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, bd.workspace(P, 1, q.device), dev_status=status)
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, f"{wl.name}: device status {int(status.item())} ({bd.strerror(int(status.item()))})"
     return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, drel=drel)
 
 
