@@ -965,27 +965,23 @@ __global__ void __launch_bounds__(256) reduce_dr_kernel(BwdArgs A) {
         const int len = p.nT - (D < 0 ? -D : D);
         const int nch = (len + A.dg_ch - 1) / A.dg_ch;
         const float *part = A.part_dg + (bh * A.nbands + band) * A.dg_nchunk * DG_STRIDE + (size_t)(65 * w) * 128 + c;
-        // two chunks' loads in flight before their (in-order) accumulation
-        int ch = 0;
-        for (; ch + 1 < nch; ch += 2) {
-          const float *p0 = part + (size_t)ch * DG_STRIDE, *p1 = p0 + DG_STRIDE;
-          float v0[9], v1[9];
+        // up to four chunks' loads in flight before their (in-order) accumulation
+        for (int ch = 0; ch < nch; ch += 4) {
+          float v[4][9];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            v0[k] = __ldg(p0 + (size_t)(8 * eg + k) * 128);
-            v1[k] = __ldg(p1 + (size_t)(8 * eg + k) * 128);
+          for (int u = 0; u < 4; ++u) {
+            const float *pu = part + (size_t)(ch + u) * DG_STRIDE;
+            const bool have = ch + u < nch;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[u][k] = have ? __ldg(pu + (size_t)(8 * eg + k) * 128) : 0.f;
+            v[u][8] = have ? __ldg(pu + (size_t)64 * 128) : 0.f;
           }
-          v0[8] = __ldg(p0 + (size_t)64 * 128);
-          v1[8] = __ldg(p1 + (size_t)64 * 128);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] = (acc[k] + v0[k]) + v1[k];
-          gs = (gs + v0[8]) + v1[8];
-        }
-        if (ch < nch) {
-          const float *p0 = part + (size_t)ch * DG_STRIDE;
+          for (int u = 0; u < 4; ++u) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[k] += __ldg(p0 + (size_t)(8 * eg + k) * 128);
-          gs += __ldg(p0 + (size_t)64 * 128);
+            for (int k = 0; k < 8; ++k) acc[k] += v[u][k];
+            gs += v[u][8];
+          }
         }
       }
     }
@@ -1004,15 +1000,26 @@ __global__ void __launch_bounds__(256) reduce_dr_kernel(BwdArgs A) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) pv[k] = 0.f;
   }
+  // sum over the 32 lanes of eight values in 9 shuffles: halve the set at xor 16, 8, 4
+  // (each lane keeps the half its bit selects), then finish at xor 2, 1; lane 4k ends
+  // with the sum of value k (a fixed order)
+  {
+    const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
+    float h4[4], h3[2];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+    for (int j = 0; j < 4; ++j) {
+      const float send = b4 ? pv[j] : pv[j + 4], keep = b4 ? pv[j + 4] : pv[j];
+      h4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
 #pragma unroll
-    for (int sh = 16; sh > 0; sh >>= 1) pv[k] += __shfl_xor_sync(0xffffffffu, pv[k], sh);
-  }
-  if (lane == 0) {
-    float *dst = A.part_uv + ((size_t)h * ntile + tile) * HD + 8 * eg;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) dst[k] = pv[k];
+    for (int j = 0; j < 2; ++j) {
+      const float send = b3 ? h4[j] : h4[j + 2], keep = b3 ? h4[j + 2] : h4[j];
+      h3[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float h2 = (b2 ? h3[1] : h3[0]) + __shfl_xor_sync(0xffffffffu, b2 ? h3[0] : h3[1], 4);
+    h2 += __shfl_xor_sync(0xffffffffu, h2, 2);
+    h2 += __shfl_xor_sync(0xffffffffu, h2, 1);
+    if ((lane & 3) == 0) A.part_uv[((size_t)h * ntile + tile) * HD + 8 * eg + (lane >> 2)] = h2;
   }
 }
 
