@@ -118,3 +118,25 @@ def test_t5_thresholds_match_oracle_buckets(lib):
     for nb, md, bidir in ((32, 128, True), (10, 40, True), (7, 20, False), (64, 1000, True)):
         bd.relpos_attn_workspace_size(bd.Params(mech=0, B=1, H=1, L=100, t5_num_buckets=nb, t5_max_distance=md,
                                                 t5_bidirectional=bidir), 0)
+
+
+def test_resolved_paths(lib):
+    """Which kernel family each pass runs (host-side dispatch, no device work): bf16
+    runs on the tensor cores except the backward of T5, DeBERTa and Shaw with c > 64;
+    float32 and an explicit CUDA-core request always run the CUDA-core kernels."""
+    TC, SIMT = bd.PATH_TC, bd.PATH_SIMT
+    want = {  # (mech, clip) -> (forward, backward) for bf16, automatic choice
+        (bd.T5, 64): (TC, SIMT),
+        (bd.SHAW, 64): (TC, TC),
+        (bd.SHAW, 65): (TC, SIMT),
+        (bd.SHAW, 100): (SIMT, SIMT),
+        (bd.TXL, 64): (TC, TC),
+        (bd.DEBERTA, 64): (TC, SIMT),
+    }
+    for (mech, clip), (f, b) in want.items():
+        P = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip)
+        assert (bd.relpos_attn_resolved_path(P, 0), bd.relpos_attn_resolved_path(P, 1)) == (f, b), (mech, clip)
+        P32 = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip, dtype=bd.F32)
+        assert bd.relpos_attn_resolved_path(P32, 0) == SIMT and bd.relpos_attn_resolved_path(P32, 1) == SIMT
+        Ps = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip, kernel_path=bd.PATH_SIMT)
+        assert bd.relpos_attn_resolved_path(Ps, 0) == SIMT and bd.relpos_attn_resolved_path(Ps, 1) == SIMT

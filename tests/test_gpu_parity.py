@@ -54,6 +54,21 @@ def test_parity_deberta_span256(path):
     compare_full(wl, inp, run_gpu(wl, inp, path))
 
 
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("clip", [1, 7, 33, 64, 100])
+@pytest.mark.parametrize("L", [300, 700])
+def test_parity_shaw_clip(clip, causal, L):
+    """Shaw's clip decides which tiles hold unclipped offsets (the tensor-core backward's
+    band tiles: only the diagonal one for small c) and where each row's clipped pairs
+    start; c > 64 runs the CUDA-core backward."""
+    wl = small_wl("shaw", torch.bfloat16, causal, L, shaw_clip=clip)
+    P = bd.Params(mech=SHAW, B=wl.B, H=wl.H, L=L, causal=causal, shaw_clip=clip)
+    want_bwd = bd.PATH_TC if clip <= 64 else bd.PATH_SIMT
+    assert bd.relpos_attn_resolved_path(P, 1) == want_bwd
+    inp = make_inputs(wl, seed=clip + L)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_parity_t5_unidirectional_and_odd_buckets(causal):
     for nb, md, bidir in ((32, 128, False), (10, 40, True), (7, 20, False)):
