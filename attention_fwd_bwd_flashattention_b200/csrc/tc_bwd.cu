@@ -405,7 +405,7 @@ constexpr int OFF_ROT = OFF_R + 3 * 16384;  // rot rows; E_lo at +0, E_hi at +32
 constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
-enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_PDS, B_PDSFREE, B_DSFREE, B_DRAIN, NB };
+enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_DPCONS, B_PDS, B_PDSFREE, B_DSFREE, B_DRAIN, NB };
 constexpr uint32_t T_S = 0, T_REL = 128, T_DQ = 384, T_DS = 448;
 }  // namespace qk
 
@@ -435,6 +435,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_TCONS), NSOFT);
     mbar_init(BAR(B_DPF), 1);
+    mbar_init(BAR(B_DPCONS), NSOFT);
     mbar_init(BAR(B_PDS), NSOFT);
     mbar_init(BAR(B_PDSFREE), 1);
     mbar_init(BAR(B_DSFREE), 1);
@@ -495,11 +496,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         if (n + 1 < nTiles) {
           if (!ctl.wait_load(BAR(B_ST0 + (st ^ 1)), ((n + 1) >> 1) & 1)) break;
           umma_k64(tbase + T_S, sbase + OFF_Q, sbase + OFF_K + 16384 * (st ^ 1), idS, false);  // S(n+1)
+          // relation block D - 2 for tile n + 1 into the slot dP(n) used, once the rows have
+          // read dP(n): it runs under their dS / E stores
+          if (!ctl.wait(BAR(B_DPCONS), n & 1)) break;
+          tc_fence_after();
+          if (block_valid(p, D - 2))
+            umma_k64(tbase + slotA, sbase + OFF_R + 16384 * slot3(D - 2), sbase + OFF_Q, idS, false);
+          umma_commit(BAR(B_SFULL));
         }
         if (!ctl.wait(BAR(B_PDS), n & 1)) break;
         tc_fence_after();
         // dQ += E_lo r_D + E_hi r_{D-1} (E in smem, freed first so the rows can skew the
-        // next tile), then the next tile's relation block, then dQ += dS K_n (dS in TMEM)
+        // next tile), then dQ += dS K_n (dS in TMEM)
         uint32_t acc = n > 0 ? 1u : 0u;
         if (block_valid(p, D)) {
 #pragma unroll
@@ -516,11 +524,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
           acc = 1u;
         }
         umma_commit(BAR(B_PDSFREE));
-        if (n + 1 < nTiles) {  // relation block D - 2 for tile n + 1, into the slot dP(n) used
-          if (block_valid(p, D - 2))
-            umma_k64(tbase + slotA, sbase + OFF_R + 16384 * slot3(D - 2), sbase + OFF_Q, idS, false);
-          umma_commit(BAR(B_SFULL));
-        }
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           umma_bf16_ts(tbase + T_DQ, tbase + T_DS + 8 * k, sdesc_sw128(sbase + OFF_K + 16384 * st + 2048 * k, 16, 1024), idDQ,
@@ -619,6 +622,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
           for (int e = 0; e < 4; ++e) x[4 * c4 + e] = dd[e];
         }
         tc_fence_before();
+        mbar_arrive(BAR(B_DPCONS));  // dP(n) read: the next relation block may overwrite it
       }
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
