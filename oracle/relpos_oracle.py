@@ -47,8 +47,13 @@ Readings where the pages are silent (listed again in the design notes):
     boundaries a = 16, 32, 64).
   * Shaw: the scale multiplies the whole logit (content and position parts).
   * T5: the bias is added unscaled.
-  * Fully masked rows (possible only with an empty key set) give O = 0 and
-    LSE = -inf and zero gradients.
+  * Variable-length batches (the speech batches of the article, section "为什么
+    相对位置注意力难做快"): an optional per-batch key length ``seqlens_k[b]``
+    masks keys j >= seqlens_k[b] of that batch (after causal masking); queries are
+    all computed.  Relative positions keep their meaning (j - i over the padded
+    length L), so the tables and index maps do not change.
+  * Fully masked rows (an empty key set: seqlens_k[b] = 0, or a causal row whose
+    keys are all padding) give O = 0 and LSE = -inf and zero gradients.
   * LSE is the natural log of the softmax denominator.
 
 All arithmetic is float64.  Inputs given in bf16 are expected to be upcast by
@@ -175,11 +180,13 @@ def index_map(mech: int, L: int, causal: bool, cfg: RelCfg, rows_i: np.ndarray, 
     return np.clip(n + k, 0, 2 * k - 1)  # delta(j, i) = clip(j - i + k)
 
 
-def _mask(L: int, causal: bool, rows_i: np.ndarray) -> np.ndarray:
-    """True where the pair is allowed."""
-    if not causal:
-        return np.ones((rows_i.size, L), dtype=bool)
-    return _rel(rows_i, L) <= 0
+def _mask(L: int, causal: bool, rows_i: np.ndarray, lk=None) -> np.ndarray:
+    """True where the pair is allowed: j <= i when causal, and j < lk (the batch's
+    key length) when one is given."""
+    allowed = np.ones((rows_i.size, L), dtype=bool) if not causal else _rel(rows_i, L) <= 0
+    if lk is not None:
+        allowed &= np.arange(L)[None, :] < int(lk)
+    return allowed
 
 
 # --------------------------------------------------------------------------
@@ -219,10 +226,14 @@ def head_bias(mech, q, k, rel_h, scale, cfg, causal, rows_i):
     return scale * (c2p + p2c)
 
 
-def head_scores(mech, q, k, rel_h, scale, cfg, causal, rows_i):
+def head_scores(mech, q, k, rel_h, scale, cfg, causal, rows_i, lk=None):
     """S rows for one (b, h): scale q_i.k_j + B_ij, -inf where masked."""
     S = scale * (q[rows_i] @ k.T) + head_bias(mech, q, k, rel_h, scale, cfg, causal, rows_i)
-    return np.where(_mask(k.shape[0], causal, rows_i), S, -np.inf)
+    return np.where(_mask(k.shape[0], causal, rows_i, lk), S, -np.inf)
+
+
+def _lk(seqlens_k, b):
+    return None if seqlens_k is None else int(seqlens_k[b])
 
 
 def _softmax_rows(S):
@@ -244,8 +255,9 @@ def _head_tables(mech, rel, h):
 # --------------------------------------------------------------------------
 # Public entry points
 # --------------------------------------------------------------------------
-def forward(mech, q, k, v, rel, causal, scale=None, cfg=RelCfg(), rows=None):
-    """O [B,H,R,d] and LSE [B,H,R] for the query rows ``rows`` (default: all).
+def forward(mech, q, k, v, rel, causal, scale=None, cfg=RelCfg(), rows=None, seqlens_k=None):
+    """O [B,H,R,d] and LSE [B,H,R] for the query rows ``rows`` (default: all);
+    ``seqlens_k`` (optional, [B]) masks each batch's keys j >= seqlens_k[b].
 
     q, k, v: [B, H, L, d]; rel: list of per-head tables (see module docstring):
     T5 [t (H,nb)], Shaw [a (H,2c+1,d)], TXL [r (H,n_off,d), u (H,d), v (H,d)],
@@ -260,14 +272,14 @@ def forward(mech, q, k, v, rel, causal, scale=None, cfg=RelCfg(), rows=None):
     for b in range(B):
         for h in range(H):
             rh = _head_tables(mech, rel, h)
-            S = head_scores(mech, q[b, h], k[b, h], rh, scale, cfg, causal, rows_i)
+            S = head_scores(mech, q[b, h], k[b, h], rh, scale, cfg, causal, rows_i, _lk(seqlens_k, b))
             P, lse = _softmax_rows(S)
             O[b, h] = P @ v[b, h]
             LSE[b, h] = lse
     return O, LSE
 
 
-def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg()):
+def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg(), seqlens_k=None):
     """Exact gradients (dq, dk, dv, drel) of  sum(O * dO).
 
     drel matches rel's structure: T5 [dt], Shaw [da], TXL [dr, du, dv],
@@ -283,7 +295,7 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg()):
         for h in range(H):
             rh = _head_tables(mech, rel, h)
             qh, kh, vh, gh = q[b, h], k[b, h], v[b, h], dO[b, h]
-            S = head_scores(mech, qh, kh, rh, scale, cfg, causal, rows_i)
+            S = head_scores(mech, qh, kh, rh, scale, cfg, causal, rows_i, _lk(seqlens_k, b))
             P, _ = _softmax_rows(S)
             O = P @ vh
             dP = gh @ vh.T
@@ -306,7 +318,7 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg()):
             elif mech == TXL:
                 r, u, vv = rh
                 idx = index_map(TXL, L, causal, cfg, rows_i)
-                allowed = _mask(L, causal, rows_i)
+                allowed = _mask(L, causal, rows_i, _lk(seqlens_k, b))
                 M = np.zeros((L, r.shape[0]))
                 sel = allowed.ravel()
                 np.add.at(M, (np.repeat(rows_i, L)[sel], idx.ravel()[sel]), dS.ravel()[sel])
@@ -330,7 +342,7 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg()):
     return dq, dk, dv, drel
 
 
-def backward_rows(mech, q, k, v, rel, causal, dO, rows, scale=None, cfg=RelCfg()):
+def backward_rows(mech, q, k, v, rel, causal, dO, rows, scale=None, cfg=RelCfg(), seqlens_k=None):
     """dq for the query rows ``rows`` only (each is a function of its own row of
     dS, which needs only that row's O, so no full pass is required)."""
     q, k, v, dO = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dO))
@@ -342,7 +354,7 @@ def backward_rows(mech, q, k, v, rel, causal, dO, rows, scale=None, cfg=RelCfg()
         for h in range(H):
             rh = _head_tables(mech, rel, h)
             qh, kh, vh, gh = q[b, h], k[b, h], v[b, h], dO[b, h]
-            S = head_scores(mech, qh, kh, rh, scale, cfg, causal, rows_i)
+            S = head_scores(mech, qh, kh, rh, scale, cfg, causal, rows_i, _lk(seqlens_k, b))
             P, _ = _softmax_rows(S)
             O = P @ vh
             dP = gh[rows_i] @ vh.T
@@ -352,7 +364,7 @@ def backward_rows(mech, q, k, v, rel, causal, dO, rows, scale=None, cfg=RelCfg()
             if mech in (SHAW, TXL, DEBERTA):
                 tab = rh[0]
                 idx = index_map(mech, L, causal, cfg, rows_i, "row")
-                allowed = _mask(L, causal, rows_i)
+                allowed = _mask(L, causal, rows_i, _lk(seqlens_k, b))
                 M = np.zeros((rows_i.size, tab.shape[0]))
                 sel = allowed.ravel()
                 np.add.at(M, (np.repeat(np.arange(rows_i.size), L)[sel], idx.ravel()[sel]), dS.ravel()[sel])

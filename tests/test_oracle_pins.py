@@ -117,7 +117,9 @@ def bf_score(mech, q, k, rel, h, i, j, L, causal, s, cfg):
     return s * (dot(q[i], k[j]) + dot(q[i], rel[0][h][c2p]) + dot(k[j], rel[1][h][p2c]))
 
 
-def brute(mech, q, k, v, rel, causal, do, s, cfg):
+def brute(mech, q, k, v, rel, causal, do, s, cfg, lk=None):
+    """Scalar loops over (i, j) from the mechanism formulas; lk[b] (optional) is the
+    batch's key length: keys j >= lk[b] do not take part."""
     B, H, L, d = q.shape
     O = np.zeros_like(q)
     LSE = np.zeros((B, H, L))
@@ -128,7 +130,10 @@ def brute(mech, q, k, v, rel, causal, do, s, cfg):
             qb, kb, vb, gb = q[b, h], k[b, h], v[b, h], do[b, h]
             P = np.zeros((L, L))
             for i in range(L):
-                keys = [j for j in range(L) if not (causal and j > i)]
+                keys = [j for j in range(L) if not (causal and j > i) and (lk is None or j < lk[b])]
+                if not keys:  # empty key set: O = 0, LSE = -inf, no gradient
+                    LSE[b, h, i] = -math.inf
+                    continue
                 sc = {j: bf_score(mech, qb, kb, rel, h, i, j, L, causal, s, cfg) for j in keys}
                 m = max(sc.values())
                 z = sum(math.exp(x - m) for x in sc.values())
@@ -140,7 +145,7 @@ def brute(mech, q, k, v, rel, causal, do, s, cfg):
             for i in range(L):
                 Di = dot(gb[i], O[b, h, i])
                 for j in range(L):
-                    if causal and j > i:
+                    if (causal and j > i) or (lk is not None and j >= lk[b]):
                         continue
                     dS = P[i, j] * (dot(gb[i], vb[j]) - Di)
                     dv[b, h, j] += P[i, j] * gb[i]
@@ -192,6 +197,59 @@ def test_oracle_vs_brute_force(mech, causal, L, d):
     np.testing.assert_allclose(L2, LSE[:, :, rows], rtol=1e-13, atol=1e-13)
     dq2 = orc.backward_rows(mech, q, k, v, rel, causal, do, rows, s, SMALL)
     np.testing.assert_allclose(dq2, dq[:, :, rows], rtol=1e-12, atol=1e-12)
+
+
+SEQ_CASES = [(mech, causal, L, lk) for mech in (T5, SHAW, TXL, DEBERTA) for causal in (False, True)
+             for (L, lk) in ((3, (2, 0)), (5, (5, 1)), (8, (3, 7)))]
+
+
+@pytest.mark.parametrize("mech,causal,L,lk", SEQ_CASES)
+def test_oracle_key_lengths_vs_brute_force(mech, causal, L, lk):
+    """Variable key lengths: the oracle's masked path against the scalar loops."""
+    q, k, v, do, rel = make_case(mech, 2, 2, L, 2, causal, SMALL, seed=L * 7 + lk[0])
+    s = 0.41
+    O, LSE = orc.forward(mech, q, k, v, rel, causal, s, SMALL, seqlens_k=lk)
+    dq, dk, dv, drel = orc.backward(mech, q, k, v, rel, causal, do, s, SMALL, seqlens_k=lk)
+    bO, bL, bdq, bdk, bdv, bdrel = brute(mech, q, k, v, rel, causal, do, s, SMALL, lk=lk)
+    np.testing.assert_array_equal(np.isneginf(LSE), np.isneginf(bL))
+    fin = np.isfinite(bL)
+    np.testing.assert_allclose(LSE[fin], bL[fin], rtol=1e-12, atol=1e-12)
+    for got, want in [(O, bO), (dq, bdq), (dk, bdk), (dv, bdv)] + list(zip(drel, bdrel)):
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    rows = np.arange(L)[1::2]
+    dq2 = orc.backward_rows(mech, q, k, v, rel, causal, do, rows, s, SMALL, seqlens_k=lk)
+    np.testing.assert_allclose(dq2, dq[:, :, rows], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mech", [T5, SHAW, TXL, DEBERTA])
+def test_padding_keys_do_not_matter(mech):
+    """Keys past a batch's length change nothing but get zero dk, dv; an empty key
+    set gives O = 0, LSE = -inf and zero gradients; a full length is no mask."""
+    L = 7
+    q, k, v, do, rel = make_case(mech, 2, 2, L, 4, False, SMALL, seed=11)
+    lk = (4, 0)
+    base = orc.forward(mech, q, k, v, rel, False, 0.3, SMALL, seqlens_k=lk)
+    gb = orc.backward(mech, q, k, v, rel, False, do, 0.3, SMALL, seqlens_k=lk)
+    k2, v2 = k.copy(), v.copy()
+    rng = np.random.default_rng(5)
+    k2[0, :, 4:] = rng.standard_normal(k2[0, :, 4:].shape)
+    v2[0, :, 4:] = rng.standard_normal(v2[0, :, 4:].shape)
+    k2[1] = rng.standard_normal(k2[1].shape)
+    v2[1] = rng.standard_normal(v2[1].shape)
+    alt = orc.forward(mech, q, k2, v2, rel, False, 0.3, SMALL, seqlens_k=lk)
+    ga = orc.backward(mech, q, k2, v2, rel, False, do, 0.3, SMALL, seqlens_k=lk)
+    np.testing.assert_allclose(alt[0], base[0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(alt[1], base[1])
+    np.testing.assert_allclose(ga[0], gb[0], rtol=1e-12, atol=1e-13)  # dq
+    for t in range(len(rel)):  # table gradients (TXL du = s sum_j c_j k_j: masked keys have c_j = 0)
+        np.testing.assert_allclose(ga[3][t], gb[3][t], rtol=1e-12, atol=1e-13)
+    assert np.all(gb[1][0, :, 4:] == 0) and np.all(gb[2][0, :, 4:] == 0)
+    assert np.all(base[0][1] == 0) and np.all(np.isneginf(base[1][1]))
+    assert all(np.all(g[1] == 0) for g in gb[:3])
+    full = orc.forward(mech, q, k, v, rel, False, 0.3, SMALL, seqlens_k=(L, L))
+    plain = orc.forward(mech, q, k, v, rel, False, 0.3, SMALL)
+    np.testing.assert_array_equal(full[0], plain[0])
+    np.testing.assert_array_equal(full[1], plain[1])
 
 
 # ----------------------------------------------------------------------------
