@@ -44,6 +44,7 @@ class relpos_params_t(ctypes.Structure):
         ("t5_bidirectional", ctypes.c_int32),
         ("shaw_clip", ctypes.c_int32),
         ("deberta_span", ctypes.c_int32),
+        ("seqlens_k", ctypes.c_void_p),
     ]
 
 
@@ -105,14 +106,19 @@ class Params:
     t5_bidirectional: bool = True
     shaw_clip: int = 64
     deberta_span: int = 256
+    seqlens_k: Optional[torch.Tensor] = None  # [B] int32 on the device, or None (all L)
 
     def c(self) -> relpos_params_t:
         scale = self.scale
         if scale is None:
             scale = 1.0 / math.sqrt(3 * self.d) if self.mech == DEBERTA else 1.0 / math.sqrt(self.d)
+        if self.seqlens_k is not None:
+            t = self.seqlens_k
+            if t.dtype != torch.int32 or t.numel() != self.B or not t.is_contiguous():
+                raise ValueError("seqlens_k must be a contiguous int32 tensor of B elements")
         return relpos_params_t(self.mech, self.dtype, int(self.causal), self.kernel_path, self.B, self.H, self.L, self.d,
                                float(scale), self.t5_num_buckets, self.t5_max_distance, int(self.t5_bidirectional),
-                               self.shaw_clip, self.deberta_span)
+                               self.shaw_clip, self.deberta_span, _ptr(self.seqlens_k))
 
     def n_rel(self) -> int:
         return {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2}[self.mech]

@@ -14,7 +14,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kVersion = 10100;  // 1.1.0: relpos_params_t.seqlens_k
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -91,6 +91,7 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   p.H = (int)P->H;
   p.L = (int)P->L;
   p.scale = P->scale;
+  p.seqlens_k = P->seqlens_k;
   p.nT = (p.L + kTile - 1) / kTile;
   switch (P->mech) {
     case RELPOS_T5: {
@@ -248,6 +249,18 @@ extern "C" int relpos_attn_workspace_size(const relpos_params_t *params, int pas
   return RELPOS_OK;
 }
 
+// seqlens_k is read by the kernels: it must be device (or managed) memory; a host
+// pointer is rejected here rather than faulting on the device.
+static int check_seqlens(const relpos_params_t *P) {
+  if (!P->seqlens_k) return RELPOS_OK;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, P->seqlens_k) != cudaSuccess) {
+    cudaGetLastError();  // reset the runtime's last-error state after the failed query
+    return RELPOS_ERR_INVALID_ARG;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) ? RELPOS_OK : RELPOS_ERR_INVALID_ARG;
+}
+
 extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, const void *k, const void *v,
                                const void *const rel[3], void *o, float *lse, void *workspace,
                                size_t workspace_bytes, int32_t *dev_status, void *stream) {
@@ -257,6 +270,7 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   if (!q || !k || !v || !rel || !o || !lse) return RELPOS_ERR_INVALID_ARG;
   for (int i = 0; i < rel_count(p.mech); ++i)
     if (!rel[i]) return RELPOS_ERR_INVALID_ARG;
+  if ((e = check_seqlens(params))) return e;
   const bool tc = use_tc(params, p, 0);
   if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
   if (tc) {  // TMA needs 16-byte aligned tensors
@@ -293,6 +307,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   if (!q || !k || !v || !rel || !o || !lse || !dout || !dq || !dk || !dv || !drel) return RELPOS_ERR_INVALID_ARG;
   for (int i = 0; i < rel_count(p.mech); ++i)
     if (!rel[i] || !drel[i]) return RELPOS_ERR_INVALID_ARG;
+  if ((e = check_seqlens(params))) return e;
   const bool tc = use_tc(params, p, 1);
   if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
   const Layout l = layout_of(p, 1, tc);

@@ -51,7 +51,16 @@ struct Prm {
   float *part_diag;    // Transformer-XL per-diagonal-shard partials
   float *gtot;         // Transformer-XL [H][n_off] diagonal sums of dS
   int *status;
+  const int *seqlens_k;  // [B] key lengths (device), or null: every batch has L keys
+  int klen;              // this CTA's key length (set by kernels that mask keys)
 };
+
+// Key length of batch b: keys j >= key_len are masked (variable-length batches).
+__device__ __forceinline__ int key_len(const Prm &p, int b) {
+  if (!p.seqlens_k) return p.L;
+  const int v = p.seqlens_k[b];
+  return v < 0 ? 0 : (v > p.L ? p.L : v);
+}
 
 // ---------------------------------------------------------------------------
 // element access

@@ -240,7 +240,7 @@ __device__ __forceinline__ void scores(const Prm &p, const Sm &sm, int h, int i0
       const int i = i0 + r, j = j0 + c;
       float s = S[a][b] * p.scale;
       if (MECH == M_T5) s += sm.aux[A_BIAS + (j - i) - dmin];
-      if (i >= p.L || j >= p.L || (p.causal && j > i)) s = -INFINITY;
+      if (i >= p.L || j >= p.klen || (p.causal && j > i)) s = -INFINITY;
       S[a][b] = s;
     }
 }
@@ -250,6 +250,7 @@ __device__ __forceinline__ void scores(const Prm &p, const Sm &sm, int h, int i0
 // ---------------------------------------------------------------------------
 template <int MECH, class T>
 __global__ void __launch_bounds__(NT, 1) fwd_kernel(Prm p) {
+  p.klen = key_len(p, blockIdx.z);
   extern __shared__ float smem[];
   const Sm sm = carve(smem);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -367,7 +368,7 @@ __device__ __forceinline__ void scatter_E(const Prm &p, const float (&dS)[4][4],
     for (int b = 0; b < 4; ++b) {
       const int r = TRANS ? tx + 16 * b : x, c = TRANS ? x : tx + 16 * b;
       const int i = i0 + r, j = j0 + c;
-      if (i >= p.L || j >= p.L || (p.causal && j > i)) continue;
+      if (i >= p.L || j >= p.klen || (p.causal && j > i)) continue;
       const int rho = COLSIDE ? rho_col(p, j - i) : rho_row<MECH>(p, j - i);
       if (has_ends<MECH>() && rho == 0)
         e0 += dS[a][b];
@@ -418,6 +419,7 @@ __global__ void __launch_bounds__(256) dvec_kernel(Prm p) {
 // ---------------------------------------------------------------------------
 template <int MECH, class T>
 __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
+  p.klen = key_len(p, blockIdx.z);
   extern __shared__ float smem[];
   const Sm sm = carve(smem);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -541,6 +543,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
 // ---------------------------------------------------------------------------
 template <int MECH, class T>
 __global__ void __launch_bounds__(NT, 1) bwd_kv_kernel(Prm p) {
+  p.klen = key_len(p, blockIdx.z);
   extern __shared__ float smem[];
   const Sm sm = carve(smem);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -660,6 +663,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_kv_kernel(Prm p) {
 // ---------------------------------------------------------------------------
 template <class T>
 __global__ void __launch_bounds__(NT, 1) bwd_diag_kernel(Prm p) {
+  p.klen = key_len(p, blockIdx.z / p.H);
   extern __shared__ float smem[];
   const Sm sm = carve(smem);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;

@@ -131,6 +131,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
   const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, j0 = n * 128;
   const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
+  const int klen = key_len(p, bh / p.H);  // keys j >= klen of this batch are masked
+  if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0, no du contribution (whole CTA, no barrier yet)
+    for (int x = tid; x < 128 * (HD / 8); x += NTHREADS) {
+      const int r = x / (HD / 8), c8 = x % (HD / 8);
+      if (j0 + r < L) {
+        const size_t off = ((size_t)bh * L + j0 + r) * HD + 8 * c8;
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dk + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dv + off) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    if (tid < HD) A.part_kv[((size_t)bh * p.nT + n) * HD + tid] = 0.f;
+    return;
+  }
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
@@ -256,7 +269,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
     auto fetch1 = [&](int t) {
       const int m = mStart + t, D = m - n, r = tid & 127, w = tid >> 7;
       const int i = m * 128 + r, ro = 128 * (w == 2 ? D : D - 1) + r + p.off;
-      if (w == 0) return (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      if (w == 0) return lse2_of(p, bh, i);
       if (w == 1) return (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
       return (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
     };
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
       // P and dS of this thread's NC keys, packed to bf16 pairs as they are made
       uint32_t pk[NC / 2], dk[NC / 2];
-      const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
+      const bool need_mask = (p.causal && m == n) || (j0 + 128 > klen);
       if (good) {
         tc_fence_after();
         const float lse2 = tv[il], Dv = tv[128 + il];
@@ -307,7 +320,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int j = j0 + cb + x0 + e;
-                  if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+                  if (j >= klen || (p.causal && j > i)) y[e] = -INFINITY;
                 }
               }
 #pragma unroll
@@ -418,7 +431,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
   const int BH = p.B * p.H;
   const int bh = (int)blockIdx.x % BH, m = p.nT - 1 - (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, i0 = m * 128;
-  const int nTiles = p.causal ? m + 1 : p.nT;
+  const int klen = key_len(p, bh / p.H);  // keys j >= klen of this batch are masked; their tiles skipped
+  const int nTiles = min(p.causal ? m + 1 : p.nT, (klen + 127) / 128);
+  if (nTiles == 0) {  // no key at all: dQ = 0 (whole CTA, before any barrier)
+    for (int x = tid; x < 128 * (HD / 8); x += NTHREADS) {
+      const int r = x / (HD / 8), c8 = x % (HD / 8);
+      if (i0 + r < L)
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dq + ((size_t)bh * L + i0 + r) * HD + 8 * c8) = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
@@ -542,7 +564,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     const int i = i0 + il;
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     float *rrow = rot + il * ROT_LD;
-    const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+    const float lse2 = lse2_of(p, bh, i);
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
     const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
     bool good = true;
@@ -585,7 +607,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         for (int e = 0; e < NC; ++e) x[e] = 0.f;
       }
       named_bar_sync(1, NSOFT);
-      const bool need_mask = (p.causal && n == m) || (j0 + 128 > L);
+      const bool need_mask = (p.causal && n == m) || (j0 + 128 > klen);
       auto probs = [&](auto masked) {  // x <- P = 2^(s c1 + r' + u' - lse2)
 #pragma unroll
         for (int c4 = 0; c4 < NC / 4; ++c4) {
@@ -599,7 +621,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = j0 + cb + 4 * c4 + e;
-              if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+              if (j >= klen || (p.causal && j > i)) y[e] = -INFINITY;
             }
           }
 #pragma unroll
@@ -701,8 +723,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
   const int band = p.causal ? D : D + (p.nT - 1);
   const int b = bh / p.H, h = bh % p.H;
   const int mlo = max(0, D), mhi = min(p.nT - 1, p.nT - 1 + D);
-  const int m0 = mlo + chunk * A.dg_ch, m1 = min(mhi, m0 + A.dg_ch - 1);
-  if (m0 > m1) return;  // whole CTA, before any barrier or TMEM allocation
+  const int m0 = mlo + chunk * A.dg_ch, m1a = min(mhi, m0 + A.dg_ch - 1);
+  if (m0 > m1a) return;  // no such chunk (never read): whole CTA, before any barrier or TMEM allocation
+  // keys j >= klen of this batch are masked: tiles whose key tile m - D lies past them are skipped
+  const int klen = key_len(p, bh / p.H);
+  const int m1 = min(m1a, (klen + 127) / 128 - 1 + D);
+  if (m0 > m1) {  // the chunk's tiles are all padding: a zero partial
+    float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
+    for (int x = tid; x < DG_STRIDE; x += NTHREADS) part[x] = 0.f;
+    return;
+  }
   const int iters = m1 - m0 + 1;
   const int L = p.L;
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
@@ -833,7 +863,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
     }
     auto fetch1 = [&](int t) {
       const int m = m0 + t, r = tid & 127, w = tid >> 7, i = m * 128 + r, j = (m - D) * 128 + r;
-      if (w == 0) return (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+      if (w == 0) return lse2_of(p, bh, i);
       if (w == 1) return (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
       return (j < L) ? A.uk[(size_t)bh * L + j] * c1 : 0.f;
     };
@@ -859,7 +889,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
       uint32_t ds[NC / 2];  // dS as bf16 pairs (x[2k+1] low, x[2k] high)
-      const bool need_mask = (p.causal && m == nn) || (j0 + 128 > L);
+      const bool need_mask = (p.causal && m == nn) || (j0 + 128 > klen);
       if (good) {
         tc_fence_after();
         const float lse2 = tv[il], Dv = tv[128 + il];
@@ -882,7 +912,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int j = j0 + cb + x0 + e;
-                  if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+                  if (j >= klen || (p.causal && j > i)) y[e] = -INFINITY;
                 }
               }
 #pragma unroll

@@ -42,6 +42,14 @@ __device__ __forceinline__ void ds_pairs(const float (&pr)[4], const uint32_t *d
   f2_split(mul2(f2(pr[2], pr[3]), add2(f2(u2f(dp[2]), u2f(dp[3])), nDv)), dd[2], dd[3]);
 }
 
+// log2-domain LSE of query row i for P = 2^(y - lse2): rows past L and rows with no
+// key (LSE = -inf) give +inf, i.e. P = 0
+__device__ __forceinline__ float lse2_of(const Prm &p, int bh, int i) {
+  if (i >= p.L) return INFINITY;
+  const float l = p.lse[(size_t)bh * p.L + i];
+  return l == -INFINITY ? INFINITY : l * LOG2E;
+}
+
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *ab, int32_t *st) {
   const bool ok = mbar_wait(bar, parity, ab, st, RELPOS_ERR_TIMEOUT_DEV);
   return __all_sync(0xffffffffu, ok);

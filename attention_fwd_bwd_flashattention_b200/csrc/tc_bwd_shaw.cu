@@ -111,6 +111,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
   const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH;
   const int L = p.L, j0 = n * 128, cl = p.clip;
   const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
+  const int klen = key_len(p, bh / p.H);  // keys j >= klen of this batch are masked
+  if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0 (whole CTA, no barrier yet)
+    for (int x = tid; x < 128 * (HD / 8); x += NTHREADS) {
+      const int r = x / (HD / 8), c8 = x % (HD / 8);
+      if (j0 + r < L) {
+        const size_t off = ((size_t)bh * L + j0 + r) * HD + 8 * c8;
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dk + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dv + off) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    return;
+  }
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
@@ -219,7 +231,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
     auto fetch1 = [&](int t) {
       const int m = mStart + t, r = tid & 127, w = tid >> 7, i = m * 128 + r;
       if (i >= L) return w == 0 ? INFINITY : 0.f;
-      if (w == 0) return p.lse[(size_t)bh * L + i] * LOG2E;
+      if (w == 0) return lse2_of(p, bh, i);
       if (w == 1) return p.Dvec[(size_t)bh * L + i];
       return A.qa[((size_t)bh * L + i) * QA_LD + (m > n ? 0 : 2 * cl)];
     };
@@ -236,7 +248,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
         ++qa_cnt;
       }
       uint32_t pk[NC / 2], dk[NC / 2];
-      const bool need_mask = (p.causal && m == n) || (j0 + 128 > L);
+      const bool need_mask = (p.causal && m == n) || (j0 + 128 > klen);
       const int d0 = j0 + cb - i;  // offset j - i of this thread's first key
       if (good) {
         tc_fence_after();
@@ -261,7 +273,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int j = j0 + cb + x0 + e;
-                  if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+                  if (j >= klen || (p.causal && j > i)) y[e] = -INFINITY;
                 }
               }
 #pragma unroll
@@ -389,7 +401,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
   const int BH = p.B * p.H;
   const int bh = (int)blockIdx.x % BH, m = p.nT - 1 - (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, i0 = m * 128, cl = p.clip;
-  const int nTiles = p.causal ? m + 1 : p.nT;
+  const int klen = key_len(p, bh / p.H);  // keys j >= klen of this batch are masked; their tiles skipped
+  const int nTiles = min(p.causal ? m + 1 : p.nT, (klen + 127) / 128);
+  if (nTiles == 0) {  // no key at all: dQ = 0 and a zero da partial (whole CTA, before any barrier)
+    for (int x = tid; x < 128 * (HD / 8); x += NTHREADS) {
+      const int r = x / (HD / 8), c8 = x % (HD / 8);
+      if (i0 + r < L)
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dq + ((size_t)bh * L + i0 + r) * HD + 8 * c8) = make_uint4(0, 0, 0, 0);
+    }
+    float *part = A.part + ((size_t)bh * p.nT + m) * (size_t)p.nrows * HD;
+    for (int x = tid; x < p.nrows * HD; x += NTHREADS) part[x] = 0.f;
+    return;
+  }
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
@@ -490,7 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
     const int i = i0 + il;
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     const float *rrow = rot + il * QA_LD;
-    const float lse2 = (i < L) ? p.lse[(size_t)bh * L + i] * LOG2E : INFINITY;
+    const float lse2 = lse2_of(p, bh, i);
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
     const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
     bool good = warp_wait(BAR(B_QD), 0, abort_flag, status);
@@ -500,7 +523,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
       const int j0 = n * 128;
       const bool band = band_tile(cl, m, n);
       good = good && warp_wait(BAR(B_SDP), n & 1, abort_flag, status);
-      const bool need_mask = (p.causal && n == m) || (j0 + 128 > L);
+      const bool need_mask = (p.causal && n == m) || (j0 + 128 > klen);
       const int d0 = j0 + cb - i;  // offset j - i of this thread's first key
       float x[NC];
       if (good) {
@@ -525,7 +548,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int j = j0 + cb + x0 + e;
-                  if (j >= L || (p.causal && j > i)) y[e] = -INFINITY;
+                  if (j >= klen || (p.causal && j > i)) y[e] = -INFINITY;
                 }
               }
 #pragma unroll

@@ -97,7 +97,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const int bh = (int)blockIdx.x % BH, m = p.nT - 1 - (int)blockIdx.x / BH;
   const int h = bh % p.H;
   const int L = p.L, i0 = m * BM;
-  const int nTiles = p.causal ? m + 1 : p.nT;
+  // keys j >= klen of this batch are masked; key tiles past them are skipped
+  const int klen = key_len(p, bh / p.H);
+  const int nTiles = min(p.causal ? m + 1 : p.nT, (klen + BN - 1) / BN);
+  if (nTiles == 0) {  // no key at all: O = 0, LSE = -inf (whole CTA, before any barrier)
+    for (int x = tid; x < BM * (HD / 8); x += NTHREADS) {
+      const int r = x / (HD / 8), c8 = x % (HD / 8);
+      if (i0 + r < L)
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.out + ((size_t)bh * L + i0 + r) * HD + 8 * c8) = make_uint4(0, 0, 0, 0);
+    }
+    if (tid < BM && i0 + tid < L) p.lse[(size_t)bh * L + i0 + tid] = -INFINITY;
+    return;
+  }
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -460,13 +471,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
       }
       // ---- mask (diagonal / ragged tiles only), row max over the row's threads ----
-      const bool need_mask = (p.causal && n == m) || (j0 + BN > L);
+      const bool need_mask = (p.causal && n == m) || (j0 + BN > klen);
       float mt = -INFINITY;
       if (need_mask) {
 #pragma unroll
         for (int t = 0; t < NC; ++t) {
           const int j = j0 + cb + t;
-          if (j >= L || (p.causal && j > i)) x[t] = -INFINITY;
+          if (j >= klen || (p.causal && j > i)) x[t] = -INFINITY;
           mt = fmaxf(mt, x[t]);
         }
       } else {

@@ -107,6 +107,15 @@ typedef struct relpos_params {
   int32_t t5_bidirectional;  /* T5: 1 bidirectional, 0 unidirectional             */
   int32_t shaw_clip;         /* Shaw: clip distance c (table rows 2c + 1)         */
   int32_t deberta_span;      /* DeBERTa: relative span k (table rows 2k)          */
+  /* Variable-length batches (optional; NULL = every batch has L keys): DEVICE
+   * pointer to B int32 key lengths.  Keys j >= seqlens_k[b] of batch b are masked
+   * (after causal masking); all L queries are computed and relative positions keep
+   * their meaning over the padded length.  Values are clamped to [0, L].  A query
+   * with no unmasked key gets O = 0, LSE = -inf and zero gradients; masked keys get
+   * dK = dV = 0.  The array is read by the kernels of the call (stream order) and
+   * must stay valid until they finish.  Variable-length speech batches: article
+   * "结构感知内核让相对位置注意力加速21倍", section "为什么相对位置注意力难做快". */
+  const int32_t *seqlens_k;
 } relpos_params_t;
 
 /* Bytes of device workspace a call needs.  pass: 0 forward, 1 backward.

@@ -22,10 +22,13 @@ def params_of(wl, path):
                      t5_max_distance=wl.t5_max_distance, t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
 
 
-def run_gpu(wl, inp, path, dev="cuda"):
+def run_gpu(wl, inp, path, dev="cuda", seqlens_k=None):
     """Forward + backward through the C ABI; the device status word must stay 0 (a
-    bounded wait that ran out inside a kernel reports RELPOS_ERR_TIMEOUT there)."""
+    bounded wait that ran out inside a kernel reports RELPOS_ERR_TIMEOUT there).
+    seqlens_k: optional per-batch key lengths (a sequence of B ints)."""
     P = params_of(wl, path)
+    if seqlens_k is not None:
+        P.seqlens_k = torch.tensor(list(seqlens_k), dtype=torch.int32, device=dev)
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
     rel = [r.to(dev) for r in inp["rel"]]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -41,7 +44,14 @@ def run_gpu(wl, inp, path, dev="cuda"):
 
 
 def maxabs(got, want):
-    return float(np.max(np.abs(got - want))) if want.size else 0.0
+    """Largest |got - want|; entries where both are the same infinity (LSE = -inf of
+    a query without keys) count as equal, an infinity on one side only as inf."""
+    if not want.size:
+        return 0.0
+    same_inf = np.isinf(want) & (got == want)
+    with np.errstate(invalid="ignore"):  # inf - inf where same_inf; masked out below
+        diff = np.abs(got - want)
+    return float(np.max(np.where(same_inf, 0.0, diff)))
 
 
 def rel_l2(got, want):
@@ -59,7 +69,7 @@ def f64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def compare_full(wl, inp, out, heads=None):
+def compare_full(wl, inp, out, heads=None, seqlens_k=None):
     """Compare every output with the oracle (optionally only some heads; table
     gradients then cover those heads, which is exact when B == 1)."""
     tol = TOL[wl.dtype]
@@ -70,8 +80,8 @@ def compare_full(wl, inp, out, heads=None):
     if heads is not None:
         q, k, v, do = q[:, hs], k[:, hs], v[:, hs], do[:, hs]
         rel = [r[hs] for r in rel]
-    O, LSE = orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg)
-    dq, dk, dv, drel = orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg)
+    O, LSE = orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, seqlens_k=seqlens_k)
+    dq, dk, dv, drel = orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg, seqlens_k=seqlens_k)
     errs = {
         "o": maxabs(f64(out["o"][:, hs]), O),
         "lse": maxabs(f64(out["lse"][:, hs]), LSE),

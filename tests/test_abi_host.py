@@ -44,17 +44,19 @@ def test_struct_layout_matches_c(tmp_path):
     prog = tmp_path / "layout.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "relpos_attn.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
-        " offsetof(relpos_params_t,scale), offsetof(relpos_params_t,t5_num_buckets), offsetof(relpos_params_t,deberta_span));return 0;}\n")
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
+        " offsetof(relpos_params_t,scale), offsetof(relpos_params_t,t5_num_buckets), offsetof(relpos_params_t,deberta_span),"
+        " offsetof(relpos_params_t,seqlens_k));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(prog), "-o", str(exe)], check=True)
     got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     S = bd.relpos_params_t
-    assert got == [ctypes.sizeof(S), S.B.offset, S.scale.offset, S.t5_num_buckets.offset, S.deberta_span.offset]
+    assert got == [ctypes.sizeof(S), S.B.offset, S.scale.offset, S.t5_num_buckets.offset, S.deberta_span.offset,
+                   S.seqlens_k.offset]
 
 
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10000
+    assert lib.relpos_attn_version() == 10100
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"

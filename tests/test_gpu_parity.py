@@ -69,6 +69,46 @@ def test_parity_shaw_clip(clip, causal, L):
     compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
 
 
+@pytest.mark.parametrize("path", [bd.PATH_SIMT, bd.PATH_AUTO], ids=["simt", "auto"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("mech", list(MECHS))
+@pytest.mark.parametrize("L,lens", [(300, (300, 171, 0)), (700, (129, 700, 384))])
+def test_parity_key_lengths(mech, causal, L, lens, path):
+    """Variable-length batches: per-batch key lengths inside a tile, on a tile
+    boundary, the full length and an empty key set (O = 0, LSE = -inf)."""
+    wl = small_wl(mech, torch.bfloat16, causal, L, B=len(lens))
+    inp = make_inputs(wl, seed=L + 3)
+    compare_full(wl, inp, run_gpu(wl, inp, path, seqlens_k=lens), seqlens_k=lens)
+
+
+def test_key_lengths_on_the_host_are_rejected():
+    wl = small_wl("txl", torch.bfloat16, False, 64, B=2)
+    P = bd.Params(mech=TXL, B=2, H=2, L=64, seqlens_k=torch.tensor([64, 3], dtype=torch.int32))
+    q = torch.zeros(2, 2, 64, 64, dtype=torch.bfloat16, device="cuda")
+    rel = [torch.zeros(2, 127, 64, dtype=torch.bfloat16, device="cuda"), torch.zeros(2, 64, dtype=torch.bfloat16, device="cuda"),
+           torch.zeros(2, 64, dtype=torch.bfloat16, device="cuda")]
+    with pytest.raises(bd.RelposError) as ei:
+        bd.forward(P, q, q, q, rel)
+    assert ei.value.code == -1
+
+
+def test_key_lengths_match_truncated_keys():
+    """A batch whose keys stop at Lk gives the same O and LSE as the same keys with
+    everything after Lk replaced (T5 and Shaw depend only on j - i)."""
+    wl = small_wl("shaw", torch.bfloat16, False, 520, B=2)
+    inp = make_inputs(wl, seed=9)
+    lens = (333, 520)
+    a = run_gpu(wl, inp, bd.PATH_AUTO, seqlens_k=lens)
+    inp2 = dict(inp)
+    for n in ("k", "v"):
+        t = inp[n].clone()
+        t[0, :, 333:] = torch.randn(t[0, :, 333:].shape, generator=torch.Generator().manual_seed(1)).to(t.dtype)
+        inp2[n] = t
+    b = run_gpu(wl, inp2, bd.PATH_AUTO, seqlens_k=lens)
+    assert torch.equal(a["o"], b["o"]) and torch.equal(a["lse"], b["lse"]) and torch.equal(a["dq"], b["dq"])
+    assert torch.all(b["dk"][0, :, 333:] == 0) and torch.all(b["dv"][0, :, 333:] == 0)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_parity_t5_unidirectional_and_odd_buckets(causal):
     for nb, md, bidir in ((32, 128, False), (10, 40, True), (7, 20, False)):
