@@ -30,7 +30,16 @@ original papers, because the pages print none of their formulas:
                                           + k_j.Qr[h, clip(j - i + k, 0, 2k-1)])
 
 with s the caller's scale (1/sqrt(d) for the first three, 1/sqrt(3d) for DeBERTa
-by default).  Transformer-XL rows: row(delta) = delta when causal (delta in [0, L)),
+by default).  ALiBi, the further bias named by the article (section "工程权衡与适用边界",
+in its list of models the method suits), is written from its own
+paper (Press et al., "Train Short, Test Long"):
+
+  ALiBi                        S_ij = s q_i.k_j - m[h] |j - i|
+
+a fixed per-head slope m[h] times the distance, added unscaled (the causal model of
+that paper sees only j <= i, so -m (i - j); without a causal mask the symmetric
+distance is the plain reading).  The slopes are the caller's input; their gradient
+sum_ij dS_ij (-|j - i|) is returned like a table gradient.  Transformer-XL rows: row(delta) = delta when causal (delta in [0, L)),
 delta + L - 1 otherwise (delta in (-L, L)).  Causal masking removes j > i.
 
 Backward (textbook softmax chain rule):
@@ -66,8 +75,8 @@ from dataclasses import dataclass
 
 import numpy as np
 
-T5, SHAW, TXL, DEBERTA = 0, 1, 2, 3
-MECH_NAMES = {T5: "t5", SHAW: "shaw", TXL: "txl", DEBERTA: "deberta"}
+T5, SHAW, TXL, DEBERTA, ALIBI = 0, 1, 2, 3, 4
+MECH_NAMES = {T5: "t5", SHAW: "shaw", TXL: "txl", DEBERTA: "deberta", ALIBI: "alibi"}
 
 
 @dataclass(frozen=True)
@@ -88,7 +97,9 @@ def default_scale(mech: int, d: int) -> float:
 
 
 def table_rows(mech: int, L: int, causal: bool, cfg: RelCfg) -> int:
-    """Number of rows of the relative table of each head."""
+    """Number of rows of the relative table of each head (ALiBi: one slope)."""
+    if mech == ALIBI:
+        return 1
     if mech == T5:
         return cfg.t5_num_buckets
     if mech == SHAW:
@@ -201,6 +212,9 @@ def head_bias(mech, q, k, rel_h, scale, cfg, causal, rows_i):
     """
     L = k.shape[0]
     qi = q[rows_i]
+    if mech == ALIBI:
+        (m,) = rel_h
+        return -float(m) * np.abs(_rel(rows_i, L)).astype(np.float64)
     if mech == T5:
         (t,) = rel_h
         return t[index_map(T5, L, causal, cfg, rows_i)]
@@ -261,7 +275,7 @@ def forward(mech, q, k, v, rel, causal, scale=None, cfg=RelCfg(), rows=None, seq
 
     q, k, v: [B, H, L, d]; rel: list of per-head tables (see module docstring):
     T5 [t (H,nb)], Shaw [a (H,2c+1,d)], TXL [r (H,n_off,d), u (H,d), v (H,d)],
-    DeBERTa [Kr (H,2k,d), Qr (H,2k,d)].
+    DeBERTa [Kr (H,2k,d), Qr (H,2k,d)], ALiBi [m (H,)].
     """
     q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
     B, H, L, d = q.shape
@@ -283,7 +297,8 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg(), seqlens_k
     """Exact gradients (dq, dk, dv, drel) of  sum(O * dO).
 
     drel matches rel's structure: T5 [dt], Shaw [da], TXL [dr, du, dv],
-    DeBERTa [dKr, dQr]; table gradients sum over the batch (tables are per head).
+    DeBERTa [dKr, dQr], ALiBi [dm]; table gradients sum over the batch (tables
+    are per head).
     """
     q, k, v, dO = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dO))
     B, H, L, d = q.shape
@@ -305,7 +320,9 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg(), seqlens_k
             # content term scale * q_i . k_j
             dq[b, h] = scale * (dS @ kh)
             dk[b, h] = scale * (dS.T @ qh)
-            if mech == T5:
+            if mech == ALIBI:
+                drel[0][h] += np.sum(dS * -np.abs(_rel(rows_i, L)))
+            elif mech == T5:
                 idx = index_map(T5, L, causal, cfg, rows_i)
                 np.add.at(drel[0][h], idx.ravel(), dS.ravel())
             elif mech == SHAW:

@@ -5,7 +5,7 @@
   forward and scalar chain-rule backward, on tiny shapes with small clip /
   span / bucket parameters so that clipping and bucketing are exercised,
 * central finite differences of sum(O * dO) for every input and parameter,
-* closed forms (L = 1; causal row 0),
+* closed forms (L = 1; causal row 0; ALiBi with q.k = 0: geometric sums),
 * zero relative term == plain softmax attention, checked against
   torch.nn.functional.scaled_dot_product_attention (fp64, CPU) and autograd,
 * row-constant terms leave O unchanged and shift LSE; the gradient of every
@@ -19,7 +19,7 @@ import pytest
 import torch
 
 import oracle as orc
-from oracle import DEBERTA, SHAW, T5, TXL, RelCfg
+from oracle import ALIBI, DEBERTA, SHAW, T5, TXL, RelCfg
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 SMALL = RelCfg(t5_num_buckets=8, t5_max_distance=6, t5_bidirectional=True, shaw_clip=2, deberta_span=2)
@@ -34,7 +34,9 @@ def make_case(mech, B, H, L, d, causal, cfg, seed=0, zero_rel=False):
     q, k, v, do = (rnd(rng, B, H, L, d) for _ in range(4))
     nrows = orc.table_rows(mech, L, causal, cfg)
     sc = 0.0 if zero_rel else 1.0
-    if mech == T5:
+    if mech == ALIBI:
+        rel = [sc * (0.05 + np.abs(rnd(rng, H, std=0.5)))]
+    elif mech == T5:
         rel = [sc * rnd(rng, H, nrows, std=0.5)]
     elif mech == SHAW:
         rel = [sc * rnd(rng, H, nrows, d, std=0.5)]
@@ -102,6 +104,8 @@ def dot(x, y):
 
 def bf_score(mech, q, k, rel, h, i, j, L, causal, s, cfg):
     """S_ij straight from the mechanism's formula."""
+    if mech == ALIBI:
+        return s * dot(q[i], k[j]) - rel[0][h] * abs(j - i)
     if mech == T5:
         return s * dot(q[i], k[j]) + rel[0][h][bf_bucket(j - i, cfg)]
     if mech == SHAW:
@@ -151,7 +155,9 @@ def brute(mech, q, k, v, rel, causal, do, s, cfg, lk=None):
                     dv[b, h, j] += P[i, j] * gb[i]
                     dq[b, h, i] += s * dS * kb[j]
                     dk[b, h, j] += s * dS * qb[i]
-                    if mech == T5:
+                    if mech == ALIBI:
+                        drel[0][h] += dS * -abs(j - i)
+                    elif mech == T5:
                         drel[0][h][bf_bucket(j - i, cfg)] += dS
                     elif mech == SHAW:
                         c = cfg.shaw_clip
@@ -177,7 +183,8 @@ def brute(mech, q, k, v, rel, causal, do, s, cfg, lk=None):
     return O, LSE, dq, dk, dv, drel
 
 
-CASES = [(mech, causal, L, d) for mech in (T5, SHAW, TXL, DEBERTA) for causal in (False, True)
+MECHS = (T5, SHAW, TXL, DEBERTA, ALIBI)
+CASES = [(mech, causal, L, d) for mech in MECHS for causal in (False, True)
          for (L, d) in ((1, 2), (2, 1), (3, 4), (5, 2), (8, 4))]
 
 
@@ -199,7 +206,7 @@ def test_oracle_vs_brute_force(mech, causal, L, d):
     np.testing.assert_allclose(dq2, dq[:, :, rows], rtol=1e-12, atol=1e-12)
 
 
-SEQ_CASES = [(mech, causal, L, lk) for mech in (T5, SHAW, TXL, DEBERTA) for causal in (False, True)
+SEQ_CASES = [(mech, causal, L, lk) for mech in MECHS for causal in (False, True)
              for (L, lk) in ((3, (2, 0)), (5, (5, 1)), (8, (3, 7)))]
 
 
@@ -221,7 +228,7 @@ def test_oracle_key_lengths_vs_brute_force(mech, causal, L, lk):
     np.testing.assert_allclose(dq2, dq[:, :, rows], rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("mech", [T5, SHAW, TXL, DEBERTA])
+@pytest.mark.parametrize("mech", MECHS)
 def test_padding_keys_do_not_matter(mech):
     """Keys past a batch's length change nothing but get zero dk, dv; an empty key
     set gives O = 0, LSE = -inf and zero gradients; a full length is no mask."""
@@ -255,7 +262,7 @@ def test_padding_keys_do_not_matter(mech):
 # ----------------------------------------------------------------------------
 # finite differences
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("mech", [T5, SHAW, TXL, DEBERTA])
+@pytest.mark.parametrize("mech", MECHS)
 @pytest.mark.parametrize("causal", [False, True])
 def test_oracle_finite_differences(mech, causal):
     L, d = 13, 4
@@ -291,7 +298,7 @@ def test_oracle_finite_differences(mech, causal):
 # ----------------------------------------------------------------------------
 # closed forms
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("mech", [T5, SHAW, TXL, DEBERTA])
+@pytest.mark.parametrize("mech", MECHS)
 def test_closed_form_L1(mech):
     q, k, v, do, rel = make_case(mech, 1, 3, 1, 8, False, RelCfg(), seed=3)
     s = orc.default_scale(mech, 8)
@@ -305,17 +312,42 @@ def test_closed_form_L1(mech):
         np.testing.assert_allclose(g, 0.0, atol=1e-13)
 
 
-@pytest.mark.parametrize("mech", [T5, SHAW, TXL, DEBERTA])
+@pytest.mark.parametrize("mech", MECHS)
 def test_closed_form_causal_row0(mech):
     q, k, v, do, rel = make_case(mech, 1, 2, 6, 4, True, SMALL, seed=5)
     O, _ = orc.forward(mech, q, k, v, rel, True, 0.5, SMALL)
     np.testing.assert_allclose(O[:, :, 0], v[:, :, 0], atol=1e-15)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_alibi_geometric_closed_form(causal):
+    """q = 0 leaves only the ALiBi term: row i's softmax weights are e^{-m |j - i|},
+    so LSE_i = ln(sum_{t=0}^{i} e^{-m t} + [not causal] sum_{t=1}^{L-1-i} e^{-m t})
+    (geometric sums), and with v_j = e^{-m j} (causal) every key contributes
+    e^{-m i} / Z_i, so O_i = (i + 1) e^{-m i} / Z_i."""
+    L, H = 50, 3
+    m = np.array([0.03, 0.5, 2.0])
+    q = np.zeros((1, H, L, 1))
+    k = np.random.default_rng(2).standard_normal((1, H, L, 1))
+    j = np.arange(L, dtype=np.float64)
+    v = np.broadcast_to(np.exp(-m[:, None] * j[None, :])[None, :, :, None], (1, H, L, 1)).copy()
+    O, LSE = orc.forward(ALIBI, q, k, v, [m], causal, 1.0)
+
+    def geo(n, mm):  # sum_{t=0}^{n-1} e^{-mm t}
+        return (1.0 - np.exp(-mm * n)) / (1.0 - np.exp(-mm))
+
+    for h in range(H):
+        i = np.arange(L)
+        Z = geo(i + 1, m[h]) + (0.0 if causal else geo(L - i, m[h]) - 1.0)
+        np.testing.assert_allclose(LSE[0, h], np.log(Z), rtol=1e-13, atol=1e-13)
+        if causal:
+            np.testing.assert_allclose(O[0, h, :, 0], (i + 1) * np.exp(-m[h] * i) / Z, rtol=1e-12)
+
+
 # ----------------------------------------------------------------------------
 # zero relative term == plain attention (independent library routine)
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("mech", [T5, SHAW, TXL, DEBERTA])
+@pytest.mark.parametrize("mech", MECHS)
 @pytest.mark.parametrize("causal", [False, True])
 def test_zero_term_is_plain_attention(mech, causal):
     L, d = 37, 16
@@ -387,7 +419,7 @@ def test_batch_sums_table_grads():
     """Per-head tables are shared across the batch: their gradient with B = 2 is
     the sum of the two single-batch gradients."""
     cfg = RelCfg(shaw_clip=3, deberta_span=3)
-    for mech in (T5, SHAW, TXL, DEBERTA):
+    for mech in MECHS:
         q, k, v, do, rel = make_case(mech, 2, 2, 9, 4, False, cfg, seed=31)
         _, _, _, dr = orc.backward(mech, q, k, v, rel, False, do, 0.5, cfg)
         parts = [orc.backward(mech, q[b:b + 1], k[b:b + 1], v[b:b + 1], rel, False, do[b:b + 1], 0.5, cfg)[3] for b in range(2)]
