@@ -8,7 +8,9 @@ fixed order, so a seed gives the same values on every machine.
 Distributions (per the workload definitions): Q, K, V, dO ~ N(0, 1); T5 bias
 table t[H, 32] ~ N(0, 0.1); Shaw table a[H, 129, d] ~ N(0, 0.02); DeBERTa Kr,
 Qr [H, 512, d] ~ N(0, 0.02); Transformer-XL u, v [H, d] ~ N(0, 0.02) and
-r = sinusoid(offset) [n_off, 512] @ W_R [512, H*d] with W_R ~ N(0, 0.02).
+r = sinusoid(offset) [n_off, 512] @ W_R [512, H*d] with W_R ~ N(0, 0.02);
+ALiBi slopes m[h] = 2^(-8 (h + 1) / H), the geometric sequence of the ALiBi paper
+(Press et al.) for its heads (fixed, not drawn).
 The sinusoid is the Transformer-XL one: [sin(delta w_k), cos(delta w_k)]
 concatenated, w_k = 10000^(-2k/512), k = 0..255.
 """
@@ -16,11 +18,12 @@ from __future__ import annotations
 
 import math
 from dataclasses import dataclass
+from typing import Optional, Tuple
 
 import torch
 
-T5, SHAW, TXL, DEBERTA = 0, 1, 2, 3
-MECH_IDS = {"t5": T5, "shaw": SHAW, "txl": TXL, "deberta": DEBERTA}
+T5, SHAW, TXL, DEBERTA, ALIBI = 0, 1, 2, 3, 4
+MECH_IDS = {"t5": T5, "shaw": SHAW, "txl": TXL, "deberta": DEBERTA, "alibi": ALIBI}
 MECH_NAMES = {v: k for k, v in MECH_IDS.items()}
 
 TXL_EMB = 512  # width of the Transformer-XL sinusoid fed to W_R
@@ -41,6 +44,7 @@ class Workload:
     t5_bidirectional: bool = True
     shaw_clip: int = 64
     deberta_span: int = 256
+    seqlens_k: Optional[Tuple[int, ...]] = None  # per-batch key lengths (variable-length batch)
 
     @property
     def scale(self) -> float:
@@ -62,6 +66,14 @@ WORKLOADS = {
 }
 for _L in (4096, 8192, 16384, 32768):
     WORKLOADS[f"txl_L{_L}_bf16"] = Workload(f"txl_L{_L}_bf16", TXL, torch.bfloat16, False, 1, 8, _L)
+# A variable-length batch of the speech-encoder shape (H = 8, d = 64, non-causal): four
+# utterances padded to 8192 frames, key lengths fixed so that runs are comparable.
+WORKLOADS["txl_varlen_B4_L8192_bf16"] = Workload("txl_varlen_B4_L8192_bf16", TXL, torch.bfloat16, False, 4, 8, 8192,
+                                                 seqlens_k=(8192, 6144, 4000, 2500))
+# ALiBi, causal decoder shape at 8K, and T5 at the same size for comparison.
+WORKLOADS["alibi_causal_L8192_bf16"] = Workload("alibi_causal_L8192_bf16", ALIBI, torch.bfloat16, True, 1, 8, 8192)
+WORKLOADS["t5_causal_L8192_bf16"] = Workload("t5_causal_L8192_bf16", T5, torch.bfloat16, True, 1, 8, 8192,
+                                             t5_bidirectional=False)
 
 
 def txl_sinusoid(n_off: int, causal: bool, L: int) -> torch.Tensor:
@@ -80,7 +92,7 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
 
     Returns dict(q, k, v, do, rel) with rel the list of relative parameters:
     T5 [t (H,nb) fp32]; Shaw [a (H,2c+1,d)]; TXL [r (H,n_off,d), u (H,d), v (H,d)];
-    DeBERTa [Kr (H,2k,d), Qr (H,2k,d)].
+    DeBERTa [Kr (H,2k,d), Qr (H,2k,d)]; ALiBi [m (H,) fp32].
     """
     g = torch.Generator(device="cpu").manual_seed(seed)
     B, H, L, d = wl.B, wl.H, wl.L, wl.d
@@ -93,7 +105,9 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
     k = nrm(B, H, L, d).to(dt)
     v = nrm(B, H, L, d).to(dt)
     do = nrm(B, H, L, d).to(dt)
-    if wl.mech == T5:
+    if wl.mech == ALIBI:
+        rel = [torch.pow(2.0, -8.0 * torch.arange(1, H + 1, dtype=torch.float32) / H)]
+    elif wl.mech == T5:
         rel = [nrm(H, wl.t5_num_buckets, std=0.1)]
     elif wl.mech == SHAW:
         rel = [nrm(H, 2 * wl.shaw_clip + 1, d, std=0.02).to(dt)]

@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 
 from attention_fwd_bwd_flashattention_b200 import binding as bd  # noqa: E402
 from attention_fwd_bwd_flashattention_b200 import dist as rdist  # noqa: E402
-from attention_fwd_bwd_flashattention_b200.inputs import DEBERTA, SHAW, T5, TXL, WORKLOADS, make_inputs  # noqa: E402
+from attention_fwd_bwd_flashattention_b200.inputs import ALIBI, DEBERTA, SHAW, T5, TXL, WORKLOADS, make_inputs  # noqa: E402
 
 DEFAULT_WORKLOAD = "txl_causal_L8192_bf16"
 METRIC = "fwd+bwd TFLOP/s and tokens/s at L=8192, % of B200 BF16 tensor peak"
@@ -47,14 +47,24 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # algorithmic FLOPs (distinct products the method must compute; recompute and
 # window duplication are not credited)
 # ----------------------------------------------------------------------------
+def pairs_of(wl):
+    """Unmasked (query, key) pairs of one head, summed over the batch: every query
+    with the keys before its batch's key length (and not after it when causal)."""
+    lens = wl.seqlens_k if wl.seqlens_k is not None else (wl.L,) * wl.B
+    tot = 0
+    for lk in lens:
+        lk = max(0, min(wl.L, lk))
+        tot += lk * (lk + 1) // 2 + (wl.L - lk) * lk if wl.causal else wl.L * lk
+    return tot
+
+
 def algo_flops(wl):
-    pairs = wl.L * (wl.L + 1) // 2 if wl.causal else wl.L * wl.L
-    U = 2.0 * wl.B * wl.H * wl.d * pairs
+    U = 2.0 * wl.H * wl.d * pairs_of(wl)
 
     def R(rows):
         return 2.0 * wl.B * wl.H * wl.L * rows * wl.d
 
-    if wl.mech == T5:
+    if wl.mech in (T5, ALIBI):
         return 2 * U, 5 * U
     if wl.mech == SHAW:
         r = R(2 * wl.shaw_clip + 1)
@@ -66,13 +76,13 @@ def algo_flops(wl):
 
 
 def fa_flops(wl):
-    pairs = wl.L * (wl.L + 1) // 2 if wl.causal else wl.L * wl.L
-    return 4.0 * pairs * wl.d * wl.B * wl.H, 10.0 * pairs * wl.d * wl.B * wl.H
+    pairs = pairs_of(wl)
+    return 4.0 * pairs * wl.d * wl.H, 10.0 * pairs * wl.d * wl.H
 
 
 def kernel_launches(wl, path):
     """Kernels this library launches per forward and per backward call (the dispatch of csrc/api.cu)."""
-    t5 = 1 if wl.mech == T5 else 0  # per-call bucket/bias preparation
+    t5 = 1 if wl.mech in (T5, ALIBI) else 0  # per-call per-offset bias preparation
     tc = path != "simt" and wl.dtype == torch.bfloat16
     if tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
         fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
@@ -83,7 +93,7 @@ def kernel_launches(wl, path):
     elif tc and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction
         bwd = 5
     else:  # D, key-tile, query-tile, then the table-gradient reductions
-        bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2}[wl.mech]
+        bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[wl.mech]
     return fwd, bwd
 
 
@@ -91,10 +101,10 @@ def kernel_launches(wl, path):
 # capture of the same build and workload, summed over the pass's captured kernels; set to
 # None whenever those kernels change.  Source: profiles/tc_kernels_txl_causal_L8192.md.
 DRAM_TRAFFIC = {
-    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (308.63e6, "tc_bwd_kv + tc_bwd_q + tc_bwd_diag + reduce_dr "
+    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (306.78e6, "tc_bwd_kv + tc_bwd_q + tc_bwd_diag + reduce_dr "
                                                    "(the relation prep, D and u/v reduction kernels, about 35 MB "
                                                    "of algorithmic traffic, were not captured)"),
-    ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.20e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
+    ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.22e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
 }
 
 
@@ -186,7 +196,8 @@ def oracle_sample(wl, rows_fraction=None):
     import oracle as orc
     from attention_fwd_bwd_flashattention_b200.inputs import to_f64
 
-    one = wl.with_(B=1, H=1)
+    lk = None if wl.seqlens_k is None else (wl.seqlens_k[0],)
+    one = wl.with_(B=1, H=1, seqlens_k=lk)
     inp = make_inputs(one, 0)
     q, k, v, do = (to_f64(inp[n]) for n in ("q", "k", "v", "do"))
     rel = [to_f64(r) for r in inp["rel"]]
@@ -195,15 +206,15 @@ def oracle_sample(wl, rows_fraction=None):
     f_fwd, f_bwd = algo_flops(one)
     t0 = time.perf_counter()
     if rows_fraction is None:
-        orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg)
-        orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg)
+        orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, seqlens_k=lk)
+        orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg, seqlens_k=lk)
         flops = f_fwd + f_bwd
         sample = f"1 of {wl.B * wl.H} (batch, head) slices at full L={wl.L}, forward + backward"
     else:
         step = max(1, int(round(1 / rows_fraction)))
         rows = np.arange(0, wl.L, step)
-        orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, rows=rows)
-        orc.backward_rows(wl.mech, q, k, v, rel, wl.causal, do, rows, wl.scale, cfg)
+        orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, rows=rows, seqlens_k=lk)
+        orc.backward_rows(wl.mech, q, k, v, rel, wl.causal, do, rows, wl.scale, cfg, seqlens_k=lk)
         flops = (f_fwd + f_bwd) * len(rows) / wl.L
         sample = f"{len(rows)} of {wl.L} query rows of 1 of {wl.B * wl.H} (batch, head) slices: O, LSE and dQ"
     return time.perf_counter() - t0, flops, sample
@@ -227,7 +238,8 @@ def run_reference(args, wl):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "mech": wl.name.split("_")[0], "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d,
-                   "causal": wl.causal, "l2": "n/a (host)"},
+                   "causal": wl.causal, "l2": "n/a (host)",
+                   "seqlens_k": list(wl.seqlens_k) if wl.seqlens_k is not None else None},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -248,6 +260,8 @@ def run_ours(args, wl):
                   dtype=bd.BF16 if wl.dtype == torch.bfloat16 else bd.F32, causal=wl.causal, scale=wl.scale,
                   kernel_path=path, t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance,
                   shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+    if wl.seqlens_k is not None:
+        P.seqlens_k = torch.tensor(wl.seqlens_k, dtype=torch.int32, device=dev)
     inp = make_inputs(wl, seed=rank)
     if rank != 0:  # the relative tables are shared by all ranks (one model)
         inp["rel"] = make_inputs(wl, seed=0)["rel"]
@@ -341,6 +355,7 @@ def run_ours(args, wl):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d, "causal": wl.causal,
+                   "seqlens_k": list(wl.seqlens_k) if wl.seqlens_k is not None else None,
                    "kernel_path": "tcgen05" if tensor_path else "cuda-core fp32",
                    "l2": "flushed before every timed step (256 MB write, untimed)",
                    "parallelism": f"dp{world} (weak; table grads all-reduced)" if world > 1 else "single GPU"},

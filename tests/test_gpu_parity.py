@@ -11,13 +11,14 @@ import torch
 
 import oracle as orc
 from attention_fwd_bwd_flashattention_b200 import binding as bd
-from attention_fwd_bwd_flashattention_b200.inputs import DEBERTA, SHAW, T5, TXL, WORKLOADS, Workload, make_inputs, to_f64
+from attention_fwd_bwd_flashattention_b200.inputs import (ALIBI, DEBERTA, SHAW, T5, TXL, WORKLOADS, Workload, make_inputs,
+                                                           to_f64)
 
 from _parity import TOL, compare_full, f64, maxabs, oracle_cfg, rel_l2, run_gpu
 
 pytestmark = pytest.mark.gpu
 
-MECHS = {"t5": T5, "shaw": SHAW, "txl": TXL, "deberta": DEBERTA}
+MECHS = {"t5": T5, "shaw": SHAW, "txl": TXL, "deberta": DEBERTA, "alibi": ALIBI}
 
 
 def small_wl(mech, dtype, causal, L, B=2, H=2, **kw):
@@ -170,13 +171,15 @@ def test_parity_shaw_L2048_full():
     compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
 
 
-@pytest.mark.parametrize("name", ["txl_causal_L8192_bf16", "deberta_L8192_bf16", "txl_L8192_bf16"])
+@pytest.mark.parametrize("name", ["txl_causal_L8192_bf16", "deberta_L8192_bf16", "txl_L8192_bf16",
+                                  "txl_varlen_B4_L8192_bf16", "alibi_causal_L8192_bf16", "t5_causal_L8192_bf16"])
 def test_parity_L8192_one_head(name):
-    """Every output of head 0 (table gradients included, B = 1) at L = 8192."""
+    """Every output of head 0 (table gradients of that head over the whole batch) at
+    L = 8192; the variable-length batch runs with its key lengths."""
     wl = WORKLOADS[name]
     inp = make_inputs(wl, 0)
-    out = run_gpu(wl, inp, bd.PATH_AUTO)
-    compare_full(wl, inp, out, heads=slice(0, 1))
+    out = run_gpu(wl, inp, bd.PATH_AUTO, seqlens_k=wl.seqlens_k)
+    compare_full(wl, inp, out, heads=slice(0, 1), seqlens_k=wl.seqlens_k)
 
 
 @pytest.mark.parametrize("name", ["txl_L16384_bf16", "txl_L32768_bf16"])
