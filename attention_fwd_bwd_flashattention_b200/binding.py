@@ -14,7 +14,7 @@ from typing import Optional, Sequence
 
 import torch
 
-T5, SHAW, TXL, DEBERTA = 0, 1, 2, 3
+T5, SHAW, TXL, DEBERTA, ALIBI = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
 
@@ -121,7 +121,7 @@ class Params:
                                self.shaw_clip, self.deberta_span, _ptr(self.seqlens_k))
 
     def n_rel(self) -> int:
-        return {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2}[self.mech]
+        return {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[self.mech]
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:

@@ -14,7 +14,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10100;  // 1.1.0: relpos_params_t.seqlens_k
+constexpr int kVersion = 10200;  // 1.1.0: relpos_params_t.seqlens_k; 1.2.0: RELPOS_ALIBI
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -78,14 +78,16 @@ static int fill_t5(const relpos_params_t *P, Prm &p) {
 static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   if (!P) return RELPOS_ERR_INVALID_ARG;
   memset(&p, 0, sizeof(p));
-  if (P->mech < RELPOS_T5 || P->mech > RELPOS_DEBERTA) return RELPOS_ERR_INVALID_ARG;
+  if (P->mech < RELPOS_T5 || P->mech > RELPOS_ALIBI) return RELPOS_ERR_INVALID_ARG;
   if (P->dtype != RELPOS_F32 && P->dtype != RELPOS_BF16) return RELPOS_ERR_INVALID_ARG;
   if (P->causal != 0 && P->causal != 1) return RELPOS_ERR_INVALID_ARG;
   if (P->kernel_path < RELPOS_PATH_AUTO || P->kernel_path > RELPOS_PATH_TC) return RELPOS_ERR_INVALID_ARG;
   if (P->d != rp::HD) return RELPOS_ERR_INVALID_ARG;
   if (P->B < 1 || P->H < 1 || P->L < 1 || P->L > kMaxL || P->B * P->H > 65535) return RELPOS_ERR_INVALID_ARG;
   if (!isfinite(P->scale)) return RELPOS_ERR_INVALID_ARG;
-  p.mech = P->mech;
+  // ALiBi is a per-offset bias like T5's: it runs on the T5 kernels with one slope
+  // per head in place of the bucket table
+  p.mech = P->mech == RELPOS_ALIBI ? (int)rp::M_T5 : P->mech;
   p.causal = P->causal;
   p.B = (int)P->B;
   p.H = (int)P->H;
@@ -100,6 +102,11 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
       p.nrows = p.nb;
       break;
     }
+    case RELPOS_ALIBI:
+      p.alibi = 1;
+      p.nb = 1;
+      p.nrows = 1;
+      break;
     case RELPOS_SHAW:
       if (P->shaw_clip < 0 || P->shaw_clip > 4096) return RELPOS_ERR_INVALID_ARG;
       p.clip = P->shaw_clip;

@@ -32,6 +32,9 @@ struct Prm {
   // (smallest distance of log buckets me+1, me+2, ...), capped at half-1.
   int nb, bidir, half, me, nthr;
   int thr[32];
+  // ALiBi runs on the T5 per-offset path (mech M_T5, one "bucket"): its bias vector
+  // is -m[h] |delta| and its slope gradient weights each offset's dS sum by -|delta|.
+  int alibi;
   int clip;   // Shaw clip c
   int span;   // DeBERTa span k
   int nT;     // number of 64-row tiles
@@ -42,8 +45,8 @@ struct Prm {
   void *out, *dq, *dk, *dv;
   float *lse, *drel0, *drel1, *drel2;
   // workspace
-  float *t5_bias;      // [H][2L-1]   t[h, bucket(delta)] at delta + L - 1
-  int *t5_bkt;         // [2L-1]      bucket(delta)
+  float *t5_bias;      // [H][2L-1]   t[h, bucket(delta)] (ALiBi: -m[h] |delta|) at delta + L - 1
+  int *t5_bkt;         // [2L-1]      bucket(delta) (ALiBi: 0)
   float *Dvec;         // [B][H][L]   D_i = dO_i . O_i
   float *part_row;     // per (b,h,query tile) partial of the query-side table gradient
   float *part_col;     // per (b,h,key tile) partial of the key-side table gradient

@@ -493,7 +493,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
         float acc = sm.aux[A_ACC + tid];
         for (int w = 0; w < TROWS - 1; ++w) {
           const int delta = dmin + w;
-          if (delta > -p.L && delta < p.L && p.t5_bkt[delta + p.L - 1] == tid) acc += sm.aux[A_G + w];
+          if (delta > -p.L && delta < p.L && p.t5_bkt[delta + p.L - 1] == tid)
+            acc += p.alibi ? -fabsf((float)delta) * sm.aux[A_G + w] : sm.aux[A_G + w];
         }
         sm.aux[A_ACC + tid] = acc;
       }
@@ -864,14 +865,21 @@ static cudaError_t run_bwd_t(const Prm &p, cudaStream_t st) {
 }  // namespace simt
 
 // T5 per-offset bucket and bias vectors (the method's per-call preprocessing):
-// bkt[delta + L - 1] = bucket(delta), bias[h][delta + L - 1] = t[h][bucket(delta)]
+// bkt[delta + L - 1] = bucket(delta), bias[h][delta + L - 1] = t[h][bucket(delta)];
+// ALiBi: bkt = 0 and bias = -m[h] |delta| (one slope per head, rel0 = m[H]).
 __global__ void t5_prep_kernel(Prm p) {
   const int x = blockIdx.x * blockDim.x + threadIdx.x;
   const int n = 2 * p.L - 1;
   if (x >= n) return;
+  const float *t = (const float *)p.rel0;
+  if (p.alibi) {
+    const float dist = (float)abs(x - (p.L - 1));
+    p.t5_bkt[x] = 0;
+    for (int h = 0; h < p.H; ++h) p.t5_bias[(size_t)h * n + x] = -(t[h] * dist);
+    return;
+  }
   const int bk = t5_bucket(p, x - (p.L - 1));
   p.t5_bkt[x] = bk;
-  const float *t = (const float *)p.rel0;
   for (int h = 0; h < p.H; ++h) p.t5_bias[(size_t)h * n + x] = t[h * p.nb + bk];
 }
 

@@ -13,7 +13,9 @@
  * the article "结构感知内核让相对位置注意力加速21倍" (section
  * "为什么相对位置注意力难做快": S = Q K^T / sqrt(d) + B, with B never
  * materialised).  The four mechanisms are the ones the paper's Hugging Face page
- * names (Community comment); their formulas follow their original papers:
+ * names (Community comment), and ALiBi is the further bias the article lists among
+ * the models the method suits (section "工程权衡与适用边界"); their formulas follow
+ * their original papers:
  *
  *   RELPOS_T5       R_ij = t[h, bucket(j - i)]                      (added unscaled)
  *   RELPOS_SHAW     R_ij = scale * q_i . a[h, clip(j - i, -c, c) + c]
@@ -21,6 +23,7 @@
  *                   row(x) = x when causal (table rows L), x + L - 1 otherwise (2L - 1)
  *   RELPOS_DEBERTA  R_ij = scale * (q_i . Kr[h, clip(i - j + k, 0, 2k - 1)]
  *                                 + k_j . Qr[h, clip(j - i + k, 0, 2k - 1)])
+ *   RELPOS_ALIBI   R_ij = -m[h] * |j - i|                           (added unscaled)
  *
  * T5 buckets: bidirectional (upper half for j > i) or unidirectional, exact
  * distances below max_exact = (buckets per side) / 2, then
@@ -40,6 +43,7 @@
  *       TXL      rel[0] = r  [H, n_off, d]  (n_off = L causal, 2L - 1 otherwise),
  *                rel[1] = u  [H, d], rel[2] = v [H, d]
  *       DeBERTa  rel[0] = Kr [H, 2k, d], rel[1] = Qr [H, 2k, d]
+ *       ALiBi    rel[0] = m  [H]  per-head slopes            float32 always
  *     Unused entries may be NULL.
  *   - LSE: float32 [B, H, L], natural log.
  *   - drel[0..2]: float32 gradients with the shapes of rel[0..2], summed over the
@@ -76,7 +80,7 @@
 extern "C" {
 #endif
 
-enum relpos_mech { RELPOS_T5 = 0, RELPOS_SHAW = 1, RELPOS_TXL = 2, RELPOS_DEBERTA = 3 };
+enum relpos_mech { RELPOS_T5 = 0, RELPOS_SHAW = 1, RELPOS_TXL = 2, RELPOS_DEBERTA = 3, RELPOS_ALIBI = 4 };
 enum relpos_dtype { RELPOS_F32 = 0, RELPOS_BF16 = 1 };
 
 /* kernel_path: which kernel family runs the call.  RELPOS_PATH_AUTO picks the
@@ -135,7 +139,9 @@ RELPOS_API int relpos_attn_fwd(const relpos_params_t *params,
                     int32_t *dev_status, void *stream);
 
 /* Backward pass: given O and LSE from relpos_attn_fwd and the output gradient
- * dO, writes dQ, dK, dV (params dtype) and drel[0..2] (float32, see above).
+ * dO, writes dQ, dK, dV (params dtype) and drel[0..2] (float32, see above; for
+ * ALiBi drel[0] = dm[H] = sum over pairs of dS_ij * -|j - i|, for callers that
+ * learn the slopes).
  * Gradients of the relative parameters are sharded by offset into partials and
  * merged by a fixed-order second pass with no atomics (same Abstract, technique
  * (3); article section "3. 基于偏移的梯度分片"). */

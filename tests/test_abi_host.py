@@ -56,13 +56,13 @@ def test_struct_layout_matches_c(tmp_path):
 
 
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10100
+    assert lib.relpos_attn_version() == 10200
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"
 
 
-@pytest.mark.parametrize("bad", [dict(d=32), dict(mech=7), dict(L=0), dict(B=0), dict(dtype=5), dict(scale=float("nan")),
+@pytest.mark.parametrize("bad", [dict(d=32), dict(mech=5), dict(L=0), dict(B=0), dict(dtype=5), dict(scale=float("nan")),
                                  dict(kernel_path=9), dict(mech=0, t5_num_buckets=1), dict(mech=0, t5_max_distance=4),
                                  dict(mech=3, deberta_span=0), dict(mech=1, shaw_clip=-1)])
 def test_invalid_params_rejected(lib, bad):
@@ -74,7 +74,7 @@ def test_invalid_params_rejected(lib, bad):
 
 
 def test_workspace_sizes(lib):
-    for mech in range(4):
+    for mech in range(5):
         for causal in (False, True):
             P = bd.Params(mech=mech, B=2, H=3, L=1000, causal=causal)
             f = bd.relpos_attn_workspace_size(P, 0)
@@ -83,9 +83,9 @@ def test_workspace_sizes(lib):
             assert f % 256 == 0 and b % 256 == 0
             # forward scratch: T5's per-offset bias vector; on the bf16 tensor-core
             # path also Transformer-XL's u.k / v.r and DeBERTa's end-row products
-            assert (f > 0) == (mech in (0, 2, 3))
+            assert (f > 0) == (mech in (0, 2, 3, 4))
             f32 = bd.relpos_attn_workspace_size(bd.Params(mech=mech, B=2, H=3, L=1000, causal=causal, dtype=bd.F32), 0)
-            assert (f32 > 0) == (mech == 0)
+            assert (f32 > 0) == (mech in (0, 4))
     with pytest.raises(bd.RelposError):
         bd.relpos_attn_workspace_size(bd.Params(mech=1, B=1, H=1, L=8), 2)
 
@@ -134,6 +134,7 @@ def test_resolved_paths(lib):
         (bd.SHAW, 100): (SIMT, SIMT),
         (bd.TXL, 64): (TC, TC),
         (bd.DEBERTA, 64): (TC, SIMT),
+        (bd.ALIBI, 64): (TC, SIMT),
     }
     for (mech, clip), (f, b) in want.items():
         P = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip)
