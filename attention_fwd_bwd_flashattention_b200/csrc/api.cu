@@ -136,7 +136,9 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
-  if (pass == 1) return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p));
+  if (pass == 1)
+    return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p)) ||
+           (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p));
   return rp::tc_supported(p);
 }
 
@@ -173,7 +175,10 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
       l.p2cE = take(sizeof(float) * BH * p.L * 2);
     }
   }
-  if (pass == 1 && tc && p.mech == rp::M_SHAW) {  // tensor-core backward (Shaw)
+  if (pass == 1 && tc && p.mech == rp::M_T5) {  // tensor-core backward (T5, ALiBi): per-query-tile partials
+    l.dvec = take(sizeof(float) * BH * p.L);
+    l.part_small = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nb);
+  } else if (pass == 1 && tc && p.mech == rp::M_SHAW) {  // tensor-core backward (Shaw)
     l.dvec = take(sizeof(float) * BH * p.L);
     l.qa = take(sizeof(float) * rp::tc_bwd_shaw_qa_floats(p));
     l.part_row = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nrows * rp::HD);
@@ -343,6 +348,10 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
       return RELPOS_ERR_INVALID_ARG;
     if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;
     if (p.mech == rp::M_SHAW) return to_status(rp::tc_bwd_shaw(p, tc_work(l, workspace), st));
+    if (p.mech == rp::M_T5) {
+      if ((e = to_status(rp::launch_t5_prep(p, st)))) return e;
+      return to_status(rp::tc_bwd_bias(p, st));
+    }
     return to_status(rp::tc_bwd(p, tc_work(l, workspace), st));
   }
   if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;

@@ -23,5 +23,7 @@ size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats);
 bool tc_bwd_shaw_supported(const Prm &p);
 size_t tc_bwd_shaw_qa_floats(const Prm &p);
 cudaError_t tc_bwd_shaw(const Prm &p, const TcWork &w, cudaStream_t st);
+bool tc_bwd_bias_supported(const Prm &p);
+cudaError_t tc_bwd_bias(const Prm &p, cudaStream_t st);
 cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st);
 }  // namespace rp

@@ -124,17 +124,18 @@ def test_t5_thresholds_match_oracle_buckets(lib):
 
 def test_resolved_paths(lib):
     """Which kernel family each pass runs (host-side dispatch, no device work): bf16
-    runs on the tensor cores except the backward of T5, DeBERTa and Shaw with c > 64;
+    runs on the tensor cores except the backward of DeBERTa, of Shaw with c > 64 and of
+    T5 whose buckets stay distinct over more than 8 tiles;
     float32 and an explicit CUDA-core request always run the CUDA-core kernels."""
     TC, SIMT = bd.PATH_TC, bd.PATH_SIMT
     want = {  # (mech, clip) -> (forward, backward) for bf16, automatic choice
-        (bd.T5, 64): (TC, SIMT),
+        (bd.T5, 64): (TC, TC),
         (bd.SHAW, 64): (TC, TC),
         (bd.SHAW, 65): (TC, SIMT),
         (bd.SHAW, 100): (SIMT, SIMT),
         (bd.TXL, 64): (TC, TC),
         (bd.DEBERTA, 64): (TC, SIMT),
-        (bd.ALIBI, 64): (TC, SIMT),
+        (bd.ALIBI, 64): (TC, TC),
     }
     for (mech, clip), (f, b) in want.items():
         P = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip)
@@ -143,3 +144,9 @@ def test_resolved_paths(lib):
         assert bd.relpos_attn_resolved_path(P32, 0) == SIMT and bd.relpos_attn_resolved_path(P32, 1) == SIMT
         Ps = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip, kernel_path=bd.PATH_SIMT)
         assert bd.relpos_attn_resolved_path(Ps, 0) == SIMT and bd.relpos_attn_resolved_path(Ps, 1) == SIMT
+    # T5 buckets distinct out to distance 547 (max_distance 1000) span 11 tiles at L = 4096
+    # (CUDA-core backward); at L = 300 all three tiles are band tiles (tensor cores)
+    wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
+    assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == SIMT
+    assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC
+    assert bd.relpos_attn_resolved_path(bd.Params(L=4096, t5_bidirectional=False, **wide), 1) == TC  # one side flat

@@ -14,7 +14,7 @@ from attention_fwd_bwd_flashattention_b200 import binding as bd
 from attention_fwd_bwd_flashattention_b200.inputs import (ALIBI, DEBERTA, SHAW, T5, TXL, WORKLOADS, Workload, make_inputs,
                                                            to_f64)
 
-from _parity import TOL, compare_full, f64, maxabs, oracle_cfg, rel_l2, run_gpu
+from _parity import TOL, compare_full, f64, maxabs, oracle_cfg, params_of, rel_l2, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -117,6 +117,24 @@ def test_parity_t5_unidirectional_and_odd_buckets(causal):
                       t5_bidirectional=bidir)
         inp = make_inputs(wl, nb)
         compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_parity_bias_family_tensor_core_backward(causal):
+    """T5 bucket layouts whose band of distinct-bias tiles is narrow, wide (up to the
+    eight-tile limit) or one-sided, and ALiBi slopes from nearly flat to sharply local,
+    on the bf16 tensor-core backward."""
+    for nb, md, bidir in ((32, 128, True), (10, 40, True), (7, 20, False), (32, 600, True), (64, 900, False)):
+        wl = Workload("t5x", T5, torch.bfloat16, causal, 1, 2, 1100, t5_num_buckets=nb, t5_max_distance=md,
+                      t5_bidirectional=bidir)
+        P = params_of(wl, bd.PATH_AUTO)
+        assert bd.relpos_attn_resolved_path(P, 1) == bd.PATH_TC, (nb, md, bidir)
+        inp = make_inputs(wl, nb)
+        compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+    wl = Workload("alibi_x", ALIBI, torch.bfloat16, causal, 2, 4, 1100)
+    inp = make_inputs(wl, 3)
+    inp["rel"] = [torch.tensor([1e-4, 0.02, 1.0, 8.0])]
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
 
 
 def test_t5_small_buckets_and_fp32_config():
