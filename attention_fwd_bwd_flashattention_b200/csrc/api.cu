@@ -138,7 +138,7 @@ static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
   if (pass == 1)
     return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p)) ||
-           (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p));
+           (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p)) || (p.mech == rp::M_DEB && rp::tc_bwd_deb_supported(p));
   return rp::tc_supported(p);
 }
 
@@ -147,6 +147,7 @@ struct Layout {
   size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot;
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
   size_t part_kv, part_dg, part_uv, qa;  // tensor-core backward partials / products
+  size_t qkr, kqr, dM, dN, dqc, dkc, dpart;  // DeBERTa tensor-core backward
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -175,7 +176,18 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
       l.p2cE = take(sizeof(float) * BH * p.L * 2);
     }
   }
-  if (pass == 1 && tc && p.mech == rp::M_T5) {  // tensor-core backward (T5, ALiBi): per-query-tile partials
+  if (pass == 1 && tc && p.mech == rp::M_DEB) {  // tensor-core backward (DeBERTa)
+    size_t tab = 0, partf = 0;
+    rp::tc_bwd_deb_sizes(p, tab, partf);
+    l.dvec = take(sizeof(float) * BH * p.L);
+    l.qkr = take(sizeof(float) * tab);
+    l.kqr = take(sizeof(float) * tab);
+    l.dM = take(2 * tab);
+    l.dN = take(2 * tab);
+    l.dqc = take(sizeof(float) * BH * p.L * rp::HD);
+    l.dkc = take(sizeof(float) * BH * p.L * rp::HD);
+    l.dpart = take(sizeof(float) * partf);
+  } else if (pass == 1 && tc && p.mech == rp::M_T5) {  // tensor-core backward (T5, ALiBi): per-query-tile partials
     l.dvec = take(sizeof(float) * BH * p.L);
     l.part_small = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nb);
   } else if (pass == 1 && tc && p.mech == rp::M_SHAW) {  // tensor-core backward (Shaw)
@@ -237,6 +249,13 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.part_dg = (float *)(b + l.part_dg);
   w.part_uv = (float *)(b + l.part_uv);
   w.qa = (float *)(b + l.qa);
+  w.qkr = (float *)(b + l.qkr);
+  w.kqr = (float *)(b + l.kqr);
+  w.dqc = (float *)(b + l.dqc);
+  w.dkc = (float *)(b + l.dkc);
+  w.dpart = (float *)(b + l.dpart);
+  w.dM = b + l.dM;
+  w.dN = b + l.dN;
   return w;
 }
 
@@ -348,6 +367,10 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
       return RELPOS_ERR_INVALID_ARG;
     if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;
     if (p.mech == rp::M_SHAW) return to_status(rp::tc_bwd_shaw(p, tc_work(l, workspace), st));
+    if (p.mech == rp::M_DEB) {
+      if (!aligned16(rel[1])) return RELPOS_ERR_INVALID_ARG;
+      return to_status(rp::tc_bwd_deb(p, tc_work(l, workspace), st));
+    }
     if (p.mech == rp::M_T5) {
       if ((e = to_status(rp::launch_t5_prep(p, st)))) return e;
       return to_status(rp::tc_bwd_bias(p, st));

@@ -14,6 +14,10 @@ struct TcWork {
   float *part_kv, *part_dg;      // backward partials (Transformer-XL)
   float *part_uv;                // [H][ceil(rows / 32)][64] dv partials per 32-offset tile
   float *qa;                     // Shaw backward: [B,H,L][132] per-row products q_i . a_rho
+  // DeBERTa backward: relation products QKr, KQr and dS K, dS^T Q (fp32), the
+  // offset-ordered dS copies M, N (bf16, [B,H,L][2k]) and the table-gradient partials
+  float *qkr, *kqr, *dqc, *dkc, *dpart;
+  void *dM, *dN;
 };
 bool tc_supported(const Prm &p);
 cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st);
@@ -23,6 +27,9 @@ size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats);
 bool tc_bwd_shaw_supported(const Prm &p);
 size_t tc_bwd_shaw_qa_floats(const Prm &p);
 cudaError_t tc_bwd_shaw(const Prm &p, const TcWork &w, cudaStream_t st);
+bool tc_bwd_deb_supported(const Prm &p);
+void tc_bwd_deb_sizes(const Prm &p, size_t &table_elems, size_t &part_floats);
+cudaError_t tc_bwd_deb(const Prm &p, const TcWork &w, cudaStream_t st);
 bool tc_bwd_bias_supported(const Prm &p);
 cudaError_t tc_bwd_bias(const Prm &p, cudaStream_t st);
 cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st);

@@ -704,6 +704,21 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t plane
   return tc::make_map(m, base, rows, planes, box_rows);
 }
 
+// [planes][rows][row_len] bf16 (row_len a multiple of 64); box = 64 x box_rows x 1 at any
+// 64-element column offset, 128B swizzle; rows and columns outside the tensor read as zeros.
+bool tc_make_map_bf16_wide(CUtensorMap *m, const void *base, uint32_t row_len, uint64_t rows, uint64_t planes,
+                           uint32_t box_rows) {
+  tc::EncodeTiledFn enc = tc::encode_fn();
+  if (!enc || row_len % 64u != 0) return false;
+  cuuint64_t dims[3] = {row_len, rows, planes};
+  cuuint64_t strides[2] = {(cuuint64_t)row_len * 2, (cuuint64_t)rows * row_len * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st) {
   if (p.mech != M_TXL && p.mech != M_DEB) return cudaSuccess;
   const size_t rows = (size_t)p.B * p.H * p.L + (p.mech == M_TXL ? (size_t)p.H * p.nrows : 0);

@@ -94,6 +94,8 @@ def kernel_launches(wl, path):
         bwd = 5
     elif tc and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
         bwd = 5
+    elif tc and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction
+        bwd = 7
     else:  # D, key-tile, query-tile, then the table-gradient reductions
         bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[wl.mech]
     return fwd, bwd

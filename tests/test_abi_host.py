@@ -124,8 +124,9 @@ def test_t5_thresholds_match_oracle_buckets(lib):
 
 def test_resolved_paths(lib):
     """Which kernel family each pass runs (host-side dispatch, no device work): bf16
-    runs on the tensor cores except the backward of DeBERTa, of Shaw with c > 64 and of
-    T5 whose buckets stay distinct over more than 8 tiles;
+    runs on the tensor cores except the backward of DeBERTa with a span that is not a
+    multiple of 32 up to 256, of Shaw with c > 64 and of T5 whose buckets stay distinct
+    over more than 8 tiles;
     float32 and an explicit CUDA-core request always run the CUDA-core kernels."""
     TC, SIMT = bd.PATH_TC, bd.PATH_SIMT
     want = {  # (mech, clip) -> (forward, backward) for bf16, automatic choice
@@ -134,7 +135,7 @@ def test_resolved_paths(lib):
         (bd.SHAW, 65): (TC, SIMT),
         (bd.SHAW, 100): (SIMT, SIMT),
         (bd.TXL, 64): (TC, TC),
-        (bd.DEBERTA, 64): (TC, SIMT),
+        (bd.DEBERTA, 64): (TC, TC),
         (bd.ALIBI, 64): (TC, TC),
     }
     for (mech, clip), (f, b) in want.items():
@@ -146,6 +147,9 @@ def test_resolved_paths(lib):
         assert bd.relpos_attn_resolved_path(Ps, 0) == SIMT and bd.relpos_attn_resolved_path(Ps, 1) == SIMT
     # T5 buckets distinct out to distance 547 (max_distance 1000) span 11 tiles at L = 4096
     # (CUDA-core backward); at L = 300 all three tiles are band tiles (tensor cores)
+    # DeBERTa: spans that are multiples of 32 up to 256 take the tensor-core backward
+    for span, want_b in ((256, TC), (32, TC), (96, TC), (24, SIMT), (288, SIMT)):
+        assert bd.relpos_attn_resolved_path(bd.Params(mech=bd.DEBERTA, B=1, H=2, L=300, deberta_span=span), 1) == want_b, span
     wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == SIMT
     assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC

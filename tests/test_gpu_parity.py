@@ -56,6 +56,27 @@ def test_parity_deberta_span256(path):
 
 
 @pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("span", [32, 96, 160, 256])
+@pytest.mark.parametrize("L", [130, 700, 1100])
+def test_parity_deberta_tensor_core_backward(span, causal, L):
+    """DeBERTa spans on the bf16 tensor-core backward (offset-ordered dS copies and
+    their GEMMs), with the band of tiles narrower than, equal to and wider than the
+    sequence."""
+    wl = Workload("deb_tc", DEBERTA, torch.bfloat16, causal, 2, 2, L, deberta_span=span)
+    assert bd.relpos_attn_resolved_path(params_of(wl, bd.PATH_AUTO), 1) == bd.PATH_TC
+    inp = make_inputs(wl, span + L)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_parity_deberta_tensor_core_key_lengths(causal):
+    wl = Workload("deb_tc_len", DEBERTA, torch.bfloat16, causal, 3, 2, 700, deberta_span=128)
+    lens = (700, 0, 257)
+    inp = make_inputs(wl, 5)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO, seqlens_k=lens), seqlens_k=lens)
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
 @pytest.mark.parametrize("clip", [1, 7, 33, 64, 100])
 @pytest.mark.parametrize("L", [300, 700])
 def test_parity_shaw_clip(clip, causal, L):
