@@ -61,13 +61,40 @@ struct DebArgs {
 __device__ __forceinline__ bool far_left(int m, int n, int k) { return 128 * (m - n) - 127 >= k; }
 __device__ __forceinline__ bool far_right(int m, int n, int k) { return 128 * (n - m) - 127 >= k; }
 
-// relation term of pair (i, j) on a band tile: QKr[i][rho] + KQr[j][rho'] (0 outside the sequence)
-__device__ __forceinline__ float band_rel(const DebArgs &A, int bh, int i, int j) {
+constexpr int RLD = 129;  // fp32 stride of the band tile's relation terms in smem (conflict-free rows and columns)
+
+// Relation terms of band tile (i0, j0) into R[il * RLD + jl] = QKr[i][rho] + KQr[j][rho']
+// (0 outside the sequence).  Warp w loads rows il = 8w .. 8w + 7 of QKr, then keys
+// jl = 8w .. 8w + 7 of KQr; every load is a coalesced run of one table row and all of
+// a warp's 32 loads of a phase are independent.  Ends with R complete for every row thread.
+__device__ __forceinline__ void band_fill(const DebArgs &A, int bh, int i0, int j0, float *R, int warp, int lane) {
   const Prm &p = A.p;
-  const int W = A.W, k = p.span;
-  if (i >= p.L || j >= p.L) return 0.f;
-  const int r = iclamp(i - j + k, 0, W - 1), r2 = iclamp(j - i + k, 0, W - 1);
-  return A.qkr[((size_t)bh * p.L + i) * W + r] + A.kqr[((size_t)bh * p.L + j) * W + r2];
+  const int L = p.L, W = A.W, k = p.span;
+  float v[32];
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int i = i0 + 8 * warp + rr;
+    const float *row = A.qkr + ((size_t)bh * L + (i < L ? i : 0)) * W;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[4 * rr + q] = (i < L) ? row[iclamp(i - j0 - (lane + 32 * q) + k, 0, W - 1)] : 0.f;
+  }
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) R[(8 * warp + rr) * RLD + lane + 32 * q] = v[4 * rr + q];
+  named_bar_sync(2, NSOFT);
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int j = j0 + 8 * warp + rr;
+    const float *row = A.kqr + ((size_t)bh * L + (j < L ? j : 0)) * W;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[4 * rr + q] = (j < L) ? row[iclamp(j - (i0 + lane + 32 * q) + k, 0, W - 1)] : 0.f;
+  }
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) R[(lane + 32 * q) * RLD + 8 * warp + rr] += v[4 * rr + q];
+  named_bar_sync(2, NSOFT);
 }
 
 // log2-domain scores y = (s_raw + R) c1 - lse2 of four keys
@@ -175,8 +202,8 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
 // ============================================================================
 namespace kvd {
 constexpr int OFF_K = 0, OFF_V = 16384, OFF_Q = 32768, OFF_DO = OFF_Q + 32768;
-constexpr int OFF_PDS = OFF_DO + 32768;  // P tile, dS tile at +32768
-constexpr int OFF_ONES = OFF_PDS + 65536;  // 128 x 64 bf16 ones, MN-major swizzled (B of dS^T 1)
+constexpr int OFF_PDS = OFF_DO + 32768;  // P tile, dS tile at +32768; band tiles: relation terms (128 x RLD fp32) first
+constexpr int OFF_ONES = OFF_PDS + 67584;  // 128 x 64 bf16 ones, MN-major swizzled (B of dS^T 1)
 constexpr int OFF_VEC = OFF_ONES + 16384;  // per tile, double-buffered: [lse2 | D | c2p end product] x 384
 constexpr int OFF_EK = OFF_VEC + 3072;     // p2c end products of the CTA's keys [2][128]
 constexpr int OFF_RED = OFF_EK + 1024;     // band column sums [2 classes][4 row quarters][128]
@@ -345,6 +372,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
       const float nv = (tid < 384 && t + 1 < iters) ? fetch1(t + 1) : 0.f;
       named_bar_sync(1, NSOFT);
       const bool fl = far_left(m, n, k), fr = far_right(m, n, k), band = !fl && !fr;
+      float *Rt = (float *)(smem + OFF_PDS);
+      if (band) {  // the relation terms overwrite the P / dS tiles: the previous tile's MMAs must be done
+        if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
+        band_fill(A, bh, m * 128, j0, Rt, warp, lane);
+      }
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
       uint32_t pk[NC / 2], dk[NC / 2];
       const bool need_mask = (p.causal && m == n) || (j0 + 128 > klen);
@@ -352,15 +384,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
         tc_fence_after();
         const float lse2 = tv[il], Dv = tv[128 + il], cE = tv[256 + il];
         const float *ekr = ek + (fl ? 0 : 128) + cb;
+        const float *Rrow = Rt + il * RLD + cb;
         const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
         auto pds = [&](auto masked, auto banded) {
 #pragma unroll
           for (int hq = 0; hq < NC / 16; ++hq) {
-            float Rb[16];
-            if constexpr (decltype(banded)::value) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) Rb[e] = band_rel(A, bh, i, j0 + cb + 16 * hq + e);
-            }
             uint32_t rs[16], rp[16];
             tmem_ld16(tl + T_S + cb + 16 * hq, rs);
             tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
@@ -370,7 +398,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
               const int x0 = 16 * hq + 4 * c4;
               float R[4], y[4], pr[4], dd[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) R[e] = decltype(banded)::value ? Rb[4 * c4 + e] : cE + ekr[x0 + e];
+              for (int e = 0; e < 4; ++e) R[e] = decltype(banded)::value ? Rrow[x0 + e] : cE + ekr[x0 + e];
               score_rel4(rs + 4 * c4, R, c12, nlse, y);
               if constexpr (decltype(masked)::value) {
 #pragma unroll
@@ -400,7 +428,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
 #pragma unroll
         for (int e = 0; e < NC / 2; ++e) pk[e] = dk[e] = 0u;
       }
-      if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
+      if (band) named_bar_sync(1, NSOFT);  // every row has read the relation terms: P / dS may overwrite them
+      else if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
       if (good) {
 #pragma unroll
         for (int cc = 0; cc < NC / 8; ++cc) {
@@ -511,10 +540,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
 // ============================================================================
 namespace qd {
 constexpr int OFF_Q = 0, OFF_DO = 16384, OFF_K = 32768, OFF_V = OFF_K + 32768;
-constexpr int OFF_VEC = OFF_V + 32768;   // p2c end products of the tile's keys, double-buffered [2][128]
+constexpr int OFF_R = OFF_V + 32768;     // band tiles: relation terms, then dS (128 x RLD fp32)
+constexpr int OFF_VEC = OFF_R + 128 * RLD * 4;  // p2c end products of the tile's keys, double-buffered [2][128]
 constexpr int OFF_RED = OFF_VEC + 1024;  // clipped row sums [2][4][128]
 constexpr int OFF_BAR = OFF_RED + 4096;
-constexpr int SMEM = 120 * 1024;  // one CTA per SM (512 TMEM columns each)
+constexpr int SMEM = OFF_BAR + 256 + 1024;  // over half the SM: one CTA per SM (512 TMEM columns each)
 enum { B_QD = 0, B_ST0, B_ST1, B_SDP, B_SDPCONS, B_PDS, B_DSFREE, B_DRAIN, NB };
 constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_DS = 320;
 static_assert(OFF_BAR + 256 + 1024 <= SMEM, "shared memory layout");
@@ -647,6 +677,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
       if (n + 1 < nTiles) nva = fetch_ek(n + 1);
       named_bar_sync(1, NSOFT);
       const bool fl = far_left(m, n, k), fr = far_right(m, n, k), band = !fl && !fr;
+      float *Rt = (float *)(smem + OFF_R);
+      if (band) band_fill(A, bh, i0, j0, Rt, warp, lane);
       good = good && warp_wait(BAR(B_SDP), n & 1, abort_flag, status);
       const bool need_mask = (p.causal && n == m) || (j0 + 128 > klen);
       float x[NC];
@@ -654,14 +686,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
         tc_fence_after();
         const float cE = fl ? cEW : cE0;
         const float *ekr = tv + cb;
+        const float *Rrow = Rt + il * RLD + cb;
         auto pds = [&](auto masked, auto banded) {
 #pragma unroll
           for (int hq = 0; hq < NC / 16; ++hq) {
-            float Rb[16];
-            if constexpr (decltype(banded)::value) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) Rb[e] = band_rel(A, bh, i, j0 + cb + 16 * hq + e);
-            }
             uint32_t rs[16], rp[16];
             tmem_ld16(tl + T_S + cb + 16 * hq, rs);
             tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
@@ -671,7 +699,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
               const int x0 = 16 * hq + 4 * c4;
               float R[4], y[4], pr[4], dd[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) R[e] = decltype(banded)::value ? Rb[4 * c4 + e] : cE + ekr[x0 + e];
+              for (int e = 0; e < 4; ++e) R[e] = decltype(banded)::value ? Rrow[x0 + e] : cE + ekr[x0 + e];
               score_rel4(rs + 4 * c4, R, c12, nlse, y);
               if constexpr (decltype(masked)::value) {
 #pragma unroll
@@ -702,21 +730,35 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
       uint32_t pk[NC / 2];
 #pragma unroll
       for (int q = 0; q < NC / 2; ++q) pk[q] = pack_bf16x2(x[2 * q], x[2 * q + 1]);
-      // ---- clipped row sums and the M entries of the tile ----
+      // ---- clipped row sums; band tiles: dS through smem into the M rows ----
       if (band) {
         const int r0 = i - j0 - cb + k;  // rho of this thread's first key (decreasing with the key)
 #pragma unroll
         for (int e = 0; e < NC; ++e) {
           const int r = r0 - e;
-          const float dsb = (e & 1) ? bf_hi(pk[e >> 1]) : bf_lo(pk[e >> 1]);
-          if (r <= 0) rs0 += dsb;
-          else if (r >= W - 1) rsW += dsb;
-          else if (i < L) *reinterpret_cast<uint16_t *>(mrow + r) = (uint16_t)((e & 1) ? (pk[e >> 1] >> 16) : (pk[e >> 1] & 0xFFFFu));
+          if (r <= 0) rs0 += x[e];
+          else if (r >= W - 1) rsW += x[e];
+        }
+        named_bar_sync(2, NSOFT);  // every row has read the relation terms
+#pragma unroll
+        for (int e = 0; e < NC; ++e) Rt[il * RLD + cb + e] = x[e];
+        named_bar_sync(2, NSOFT);
+        // warp w writes rows 8w .. 8w + 7: M[i][rho] for the interior rho of the tile's keys
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+          const int ir = i0 + 8 * warp + rr;
+          if (ir >= L) continue;
+          __nv_bfloat16 *mr = A.M + ((size_t)bh * L + ir) * W;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int jl = lane + 32 * q, r = ir - j0 - jl + k;
+            if (r >= 1 && r <= W - 2) mr[r] = __float2bfloat16_rn(Rt[(8 * warp + rr) * RLD + jl]);
+          }
         }
       } else {
         float s = 0.f;
 #pragma unroll
-        for (int e = 0; e < NC; ++e) s += (e & 1) ? bf_hi(pk[e >> 1]) : bf_lo(pk[e >> 1]);
+        for (int e = 0; e < NC; ++e) s += x[e];
         if (fl) rsW += s; else rs0 += s;
       }
       // ---- dS -> TMEM for dQ += dS K ----
