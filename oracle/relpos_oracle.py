@@ -30,7 +30,11 @@ original papers, because the pages print none of their formulas:
                                           + k_j.Qr[h, clip(j - i + k, 0, 2k-1)])
 
 with s the caller's scale (1/sqrt(d) for the first three, 1/sqrt(3d) for DeBERTa
-by default).  ALiBi, the further bias named by the article (section "工程权衡与适用边界",
+by default).  Shaw's value-side term (the second relative table of Shaw et al.,
+optional: ``RelCfg.shaw_value``) adds the same clipped offset's table row to every
+value a query averages:
+
+  O_i = sum_j P_ij (v_j + aV[h, clip(j - i, -c, c) + c])  ALiBi, the further bias named by the article (section "工程权衡与适用边界",
 in its list of models the method suits), is written from its own
 paper (Press et al., "Train Short, Test Long"):
 
@@ -88,6 +92,7 @@ class RelCfg:
     t5_bidirectional: bool = True
     shaw_clip: int = 64
     deberta_span: int = 256
+    shaw_value: bool = False  # Shaw: rel[1] = aV, the value-side table
 
 
 def default_scale(mech: int, d: int) -> float:
@@ -219,7 +224,7 @@ def head_bias(mech, q, k, rel_h, scale, cfg, causal, rows_i):
         (t,) = rel_h
         return t[index_map(T5, L, causal, cfg, rows_i)]
     if mech == SHAW:
-        (a,) = rel_h
+        a = rel_h[0]  # rel_h[1], the value-side table, does not enter the scores
         qa = qi @ a.T  # [rows, 2c+1]: every q_i . a_r
         idx = index_map(SHAW, L, causal, cfg, rows_i)
         return scale * np.take_along_axis(qa, idx, axis=1)
@@ -266,6 +271,19 @@ def _head_tables(mech, rel, h):
     return tuple(np.asarray(x[h], dtype=np.float64) for x in rel)
 
 
+def _value_term(mech, cfg):
+    return mech == SHAW and cfg.shaw_value
+
+
+def _by_offset(X, mech, L, causal, cfg, rows_i, nrows):
+    """Pe[r, rho] = sum of X[r, j] over the keys j whose pair (rows_i[r], j) reads
+    table row rho (X is zero on masked pairs)."""
+    idx = index_map(mech, L, causal, cfg, rows_i)
+    Pe = np.zeros((rows_i.size, nrows))
+    np.add.at(Pe, (np.repeat(np.arange(rows_i.size), L), idx.ravel()), X.ravel())
+    return Pe
+
+
 # --------------------------------------------------------------------------
 # Public entry points
 # --------------------------------------------------------------------------
@@ -289,6 +307,8 @@ def forward(mech, q, k, v, rel, causal, scale=None, cfg=RelCfg(), rows=None, seq
             S = head_scores(mech, q[b, h], k[b, h], rh, scale, cfg, causal, rows_i, _lk(seqlens_k, b))
             P, lse = _softmax_rows(S)
             O[b, h] = P @ v[b, h]
+            if _value_term(mech, cfg):
+                O[b, h] += _by_offset(P, mech, L, causal, cfg, rows_i, rh[1].shape[0]) @ rh[1]
             LSE[b, h] = lse
     return O, LSE
 
@@ -296,7 +316,7 @@ def forward(mech, q, k, v, rel, causal, scale=None, cfg=RelCfg(), rows=None, seq
 def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg(), seqlens_k=None):
     """Exact gradients (dq, dk, dv, drel) of  sum(O * dO).
 
-    drel matches rel's structure: T5 [dt], Shaw [da], TXL [dr, du, dv],
+    drel matches rel's structure: T5 [dt], Shaw [da] (+ daV with the value term), TXL [dr, du, dv],
     DeBERTa [dKr, dQr], ALiBi [dm]; table gradients sum over the batch (tables
     are per head).
     """
@@ -314,6 +334,12 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg(), seqlens_k
             P, _ = _softmax_rows(S)
             O = P @ vh
             dP = gh @ vh.T
+            if _value_term(mech, cfg):  # O_i += sum_j P_ij aV_rho: dP_ij += dO_i . aV_rho, daV += Pe^T dO
+                aV = rh[1]
+                Pe = _by_offset(P, mech, L, causal, cfg, rows_i, aV.shape[0])
+                O = O + Pe @ aV
+                dP = dP + np.take_along_axis(gh @ aV.T, index_map(mech, L, causal, cfg, rows_i), axis=1)
+                drel[1][h] += Pe.T @ gh
             D = np.sum(gh * O, axis=1)
             dS = P * (dP - D[:, None])
             dv[b, h] = P.T @ gh
@@ -326,7 +352,7 @@ def backward(mech, q, k, v, rel, causal, dO, scale=None, cfg=RelCfg(), seqlens_k
                 idx = index_map(T5, L, causal, cfg, rows_i)
                 np.add.at(drel[0][h], idx.ravel(), dS.ravel())
             elif mech == SHAW:
-                (a,) = rh
+                a = rh[0]
                 idx = index_map(SHAW, L, causal, cfg, rows_i)
                 M = np.zeros((L, a.shape[0]))  # M[i, r] = sum_{j: idx=r} dS_ij
                 np.add.at(M, (np.repeat(rows_i, L), idx.ravel()), dS.ravel())
@@ -375,6 +401,10 @@ def backward_rows(mech, q, k, v, rel, causal, dO, rows, scale=None, cfg=RelCfg()
             P, _ = _softmax_rows(S)
             O = P @ vh
             dP = gh[rows_i] @ vh.T
+            if _value_term(mech, cfg):
+                aV = rh[1]
+                O = O + _by_offset(P, mech, L, causal, cfg, rows_i, aV.shape[0]) @ aV
+                dP = dP + np.take_along_axis(gh[rows_i] @ aV.T, index_map(mech, L, causal, cfg, rows_i), axis=1)
             D = np.sum(gh[rows_i] * O, axis=1)
             dS = P * (dP - D[:, None])
             g = scale * (dS @ kh)

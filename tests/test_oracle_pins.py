@@ -121,9 +121,16 @@ def bf_score(mech, q, k, rel, h, i, j, L, causal, s, cfg):
     return s * (dot(q[i], k[j]) + dot(q[i], rel[0][h][c2p]) + dot(k[j], rel[1][h][p2c]))
 
 
+def bf_value_row(cfg, i, j):
+    c = cfg.shaw_clip
+    return max(-c, min(c, j - i)) + c
+
+
 def brute(mech, q, k, v, rel, causal, do, s, cfg, lk=None):
     """Scalar loops over (i, j) from the mechanism formulas; lk[b] (optional) is the
-    batch's key length: keys j >= lk[b] do not take part."""
+    batch's key length: keys j >= lk[b] do not take part.  With Shaw's value term
+    (cfg.shaw_value) every value v_j is read as v_j + aV[row(i, j)]."""
+    val = mech == SHAW and cfg.shaw_value
     B, H, L, d = q.shape
     O = np.zeros_like(q)
     LSE = np.zeros((B, H, L))
@@ -145,14 +152,18 @@ def brute(mech, q, k, v, rel, causal, do, s, cfg, lk=None):
                 for j in keys:
                     P[i, j] = math.exp(sc[j] - m) / z
                 for c in range(d):
-                    O[b, h, i, c] = sum(P[i, j] * vb[j, c] for j in keys)
+                    O[b, h, i, c] = sum(P[i, j] * (vb[j, c] + (rel[1][h][bf_value_row(cfg, i, j)][c] if val else 0.0))
+                                        for j in keys)
             for i in range(L):
                 Di = dot(gb[i], O[b, h, i])
                 for j in range(L):
                     if (causal and j > i) or (lk is not None and j >= lk[b]):
                         continue
-                    dS = P[i, j] * (dot(gb[i], vb[j]) - Di)
+                    vj = vb[j] + (rel[1][h][bf_value_row(cfg, i, j)] if val else 0.0)
+                    dS = P[i, j] * (dot(gb[i], vj) - Di)
                     dv[b, h, j] += P[i, j] * gb[i]
+                    if val:
+                        drel[1][h][bf_value_row(cfg, i, j)] += P[i, j] * gb[i]
                     dq[b, h, i] += s * dS * kb[j]
                     dk[b, h, j] += s * dS * qb[i]
                     if mech == ALIBI:
@@ -257,6 +268,74 @@ def test_padding_keys_do_not_matter(mech):
     plain = orc.forward(mech, q, k, v, rel, False, 0.3, SMALL)
     np.testing.assert_array_equal(full[0], plain[0])
     np.testing.assert_array_equal(full[1], plain[1])
+
+
+# ----------------------------------------------------------------------------
+# Shaw's value-side term
+# ----------------------------------------------------------------------------
+VAL = RelCfg(shaw_clip=2, shaw_value=True)
+
+
+def value_case(B, H, L, d, seed):
+    rng = np.random.default_rng(seed)
+    q, k, v, do = (rnd(rng, B, H, L, d) for _ in range(4))
+    rel = [rnd(rng, H, 2 * VAL.shaw_clip + 1, d, std=0.5), rnd(rng, H, 2 * VAL.shaw_clip + 1, d, std=0.5)]
+    return q, k, v, do, rel
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("L,lk", [(1, None), (3, None), (7, None), (8, (8, 3))])
+def test_shaw_value_term_vs_brute_force(causal, L, lk):
+    q, k, v, do, rel = value_case(2, 2, L, 3, seed=L + 5)
+    s = 0.45
+    O, LSE = orc.forward(SHAW, q, k, v, rel, causal, s, VAL, seqlens_k=lk)
+    dq, dk, dv, drel = orc.backward(SHAW, q, k, v, rel, causal, do, s, VAL, seqlens_k=lk)
+    bO, bL, bdq, bdk, bdv, bdrel = brute(SHAW, q, k, v, rel, causal, do, s, VAL, lk=lk)
+    for got, want in [(O, bO), (LSE, bL), (dq, bdq), (dk, bdk), (dv, bdv)] + list(zip(drel, bdrel)):
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    rows = np.arange(L)[::2]
+    dq2 = orc.backward_rows(SHAW, q, k, v, rel, causal, do, rows, s, VAL, seqlens_k=lk)
+    np.testing.assert_allclose(dq2, dq[:, :, rows], rtol=1e-12, atol=1e-12)
+    O2, _ = orc.forward(SHAW, q, k, v, rel, causal, s, VAL, rows=rows, seqlens_k=lk)
+    np.testing.assert_allclose(O2, O[:, :, rows], rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_shaw_value_term_finite_differences(causal):
+    q, k, v, do, rel = value_case(1, 2, 11, 4, seed=3)
+    s = 0.4
+
+    def loss(rel_):
+        return float(np.sum(orc.forward(SHAW, q, k, v, rel_, causal, s, VAL)[0] * do))
+
+    _, _, _, drel = orc.backward(SHAW, q, k, v, rel, causal, do, s, VAL)
+    rng = np.random.default_rng(8)
+    for n in range(2):
+        e = rng.standard_normal(rel[n].shape)
+        rp, rm = list(rel), list(rel)
+        rp[n] = rel[n] + 1e-6 * e
+        rm[n] = rel[n] - 1e-6 * e
+        fd = (loss(rp) - loss(rm)) / 2e-6
+        an = float(np.sum(drel[n] * e))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (n, fd, an)
+
+
+def test_shaw_value_term_constant_rows_shift_the_output():
+    """aV rows all equal to w: each row of P sums to one, so O = O_plain + w, the
+    scores (LSE, dq, dk) do not change, and the daV rows add up to sum_i dO_i."""
+    q, k, v, do, rel = value_case(2, 2, 9, 4, seed=4)
+    w = np.random.default_rng(1).standard_normal((2, 4))
+    aV = np.repeat(w[:, None, :], 2 * VAL.shaw_clip + 1, axis=1)
+    plain = RelCfg(shaw_clip=2)
+    O0, L0 = orc.forward(SHAW, q, k, v, rel[:1], False, 0.5, plain)
+    O1, L1 = orc.forward(SHAW, q, k, v, [rel[0], aV], False, 0.5, VAL)
+    np.testing.assert_allclose(O1, O0 + w[None, :, None, :], atol=1e-12)
+    np.testing.assert_array_equal(L1, L0)
+    g0 = orc.backward(SHAW, q, k, v, rel[:1], False, do, 0.5, plain)
+    g1 = orc.backward(SHAW, q, k, v, [rel[0], aV], False, do, 0.5, VAL)
+    for a, b in zip(list(g0[:3]) + [g0[3][0]], list(g1[:3]) + [g1[3][0]]):
+        np.testing.assert_allclose(b, a, atol=1e-11)
+    np.testing.assert_allclose(g1[3][1].sum(axis=1), do.sum(axis=(0, 2)), atol=1e-11)
 
 
 # ----------------------------------------------------------------------------
