@@ -45,6 +45,7 @@ class relpos_params_t(ctypes.Structure):
         ("shaw_clip", ctypes.c_int32),
         ("deberta_span", ctypes.c_int32),
         ("seqlens_k", ctypes.c_void_p),
+        ("shaw_value", ctypes.c_int32),
     ]
 
 
@@ -107,6 +108,7 @@ class Params:
     shaw_clip: int = 64
     deberta_span: int = 256
     seqlens_k: Optional[torch.Tensor] = None  # [B] int32 on the device, or None (all L)
+    shaw_value: bool = False  # Shaw: rel[1] = aV, the value-side table
 
     def c(self) -> relpos_params_t:
         scale = self.scale
@@ -118,9 +120,11 @@ class Params:
                 raise ValueError("seqlens_k must be a contiguous int32 tensor of B elements")
         return relpos_params_t(self.mech, self.dtype, int(self.causal), self.kernel_path, self.B, self.H, self.L, self.d,
                                float(scale), self.t5_num_buckets, self.t5_max_distance, int(self.t5_bidirectional),
-                               self.shaw_clip, self.deberta_span, _ptr(self.seqlens_k))
+                               self.shaw_clip, self.deberta_span, _ptr(self.seqlens_k), int(self.shaw_value))
 
     def n_rel(self) -> int:
+        if self.mech == SHAW and self.shaw_value:
+            return 2
         return {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[self.mech]
 
 

@@ -14,7 +14,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10200;  // 1.1.0: relpos_params_t.seqlens_k; 1.2.0: RELPOS_ALIBI
+constexpr int kVersion = 10300;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -85,6 +85,7 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   if (P->d != rp::HD) return RELPOS_ERR_INVALID_ARG;
   if (P->B < 1 || P->H < 1 || P->L < 1 || P->L > kMaxL || P->B * P->H > 65535) return RELPOS_ERR_INVALID_ARG;
   if (!isfinite(P->scale)) return RELPOS_ERR_INVALID_ARG;
+  if (P->shaw_value != 0 && (P->shaw_value != 1 || P->mech != RELPOS_SHAW)) return RELPOS_ERR_INVALID_ARG;
   // ALiBi is a per-offset bias like T5's: it runs on the T5 kernels with one slope
   // per head in place of the bucket table
   p.mech = P->mech == RELPOS_ALIBI ? (int)rp::M_T5 : P->mech;
@@ -111,6 +112,7 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
       if (P->shaw_clip < 0 || P->shaw_clip > 4096) return RELPOS_ERR_INVALID_ARG;
       p.clip = P->shaw_clip;
       p.nrows = 2 * p.clip + 1;
+      p.shaw_v = P->shaw_value;
       break;
     case RELPOS_TXL:
       p.nrows = p.causal ? p.L : 2 * p.L - 1;
@@ -136,6 +138,7 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
+  if (p.shaw_v) return false;  // Shaw's value-side term runs on the CUDA-core kernels
   if (pass == 1)
     return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p)) ||
            (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p)) || (p.mech == rp::M_DEB && rp::tc_bwd_deb_supported(p));
@@ -144,7 +147,7 @@ static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
 
 // ---- workspace layout ------------------------------------------------------
 struct Layout {
-  size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot;
+  size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot, part_val;
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
   size_t part_kv, part_dg, part_uv, qa;  // tensor-core backward partials / products
   size_t qkr, kqr, dM, dN, dqc, dkc, dpart;  // DeBERTa tensor-core backward
@@ -208,7 +211,10 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
     const size_t tab = (size_t)p.nrows * rp::HD;
     switch (p.mech) {
       case rp::M_T5: l.part_small = take(sizeof(float) * BH * p.nT * p.nb); break;
-      case rp::M_SHAW: l.part_row = take(sizeof(float) * BH * p.nT * tab); break;
+      case rp::M_SHAW:
+        l.part_row = take(sizeof(float) * BH * p.nT * tab);
+        if (p.shaw_v) l.part_val = take(sizeof(float) * BH * p.nT * tab);
+        break;
       case rp::M_DEB:
         l.part_row = take(sizeof(float) * BH * p.nT * tab);
         l.part_col = take(sizeof(float) * BH * p.nT * tab);
@@ -236,6 +242,7 @@ static void bind_workspace(Prm &p, const Layout &l, void *ws) {
   p.part_small = (float *)(b + l.part_small);
   p.part_diag = (float *)(b + l.part_diag);
   p.gtot = (float *)(b + l.gtot);
+  p.part_val = (float *)(b + l.part_val);
 }
 
 static rp::TcWork tc_work(const Layout &l, void *ws) {
@@ -261,7 +268,9 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
 
 static bool aligned16(const void *x) { return ((uintptr_t)x & 15) == 0; }
 
-static int rel_count(int mech) { return mech == rp::M_TXL ? 3 : (mech == rp::M_DEB ? 2 : 1); }
+static int rel_count(const Prm &p) {
+  return p.mech == rp::M_TXL ? 3 : ((p.mech == rp::M_DEB || p.shaw_v) ? 2 : 1);
+}
 
 static int to_status(cudaError_t e) {
   if (e == cudaSuccess) return RELPOS_OK;
@@ -299,7 +308,7 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   int e = validate_and_fill(params, p);
   if (e) return e;
   if (!q || !k || !v || !rel || !o || !lse) return RELPOS_ERR_INVALID_ARG;
-  for (int i = 0; i < rel_count(p.mech); ++i)
+  for (int i = 0; i < rel_count(p); ++i)
     if (!rel[i]) return RELPOS_ERR_INVALID_ARG;
   if ((e = check_seqlens(params))) return e;
   const bool tc = use_tc(params, p, 0);
@@ -316,8 +325,8 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   p.k = k;
   p.v = v;
   p.rel0 = rel[0];
-  p.rel1 = rel_count(p.mech) > 1 ? rel[1] : nullptr;
-  p.rel2 = rel_count(p.mech) > 2 ? rel[2] : nullptr;
+  p.rel1 = rel_count(p) > 1 ? rel[1] : nullptr;
+  p.rel2 = rel_count(p) > 2 ? rel[2] : nullptr;
   p.out = o;
   p.lse = lse;
   p.status = dev_status;
@@ -336,7 +345,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   int e = validate_and_fill(params, p);
   if (e) return e;
   if (!q || !k || !v || !rel || !o || !lse || !dout || !dq || !dk || !dv || !drel) return RELPOS_ERR_INVALID_ARG;
-  for (int i = 0; i < rel_count(p.mech); ++i)
+  for (int i = 0; i < rel_count(p); ++i)
     if (!rel[i] || !drel[i]) return RELPOS_ERR_INVALID_ARG;
   if ((e = check_seqlens(params))) return e;
   const bool tc = use_tc(params, p, 1);
@@ -350,15 +359,15 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   p.o = o;
   p.dout = dout;
   p.rel0 = rel[0];
-  p.rel1 = rel_count(p.mech) > 1 ? rel[1] : nullptr;
-  p.rel2 = rel_count(p.mech) > 2 ? rel[2] : nullptr;
+  p.rel1 = rel_count(p) > 1 ? rel[1] : nullptr;
+  p.rel2 = rel_count(p) > 2 ? rel[2] : nullptr;
   p.lse = (float *)lse;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
   p.drel0 = drel[0];
-  p.drel1 = rel_count(p.mech) > 1 ? drel[1] : nullptr;
-  p.drel2 = rel_count(p.mech) > 2 ? drel[2] : nullptr;
+  p.drel1 = rel_count(p) > 1 ? drel[1] : nullptr;
+  p.drel2 = rel_count(p) > 2 ? drel[2] : nullptr;
   p.status = dev_status;
   cudaStream_t st = (cudaStream_t)stream;
   const bool bf16 = params->dtype == RELPOS_BF16;

@@ -36,6 +36,7 @@ struct Prm {
   // is -m[h] |delta| and its slope gradient weights each offset's dS sum by -|delta|.
   int alibi;
   int clip;   // Shaw clip c
+  int shaw_v;  // Shaw: value-side table rel1 = aV (O_i += sum_j P_ij aV[row(j - i)])
   int span;   // DeBERTa span k
   int nT;     // number of 64-row tiles
   int diag_ch, diag_nchunk, nbands;  // Transformer-XL diagonal shards
@@ -52,6 +53,7 @@ struct Prm {
   float *part_col;     // per (b,h,key tile) partial of the key-side table gradient
   float *part_small;   // T5 bucket partials / Transformer-XL du partials
   float *part_diag;    // Transformer-XL per-diagonal-shard partials
+  float *part_val;     // Shaw value term: per (b,h,query tile) partial of daV
   float *gtot;         // Transformer-XL [H][n_off] diagonal sums of dS
   int *status;
   const int *seqlens_k;  // [B] key lengths (device), or null: every batch has L keys

@@ -245,6 +245,10 @@ __device__ __forceinline__ void scores(const Prm &p, const Sm &sm, int h, int i0
     }
 }
 
+template <int MECH, bool COLSIDE, bool TRANS>
+__device__ __forceinline__ void scatter_E(const Prm &p, const float (&dS)[4][4], float *E, int i0, int j0, int lo, int nw);
+__device__ __forceinline__ void zero_W(float *W, int nw);
+
 // ---------------------------------------------------------------------------
 // forward: one CTA per (query tile, head, batch)
 // ---------------------------------------------------------------------------
@@ -307,6 +311,17 @@ __global__ void __launch_bounds__(NT, 1) fwd_kernel(Prm p) {
       for (int c = 0; c < 4; ++c) sm.P[(ty + 16 * a) * LDX + tx + 16 * c] = S[a][c];
     __syncthreads();
     mm_nn<4, 4>(sm.P, LDX, sm.V, LDX, BN, O);
+    if (MECH == M_SHAW && p.shaw_v) {
+      // value term: O_i += sum_rho Pe[i][rho] aV_rho, Pe = P by table row (window of the tile)
+      int lo, nw;
+      row_window<MECH>(p, j0 - (i0 + BM - 1), j0 + BN - 1 - i0, lo, nw);
+      zero_W(sm.W, 0);
+      __syncthreads();
+      scatter_E<MECH, false, false>(p, S, sm.W, i0, j0, lo, nw);
+      load_tab((const T *)p.rel1 + (size_t)h * p.nrows * HD, lo, nw, sm.T);
+      __syncthreads();
+      mm_nn<4, 4>(sm.W, WS, sm.T, LDX, nw, O);
+    }
   }
   T *Og = (T *)p.out + base;
 #pragma unroll
@@ -388,6 +403,30 @@ __device__ __forceinline__ void scatter_E(const Prm &p, const float (&dS)[4][4],
   }
 }
 
+// Shaw value term in dP: dP_ij += dO_i . aV[row(j - i)] for the tile's pairs (TRANS as in
+// scores()).  The window products dO . aV_w come from one small GEMM; contains
+// __syncthreads() and uses T / W, which scores() has finished with.
+template <bool TRANS, class T>
+__device__ __forceinline__ void value_dp(const Prm &p, const Sm &sm, int h, int i0, int j0, int dmin, int dmax,
+                                         float (&dP)[4][4]) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  int lo, nw;
+  row_window<M_SHAW>(p, dmin, dmax, lo, nw);
+  __syncthreads();
+  load_tab((const T *)p.rel1 + (size_t)h * p.nrows * HD, lo, nw, sm.T);
+  __syncthreads();
+  window_gemm(sm.dO, sm.T, nw, sm.W);  // W[r][w] = dO_r . aV_{lo + w}
+  __syncthreads();
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int r = TRANS ? tx + 16 * b : ty + 16 * a, c = TRANS ? ty + 16 * a : tx + 16 * b;
+      const int w = rho_row<M_SHAW>(p, (j0 + c) - (i0 + r)) - lo;
+      if (w >= 0 && w < nw) dP[a][b] += sm.W[r * WS + w];
+    }
+}
+
 __device__ __forceinline__ void zero_W(float *W, int nw) {
   for (int x = threadIdx.x; x < BM * WS; x += NT) W[x] = 0.f;
   (void)nw;
@@ -437,9 +476,14 @@ __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
   }
   // this CTA's partial of the query-side table gradient (Shaw a, DeBERTa Kr)
   float *part = nullptr;
+  float *partv = nullptr;  // Shaw value term: daV partial of this CTA
   if (MECH == M_SHAW || MECH == M_DEB) {
     part = p.part_row + (bh * p.nT + m) * (size_t)p.nrows * HD;
     for (int x = tid; x < p.nrows * HD; x += NT) part[x] = 0.f;
+  }
+  if (MECH == M_SHAW && p.shaw_v) {
+    partv = p.part_val + (bh * p.nT + m) * (size_t)p.nrows * HD;
+    for (int x = tid; x < p.nrows * HD; x += NT) partv[x] = 0.f;
   }
   if (MECH == M_T5 && tid < 64) sm.aux[A_ACC + tid] = 0.f;
   float dQ[4][4];
@@ -464,6 +508,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) dP[a][c] = 0.f;
     mm_nt<4, 4>(sm.dO, LDX, sm.V, LDX, HD, dP);
+    if (MECH == M_SHAW && p.shaw_v) value_dp<false, T>(p, sm, h, i0, j0, dmin, dmax, dP);
     probs_and_ds<false>(sm, S, dP, dS);
     __syncthreads();  // everyone is done reading W / T of the score stage
 #pragma unroll
@@ -518,6 +563,26 @@ __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
           if (w < nw) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) part[(size_t)(lo + w) * HD + tx + 16 * e] += p.scale * G[a][e];
+          }
+        }
+        if (MECH == M_SHAW && p.shaw_v) {  // daV[rho] += sum_i Pe[i][rho] dO_i (Pe: P by table row)
+          __syncthreads();
+          zero_W(sm.W, 0);
+          __syncthreads();
+          scatter_E<MECH, false, false>(p, S, sm.W, i0, j0, lo, nw);
+          __syncthreads();
+#pragma unroll
+          for (int a = 0; a < 8; ++a)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) G[a][e] = 0.f;
+          mm_tn<8, 4>(sm.W, WS, sm.dO, LDX, BM, G);
+#pragma unroll
+          for (int a = 0; a < 8; ++a) {
+            const int w = ty + 16 * a;
+            if (w < nw) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) partv[(size_t)(lo + w) * HD + tx + 16 * e] += G[a][e];
+            }
           }
         }
       }
@@ -588,6 +653,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_kv_kernel(Prm p) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) dP[a][c] = 0.f;
     mm_nt<4, 4>(sm.V, LDX, sm.dO, LDX, HD, dP);
+    if (MECH == M_SHAW && p.shaw_v) value_dp<true, T>(p, sm, h, i0, j0, dmin, dmax, dP);
     probs_and_ds<true>(sm, S, dP, dS);
     __syncthreads();
 #pragma unroll
@@ -855,6 +921,10 @@ static cudaError_t run_bwd_t(const Prm &p, cudaStream_t st) {
   const size_t n = (size_t)p.H * p.nrows * HD;
   reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_row, p.drel0);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (MECH == M_SHAW && p.shaw_v) {
+    reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_val, p.drel1);
+    return cudaGetLastError();
+  }
   if (MECH == M_DEB) {
     reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_col, p.drel1);
     return cudaGetLastError();

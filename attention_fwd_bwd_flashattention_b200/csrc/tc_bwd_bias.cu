@@ -592,15 +592,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_bias_q_kernel(const __grid
   }
 }
 
-// dt[h][b] (ALiBi: dm[h]) = sum over batches and query tiles of the partials, in a fixed order
+// dt[h][b] (ALiBi: dm[h]) = sum over batches and query tiles of the partials, in a fixed
+// order: one warp per output, lane l takes partials l, l + 32, ..., then a shuffle tree
 __global__ void reduce_bias_kernel(Prm p, const float *part) {
-  const int x = blockIdx.x * blockDim.x + threadIdx.x;
+  const int x = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (x >= p.H * p.nb) return;
-  const int h = x / p.nb, b = x % p.nb;
+  const int h = x / p.nb, b = x % p.nb, n = p.B * p.nT;
   float acc = 0.f;
-  for (int bb = 0; bb < p.B; ++bb)
-    for (int m = 0; m < p.nT; ++m) acc += part[(((size_t)bb * p.H + h) * p.nT + m) * p.nb + b];
-  p.drel0[x] = acc;
+  for (int t = lane; t < n; t += 32) {
+    const int bb = t / p.nT, m = t % p.nT;
+    acc += part[(((size_t)bb * p.H + h) * p.nT + m) * p.nb + b];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) p.drel0[x] = acc;
 }
 
 // Smallest a in [1, L - 1] from which every offset sign * a' (a' >= a) has the bias of
@@ -662,7 +667,7 @@ cudaError_t tc_bwd_bias(const Prm &p0, cudaStream_t st) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   tc_bwd_bias_q_kernel<<<tiles, NTHREADS, qb::SMEM, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reduce_bias_kernel<<<(unsigned)((p0.H * p0.nb + 255) / 256), 256, 0, st>>>(a.p, a.part);
+  reduce_bias_kernel<<<(unsigned)((p0.H * p0.nb + 7) / 8), 256, 0, st>>>(a.p, a.part);
   return cudaGetLastError();
 }
 

@@ -45,6 +45,7 @@ class Workload:
     shaw_clip: int = 64
     deberta_span: int = 256
     seqlens_k: Optional[Tuple[int, ...]] = None  # per-batch key lengths (variable-length batch)
+    shaw_value: bool = False  # Shaw: also the value-side table aV
 
     @property
     def scale(self) -> float:
@@ -71,6 +72,9 @@ for _L in (4096, 8192, 16384, 32768):
 WORKLOADS["txl_varlen_B4_L8192_bf16"] = Workload("txl_varlen_B4_L8192_bf16", TXL, torch.bfloat16, False, 4, 8, 8192,
                                                  seqlens_k=(8192, 6144, 4000, 2500))
 # ALiBi, causal decoder shape at 8K, and T5 at the same size for comparison.
+# Shaw with its value-side table as well (CUDA-core kernels), the Shaw shape at 2K.
+WORKLOADS["shaw_value_L2048_bf16"] = Workload("shaw_value_L2048_bf16", SHAW, torch.bfloat16, False, 2, 8, 2048,
+                                              shaw_value=True)
 WORKLOADS["alibi_causal_L8192_bf16"] = Workload("alibi_causal_L8192_bf16", ALIBI, torch.bfloat16, True, 1, 8, 8192)
 WORKLOADS["t5_causal_L8192_bf16"] = Workload("t5_causal_L8192_bf16", T5, torch.bfloat16, True, 1, 8, 8192,
                                              t5_bidirectional=False)
@@ -91,7 +95,7 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
     """All inputs of one workload as CPU tensors in the workload's dtype.
 
     Returns dict(q, k, v, do, rel) with rel the list of relative parameters:
-    T5 [t (H,nb) fp32]; Shaw [a (H,2c+1,d)]; TXL [r (H,n_off,d), u (H,d), v (H,d)];
+    T5 [t (H,nb) fp32]; Shaw [a (H,2c+1,d)] (+ aV with the value term); TXL [r (H,n_off,d), u (H,d), v (H,d)];
     DeBERTa [Kr (H,2k,d), Qr (H,2k,d)]; ALiBi [m (H,) fp32].
     """
     g = torch.Generator(device="cpu").manual_seed(seed)
@@ -111,6 +115,8 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
         rel = [nrm(H, wl.t5_num_buckets, std=0.1)]
     elif wl.mech == SHAW:
         rel = [nrm(H, 2 * wl.shaw_clip + 1, d, std=0.02).to(dt)]
+        if wl.shaw_value:
+            rel.append(nrm(H, 2 * wl.shaw_clip + 1, d, std=0.02).to(dt))
     elif wl.mech == TXL:
         n_off = L if wl.causal else 2 * L - 1
         W_R = nrm(TXL_EMB, H * d, std=0.02).to(torch.float64)

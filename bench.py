@@ -68,6 +68,8 @@ def algo_flops(wl):
         return 2 * U, 5 * U
     if wl.mech == SHAW:
         r = R(2 * wl.shaw_clip + 1)
+        if wl.shaw_value:  # value side: Pe aV forward; dO aV^T and Pe^T dO backward
+            return 2 * U + 2 * r, 5 * U + 5 * r
         return 2 * U + r, 5 * U + 3 * r
     if wl.mech == TXL:
         return 3 * U, 8 * U
@@ -205,8 +207,9 @@ def oracle_sample(wl, rows_fraction=None):
     inp = make_inputs(one, 0)
     q, k, v, do = (to_f64(inp[n]) for n in ("q", "k", "v", "do"))
     rel = [to_f64(r) for r in inp["rel"]]
-    cfg = orc.RelCfg(t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance, shaw_clip=wl.shaw_clip,
-                     deberta_span=wl.deberta_span)
+    cfg = orc.RelCfg(t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance,
+                     t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span,
+                     shaw_value=wl.shaw_value)
     f_fwd, f_bwd = algo_flops(one)
     t0 = time.perf_counter()
     if rows_fraction is None:
@@ -263,7 +266,8 @@ def run_ours(args, wl):
     P = bd.Params(mech=wl.mech, B=wl.B, H=wl.H, L=wl.L, d=wl.d,
                   dtype=bd.BF16 if wl.dtype == torch.bfloat16 else bd.F32, causal=wl.causal, scale=wl.scale,
                   kernel_path=path, t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance,
-                  shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+                  t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span,
+                  shaw_value=wl.shaw_value)
     if wl.seqlens_k is not None:
         P.seqlens_k = torch.tensor(wl.seqlens_k, dtype=torch.int32, device=dev)
     inp = make_inputs(wl, seed=rank)

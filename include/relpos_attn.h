@@ -39,7 +39,7 @@
  *     (float32 or bfloat16).  d must be 64.
  *   - Relative parameters rel[0..2] (contiguous, params' dtype unless noted):
  *       T5       rel[0] = t  [H, num_buckets]            float32 always
- *       Shaw     rel[0] = a  [H, 2c + 1, d]
+ *       Shaw     rel[0] = a  [H, 2c + 1, d]  (+ rel[1] = aV [H, 2c + 1, d] with shaw_value)
  *       TXL      rel[0] = r  [H, n_off, d]  (n_off = L causal, 2L - 1 otherwise),
  *                rel[1] = u  [H, d], rel[2] = v [H, d]
  *       DeBERTa  rel[0] = Kr [H, 2k, d], rel[1] = Qr [H, 2k, d]
@@ -120,6 +120,13 @@ typedef struct relpos_params {
    * must stay valid until they finish.  Variable-length speech batches: article
    * "结构感知内核让相对位置注意力加速21倍", section "为什么相对位置注意力难做快". */
   const int32_t *seqlens_k;
+  /* Shaw only (0 or 1): 1 adds the value-side term of Shaw et al.,
+   *     O_i = sum_j P_ij (v_j + aV[h, clip(j - i, -c, c) + c]),
+   * with rel[1] = aV [H, 2c + 1, d] (params' dtype) and drel[1] = daV (float32).
+   * The paper's Hugging Face page names Shaw among the mechanisms the method covers
+   * (Community comment); the value side is the second table of Shaw's own paper.
+   * Such calls run on the CUDA-core kernels (RELPOS_PATH_TC is rejected). */
+  int32_t shaw_value;
 } relpos_params_t;
 
 /* Bytes of device workspace a call needs.  pass: 0 forward, 1 backward.

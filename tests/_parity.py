@@ -13,13 +13,14 @@ TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 
 def oracle_cfg(wl):
     return orc.RelCfg(t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance, t5_bidirectional=wl.t5_bidirectional,
-                      shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+                      shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span, shaw_value=wl.shaw_value)
 
 
 def params_of(wl, path):
     return bd.Params(mech=wl.mech, B=wl.B, H=wl.H, L=wl.L, d=wl.d, dtype=bd.BF16 if wl.dtype == torch.bfloat16 else bd.F32,
                      causal=wl.causal, scale=wl.scale, kernel_path=path, t5_num_buckets=wl.t5_num_buckets,
-                     t5_max_distance=wl.t5_max_distance, t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span)
+                     t5_max_distance=wl.t5_max_distance, t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span,
+                     shaw_value=wl.shaw_value)
 
 
 def run_gpu(wl, inp, path, dev="cuda", seqlens_k=None):

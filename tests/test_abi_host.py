@@ -44,19 +44,19 @@ def test_struct_layout_matches_c(tmp_path):
     prog = tmp_path / "layout.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "relpos_attn.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
         " offsetof(relpos_params_t,scale), offsetof(relpos_params_t,t5_num_buckets), offsetof(relpos_params_t,deberta_span),"
-        " offsetof(relpos_params_t,seqlens_k));return 0;}\n")
+        " offsetof(relpos_params_t,seqlens_k), offsetof(relpos_params_t,shaw_value));return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(prog), "-o", str(exe)], check=True)
     got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     S = bd.relpos_params_t
     assert got == [ctypes.sizeof(S), S.B.offset, S.scale.offset, S.t5_num_buckets.offset, S.deberta_span.offset,
-                   S.seqlens_k.offset]
+                   S.seqlens_k.offset, S.shaw_value.offset]
 
 
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10200
+    assert lib.relpos_attn_version() == 10300
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"
@@ -64,7 +64,8 @@ def test_version_and_strerror(lib):
 
 @pytest.mark.parametrize("bad", [dict(d=32), dict(mech=5), dict(L=0), dict(B=0), dict(dtype=5), dict(scale=float("nan")),
                                  dict(kernel_path=9), dict(mech=0, t5_num_buckets=1), dict(mech=0, t5_max_distance=4),
-                                 dict(mech=3, deberta_span=0), dict(mech=1, shaw_clip=-1)])
+                                 dict(mech=3, deberta_span=0), dict(mech=1, shaw_clip=-1), dict(shaw_value=2),
+                                 dict(mech=0, shaw_value=1)])
 def test_invalid_params_rejected(lib, bad):
     kw = dict(mech=1, B=1, H=2, L=64)
     kw.update(bad)
@@ -150,6 +151,11 @@ def test_resolved_paths(lib):
     # DeBERTa: spans that are multiples of 32 up to 256 take the tensor-core backward
     for span, want_b in ((256, TC), (32, TC), (96, TC), (24, SIMT), (288, SIMT)):
         assert bd.relpos_attn_resolved_path(bd.Params(mech=bd.DEBERTA, B=1, H=2, L=300, deberta_span=span), 1) == want_b, span
+    # Shaw's value-side term: CUDA-core kernels in both passes
+    Pv = bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True)
+    assert (bd.relpos_attn_resolved_path(Pv, 0), bd.relpos_attn_resolved_path(Pv, 1)) == (SIMT, SIMT)
+    with pytest.raises(bd.RelposError):
+        bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, kernel_path=bd.PATH_TC), 0)
     wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == SIMT
     assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC

@@ -55,6 +55,26 @@ def test_parity_deberta_span256(path):
     compare_full(wl, inp, run_gpu(wl, inp, path))
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("clip,L", [(3, 17), (3, 130), (64, 300), (100, 257)])
+def test_parity_shaw_value_term(clip, L, causal, dtype):
+    """Shaw with the value-side table aV: O, LSE, dQ, dK, dV, da and daV."""
+    wl = Workload("shaw_val", SHAW, dtype, causal, 2, 2, L, shaw_clip=clip, shaw_value=True)
+    inp = make_inputs(wl, clip + L)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+def test_parity_shaw_value_term_key_lengths_and_full_size():
+    wl = Workload("shaw_val_len", SHAW, torch.bfloat16, False, 3, 2, 500, shaw_clip=20, shaw_value=True)
+    lens = (500, 0, 201)
+    inp = make_inputs(wl, 7)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO, seqlens_k=lens), seqlens_k=lens)
+    wl = WORKLOADS["shaw_value_L2048_bf16"]
+    inp = make_inputs(wl, 0)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO), heads=slice(0, 2))
+
+
 @pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
 @pytest.mark.parametrize("span", [32, 96, 160, 256])
 @pytest.mark.parametrize("L", [130, 700, 1100])
