@@ -304,14 +304,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
         auto pds = [&](auto masked) {
 #pragma unroll
-          for (int hq = 0; hq < NC / 16; ++hq) {
-            uint32_t rs[16], rp[16];
-            tmem_ld16(tl + T_S + cb + 16 * hq, rs);
-            tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+          for (int hq = 0; hq < NC / 8; ++hq) {
+            uint32_t rs[8], rp[8];
+            tmem_ld8(tl + T_S + cb + 8 * hq, rs);
+            tmem_ld8(tl + T_DP + cb + 8 * hq, rp);
             tmem_wait_ld();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const int x0 = 16 * hq + 4 * c4;
+            for (int c4 = 0; c4 < 2; ++c4) {
+              const int x0 = 8 * hq + 4 * c4;
               const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + x0);
               const float4 uk = *reinterpret_cast<const float4 *>(vec + cb + x0);
               float y[4], pr[4], dd[4];

@@ -256,14 +256,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
         const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
         auto pds = [&](auto masked, auto banded) {
 #pragma unroll
-          for (int hq = 0; hq < NC / 16; ++hq) {
-            uint32_t rs[16], rp[16];
-            tmem_ld16(tl + T_S + cb + 16 * hq, rs);
-            tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+          for (int hq = 0; hq < NC / 8; ++hq) {
+            uint32_t rs[8], rp[8];
+            tmem_ld8(tl + T_S + cb + 8 * hq, rs);
+            tmem_ld8(tl + T_DP + cb + 8 * hq, rp);
             tmem_wait_ld();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const int x0 = 16 * hq + 4 * c4;
+            for (int c4 = 0; c4 < 2; ++c4) {
+              const int x0 = 8 * hq + 4 * c4;
               float R[4], y[4], pr[4], dd[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
@@ -531,14 +531,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
         const float rend = band ? 0.f : rrow[m > n ? 0 : 2 * cl];
         auto pds = [&](auto masked, auto banded) {
 #pragma unroll
-          for (int hq = 0; hq < NC / 16; ++hq) {
-            uint32_t rs[16], rp[16];
-            tmem_ld16(tl + T_S + cb + 16 * hq, rs);
-            tmem_ld16(tl + T_DP + cb + 16 * hq, rp);
+          for (int hq = 0; hq < NC / 8; ++hq) {
+            uint32_t rs[8], rp[8];
+            tmem_ld8(tl + T_S + cb + 8 * hq, rs);
+            tmem_ld8(tl + T_DP + cb + 8 * hq, rp);
             tmem_wait_ld();
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const int x0 = 16 * hq + 4 * c4;
+            for (int c4 = 0; c4 < 2; ++c4) {
+              const int x0 = 8 * hq + 4 * c4;
               float R[4], y[4], pr[4], dd[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
