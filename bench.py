@@ -136,17 +136,24 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        t_end = time.time() + 5.0  # let the sampler produce its first line before the timed region
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        """Wall-clock bounds of the timed region: only samples read in it count."""
+        self.t0, self.t1 = t0, t1
 
     def stop(self):
         if self.proc is None:
@@ -160,7 +167,9 @@ class ClockSampler:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
+        inside = [ln for ts, ln in self.lines if t0 <= ts <= t1 + 0.15]  # a line is read just after its sample
+        for ln in inside:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -228,11 +237,12 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    frac = (1 / 64) * min(1.0, 20 / max(1, args.steps))  # bounded total CPU time for any --steps
     for _ in range(args.warmup):
-        oracle_sample(wl, rows_fraction=1 / 64)
+        oracle_sample(wl, rows_fraction=frac)
     secs, flops = 0.0, 0.0
     for _ in range(args.steps):
-        s, f, sample = oracle_sample(wl, rows_fraction=1 / 64)
+        s, f, sample = oracle_sample(wl, rows_fraction=frac)
         secs += s
         flops += f
     value = flops / secs / 1e12
@@ -299,6 +309,7 @@ def run_ours(args, wl):
     clocks.start()
     rdist.barrier()
     torch.cuda.synchronize()
+    t_wall0 = time.time()
     for s in range(args.steps):
         flush.fill_(float(s))
         ev[s][0].record(stream)
@@ -309,6 +320,7 @@ def run_ours(args, wl):
             rdist.allreduce_table_grads(drel)
         ev[s][2].record(stream)
     torch.cuda.synchronize()
+    clocks.mark(t_wall0, time.time())
     rdist.barrier()
     clk = clocks.stop()
     fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
@@ -384,54 +396,81 @@ def run_ours(args, wl):
 
 
 def run_e2e(args, wl, P, inp, dev, stream, world):
-    """Same metric through the public entry points, with the step's inputs copied
-    from pinned host memory and its results (dQ, dK, dV, drel) copied back."""
+    """Same metric through the public entry points, with every step's inputs copied
+    from pinned host memory and its results (dQ, dK, dV, drel) copied back.  Steps are
+    pipelined over two buffer sets: step k's host-to-device copies (one stream) and
+    step k - 1's device-to-host copies (another) overlap step k - 1's / k's kernels (the
+    compute stream); events order every reuse of a buffer.  The timed region runs from
+    the first input copy to the last result copy."""
     host_in = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
     host_rel = [r.pin_memory() for r in inp["rel"]]
-    q, k, v, do = (torch.empty_like(host_in[n], device=dev) for n in ("q", "k", "v", "do"))
-    rel = [torch.empty_like(r, device=dev) for r in host_rel]
     ws_f = bd.workspace(P, 0, dev)
     ws_b = bd.workspace(P, 1, dev)
-    o = torch.empty_like(q)
-    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    drel = [torch.empty(r.shape, dtype=torch.float32, device=dev) for r in rel[: P.n_rel()]]
-    out_host = [torch.empty_like(t, device="cpu").pin_memory() for t in [dq, dk, dv] + drel]
+
+    def buffers():
+        b = {n: torch.empty_like(host_in[n], device=dev) for n in ("q", "k", "v", "do")}
+        b["rel"] = [torch.empty_like(r, device=dev) for r in host_rel]
+        b["o"] = torch.empty_like(b["q"])
+        b["lse"] = torch.empty(b["q"].shape[:3], dtype=torch.float32, device=dev)
+        b["dq"], b["dk"], b["dv"] = (torch.empty_like(b["q"]) for _ in range(3))
+        b["drel"] = [torch.empty(r.shape, dtype=torch.float32, device=dev) for r in b["rel"][: P.n_rel()]]
+        b["out"] = [torch.empty_like(t, device="cpu").pin_memory() for t in [b["dq"], b["dk"], b["dv"]] + b["drel"]]
+        return b
+
+    bufs = [buffers(), buffers()]
     h2d = sum(t.numel() * t.element_size() for t in list(host_in.values()) + host_rel)
-    d2h = sum(t.numel() * t.element_size() for t in out_host)
+    d2h = sum(t.numel() * t.element_size() for t in bufs[0]["out"])
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def step():
-        for dst, src in zip([q, k, v, do], [host_in[n] for n in ("q", "k", "v", "do")]):
-            dst.copy_(src, non_blocking=True)
-        for dst, src in zip(rel, host_rel):
-            dst.copy_(src, non_blocking=True)
-        bd.relpos_attn_fwd(P, q, k, v, rel, o, lse, ws_f, stream=stream)
-        bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, ws_b, stream=stream)
-        if world > 1:
-            rdist.allreduce_table_grads(drel)
-        for dst, src in zip(out_host, [dq, dk, dv] + drel):
-            dst.copy_(src, non_blocking=True)
+    def step(kk):
+        i = kk & 1
+        B = bufs[i]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_done[i])  # the kernels of step kk - 2 are done with these inputs
+            for n in ("q", "k", "v", "do"):
+                B[n].copy_(host_in[n], non_blocking=True)
+            for dst, src in zip(B["rel"], host_rel):
+                dst.copy_(src, non_blocking=True)
+            ev_in[i].record(s_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[i])
+            stream.wait_event(ev_out[i])  # step kk - 2's results have left these buffers
+            bd.relpos_attn_fwd(P, B["q"], B["k"], B["v"], B["rel"], B["o"], B["lse"], ws_f, stream=stream)
+            bd.relpos_attn_bwd(P, B["q"], B["k"], B["v"], B["rel"], B["o"], B["lse"], B["do"], B["dq"], B["dk"], B["dv"],
+                               B["drel"], ws_b, stream=stream)
+            if world > 1:
+                rdist.allreduce_table_grads(B["drel"])
+            ev_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i])
+            for dst, src in zip(B["out"], [B["dq"], B["dk"], B["dv"]] + B["drel"]):
+                dst.copy_(src, non_blocking=True)
+            ev_out[i].record(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        step()
+    for kk in range(max(1, args.warmup)):
+        step(kk)
     torch.cuda.synchronize()
     rdist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
+    e0.record(s_in)
+    for kk in range(args.steps):
+        step(kk)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = rdist.max_over_ranks(e0.elapsed_time(e1)) / args.steps
     f_fwd, f_bwd = algo_flops(wl)
     return {"value": world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipeline": "two buffer sets; host-to-device, kernels and device-to-host on three streams"}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)  # about half a second of timed work at the default workload
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
