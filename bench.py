@@ -85,7 +85,7 @@ def fa_flops(wl):
 def kernel_launches(wl, path):
     """Kernels this library launches per forward and per backward call (the dispatch of csrc/api.cu)."""
     t5 = 1 if wl.mech in (T5, ALIBI) else 0  # per-call per-offset bias preparation
-    tc = path != "simt" and wl.dtype == torch.bfloat16
+    tc = path != "simt" and wl.dtype == torch.bfloat16 and not wl.shaw_value  # the value side runs on CUDA cores
     if tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
         fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
     else:
@@ -98,8 +98,8 @@ def kernel_launches(wl, path):
         bwd = 5
     elif tc and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction
         bwd = 7
-    else:  # D, key-tile, query-tile, then the table-gradient reductions
-        bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[wl.mech]
+    else:  # D, key-tile, query-tile, then the table-gradient reductions (Shaw's value side: one more)
+        bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[wl.mech] + (1 if wl.shaw_value else 0)
     return fwd, bwd
 
 
