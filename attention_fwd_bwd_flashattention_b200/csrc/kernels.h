@@ -14,6 +14,7 @@ struct TcWork {
   float *part_kv, *part_dg;      // backward partials (Transformer-XL)
   float *part_uv;                // [H][ceil(rows / 32)][64] dv partials per 32-offset tile
   float *qa;                     // Shaw backward: [B,H,L][132] per-row products q_i . a_rho
+  void *etiles;                  // Transformer-XL backward: the query-tile kernel's E tiles (or null)
   // DeBERTa backward: relation products QKr, KQr and dS K, dS^T Q (fp32), the
   // offset-ordered dS copies M, N (bf16, [B,H,L][2k]) and the table-gradient partials
   float *qkr, *kqr, *dqc, *dkc, *dpart;
@@ -24,6 +25,7 @@ cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st);
 cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st);
 cudaError_t tc_bwd(const Prm &p, const TcWork &w, cudaStream_t st);
 size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats);
+size_t tc_bwd_etile_bytes(const Prm &p);
 bool tc_bwd_shaw_supported(const Prm &p);
 size_t tc_bwd_shaw_qa_floats(const Prm &p);
 cudaError_t tc_bwd_shaw(const Prm &p, const TcWork &w, cudaStream_t st);

@@ -107,9 +107,6 @@ def kernel_launches(wl, path):
 # capture of the same build and workload, summed over the pass's captured kernels; set to
 # None whenever those kernels change.  Source: profiles/tc_kernels_txl_causal_L8192.md.
 DRAM_TRAFFIC = {
-    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (306.21e6, "tc_bwd_kv + tc_bwd_q + tc_bwd_diag + reduce_dr "
-                                                   "(the relation prep, D and u/v reduction kernels, about 35 MB "
-                                                   "of algorithmic traffic, were not captured)"),
     ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.21e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
 }
 
