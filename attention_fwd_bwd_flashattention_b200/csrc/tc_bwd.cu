@@ -52,6 +52,9 @@ struct BwdArgs {
   int dg_ch, dg_nchunk, nbands;
   CUtensorMap me;        // stored E tiles: [planes][128][64] bf16, four planes (16 KB) per tile
   int e_stored;          // 1: the query-tile kernel stores E and the diagonal partials come from it
+  CUtensorMap mpd;       // stored P / dS tiles, same plane layout (P keys 0-63, 64-127, dS likewise)
+  __nv_bfloat16 *pd;     // their base
+  int pd_stored;         // 1: the query-tile kernel stores P and dS and dK / dV come from them
 };
 
 // First of the four 16 KB planes (E_lo columns 0-63, 64-127, E_hi likewise) of tile (m, n)
@@ -420,6 +423,169 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
 }
 
 // ============================================================================
+// key-tile kernel from stored P / dS: dV += P^T dO, [dK | c] += dS^T [Q | 1] streaming the
+// query-tile kernel's tiles (no recompute); the same epilogue as tc_bwd_kv_kernel
+// ============================================================================
+namespace kvs {
+constexpr int OFF_P = 0;                    // 2 stages x 64 KB: P (two 64-key halves), dS at +32 KB
+constexpr int OFF_Q = 2 * 65536;            // 2 stages x 16 KB
+constexpr int OFF_DO = OFF_Q + 32768;       // 2 stages x 16 KB
+constexpr int OFF_ONES = OFF_DO + 32768;    // 128 x 64 bf16 ones (second N atom of [Q | 1])
+constexpr int OFF_VEC = OFF_ONES + 16384;   // c_j of the tile's keys (du)
+constexpr int OFF_BAR = OFF_VEC + 512;
+constexpr int SMEM = OFF_BAR + 256 + 1024;
+constexpr int NTH = 160;  // four epilogue warps (TMEM lane quarters = keys) and one control warp
+enum { B_LD0 = 0, B_LD1, B_FR0, B_FR1, B_DONE, B_DRAIN, NB };
+constexpr uint32_t T_DV = 0, T_DK = 64;  // dK | c: 80 columns
+}  // namespace kvs
+
+__global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_constant__ BwdArgs A) {
+  using namespace kvs;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Prm &p = A.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int BH = p.B * p.H;
+  const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH, h = bh % p.H;
+  const int L = p.L, j0 = n * 128;
+  const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
+  const int klen = key_len(p, bh / p.H);
+  if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0, no du contribution (whole CTA, no barrier yet)
+    for (int x = tid; x < 128 * (HD / 8); x += NTH) {
+      const int r = x / (HD / 8), c8 = x % (HD / 8);
+      if (j0 + r < L) {
+        const size_t off = ((size_t)bh * L + j0 + r) * HD + 8 * c8;
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dk + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>((__nv_bfloat16 *)p.dv + off) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    if (tid < HD) A.part_kv[((size_t)bh * p.nT + n) * HD + tid] = 0.f;
+    return;
+  }
+  const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NB);
+  float *vec = (float *)(smem + OFF_VEC);
+  int32_t *status = p.status;
+  if (tid == 0) {
+    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  for (int x = tid; x < 16384 / 16; x += NTH) {
+    const uint32_t one2 = 0x3F803F80u;
+    *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
+  }
+  fence_async_smem();
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  if (warp == 4) {
+    if (lane == 0) {
+      Ctl ctl;
+      ctl.np = 0;
+      ctl.ab = abort_flag;
+      ctl.st = status;
+      prefetch_tmap(&A.mpd);
+      prefetch_tmap(&A.mq);
+      prefetch_tmap(&A.mdo);
+      const uint32_t idAcc = idesc_bf16(128, 64, true, true);
+      const uint32_t idK = idesc_bf16(128, 80, true, true);
+      auto issue = [&](int t) {
+        const int st = t & 1, m = mStart + t, pl = e_plane(p, bh, m, n);
+        ctl.expect(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1), 65536u + 32768u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tma_load_3d(sbase + OFF_P + 65536 * st + 16384 * q, &A.mpd, BAR(B_LD0 + st), 0, 0, pl + q);
+        tma_load_3d(sbase + OFF_Q + 16384 * st, &A.mq, BAR(B_LD0 + st), 0, m * 128, bh);
+        tma_load_3d(sbase + OFF_DO + 16384 * st, &A.mdo, BAR(B_LD0 + st), 0, m * 128, bh);
+      };
+      issue(0);
+      if (iters > 1) issue(1);
+      for (int t = 0; t < iters; ++t) {
+        const int st = t & 1;
+        if (!ctl.wait_load(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t lbo = (uint32_t)(OFF_ONES - OFF_Q - 16384 * st);  // Q atom -> ones atom
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
+          umma_bf16(tbase + T_DV, sdesc_sw128(sbase + OFF_P + 65536 * st + 2048 * k, 16384, 1024),
+                    sdesc_sw128(sbase + OFF_DO + 16384 * st + 2048 * k, 16, 1024), idAcc, acc);
+          umma_bf16(tbase + T_DK, sdesc_sw128(sbase + OFF_P + 65536 * st + 32768 + 2048 * k, 16384, 1024),
+                    sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, lbo, 1024), idK, acc);
+        }
+        umma_commit(BAR(B_FR0 + st));
+        if (t + 2 < iters) {  // this stage is free once its MMAs are done
+          if (!ctl.wait(BAR(B_FR0 + st), (uint32_t)((t >> 1) & 1))) break;
+          issue(t + 2);
+        }
+      }
+      umma_commit(BAR(B_DONE));
+      ctl.drain(BAR(B_DRAIN));
+    }
+    __syncwarp();
+  } else {  // epilogue: lane il is key j0 + il; this thread takes all 64 columns
+    const int il = 32 * warp + lane, j = j0 + il;
+    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
+    float csum = 0.f;
+    if (warp_wait(BAR(B_DONE), 0, abort_flag, status)) {
+      tc_fence_after();
+      uint32_t c8r[8];
+      tmem_ld8(tl + T_DK + 64, c8r);
+      tmem_wait_ld();
+      csum = j < L ? u2f(c8r[0]) : 0.f;
+      const __nv_bfloat16 *u = (const __nv_bfloat16 *)p.rel1 + (size_t)h * HD;
+#pragma unroll
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t rv[32], rk[32];
+        tmem_ld32(tl + T_DV + c0, rv);
+        tmem_ld32(tl + T_DK + c0, rk);
+        tmem_wait_ld();
+        if (j < L) {
+          __nv_bfloat16 *dvp = (__nv_bfloat16 *)p.dv + ((size_t)bh * L + j) * HD + c0;
+          __nv_bfloat16 *dkp = (__nv_bfloat16 *)p.dk + ((size_t)bh * L + j) * HD + c0;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float kv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) kv[e] = p.scale * (u2f(rk[8 * c8 + e]) + csum * __bfloat162float(u[c0 + 8 * c8 + e]));
+            uint4 wv, wk;
+            wv.x = pack_bf16x2(u2f(rv[8 * c8 + 0]), u2f(rv[8 * c8 + 1]));
+            wv.y = pack_bf16x2(u2f(rv[8 * c8 + 2]), u2f(rv[8 * c8 + 3]));
+            wv.z = pack_bf16x2(u2f(rv[8 * c8 + 4]), u2f(rv[8 * c8 + 5]));
+            wv.w = pack_bf16x2(u2f(rv[8 * c8 + 6]), u2f(rv[8 * c8 + 7]));
+            wk.x = pack_bf16x2(kv[0], kv[1]);
+            wk.y = pack_bf16x2(kv[2], kv[3]);
+            wk.z = pack_bf16x2(kv[4], kv[5]);
+            wk.w = pack_bf16x2(kv[6], kv[7]);
+            *reinterpret_cast<uint4 *>(dvp + 8 * c8) = wv;
+            *reinterpret_cast<uint4 *>(dkp + 8 * c8) = wk;
+          }
+        }
+      }
+    }
+    // du partial: s * sum_j c_j k_j over this key tile (fixed order)
+    vec[il] = csum;
+    named_bar_sync(1, 128);
+    if (tid < HD) {
+      const __nv_bfloat16 *kp = (const __nv_bfloat16 *)p.k + (size_t)bh * L * HD;
+      float acc = 0.f;
+      for (int jj = 0; jj < 128 && j0 + jj < L; ++jj) acc = fmaf(vec[jj], __bfloat162float(kp[(size_t)(j0 + jj) * HD + tid]), acc);
+      A.part_kv[((size_t)bh * p.nT + n) * HD + tid] = p.scale * acc;
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// ============================================================================
 // query-tile kernel: dQ
 // ============================================================================
 namespace qk {
@@ -653,6 +819,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         }
       };
       if (need_mask) probs(std::true_type{}); else probs(std::false_type{});
+      // row-major bf16 P / dS planes of this tile for the key-tile kernel: row il, keys cb .. cb + 31
+      __nv_bfloat16 *pdrow = A.pd_stored ? A.pd + (size_t)(e_plane(p, bh, m, n) + (qt >> 1)) * 8192 + il * 64 + 32 * (qt & 1)
+                                         : nullptr;
+      if (A.pd_stored && good) {
+#pragma unroll
+        for (int c8 = 0; c8 < NC / 8; ++c8)
+          *reinterpret_cast<uint4 *>(pdrow + 8 * c8) =
+              make_uint4(pack_bf16x2(x[8 * c8], x[8 * c8 + 1]), pack_bf16x2(x[8 * c8 + 2], x[8 * c8 + 3]),
+                         pack_bf16x2(x[8 * c8 + 4], x[8 * c8 + 5]), pack_bf16x2(x[8 * c8 + 6], x[8 * c8 + 7]));
+      }
       good = good && warp_wait(BAR(B_DPF), n & 1, abort_flag, status);
       if (good) {
         tc_fence_after();
@@ -675,6 +851,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        if (A.pd_stored) {
+#pragma unroll
+          for (int c8 = 0; c8 < NC / 8; ++c8)
+            *reinterpret_cast<uint4 *>(pdrow + 2 * 8192 + 8 * c8) = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+        }
         // the previous tile's dS K MMAs read T_DS: wait for them (long done in practice)
         if (n >= 1 && !warp_wait(BAR(B_DSFREE), (n - 1) & 1, abort_flag, status)) good = false;
         if (good) tmem_st16(tl + T_DS + 16 * qt, pk);
@@ -1248,13 +1429,13 @@ void tc_bwd_shape(const Prm &p, int &nT, int &nbands, int &ch, int &nchunk) {
   nchunk = (nT + ch - 1) / ch;
 }
 
-// Bytes of the stored-E buffer (64 KB per tile of the backward), or 0 when over 16 GiB (the
-// diagonal kernel then recomputes E).
+// Bytes of each stored-tile buffer (E; P and dS): 64 KB per tile of the backward, or 0 when
+// the two together would exceed 16 GiB (the key-tile and diagonal kernels then recompute).
 size_t tc_bwd_etile_bytes(const Prm &p) {
   const size_t nT = ((size_t)p.L + 127) / 128;
   const size_t ntiles = p.causal ? nT * (nT + 1) / 2 : nT * nT;
   const size_t bytes = (size_t)p.B * p.H * ntiles * 65536;
-  return bytes <= ((size_t)16 << 30) ? bytes : 0;
+  return 2 * bytes <= ((size_t)16 << 30) ? bytes : 0;
 }
 
 size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats) {
@@ -1286,6 +1467,9 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   const uint64_t BH = (uint64_t)p0.B * p0.H;
   a.e_stored = w.etiles != nullptr;
   if (a.e_stored && !tc_make_map(&a.me, w.etiles, 128, tc_bwd_etile_bytes(p0) / 16384, 128)) return cudaErrorInvalidValue;
+  a.pd_stored = a.e_stored && w.pdtiles != nullptr;
+  a.pd = (__nv_bfloat16 *)w.pdtiles;
+  if (a.pd_stored && !tc_make_map(&a.mpd, w.pdtiles, 128, tc_bwd_etile_bytes(p0) / 16384, 128)) return cudaErrorInvalidValue;
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
         tc_make_map(&a.mv, p0.v, p0.L, BH, 128) && tc_make_map(&a.mdo, p0.dout, p0.L, BH, 128) &&
         tc_make_map(&a.mr, p0.rel0, p0.nrows, p0.H, 128)))
@@ -1297,9 +1481,17 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_bwd_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dg::SMEM)) != cudaSuccess)
     return e;
   const unsigned tiles = (unsigned)(nT * p0.H * p0.B);
-  tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
+  if (a.pd_stored) {  // the query-tile kernel first: the key-tile pass streams its P / dS tiles
+    if ((e = cudaFuncSetAttribute(tc_bwd_kvs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess)
+      return e;
+    tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    tc_bwd_kvs_kernel<<<tiles, kvs::NTH, kvs::SMEM, st>>>(a);
+  } else {
+    tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.e_stored) {
     if ((e = cudaFuncSetAttribute(tc_bwd_dgs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dgs::SMEM)) != cudaSuccess)
