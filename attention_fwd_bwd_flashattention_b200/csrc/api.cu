@@ -151,7 +151,7 @@ struct Layout {
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
   size_t part_kv, part_dg, part_uv, qa;  // tensor-core backward partials / products
   size_t qkr, kqr, dM, dN, dqc, dkc, dpart;  // DeBERTa tensor-core backward
-  size_t etiles, pdtiles;                    // Transformer-XL tensor-core backward: stored E, P / dS tiles (0: none)
+  size_t pdtiles;                            // Transformer-XL tensor-core backward: stored P / dS tiles (0: none)
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -208,10 +208,7 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
     l.part_dg = take(sizeof(float) * dgf);
     l.part_uv = take(sizeof(float) * (size_t)p.H * ((p.nrows + 31) / 32) * rp::HD);
     const size_t eb = rp::tc_bwd_etile_bytes(p);
-    if (eb) {
-      l.etiles = take(eb);
-      l.pdtiles = take(eb);
-    }
+    if (eb) l.pdtiles = take(eb);
   } else if (pass == 1) {
     l.dvec = take(sizeof(float) * BH * p.L);
     const size_t tab = (size_t)p.nrows * rp::HD;
@@ -269,7 +266,6 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.dpart = (float *)(b + l.dpart);
   w.dM = b + l.dM;
   w.dN = b + l.dN;
-  w.etiles = l.etiles ? b + l.etiles : nullptr;
   w.pdtiles = l.pdtiles ? b + l.pdtiles : nullptr;
   return w;
 }

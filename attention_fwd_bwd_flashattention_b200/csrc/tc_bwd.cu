@@ -50,15 +50,13 @@ struct BwdArgs {
   float *part_dg;        // [B,H,nbands,nchunk][2][65][128] diagonal partials (G then g)
   float *part_uv;        // [H][ceil(rows / 32)][64] dv partials per 32-offset tile
   int dg_ch, dg_nchunk, nbands;
-  CUtensorMap me;        // stored E tiles: [planes][128][64] bf16, four planes (16 KB) per tile
-  int e_stored;          // 1: the query-tile kernel stores E and the diagonal partials come from it
-  CUtensorMap mpd;       // stored P / dS tiles, same plane layout (P keys 0-63, 64-127, dS likewise)
-  __nv_bfloat16 *pd;     // their base
-  int pd_stored;         // 1: the query-tile kernel stores P and dS and dK / dV come from them
+  CUtensorMap mpd;       // stored P / dS tiles: [planes][128][64] bf16, four 16 KB planes per tile
+  __nv_bfloat16 *pd;     // (P keys 0-63, P keys 64-127, dS likewise) and their base
+  int pd_stored;         // 1: the query-tile kernel stores P and dS; dK / dV and dr come from them
 };
 
-// First of the four 16 KB planes (E_lo columns 0-63, 64-127, E_hi likewise) of tile (m, n)
-// of (batch, head) bh in the stored-E buffer: causal tiles n <= m row by row, else all.
+// First of the four 16 KB planes of tile (m, n) of (batch, head) bh in the stored-tile
+// buffer: causal tiles n <= m row by row, else all.
 __device__ __forceinline__ int e_plane(const Prm &p, int bh, int m, int n) {
   const int ntiles = p.causal ? p.nT * (p.nT + 1) / 2 : p.nT * p.nT;
   const int idx = p.causal ? m * (m + 1) / 2 + n : m * p.nT + n;
@@ -594,7 +592,7 @@ constexpr int OFF_ROT = OFF_R + 3 * 16384;  // rot rows; E_lo at +0, E_hi at +32
 constexpr int OFF_VEC = OFF_ROT + 128 * ROT_LD * 4;
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
-enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_DPCONS, B_PDS, B_PDSFREE, B_DSFREE, B_ESFREE, B_DRAIN, NB };
+enum { B_QD = 0, B_ST0, B_ST1, B_SFULL, B_TCONS, B_DPF, B_DPCONS, B_PDS, B_PDSFREE, B_DSFREE, B_DRAIN, NB };
 constexpr uint32_t T_S = 0, T_REL = 128, T_DQ = 384, T_DS = 448;
 }  // namespace qk
 
@@ -637,7 +635,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
     mbar_init(BAR(B_PDS), NSOFT);
     mbar_init(BAR(B_PDSFREE), 1);
     mbar_init(BAR(B_DSFREE), 1);
-    mbar_init(BAR(B_ESFREE), 1);
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -659,7 +656,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       prefetch_tmap(&A.mv);
       prefetch_tmap(&A.mdo);
       prefetch_tmap(&A.mr);
-      if (A.e_stored) prefetch_tmap(&A.me);
       const uint32_t idS = idesc_bf16(128, 128, false);
       const uint32_t idDQ = idesc_bf16(128, 64, true);
       ctl.expect(BAR(B_QD), 0, 32768);
@@ -706,12 +702,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         }
         if (!ctl.wait(BAR(B_PDS), n & 1)) break;
         tc_fence_after();
-        if (A.e_stored) {  // the tile's E (offset-ordered dS) to HBM, for the diagonal partials
-          const int pl = e_plane(p, bh, m, n);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tma_store_3d(&A.me, sbase + OFF_ROT + 16384 * q, 0, 0, pl + q);
-          bulk_commit();
-        }
         // dQ += E_lo r_D + E_hi r_{D-1} (E in smem, freed first so the rows can skew the
         // next tile), then dQ += dS K_n (dS in TMEM)
         uint32_t acc = n > 0 ? 1u : 0u;
@@ -735,16 +725,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
           umma_bf16_ts(tbase + T_DQ, tbase + T_DS + 8 * k, sdesc_sw128(sbase + OFF_K + 16384 * st + 2048 * k, 16, 1024), idDQ,
                        (acc || k > 0) ? 1u : 0u);
         umma_commit(BAR(B_DSFREE));
-        if (A.e_stored) {  // the stores have read E: the rows may overwrite it
-          bulk_wait_read0();
-          mbar_arrive(BAR(B_ESFREE));
-        }
         if (n + 2 < nTiles) {  // K_n, V_n and the tile's relation block slot are free once dS K_n is done
           if (!ctl.wait(BAR(B_DSFREE), n & 1)) break;
           issue_stage(n + 2);
         }
       }
-      bulk_wait0();  // every E store is complete (none are issued without e_stored)
       ctl.drain(BAR(B_DRAIN));
     }
     __syncwarp();
@@ -773,7 +758,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
-      if (n >= 1 && A.e_stored) good = good && warp_wait(BAR(B_ESFREE), (n - 1) & 1, abort_flag, status);
       const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
       float x[NC];
       if (good) {
@@ -1176,21 +1160,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
 }
 
 // ============================================================================
-// diagonal kernel from stored E: the same partials as tc_bwd_diag_kernel, streaming the
-// query-tile kernel's E tiles of the band (no recompute of S, P or dS)
+// diagonal kernel from the stored dS tiles: the same partials as tc_bwd_diag_kernel with
+// no recompute of S, P or dS -- the rows rebuild E (offset order) from each stored dS tile
 // ============================================================================
 namespace dgs {
-constexpr int OFF_E = 0;                 // 2 stages x 64 KB: E_lo (two 64-column halves), E_hi
-constexpr int OFF_Q = 2 * 65536;         // 2 stages x 16 KB
-constexpr int OFF_ONES = OFF_Q + 32768;  // 128 x 64 bf16 ones (second N atom of [Q | 1])
+constexpr int OFF_DS = 0;                  // 2 stages x 32 KB: dS (two 64-key halves)
+constexpr int OFF_Q = 2 * 32768;           // 2 stages x 16 KB
+constexpr int OFF_E = OFF_Q + 32768;       // E_lo, E_hi (64 KB)
+constexpr int OFF_ONES = OFF_E + 65536;    // 128 x 64 bf16 ones (second N atom of [Q | 1])
 constexpr int OFF_BAR = OFF_ONES + 16384;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
-constexpr int NTH = 160;  // four epilogue warps (TMEM lane quarters) and one control warp
-enum { B_LD0 = 0, B_LD1, B_FR0, B_FR1, B_DONE, B_DRAIN, NB };
+enum { B_LD0 = 0, B_LD1, B_EFULL, B_EFREE, B_DRAIN, NB };
 constexpr uint32_t T_GLO = 0, T_GHI = 128;  // G | g: 80 columns each
 }  // namespace dgs
 
-__global__ void __launch_bounds__(dgs::NTH, 1) tc_bwd_dgs_kernel(const __grid_constant__ BwdArgs A) {
+__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_dgs_kernel(const __grid_constant__ BwdArgs A) {
   using namespace dgs;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1208,7 +1192,7 @@ __global__ void __launch_bounds__(dgs::NTH, 1) tc_bwd_dgs_kernel(const __grid_co
   const int m1 = min(m1a, (klen + 127) / 128 - 1 + D);  // the tiles the query-tile kernel stored
   float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
   if (m0 > m1) {  // the chunk's tiles are all padding: a zero partial
-    for (int x = tid; x < DG_STRIDE; x += NTH) part[x] = 0.f;
+    for (int x = tid; x < DG_STRIDE; x += NTHREADS) part[x] = 0.f;
     return;
   }
   const int iters = m1 - m0 + 1;
@@ -1218,11 +1202,11 @@ __global__ void __launch_bounds__(dgs::NTH, 1) tc_bwd_dgs_kernel(const __grid_co
   uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NB);
   int32_t *status = p.status;
   if (tid == 0) {
-    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), 1);
+    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), k == B_EFULL ? NSOFT : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int x = tid; x < 16384 / 16; x += NTH) {
+  for (int x = tid; x < 16384 / 16; x += NTHREADS) {
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
@@ -1232,20 +1216,20 @@ __global__ void __launch_bounds__(dgs::NTH, 1) tc_bwd_dgs_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  if (warp == 4) {
+  if (warp == CTRL_WARP) {
     if (lane == 0) {
       Ctl ctl;
       ctl.np = 0;
       ctl.ab = abort_flag;
       ctl.st = status;
-      prefetch_tmap(&A.me);
+      prefetch_tmap(&A.mpd);
       prefetch_tmap(&A.mq);
       const uint32_t idG = idesc_bf16(128, 80, true, true);
-      auto issue = [&](int t) {
+      auto issue = [&](int t) {  // dS planes of tile (m, m - D) and Q_m
         const int st = t & 1, m = m0 + t, pl = e_plane(p, bh, m, m - D);
-        ctl.expect(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1), 65536u + 16384u);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tma_load_3d(sbase + OFF_E + 65536 * st + 16384 * q, &A.me, BAR(B_LD0 + st), 0, 0, pl + q);
+        ctl.expect(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1), 32768u + 16384u);
+        tma_load_3d(sbase + OFF_DS + 32768 * st, &A.mpd, BAR(B_LD0 + st), 0, 0, pl + 2);
+        tma_load_3d(sbase + OFF_DS + 32768 * st + 16384, &A.mpd, BAR(B_LD0 + st), 0, 0, pl + 3);
         tma_load_3d(sbase + OFF_Q + 16384 * st, &A.mq, BAR(B_LD0 + st), 0, m * 128, bh);
       };
       issue(0);
@@ -1253,46 +1237,70 @@ __global__ void __launch_bounds__(dgs::NTH, 1) tc_bwd_dgs_kernel(const __grid_co
       for (int t = 0; t < iters; ++t) {
         const int st = t & 1;
         if (!ctl.wait_load(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1))) break;
+        if (!ctl.wait(BAR(B_EFULL), t & 1)) break;  // the rows have built E(t) (and read dS(t))
         tc_fence_after();
         const uint32_t lbo = (uint32_t)(OFF_ONES - OFF_Q - 16384 * st);  // Q atom -> ones atom
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // [G | g]_lo, [G | g]_hi += E^T [Q | 1]
           const uint32_t acc = (t > 0 || k > 0) ? 1u : 0u;
           const uint64_t bq = sdesc_sw128(sbase + OFF_Q + 16384 * st + 2048 * k, lbo, 1024);
-          umma_bf16(tbase + T_GLO, sdesc_sw128(sbase + OFF_E + 65536 * st + 2048 * k, 16384, 1024), bq, idG, acc);
-          umma_bf16(tbase + T_GHI, sdesc_sw128(sbase + OFF_E + 65536 * st + 32768 + 2048 * k, 16384, 1024), bq, idG, acc);
+          umma_bf16(tbase + T_GLO, sdesc_sw128(sbase + OFF_E + 2048 * k, 16384, 1024), bq, idG, acc);
+          umma_bf16(tbase + T_GHI, sdesc_sw128(sbase + OFF_E + 32768 + 2048 * k, 16384, 1024), bq, idG, acc);
         }
-        umma_commit(BAR(B_FR0 + st));
-        if (t + 2 < iters) {  // this stage is free once its MMAs are done
-          if (!ctl.wait(BAR(B_FR0 + st), (uint32_t)((t >> 1) & 1))) break;
+        umma_commit(BAR(B_EFREE));
+        if (t + 2 < iters) {  // stage st (dS read by the rows, Q by these MMAs) is free
+          if (!ctl.wait(BAR(B_EFREE), t & 1)) break;
           issue(t + 2);
         }
       }
-      umma_commit(BAR(B_DONE));
       ctl.drain(BAR(B_DRAIN));
     }
     __syncwarp();
-  } else {  // epilogue: lane il = offset c of both blocks; [block][65][128 offsets] partial layout
-    const int il = 32 * warp + lane;
-    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
-    if (warp_wait(BAR(B_DONE), 0, abort_flag, status)) {
-      tc_fence_after();
+  } else {
+    const int g = warp & 3, qt = warp >> 2, il = 32 * g + lane, cb = NC * qt;
+    const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
+    bool good = true;
+    for (int t = 0; t < iters; ++t) {
+      const int st = t & 1;
+      good = good && warp_wait(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1), abort_flag, status);
+      if (t >= 1) good = good && warp_wait(BAR(B_EFREE), (t - 1) & 1, abort_flag, status);  // E(t - 1) read
+      if (good) {
+        // this thread's 32 dS values (row il, keys cb .. cb + 31) from the swizzled stage,
+        // as bf16 pairs (x[2k+1] low, x[2k] high) for store_E
+        uint32_t ds[NC / 2];
+        const uint8_t *src = smem + OFF_DS + 32768 * st + 16384 * (qt >> 1) + 128 * il;
 #pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        const uint32_t col = blk ? T_GHI : T_GLO;
-        float *pb = part + (size_t)(65 * blk) * 128 + il;
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tl + col + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pb[(size_t)(c0 + e) * 128] = u2f(r[e]);
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(src + (((4 * (qt & 1) + c) ^ (il & 7)) << 4));
+          ds[4 * c] = prmt(v.x, v.x, 0x1032u);
+          ds[4 * c + 1] = prmt(v.y, v.y, 0x1032u);
+          ds[4 * c + 2] = prmt(v.z, v.z, 0x1032u);
+          ds[4 * c + 3] = prmt(v.w, v.w, 0x1032u);
         }
-        uint32_t g8[8];
-        tmem_ld8(tl + col + 64, g8);
-        tmem_wait_ld();
-        pb[(size_t)64 * 128] = u2f(g8[0]);
+        store_E(smem + OFF_E, il, cb, ds);
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_EFULL));
+      }
+    }
+    // ---- epilogue: lane il is offset c = il of both blocks; 16 columns per thread ----
+    good = good && warp_wait(BAR(B_EFREE), (iters - 1) & 1, abort_flag, status);
+    if (good) {
+      tc_fence_after();
+      uint32_t rlo[16], rhi[16], glo[16], ghi[16];
+      tmem_ld16(tl + T_GLO + 16 * qt, rlo);
+      tmem_ld16(tl + T_GHI + 16 * qt, rhi);
+      tmem_ld16(tl + T_GLO + 64, glo);
+      tmem_ld16(tl + T_GHI + 64, ghi);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        part[(size_t)(16 * qt + e) * 128 + il] = u2f(rlo[e]);
+        part[(size_t)(65 + 16 * qt + e) * 128 + il] = u2f(rhi[e]);
+      }
+      if (qt == 0) {
+        part[(size_t)64 * 128 + il] = u2f(glo[0]);
+        part[(size_t)(65 + 64) * 128 + il] = u2f(ghi[0]);
       }
     }
     tc_fence_before();
@@ -1429,13 +1437,13 @@ void tc_bwd_shape(const Prm &p, int &nT, int &nbands, int &ch, int &nchunk) {
   nchunk = (nT + ch - 1) / ch;
 }
 
-// Bytes of each stored-tile buffer (E; P and dS): 64 KB per tile of the backward, or 0 when
-// the two together would exceed 16 GiB (the key-tile and diagonal kernels then recompute).
+// Bytes of the stored P / dS tile buffer: 64 KB per tile of the backward, or 0 when over
+// 16 GiB (the key-tile and diagonal kernels then recompute S, P and dS).
 size_t tc_bwd_etile_bytes(const Prm &p) {
   const size_t nT = ((size_t)p.L + 127) / 128;
   const size_t ntiles = p.causal ? nT * (nT + 1) / 2 : nT * nT;
   const size_t bytes = (size_t)p.B * p.H * ntiles * 65536;
-  return 2 * bytes <= ((size_t)16 << 30) ? bytes : 0;
+  return bytes <= ((size_t)16 << 30) ? bytes : 0;
 }
 
 size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats) {
@@ -1465,9 +1473,7 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   a.part_uv = w.part_uv;
   a.p.part_small = w.part_kv;
   const uint64_t BH = (uint64_t)p0.B * p0.H;
-  a.e_stored = w.etiles != nullptr;
-  if (a.e_stored && !tc_make_map(&a.me, w.etiles, 128, tc_bwd_etile_bytes(p0) / 16384, 128)) return cudaErrorInvalidValue;
-  a.pd_stored = a.e_stored && w.pdtiles != nullptr;
+  a.pd_stored = w.pdtiles != nullptr;
   a.pd = (__nv_bfloat16 *)w.pdtiles;
   if (a.pd_stored && !tc_make_map(&a.mpd, w.pdtiles, 128, tc_bwd_etile_bytes(p0) / 16384, 128)) return cudaErrorInvalidValue;
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
@@ -1493,10 +1499,10 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
     tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (a.e_stored) {
+  if (a.pd_stored) {
     if ((e = cudaFuncSetAttribute(tc_bwd_dgs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dgs::SMEM)) != cudaSuccess)
       return e;
-    tc_bwd_dgs_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), dgs::NTH, dgs::SMEM, st>>>(a);
+    tc_bwd_dgs_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dgs::SMEM, st>>>(a);
   } else {
     tc_bwd_diag_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a);
   }

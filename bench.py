@@ -107,10 +107,6 @@ def kernel_launches(wl, path):
 # capture of the same build and workload, summed over the pass's captured kernels; set to
 # None whenever those kernels change.  Source: profiles/tc_kernels_txl_causal_L8192.md.
 DRAM_TRAFFIC = {
-    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (4722.8e6, "tc_bwd_q + tc_bwd_kvs + tc_bwd_dgs + reduce_dr (includes "
-                                                   "the 2.1 GB of stored E, P and dS tiles written once and read "
-                                                   "once; the relation prep, D and u/v reduction kernels were "
-                                                   "not captured)"),
     ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.26e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
 }
 
