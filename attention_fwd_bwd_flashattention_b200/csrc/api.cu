@@ -207,7 +207,7 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
     l.part_kv = take(sizeof(float) * kvf);
     l.part_dg = take(sizeof(float) * dgf);
     l.part_uv = take(sizeof(float) * (size_t)p.H * ((p.nrows + 31) / 32) * rp::HD);
-    const size_t eb = rp::tc_bwd_etile_bytes(p);
+    const size_t eb = rp::tc_bwd_tile_bytes(p);
     if (eb) l.pdtiles = take(eb);
   } else if (pass == 1) {
     l.dvec = take(sizeof(float) * BH * p.L);

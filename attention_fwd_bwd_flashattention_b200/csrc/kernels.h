@@ -25,7 +25,7 @@ cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st);
 cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st);
 cudaError_t tc_bwd(const Prm &p, const TcWork &w, cudaStream_t st);
 size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats);
-size_t tc_bwd_etile_bytes(const Prm &p);
+size_t tc_bwd_tile_bytes(const Prm &p);
 bool tc_bwd_shaw_supported(const Prm &p);
 size_t tc_bwd_shaw_qa_floats(const Prm &p);
 cudaError_t tc_bwd_shaw(const Prm &p, const TcWork &w, cudaStream_t st);

@@ -27,6 +27,12 @@
 //                     Kernels", Abstract, technique (3)).
 // A fixed-order reduction turns the partials into dr = s (G + g v), dv = s sum g r
 // and du = s sum_j c_j k_j.
+//
+// Stored tiles (whenever the buffer fits in 16 GiB): the query-tile kernel runs first and
+// its row threads also write every tile's P and dS (bf16, 64 KB per tile) to a workspace
+// buffer; the key-tile and diagonal work then stream those tiles instead of recomputing
+// S, P and dS (tc_bwd_kvs_kernel: dV, [dK | c] MMAs only; tc_bwd_dgs_kernel: E rebuilt in
+// smem from the stored dS, then the G MMAs).  The results are bitwise the same.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -57,7 +63,7 @@ struct BwdArgs {
 
 // First of the four 16 KB planes of tile (m, n) of (batch, head) bh in the stored-tile
 // buffer: causal tiles n <= m row by row, else all.
-__device__ __forceinline__ int e_plane(const Prm &p, int bh, int m, int n) {
+__device__ __forceinline__ int tile_plane(const Prm &p, int bh, int m, int n) {
   const int ntiles = p.causal ? p.nT * (p.nT + 1) / 2 : p.nT * p.nT;
   const int idx = p.causal ? m * (m + 1) / 2 + n : m * p.nT + n;
   return (bh * ntiles + idx) * 4;
@@ -493,7 +499,7 @@ __global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_co
       const uint32_t idAcc = idesc_bf16(128, 64, true, true);
       const uint32_t idK = idesc_bf16(128, 80, true, true);
       auto issue = [&](int t) {
-        const int st = t & 1, m = mStart + t, pl = e_plane(p, bh, m, n);
+        const int st = t & 1, m = mStart + t, pl = tile_plane(p, bh, m, n);
         ctl.expect(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1), 65536u + 32768u);
 #pragma unroll
         for (int q = 0; q < 4; ++q) tma_load_3d(sbase + OFF_P + 65536 * st + 16384 * q, &A.mpd, BAR(B_LD0 + st), 0, 0, pl + q);
@@ -804,7 +810,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       };
       if (need_mask) probs(std::true_type{}); else probs(std::false_type{});
       // row-major bf16 P / dS planes of this tile for the key-tile kernel: row il, keys cb .. cb + 31
-      __nv_bfloat16 *pdrow = A.pd_stored ? A.pd + (size_t)(e_plane(p, bh, m, n) + (qt >> 1)) * 8192 + il * 64 + 32 * (qt & 1)
+      __nv_bfloat16 *pdrow = A.pd_stored ? A.pd + (size_t)(tile_plane(p, bh, m, n) + (qt >> 1)) * 8192 + il * 64 + 32 * (qt & 1)
                                          : nullptr;
       if (A.pd_stored && good) {
 #pragma unroll
@@ -1226,7 +1232,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_dgs_kernel(const __grid_co
       prefetch_tmap(&A.mq);
       const uint32_t idG = idesc_bf16(128, 80, true, true);
       auto issue = [&](int t) {  // dS planes of tile (m, m - D) and Q_m
-        const int st = t & 1, m = m0 + t, pl = e_plane(p, bh, m, m - D);
+        const int st = t & 1, m = m0 + t, pl = tile_plane(p, bh, m, m - D);
         ctl.expect(BAR(B_LD0 + st), (uint32_t)((t >> 1) & 1), 32768u + 16384u);
         tma_load_3d(sbase + OFF_DS + 32768 * st, &A.mpd, BAR(B_LD0 + st), 0, 0, pl + 2);
         tma_load_3d(sbase + OFF_DS + 32768 * st + 16384, &A.mpd, BAR(B_LD0 + st), 0, 0, pl + 3);
@@ -1439,7 +1445,7 @@ void tc_bwd_shape(const Prm &p, int &nT, int &nbands, int &ch, int &nchunk) {
 
 // Bytes of the stored P / dS tile buffer: 64 KB per tile of the backward, or 0 when over
 // 16 GiB (the key-tile and diagonal kernels then recompute S, P and dS).
-size_t tc_bwd_etile_bytes(const Prm &p) {
+size_t tc_bwd_tile_bytes(const Prm &p) {
   const size_t nT = ((size_t)p.L + 127) / 128;
   const size_t ntiles = p.causal ? nT * (nT + 1) / 2 : nT * nT;
   const size_t bytes = (size_t)p.B * p.H * ntiles * 65536;
@@ -1475,7 +1481,7 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   const uint64_t BH = (uint64_t)p0.B * p0.H;
   a.pd_stored = w.pdtiles != nullptr;
   a.pd = (__nv_bfloat16 *)w.pdtiles;
-  if (a.pd_stored && !tc_make_map(&a.mpd, w.pdtiles, 128, tc_bwd_etile_bytes(p0) / 16384, 128)) return cudaErrorInvalidValue;
+  if (a.pd_stored && !tc_make_map(&a.mpd, w.pdtiles, 128, tc_bwd_tile_bytes(p0) / 16384, 128)) return cudaErrorInvalidValue;
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
         tc_make_map(&a.mv, p0.v, p0.L, BH, 128) && tc_make_map(&a.mdo, p0.dout, p0.L, BH, 128) &&
         tc_make_map(&a.mr, p0.rel0, p0.nrows, p0.H, 128)))
