@@ -65,6 +65,9 @@ Readings where the pages are silent (listed again in the design notes):
     masks keys j >= seqlens_k[b] of that batch (after causal masking); queries are
     all computed.  Relative positions keep their meaning (j - i over the padded
     length L), so the tables and index maps do not change.
+  * Transformer-XL memory (``txl_memory_forward`` / ``txl_memory_backward``): the L
+    queries of the current segment sit at absolute positions M .. M + L - 1 over the M
+    cached keys / values followed by the segment's L; causal, r has M + L rows.
   * Fully masked rows (an empty key set: seqlens_k[b] = 0, or a causal row whose
     keys are all padding) give O = 0 and LSE = -inf and zero gradients.
   * LSE is the natural log of the softmax denominator.
@@ -418,3 +421,38 @@ def backward_rows(mech, q, k, v, rel, causal, dO, rows, scale=None, cfg=RelCfg()
                 g += scale * (M @ tab)
             dq[b, h] = g
     return dq
+
+
+# --------------------------------------------------------------------------
+# Transformer-XL with memory (Dai et al.): the current segment's L queries attend to the
+# cached previous segment's M keys / values followed by the segment's own L; query i sits
+# at absolute position M + i, so S_ij = s ((q_i + u).k_j + (q_i + v).r[M + i - j]) for
+# keys j <= M + i (causal), and r has M + L rows.  This is exactly the causal attention of
+# the concatenated M + L positions read at its last L query rows, which is how it is
+# computed here (the first M query rows are placeholders with zero output gradient).
+# --------------------------------------------------------------------------
+def _with_memory(q, m_len):
+    B, H, L, d = q.shape
+    return np.concatenate([np.zeros((B, H, m_len, d)), np.asarray(q, dtype=np.float64)], axis=2)
+
+
+def txl_memory_forward(q, k, v, rel, scale=None, cfg=RelCfg()):
+    """O [B,H,L,d] and LSE [B,H,L] of Transformer-XL with memory: q [B,H,L,d] is the
+    current segment, k and v [B,H,M+L,d] the memory followed by the segment, rel =
+    [r (H, M+L, d), u (H, d), v (H, d)]."""
+    m_len = np.shape(k)[2] - np.shape(q)[2]
+    assert m_len >= 0, "keys must cover the memory and the segment"
+    qf = _with_memory(q, m_len)
+    rows = np.arange(m_len, qf.shape[2])
+    return forward(TXL, qf, k, v, rel, True, scale, cfg, rows=rows)
+
+
+def txl_memory_backward(q, k, v, rel, dO, scale=None, cfg=RelCfg()):
+    """Gradients (dq [B,H,L,d], dk, dv [B,H,M+L,d], drel) of sum(O * dO) for
+    txl_memory_forward; the memory's keys and values get gradients like any key."""
+    m_len = np.shape(k)[2] - np.shape(q)[2]
+    assert m_len >= 0, "keys must cover the memory and the segment"
+    qf = _with_memory(q, m_len)
+    gf = _with_memory(dO, m_len)
+    dq, dk, dv, drel = backward(TXL, qf, k, v, rel, True, gf, scale, cfg)
+    return dq[:, :, m_len:], dk, dv, drel

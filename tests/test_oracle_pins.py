@@ -504,3 +504,78 @@ def test_batch_sums_table_grads():
         parts = [orc.backward(mech, q[b:b + 1], k[b:b + 1], v[b:b + 1], rel, False, do[b:b + 1], 0.5, cfg)[3] for b in range(2)]
         for n in range(len(rel)):
             np.testing.assert_allclose(dr[n], parts[0][n] + parts[1][n], rtol=1e-12, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# Transformer-XL with memory (keys: M cached positions, then the L of the segment)
+# ----------------------------------------------------------------------------
+def brute_txl_memory(q, k, v, rel, do, s):
+    """Scalar loops: query i at absolute position M + i, keys j <= M + i,
+    S_ij = s ((q_i + u).k_j + (q_i + v).r[M + i - j])."""
+    r, u, vv = rel
+    B, H, L, d = q.shape
+    LK = k.shape[2]
+    M = LK - L
+    O = np.zeros_like(q)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    drel = [np.zeros_like(x) for x in rel]
+    for b in range(B):
+        for h in range(H):
+            for i in range(L):
+                a = M + i
+                keys = list(range(a + 1))
+                sc = [s * (dot(q[b, h, i] + u[h], k[b, h, j]) + dot(q[b, h, i] + vv[h], r[h][a - j])) for j in keys]
+                mx = max(sc)
+                z = sum(math.exp(x - mx) for x in sc)
+                P = [math.exp(x - mx) / z for x in sc]
+                O[b, h, i] = sum(pj * v[b, h, j] for pj, j in zip(P, keys))
+                Di = dot(do[b, h, i], O[b, h, i])
+                for pj, j in zip(P, keys):
+                    dS = pj * (dot(do[b, h, i], v[b, h, j]) - Di)
+                    dv[b, h, j] += pj * do[b, h, i]
+                    dq[b, h, i] += s * dS * (k[b, h, j] + r[h][a - j])
+                    dk[b, h, j] += s * dS * (q[b, h, i] + u[h])
+                    drel[0][h][a - j] += s * dS * (q[b, h, i] + vv[h])
+                    drel[1][h] += s * dS * k[b, h, j]
+                    drel[2][h] += s * dS * r[h][a - j]
+    return O, dq, dk, dv, drel
+
+
+@pytest.mark.parametrize("M,L", [(0, 5), (3, 4), (6, 2), (5, 1)])
+def test_txl_memory_vs_brute_force(M, L):
+    rng = np.random.default_rng(M * 10 + L)
+    d, H = 3, 2
+    q, do = rnd(rng, 2, H, L, d), rnd(rng, 2, H, L, d)
+    k, v = rnd(rng, 2, H, M + L, d), rnd(rng, 2, H, M + L, d)
+    rel = [rnd(rng, H, M + L, d, std=0.5), rnd(rng, H, d, std=0.5), rnd(rng, H, d, std=0.5)]
+    s = 0.43
+    O, _ = orc.txl_memory_forward(q, k, v, rel, s)
+    dq, dk, dv, drel = orc.txl_memory_backward(q, k, v, rel, do, s)
+    bO, bdq, bdk, bdv, bdrel = brute_txl_memory(q, k, v, rel, do, s)
+    for got, want in [(O, bO), (dq, bdq), (dk, bdk), (dv, bdv)] + list(zip(drel, bdrel)):
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_txl_memory_finite_differences():
+    rng = np.random.default_rng(17)
+    M, L, d, H = 4, 5, 3, 2
+    q, do = rnd(rng, 1, H, L, d), rnd(rng, 1, H, L, d)
+    k, v = rnd(rng, 1, H, M + L, d), rnd(rng, 1, H, M + L, d)
+    rel = [rnd(rng, H, M + L, d, std=0.5), rnd(rng, H, d, std=0.5), rnd(rng, H, d, std=0.5)]
+    s = 0.37
+    dq, dk, dv, drel = orc.txl_memory_backward(q, k, v, rel, do, s)
+
+    def loss(q_, k_, v_, rel_):
+        return float(np.sum(orc.txl_memory_forward(q_, k_, v_, rel_, s)[0] * do))
+
+    e = np.random.default_rng(2)
+    for name, x, g in [("q", q, dq), ("k", k, dk), ("v", v, dv), ("r", rel[0], drel[0])]:
+        dirn = e.standard_normal(x.shape)
+        args = {"q": q, "k": k, "v": v, "r": rel[0]}
+        plus, minus = dict(args), dict(args)
+        plus[name] = x + 1e-6 * dirn
+        minus[name] = x - 1e-6 * dirn
+        fd = (loss(plus["q"], plus["k"], plus["v"], [plus["r"]] + rel[1:]) -
+              loss(minus["q"], minus["k"], minus["v"], [minus["r"]] + rel[1:])) / 2e-6
+        an = float(np.sum(g * dirn))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
