@@ -46,6 +46,7 @@ class relpos_params_t(ctypes.Structure):
         ("deberta_span", ctypes.c_int32),
         ("seqlens_k", ctypes.c_void_p),
         ("shaw_value", ctypes.c_int32),
+        ("mem_len", ctypes.c_int64),
     ]
 
 
@@ -109,6 +110,7 @@ class Params:
     deberta_span: int = 256
     seqlens_k: Optional[torch.Tensor] = None  # [B] int32 on the device, or None (all L)
     shaw_value: bool = False  # Shaw: rel[1] = aV, the value-side table
+    mem_len: int = 0  # Transformer-XL (causal): memory length M; k, v and r then have M + L rows
 
     def c(self) -> relpos_params_t:
         scale = self.scale
@@ -120,7 +122,8 @@ class Params:
                 raise ValueError("seqlens_k must be a contiguous int32 tensor of B elements")
         return relpos_params_t(self.mech, self.dtype, int(self.causal), self.kernel_path, self.B, self.H, self.L, self.d,
                                float(scale), self.t5_num_buckets, self.t5_max_distance, int(self.t5_bidirectional),
-                               self.shaw_clip, self.deberta_span, _ptr(self.seqlens_k), int(self.shaw_value))
+                               self.shaw_clip, self.deberta_span, _ptr(self.seqlens_k), int(self.shaw_value),
+                               int(self.mem_len))
 
     def n_rel(self) -> int:
         if self.mech == SHAW and self.shaw_value:

@@ -14,7 +14,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10300;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value
+constexpr int kVersion = 10400;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -86,13 +86,17 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   if (P->B < 1 || P->H < 1 || P->L < 1 || P->L > kMaxL || P->B * P->H > 65535) return RELPOS_ERR_INVALID_ARG;
   if (!isfinite(P->scale)) return RELPOS_ERR_INVALID_ARG;
   if (P->shaw_value != 0 && (P->shaw_value != 1 || P->mech != RELPOS_SHAW)) return RELPOS_ERR_INVALID_ARG;
+  if (P->mem_len < 0 || P->L + P->mem_len > kMaxL) return RELPOS_ERR_INVALID_ARG;
+  if (P->mem_len > 0 && (P->mech != RELPOS_TXL || P->causal != 1)) return RELPOS_ERR_INVALID_ARG;
   // ALiBi is a per-offset bias like T5's: it runs on the T5 kernels with one slope
   // per head in place of the bucket table
   p.mech = P->mech == RELPOS_ALIBI ? (int)rp::M_T5 : P->mech;
   p.causal = P->causal;
   p.B = (int)P->B;
   p.H = (int)P->H;
-  p.L = (int)P->L;
+  p.L = (int)(P->L + P->mem_len);  // the kernels see the memory and the segment as one causal sequence
+  p.mem_len = (int)P->mem_len;
+  p.esize = P->dtype == RELPOS_BF16 ? 2 : 4;
   p.scale = P->scale;
   p.seqlens_k = P->seqlens_k;
   p.nT = (p.L + kTile - 1) / kTile;
@@ -152,6 +156,7 @@ struct Layout {
   size_t part_kv, part_dg, part_uv, qa;  // tensor-core backward partials / products
   size_t qkr, kqr, dM, dN, dqc, dkc, dpart;  // DeBERTa tensor-core backward
   size_t pdtiles;                            // Transformer-XL tensor-core backward: stored P / dS tiles (0: none)
+  size_t mq, mo, mlse, mdo, mdq;             // Transformer-XL memory: query-side tensors padded to M + L rows
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -229,6 +234,16 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
         break;
     }
   }
+  if (p.mem_len > 0) {  // the query-side tensors at M + L rows, the first M rows placeholders
+    const size_t rows = BH * (size_t)p.L, rb = (size_t)p.esize * rp::HD;
+    l.mq = take(rows * rb);
+    l.mo = take(rows * rb);
+    l.mlse = take(rows * sizeof(float));
+    if (pass == 1) {
+      l.mdo = take(rows * rb);
+      l.mdq = take(rows * rb);
+    }
+  }
   l.total = off;
   return l;
 }
@@ -282,6 +297,26 @@ static int to_status(cudaError_t e) {
   return RELPOS_ERR_LAUNCH;
 }
 
+__global__ void fill_f32_kernel(float *x, size_t n, float v) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) x[i] = v;
+}
+
+// Transformer-XL memory: a [B,H,L,..] tensor into rows M .. M + L - 1 of each (batch, head)
+// plane of a [B,H,M+L,..] one (rows 0 .. M - 1 set to zero), and back.
+static cudaError_t pad_rows(void *dst, const void *src, size_t rb, const Prm &p, cudaStream_t st) {
+  const int M = p.mem_len, Ls = p.L - M, BH = p.B * p.H;
+  cudaError_t e = cudaMemsetAsync(dst, 0, (size_t)BH * p.L * rb, st);
+  if (e != cudaSuccess) return e;
+  return cudaMemcpy2DAsync((char *)dst + (size_t)M * rb, (size_t)p.L * rb, src, (size_t)Ls * rb, (size_t)Ls * rb, BH,
+                           cudaMemcpyDeviceToDevice, st);
+}
+static cudaError_t unpad_rows(void *dst, const void *src, size_t rb, const Prm &p, cudaStream_t st) {
+  const int M = p.mem_len, Ls = p.L - M, BH = p.B * p.H;
+  return cudaMemcpy2DAsync(dst, (size_t)Ls * rb, (const char *)src + (size_t)M * rb, (size_t)p.L * rb, (size_t)Ls * rb, BH,
+                           cudaMemcpyDeviceToDevice, st);
+}
+
 }  // namespace
 
 extern "C" int relpos_attn_workspace_size(const relpos_params_t *params, int pass, size_t *bytes) {
@@ -325,6 +360,7 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   const Layout l = layout_of(p, 0, tc);
   if (l.total > 0 && (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255))) return RELPOS_ERR_WORKSPACE;
   bind_workspace(p, l, workspace);
+  cudaStream_t st = (cudaStream_t)stream;
   p.q = q;
   p.k = k;
   p.v = v;
@@ -334,11 +370,20 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   p.out = o;
   p.lse = lse;
   p.status = dev_status;
-  cudaStream_t st = (cudaStream_t)stream;
+  const size_t rb = (size_t)p.esize * rp::HD;
+  char *wb = (char *)workspace;
+  if (p.mem_len > 0) {  // the segment's queries at rows M .. M + L - 1 of the padded sequence
+    if ((e = to_status(pad_rows(wb + l.mq, q, rb, p, st)))) return e;
+    p.q = wb + l.mq;
+    p.out = wb + l.mo;
+    p.lse = (float *)(wb + l.mlse);
+  }
   const bool bf16 = params->dtype == RELPOS_BF16;
   if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
-  if (tc) return to_status(rp::tc_fwd(p, tc_work(l, workspace), st));
-  return to_status(rp::simt_fwd(p, bf16, st));
+  e = tc ? to_status(rp::tc_fwd(p, tc_work(l, workspace), st)) : to_status(rp::simt_fwd(p, bf16, st));
+  if (e || p.mem_len == 0) return e;
+  if ((e = to_status(unpad_rows(o, wb + l.mo, rb, p, st)))) return e;
+  return to_status(unpad_rows(lse, wb + l.mlse, sizeof(float), p, st));
 }
 
 extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, const void *k, const void *v,
@@ -378,20 +423,45 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   if (tc) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(rel[0]))
       return RELPOS_ERR_INVALID_ARG;
-    if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;
-    if (p.mech == rp::M_SHAW) return to_status(rp::tc_bwd_shaw(p, tc_work(l, workspace), st));
-    if (p.mech == rp::M_DEB) {
-      if (!aligned16(rel[1])) return RELPOS_ERR_INVALID_ARG;
-      return to_status(rp::tc_bwd_deb(p, tc_work(l, workspace), st));
-    }
-    if (p.mech == rp::M_T5) {
-      if ((e = to_status(rp::launch_t5_prep(p, st)))) return e;
-      return to_status(rp::tc_bwd_bias(p, st));
-    }
-    return to_status(rp::tc_bwd(p, tc_work(l, workspace), st));
+    if (p.mech == rp::M_DEB && !aligned16(rel[1])) return RELPOS_ERR_INVALID_ARG;
   }
-  if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
-  return to_status(rp::simt_bwd(p, bf16, st));
+  const size_t rb = (size_t)p.esize * rp::HD;
+  char *wb = (char *)workspace;
+  if (p.mem_len > 0) {  // placeholder rows 0 .. M - 1: zero q, O and dO, LSE = +inf, so P = 0 and dS = 0 there
+    if ((e = to_status(pad_rows(wb + l.mq, q, rb, p, st)))) return e;
+    if ((e = to_status(pad_rows(wb + l.mo, o, rb, p, st)))) return e;
+    if ((e = to_status(pad_rows(wb + l.mdo, dout, rb, p, st)))) return e;
+    const size_t n = (size_t)p.B * p.H * p.L;
+    fill_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((float *)(wb + l.mlse), n, INFINITY);
+    if ((e = to_status(cudaGetLastError()))) return e;
+    if ((e = to_status(cudaMemcpy2DAsync(wb + l.mlse + (size_t)p.mem_len * sizeof(float), (size_t)p.L * sizeof(float), lse,
+                                         (size_t)(p.L - p.mem_len) * sizeof(float), (size_t)(p.L - p.mem_len) * sizeof(float),
+                                         (size_t)p.B * p.H, cudaMemcpyDeviceToDevice, st))))
+      return e;
+    p.q = wb + l.mq;
+    p.o = wb + l.mo;
+    p.dout = wb + l.mdo;
+    p.lse = (float *)(wb + l.mlse);
+    p.dq = wb + l.mdq;
+  }
+  if (tc) {
+    if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;
+    if (p.mech == rp::M_SHAW) {
+      e = to_status(rp::tc_bwd_shaw(p, tc_work(l, workspace), st));
+    } else if (p.mech == rp::M_DEB) {
+      e = to_status(rp::tc_bwd_deb(p, tc_work(l, workspace), st));
+    } else if (p.mech == rp::M_T5) {
+      if ((e = to_status(rp::launch_t5_prep(p, st)))) return e;
+      e = to_status(rp::tc_bwd_bias(p, st));
+    } else {
+      e = to_status(rp::tc_bwd(p, tc_work(l, workspace), st));
+    }
+  } else {
+    if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
+    e = to_status(rp::simt_bwd(p, bf16, st));
+  }
+  if (e || p.mem_len == 0) return e;
+  return to_status(unpad_rows(dq, wb + l.mdq, rb, p, st));
 }
 
 extern "C" int relpos_attn_resolved_path(const relpos_params_t *params, int pass) {

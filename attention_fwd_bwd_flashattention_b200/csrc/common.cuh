@@ -37,6 +37,7 @@ struct Prm {
   int alibi;
   int clip;   // Shaw clip c
   int shaw_v;  // Shaw: value-side table rel1 = aV (O_i += sum_j P_ij aV[row(j - i)])
+  int mem_len, esize;  // host bookkeeping: Transformer-XL memory length (L counts it), element bytes
   int span;   // DeBERTa span k
   int nT;     // number of 64-row tiles
   int diag_ch, diag_nchunk, nbands;  // Transformer-XL diagonal shards

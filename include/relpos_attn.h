@@ -127,6 +127,14 @@ typedef struct relpos_params {
    * (Community comment); the value side is the second table of Shaw's own paper.
    * Such calls run on the CUDA-core kernels (RELPOS_PATH_TC is rejected). */
   int32_t shaw_value;
+  /* Transformer-XL only, causal only (0 = none): length M of the cached memory of the
+   * previous segment.  The L queries (q, o, lse, dq, dO: [B, H, L, d]) sit at positions
+   * M .. M + L - 1 over M + L keys (k, v, dk, dv: [B, H, M + L, d]: the memory, then the
+   * segment); r has M + L rows and seqlens_k counts keys over the M + L.  Computed as the
+   * causal attention of the M + L positions read at its last L query rows (the first M
+   * rows' work is done and discarded).  Transformer-XL's segment-level recurrence; the
+   * mechanism is one of those the paper's Hugging Face page names (Community comment). */
+  int64_t mem_len;
 } relpos_params_t;
 
 /* Bytes of device workspace a call needs.  pass: 0 forward, 1 backward.

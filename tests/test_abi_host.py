@@ -44,19 +44,20 @@ def test_struct_layout_matches_c(tmp_path):
     prog = tmp_path / "layout.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "relpos_attn.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(relpos_params_t), offsetof(relpos_params_t,B),"
         " offsetof(relpos_params_t,scale), offsetof(relpos_params_t,t5_num_buckets), offsetof(relpos_params_t,deberta_span),"
-        " offsetof(relpos_params_t,seqlens_k), offsetof(relpos_params_t,shaw_value));return 0;}\n")
+        " offsetof(relpos_params_t,seqlens_k), offsetof(relpos_params_t,shaw_value), offsetof(relpos_params_t,mem_len));"
+        "return 0;}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(prog), "-o", str(exe)], check=True)
     got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     S = bd.relpos_params_t
     assert got == [ctypes.sizeof(S), S.B.offset, S.scale.offset, S.t5_num_buckets.offset, S.deberta_span.offset,
-                   S.seqlens_k.offset, S.shaw_value.offset]
+                   S.seqlens_k.offset, S.shaw_value.offset, S.mem_len.offset]
 
 
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10300
+    assert lib.relpos_attn_version() == 10400
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"
@@ -65,7 +66,8 @@ def test_version_and_strerror(lib):
 @pytest.mark.parametrize("bad", [dict(d=32), dict(mech=5), dict(L=0), dict(B=0), dict(dtype=5), dict(scale=float("nan")),
                                  dict(kernel_path=9), dict(mech=0, t5_num_buckets=1), dict(mech=0, t5_max_distance=4),
                                  dict(mech=3, deberta_span=0), dict(mech=1, shaw_clip=-1), dict(shaw_value=2),
-                                 dict(mech=0, shaw_value=1)])
+                                 dict(mech=0, shaw_value=1), dict(mech=2, causal=True, mem_len=-1),
+                                 dict(mech=2, causal=False, mem_len=64), dict(mech=1, causal=True, mem_len=64)])
 def test_invalid_params_rejected(lib, bad):
     kw = dict(mech=1, B=1, H=2, L=64)
     kw.update(bad)
@@ -89,6 +91,14 @@ def test_workspace_sizes(lib):
             assert (f32 > 0) == (mech in (0, 4))
     with pytest.raises(bd.RelposError):
         bd.relpos_attn_workspace_size(bd.Params(mech=1, B=1, H=1, L=8), 2)
+
+
+def test_memory_adds_padded_query_buffers(lib):
+    """Transformer-XL memory: the workspace grows by the query-side tensors at M + L rows."""
+    for pass_ in (0, 1):
+        base = bd.relpos_attn_workspace_size(bd.Params(mech=bd.TXL, B=2, H=2, L=300, causal=True), pass_)
+        mem = bd.relpos_attn_workspace_size(bd.Params(mech=bd.TXL, B=2, H=2, L=300, causal=True, mem_len=100), pass_)
+        assert mem >= base + 2 * 2 * 400 * (64 * 2 * (2 if pass_ == 0 else 4) + 4)
 
 
 def test_backward_workspace_holds_the_stored_tiles(lib):

@@ -56,6 +56,40 @@ def test_parity_deberta_span256(path):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("M,L", [(64, 130), (100, 300), (256, 256), (5, 1)])
+def test_parity_txl_memory(M, L, dtype):
+    """Transformer-XL with M cached keys / values before the segment's L: every output
+    against the oracle's memory formula."""
+    g = torch.Generator().manual_seed(M * 7 + L)
+    B, H, d = 2, 2, 64
+
+    def rn(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g) * std).to(dtype)
+
+    q, do = rn(B, H, L, d), rn(B, H, L, d)
+    k, v = rn(B, H, M + L, d), rn(B, H, M + L, d)
+    rel = [rn(H, M + L, d, std=0.3), rn(H, d, std=0.3), rn(H, d, std=0.3)]
+    s = 1.0 / 8.0
+    P = bd.Params(mech=TXL, B=B, H=H, L=L, dtype=bd.BF16 if dtype == torch.bfloat16 else bd.F32, causal=True,
+                  scale=s, mem_len=M)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    reld = [r.to(dev) for r in rel]
+    o, lse = bd.forward(P, qd, kd, vd, reld)
+    dq, dk, dv, drel = bd.backward(P, qd, kd, vd, reld, o, lse, dod)
+    torch.cuda.synchronize()
+    Q, K, V, G = (to_f64(t) for t in (q, k, v, do))
+    R = [to_f64(r) for r in rel]
+    O, LSE = orc.txl_memory_forward(Q, K, V, R, s)
+    dQ, dK, dV, dR = orc.txl_memory_backward(Q, K, V, R, G, s)
+    tol = TOL[dtype]
+    assert maxabs(f64(o), O) <= tol
+    assert maxabs(f64(lse), LSE) <= tol
+    for got, want in [(dq, dQ), (dk, dK), (dv, dV)] + list(zip(drel, dR)):
+        assert rel_l2(f64(got), want) <= tol
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
 @pytest.mark.parametrize("clip,L", [(3, 17), (3, 130), (64, 300), (100, 257)])
 def test_parity_shaw_value_term(clip, L, causal, dtype):
