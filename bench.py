@@ -108,6 +108,8 @@ def kernel_launches(wl, path):
 # None whenever those kernels change.  Source: profiles/tc_kernels_txl_causal_L8192.md.
 DRAM_TRAFFIC = {
     ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.26e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
+    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (
+        3045.74e6, "dvec, tc_bwd_q, tc_bwd_kvs, tc_bwd_dgs, reduce_dr, reduce_uv (the relation prep kernel not captured)"),
 }
 
 
