@@ -161,7 +161,8 @@ struct Layout {
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-static Layout layout_of(const Prm &p, int pass, bool tc) {
+// lean: the smallest backward workspace (no stored P / dS tiles)
+static Layout layout_of(const Prm &p, int pass, bool tc, bool lean = false) {
   Layout l;
   memset(&l, 0, sizeof(l));
   size_t off = 0;
@@ -212,7 +213,7 @@ static Layout layout_of(const Prm &p, int pass, bool tc) {
     l.part_kv = take(sizeof(float) * kvf);
     l.part_dg = take(sizeof(float) * dgf);
     l.part_uv = take(sizeof(float) * (size_t)p.H * ((p.nrows + 31) / 32) * rp::HD);
-    const size_t eb = rp::tc_bwd_tile_bytes(p);
+    const size_t eb = lean ? 0 : rp::tc_bwd_tile_bytes(p);
     if (eb) l.pdtiles = take(eb);
   } else if (pass == 1) {
     l.dvec = take(sizeof(float) * BH * p.L);
@@ -321,10 +322,11 @@ static cudaError_t unpad_rows(void *dst, const void *src, size_t rb, const Prm &
 
 extern "C" int relpos_attn_workspace_size(const relpos_params_t *params, int pass, size_t *bytes) {
   Prm p;
-  if (!bytes || (pass != 0 && pass != 1)) return RELPOS_ERR_INVALID_ARG;
+  if (!bytes || pass < 0 || pass > 2) return RELPOS_ERR_INVALID_ARG;
   int e = validate_and_fill(params, p);
   if (e) return e;
-  *bytes = layout_of(p, pass, use_tc(params, p, pass)).total;
+  const int ps = pass == 0 ? 0 : 1;
+  *bytes = layout_of(p, ps, use_tc(params, p, ps), pass == 2).total;
   return RELPOS_OK;
 }
 
@@ -399,7 +401,8 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   if ((e = check_seqlens(params))) return e;
   const bool tc = use_tc(params, p, 1);
   if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
-  const Layout l = layout_of(p, 1, tc);
+  Layout l = layout_of(p, 1, tc);
+  if (workspace_bytes < l.total && l.pdtiles) l = layout_of(p, 1, tc, true);  // too small for the stored tiles: recompute
   if (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255)) return RELPOS_ERR_WORKSPACE;
   bind_workspace(p, l, workspace);
   p.q = q;

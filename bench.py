@@ -113,6 +113,18 @@ DRAM_TRAFFIC = {
 }
 
 
+def median_iqr(xs):
+    """(median, interquartile range) of a list of timings (linear interpolation)."""
+    ys = sorted(xs)
+
+    def q(f):
+        x = f * (len(ys) - 1)
+        lo = int(math.floor(x))
+        hi = min(lo + 1, len(ys) - 1)
+        return ys[lo] + (ys[hi] - ys[lo]) * (x - lo)
+    return q(0.5), q(0.75) - q(0.25)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -329,7 +341,12 @@ def run_ours(args, wl):
     bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
     tot_ms = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
     tot_ms = rdist.max_over_ranks(tot_ms)
-    peak_mem = torch.cuda.max_memory_allocated(dev) - base_mem
+    alloc_in_steps = torch.cuda.max_memory_allocated(dev) - base_mem  # 0: the library allocates nothing
+    # device memory of one fwd + bwd step: every buffer the two calls read or write
+    step_bufs = [q, k, v, do, o, lse, dq, dk, dv, *rel, *drel, ws_f, ws_b]
+    step_mem = sum(t.numel() * t.element_size() for t in step_bufs if t is not None)
+    ws_sizes = {"fwd": bd.relpos_attn_workspace_size(P, 0), "bwd": bd.relpos_attn_workspace_size(P, 1),
+                "bwd_smallest": bd.relpos_attn_workspace_size(P, 2)}
 
     f_fwd, f_bwd = algo_flops(wl)
     fa_f, fa_b = fa_flops(wl)
@@ -384,7 +401,12 @@ def run_ours(args, wl):
         "fa_convention_tflops": world * (fa_f + fa_b) / (ms_step * 1e-3) / 1e12,
         "frac_of_dense_bf16_datasheet": value / world / 2250.0,
         "frac_of_measured_bf16": value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
-        "peak_mem_bytes": int(peak_mem),
+        "peak_mem_bytes": int(step_mem),
+        "peak_mem_smallest_workspace_bytes": int(step_mem - ws_sizes["bwd"] + ws_sizes["bwd_smallest"]),
+        "workspace_bytes": ws_sizes,
+        "alloc_during_steps_bytes": int(alloc_in_steps),
+        "timing_ms": {"fwd_median": median_iqr(fwd_ms)[0], "fwd_iqr": median_iqr(fwd_ms)[1],
+                      "bwd_median": median_iqr(bwd_ms)[0], "bwd_iqr": median_iqr(bwd_ms)[1]},
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -137,7 +137,15 @@ typedef struct relpos_params {
   int64_t mem_len;
 } relpos_params_t;
 
-/* Bytes of device workspace a call needs.  pass: 0 forward, 1 backward.
+/* Bytes of device workspace a call needs.  pass: 0 forward, 1 backward,
+ * 2 backward at its smallest.  relpos_attn_bwd accepts any workspace of at least
+ * the pass-2 size.  Between that and the pass-1 size, the Transformer-XL
+ * tensor-core backward recomputes S, P and dS in its key-tile and diagonal kernels.
+ * With the pass-1 size or more, the query-tile kernel writes every tile's P and dS
+ * (64 KB per 128 x 128 tile, e.g. 1.1 GB at B = 1, H = 8, L = 8192 causal) and those
+ * kernels stream them back: faster, but the memory grows with L^2.  Other calls
+ * need the same size for passes 1 and 2.  The split trades memory for time and is
+ * no part of the method.
  * Returns RELPOS_OK and sets *bytes, or RELPOS_ERR_INVALID_ARG. */
 RELPOS_API int relpos_attn_workspace_size(const relpos_params_t *params, int pass, size_t *bytes);
 

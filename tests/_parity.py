@@ -23,10 +23,11 @@ def params_of(wl, path):
                      shaw_value=wl.shaw_value)
 
 
-def run_gpu(wl, inp, path, dev="cuda", seqlens_k=None):
+def run_gpu(wl, inp, path, dev="cuda", seqlens_k=None, bwd_pass=1):
     """Forward + backward through the C ABI; the device status word must stay 0 (a
     bounded wait that ran out inside a kernel reports RELPOS_ERR_TIMEOUT there).
-    seqlens_k: optional per-batch key lengths (a sequence of B ints)."""
+    seqlens_k: optional per-batch key lengths (a sequence of B ints).
+    bwd_pass: the workspace-size pass of the backward's workspace (2: the smallest)."""
     P = params_of(wl, path)
     if seqlens_k is not None:
         P.seqlens_k = torch.tensor(list(seqlens_k), dtype=torch.int32, device=dev)
@@ -38,7 +39,7 @@ def run_gpu(wl, inp, path, dev="cuda", seqlens_k=None):
     bd.relpos_attn_fwd(P, q, k, v, rel, o, lse, bd.workspace(P, 0, q.device), dev_status=status)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     drel = [torch.empty(r.shape, dtype=torch.float32, device=dev) for r in rel[: P.n_rel()]]
-    bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, bd.workspace(P, 1, q.device), dev_status=status)
+    bd.relpos_attn_bwd(P, q, k, v, rel, o, lse, do, dq, dk, dv, drel, bd.workspace(P, bwd_pass, q.device), dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0, f"{wl.name}: device status {int(status.item())} ({bd.strerror(int(status.item()))})"
     return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, drel=drel)

@@ -90,7 +90,7 @@ def test_workspace_sizes(lib):
             f32 = bd.relpos_attn_workspace_size(bd.Params(mech=mech, B=2, H=3, L=1000, causal=causal, dtype=bd.F32), 0)
             assert (f32 > 0) == (mech in (0, 4))
     with pytest.raises(bd.RelposError):
-        bd.relpos_attn_workspace_size(bd.Params(mech=1, B=1, H=1, L=8), 2)
+        bd.relpos_attn_workspace_size(bd.Params(mech=1, B=1, H=1, L=8), 3)
 
 
 def test_memory_adds_padded_query_buffers(lib):
@@ -99,6 +99,28 @@ def test_memory_adds_padded_query_buffers(lib):
         base = bd.relpos_attn_workspace_size(bd.Params(mech=bd.TXL, B=2, H=2, L=300, causal=True), pass_)
         mem = bd.relpos_attn_workspace_size(bd.Params(mech=bd.TXL, B=2, H=2, L=300, causal=True, mem_len=100), pass_)
         assert mem >= base + 2 * 2 * 400 * (64 * 2 * (2 if pass_ == 0 else 4) + 4)
+
+
+def test_smallest_backward_workspace(lib):
+    """pass 2: the smallest backward workspace; it leaves out only the Transformer-XL
+    tensor-core backward's stored P / dS tiles (64 KB per 128 x 128 tile)."""
+    ws = bd.relpos_attn_workspace_size
+    txl = bd.Params(mech=bd.TXL, B=1, H=2, L=1000, dtype=bd.BF16, causal=True)
+    assert ws(txl, 1) - ws(txl, 2) == 2 * (8 * 9 // 2) * 65536
+    txl_full = bd.Params(mech=bd.TXL, B=1, H=2, L=1000, dtype=bd.BF16, causal=False)
+    assert ws(txl_full, 1) - ws(txl_full, 2) == 2 * 64 * 65536
+    mem = bd.Params(mech=bd.TXL, B=1, H=2, L=1000, dtype=bd.BF16, causal=True, mem_len=24)
+    assert ws(mem, 1) - ws(mem, 2) == 2 * (8 * 9 // 2) * 65536
+    same = [bd.Params(mech=bd.TXL, B=1, H=2, L=1000, dtype=bd.F32, causal=True),
+            bd.Params(mech=bd.T5, B=1, H=2, L=1000, dtype=bd.BF16),
+            bd.Params(mech=bd.SHAW, B=1, H=2, L=1000, dtype=bd.BF16),
+            bd.Params(mech=bd.DEBERTA, B=1, H=2, L=1000, dtype=bd.BF16),
+            bd.Params(mech=bd.TXL, B=1, H=2, L=1000, dtype=bd.BF16, kernel_path=bd.PATH_SIMT)]
+    for P in same:
+        assert ws(P, 2) == ws(P, 1)
+    for bad in (-1, 3):
+        with pytest.raises(bd.RelposError):
+            ws(txl, bad)
 
 
 def test_backward_workspace_holds_the_stored_tiles(lib):

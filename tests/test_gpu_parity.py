@@ -55,6 +55,18 @@ def test_parity_deberta_span256(path):
     compare_full(wl, inp, run_gpu(wl, inp, path))
 
 
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("L", [130, 700])
+def test_parity_txl_smallest_backward_workspace(L, causal):
+    """Transformer-XL bf16 backward given only the smallest workspace: the kernels that
+    recompute S, P and dS instead of storing the tiles; every output against the oracle."""
+    wl = small_wl("txl", torch.bfloat16, causal, L)
+    P = params_of(wl, bd.PATH_AUTO)
+    assert bd.relpos_attn_workspace_size(P, 2) < bd.relpos_attn_workspace_size(P, 1)
+    inp = make_inputs(wl, seed=L + 1)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO, bwd_pass=2))
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
 @pytest.mark.parametrize("M,L", [(64, 130), (100, 300), (256, 256), (5, 1)])
 def test_parity_txl_memory(M, L, dtype):
