@@ -34,17 +34,21 @@ by default).  Shaw's value-side term (the second relative table of Shaw et al.,
 optional: ``RelCfg.shaw_value``) adds the same clipped offset's table row to every
 value a query averages:
 
-  O_i = sum_j P_ij (v_j + aV[h, clip(j - i, -c, c) + c])  ALiBi, the further bias named by the article (section "工程权衡与适用边界",
-in its list of models the method suits), is written from its own
-paper (Press et al., "Train Short, Test Long"):
+  O_i = sum_j P_ij (v_j + aV[h, clip(j - i, -c, c) + c])
+
+ALiBi, the further bias named by the article (section "工程权衡与适用边界", in its
+list of models the method suits), is written from its own paper (Press et al.,
+"Train Short, Test Long"):
 
   ALiBi                        S_ij = s q_i.k_j - m[h] |j - i|
 
 a fixed per-head slope m[h] times the distance, added unscaled (the causal model of
 that paper sees only j <= i, so -m (i - j); without a causal mask the symmetric
 distance is the plain reading).  The slopes are the caller's input; their gradient
-sum_ij dS_ij (-|j - i|) is returned like a table gradient.  Transformer-XL rows: row(delta) = delta when causal (delta in [0, L)),
-delta + L - 1 otherwise (delta in (-L, L)).  Causal masking removes j > i.
+sum_ij dS_ij (-|j - i|) is returned like a table gradient.
+
+Transformer-XL rows: row(delta) = delta when causal (delta in [0, L)), delta + L - 1
+otherwise (delta in (-L, L)).  Causal masking removes j > i.
 
 Backward (textbook softmax chain rule):
   dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P o (dP - D),  dV = P^T dO,
@@ -74,6 +78,22 @@ Readings where the pages are silent (listed again in the design notes):
 
 All arithmetic is float64.  Inputs given in bf16 are expected to be upcast by
 the caller (the oracle then sees exactly the values the GPU sees).
+
+Pins (tests/test_oracle_pins.py, tests/test_oracle_autograd.py; none of them calls
+this module to make its expected values):
+  * ``t5_bucket``: a hand-written golden table (tests/golden), the float formula away
+    from the exact ties, the unidirectional variant;
+  * ``forward`` / ``backward`` / ``backward_rows`` for every mechanism, with key
+    lengths and the Shaw value table: scalar Python loops written from each formula
+    (forward and scalar chain rule) on tiny shapes, central finite differences, and
+    torch.autograd of a dense torch restatement (1e-11);
+  * closed forms: L = 1, causal row 0, ALiBi geometric sums; zero relative term ==
+    torch's scaled_dot_product_attention; row-constant terms; query-side table
+    gradients summing to zero; batch sums; padding keys;
+  * ``txl_memory_forward`` / ``txl_memory_backward``: scalar loops with the explicit
+    memory offset, finite differences, autograd of a direct restatement.
+Parity unpinned: no function.  The conventions the pages leave open (listed above
+under "Readings") are pinned only as readings: the pages print no worked example.
 """
 from __future__ import annotations
 
