@@ -56,8 +56,10 @@
  *   - stream: a cudaStream_t (NULL = the legacy default stream).  All work is
  *     enqueued on it asynchronously.
  *
- * Errors: every call returns RELPOS_OK (0) or a negative RELPOS_ERR_* code and
- * enqueues nothing on error.  Launch failures are reported as RELPOS_ERR_LAUNCH.
+ * Errors: every call returns RELPOS_OK (0) or a negative RELPOS_ERR_* code.  Argument
+ * errors (RELPOS_ERR_INVALID_ARG, _WORKSPACE, _UNSUPPORTED) are found before anything
+ * is enqueued; after a launch or runtime failure (RELPOS_ERR_LAUNCH, _CUDA) the work
+ * enqueued before it may still run, and the outputs are undefined.
  * Nothing aborts, traps or throws across this boundary.
  *
  * Determinism: the backward pass uses no atomic operations; the relative-table
