@@ -83,10 +83,11 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   if (P->causal != 0 && P->causal != 1) return RELPOS_ERR_INVALID_ARG;
   if (P->kernel_path < RELPOS_PATH_AUTO || P->kernel_path > RELPOS_PATH_TC) return RELPOS_ERR_INVALID_ARG;
   if (P->d != rp::HD) return RELPOS_ERR_INVALID_ARG;
-  if (P->B < 1 || P->H < 1 || P->L < 1 || P->L > kMaxL || P->B * P->H > 65535) return RELPOS_ERR_INVALID_ARG;
+  if (P->B < 1 || P->H < 1 || P->L < 1 || P->L > kMaxL) return RELPOS_ERR_INVALID_ARG;
+  if (P->B > 65535 || P->H > 65535 || P->B * P->H > 65535) return RELPOS_ERR_INVALID_ARG;  // no overflow: both <= 2^16
   if (!isfinite(P->scale)) return RELPOS_ERR_INVALID_ARG;
   if (P->shaw_value != 0 && (P->shaw_value != 1 || P->mech != RELPOS_SHAW)) return RELPOS_ERR_INVALID_ARG;
-  if (P->mem_len < 0 || P->L + P->mem_len > kMaxL) return RELPOS_ERR_INVALID_ARG;
+  if (P->mem_len < 0 || P->mem_len > kMaxL - P->L) return RELPOS_ERR_INVALID_ARG;
   if (P->mem_len > 0 && (P->mech != RELPOS_TXL || P->causal != 1)) return RELPOS_ERR_INVALID_ARG;
   // ALiBi is a per-offset bias like T5's: it runs on the T5 kernels with one slope
   // per head in place of the bucket table

@@ -67,7 +67,10 @@ def test_version_and_strerror(lib):
                                  dict(kernel_path=9), dict(mech=0, t5_num_buckets=1), dict(mech=0, t5_max_distance=4),
                                  dict(mech=3, deberta_span=0), dict(mech=1, shaw_clip=-1), dict(shaw_value=2),
                                  dict(mech=0, shaw_value=1), dict(mech=2, causal=True, mem_len=-1),
-                                 dict(mech=2, causal=False, mem_len=64), dict(mech=1, causal=True, mem_len=64)])
+                                 dict(mech=2, causal=False, mem_len=64), dict(mech=1, causal=True, mem_len=64),
+                                 dict(B=1 << 40, H=1 << 40), dict(B=65536, H=1), dict(B=256, H=257),
+                                 dict(mech=2, causal=True, mem_len=(1 << 63) - 1), dict(mech=2, causal=True, mem_len=1 << 20),
+                                 dict(L=(1 << 20) + 1), dict(causal=2)])
 def test_invalid_params_rejected(lib, bad):
     kw = dict(mech=1, B=1, H=2, L=64)
     kw.update(bad)
