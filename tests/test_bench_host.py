@@ -1,0 +1,73 @@
+"""Host logic of bench.py: the FLOP accounting and the timing statistics.
+
+The algorithmic FLOP totals of the workloads were worked out by hand from the
+counting rule (U = 2 B H d #pairs; T5 2U / 5U, Shaw 2U + R / 5U + 3R, Transformer-XL
+3U / 8U, DeBERTa 2U + 2R / 5U + 6R with R = 2 B H L rows d) and rounded to three
+digits; the bench's own functions must reproduce them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import bench
+from attention_fwd_bwd_flashattention_b200.inputs import WORKLOADS
+
+HAND = {  # workload: (fwd, bwd) flop, or (None, total)
+    "t5_L128_fp32": (None, 2.94e7),
+    "shaw_L2048_bf16": (1.77e10, 4.46e10),
+    "txl_causal_L8192_bf16": (1.03e11, 2.75e11),
+    "deberta_L8192_bf16": (2.19e11, 5.54e11),
+    "txl_L4096_bf16": (None, 1.89e11),
+    "txl_L8192_bf16": (None, 7.56e11),
+    "txl_L16384_bf16": (None, 3.02e12),
+    "txl_L32768_bf16": (None, 1.21e13),
+}
+
+
+@pytest.mark.parametrize("name", list(HAND))
+def test_algorithmic_flops_match_hand_totals(name):
+    f, b = bench.algo_flops(WORKLOADS[name])
+    want_f, want = HAND[name]
+    if want_f is None:
+        assert abs((f + b) / want - 1) < 0.01, (f + b, want)
+    else:
+        assert abs(f / want_f - 1) < 0.01, (f, want_f)
+        assert abs(b / want - 1) < 0.01, (b, want)
+
+
+def brute_pairs(L, B, causal, lens):
+    n = 0
+    for b in range(B):
+        lk = L if lens is None else max(0, min(L, lens[b]))
+        for i, j in itertools.product(range(L), range(L)):
+            n += (j < lk) and (not causal or j <= i)
+    return n
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("lens", [None, (9, 0, 23, 40)])
+def test_pairs_of_counts_unmasked_pairs(causal, lens):
+    wl = WORKLOADS["txl_L4096_bf16"].with_(B=4, L=23, causal=causal, seqlens_k=lens)
+    assert bench.pairs_of(wl) == brute_pairs(23, 4, causal, lens)
+
+
+def test_fa_convention_flops():
+    wl = WORKLOADS["txl_causal_L8192_bf16"]
+    f, b = bench.fa_flops(wl)
+    pairs = 8192 * 8193 // 2
+    assert f == 4.0 * pairs * 64 * 8 and b == 2.5 * f
+
+
+@pytest.mark.parametrize("xs", [[1.0], [2.0, 1.0], [3.0, 1.0, 2.0, 5.0, 4.0], [1.5, 2.5, 0.3, 9.0, 2.0, 2.0, 7.1]])
+def test_median_iqr(xs):
+    m, iqr = bench.median_iqr(xs)
+    assert math.isclose(m, float(np.median(xs)))
+    assert math.isclose(iqr, float(np.percentile(xs, 75) - np.percentile(xs, 25)), abs_tol=1e-12)
+
+
+def test_kernel_launch_counts_of_the_default_workload():
+    """Transformer-XL bf16: relation prep + forward; D, relation prep, query-tile, the two
+    tile-streaming kernels, dr and u / v reductions (the ncu launch list's kernels)."""
+    assert bench.kernel_launches(WORKLOADS["txl_causal_L8192_bf16"], "auto") == (2, 7)
