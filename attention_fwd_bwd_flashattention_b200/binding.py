@@ -50,8 +50,22 @@ class relpos_params_t(ctypes.Structure):
     ]
 
 
+TRACE_MAX = 64
+
+
+class relpos_trace_t(ctypes.Structure):
+    _fields_ = [
+        ("events", ctypes.POINTER(ctypes.c_void_p)),
+        ("capacity", ctypes.c_int32),
+        ("count", ctypes.c_int32),
+        ("dropped", ctypes.c_int32),
+        ("names", ctypes.c_char_p * TRACE_MAX),
+    ]
+
+
 EXPORTS = ("relpos_attn_workspace_size", "relpos_attn_fwd", "relpos_attn_bwd", "relpos_attn_fwd_noalloc",
-           "relpos_attn_resolved_path", "relpos_strerror", "relpos_attn_version")
+           "relpos_attn_resolved_path", "relpos_selftest_wait", "relpos_trace_begin", "relpos_trace_end",
+           "relpos_strerror", "relpos_attn_version")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -80,6 +94,12 @@ def load() -> ctypes.CDLL:
     lib.relpos_attn_fwd_noalloc.restype = ctypes.c_int
     lib.relpos_attn_resolved_path.argtypes = [P, ctypes.c_int]
     lib.relpos_attn_resolved_path.restype = ctypes.c_int
+    lib.relpos_selftest_wait.argtypes = [ctypes.c_uint64, vp, vp, vp]
+    lib.relpos_selftest_wait.restype = ctypes.c_int
+    lib.relpos_trace_begin.argtypes = [ctypes.POINTER(relpos_trace_t)]
+    lib.relpos_trace_begin.restype = ctypes.c_int
+    lib.relpos_trace_end.argtypes = []
+    lib.relpos_trace_end.restype = ctypes.c_int
     lib.relpos_strerror.argtypes = [ctypes.c_int]
     lib.relpos_strerror.restype = ctypes.c_char_p
     lib.relpos_attn_version.argtypes = []
@@ -190,6 +210,45 @@ def relpos_attn_fwd_noalloc(params: Params, q, k, v, rel, o, lse, dev_status=Non
                                         _ptr(lse), _ptr(dev_status), _stream(stream))
     if rc != 0:
         raise RelposError(rc, "relpos_attn_fwd_noalloc")
+
+
+def relpos_selftest_wait(limit_ns: int, dev_status, dev_elapsed_ns, stream=None) -> None:
+    """Bounded-wait self-test (see include/relpos_attn.h): dev_status int32 [1] and
+    dev_elapsed_ns int64 [1] device tensors receive RELPOS_ERR_TIMEOUT and the wait's
+    duration."""
+    rc = load().relpos_selftest_wait(int(limit_ns), _ptr(dev_status), _ptr(dev_elapsed_ns), _stream(stream))
+    if rc != 0:
+        raise RelposError(rc, "relpos_selftest_wait")
+
+
+class Trace:
+    """Device time of every kernel the library launches from this thread while the
+    context is active (relpos_trace_begin / relpos_trace_end): each kernel is bracketed
+    by two CUDA events on its launch stream.  After synchronising, ``kernels()`` gives
+    [(name, milliseconds)] in launch order."""
+
+    def __init__(self, capacity: int = TRACE_MAX):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.events:  # torch creates the CUDA event at its first record
+            e.record()
+        self._handles = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.events])
+        self.c = relpos_trace_t()
+        self.c.events = ctypes.cast(self._handles, ctypes.POINTER(ctypes.c_void_p))
+        self.c.capacity = capacity
+
+    def __enter__(self):
+        rc = load().relpos_trace_begin(ctypes.byref(self.c))
+        if rc != 0:
+            raise RelposError(rc, "relpos_trace_begin")
+        return self
+
+    def __exit__(self, *exc):
+        load().relpos_trace_end()
+        return False
+
+    def kernels(self):
+        return [(self.c.names[k].decode(), self.events[2 * k].elapsed_time(self.events[2 * k + 1]))
+                for k in range(self.c.count)]
 
 
 def relpos_attn_bwd(params: Params, q, k, v, rel, o, lse, dout, dq, dk, dv, drel, workspace, dev_status=None,

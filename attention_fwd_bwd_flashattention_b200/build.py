@@ -5,6 +5,7 @@ without a GPU.  The shared library exports exactly the C ABI of include/relpos_a
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -45,15 +46,37 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    """Compile (if stale) and return the path of the shared library."""
+    """Compile (if stale) and return the path of the shared library.  Each source is
+    compiled by its own nvcc process (in parallel), then the objects are linked."""
     if not force and up_to_date():
         return lib_path()
     os.makedirs(LIBDIR, exist_ok=True)
+    objdir = os.path.join(LIBDIR, "obj")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "--expt-relaxed-constexpr",
+             "-I", INCLUDE, "-I", CSRC, *(extra or [])]
+
+    def compile_one(src):
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc(), *flags, "-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, r
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(sources()), os.cpu_count() or 1))) as ex:
+        results = list(ex.map(compile_one, sources()))
+    failed = False
+    for src, _, r in results:
+        if r.stdout or r.stderr:
+            print(r.stdout + r.stderr, file=sys.stderr, end="")
+        if r.returncode != 0:
+            print(f"nvcc failed: {src}", file=sys.stderr)
+            failed = True
+    if failed:
+        raise subprocess.CalledProcessError(1, "nvcc")
     tmp = lib_path() + ".tmp"
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
-           "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
-    if extra:
-        cmd[1:1] = list(extra)
+    cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *[o for _, o, _ in results]]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)

@@ -14,7 +14,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10400;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len
+constexpr int kVersion = 10600;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len; 1.5.0: relpos_selftest_wait; 1.6.0: relpos_trace_begin / _end
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -436,7 +436,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
     if ((e = to_status(pad_rows(wb + l.mo, o, rb, p, st)))) return e;
     if ((e = to_status(pad_rows(wb + l.mdo, dout, rb, p, st)))) return e;
     const size_t n = (size_t)p.B * p.H * p.L;
-    fill_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((float *)(wb + l.mlse), n, INFINITY);
+    RP_TRACED("fill_f32_kernel", st, fill_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((float *)(wb + l.mlse), n, INFINITY));
     if ((e = to_status(cudaGetLastError()))) return e;
     if ((e = to_status(cudaMemcpy2DAsync(wb + l.mlse + (size_t)p.mem_len * sizeof(float), (size_t)p.L * sizeof(float), lse,
                                          (size_t)(p.L - p.mem_len) * sizeof(float), (size_t)(p.L - p.mem_len) * sizeof(float),

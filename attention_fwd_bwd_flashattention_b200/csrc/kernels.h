@@ -4,6 +4,18 @@
 #include "common.cuh"
 
 namespace rp {
+// Every kernel launch of the library goes through RP_TRACED: an NVTX range around the
+// launch and, when the calling thread registered a trace (relpos_trace_begin), CUDA
+// events on the launch stream before and after the kernel.
+void trace_pre(const char *name, cudaStream_t st);
+void trace_post(cudaStream_t st);
+#define RP_TRACED(name, st, ...)   \
+  do {                             \
+    ::rp::trace_pre(name, st);     \
+    __VA_ARGS__;                   \
+    ::rp::trace_post(st);          \
+  } while (0)
+
 cudaError_t launch_t5_prep(const Prm &p, cudaStream_t st);
 cudaError_t simt_fwd(const Prm &p, bool bf16, cudaStream_t st);
 cudaError_t simt_bwd(const Prm &p, bool bf16, cudaStream_t st);

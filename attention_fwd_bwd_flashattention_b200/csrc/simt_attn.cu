@@ -883,7 +883,7 @@ static cudaError_t run_fwd_t(const Prm &p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nT, p.H, p.B);
-  k<<<grid, NT, SMEM_BYTES, st>>>(p);
+  RP_TRACED("simt_fwd_kernel", st, k<<<grid, NT, SMEM_BYTES, st>>>(p));
   return cudaGetLastError();
 }
 
@@ -891,42 +891,42 @@ template <int MECH, class T>
 static cudaError_t run_bwd_t(const Prm &p, cudaStream_t st) {
   cudaError_t e;
   const size_t rows = (size_t)p.B * p.H * p.L;
-  dvec_kernel<T><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p);
+  RP_TRACED("dvec_kernel", st, dvec_kernel<T><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   auto kq = bwd_q_kernel<MECH, T>;
   auto kkv = bwd_kv_kernel<MECH, T>;
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess) return e;
   dim3 grid(p.nT, p.H, p.B);
-  kkv<<<grid, NT, SMEM_BYTES, st>>>(p);
+  RP_TRACED("simt_bwd_kv_kernel", st, kkv<<<grid, NT, SMEM_BYTES, st>>>(p));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kq<<<grid, NT, SMEM_BYTES, st>>>(p);
+  RP_TRACED("simt_bwd_q_kernel", st, kq<<<grid, NT, SMEM_BYTES, st>>>(p));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (MECH == M_TXL) {
     auto kd = bwd_diag_kernel<T>;
     if ((e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess) return e;
     dim3 gd(p.nbands, p.diag_nchunk, p.B * p.H);
-    kd<<<gd, NT, SMEM_BYTES, st>>>(p);
+    RP_TRACED("simt_bwd_diag_kernel", st, kd<<<gd, NT, SMEM_BYTES, st>>>(p));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t n = (size_t)p.H * p.nrows * HD;
-    reduce_txl_dr_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p);
+    RP_TRACED("reduce_txl_dr_kernel", st, reduce_txl_dr_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    reduce_txl_uv_kernel<T><<<p.H * HD, 256, 0, st>>>(p);
+    RP_TRACED("reduce_txl_uv_kernel", st, reduce_txl_uv_kernel<T><<<p.H * HD, 256, 0, st>>>(p));
     return cudaGetLastError();
   }
   if (MECH == M_T5) {
-    reduce_t5_kernel<<<(p.H * p.nb + 255) / 256, 256, 0, st>>>(p);
+    RP_TRACED("reduce_t5_kernel", st, reduce_t5_kernel<<<(p.H * p.nb + 255) / 256, 256, 0, st>>>(p));
     return cudaGetLastError();
   }
   const size_t n = (size_t)p.H * p.nrows * HD;
-  reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_row, p.drel0);
+  RP_TRACED("reduce_tiles_kernel", st, reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_row, p.drel0));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (MECH == M_SHAW && p.shaw_v) {
-    reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_val, p.drel1);
+    RP_TRACED("reduce_tiles_kernel", st, reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_val, p.drel1));
     return cudaGetLastError();
   }
   if (MECH == M_DEB) {
-    reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_col, p.drel1);
+    RP_TRACED("reduce_tiles_kernel", st, reduce_tiles_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, p.part_col, p.drel1));
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -956,15 +956,15 @@ __global__ void t5_prep_kernel(Prm p) {
 cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st) {
   const size_t rows = (size_t)p.B * p.H * p.L;
   if (bf16)
-    simt::dvec_kernel<__nv_bfloat16><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p);
+    RP_TRACED("dvec_kernel", st, simt::dvec_kernel<__nv_bfloat16><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p));
   else
-    simt::dvec_kernel<float><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p);
+    RP_TRACED("dvec_kernel", st, simt::dvec_kernel<float><<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p));
   return cudaGetLastError();
 }
 
 cudaError_t launch_t5_prep(const Prm &p, cudaStream_t st) {
   const int n = 2 * p.L - 1;
-  t5_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(p);
+  RP_TRACED("t5_prep_kernel", st, t5_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(p));
   return cudaGetLastError();
 }
 

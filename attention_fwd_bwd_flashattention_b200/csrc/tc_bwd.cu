@@ -1496,26 +1496,26 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if (a.pd_stored) {  // the query-tile kernel first: the key-tile pass streams its P / dS tiles
     if ((e = cudaFuncSetAttribute(tc_bwd_kvs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess)
       return e;
-    tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
+    RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    tc_bwd_kvs_kernel<<<tiles, kvs::NTH, kvs::SMEM, st>>>(a);
+    RP_TRACED("tc_bwd_kvs_kernel", st, tc_bwd_kvs_kernel<<<tiles, kvs::NTH, kvs::SMEM, st>>>(a));
   } else {
-    tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a);
+    RP_TRACED("tc_bwd_kv_kernel", st, tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a);
+    RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.pd_stored) {
     if ((e = cudaFuncSetAttribute(tc_bwd_dgs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dgs::SMEM)) != cudaSuccess)
       return e;
-    tc_bwd_dgs_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dgs::SMEM, st>>>(a);
+    RP_TRACED("tc_bwd_dgs_kernel", st, tc_bwd_dgs_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dgs::SMEM, st>>>(a));
   } else {
-    tc_bwd_diag_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a);
+    RP_TRACED("tc_bwd_diag_kernel", st, tc_bwd_diag_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reduce_dr_kernel<<<(unsigned)(p0.H * ((p0.nrows + 31) / 32)), 256, 0, st>>>(a);
+  RP_TRACED("reduce_dr_kernel", st, reduce_dr_kernel<<<(unsigned)(p0.H * ((p0.nrows + 31) / 32)), 256, 0, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reduce_uv_kernel<<<p0.H, 256, 0, st>>>(a);
+  RP_TRACED("reduce_uv_kernel", st, reduce_uv_kernel<<<p0.H, 256, 0, st>>>(a));
   return cudaGetLastError();
 }
 

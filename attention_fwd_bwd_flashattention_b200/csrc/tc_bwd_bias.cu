@@ -663,11 +663,11 @@ cudaError_t tc_bwd_bias(const Prm &p0, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_bwd_bias_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qb::SMEM)) != cudaSuccess)
     return e;
   const unsigned tiles = (unsigned)(a.p.nT * BH);
-  tc_bwd_bias_kv_kernel<<<tiles, NTHREADS, kvb::SMEM, st>>>(a);
+  RP_TRACED("tc_bwd_bias_kv_kernel", st, tc_bwd_bias_kv_kernel<<<tiles, NTHREADS, kvb::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_bwd_bias_q_kernel<<<tiles, NTHREADS, qb::SMEM, st>>>(a);
+  RP_TRACED("tc_bwd_bias_q_kernel", st, tc_bwd_bias_q_kernel<<<tiles, NTHREADS, qb::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reduce_bias_kernel<<<(unsigned)((p0.H * p0.nb + 7) / 8), 256, 0, st>>>(a.p, a.part);
+  RP_TRACED("reduce_bias_kernel", st, reduce_bias_kernel<<<(unsigned)((p0.H * p0.nb + 7) / 8), 256, 0, st>>>(a.p, a.part));
   return cudaGetLastError();
 }
 

@@ -1064,18 +1064,18 @@ cudaError_t tc_bwd_deb(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(deb_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rw::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(deb_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tk::SMEM)) != cudaSuccess) return e;
   const unsigned tiles = (unsigned)(a.p.nT * BH);
-  deb_tables_kernel<<<dim3(tiles, 2), 128, tb::SMEM, st>>>(a);
+  RP_TRACED("deb_tables_kernel", st, deb_tables_kernel<<<dim3(tiles, 2), 128, tb::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  deb_kv_kernel<<<tiles, NTHREADS, kvd::SMEM, st>>>(a);
+  RP_TRACED("deb_kv_kernel", st, deb_kv_kernel<<<tiles, NTHREADS, kvd::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  deb_q_kernel<<<tiles, NTHREADS, qd::SMEM, st>>>(a);
+  RP_TRACED("deb_q_kernel", st, deb_q_kernel<<<tiles, NTHREADS, qd::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  deb_rows_kernel<<<dim3(tiles, 2), 128, rw::SMEM, st>>>(a);
+  RP_TRACED("deb_rows_kernel", st, deb_rows_kernel<<<dim3(tiles, 2), 128, rw::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  deb_table_kernel<<<dim3((unsigned)(p0.H * ((a.W + 127) / 128)), (unsigned)(p0.B * a.nch), 2), 128, tk::SMEM, st>>>(a);
+  RP_TRACED("deb_table_kernel", st, deb_table_kernel<<<dim3((unsigned)(p0.H * ((a.W + 127) / 128)), (unsigned)(p0.B * a.nch), 2), 128, tk::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t n = 2 * (size_t)p0.H * a.W * HD;
-  reduce_deb_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a);
+  RP_TRACED("reduce_deb_table_kernel", st, reduce_deb_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a));
   return cudaGetLastError();
 }
 

@@ -703,19 +703,19 @@ cudaError_t tc_bwd_shaw(const Prm &p0, const TcWork &w, cudaStream_t st) {
     return cudaErrorInvalidValue;
   cudaError_t e;
   const unsigned qa_blocks = (unsigned)(BH * ((p0.L + 31) / 32));
-  shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, w.qa);
+  RP_TRACED("shaw_qa_kernel", st, shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, w.qa));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(tc_bwd_shaw_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(tc_bwd_shaw_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qs::SMEM)) != cudaSuccess)
     return e;
   const unsigned tiles = (unsigned)(a.p.nT * BH);
-  tc_bwd_shaw_kv_kernel<<<tiles, NTHREADS, kvs::SMEM, st>>>(a);
+  RP_TRACED("tc_bwd_shaw_kv_kernel", st, tc_bwd_shaw_kv_kernel<<<tiles, NTHREADS, kvs::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_bwd_shaw_q_kernel<<<tiles, NTHREADS, qs::SMEM, st>>>(a);
+  RP_TRACED("tc_bwd_shaw_q_kernel", st, tc_bwd_shaw_q_kernel<<<tiles, NTHREADS, qs::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t n = (size_t)p0.H * p0.nrows * HD;
-  reduce_shaw_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.p, a.part);
+  RP_TRACED("reduce_shaw_kernel", st, reduce_shaw_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.p, a.part));
   return cudaGetLastError();
 }
 

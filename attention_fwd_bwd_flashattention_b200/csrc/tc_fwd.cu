@@ -678,7 +678,7 @@ static cudaError_t launch_fwd_t(const FwdArgs &a, cudaStream_t st) {
   auto k = tc_fwd_kernel<MECH>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)(a.p.nT * a.p.H * a.p.B), NTHREADS, SMEM_BYTES, st>>>(a);
+  RP_TRACED("tc_fwd_kernel", st, k<<<(unsigned)(a.p.nT * a.p.H * a.p.B), NTHREADS, SMEM_BYTES, st>>>(a));
   return cudaGetLastError();
 }
 
@@ -722,7 +722,7 @@ bool tc_make_map_bf16_wide(CUtensorMap *m, const void *base, uint32_t row_len, u
 cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st) {
   if (p.mech != M_TXL && p.mech != M_DEB) return cudaSuccess;
   const size_t rows = (size_t)p.B * p.H * p.L + (p.mech == M_TXL ? (size_t)p.H * p.nrows : 0);
-  tc::tc_prep_kernel<<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE);
+  RP_TRACED("tc_prep_kernel", st, tc::tc_prep_kernel<<<(unsigned)((8 * rows + 255) / 256), 256, 0, st>>>(p, w.uk, w.vr, w.c2pE, w.p2cE));
   return cudaGetLastError();
 }
 

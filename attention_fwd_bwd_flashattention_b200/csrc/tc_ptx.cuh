@@ -48,19 +48,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for phase `parity` of an mbarrier, for at most ~2 s.  On expiry the CTA's
 // abort flag is raised, the caller's status word gets `code`, and false is
 // returned; every later wait of the CTA then returns at once.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
-                                          int code) {
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
+                                              int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (*abort_flag) return false;
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > 2000000000ull) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
       if (status) *status = code;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, int32_t *status,
+                                          int code) {
+  return mbar_wait_for(bar, parity, abort_flag, status, code, 2000000000ull);
 }
 
 // ---------------------------------------------------------------------------

@@ -46,6 +46,10 @@ class Workload:
     deberta_span: int = 256
     seqlens_k: Optional[Tuple[int, ...]] = None  # per-batch key lengths (variable-length batch)
     shaw_value: bool = False  # Shaw: also the value-side table aV
+    # std of the drawn Shaw (a, aV) and DeBERTa (Kr, Qr) tables instead of the workload's
+    # 0.02; None keeps 0.02.  Parity tests draw them at O(1) so that the relative term
+    # moves the outputs by far more than the tolerance.
+    rel_std: Optional[float] = None
 
     @property
     def scale(self) -> float:
@@ -114,9 +118,10 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
     elif wl.mech == T5:
         rel = [nrm(H, wl.t5_num_buckets, std=0.1)]
     elif wl.mech == SHAW:
-        rel = [nrm(H, 2 * wl.shaw_clip + 1, d, std=0.02).to(dt)]
+        sd = 0.02 if wl.rel_std is None else wl.rel_std
+        rel = [nrm(H, 2 * wl.shaw_clip + 1, d, std=sd).to(dt)]
         if wl.shaw_value:
-            rel.append(nrm(H, 2 * wl.shaw_clip + 1, d, std=0.02).to(dt))
+            rel.append(nrm(H, 2 * wl.shaw_clip + 1, d, std=sd).to(dt))
     elif wl.mech == TXL:
         n_off = L if wl.causal else 2 * L - 1
         W_R = nrm(TXL_EMB, H * d, std=0.02).to(torch.float64)
@@ -125,7 +130,8 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
         r = (txl_sinusoid(n_off, wl.causal, L) @ W_R).reshape(n_off, H, d).permute(1, 0, 2).contiguous()
         rel = [r.to(dt), u, vv]
     else:
-        rel = [nrm(H, 2 * wl.deberta_span, d, std=0.02).to(dt), nrm(H, 2 * wl.deberta_span, d, std=0.02).to(dt)]
+        sd = 0.02 if wl.rel_std is None else wl.rel_std
+        rel = [nrm(H, 2 * wl.deberta_span, d, std=sd).to(dt), nrm(H, 2 * wl.deberta_span, d, std=sd).to(dt)]
     return dict(q=q, k=k, v=v, do=do, rel=rel)
 
 

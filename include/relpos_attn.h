@@ -192,7 +192,9 @@ RELPOS_API int relpos_attn_bwd(const relpos_params_t *params,
  * rejected with RELPOS_ERR_WORKSPACE before anything is enqueued.  It allocates
  * nothing.  All calls share the array: calls that may overlap on the GPU race and
  * must be ordered by the caller.  The first call on a device looks up the array's
- * device address (with that device current); make it before any stream capture. */
+ * device address (with that device current); make it before any stream capture.
+ * The address is kept for the life of the process: do not use this entry point after
+ * cudaDeviceReset, nor from a context other than the device's primary context. */
 RELPOS_API int relpos_attn_fwd_noalloc(const relpos_params_t *params,
                                        const void *q, const void *k, const void *v,
                                        const void *const rel[3],
@@ -204,6 +206,44 @@ RELPOS_API int relpos_attn_fwd_noalloc(const relpos_params_t *params,
  * or a negative RELPOS_ERR_* code (RELPOS_ERR_UNSUPPORTED when RELPOS_PATH_TC is
  * forced where it does not apply). */
 RELPOS_API int relpos_attn_resolved_path(const relpos_params_t *params, int pass);
+
+/* Self-test of the bounded device waits (failure detection; no counterpart in the
+ * paper).  Launches one warp that waits on a device barrier nothing ever completes,
+ * through the wait routine of the tensor-core kernels, with a limit of limit_ns
+ * (1 ms .. 10 s) instead of their 2 s.  When the kernel has run, *dev_status holds
+ * RELPOS_ERR_TIMEOUT and *dev_elapsed_ns the nanoseconds the wait took (the limit plus
+ * at most about 1 ms); the context stays usable.  dev_status and dev_elapsed_ns are
+ * device pointers.  Returns RELPOS_ERR_INVALID_ARG for a null or host pointer or a
+ * limit out of range, RELPOS_ERR_LAUNCH if the launch fails, else RELPOS_OK. */
+RELPOS_API int relpos_selftest_wait(uint64_t limit_ns, int32_t *dev_status,
+                                    unsigned long long *dev_elapsed_ns, void *stream);
+
+/* Tracing (no counterpart in the paper; a measurement aid).  Every kernel the library
+ * launches is wrapped in an NVTX range named after the kernel, which NVTX-aware
+ * profilers show and which costs nothing when none is attached.  A caller that wants
+ * per-kernel device times without a profiler registers a relpos_trace_t with
+ * relpos_trace_begin: until relpos_trace_end, every kernel that this library launches
+ * from the SAME host thread is bracketed by two of the caller's CUDA events, recorded on
+ * the launch stream: kernel k of the traced calls (in launch order) between
+ * events[2k] and events[2k + 1], its static name in names[k].  The caller creates the
+ * 2 * capacity events (cudaEvent_t, timing enabled), keeps the struct alive while it is
+ * registered, and reads the times with cudaEventElapsedTime after synchronising.
+ * Kernels past capacity are not recorded and counted in `dropped`.  Registration is per
+ * host thread: calls from other threads are neither traced nor affected. */
+#define RELPOS_TRACE_MAX 64
+typedef struct relpos_trace {
+  void *const *events;                 /* in: 2 * capacity cudaEvent_t handles        */
+  int32_t capacity;                    /* in: kernels to record, 1 .. RELPOS_TRACE_MAX */
+  int32_t count;                       /* out: kernels recorded                       */
+  int32_t dropped;                     /* out: kernels launched past capacity         */
+  const char *names[RELPOS_TRACE_MAX]; /* out: name of kernel k                       */
+} relpos_trace_t;
+
+/* Starts recording this thread's launches into *trace (count and dropped reset).
+ * Returns RELPOS_ERR_INVALID_ARG for a null struct or event, or a capacity out of range. */
+RELPOS_API int relpos_trace_begin(relpos_trace_t *trace);
+/* Stops recording for this thread.  Always RELPOS_OK. */
+RELPOS_API int relpos_trace_end(void);
 
 /* Static, NUL-terminated description of a status code. */
 RELPOS_API const char *relpos_strerror(int status);

@@ -56,8 +56,35 @@ def test_struct_layout_matches_c(tmp_path):
                    S.seqlens_k.offset, S.shaw_value.offset, S.mem_len.offset]
 
 
+def test_trace_struct_layout_matches_c(tmp_path):
+    prog = tmp_path / "trace.c"
+    prog.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "relpos_attn.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %d\\n\", sizeof(relpos_trace_t), offsetof(relpos_trace_t,capacity),"
+        " offsetof(relpos_trace_t,count), offsetof(relpos_trace_t,dropped), offsetof(relpos_trace_t,names), RELPOS_TRACE_MAX);"
+        "return 0;}\n")
+    exe = tmp_path / "trace"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(prog), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    T = bd.relpos_trace_t
+    assert got == [ctypes.sizeof(T), T.capacity.offset, T.count.offset, T.dropped.offset, T.names.offset, bd.TRACE_MAX]
+
+
+def test_trace_registration_is_validated(lib):
+    t = bd.relpos_trace_t()
+    assert lib.relpos_trace_begin(None) == -1
+    assert lib.relpos_trace_begin(ctypes.byref(t)) == -1  # no events
+    arr = (ctypes.c_void_p * 2)(None, None)
+    t.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    t.capacity = 1
+    assert lib.relpos_trace_begin(ctypes.byref(t)) == -1  # null event handles
+    t.capacity = bd.TRACE_MAX + 1
+    assert lib.relpos_trace_begin(ctypes.byref(t)) == -1
+    assert lib.relpos_trace_end() == 0
+
+
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10400
+    assert lib.relpos_attn_version() == 10600
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"

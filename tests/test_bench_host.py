@@ -71,3 +71,20 @@ def test_kernel_launch_counts_of_the_default_workload():
     """Transformer-XL bf16: relation prep + forward; D, relation prep, query-tile, the two
     tile-streaming kernels, dr and u / v reductions (the ncu launch list's kernels)."""
     assert bench.kernel_launches(WORKLOADS["txl_causal_L8192_bf16"], "auto") == (2, 7)
+
+
+def test_txl_backward_credit_splits_8U():
+    """The Transformer-XL backward's algorithmic 8U, split over the kernels of each
+    variant: query-tile 5U with the streaming (2U + 1U) or recomputing (2U + 1U) kernels."""
+    c = bench.KERNEL_CREDIT_U
+    T = bench.TXL
+    assert c[(T, "tc_bwd_q_kernel")] + c[(T, "tc_bwd_kvs_kernel")] + c[(T, "tc_bwd_dgs_kernel")] == 8
+    assert c[(T, "tc_bwd_q_kernel")] + c[(T, "tc_bwd_kv_kernel")] + c[(T, "tc_bwd_diag_kernel")] == 8
+
+
+def test_kernel_table_shares():
+    k = {"a": [1.0, 1.0], "b": [0.25, 0.25, 0.25, 0.25]}
+    t = bench.kernel_table(k, 2, 2.0)
+    assert list(t) == ["a", "b"]
+    assert t["a"] == {"launches_per_step": 1.0, "ms_per_launch": 1.0, "share_of_step": 0.5}
+    assert t["b"]["launches_per_step"] == 2.0 and math.isclose(t["b"]["share_of_step"], 0.25)

@@ -313,3 +313,73 @@ def test_parity_long_sampled(name):
     assert np.max(np.abs(dk_sum)) <= tol * np.linalg.norm(f64(out["dk"][0, 0])) + 1e-3
     dr_sum = f64(out["drel"][0].sum(dim=1))
     assert np.max(np.abs(dr_sum)) <= tol * float(torch.linalg.norm(out["drel"][0][0])) + 1e-4
+
+
+def test_bounded_wait_runs_out_and_reports():
+    """Failure detection: a device wait on a barrier nothing completes gives up after its
+    limit, writes RELPOS_ERR_TIMEOUT to the status word and returns; the context stays
+    usable (a forward pass runs and matches the oracle afterwards)."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    elapsed = torch.zeros(1, dtype=torch.int64, device="cuda")
+    limit = 50_000_000  # 50 ms
+    bd.relpos_selftest_wait(limit, status, elapsed)
+    torch.cuda.synchronize()
+    assert int(status.item()) == -5, bd.strerror(int(status.item()))
+    assert limit <= int(elapsed.item()) < limit + 20_000_000
+    with pytest.raises(bd.RelposError):
+        bd.relpos_selftest_wait(limit, torch.zeros(1, dtype=torch.int32), elapsed)  # host status word
+    wl = small_wl("txl", torch.bfloat16, True, 130)
+    inp = make_inputs(wl, seed=7)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+# --------------------------------------------------------------------------
+# Shaw and DeBERTa with their tables drawn at std 1.0: at the workloads' 0.02 the
+# relative term moves the outputs by about the tolerance, at 1.0 a gather one offset
+# off, a flipped offset sign, a dropped term or swapped tables moves them by many
+# tolerances (tests/test_parity_power.py, with the oracle alone, on these shapes)
+# --------------------------------------------------------------------------
+O1_L = [130, 300, 700, 1100]
+
+
+@pytest.mark.parametrize("path", [bd.PATH_SIMT, bd.PATH_AUTO], ids=["simt", "auto"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("clip", [1, 7, 64, 100])
+@pytest.mark.parametrize("L", O1_L)
+def test_parity_shaw_o1_tables(L, clip, causal, path):
+    wl = Workload("shaw_o1", SHAW, torch.bfloat16, causal, 2, 2, L, shaw_clip=clip, rel_std=1.0)
+    inp = make_inputs(wl, seed=clip + L)
+    compare_full(wl, inp, run_gpu(wl, inp, path))
+
+
+@pytest.mark.parametrize("path", [bd.PATH_SIMT, bd.PATH_AUTO], ids=["simt", "auto"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("span", [32, 96, 256, 40])
+@pytest.mark.parametrize("L", O1_L)
+def test_parity_deberta_o1_tables(L, span, causal, path):
+    wl = Workload("deb_o1", DEBERTA, torch.bfloat16, causal, 2, 2, L, deberta_span=span, rel_std=1.0)
+    inp = make_inputs(wl, seed=span + L)
+    compare_full(wl, inp, run_gpu(wl, inp, path))
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("clip,L", [(3, 130), (64, 300), (100, 700)])
+def test_parity_shaw_value_o1_tables(clip, L, causal):
+    wl = Workload("shaw_val_o1", SHAW, torch.bfloat16, causal, 2, 2, L, shaw_clip=clip, shaw_value=True, rel_std=1.0)
+    inp = make_inputs(wl, clip + L)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+def test_parity_shaw_L2048_o1_tables():
+    """The Shaw workload's shape (B2 H8 L2048, clip 64), tables at std 1.0: every output."""
+    wl = WORKLOADS["shaw_L2048_bf16"].with_(rel_std=1.0)
+    inp = make_inputs(wl, 0)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+def test_parity_deberta_L8192_o1_tables_one_head():
+    """The DeBERTa workload's shape (B1 H12 L8192, span 256), tables at std 1.0: every
+    output of head 0 (its table gradients included)."""
+    wl = WORKLOADS["deberta_L8192_bf16"].with_(rel_std=1.0)
+    inp = make_inputs(wl, 0)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO), heads=slice(0, 1))

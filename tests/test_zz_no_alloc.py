@@ -41,6 +41,62 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     assert e.value.code == -2
 
 
+# T5, bf16, causal, B = 1, H = 64: at L = 32264 the forward scratch (per-offset bias
+# vectors and buckets) is exactly the size of the built-in array, one more row is too big
+AT_LIMIT = dict(mech=T5, B=1, H=64, L=32264, dtype=bd.BF16, causal=True)
+
+
+def test_noalloc_size_check_at_the_limit():
+    assert bd.relpos_attn_workspace_size(bd.Params(**AT_LIMIT), 0) == bd.NOALLOC_SCRATCH_BYTES
+    P = bd.Params(**dict(AT_LIMIT, L=AT_LIMIT["L"] + 1))
+    assert bd.relpos_attn_workspace_size(P, 0) > bd.NOALLOC_SCRATCH_BYTES
+    fake = torch.empty(0)
+    null_stream = type("S", (), {"cuda_stream": 0})()
+    with pytest.raises(bd.RelposError) as e:
+        bd.relpos_attn_fwd_noalloc(P, fake, fake, fake, [fake], fake, fake, stream=null_stream)
+    assert e.value.code == -2
+
+
+def _check_twice(P, q, k, v, rel, tol):
+    o_ref, lse_ref = bd.forward(P, q, k, v, rel)
+    for _ in range(2):
+        o = torch.full_like(q, float("nan"))
+        lse = torch.full(q.shape[:3], float("nan"), dtype=torch.float32, device=q.device)
+        bd.relpos_attn_fwd_noalloc(P, q, k, v, rel, o, lse)
+        torch.cuda.synchronize()
+        assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+        assert (o.float() - o_ref.float()).abs().max().item() <= tol
+        assert (lse - lse_ref).abs().max().item() <= tol
+
+
+@pytest.mark.gpu
+def test_noalloc_txl_memory_twice():
+    """Transformer-XL with memory (M = 100 cached keys before a 300-query segment): the
+    call that takes most from the array (padded q, O and LSE rows beside u.k and v.r)."""
+    dev = torch.device("cuda", 0)
+    g = torch.Generator().manual_seed(11)
+    B, H, L, M, d = 2, 2, 300, 100, 64
+
+    def rn(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g) * std).to(torch.bfloat16).to(dev)
+
+    q, k, v = rn(B, H, L, d), rn(B, H, M + L, d), rn(B, H, M + L, d)
+    rel = [rn(H, M + L, d, std=0.3), rn(H, d, std=0.3), rn(H, d, std=0.3)]
+    P = bd.Params(mech=TXL, B=B, H=H, L=L, dtype=bd.BF16, causal=True, scale=0.125, mem_len=M)
+    _check_twice(P, q, k, v, rel, TOL[torch.bfloat16])
+
+
+@pytest.mark.gpu
+def test_noalloc_at_the_scratch_limit_twice():
+    dev = torch.device("cuda", 0)
+    P = bd.Params(**AT_LIMIT)
+    g = torch.Generator().manual_seed(12)
+    shape = (P.B, P.H, P.L, 64)
+    q, k, v = (torch.randn(*shape, generator=g).to(torch.bfloat16).to(dev) for _ in range(3))
+    rel = [(torch.randn(P.H, 32, generator=g) * 0.1).to(dev)]
+    _check_twice(P, q, k, v, rel, TOL[torch.bfloat16])
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("wl", CASES, ids=[w.name for w in CASES])
 def test_noalloc_matches_regular_entry_point_twice(wl):
