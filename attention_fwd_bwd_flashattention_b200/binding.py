@@ -59,6 +59,7 @@ class relpos_trace_t(ctypes.Structure):
         ("capacity", ctypes.c_int32),
         ("count", ctypes.c_int32),
         ("dropped", ctypes.c_int32),
+        ("only", ctypes.c_char_p),
         ("names", ctypes.c_char_p * TRACE_MAX),
     ]
 
@@ -225,9 +226,10 @@ class Trace:
     """Device time of every kernel the library launches from this thread while the
     context is active (relpos_trace_begin / relpos_trace_end): each kernel is bracketed
     by two CUDA events on its launch stream.  After synchronising, ``kernels()`` gives
-    [(name, milliseconds)] in launch order."""
+    [(name, milliseconds)] in launch order.  ``only``: record only the kernels of that
+    name (two events per launch of it, nothing between the others)."""
 
-    def __init__(self, capacity: int = TRACE_MAX):
+    def __init__(self, capacity: int = TRACE_MAX, only: Optional[str] = None):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
         for e in self.events:  # torch creates the CUDA event at its first record
             e.record()
@@ -235,6 +237,8 @@ class Trace:
         self.c = relpos_trace_t()
         self.c.events = ctypes.cast(self._handles, ctypes.POINTER(ctypes.c_void_p))
         self.c.capacity = capacity
+        self._only = None if only is None else only.encode()
+        self.c.only = self._only
 
     def __enter__(self):
         rc = load().relpos_trace_begin(ctypes.byref(self.c))

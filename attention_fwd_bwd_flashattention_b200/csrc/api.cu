@@ -143,7 +143,7 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
-  if (p.shaw_v) return false;  // Shaw's value-side term runs on the CUDA-core kernels
+  if (p.shaw_v && pass == 1) return false;  // the backward of Shaw's value-side term runs on the CUDA-core kernels
   if (pass == 1)
     return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p)) ||
            (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p)) || (p.mech == rp::M_DEB && rp::tc_bwd_deb_supported(p));
@@ -346,6 +346,7 @@ static int check_seqlens(const relpos_params_t *P) {
 extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, const void *k, const void *v,
                                const void *const rel[3], void *o, float *lse, void *workspace,
                                size_t workspace_bytes, int32_t *dev_status, void *stream) {
+  cudaGetLastError();  // an error left by an earlier, unrelated call in this thread is not ours
   Prm p;
   int e = validate_and_fill(params, p);
   if (e) return e;
@@ -393,6 +394,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
                                const void *const rel[3], const void *o, const float *lse, const void *dout,
                                void *dq, void *dk, void *dv, float *const drel[3], void *workspace,
                                size_t workspace_bytes, int32_t *dev_status, void *stream) {
+  cudaGetLastError();  // an error left by an earlier, unrelated call in this thread is not ours
   Prm p;
   int e = validate_and_fill(params, p);
   if (e) return e;

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(32, 1) wait_selftest_kernel(int32_t *status, u
 
 extern "C" int relpos_selftest_wait(uint64_t limit_ns, int32_t *dev_status, unsigned long long *dev_elapsed_ns,
                                     void *stream) {
+  cudaGetLastError();  // an error left by an earlier, unrelated call in this thread is not ours
   if (!dev_status || !dev_elapsed_ns || limit_ns < 1000000ull || limit_ns > 10000000000ull) return RELPOS_ERR_INVALID_ARG;
   cudaPointerAttributes a1, a2;
   if (cudaPointerGetAttributes(&a1, dev_status) != cudaSuccess || cudaPointerGetAttributes(&a2, dev_elapsed_ns) != cudaSuccess) {

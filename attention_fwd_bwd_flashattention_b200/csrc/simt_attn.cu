@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(NT, 1) fwd_kernel(Prm p) {
   extern __shared__ float smem[];
   const Sm sm = carve(smem);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int m = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int m = (int)blockIdx.x + p.mem_len / BM, h = blockIdx.y, b = blockIdx.z;  // memory-placeholder tiles skipped
   const int L = p.L, i0 = m * BM;
   const size_t base = ((size_t)b * p.H + h) * (size_t)L * HD;
   const T *Qg = (const T *)p.q + base, *Kg = (const T *)p.k + base, *Vg = (const T *)p.v + base;
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_q_kernel(Prm p) {
   extern __shared__ float smem[];
   const Sm sm = carve(smem);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int m = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int m = (int)blockIdx.x + p.mem_len / BM, h = blockIdx.y, b = blockIdx.z;  // memory-placeholder tiles skipped
   const int L = p.L, i0 = m * BM;
   const size_t bh = (size_t)b * p.H + h, base = bh * (size_t)L * HD;
   const T *Qg = (const T *)p.q + base, *Kg = (const T *)p.k + base, *Vg = (const T *)p.v + base,
@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_kv_kernel(Prm p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) dK[a][e] = dV[a][e] = 0.f;
   }
-  const int mStart = p.causal ? n : 0;
+  const int mStart = max(p.causal ? n : 0, p.mem_len / BM);  // memory-placeholder query tiles skipped
   for (int m = mStart; m < p.nT; ++m) {
     const int i0 = m * BM;
     const int dmin = j0 - (i0 + BM - 1), dmax = j0 + BN - 1 - i0;
@@ -739,7 +739,8 @@ __global__ void __launch_bounds__(NT, 1) bwd_diag_kernel(Prm p) {
   const int Delta = p.causal ? band : band - (p.nT - 1);
   const int mlo = max(0, Delta), mhi = min(p.nT - 1, p.nT - 1 + Delta);
   const int m0 = mlo + chunk * p.diag_ch, m1 = min(mhi, m0 + p.diag_ch - 1);
-  if (m0 > m1) return;
+  if (m0 > m1) return;  // no such chunk (never read)
+  const int mfirst = max(m0, p.mem_len / BM);  // memory-placeholder query tiles skipped (the partial still written)
   const int L = p.L;
   const size_t bh = (size_t)b * p.H + h, base = bh * (size_t)L * HD;
   const T *Qg = (const T *)p.q + base, *Kg = (const T *)p.k + base, *Vg = (const T *)p.v + base,
@@ -751,7 +752,7 @@ __global__ void __launch_bounds__(NT, 1) bwd_diag_kernel(Prm p) {
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int e = 0; e < 4; ++e) G[a][e] = 0.f;
-  for (int m = m0; m <= m1; ++m) {
+  for (int m = mfirst; m <= m1; ++m) {
     const int n = m - Delta, i0 = m * BM, j0 = n * BN;
     __syncthreads();
     load_rows(Qg, i0, L, sm.Q);
@@ -882,7 +883,7 @@ static cudaError_t run_fwd_t(const Prm &p, cudaStream_t st) {
   auto k = fwd_kernel<MECH, T>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nT, p.H, p.B);
+  dim3 grid(p.nT - p.mem_len / BM, p.H, p.B);  // no memory-placeholder query tiles
   RP_TRACED("simt_fwd_kernel", st, k<<<grid, NT, SMEM_BYTES, st>>>(p));
   return cudaGetLastError();
 }
@@ -897,10 +898,10 @@ static cudaError_t run_bwd_t(const Prm &p, cudaStream_t st) {
   auto kkv = bwd_kv_kernel<MECH, T>;
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess) return e;
-  dim3 grid(p.nT, p.H, p.B);
+  dim3 grid(p.nT, p.H, p.B), gq(p.nT - p.mem_len / BM, p.H, p.B);  // no memory-placeholder query tiles
   RP_TRACED("simt_bwd_kv_kernel", st, kkv<<<grid, NT, SMEM_BYTES, st>>>(p));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  RP_TRACED("simt_bwd_q_kernel", st, kq<<<grid, NT, SMEM_BYTES, st>>>(p));
+  RP_TRACED("simt_bwd_q_kernel", st, kq<<<gq, NT, SMEM_BYTES, st>>>(p));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (MECH == M_TXL) {
     auto kd = bwd_diag_kernel<T>;

@@ -147,7 +147,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
   const int BH = p.B * p.H;
   const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, j0 = n * 128;
-  const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
+  // query tiles holding only Transformer-XL memory placeholders (rows < mem_len) are skipped
+  const int mStart = max(p.causal ? n : 0, p.mem_len / 128), iters = p.nT - mStart;
   const int klen = key_len(p, bh / p.H);  // keys j >= klen of this batch are masked
   if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0, no du contribution (whole CTA, no barrier yet)
     for (int x = tid; x < 128 * (HD / 8); x += NTHREADS) {
@@ -452,7 +453,8 @@ __global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_co
   const int BH = p.B * p.H;
   const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH, h = bh % p.H;
   const int L = p.L, j0 = n * 128;
-  const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
+  // query tiles holding only Transformer-XL memory placeholders (rows < mem_len) are skipped
+  const int mStart = max(p.causal ? n : 0, p.mem_len / 128), iters = p.nT - mStart;
   const int klen = key_len(p, bh / p.H);
   if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0, no du contribution (whole CTA, no barrier yet)
     for (int x = tid; x < 128 * (HD / 8); x += NTH) {
@@ -918,8 +920,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
   const int band = p.causal ? D : D + (p.nT - 1);
   const int b = bh / p.H, h = bh % p.H;
   const int mlo = max(0, D), mhi = min(p.nT - 1, p.nT - 1 + D);
-  const int m0 = mlo + chunk * A.dg_ch, m1a = min(mhi, m0 + A.dg_ch - 1);
-  if (m0 > m1a) return;  // no such chunk (never read): whole CTA, before any barrier or TMEM allocation
+  const int mc = mlo + chunk * A.dg_ch, m1a = min(mhi, mc + A.dg_ch - 1);
+  if (mc > m1a) return;  // no such chunk (never read): whole CTA, before any barrier or TMEM allocation
+  const int m0 = max(mc, p.mem_len / 128);  // memory-placeholder query tiles are skipped
   // keys j >= klen of this batch are masked: tiles whose key tile m - D lies past them are skipped
   const int klen = key_len(p, bh / p.H);
   const int m1 = min(m1a, (klen + 127) / 128 - 1 + D);
@@ -1192,8 +1195,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_dgs_kernel(const __grid_co
   const int D = p.causal ? rank : ((rank & 1) ? (rank + 1) / 2 : -(rank / 2));
   const int band = p.causal ? D : D + (p.nT - 1);
   const int mlo = max(0, D), mhi = min(p.nT - 1, p.nT - 1 + D);
-  const int m0 = mlo + chunk * A.dg_ch, m1a = min(mhi, m0 + A.dg_ch - 1);
-  if (m0 > m1a) return;  // no such chunk (never read)
+  const int mc = mlo + chunk * A.dg_ch, m1a = min(mhi, mc + A.dg_ch - 1);
+  if (mc > m1a) return;  // no such chunk (never read)
+  const int m0 = max(mc, p.mem_len / 128);  // memory-placeholder query tiles are skipped
   const int klen = key_len(p, bh / p.H);
   const int m1 = min(m1a, (klen + 127) / 128 - 1 + D);  // the tiles the query-tile kernel stored
   float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
@@ -1493,16 +1497,17 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_bwd_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dg::SMEM)) != cudaSuccess)
     return e;
   const unsigned tiles = (unsigned)(nT * p0.H * p0.B);
+  const unsigned qtiles = (unsigned)((nT - p0.mem_len / 128) * p0.H * p0.B);  // no memory-placeholder query tiles
   if (a.pd_stored) {  // the query-tile kernel first: the key-tile pass streams its P / dS tiles
     if ((e = cudaFuncSetAttribute(tc_bwd_kvs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess)
       return e;
-    RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a));
+    RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<qtiles, NTHREADS, qk::SMEM, st>>>(a));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     RP_TRACED("tc_bwd_kvs_kernel", st, tc_bwd_kvs_kernel<<<tiles, kvs::NTH, kvs::SMEM, st>>>(a));
   } else {
     RP_TRACED("tc_bwd_kv_kernel", st, tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<tiles, NTHREADS, qk::SMEM, st>>>(a));
+    RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<qtiles, NTHREADS, qk::SMEM, st>>>(a));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.pd_stored) {

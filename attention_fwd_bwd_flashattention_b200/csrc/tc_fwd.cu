@@ -66,6 +66,7 @@ enum {
 };
 
 constexpr uint32_t TM_S = 0, TM_REL = 128, TM_O = 384, TM_COLS = 512;
+constexpr uint32_t TM_P = 128;  // Shaw with the value table: P (bf16 pairs, 64 columns) as the PV MMA's A operand
 
 struct FwdArgs {
   CUtensorMap mq, mk, mv, mt0, mt1;
@@ -86,8 +87,52 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int MECH>
+// Shaw's value side: this thread's NC probabilities of row il written into the
+// offset-order tile Pe at column (delta + c) & 127 (delta = j - i), in the layout of the
+// P tile (128-byte-swizzled K-major, 64-column halves 16 KB apart).  Clipped pairs are
+// passed as 0, so the row's 128 keys fill every column once.  pk[k] = (v[2k], v[2k+1]);
+// C0 = column of v[0].  Aligned bf16 pairs; when C0 is odd the first and the last value
+// share their pair with a neighbouring thread's and are written alone.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t pe_off(uint32_t t, uint32_t rowb, uint32_t r7) {  // t = 2 col, col even
+  return ((t << 7) & 0x4000u) + rowb + ((t & 126u) ^ r7);
+}
+__device__ __forceinline__ void store_pe(uint8_t *E, int il, uint32_t C0, const uint32_t (&pk)[NC / 2]) {
+  const bool odd = (C0 & 1u) != 0;
+  const uint32_t rowb = 128u * (uint32_t)il, r7 = (uint32_t)(il & 7) << 4;
+  const uint32_t sel = odd ? 0x5432u : 0x3210u;  // odd: (high half of pk[k], low half of pk[k+1])
+  const uint32_t B0 = (C0 + (odd ? 1u : 0u)) & 127u;
+#pragma unroll
+  for (int k = 0; k < NC / 2 - 1; ++k) {
+    const uint32_t col = (B0 + 2u * k) & 127u;
+    *reinterpret_cast<uint32_t *>(E + pe_off(2u * col, rowb, r7)) = prmt(pk[k], pk[k + 1], sel);
+  }
+  if (!odd) {
+    const uint32_t col = (B0 + 2u * (NC / 2 - 1)) & 127u;
+    *reinterpret_cast<uint32_t *>(E + pe_off(2u * col, rowb, r7)) = pk[NC / 2 - 1];
+  } else {
+    const uint32_t c0 = (C0 - 1u) & 127u, c31 = (C0 + NC - 1) & 127u;
+    *reinterpret_cast<uint16_t *>(E + pe_off(2u * c0, rowb, r7) + 2u) = (uint16_t)(pk[0] & 0xFFFFu);
+    *reinterpret_cast<uint16_t *>(E + pe_off(2u * c31, rowb, r7)) = (uint16_t)(pk[NC / 2 - 1] >> 16);
+  }
+}
+
+// Shaw band tile: some of its offsets 128 (n - m) + [-127, 127] are unclipped.
+__device__ __forceinline__ bool shaw_band(int clip, int m, int n) {
+  const int D = m - n;
+  return 128 * (D < 0 ? -D : D) - 127 < clip;
+}
+
+// VAL (Shaw only): the value-side table aV (rel1) adds sum_j P_ij aV[clip(j - i) + c] to
+// every O_i: band tiles through one more MMA O += Pe aV[0..127] with P in offset order,
+// the clipped pairs through two per-row sums applied to aV[0] / aV[2c] in the epilogue.
+template <int MECH, bool VAL = false>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ FwdArgs A) {
+  constexpr bool SV = MECH == M_SHAW && VAL;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
@@ -194,6 +239,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           umma_commit(BAR(B_PFULLPRO));
           ok = wait_bar(B_PFREEPRO, 0);
         }
+        if (SV && ok) {  // the QA MMA is done with the table a: aV rows 0..127 take its place
+          expect(B_PLOAD, 1, 16384);
+          tma_load_3d(sbase + OFF_R, &A.mt1, BAR(B_PLOAD), 0, 0, h);
+        }
       }
       if (MECH == M_TXL) {  // first relation block: offsets 128 m + [0, 128)
         expect(B_PLOAD, 0, 16384);
@@ -214,16 +263,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       };
       auto issue_pv = [&](int n) {  // O (+)= P(n) V(n)
         const int ps = n & 1;
+        if constexpr (SV) {  // P from TMEM; on band tiles also O += Pe aV (Pe in the P smem tile)
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
-                    sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024), idPV, (n > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 8; ++k)
+            umma_bf16_ts(tbase + TM_O, tbase + TM_P + 8 * k, sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024),
+                         idPV, (n > 0 || k > 0) ? 1u : 0u);
+          if (shaw_band(p.clip, m, n)) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
+                        sdesc_sw128(sbase + OFF_R + 2048 * k, 16, 1024), idPV, 1u);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
+                      sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024), idPV, (n > 0 || k > 0) ? 1u : 0u);
+        }
         umma_commit(BAR(B_PV));
       };
       if (ok) {
         issue_kv(0);
         if (nTiles > 1) issue_kv(1);
       }
+      if (SV && ok) ok = wait_load(B_PLOAD, 1);  // aV staged before the first PV
       for (int n = 0; ok && n < nTiles; ++n) {
         const int st = n & 1;
         const int Delta = m - n;
@@ -293,6 +356,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     float *rrow = rot + il * ROT_LD;
     float *red = (float *)(smem + OFF_RED);
     float m2 = -INFINITY, lsum = 0.f;
+    float sL = 0.f, sR = 0.f;  // Shaw value side: mass of the row's keys clipped left (delta <= -c) / right (>= c)
     float cE0 = 0.f, cE1 = 0.f;
     bool good = true;  // warp-uniform: false once any wait of the CTA ran out
     if (MECH == M_DEB && i < L) {
@@ -509,6 +573,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           }
           if (need) {
             lsum *= alpha;
+            if (SV) {
+              sL *= alpha;
+              sR *= alpha;
+            }
             m2 = mt;
           }
         }
@@ -520,7 +588,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         lsum += x[t];
       }
       if (n >= 1) good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
-      if (good) {
+      if constexpr (SV) {
+        const int d0 = j0 + cb - i;  // delta of this thread's first key
+        const int eLo = max(0, 1 - p.clip - d0), eHi = min(NC - 1, p.clip - 1 - d0);  // unclipped: eLo..eHi
+#pragma unroll
+        for (int e = 0; e < NC; ++e) {
+          if (e < eLo) sL += x[e];
+          else if (e > eHi) sR += x[e];
+        }
+        if (good) {
+          uint32_t pk[NC / 2];
+#pragma unroll
+          for (int k = 0; k < NC / 2; ++k) pk[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
+          tmem_st16(tl + TM_P + 16 * qt, pk);
+          if (shaw_band(p.clip, m, n)) {
+#pragma unroll
+            for (int k = 0; k < NC / 2; ++k) {
+              const float v0 = (2 * k >= eLo && 2 * k <= eHi) ? x[2 * k] : 0.f;
+              const float v1 = (2 * k + 1 >= eLo && 2 * k + 1 <= eHi) ? x[2 * k + 1] : 0.f;
+              pk[k] = pack_bf16x2(v0, v1);
+            }
+            store_pe(smem + OFF_P, il, (uint32_t)(d0 + p.clip) & 127u, pk);
+          }
+          tmem_wait_st();
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(BAR(B_PFULL));
+        }
+      } else if (good) {
         // P quarter-row -> smem sub-tile qt / 2, K-major 128B swizzle: chunk c of row r at chunk c ^ (r & 7)
 #pragma unroll
         for (int cc = 0; cc < NC / 8; ++cc) {
@@ -540,10 +635,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     // ---- epilogue: O / l (l summed over the row's threads), LSE ----
     float *rl = red + TPR * 128 * (nTiles & 1);
     rl[128 * qt + il] = lsum;
+    if (SV) {  // the per-tile vector buffer is unused by Shaw: it carries the clipped sums
+      vec[128 * qt + il] = sL;
+      vec[512 + 128 * qt + il] = sR;
+    }
     named_bar_sync(1, NSOFT);
-    float ltot = 0.f;
+    float ltot = 0.f, sLt = 0.f, sRt = 0.f;
 #pragma unroll
     for (int u = 0; u < TPR; ++u) ltot += rl[128 * u + il];
+    if (SV) {
+#pragma unroll
+      for (int u = 0; u < TPR; ++u) {
+        sLt += vec[128 * u + il];
+        sRt += vec[512 + 128 * u + il];
+      }
+    }
     good = good && warp_wait(BAR(B_PV), (nTiles - 1) & 1, abort_flag, status);
     if (good) {
       tc_fence_after();
@@ -552,6 +658,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       uint32_t r[16];
       tmem_ld16(tl + TM_O + 16 * qt, r);
       tmem_wait_ld();
+      if (SV) {  // clipped pairs: O += sL aV[0] + sR aV[2c]
+        const __nv_bfloat16 *a0 = (const __nv_bfloat16 *)p.rel1 + (size_t)h * p.nrows * HD + 16 * qt;
+        const __nv_bfloat16 *a1 = a0 + (size_t)(2 * p.clip) * HD;
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          r[e] = __float_as_uint(u2f(r[e]) + sLt * __bfloat162float(a0[e]) + sRt * __bfloat162float(a1[e]));
+      }
       if (i < L) {
 #pragma unroll
         for (int c8 = 0; c8 < 2; ++c8) {
@@ -673,12 +786,13 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MECH>
+template <int MECH, bool VAL = false>
 static cudaError_t launch_fwd_t(const FwdArgs &a, cudaStream_t st) {
-  auto k = tc_fwd_kernel<MECH>;
+  auto k = tc_fwd_kernel<MECH, VAL>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  RP_TRACED("tc_fwd_kernel", st, k<<<(unsigned)(a.p.nT * a.p.H * a.p.B), NTHREADS, SMEM_BYTES, st>>>(a));
+  // query tiles holding only Transformer-XL memory placeholders (rows < mem_len) are not launched
+  RP_TRACED("tc_fwd_kernel", st, k<<<(unsigned)((a.p.nT - a.p.mem_len / BM) * a.p.H * a.p.B), NTHREADS, SMEM_BYTES, st>>>(a));
   return cudaGetLastError();
 }
 
@@ -728,6 +842,7 @@ cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st) {
 
 bool tc_supported(const Prm &p) {
   if (p.mech == M_SHAW && 2 * p.clip + 1 > 131) return false;  // QA row must fit the 132-float smem row
+  if (p.shaw_v && p.clip > 64) return false;  // the unclipped offsets 1 .. 2c - 1 must fit the 128 columns of Pe
   return true;
 }
 
@@ -747,6 +862,7 @@ cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st) {
   if (p.mech == M_SHAW) {
     a.shaw_n = ((2 * p.clip + 1) + 15) / 16 * 16;
     ok = ok && make_map(&a.mt0, p.rel0, p.nrows, p.H, a.shaw_n);
+    if (p.shaw_v) ok = ok && make_map(&a.mt1, p.rel1, p.nrows, p.H, 128);  // aV rows 0..127 (past 2c: zeros)
   }
   if (p.mech == M_DEB) ok = ok && make_map(&a.mt0, p.rel0, p.nrows, p.H, 256) && make_map(&a.mt1, p.rel1, p.nrows, p.H, 256);
   if (!ok) return cudaErrorInvalidValue;
@@ -754,7 +870,7 @@ cudaError_t tc_fwd(const Prm &p, const TcWork &w, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   switch (p.mech) {
     case M_T5: return launch_fwd_t<M_T5>(a, st);
-    case M_SHAW: return launch_fwd_t<M_SHAW>(a, st);
+    case M_SHAW: return p.shaw_v ? launch_fwd_t<M_SHAW, true>(a, st) : launch_fwd_t<M_SHAW>(a, st);
     case M_TXL: return launch_fwd_t<M_TXL>(a, st);
     default: return launch_fwd_t<M_DEB>(a, st);
   }

@@ -4,6 +4,8 @@
 // one kernel of a pass can be timed on the device without a profiler.  The events are
 // the caller's; the registration is per host thread, so calls made from other threads
 // are not traced and no state is shared between threads.
+#include <string.h>
+
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
@@ -17,7 +19,7 @@ static thread_local relpos_trace_t *t_trace = nullptr;
 void trace_pre(const char *name, cudaStream_t st) {
   nvtxRangePushA(name);
   relpos_trace_t *t = t_trace;
-  if (!t) return;
+  if (!t || (t->only && strcmp(t->only, name) != 0)) return;
   if (t->count >= t->capacity) {
     ++t->dropped;
     return;
@@ -29,6 +31,7 @@ void trace_pre(const char *name, cudaStream_t st) {
 void trace_post(cudaStream_t st) {
   nvtxRangePop();
   relpos_trace_t *t = t_trace;
+  // the kernel just launched was recorded by trace_pre iff its slot holds a name
   if (!t || t->count >= t->capacity || t->names[t->count] == nullptr) return;
   cudaEventRecord((cudaEvent_t)t->events[2 * t->count + 1], st);
   ++t->count;

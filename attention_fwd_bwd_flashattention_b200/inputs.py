@@ -50,6 +50,9 @@ class Workload:
     # 0.02; None keeps 0.02.  Parity tests draw them at O(1) so that the relative term
     # moves the outputs by far more than the tolerance.
     rel_std: Optional[float] = None
+    # Transformer-XL (causal) memory: M cached keys / values before the segment's L
+    # queries; k, v and r then have M + L rows
+    mem_len: int = 0
 
     @property
     def scale(self) -> float:
@@ -80,6 +83,10 @@ WORKLOADS["txl_varlen_B4_L8192_bf16"] = Workload("txl_varlen_B4_L8192_bf16", TXL
 WORKLOADS["shaw_value_L2048_bf16"] = Workload("shaw_value_L2048_bf16", SHAW, torch.bfloat16, False, 2, 8, 2048,
                                               shaw_value=True)
 WORKLOADS["alibi_causal_L8192_bf16"] = Workload("alibi_causal_L8192_bf16", ALIBI, torch.bfloat16, True, 1, 8, 8192)
+# Transformer-XL with a segment memory as long as the segment (M = L = 4096): the same
+# 8192 causal positions as the 8K workload, the first 4096 of them cached keys only.
+WORKLOADS["txl_mem_M4096_L4096_bf16"] = Workload("txl_mem_M4096_L4096_bf16", TXL, torch.bfloat16, True, 1, 8, 4096,
+                                                 mem_len=4096)
 WORKLOADS["t5_causal_L8192_bf16"] = Workload("t5_causal_L8192_bf16", T5, torch.bfloat16, True, 1, 8, 8192,
                                              t5_bidirectional=False)
 
@@ -109,9 +116,10 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
     def nrm(*shape, std=1.0):
         return (torch.randn(*shape, generator=g, dtype=torch.float32) * std)
 
+    Lk = L + wl.mem_len  # keys and values: the memory, then the segment
     q = nrm(B, H, L, d).to(dt)
-    k = nrm(B, H, L, d).to(dt)
-    v = nrm(B, H, L, d).to(dt)
+    k = nrm(B, H, Lk, d).to(dt)
+    v = nrm(B, H, Lk, d).to(dt)
     do = nrm(B, H, L, d).to(dt)
     if wl.mech == ALIBI:
         rel = [torch.pow(2.0, -8.0 * torch.arange(1, H + 1, dtype=torch.float32) / H)]
@@ -123,11 +131,11 @@ def make_inputs(wl: Workload, seed: int = 0) -> dict:
         if wl.shaw_value:
             rel.append(nrm(H, 2 * wl.shaw_clip + 1, d, std=sd).to(dt))
     elif wl.mech == TXL:
-        n_off = L if wl.causal else 2 * L - 1
+        n_off = Lk if wl.causal else 2 * L - 1
         W_R = nrm(TXL_EMB, H * d, std=0.02).to(torch.float64)
         u = nrm(H, d, std=0.02).to(dt)
         vv = nrm(H, d, std=0.02).to(dt)
-        r = (txl_sinusoid(n_off, wl.causal, L) @ W_R).reshape(n_off, H, d).permute(1, 0, 2).contiguous()
+        r = (txl_sinusoid(n_off, wl.causal, Lk) @ W_R).reshape(n_off, H, d).permute(1, 0, 2).contiguous()
         rel = [r.to(dt), u, vv]
     else:
         sd = 0.02 if wl.rel_std is None else wl.rel_std

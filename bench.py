@@ -49,7 +49,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ----------------------------------------------------------------------------
 def pairs_of(wl):
     """Unmasked (query, key) pairs of one head, summed over the batch: every query
-    with the keys before its batch's key length (and not after it when causal)."""
+    with the keys before its batch's key length (and not after it when causal); with a
+    Transformer-XL memory of M keys, query i sees the M cached keys and i + 1 of the
+    segment's."""
+    if wl.mem_len:
+        return wl.B * (wl.L * wl.mem_len + wl.L * (wl.L + 1) // 2)
     lens = wl.seqlens_k if wl.seqlens_k is not None else (wl.L,) * wl.B
     tot = 0
     for lk in lens:
@@ -85,32 +89,23 @@ def fa_flops(wl):
 def kernel_launches(wl, path):
     """Kernels this library launches per forward and per backward call (the dispatch of csrc/api.cu)."""
     t5 = 1 if wl.mech in (T5, ALIBI) else 0  # per-call per-offset bias preparation
-    tc = path != "simt" and wl.dtype == torch.bfloat16 and not wl.shaw_value  # the value side runs on CUDA cores
+    tc = path != "simt" and wl.dtype == torch.bfloat16
+    tc_bwd = tc and not wl.shaw_value  # the value side's backward runs on CUDA cores
     if tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
         fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
     else:
         fwd = 1 + t5
-    if tc and wl.mech == TXL:  # D, relation prep, key-tile, query-tile, diagonal, dr and u/v reductions
+    if tc_bwd and wl.mech == TXL:  # D, relation prep, key-tile, query-tile, diagonal, dr and u/v reductions
         bwd = 7
-    elif tc and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction
+    elif tc_bwd and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction
         bwd = 5
-    elif tc and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
+    elif tc_bwd and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
         bwd = 5
-    elif tc and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction
+    elif tc_bwd and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction
         bwd = 7
     else:  # D, key-tile, query-tile, then the table-gradient reductions (Shaw's value side: one more)
         bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[wl.mech] + (1 if wl.shaw_value else 0)
     return fwd, bwd
-
-
-# DRAM traffic per call (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
-# capture of the same build and workload, summed over the pass's captured kernels; set to
-# None whenever those kernels change.  Source: profiles/tc_kernels_txl_causal_L8192.md.
-DRAM_TRAFFIC = {
-    ("txl_causal_L8192_bf16", "relpos_attn_fwd"): (34.26e6, "tc_fwd_kernel (the relation prep kernel not captured)"),
-    ("txl_causal_L8192_bf16", "relpos_attn_bwd"): (
-        3045.74e6, "dvec, tc_bwd_q, tc_bwd_kvs, tc_bwd_dgs, reduce_dr, reduce_uv (the relation prep kernel not captured)"),
-}
 
 
 def median_iqr(xs):
@@ -276,6 +271,11 @@ def oracle_sample(wl, rows_fraction=None):
                      shaw_value=wl.shaw_value)
     f_fwd, f_bwd = algo_flops(one)
     t0 = time.perf_counter()
+    if wl.mem_len:  # the memory formula on the whole slice (no row sampling)
+        orc.txl_memory_forward(q, k, v, rel, wl.scale, cfg)
+        orc.txl_memory_backward(q, k, v, rel, do, wl.scale, cfg)
+        return (time.perf_counter() - t0, f_fwd + f_bwd,
+                f"1 of {wl.B * wl.H} (batch, head) slices, memory {wl.mem_len} + segment {wl.L}, forward + backward")
     if rows_fraction is None:
         orc.forward(wl.mech, q, k, v, rel, wl.causal, wl.scale, cfg, seqlens_k=lk)
         orc.backward(wl.mech, q, k, v, rel, wl.causal, do, wl.scale, cfg, seqlens_k=lk)
@@ -337,7 +337,6 @@ KERNEL_CREDIT_U = {
 # removed whenever that kernel changes.
 KERNEL_TRAFFIC = {
     ("txl_causal_L8192_bf16", "tc_bwd_q_kernel"): 1126.0e6,
-    ("txl_causal_L8192_bf16", "tc_fwd_kernel"): 34.26e6,
 }
 # Further workloads timed by the default run (one line, sub-record "workloads"): the other
 # configuration quoted at L = 8192 (DeBERTa), the Shaw configuration, and one point of the
@@ -350,7 +349,7 @@ def params_of(wl, path):
                   dtype=bd.BF16 if wl.dtype == torch.bfloat16 else bd.F32, causal=wl.causal, scale=wl.scale,
                   kernel_path=path, t5_num_buckets=wl.t5_num_buckets, t5_max_distance=wl.t5_max_distance,
                   t5_bidirectional=wl.t5_bidirectional, shaw_clip=wl.shaw_clip, deberta_span=wl.deberta_span,
-                  shaw_value=wl.shaw_value)
+                  shaw_value=wl.shaw_value, mem_len=wl.mem_len)
     return P
 
 
@@ -395,18 +394,28 @@ class Case:
 
 def time_case(c, steps, warmup, flush, stream, world, on_region=None):
     """W untimed steps, then `steps` steps each timed with CUDA events on the launching
-    stream (fwd and bwd separately), L2 flushed before each (untimed); every kernel the
-    library launches in the timed steps is bracketed by its own events (bd.Trace).
-    Returns (fwd_ms, bwd_ms, kernels) with kernels = {name: [ms of each launch]}."""
-    for _ in range(warmup):
+    stream (fwd and bwd separately), L2 flushed before each (untimed).  The warm-up steps
+    trace every kernel the library launches (bd.Trace: events around each launch) to
+    find the one with the largest share; in the timed steps only that kernel is
+    bracketed by its own events (two per launch, nothing between the other kernels).
+    Returns (fwd_ms, bwd_ms, warm, dom) with warm = {name: [ms of each warm-up launch]}
+    and dom = (name, [ms of each timed launch])."""
+    warm_traces = [bd.Trace(32) for _ in range(warmup)]
+    for w in range(warmup):
         flush.fill_(1.0)
-        c.fwd(stream)
-        c.bwd(stream)
+        with warm_traces[w]:
+            c.fwd(stream)
+            c.bwd(stream)
         if world > 1:
             rdist.allreduce_table_grads(c.drel)
     torch.cuda.synchronize()
+    warm = {}
+    for t in warm_traces[1:] or warm_traces:  # the first warm-up step includes one-time set-up
+        for name, ms in t.kernels():
+            warm.setdefault(name, []).append(ms)
+    dom_name = max(warm, key=lambda n: sum(warm[n])) if warm else None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-    traces = [bd.Trace(16) for _ in range(steps)]
+    traces = [bd.Trace(8, only=dom_name) for _ in range(steps)]
     torch.cuda.synchronize()
     rdist.barrier()
     torch.cuda.synchronize()
@@ -427,11 +436,8 @@ def time_case(c, steps, warmup, flush, stream, world, on_region=None):
     rdist.barrier()
     fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    kernels = {}
-    for t in traces:
-        for name, ms in t.kernels():
-            kernels.setdefault(name, []).append(ms)
-    return fwd_ms, bwd_ms, kernels
+    dom_ms = [ms for t in traces for _, ms in t.kernels()]
+    return fwd_ms, bwd_ms, warm, (dom_name, dom_ms)
 
 
 def kernel_table(kernels, steps, step_ms):
@@ -443,12 +449,11 @@ def kernel_table(kernels, steps, step_ms):
 def side_workload(name, dev, rank, world, flush, stream, peaks, steps):
     wl = WORKLOADS[name]
     c = Case(wl, dev, rank, bd.PATH_AUTO)
-    fwd_ms, bwd_ms, kernels = time_case(c, steps, 3, flush, stream, world)
+    fwd_ms, bwd_ms, warm, (dom, dom_ms) = time_case(c, steps, 3, flush, stream, world)
     f_fwd, f_bwd = algo_flops(wl)
     fm, bm = median_iqr(fwd_ms)[0], median_iqr(bwd_ms)[0]
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    ktab = kernel_table(kernels, steps, fm + bm)
-    dom = next(iter(ktab)) if ktab else None
+    ktab = kernel_table({dom: dom_ms}, steps, fm + bm) if dom else {}
     out = {"workload": name, "B": wl.B, "H": wl.H, "L": wl.L, "causal": wl.causal, "kernel_path": c.paths(),
            "steps": steps, "fwd_ms_median": fm, "bwd_ms_median": bm,
            "fwd_tflops": f_fwd / (fm * 1e-3) / 1e12, "bwd_tflops": f_bwd / (bm * 1e-3) / 1e12,
@@ -478,7 +483,8 @@ def run_ours(args, wl):
     base_mem = torch.cuda.memory_allocated(dev)
     clocks = ClockSampler(dev)
     clocks.start()
-    fwd_ms, bwd_ms, kernels = time_case(c, args.steps, args.warmup, flush, stream, world, on_region=clocks.mark)
+    fwd_ms, bwd_ms, warm, (dom, dom_ms) = time_case(c, args.steps, args.warmup, flush, stream, world,
+                                                    on_region=clocks.mark)
     clk = clocks.stop()
     tot_ms = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
     tot_ms = rdist.max_over_ranks(tot_ms)
@@ -497,8 +503,10 @@ def run_ours(args, wl):
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     fwd_avg = statistics.mean(fwd_ms)
     bwd_avg = statistics.mean(bwd_ms)
-    tensor_path = path_name == "auto" and wl.dtype == torch.bfloat16 and bd.tc_available(P)
-    ktab = kernel_table(kernels, args.steps, ms_step)
+    # every kernel's share from the traced warm-up steps; the dominant kernel's time from
+    # its own events in the timed steps
+    ktab_warm = kernel_table(warm, max(1, args.warmup - 1), statistics.mean(fwd_ms) + statistics.mean(bwd_ms))
+    ktab = {dom: kernel_table({dom: dom_ms}, args.steps, ms_step)[dom]}
     U = 2.0 * wl.H * wl.d * pairs_of(wl)
     # each pass timed as one unit with events (its helper kernels included): a pass of about
     # a millisecond timed by itself, so the burst peak is the denominator
@@ -506,30 +514,35 @@ def run_ours(args, wl):
     for name, fl, ms in (("relpos_attn_fwd", f_fwd, fwd_avg), ("relpos_attn_bwd", f_bwd, bwd_avg)):
         ach = fl / (ms * 1e-3) / 1e12
         passes.append({"pass": name, "achieved": ach, "ms": ms, "frac_of_burst": ach / burst})
-    if tensor_path:
+    pass_tc = [path_name == "auto" and wl.dtype == torch.bfloat16 and bd.tc_available(P, ps) for ps in (0, 1)]
+    dom_tc = not dom.startswith("simt_")
+    credit = None
+    if dom_tc:
         # the dominant kernel: the one with the largest share of the step, timed with its own
         # events around every launch in the timed region; credited with the algorithmic FLOPs
         # of the products it computes (the forward kernel: the whole forward)
-        dom = next(iter(ktab))
         credit = f_fwd if dom == "tc_fwd_kernel" else (KERNEL_CREDIT_U.get((wl.mech, dom), 0) * U or None)
-        if credit is not None:
-            per_launch = credit / ktab[dom]["launches_per_step"]
-            ach = per_launch / (ktab[dom]["ms_per_launch"] * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s", "frac": ach / burst,
-                    "traffic": KERNEL_TRAFFIC.get((wl.name, dom)), "kernel": dom, "flops_per_launch": per_launch,
-                    "ms_per_launch": ktab[dom]["ms_per_launch"], "share_of_step": ktab[dom]["share_of_step"],
-                    "peak_kind": f"bf16 burst ({peak_src}): kernel timed by itself with events"}
-        else:  # no per-kernel credit: the dominant pass
-            dp = max(passes, key=lambda x: x["ms"])
+    if credit is not None:
+        per_launch = credit / ktab[dom]["launches_per_step"]
+        ach = per_launch / (ktab[dom]["ms_per_launch"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s", "frac": ach / burst,
+                "traffic": KERNEL_TRAFFIC.get((wl.name, dom)), "kernel": dom, "flops_per_launch": per_launch,
+                "ms_per_launch": ktab[dom]["ms_per_launch"], "share_of_step": ktab[dom]["share_of_step"],
+                "peak_kind": f"bf16 burst ({peak_src}): kernel timed by itself with events"}
+    else:  # no per-kernel credit: the dominant pass, against the peak of the kernel family it runs on
+        di = 0 if fwd_avg > bwd_avg else 1
+        dp = passes[di]
+        if pass_tc[di]:
             roof = {"bound": "tensor", "achieved": dp["achieved"], "peak": burst, "unit": "TFLOP/s",
                     "frac": dp["frac_of_burst"], "traffic": None, "kernel": dp["pass"],
                     "peak_kind": f"bf16 burst ({peak_src}): pass timed as one unit"}
-    else:
-        # CUDA-core path: fp32 FFMA bound, peak = 148 SMs x 128 lanes x 2 flop x max SM clock
-        dp = max(passes, key=lambda x: x["ms"])
-        peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        roof = {"bound": "alu", "achieved": dp["achieved"], "peak": peak, "unit": "TFLOP/s", "frac": dp["achieved"] / peak,
-                "traffic": None, "kernel": dp["pass"], "peak_kind": "fp32 FFMA, 148 SM x 128 lanes x 2 x max clock"}
+        else:
+            # CUDA-core path: fp32 FFMA bound, peak = 148 SMs x 128 lanes x 2 flop x max SM clock
+            peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            roof = {"bound": "alu", "achieved": dp["achieved"], "peak": peak, "unit": "TFLOP/s",
+                    "frac": dp["achieved"] / peak, "traffic": None, "kernel": dp["pass"],
+                    "peak_kind": "fp32 FFMA, 148 SM x 128 lanes x 2 x max clock"}
+    tensor_path = pass_tc[0] and pass_tc[1]
 
     # ---- end to end through the public API: pinned host in, host out ----
     e2e = run_e2e(args, wl, c, dev, stream, world)
@@ -552,8 +565,8 @@ def run_ours(args, wl):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d, "causal": wl.causal,
-                   "seqlens_k": list(wl.seqlens_k) if wl.seqlens_k is not None else None,
-                   "kernel_path": "tcgen05" if tensor_path else "cuda-core fp32",
+                   "seqlens_k": list(wl.seqlens_k) if wl.seqlens_k is not None else None, "mem_len": wl.mem_len,
+                   "kernel_path": c.paths(),
                    "l2": "flushed before every timed step (256 MB write, untimed)",
                    "parallelism": f"dp{world} (weak; table grads all-reduced)" if world > 1 else "single GPU"},
         "tokens_per_s": tokens,
@@ -570,12 +583,12 @@ def run_ours(args, wl):
                       "bwd_median": median_iqr(bwd_ms)[0], "bwd_iqr": median_iqr(bwd_ms)[1]},
         "roofline": roof,
         "roofline_passes": passes,
-        "kernels": ktab,
+        "kernels_warmup": ktab_warm,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        # launches of this library's kernels in the timed steps, counted by the trace (the
-        # dispatch table of csrc/api.cu gives the same number: gpu_launches_expected)
-        "gpu_launches": sum(len(v) for v in kernels.values()),
+        # launches of this library's kernels in the timed steps: the traced warm-up steps'
+        # count per step (the dispatch table of csrc/api.cu gives gpu_launches_expected)
+        "gpu_launches": round(sum(len(v) for v in warm.values()) / max(1, args.warmup - 1) * args.steps),
         "gpu_launches_expected": (fl + bl) * args.steps,
         "clocks": clk,
         "workloads": side,

@@ -56,7 +56,9 @@
  *   - stream: a cudaStream_t (NULL = the legacy default stream).  All work is
  *     enqueued on it asynchronously.
  *
- * Errors: every call returns RELPOS_OK (0) or a negative RELPOS_ERR_* code.  Argument
+ * Errors: every call returns RELPOS_OK (0) or a negative RELPOS_ERR_* code.  The entry
+ * points clear the calling thread's CUDA "last error" before they enqueue anything, so
+ * that an error left by an earlier, unrelated runtime call is not reported as theirs.  Argument
  * errors (RELPOS_ERR_INVALID_ARG, _WORKSPACE, _UNSUPPORTED) are found before anything
  * is enqueued; after a launch or runtime failure (RELPOS_ERR_LAUNCH, _CUDA) the work
  * enqueued before it may still run, and the outputs are undefined.
@@ -127,7 +129,8 @@ typedef struct relpos_params {
    * with rel[1] = aV [H, 2c + 1, d] (params' dtype) and drel[1] = daV (float32).
    * The paper's Hugging Face page names Shaw among the mechanisms the method covers
    * (Community comment); the value side is the second table of Shaw's own paper.
-   * Such calls run on the CUDA-core kernels (RELPOS_PATH_TC is rejected). */
+   * The forward runs on the tensor-core kernels for bf16 and c <= 64, the backward on
+   * the CUDA-core kernels (RELPOS_PATH_TC is rejected for it). */
   int32_t shaw_value;
   /* Transformer-XL only, causal only (0 = none): length M of the cached memory of the
    * previous segment.  The L queries (q, o, lse, dq, dO: [B, H, L, d]) sit at positions
@@ -228,14 +231,17 @@ RELPOS_API int relpos_selftest_wait(uint64_t limit_ns, int32_t *dev_status,
  * events[2k] and events[2k + 1], its static name in names[k].  The caller creates the
  * 2 * capacity events (cudaEvent_t, timing enabled), keeps the struct alive while it is
  * registered, and reads the times with cudaEventElapsedTime after synchronising.
- * Kernels past capacity are not recorded and counted in `dropped`.  Registration is per
- * host thread: calls from other threads are neither traced nor affected. */
+ * Kernels past capacity are not recorded and counted in `dropped`.  With `only` set,
+ * kernels of other names are neither recorded nor counted (their NVTX ranges remain), so
+ * that one kernel can be timed with two events per launch.  Registration is per host
+ * thread: calls from other threads are neither traced nor affected. */
 #define RELPOS_TRACE_MAX 64
 typedef struct relpos_trace {
   void *const *events;                 /* in: 2 * capacity cudaEvent_t handles        */
   int32_t capacity;                    /* in: kernels to record, 1 .. RELPOS_TRACE_MAX */
   int32_t count;                       /* out: kernels recorded                       */
   int32_t dropped;                     /* out: kernels launched past capacity         */
+  const char *only;                    /* in: NULL, or record only kernels of this name */
   const char *names[RELPOS_TRACE_MAX]; /* out: name of kernel k                       */
 } relpos_trace_t;
 

@@ -60,14 +60,16 @@ def test_trace_struct_layout_matches_c(tmp_path):
     prog = tmp_path / "trace.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "relpos_attn.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %d\\n\", sizeof(relpos_trace_t), offsetof(relpos_trace_t,capacity),"
-        " offsetof(relpos_trace_t,count), offsetof(relpos_trace_t,dropped), offsetof(relpos_trace_t,names), RELPOS_TRACE_MAX);"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %d\\n\", sizeof(relpos_trace_t), offsetof(relpos_trace_t,capacity),"
+        " offsetof(relpos_trace_t,count), offsetof(relpos_trace_t,dropped), offsetof(relpos_trace_t,only),"
+        " offsetof(relpos_trace_t,names), RELPOS_TRACE_MAX);"
         "return 0;}\n")
     exe = tmp_path / "trace"
     subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(prog), "-o", str(exe)], check=True)
     got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     T = bd.relpos_trace_t
-    assert got == [ctypes.sizeof(T), T.capacity.offset, T.count.offset, T.dropped.offset, T.names.offset, bd.TRACE_MAX]
+    assert got == [ctypes.sizeof(T), T.capacity.offset, T.count.offset, T.dropped.offset, T.only.offset, T.names.offset,
+                   bd.TRACE_MAX]
 
 
 def test_trace_registration_is_validated(lib):
@@ -226,11 +228,13 @@ def test_resolved_paths(lib):
     # DeBERTa: spans that are multiples of 32 up to 256 take the tensor-core backward
     for span, want_b in ((256, TC), (32, TC), (96, TC), (24, SIMT), (288, SIMT)):
         assert bd.relpos_attn_resolved_path(bd.Params(mech=bd.DEBERTA, B=1, H=2, L=300, deberta_span=span), 1) == want_b, span
-    # Shaw's value-side term: CUDA-core kernels in both passes
+    # Shaw's value-side term: tensor-core forward for c <= 64, CUDA-core backward
     Pv = bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True)
-    assert (bd.relpos_attn_resolved_path(Pv, 0), bd.relpos_attn_resolved_path(Pv, 1)) == (SIMT, SIMT)
+    assert (bd.relpos_attn_resolved_path(Pv, 0), bd.relpos_attn_resolved_path(Pv, 1)) == (TC, SIMT)
+    Pv65 = bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, shaw_clip=65)
+    assert (bd.relpos_attn_resolved_path(Pv65, 0), bd.relpos_attn_resolved_path(Pv65, 1)) == (SIMT, SIMT)
     with pytest.raises(bd.RelposError):
-        bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, kernel_path=bd.PATH_TC), 0)
+        bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, kernel_path=bd.PATH_TC), 1)
     wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == SIMT
     assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC

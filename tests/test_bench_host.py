@@ -88,3 +88,10 @@ def test_kernel_table_shares():
     assert list(t) == ["a", "b"]
     assert t["a"] == {"launches_per_step": 1.0, "ms_per_launch": 1.0, "share_of_step": 0.5}
     assert t["b"]["launches_per_step"] == 2.0 and math.isclose(t["b"]["share_of_step"], 0.25)
+
+
+def test_pairs_of_memory_workload():
+    """Queries at positions M .. M + L - 1, each over every key up to its own position."""
+    wl = WORKLOADS["txl_mem_M4096_L4096_bf16"].with_(H=1, L=23, mem_len=9)
+    want = sum(9 + i + 1 for i in range(23))
+    assert bench.pairs_of(wl) == want

@@ -68,10 +68,12 @@ def test_parity_txl_smallest_backward_workspace(L, causal):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("M,L", [(64, 130), (100, 300), (256, 256), (5, 1)])
+@pytest.mark.parametrize("M,L", [(64, 130), (100, 300), (256, 256), (5, 1), (128, 128), (300, 200), (1000, 700)])
 def test_parity_txl_memory(M, L, dtype):
     """Transformer-XL with M cached keys / values before the segment's L: every output
-    against the oracle's memory formula."""
+    against the oracle's memory formula.  Query tiles that hold only memory placeholders
+    (floor(M / 128) of them on the tensor cores, floor(M / 64) on the CUDA cores) are not
+    computed at all; the cases put M below, on and across those tile boundaries."""
     g = torch.Generator().manual_seed(M * 7 + L)
     B, H, d = 2, 2, 64
 
