@@ -24,7 +24,10 @@ _lib = None
 
 class RelposError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {strerror(code)} ({code})")
+        detail = ""
+        if code == -4:  # RELPOS_ERR_LAUNCH: name the CUDA error behind it
+            detail = f"; cudaError {load().relpos_last_cuda_error()}"
+        super().__init__(f"{what}: {strerror(code)} ({code}{detail})")
         self.code = code
 
 
@@ -66,7 +69,7 @@ class relpos_trace_t(ctypes.Structure):
 
 EXPORTS = ("relpos_attn_workspace_size", "relpos_attn_fwd", "relpos_attn_bwd", "relpos_attn_fwd_noalloc",
            "relpos_attn_resolved_path", "relpos_selftest_wait", "relpos_trace_begin", "relpos_trace_end",
-           "relpos_strerror", "relpos_attn_version")
+           "relpos_last_cuda_error", "relpos_strerror", "relpos_attn_version")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -103,6 +106,8 @@ def load() -> ctypes.CDLL:
     lib.relpos_trace_end.restype = ctypes.c_int
     lib.relpos_strerror.argtypes = [ctypes.c_int]
     lib.relpos_strerror.restype = ctypes.c_char_p
+    lib.relpos_last_cuda_error.argtypes = []
+    lib.relpos_last_cuda_error.restype = ctypes.c_int
     lib.relpos_attn_version.argtypes = []
     lib.relpos_attn_version.restype = ctypes.c_int
     _lib = lib

@@ -293,8 +293,12 @@ static int rel_count(const Prm &p) {
   return p.mech == rp::M_TXL ? 3 : ((p.mech == rp::M_DEB || p.shaw_v) ? 2 : 1);
 }
 
+// CUDA error behind this thread's last RELPOS_ERR_LAUNCH (relpos_last_cuda_error)
+static thread_local int t_last_cuda = 0;
+
 static int to_status(cudaError_t e) {
   if (e == cudaSuccess) return RELPOS_OK;
+  t_last_cuda = (int)e;
   cudaGetLastError();  // clear a sticky launch-configuration error
   return RELPOS_ERR_LAUNCH;
 }
@@ -494,3 +498,5 @@ extern "C" const char *relpos_strerror(int status) {
 }
 
 extern "C" int relpos_attn_version(void) { return kVersion; }
+
+extern "C" int relpos_last_cuda_error(void) { return t_last_cuda; }

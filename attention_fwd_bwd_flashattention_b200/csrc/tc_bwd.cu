@@ -292,11 +292,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
       return (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
     };
     vec[128 + tid] = fetch1(0);
+    named_bar_sync(1, NSOFT);  // tile 0's terms; later tiles' are written before the previous tile's last barrier
     for (int t = 0; t < iters; ++t) {
       const int m = mStart + t, D = m - n, i = m * 128 + il;
       const float *tv = vec + 128 + 512 * (t & 1);
       const float nv = (t + 1 < iters) ? fetch1(t + 1) : 0.f;
-      named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
       const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
@@ -355,6 +355,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(BAR(B_SDPCONS));  // S / dP read: T(t + 1) may overwrite them
       }
+      // tile t + 1's terms into the other buffer (tile t - 1's, read before the previous
+      // tile's last barrier); the barrier below makes them visible
+      vec[128 + 512 * ((t + 1) & 1) + tid] = nv;
       named_bar_sync(1, NSOFT);  // every rot row read; the P / dS tiles overwrite them
       if (good) {
 #pragma unroll
@@ -369,7 +372,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
-      vec[128 + 512 * ((t + 1) & 1) + tid] = nv;  // tile t - 1's terms were last read before this tile's first barrier
     }
     // ---- epilogue: lanes are keys now; this thread takes 16 of the 64 columns ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
@@ -759,11 +761,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       return (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
     };
     if (tid < 384) vec[tid] = fetch1(0);
+    named_bar_sync(1, NSOFT);  // tile 0's terms; later tiles' are written before the previous tile's last barrier
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * 128, D = m - n;
       const float *tu = vec + 384 * (n & 1);
       const float nv = (tid < 384 && n + 1 < nTiles) ? fetch1(n + 1) : 0.f;
-      named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       if (n >= 1) good = good && warp_wait(BAR(B_PDSFREE), (n - 1) & 1, abort_flag, status);
       const bool hasA = block_valid(p, D), hasB = block_valid(p, D - 1);
@@ -838,6 +840,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         tc_fence_before();
         mbar_arrive(BAR(B_DPCONS));  // dP(n) read: the next relation block may overwrite it
       }
+      // tile n + 1's terms into the other buffer (tile n - 1's, read before the previous
+      // tile's last barrier); the barrier below makes them visible
+      if (tid < 384) vec[384 * ((n + 1) & 1) + tid] = nv;
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
         uint32_t pk[16];
@@ -859,7 +864,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
-      if (tid < 384) vec[384 * ((n + 1) & 1) + tid] = nv;  // tile n - 1's terms were read before this tile's first barrier
     }
     good = good && warp_wait(BAR(B_DSFREE), (nTiles - 1) & 1, abort_flag, status);  // last dQ MMAs done
     if (good) {
@@ -1066,11 +1070,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       return (j < L) ? A.uk[(size_t)bh * L + j] * c1 : 0.f;
     };
     if (tid < 384) vec[256 + tid] = fetch1(0);
+    named_bar_sync(1, NSOFT);  // the band's terms and tile 0's; later tiles' are written before the previous tile's last barrier
     for (int t = 0; t < iters; ++t) {
       const int m = m0 + t, nn = m - D, i = m * 128 + il, j0 = nn * 128;
       const float *tv = vec + 256 + 384 * (t & 1), *tu = tv + 256;
       const float nv = (tid < 384 && t + 1 < iters) ? fetch1(t + 1) : 0.f;
-      named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_TFULL), t & 1, abort_flag, status);
       if (t >= 1) good = good && warp_wait(BAR(B_PDSFREE), (t - 1) & 1, abort_flag, status);
       if (good) {
@@ -1128,6 +1132,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
 #pragma unroll
         for (int x = 0; x < NC / 2; ++x) ds[x] = 0u;
       }
+      // tile t + 1's terms into the other buffer (tile t - 1's, read before the previous
+      // tile's last barrier); the barrier below makes them visible
+      if (tid < 384) vec[256 + 384 * ((t + 1) & 1) + tid] = nv;
       named_bar_sync(1, NSOFT);  // every rot row read: E overwrites them
       if (good) {
         store_E(smem + OFF_ROT, il, cb, ds);
@@ -1135,7 +1142,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
-      if (tid < 384) vec[256 + 384 * ((t + 1) & 1) + tid] = nv;  // tile t - 1's terms were read before this tile's first barrier
     }
     // ---- epilogue: lane il now is offset c = il of both blocks; 16 columns per thread ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);

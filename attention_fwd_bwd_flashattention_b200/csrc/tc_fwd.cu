@@ -81,6 +81,11 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 // A wait whose result is the same on all 32 lanes (tcgen05.ld/st are warp-collective).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *ab, int32_t *st) {
   const bool ok = mbar_wait(bar, parity, ab, st, RELPOS_ERR_TIMEOUT_DEV);
@@ -386,8 +391,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     auto fetch_vec = [&](int n) {
       const int j0 = n * BN;
       float va = 0.f;
-      if (MECH == M_TXL) {
-        if (tid < 128 && j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid];
+      if (MECH == M_TXL) {  // u.k, pre-scaled by c1
+        if (tid < 128 && j0 + tid < L) va = A.uk[(size_t)bh * L + j0 + tid] * c1;
       } else if (MECH == M_T5) {
         const int idx = j0 - i0 - 127 + tid + L - 1;
         if (tid < 255 && idx >= 0 && idx < 2 * L - 1) va = p.t5_bias[(size_t)h * (2 * L - 1) + idx];
@@ -397,12 +402,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       }
       return va;
     };
-    // TXL: this thread's v.r, offset il of blocks Delta and Delta - 1, one key tile ahead
+    // TXL: this thread's v.r (pre-scaled by c1), offset il of blocks Delta and Delta - 1,
+    // one key tile ahead
     auto fetch_vr = [&](int n, float &va, float &vb) {
       if (MECH == M_TXL) {
         const int ra = 128 * (m - n) + il + p.off, rb = ra - 128;
-        va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] : 0.f;
-        vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] : 0.f;
+        va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] * c1 : 0.f;
+        vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] * c1 : 0.f;
       }
     };
     float nva = fetch_vec(0), nvrA = 0.f, nvrB = 0.f;
@@ -416,7 +422,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         nva = fetch_vec(n + 1);
         fetch_vr(n + 1, nvrA, nvrB);
       }
-      named_bar_sync(1, NSOFT);
+      // the per-tile vectors written above are read only after a later barrier of this tile
+      // (Transformer-XL: the one after the skew; the other mechanisms: this one)
+      if (MECH != M_TXL) named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       float x[NC];
       if (good) {
@@ -434,21 +442,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (MECH == M_TXL) {
         if (good) {
           const bool hasB = !(p.causal && Delta == 0);
-          txl_skew<ROT_LD, SK_ADD>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane, 1.f,
-                                   vrA, vrB, rot);
+          // relation terms in key order, already c1 (T + v.r)
+          txl_skew<ROT_LD, SK_PACKED>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane,
+                                      c1, vrA, vrB, rot);
           tc_fence_before();
           mbar_arrive(BAR(B_SFREE));
         }
         named_bar_sync(1, NSOFT);
+        // log2-domain score s c1 + (r' + u'): one f32x2 add and one f32x2 FMA per two keys
         const uint64_t c12 = f2(c1, c1);
 #pragma unroll
         for (int c4 = 0; c4 < NC / 4; ++c4) {
           const float4 rr = *reinterpret_cast<const float4 *>(rrow + cb + 4 * c4);
           const float4 uk = *reinterpret_cast<const float4 *>(tv + cb + 4 * c4);
-          x[4 * c4 + 0] = (x[4 * c4 + 0] + rr.x + uk.x) * c1;
-          x[4 * c4 + 1] = (x[4 * c4 + 1] + rr.y + uk.y) * c1;
-          x[4 * c4 + 2] = (x[4 * c4 + 2] + rr.z + uk.z) * c1;
-          x[4 * c4 + 3] = (x[4 * c4 + 3] + rr.w + uk.w) * c1;
+          f2_split(fma2(f2(x[4 * c4 + 0], x[4 * c4 + 1]), c12, add2(f2(rr.x, rr.y), f2(uk.x, uk.y))), x[4 * c4 + 0],
+                   x[4 * c4 + 1]);
+          f2_split(fma2(f2(x[4 * c4 + 2], x[4 * c4 + 3]), c12, add2(f2(rr.z, rr.w), f2(uk.z, uk.w))), x[4 * c4 + 2],
+                   x[4 * c4 + 3]);
         }
       } else if (MECH == M_T5) {
         if (good) {
@@ -542,12 +552,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int t = 0; t < NC; ++t) {
           const int j = j0 + cb + t;
           if (j >= klen || (p.causal && j > i)) x[t] = -INFINITY;
-          mt = fmaxf(mt, x[t]);
         }
-      } else {
-#pragma unroll
-        for (int t = 0; t < NC; ++t) mt = fmaxf(mt, x[t]);
       }
+#pragma unroll
+      for (int t = 0; t < NC; t += 2) mt = fmax3(mt, x[t], x[t + 1]);
       float *rd = red + TPR * 128 * (n & 1);
       rd[128 * qt + il] = mt;
       named_bar_sync(1, NSOFT);
@@ -582,10 +590,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
       }
       const float msub = (m2 == -INFINITY) ? 0.f : m2;
+      {
+        const uint64_t nm = f2(-msub, -msub);
+        uint64_t ls = f2(0.f, 0.f);
 #pragma unroll
-      for (int t = 0; t < NC; ++t) {
-        x[t] = ex2(x[t] - msub);
-        lsum += x[t];
+        for (int t = 0; t < NC; t += 2) {
+          float a, b;
+          f2_split(add2(f2(x[t], x[t + 1]), nm), a, b);
+          x[t] = ex2(a);
+          x[t + 1] = ex2(b);
+          ls = add2(ls, f2(x[t], x[t + 1]));
+        }
+        float l0, l1;
+        f2_split(ls, l0, l1);
+        lsum += l0 + l1;
       }
       if (n >= 1) good = good && warp_wait(BAR(B_PV), (n - 1) & 1, abort_flag, status);
       if constexpr (SV) {

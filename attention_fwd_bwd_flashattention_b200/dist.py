@@ -1,8 +1,16 @@
 """Process-group plumbing for running the kernels data-parallel over GPUs.
 
-One process per GPU (torchrun).  Every rank runs its own batch; the relative
-tables are shared, so their gradients are summed across ranks with one
-all-reduce (NCCL on GPUs, gloo on CPU in tests).  Timing is reduced with MAX.
+One process per GPU (torchrun).  Every (batch, head) slice of the attention is
+independent in both passes, so the work splits over ranks in two ways:
+
+  * batch: every rank runs its own batch entries; the relative tables are shared by
+    the batch, so their gradients are summed across ranks with one all-reduce per
+    table (NCCL on GPUs, gloo on CPU in tests) -- data-parallel training;
+  * heads: every rank runs a contiguous block of heads of the same batch with the
+    matching rows of the (per-head) tables; nothing is exchanged -- the split for
+    one long sequence (B = 1).
+
+Timing is reduced with MAX.
 """
 from __future__ import annotations
 
@@ -53,6 +61,36 @@ def allreduce_table_grads(drel: List[torch.Tensor]) -> None:
         return
     for g in drel:
         dist.all_reduce(g, op=dist.ReduceOp.SUM)
+
+
+def shard_range(n: int, rank: int, world: int):
+    """Contiguous block [lo, hi) of n items for `rank` (sizes differ by at most one)."""
+    base, extra = divmod(n, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def shard_inputs(inp: dict, mode: str, rank: int, world: int) -> dict:
+    """This rank's part of a workload's inputs (dict q, k, v, do [B,H,L,d] and rel, the
+    per-head tables [H,...]): batch entries (tables whole) or heads (tables' rows of
+    those heads)."""
+    if mode not in ("batch", "heads"):
+        raise ValueError(mode)
+    dim = 0 if mode == "batch" else 1
+    lo, hi = shard_range(inp["q"].shape[dim], rank, world)
+    out = {n: inp[n].narrow(dim, lo, hi - lo) for n in ("q", "k", "v", "do")}
+    out["rel"] = list(inp["rel"]) if mode == "batch" else [r.narrow(0, lo, hi - lo) for r in inp["rel"]]
+    return out
+
+
+def gather_shards(t: torch.Tensor, dim: int) -> torch.Tensor:
+    """Concatenate every rank's equally sized block of a tensor along `dim`, in rank
+    order (all-gather)."""
+    if not active():
+        return t
+    parts = [torch.empty_like(t) for _ in range(dist.get_world_size())]
+    dist.all_gather(parts, t.contiguous())
+    return torch.cat(parts, dim=dim)
 
 
 def shutdown():

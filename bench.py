@@ -357,14 +357,15 @@ class Case:
     """Device buffers of one workload: inputs drawn on the host (seeded), outputs,
     gradients and both workspaces."""
 
-    def __init__(self, wl, dev, rank, path):
+    def __init__(self, wl, dev, rank, path, inp=None):
         self.wl = wl
         self.P = params_of(wl, path)
         if wl.seqlens_k is not None:
             self.P.seqlens_k = torch.tensor(wl.seqlens_k, dtype=torch.int32, device=dev)
-        inp = make_inputs(wl, seed=rank)
-        if rank != 0:  # the relative tables are shared by all ranks (one model)
-            inp["rel"] = make_inputs(wl, seed=0)["rel"]
+        if inp is None:
+            inp = make_inputs(wl, seed=rank)
+            if rank != 0:  # the relative tables are shared by all ranks (one model)
+                inp["rel"] = make_inputs(wl, seed=0)["rel"]
         self.inp = inp
         self.q, self.k, self.v, self.do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
         self.rel = [r.to(dev) for r in inp["rel"]]
@@ -392,7 +393,7 @@ class Case:
         return {"fwd": name[bd.relpos_attn_resolved_path(self.P, 0)], "bwd": name[bd.relpos_attn_resolved_path(self.P, 1)]}
 
 
-def time_case(c, steps, warmup, flush, stream, world, on_region=None):
+def time_case(c, steps, warmup, flush, stream, reduce_grads, on_region=None):
     """W untimed steps, then `steps` steps each timed with CUDA events on the launching
     stream (fwd and bwd separately), L2 flushed before each (untimed).  The warm-up steps
     trace every kernel the library launches (bd.Trace: events around each launch) to
@@ -406,7 +407,7 @@ def time_case(c, steps, warmup, flush, stream, world, on_region=None):
         with warm_traces[w]:
             c.fwd(stream)
             c.bwd(stream)
-        if world > 1:
+        if reduce_grads:
             rdist.allreduce_table_grads(c.drel)
     torch.cuda.synchronize()
     warm = {}
@@ -427,7 +428,7 @@ def time_case(c, steps, warmup, flush, stream, world, on_region=None):
             c.fwd(stream)
             ev[s][1].record(stream)
             c.bwd(stream)
-        if world > 1:
+        if reduce_grads:
             rdist.allreduce_table_grads(c.drel)
         ev[s][2].record(stream)
     torch.cuda.synchronize()
@@ -449,7 +450,7 @@ def kernel_table(kernels, steps, step_ms):
 def side_workload(name, dev, rank, world, flush, stream, peaks, steps):
     wl = WORKLOADS[name]
     c = Case(wl, dev, rank, bd.PATH_AUTO)
-    fwd_ms, bwd_ms, warm, (dom, dom_ms) = time_case(c, steps, 3, flush, stream, world)
+    fwd_ms, bwd_ms, warm, (dom, dom_ms) = time_case(c, steps, 3, flush, stream, False)
     f_fwd, f_bwd = algo_flops(wl)
     fm, bm = median_iqr(fwd_ms)[0], median_iqr(bwd_ms)[0]
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -474,7 +475,14 @@ def run_ours(args, wl):
     dev = torch.device("cuda", local)
     path_name = "simt" if args.path == "simt" else "auto"
     path = bd.PATH_SIMT if args.path == "simt" else bd.PATH_AUTO
-    c = Case(wl, dev, rank, path)
+    # N > 1: each rank its own batch of the workload (weak scaling, table gradients
+    # all-reduced) or its block of the workload's heads (strong scaling, no collective)
+    mode = "single" if world == 1 else args.shard
+    if mode == "heads":
+        lo, hi = rdist.shard_range(wl.H, rank, world)
+        c = Case(wl.with_(H=hi - lo), dev, rank, path, inp=rdist.shard_inputs(make_inputs(wl, seed=0), "heads", rank, world))
+    else:
+        c = Case(wl, dev, rank, path)
     P = c.P
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -483,7 +491,7 @@ def run_ours(args, wl):
     base_mem = torch.cuda.memory_allocated(dev)
     clocks = ClockSampler(dev)
     clocks.start()
-    fwd_ms, bwd_ms, warm, (dom, dom_ms) = time_case(c, args.steps, args.warmup, flush, stream, world,
+    fwd_ms, bwd_ms, warm, (dom, dom_ms) = time_case(c, args.steps, args.warmup, flush, stream, mode == "batch",
                                                     on_region=clocks.mark)
     clk = clocks.stop()
     tot_ms = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
@@ -494,11 +502,14 @@ def run_ours(args, wl):
     ws_sizes = {"fwd": bd.relpos_attn_workspace_size(P, 0), "bwd": bd.relpos_attn_workspace_size(P, 1),
                 "bwd_smallest": bd.relpos_attn_workspace_size(P, 2)}
 
-    f_fwd, f_bwd = algo_flops(wl)
+    f_fwd, f_bwd = algo_flops(c.wl)  # this rank's work
     fa_f, fa_b = fa_flops(wl)
     ms_step = tot_ms / args.steps
-    value = world * (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
-    tokens = world * wl.B * wl.L / (ms_step * 1e-3)
+    # whole-job work per step: every rank's batch (weak), or the workload's heads once (strong)
+    job = (1 if mode == "heads" else world)
+    job_flops = sum(algo_flops(wl)) * job
+    value = job_flops / (ms_step * 1e-3) / 1e12
+    tokens = job * wl.B * wl.L / (ms_step * 1e-3)
     peaks, peak_src = load_peaks()
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     fwd_avg = statistics.mean(fwd_ms)
@@ -545,7 +556,7 @@ def run_ours(args, wl):
     tensor_path = pass_tc[0] and pass_tc[1]
 
     # ---- end to end through the public API: pinned host in, host out ----
-    e2e = run_e2e(args, wl, c, dev, stream, world)
+    e2e = run_e2e(args, wl, c, dev, stream, world, mode)
 
     side = []
     if not args.no_side_workloads and world == 1 and path_name == "auto":
@@ -562,18 +573,20 @@ def run_ours(args, wl):
     fl, bl = kernel_launches(wl, path_name if not tensor_path else "tc")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if mode == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "L": wl.L, "d": wl.d, "causal": wl.causal,
                    "seqlens_k": list(wl.seqlens_k) if wl.seqlens_k is not None else None, "mem_len": wl.mem_len,
                    "kernel_path": c.paths(),
                    "l2": "flushed before every timed step (256 MB write, untimed)",
-                   "parallelism": f"dp{world} (weak; table grads all-reduced)" if world > 1 else "single GPU"},
+                   "parallelism": {"single": "single GPU", "batch": f"dp{world} (weak; table grads all-reduced)",
+                                   "heads": f"heads split over {world} GPUs (strong; no collective)"}[mode]},
         "tokens_per_s": tokens,
         "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
         "fwd_tflops": f_fwd / (fwd_avg * 1e-3) / 1e12, "bwd_tflops": f_bwd / (bwd_avg * 1e-3) / 1e12,
-        "fa_convention_tflops": world * (fa_f + fa_b) / (ms_step * 1e-3) / 1e12,
-        "frac_of_dense_bf16_datasheet": value / world / 2250.0,
+        "fa_convention_tflops": job * (fa_f + fa_b) / (ms_step * 1e-3) / 1e12,
+        "frac_of_dense_bf16_datasheet": value / world / 2250.0,  # per GPU
         "frac_of_measured_bf16": value / world / burst,
         "peak_mem_bytes": int(step_mem),
         "peak_mem_smallest_workspace_bytes": int(step_mem - ws_sizes["bwd"] + ws_sizes["bwd_smallest"]),
@@ -599,7 +612,7 @@ def run_ours(args, wl):
     return 0
 
 
-def run_e2e(args, wl, c, dev, stream, world):
+def run_e2e(args, wl, c, dev, stream, world, mode="single"):
     """Same metric through the public entry points, with every step's inputs copied
     from pinned host memory and its results (O, LSE, dQ, dK, dV, drel) copied back.  Steps are
     pipelined over two buffer sets: step k's host-to-device copies (one stream) and
@@ -649,7 +662,7 @@ def run_e2e(args, wl, c, dev, stream, world):
             bd.relpos_attn_fwd(P, B["q"], B["k"], B["v"], B["rel"], B["o"], B["lse"], ws_f, stream=stream)
             bd.relpos_attn_bwd(P, B["q"], B["k"], B["v"], B["rel"], B["o"], B["lse"], B["do"], B["dq"], B["dk"], B["dv"],
                                B["drel"], ws_b, stream=stream)
-            if world > 1:
+            if mode == "batch":
                 rdist.allreduce_table_grads(B["drel"])
             ev_done[i].record(stream)
         with torch.cuda.stream(s_out):
@@ -669,8 +682,8 @@ def run_e2e(args, wl, c, dev, stream, world):
     e1.record(s_out)
     torch.cuda.synchronize()
     ms = rdist.max_over_ranks(e0.elapsed_time(e1)) / args.steps
-    f_fwd, f_bwd = algo_flops(wl)
-    return {"value": world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+    job_flops = sum(algo_flops(wl)) * (1 if mode == "heads" else world)
+    return {"value": job_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "pipeline": "two buffer sets; host-to-device, kernels and device-to-host on three streams"}
 
@@ -685,6 +698,8 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "simt"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side-workloads", action="store_true", help="time only the main workload")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="N > 1: each rank its own batch (weak scaling) or a block of the heads (strong scaling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     wl = WORKLOADS[args.workload]

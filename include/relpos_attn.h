@@ -254,6 +254,10 @@ RELPOS_API int relpos_trace_end(void);
 /* Static, NUL-terminated description of a status code. */
 RELPOS_API const char *relpos_strerror(int status);
 
+/* The cudaError_t value behind the last RELPOS_ERR_LAUNCH that a call made from this
+ * host thread returned (0 if none has): a diagnostic for callers. */
+RELPOS_API int relpos_last_cuda_error(void);
+
 /* ABI version: major * 10000 + minor * 100 + patch. */
 RELPOS_API int relpos_attn_version(void);
 
