@@ -6,6 +6,7 @@ compiled library is missing this module raises; there is no other code path.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -168,6 +169,14 @@ def _ptr_array(ts: Sequence[Optional[torch.Tensor]]):
     return arr
 
 
+def _on_device_of(t):
+    """The library launches on the calling thread's current CUDA device: make the
+    tensor's device current for the call (as torch's own ops do)."""
+    if isinstance(t, torch.Tensor) and t.is_cuda:
+        return torch.cuda.device(t.device)
+    return contextlib.nullcontext()
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -202,8 +211,9 @@ def tc_available(params: Params, pass_: int = 0) -> bool:
 def relpos_attn_fwd(params: Params, q, k, v, rel, o, lse, workspace, dev_status=None, stream=None) -> None:
     cp = params.c()
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = load().relpos_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o), _ptr(lse),
-                                _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    with _on_device_of(q):
+        rc = load().relpos_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o), _ptr(lse),
+                                    _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
     if rc != 0:
         raise RelposError(rc, "relpos_attn_fwd")
 
@@ -212,8 +222,9 @@ def relpos_attn_fwd_noalloc(params: Params, q, k, v, rel, o, lse, dev_status=Non
     """Forward pass that allocates nothing: its scratch is the library's built-in
     device array (see relpos_attn_fwd_noalloc in include/relpos_attn.h)."""
     cp = params.c()
-    rc = load().relpos_attn_fwd_noalloc(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o),
-                                        _ptr(lse), _ptr(dev_status), _stream(stream))
+    with _on_device_of(q):
+        rc = load().relpos_attn_fwd_noalloc(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o),
+                                            _ptr(lse), _ptr(dev_status), _stream(stream))
     if rc != 0:
         raise RelposError(rc, "relpos_attn_fwd_noalloc")
 
@@ -264,9 +275,10 @@ def relpos_attn_bwd(params: Params, q, k, v, rel, o, lse, dout, dq, dk, dv, drel
                     stream=None) -> None:
     cp = params.c()
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = load().relpos_attn_bwd(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o), _ptr(lse),
-                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr_array(drel), _ptr(workspace), ws_bytes,
-                                _ptr(dev_status), _stream(stream))
+    with _on_device_of(q):
+        rc = load().relpos_attn_bwd(ctypes.byref(cp), _ptr(q), _ptr(k), _ptr(v), _ptr_array(rel), _ptr(o), _ptr(lse),
+                                    _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr_array(drel), _ptr(workspace), ws_bytes,
+                                    _ptr(dev_status), _stream(stream))
     if rc != 0:
         raise RelposError(rc, "relpos_attn_bwd")
 

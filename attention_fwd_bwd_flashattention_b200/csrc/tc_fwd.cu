@@ -60,9 +60,11 @@ constexpr int OFF_BAR = OFF_RED + 2 * TPR * 128 * 4;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 
+// B_K0 / B_K1: K (and the Transformer-XL relation block) of the even / odd key tiles;
+// B_V0 / B_V1: V of the even / odd key tiles (loaded on their own schedule)
 enum {
-  B_Q = 0, B_KV0 = 1, B_KV1 = 2, B_SFULL = 3, B_SFREE = 4, B_PFULL = 5, B_PV = 6, B_PLOAD = 7, B_PFULLPRO = 8,
-  B_PFREEPRO = 9, B_RLOAD = 10, B_RFREE = 11, B_GFULL = 12, B_DRAIN = 13, NBARS = 14
+  B_Q = 0, B_K0 = 1, B_K1 = 2, B_SFULL = 3, B_SFREE = 4, B_PFULL = 5, B_PV = 6, B_PLOAD = 7, B_PFULLPRO = 8,
+  B_PFREEPRO = 9, B_RLOAD = 10, B_RFREE = 11, B_GFULL = 12, B_DRAIN = 13, B_V0 = 14, B_V1 = 15, NBARS = 16
 };
 
 constexpr uint32_t TM_S = 0, TM_REL = 128, TM_O = 384, TM_COLS = 512;
@@ -169,8 +171,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 
   if (tid == 0) {
     mbar_init(BAR(B_Q), 1);
-    mbar_init(BAR(B_KV0), 1);
-    mbar_init(BAR(B_KV1), 1);
+    mbar_init(BAR(B_K0), 1);
+    mbar_init(BAR(B_K1), 1);
+    mbar_init(BAR(B_V0), 1);
+    mbar_init(BAR(B_V1), 1);
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_SFREE), NSOFT);
     mbar_init(BAR(B_PFULL), NSOFT);
@@ -205,8 +209,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       const uint32_t idPV = idesc_bf16(128, 64, true);
       const uint32_t idW = idesc_bf16(128, 256, false);
       // TMA loads issued but not yet waited for, drained before exit on abort
-      uint32_t pend_bar[8];
-      uint32_t pend_par[8];
+      uint32_t pend_bar[10];
+      uint32_t pend_par[10];
       int npend = 0;
       auto expect = [&](int bi, uint32_t par, uint32_t bytes) {
         mbar_expect_tx(BAR(bi), bytes);
@@ -256,15 +260,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       auto needs_new_block = [&](int n) {  // TXL: block (m - n - 1), unless it is entirely masked
         return !(p.causal && m - n - 1 < 0);
       };
-      auto issue_kv = [&](int n) {
+      // K(n) and the relation block tile n adds (TXL) go into stage n & 1 as soon as S(n - 2),
+      // their previous reader, is complete; V(n) goes into stage n & 1 once PV(n - 2) is: the
+      // loads of a key tile are issued about one tile ahead of their first use
+      auto issue_k = [&](int n) {
         const int st = n & 1;
-        uint32_t bytes = 32768;
+        uint32_t bytes = 16384;
         if (MECH == M_TXL && needs_new_block(n)) bytes += 16384;
-        expect(B_KV0 + st, (uint32_t)((n >> 1) & 1), bytes);
-        tma_load_3d(sbase + OFF_K + 16384 * st, &A.mk, BAR(B_KV0 + st), 0, n * BN, bh);
-        tma_load_3d(sbase + OFF_V + 16384 * st, &A.mv, BAR(B_KV0 + st), 0, n * BN, bh);
+        expect(B_K0 + st, (uint32_t)((n >> 1) & 1), bytes);
+        tma_load_3d(sbase + OFF_K + 16384 * st, &A.mk, BAR(B_K0 + st), 0, n * BN, bh);
         if (MECH == M_TXL && needs_new_block(n))
-          tma_load_3d(sbase + OFF_R + 16384 * st, &A.mt0, BAR(B_KV0 + st), 0, 128 * (m - n - 1) + p.off, h);
+          tma_load_3d(sbase + OFF_R + 16384 * st, &A.mt0, BAR(B_K0 + st), 0, 128 * (m - n - 1) + p.off, h);
+      };
+      auto issue_v = [&](int n) {
+        const int st = n & 1;
+        expect(B_V0 + st, (uint32_t)((n >> 1) & 1), 16384);
+        tma_load_3d(sbase + OFF_V + 16384 * st, &A.mv, BAR(B_V0 + st), 0, n * BN, bh);
       };
       auto issue_pv = [&](int n) {  // O (+)= P(n) V(n)
         const int ps = n & 1;
@@ -288,14 +299,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         umma_commit(BAR(B_PV));
       };
       if (ok) {
-        issue_kv(0);
-        if (nTiles > 1) issue_kv(1);
+        issue_k(0);
+        issue_v(0);
+        if (nTiles > 1) {
+          issue_k(1);
+          issue_v(1);
+        }
       }
       if (SV && ok) ok = wait_load(B_PLOAD, 1);  // aV staged before the first PV
       for (int n = 0; ok && n < nTiles; ++n) {
         const int st = n & 1;
         const int Delta = m - n;
-        if (!wait_load(B_KV0 + st, (n >> 1) & 1)) break;
+        if (!wait_load(B_K0 + st, (n >> 1) & 1)) break;
         if (n == 0) {
           if (MECH != M_SHAW && !wait_load(B_Q, 0)) break;
           if (MECH == M_TXL && !wait_load(B_PLOAD, 0)) break;
@@ -319,6 +334,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           umma_k64(tbase + TM_REL, sbase + OFF_Q, sbase + OFF_R, idW, false);
         }
         umma_commit(BAR(B_SFULL));
+        // K(n + 1) into the stage of tile n - 1: the rows released S(n - 1) (B_SFREE), so
+        // S(n - 1) and every MMA committed with it (and DeBERTa's p2c product of tile n - 1,
+        // which the rows read before that release) are complete
+        if (n >= 1 && n + 1 < nTiles) issue_k(n + 1);
         if (band) {
           if (!wait_bar(B_RFREE, band_cnt & 1)) break;
           tc_fence_after();
@@ -330,17 +349,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           umma_commit(BAR(B_GFULL));
           ++band_cnt;
         }
+        // V(n) into the stage of tile n - 2 once PV(n - 2) is complete (committed one tile ago)
+        if (n >= 2) {
+          if (!wait_bar(B_PV, (n - 2) & 1)) break;
+          issue_v(n);
+        }
         if (n >= 1) {
           if (!wait_bar(B_PFULL, (n - 1) & 1)) break;
+          if (!wait_load(B_V0 + ((n - 1) & 1), ((n - 1) >> 1) & 1)) break;
           tc_fence_after();
           issue_pv(n - 1);
-          if (n + 1 < nTiles) {  // refill the stage tile n-1 used
-            if (!wait_bar(B_PV, (n - 1) & 1)) break;
-            issue_kv(n + 1);
-          }
         }
       }
-      if (ok && !*abort_flag && wait_bar(B_PFULL, (nTiles - 1) & 1)) {
+      if (ok && !*abort_flag && wait_bar(B_PFULL, (nTiles - 1) & 1) &&
+          wait_load(B_V0 + ((nTiles - 1) & 1), ((nTiles - 1) >> 1) & 1)) {
         tc_fence_after();
         issue_pv(nTiles - 1);
       }
