@@ -6,6 +6,8 @@
 
 #include <vector>
 
+#include <cuda.h>
+
 #include "relpos_attn.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -293,6 +295,34 @@ static int rel_count(const Prm &p) {
   return p.mech == rp::M_TXL ? 3 : ((p.mech == rp::M_DEB || p.shaw_v) ? 2 : 1);
 }
 
+// The calling thread's CUDA context.  The runtime binds the current device's primary
+// context lazily, on the first runtime call that needs it, but the tensor-map encoder (a
+// driver call, made before any launch) needs a current context already: in a host thread
+// that has made no CUDA call yet it would fail.  When no context is current, make the
+// current device's primary context current (cudaSetDevice on the device cudaGetDevice
+// reports: what the runtime's lazy binding would do); a current context is left alone.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+static int ensure_context() {
+  static CtxGetCurrentFn fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return (CtxGetCurrentFn) nullptr;
+    }
+    return (CtxGetCurrentFn)f;
+  }();
+  CUcontext ctx = nullptr;
+  if (fn && fn(&ctx) == CUDA_SUCCESS && ctx) return RELPOS_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return RELPOS_ERR_CUDA;
+  }
+  return RELPOS_OK;
+}
+
 // CUDA error behind this thread's last RELPOS_ERR_LAUNCH (relpos_last_cuda_error)
 static thread_local int t_last_cuda = 0;
 
@@ -367,6 +397,7 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   }
   const Layout l = layout_of(p, 0, tc);
   if (l.total > 0 && (!workspace || workspace_bytes < l.total || ((uintptr_t)workspace & 255))) return RELPOS_ERR_WORKSPACE;
+  if ((e = ensure_context())) return e;  // argument errors are all found above
   bind_workspace(p, l, workspace);
   cudaStream_t st = (cudaStream_t)stream;
   p.q = q;
@@ -435,6 +466,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
       return RELPOS_ERR_INVALID_ARG;
     if (p.mech == rp::M_DEB && !aligned16(rel[1])) return RELPOS_ERR_INVALID_ARG;
   }
+  if ((e = ensure_context())) return e;  // argument errors are all found above
   const size_t rb = (size_t)p.esize * rp::HD;
   char *wb = (char *)workspace;
   if (p.mem_len > 0) {  // placeholder rows 0 .. M - 1: zero q, O and dO, LSE = +inf, so P = 0 and dS = 0 there

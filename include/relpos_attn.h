@@ -55,8 +55,10 @@
  *     to 0 and reads it back after synchronising).  NULL disables it.
  *   - stream: a cudaStream_t (NULL = the legacy default stream).  All work is
  *     enqueued on it asynchronously, on the calling thread's current CUDA device,
- *     which must be the device that holds the pointers and the stream (a host
- *     thread that has not made any device current should call cudaSetDevice first).
+ *     which must be the device that holds the pointers and the stream.  A host
+ *     thread with no current CUDA context gets the current device's primary context
+ *     made current (as the runtime's first call there would do); a current context is
+ *     left as it is.
  *
  * Errors: every call returns RELPOS_OK (0) or a negative RELPOS_ERR_* code.  The entry
  * points clear the calling thread's CUDA "last error" before they enqueue anything, so
