@@ -1,6 +1,8 @@
 // CUDA-core (fp32 FFMA) kernels for relative-position attention, forward and
-// backward, all four mechanisms.  This is the float32 path of the library and
-// the reference-grade GPU path every other kernel is compared with.
+// backward, all four mechanisms.  This is the float32 path of the library (and the
+// bfloat16 path of the cases the tensor-core kernels do not take).  Like every other
+// kernel of the library it is checked against the fp64 CPU oracle, element by element
+// on the same inputs; no kernel serves as another's reference.
 //
 // The structure is the method's, at 64 x 64 tiles:
 //  * offset-aware tiling: a query tile x key tile pair touches the offset window
