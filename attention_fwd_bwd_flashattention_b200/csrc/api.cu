@@ -145,7 +145,6 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
-  if (p.shaw_v && pass == 1) return false;  // the backward of Shaw's value-side term runs on the CUDA-core kernels
   if (pass == 1)
     return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p)) ||
            (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p)) || (p.mech == rp::M_DEB && rp::tc_bwd_deb_supported(p));
@@ -156,7 +155,7 @@ static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
 struct Layout {
   size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot, part_val;
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
-  size_t part_kv, part_dg, part_uv, qa;  // tensor-core backward partials / products
+  size_t part_kv, part_dg, part_uv, qa, da;  // tensor-core backward partials / products
   size_t qkr, kqr, dM, dN, dqc, dkc, dpart;  // DeBERTa tensor-core backward
   size_t pdtiles;                            // Transformer-XL tensor-core backward: stored P / dS tiles (0: none)
   size_t mq, mo, mlse, mdo, mdq;             // Transformer-XL memory: query-side tensors padded to M + L rows
@@ -207,6 +206,10 @@ static Layout layout_of(const Prm &p, int pass, bool tc, bool lean = false) {
     l.dvec = take(sizeof(float) * BH * p.L);
     l.qa = take(sizeof(float) * rp::tc_bwd_shaw_qa_floats(p));
     l.part_row = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nrows * rp::HD);
+    if (p.shaw_v) {  // value side: dO . aV by row and the daV partials
+      l.da = take(sizeof(float) * rp::tc_bwd_shaw_qa_floats(p));
+      l.part_val = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nrows * rp::HD);
+    }
   } else if (pass == 1 && tc) {  // tensor-core backward (Transformer-XL)
     size_t kvf = 0;
     const size_t dgf = rp::tc_bwd_part_floats(p, kvf);
@@ -278,6 +281,7 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.part_dg = (float *)(b + l.part_dg);
   w.part_uv = (float *)(b + l.part_uv);
   w.qa = (float *)(b + l.qa);
+  w.da = (float *)(b + l.da);
   w.qkr = (float *)(b + l.qkr);
   w.kqr = (float *)(b + l.kqr);
   w.dqc = (float *)(b + l.dqc);

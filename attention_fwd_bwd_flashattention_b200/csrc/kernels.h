@@ -26,6 +26,7 @@ struct TcWork {
   float *part_kv, *part_dg;      // backward partials (Transformer-XL)
   float *part_uv;                // [H][ceil(rows / 32)][64] dv partials per 32-offset tile
   float *qa;                     // Shaw backward: [B,H,L][132] per-row products q_i . a_rho
+  float *da;                     // Shaw value side: [B,H,L][132] per-row products dO_i . aV_rho
   void *pdtiles;                 // Transformer-XL backward: the query-tile kernel's P / dS tiles (or null)
   // DeBERTa backward: relation products QKr, KQr and dS K, dS^T Q (fp32), the
   // offset-ordered dS copies M, N (bf16, [B,H,L][2k]) and the table-gradient partials

@@ -21,6 +21,14 @@
 //                     end) and applied to a_0 / a_2c at the end.  The CTA writes its
 //                     partial of da (offset-sharded gradient, technique (3)); a fixed-
 //                     order reduction over query tiles finishes da.
+//
+// Shaw's value-side table aV (O_i += sum_j P_ij aV_rho, the VAL variants): dP_ij gains
+// DA[i][rho] = dO_i . aV_rho (a second per-row product table, gathered like QA but
+// read from L2: band tiles by offset, other tiles one end value per row), so both
+// kernels form dS = P (dP + DA - D); the query-tile kernel also writes P in offset order
+// (Pe, into the E tile once E's MMAs are done) on band tiles and accumulates
+// GV += Pe^T dO in TMEM, the clipped pairs' probability mass per row going to the end
+// rows aV_0 / aV_2c: one daV partial per query tile, reduced in a fixed order.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -41,7 +49,9 @@ struct ShawArgs {
   CUtensorMap mq, mk, mv, mdo, ma, mqa;
   Prm p;            // nT counts 128-row tiles
   const float *qa;  // [B,H,L][132]
+  const float *da;  // value side: [B,H,L][132] per-row products dO_i . aV_rho
   float *part;      // [B,H,nT][rows][64] da partial per query tile
+  float *part_v;    // value side: [B,H,nT][rows][64] daV partial per query tile
 };
 
 __device__ __forceinline__ bool band_tile(int c, int m, int n) {
@@ -50,17 +60,20 @@ __device__ __forceinline__ bool band_tile(int c, int m, int n) {
 }
 
 // ---------------------------------------------------------------------------
-// QA[b,h,i][rho] = q_i . a_rho: one CTA per 32 query rows of one (b,h); lanes take
-// consecutive rho (coalesced row stores), warps take rows.
+// QA[b,h,i][rho] = q_i . a_rho (and, for the value side, DA[b,h,i][rho] = dO_i . aV_rho):
+// X[b,h,i][rho] = x_i . T_rho for rows x [B,H,L,64] and a table T [H,rows,64].  One CTA
+// per 32 rows of one (b,h); lanes take consecutive rho (coalesced row stores), warps
+// take rows.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) shaw_qa_kernel(Prm p, float *qa) {
+__global__ void __launch_bounds__(256) shaw_qa_kernel(Prm p, const __nv_bfloat16 *xrows, const __nv_bfloat16 *table,
+                                                      float *qa) {
   __shared__ float As[QA_LD][65];
   __shared__ float Qs[32][65];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int tiles = (p.L + 31) / 32;
   const int bh = (int)blockIdx.x / tiles, i0 = ((int)blockIdx.x % tiles) * 32, h = bh % p.H;
-  const __nv_bfloat16 *a = (const __nv_bfloat16 *)p.rel0 + (size_t)h * p.nrows * HD;
-  const __nv_bfloat16 *q = (const __nv_bfloat16 *)p.q + ((size_t)bh * p.L) * HD;
+  const __nv_bfloat16 *a = table + (size_t)h * p.nrows * HD;
+  const __nv_bfloat16 *q = xrows + ((size_t)bh * p.L) * HD;
   for (int x = tid; x < QA_LD * HD; x += 256) {
     const int r = x / HD, d = x % HD;
     As[r][d] = r < p.nrows ? __bfloat162float(a[(size_t)r * HD + d]) : 0.f;
@@ -101,6 +114,14 @@ enum { B_KV = 0, B_ST0, B_ST1, B_QA, B_SDP, B_SDPCONS, B_PDS, B_PDSFREE, B_DRAIN
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320;
 }  // namespace kvs
 
+// dS = P (dP + DA - D) for four keys (value side: DA the dO . aV terms), nDv = (-D, -D)
+__device__ __forceinline__ void ds_pairs_da(const float (&pr)[4], const uint32_t *dp, const float *da, uint64_t nDv,
+                                            float (&dd)[4]) {
+  f2_split(mul2(f2(pr[0], pr[1]), add2(add2(f2(u2f(dp[0]), u2f(dp[1])), f2(da[0], da[1])), nDv)), dd[0], dd[1]);
+  f2_split(mul2(f2(pr[2], pr[3]), add2(add2(f2(u2f(dp[2]), u2f(dp[3])), f2(da[2], da[3])), nDv)), dd[2], dd[3]);
+}
+
+template <bool VAL>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __grid_constant__ ShawArgs A) {
   using namespace kvs;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -227,21 +248,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
     bool good = true;
     int qa_cnt = 0;
     // per-tile row terms staged through smem one tile ahead (one element per thread):
-    // [lse2 of the rows | D of the rows | QA of the clipped end row the tile sees]
+    // [lse2 of the rows | D of the rows | QA of the clipped end row the tile sees
+    //  | value side: DA of that end row]
+    constexpr int NV = VAL ? 512 : 384;
     auto fetch1 = [&](int t) {
       const int m = mStart + t, r = tid & 127, w = tid >> 7, i = m * 128 + r;
       if (i >= L) return w == 0 ? INFINITY : 0.f;
       if (w == 0) return lse2_of(p, bh, i);
       if (w == 1) return p.Dvec[(size_t)bh * L + i];
-      return A.qa[((size_t)bh * L + i) * QA_LD + (m > n ? 0 : 2 * cl)];
+      return (w == 2 ? A.qa : A.da)[((size_t)bh * L + i) * QA_LD + (m > n ? 0 : 2 * cl)];
     };
-    if (tid < 384) vec[tid] = fetch1(0);
+    if (tid < NV) vec[tid] = fetch1(0);
     for (int t = 0; t < iters; ++t) {
       const int m = mStart + t, i = m * 128 + il;
-      const float *tv = vec + 384 * (t & 1);
-      const float nv = (tid < 384 && t + 1 < iters) ? fetch1(t + 1) : 0.f;
+      const float *tv = vec + NV * (t & 1);
+      const float nv = (tid < NV && t + 1 < iters) ? fetch1(t + 1) : 0.f;
       named_bar_sync(1, NSOFT);
       const bool band = band_tile(cl, m, n);
+      // value side: row i of DA (dO_i . aV_rho), gathered by offset on band tiles; other tiles
+      // take the row's end value
+      const float *darow = (VAL && band && i < L) ? A.da + ((size_t)bh * L + i) * QA_LD + cl : nullptr;
       good = good && warp_wait(BAR(B_SDP), t & 1, abort_flag, status);
       if (band) {
         good = good && warp_wait(BAR(B_QA), qa_cnt & 1, abort_flag, status);
@@ -278,7 +304,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
               }
 #pragma unroll
               for (int e = 0; e < 4; ++e) pr[e] = ex2(y[e]);
-              ds_pairs(pr, rp + 4 * c4, nDv, dd);
+              if constexpr (VAL) {
+                float da4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) da4[e] = darow ? __ldg(darow + iclamp(d0 + x0 + e, -cl, cl)) : tv[384 + il];
+                ds_pairs_da(pr, rp + 4 * c4, da4, nDv, dd);
+              } else {
+                ds_pairs(pr, rp + 4 * c4, nDv, dd);
+              }
               pk[x0 / 2] = pack_bf16x2(pr[0], pr[1]);
               pk[x0 / 2 + 1] = pack_bf16x2(pr[2], pr[3]);
               dk[x0 / 2] = pack_bf16x2(dd[0], dd[1]);
@@ -310,7 +343,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_kv_kernel(const __gri
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
       }
-      if (tid < 384) vec[384 * ((t + 1) & 1) + tid] = nv;  // tile t - 1's terms were read before this tile's first barrier
+      if (tid < NV) vec[NV * ((t + 1) & 1) + tid] = nv;  // tile t - 1's terms were read before this tile's first barrier
     }
     // ---- epilogue: lanes are keys; this thread takes 16 of the 64 columns ----
     good = good && warp_wait(BAR(B_PDSFREE), (iters - 1) & 1, abort_flag, status);
@@ -360,8 +393,9 @@ constexpr int OFF_ROT = OFF_E + 32768;   // the CTA's QA rows, 128 x 132 fp32
 constexpr int OFF_VEC = OFF_ROT + 128 * QA_LD * 4;  // clipped-sum exchange [2][4][128]
 constexpr int OFF_BAR = OFF_VEC + 4096;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
-enum { B_QD = 0, B_ST0, B_ST1, B_SDP, B_SDPCONS, B_PDS, B_EFREE, B_DSFREE, B_DRAIN, NB };
-constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_DS = 320, T_G = 384;
+// B_PEFULL / B_PEFREE (value side): Pe written into the E tile / GV MMAs done with it
+enum { B_QD = 0, B_ST0, B_ST1, B_SDP, B_SDPCONS, B_PDS, B_EFREE, B_DSFREE, B_DRAIN, B_PEFULL, B_PEFREE, NB };
+constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_DS = 320, T_G = 384, T_GV = 448;
 }  // namespace qs
 
 // dS of this thread's NC keys into the offset-order tile E (row il): column
@@ -392,6 +426,7 @@ __device__ __forceinline__ void store_Es(uint8_t *E, int il, uint32_t C0, const 
   }
 }
 
+template <bool VAL>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid_constant__ ShawArgs A) {
   using namespace qs;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -411,6 +446,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
     }
     float *part = A.part + ((size_t)bh * p.nT + m) * (size_t)p.nrows * HD;
     for (int x = tid; x < p.nrows * HD; x += NTHREADS) part[x] = 0.f;
+    if (VAL) {
+      float *pv = A.part_v + ((size_t)bh * p.nT + m) * (size_t)p.nrows * HD;
+      for (int x = tid; x < p.nrows * HD; x += NTHREADS) pv[x] = 0.f;
+    }
     return;
   }
   const uint32_t sbase = smem_u32(smem), bar0 = sbase + OFF_BAR;
@@ -423,7 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
   const float c1 = p.scale * LOG2E;
 
   if (tid == 0) {
-    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), (k == B_SDPCONS || k == B_PDS) ? NSOFT : 1);
+    for (int k = 0; k < NB; ++k) mbar_init(BAR(k), (k == B_SDPCONS || k == B_PDS || k == B_PEFULL) ? NSOFT : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -483,7 +522,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
         }
         if (!ctl.wait(BAR(B_PDS), n & 1)) break;
         tc_fence_after();
-        if (band_tile(cl, m, n)) {  // dQ += E a, G += E^T Q (E in smem)
+        const bool bt = band_tile(cl, m, n);
+        if (bt) {  // dQ += E a, G += E^T Q (E in smem)
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             umma_bf16(tbase + T_DQ, sdesc_sw128(sbase + OFF_E + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
@@ -492,14 +532,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
                       sdesc_sw128(sbase + OFF_Q + 2048 * k, 16, 1024), idG, (nband > 0 || k > 0) ? 1u : 0u);
           }
           umma_commit(BAR(B_EFREE));
-          ++nband;
         }
         // dQ += dS K_n (dS from TMEM)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           umma_bf16_ts(tbase + T_DQ, tbase + T_DS + 8 * k, sdesc_sw128(sbase + OFF_K + 16384 * st + 2048 * k, 16, 1024), idDQ,
-                       (n > 0 || k > 0 || band_tile(cl, m, n)) ? 1u : 0u);
+                       (n > 0 || k > 0 || bt) ? 1u : 0u);
         umma_commit(BAR(B_DSFREE));
+        if (VAL && bt) {  // GV += Pe^T dO, Pe written by the rows into the E tile once E's MMAs were done
+          if (!ctl.wait(BAR(B_PEFULL), nband & 1)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            umma_bf16(tbase + T_GV, sdesc_sw128(sbase + OFF_E + 2048 * k, 16384, 1024),
+                      sdesc_sw128(sbase + OFF_DO + 2048 * k, 16, 1024), idG, (nband > 0 || k > 0) ? 1u : 0u);
+          umma_commit(BAR(B_PEFREE));
+        }
+        if (bt) ++nband;
         if (n + 2 < nTiles) {  // K_n, V_n free once dS K_n is done
           if (!ctl.wait(BAR(B_DSFREE), n & 1)) break;
           issue_stage(n + 2);
@@ -518,13 +567,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
     const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
     bool good = warp_wait(BAR(B_QD), 0, abort_flag, status);
     float rsL = 0.f, rsR = 0.f;  // dS of clipped pairs, left (rho = 0) / right (rho = 2c)
+    float psL = 0.f, psR = 0.f;  // value side: P of the clipped pairs, left / right
+    // value side: row i of DA (dO_i . aV_rho), its end values and a pointer to the rest
+    const float *darow = (VAL && i < L) ? A.da + ((size_t)bh * L + i) * QA_LD + cl : nullptr;
+    const float daL = darow ? darow[-cl] : 0.f, daR = darow ? darow[cl] : 0.f;
     int nband = 0;
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * 128;
       const bool band = band_tile(cl, m, n);
+      const int d0 = j0 + cb - i;  // offset j - i of this thread's first key
+      // clipped pairs: keys with j - i <= -c (left) or >= c (right); unclipped ones go to E
+      const int eLo = max(0, 1 - cl - d0), eHi = min(NC - 1, cl - 1 - d0);  // unclipped: eLo..eHi
+      const float dend = m > n ? daL : daR;  // value side: dO_i . aV of the row's clipped end
+      uint32_t ppk[VAL ? NC / 2 : 1];  // value side, band tiles: P of the unclipped pairs (Pe), bf16 pairs
       good = good && warp_wait(BAR(B_SDP), n & 1, abort_flag, status);
       const bool need_mask = (p.causal && n == m) || (j0 + 128 > klen);
-      const int d0 = j0 + cb - i;  // offset j - i of this thread's first key
       float x[NC];
       if (good) {
         tc_fence_after();
@@ -553,7 +610,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
               }
 #pragma unroll
               for (int e = 0; e < 4; ++e) pr[e] = ex2(y[e]);
-              ds_pairs(pr, rp + 4 * c4, nDv, dd);
+              if constexpr (VAL) {
+                // dO_i . aV of the four keys: band tiles gather row i of DA by offset (L1 / L2)
+                float da4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  da4[e] = (decltype(banded)::value && darow) ? __ldg(darow + iclamp(d0 + x0 + e, -cl, cl)) : dend;
+                ds_pairs_da(pr, rp + 4 * c4, da4, nDv, dd);
+                float pe[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int ee = x0 + e;
+                  if (ee < eLo) psL += pr[e];
+                  else if (ee > eHi) psR += pr[e];
+                  pe[e] = (ee >= eLo && ee <= eHi) ? pr[e] : 0.f;
+                }
+                if constexpr (decltype(banded)::value) {
+                  ppk[x0 / 2] = pack_bf16x2(pe[0], pe[1]);
+                  ppk[x0 / 2 + 1] = pack_bf16x2(pe[2], pe[3]);
+                }
+              } else {
+                ds_pairs(pr, rp + 4 * c4, nDv, dd);
+              }
 #pragma unroll
               for (int e = 0; e < 4; ++e) x[x0 + e] = dd[e];
             }
@@ -570,8 +648,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < NC; ++e) x[e] = 0.f;
       }
-      // clipped pairs: keys with j - i <= -c (left) or >= c (right); unclipped ones go to E
-      const int eLo = max(0, 1 - cl - d0), eHi = min(NC - 1, cl - 1 - d0);  // unclipped: eLo..eHi
 #pragma unroll
       for (int e = 0; e < NC; ++e) {
         if (e < eLo) rsL += x[e];
@@ -585,7 +661,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
         if (n >= 1 && !warp_wait(BAR(B_DSFREE), (n - 1) & 1, abort_flag, status)) good = false;
         if (good) tmem_st16(tl + T_DS + 16 * qt, pk);
         if (good && band) {
-          if (nband >= 1 && !warp_wait(BAR(B_EFREE), (nband - 1) & 1, abort_flag, status)) good = false;
+          // the E tile's last reader of the previous band tile: its E MMAs (value side: its GV MMAs)
+          if (nband >= 1 && !warp_wait(BAR(VAL ? B_PEFREE : B_EFREE), (nband - 1) & 1, abort_flag, status)) good = false;
 #pragma unroll
           for (int k = 0; k < NC / 2; ++k) {
             const float v0 = (2 * k >= eLo && 2 * k <= eHi) ? x[2 * k] : 0.f;
@@ -594,11 +671,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
           }
           if (good) store_Es(smem + OFF_E, il, (uint32_t)(d0 + cl) & 127u, pk);
         }
-        if (band) ++nband;
         tmem_wait_st();
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_PDS));
+        if constexpr (VAL) {
+          if (band) {  // Pe into the E tile once this tile's E MMAs are done
+            if (!warp_wait(BAR(B_EFREE), nband & 1, abort_flag, status)) good = false;
+            if (good) {
+              store_Es(smem + OFF_E, il, (uint32_t)(d0 + cl) & 127u, ppk);
+              fence_async_smem();
+              tc_fence_before();
+              mbar_arrive(BAR(B_PEFULL));
+            }
+          }
+        }
+        if (band) ++nband;
       }
     }
     // ---- epilogue ----
@@ -609,6 +697,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
     const float sL = ((vec[il] + vec[128 + il]) + vec[256 + il]) + vec[384 + il];
     const float sR = ((vec[512 + il] + vec[640 + il]) + vec[768 + il]) + vec[896 + il];
     good = good && warp_wait(BAR(B_DSFREE), (nTiles - 1) & 1, abort_flag, status);  // every MMA done
+    if (VAL && nband > 0) good = good && warp_wait(BAR(B_PEFREE), (nband - 1) & 1, abort_flag, status);  // and GV's
     const __nv_bfloat16 *a = (const __nv_bfloat16 *)p.rel0 + (size_t)h * p.nrows * HD;
     if (good) {
       tc_fence_after();
@@ -642,6 +731,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
 #pragma unroll
         for (int e = 0; e < 16; ++e) part[(size_t)rho * HD + 16 * qt + e] = (nband > 0) ? p.scale * u2f(gr[e]) : 0.f;
       }
+      if (VAL) {  // daV partial: rows 1..2c-1 from GV (TMEM lane = rho)
+        float *pv = A.part_v + ((size_t)bh * p.nT + m) * (size_t)p.nrows * HD;
+        tmem_ld16(tl + T_GV + 16 * qt, gr);
+        tmem_wait_ld();
+        if (rho >= 1 && rho <= 2 * cl - 1) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pv[(size_t)rho * HD + 16 * qt + e] = (nband > 0) ? u2f(gr[e]) : 0.f;
+        }
+      }
     }
     named_bar_sync(1, NSOFT);
     vec[il] = sL;  // row sums for the end rows of da (one copy per row)
@@ -655,6 +753,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
       float *part = A.part + ((size_t)bh * p.nT + m) * (size_t)p.nrows * HD;
       part[(size_t)(side ? 2 * cl : 0) * HD + d] = p.scale * acc;
     }
+    if (VAL) {  // daV[0][d] = sum_i psL_i dO_i[d], daV[2c][d] = sum_i psR_i dO_i[d] (row sums in a fixed order)
+      named_bar_sync(1, NSOFT);
+      vec[qt * 128 + il] = psL;
+      vec[512 + qt * 128 + il] = psR;
+      named_bar_sync(1, NSOFT);
+      const float pL = ((vec[il] + vec[128 + il]) + vec[256 + il]) + vec[384 + il];
+      const float pR = ((vec[512 + il] + vec[640 + il]) + vec[768 + il]) + vec[896 + il];
+      named_bar_sync(1, NSOFT);
+      vec[il] = pL;
+      vec[128 + il] = pR;
+      named_bar_sync(1, NSOFT);
+      if (tid < 2 * HD) {
+        const int d = tid & (HD - 1), side = tid >> 6;
+        const __nv_bfloat16 *gp = (const __nv_bfloat16 *)p.dout + ((size_t)bh * L + i0) * HD + d;
+        float acc = 0.f;
+        for (int rr = 0; rr < 128 && i0 + rr < L; ++rr) acc = fmaf(vec[128 * side + rr], __bfloat162float(gp[(size_t)rr * HD]), acc);
+        float *pv = A.part_v + ((size_t)bh * p.nT + m) * (size_t)p.nrows * HD;
+        pv[(size_t)(side ? 2 * cl : 0) * HD + d] = acc;
+      }
+    }
     tc_fence_before();
   }
   __syncthreads();
@@ -664,8 +782,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_shaw_q_kernel(const __grid
   }
 }
 
-// da = sum over batches and query tiles of the partials, in a fixed order
-__global__ void reduce_shaw_kernel(Prm p, const float *part) {
+// da (daV) = sum over batches and query tiles of the partials, in a fixed order
+__global__ void reduce_shaw_kernel(Prm p, const float *part, float *out) {
   const size_t per = (size_t)p.nrows * HD;
   const size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (x >= (size_t)p.H * per) return;
@@ -674,7 +792,7 @@ __global__ void reduce_shaw_kernel(Prm p, const float *part) {
   float acc = 0.f;
   for (int b = 0; b < p.B; ++b)
     for (int t = 0; t < p.nT; ++t) acc += part[(((size_t)b * p.H + h) * p.nT + t) * per + re];
-  p.drel0[x] = acc;
+  out[x] = acc;
 }
 
 }  // namespace tcs
@@ -687,14 +805,34 @@ bool tc_bwd_shaw_supported(const Prm &p) { return p.clip >= 1 && p.clip <= 64; }
 
 size_t tc_bwd_shaw_qa_floats(const Prm &p) { return (size_t)p.B * p.H * p.L * tcs::QA_LD; }
 
+template <bool VAL>
+static cudaError_t run_shaw_bwd(const tcs::ShawArgs &a, cudaStream_t st) {
+  using namespace tcs;
+  cudaError_t e;
+  auto kkv = tc_bwd_shaw_kv_kernel<VAL>;
+  auto kq = tc_bwd_shaw_q_kernel<VAL>;
+  if ((e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, qs::SMEM)) != cudaSuccess) return e;
+  const unsigned tiles = (unsigned)(a.p.nT * a.p.B * a.p.H);
+  RP_TRACED("tc_bwd_shaw_kv_kernel", st, kkv<<<tiles, NTHREADS, kvs::SMEM, st>>>(a));
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  RP_TRACED("tc_bwd_shaw_q_kernel", st, kq<<<tiles, NTHREADS, qs::SMEM, st>>>(a));
+  return cudaGetLastError();
+}
+
 cudaError_t tc_bwd_shaw(const Prm &p0, const TcWork &w, cudaStream_t st) {
   using namespace tcs;
+  typedef __nv_bfloat16 bf;
   ShawArgs a;
   memset(&a, 0, sizeof(a));
   a.p = p0;
   a.p.nT = (p0.L + 127) / 128;
   a.qa = w.qa;
   a.part = p0.part_row;
+  if (p0.shaw_v) {
+    a.da = w.da;
+    a.part_v = p0.part_val;
+  }
   const uint64_t BH = (uint64_t)p0.B * p0.H;
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
         tc_make_map(&a.mv, p0.v, p0.L, BH, 128) && tc_make_map(&a.mdo, p0.dout, p0.L, BH, 128) &&
@@ -703,20 +841,23 @@ cudaError_t tc_bwd_shaw(const Prm &p0, const TcWork &w, cudaStream_t st) {
     return cudaErrorInvalidValue;
   cudaError_t e;
   const unsigned qa_blocks = (unsigned)(BH * ((p0.L + 31) / 32));
-  RP_TRACED("shaw_qa_kernel", st, shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, w.qa));
+  RP_TRACED("shaw_qa_kernel", st, shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, (const bf *)p0.q, (const bf *)p0.rel0, w.qa));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(tc_bwd_shaw_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(tc_bwd_shaw_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qs::SMEM)) != cudaSuccess)
-    return e;
-  const unsigned tiles = (unsigned)(a.p.nT * BH);
-  RP_TRACED("tc_bwd_shaw_kv_kernel", st, tc_bwd_shaw_kv_kernel<<<tiles, NTHREADS, kvs::SMEM, st>>>(a));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  RP_TRACED("tc_bwd_shaw_q_kernel", st, tc_bwd_shaw_q_kernel<<<tiles, NTHREADS, qs::SMEM, st>>>(a));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (p0.shaw_v) {  // DA = dO aV^T by row, for the value side
+    RP_TRACED("shaw_qa_kernel", st,
+              shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, (const bf *)p0.dout, (const bf *)p0.rel1, w.da));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = p0.shaw_v ? run_shaw_bwd<true>(a, st) : run_shaw_bwd<false>(a, st)) != cudaSuccess) return e;
   const size_t n = (size_t)p0.H * p0.nrows * HD;
-  RP_TRACED("reduce_shaw_kernel", st, reduce_shaw_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.p, a.part));
-  return cudaGetLastError();
+  RP_TRACED("reduce_shaw_kernel", st, reduce_shaw_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.p, a.part, p0.drel0));
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (p0.shaw_v) {
+    RP_TRACED("reduce_shaw_kernel", st,
+              reduce_shaw_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(a.p, a.part_v, p0.drel1));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace rp

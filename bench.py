@@ -90,15 +90,15 @@ def kernel_launches(wl, path):
     """Kernels this library launches per forward and per backward call (the dispatch of csrc/api.cu)."""
     t5 = 1 if wl.mech in (T5, ALIBI) else 0  # per-call per-offset bias preparation
     tc = path != "simt" and wl.dtype == torch.bfloat16
-    tc_bwd = tc and not wl.shaw_value  # the value side's backward runs on CUDA cores
+    tc_bwd = tc and not (wl.mech == SHAW and wl.shaw_clip > 64)  # wider Shaw clips: CUDA-core backward
     if tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
         fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
     else:
         fwd = 1 + t5
     if tc_bwd and wl.mech == TXL:  # D, relation prep, key-tile, query-tile, diagonal, dr and u/v reductions
         bwd = 7
-    elif tc_bwd and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction
-        bwd = 5
+    elif tc_bwd and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction; the value
+        bwd = 7 if wl.shaw_value else 5  # side adds the dO.aV products and the daV reduction
     elif tc_bwd and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
         bwd = 5
     elif tc_bwd and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction

@@ -133,8 +133,7 @@ typedef struct relpos_params {
    * with rel[1] = aV [H, 2c + 1, d] (params' dtype) and drel[1] = daV (float32).
    * The paper's Hugging Face page names Shaw among the mechanisms the method covers
    * (Community comment); the value side is the second table of Shaw's own paper.
-   * The forward runs on the tensor-core kernels for bf16 and c <= 64, the backward on
-   * the CUDA-core kernels (RELPOS_PATH_TC is rejected for it). */
+   * Both passes run on the tensor-core kernels for bf16 and c <= 64. */
   int32_t shaw_value;
   /* Transformer-XL only, causal only (0 = none): length M of the cached memory of the
    * previous segment.  The L queries (q, o, lse, dq, dO: [B, H, L, d]) sit at positions

@@ -228,13 +228,14 @@ def test_resolved_paths(lib):
     # DeBERTa: spans that are multiples of 32 up to 256 take the tensor-core backward
     for span, want_b in ((256, TC), (32, TC), (96, TC), (24, SIMT), (288, SIMT)):
         assert bd.relpos_attn_resolved_path(bd.Params(mech=bd.DEBERTA, B=1, H=2, L=300, deberta_span=span), 1) == want_b, span
-    # Shaw's value-side term: tensor-core forward for c <= 64, CUDA-core backward
+    # Shaw's value-side term: tensor cores in both passes for c <= 64
     Pv = bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True)
-    assert (bd.relpos_attn_resolved_path(Pv, 0), bd.relpos_attn_resolved_path(Pv, 1)) == (TC, SIMT)
+    assert (bd.relpos_attn_resolved_path(Pv, 0), bd.relpos_attn_resolved_path(Pv, 1)) == (TC, TC)
     Pv65 = bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, shaw_clip=65)
     assert (bd.relpos_attn_resolved_path(Pv65, 0), bd.relpos_attn_resolved_path(Pv65, 1)) == (SIMT, SIMT)
     with pytest.raises(bd.RelposError):
-        bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, kernel_path=bd.PATH_TC), 1)
+        bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, shaw_clip=65,
+                                               kernel_path=bd.PATH_TC), 1)
     wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == SIMT
     assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC
