@@ -61,38 +61,66 @@ __device__ __forceinline__ bool band_tile(int c, int m, int n) {
 
 // ---------------------------------------------------------------------------
 // QA[b,h,i][rho] = q_i . a_rho (and, for the value side, DA[b,h,i][rho] = dO_i . aV_rho):
-// X[b,h,i][rho] = x_i . T_rho for rows x [B,H,L,64] and a table T [H,rows,64].  One CTA
-// per 32 rows of one (b,h); lanes take consecutive rho (coalesced row stores), warps
-// take rows.
+// X[b,h,i][rho] = x_i . T_rho for rows x [B,H,L,64] and a table T [H,rows,64], rho < 132
+// (rows past the table give 0).  One CTA per 64 rows of one (b,h), both operands staged
+// transposed (d-major) in smem; each thread accumulates a 4-row x 8-column register
+// tile of rho < 128 (one f32 FMA per product, fixed order over d) and one of the 256
+// products of rho = 128..131.
 // ---------------------------------------------------------------------------
+constexpr int QA_ROWS = 64;
+constexpr int QA_XS = QA_ROWS + 4;  // padded smem row of x^T (floats)
+constexpr int QA_TS = QA_LD + 4;    // padded smem row of T^T (floats)
+constexpr int QA_SMEM = (HD * QA_XS + HD * QA_TS) * 4;
 __global__ void __launch_bounds__(256) shaw_qa_kernel(Prm p, const __nv_bfloat16 *xrows, const __nv_bfloat16 *table,
                                                       float *qa) {
-  __shared__ float As[QA_LD][65];
-  __shared__ float Qs[32][65];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int tiles = (p.L + 31) / 32;
-  const int bh = (int)blockIdx.x / tiles, i0 = ((int)blockIdx.x % tiles) * 32, h = bh % p.H;
+  extern __shared__ __align__(16) float qsm[];
+  float *Xs = qsm;               // [64 d][QA_XS]: x^T
+  float *Ts = qsm + HD * QA_XS;  // [64 d][QA_TS]: T^T
+  const int tid = threadIdx.x;
+  const int tiles = (p.L + QA_ROWS - 1) / QA_ROWS;
+  const int bh = (int)blockIdx.x / tiles, i0 = ((int)blockIdx.x % tiles) * QA_ROWS, h = bh % p.H;
   const __nv_bfloat16 *a = table + (size_t)h * p.nrows * HD;
   const __nv_bfloat16 *q = xrows + ((size_t)bh * p.L) * HD;
   for (int x = tid; x < QA_LD * HD; x += 256) {
     const int r = x / HD, d = x % HD;
-    As[r][d] = r < p.nrows ? __bfloat162float(a[(size_t)r * HD + d]) : 0.f;
+    Ts[d * QA_TS + r] = r < p.nrows ? __bfloat162float(a[(size_t)r * HD + d]) : 0.f;
   }
-  for (int x = tid; x < 32 * HD; x += 256) {
+  for (int x = tid; x < QA_ROWS * HD; x += 256) {
     const int r = x / HD, d = x % HD;
-    Qs[r][d] = (i0 + r < p.L) ? __bfloat162float(q[(size_t)(i0 + r) * HD + d]) : 0.f;
+    Xs[d * QA_XS + r] = (i0 + r < p.L) ? __bfloat162float(q[(size_t)(i0 + r) * HD + d]) : 0.f;
   }
   __syncthreads();
-  for (int r = w; r < 32; r += 8) {
-    if (i0 + r >= p.L) break;
-    float *out = qa + ((size_t)bh * p.L + i0 + r) * QA_LD;
-    for (int rho = lane; rho < QA_LD; rho += 32) {
-      float acc = 0.f;
-#pragma unroll 16
-      for (int d = 0; d < HD; ++d) acc = fmaf(Qs[r][d], As[rho][d], acc);
-      out[rho] = acc;
+  const int r4 = tid >> 4, c8 = tid & 15;  // rows 4 r4 .. +3, columns 8 c8 .. +7
+  float acc[4][8];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+  const int tr = tid >> 2, tc = 128 + (tid & 3);  // the tail product of this thread
+  float tail = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < HD; ++d) {
+    const float4 xv = *reinterpret_cast<const float4 *>(Xs + d * QA_XS + 4 * r4);
+    const float4 t0 = *reinterpret_cast<const float4 *>(Ts + d * QA_TS + 8 * c8);
+    const float4 t1 = *reinterpret_cast<const float4 *>(Ts + d * QA_TS + 8 * c8 + 4);
+    const float xr[4] = {xv.x, xv.y, xv.z, xv.w};
+    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(xr[r], tv[c], acc[r][c]);
+    tail = fmaf(Xs[d * QA_XS + tr], Ts[d * QA_TS + tc], tail);
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + 4 * r4 + r;
+    if (i < p.L) {
+      float *out = qa + ((size_t)bh * p.L + i) * QA_LD + 8 * c8;
+      *reinterpret_cast<float4 *>(out) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+      *reinterpret_cast<float4 *>(out + 4) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
     }
   }
+  if (i0 + tr < p.L) qa[((size_t)bh * p.L + i0 + tr) * QA_LD + tc] = tail;
 }
 
 // log2-domain scores of four keys, y = (s + R) c1 - lse2, with the relation terms R
@@ -840,12 +868,15 @@ cudaError_t tc_bwd_shaw(const Prm &p0, const TcWork &w, cudaStream_t st) {
         tc_make_map_f32_rows(&a.mqa, w.qa, QA_LD, p0.L, BH, 128)))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  const unsigned qa_blocks = (unsigned)(BH * ((p0.L + 31) / 32));
-  RP_TRACED("shaw_qa_kernel", st, shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, (const bf *)p0.q, (const bf *)p0.rel0, w.qa));
+  const unsigned qa_blocks = (unsigned)(BH * ((p0.L + QA_ROWS - 1) / QA_ROWS));
+  if ((e = cudaFuncSetAttribute(shaw_qa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QA_SMEM)) != cudaSuccess)
+    return e;
+  RP_TRACED("shaw_qa_kernel", st,
+            shaw_qa_kernel<<<qa_blocks, 256, QA_SMEM, st>>>(a.p, (const bf *)p0.q, (const bf *)p0.rel0, w.qa));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (p0.shaw_v) {  // DA = dO aV^T by row, for the value side
     RP_TRACED("shaw_qa_kernel", st,
-              shaw_qa_kernel<<<qa_blocks, 256, 0, st>>>(a.p, (const bf *)p0.dout, (const bf *)p0.rel1, w.da));
+              shaw_qa_kernel<<<qa_blocks, 256, QA_SMEM, st>>>(a.p, (const bf *)p0.dout, (const bf *)p0.rel1, w.da));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = p0.shaw_v ? run_shaw_bwd<true>(a, st) : run_shaw_bwd<false>(a, st)) != cudaSuccess) return e;

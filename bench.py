@@ -357,7 +357,7 @@ class Case:
     """Device buffers of one workload: inputs drawn on the host (seeded), outputs,
     gradients and both workspaces."""
 
-    def __init__(self, wl, dev, rank, path, inp=None):
+    def __init__(self, wl, dev, rank, path, inp=None, bwd_pass=1):
         self.wl = wl
         self.P = params_of(wl, path)
         if wl.seqlens_k is not None:
@@ -370,7 +370,7 @@ class Case:
         self.q, self.k, self.v, self.do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
         self.rel = [r.to(dev) for r in inp["rel"]]
         self.ws_f = bd.workspace(self.P, 0, dev)
-        self.ws_b = bd.workspace(self.P, 1, dev)
+        self.ws_b = bd.workspace(self.P, bwd_pass, dev)  # 2: the smallest backward workspace
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty(self.q.shape[:3], dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
@@ -469,6 +469,24 @@ def side_workload(name, dev, rank, world, flush, stream, peaks, steps):
     return out
 
 
+def lean_backward(wl, dev, flush, stream, peaks, steps):
+    """The same step with the smallest backward workspace (relpos_attn_workspace_size pass
+    2): no stored P / dS tiles, memory O(L); timed like the main step."""
+    c = Case(wl, dev, 0, bd.PATH_AUTO, bwd_pass=2)
+    fwd_ms, bwd_ms, warm, _ = time_case(c, steps, 3, flush, stream, False)
+    f_fwd, f_bwd = algo_flops(wl)
+    fm, bm = median_iqr(fwd_ms)[0], median_iqr(bwd_ms)[0]
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    out = {"workspace": "smallest (pass 2)", "steps": steps, "fwd_ms_median": fm, "bwd_ms_median": bm,
+           "fwd_bwd_tflops": (f_fwd + f_bwd) / ((fm + bm) * 1e-3) / 1e12,
+           "frac_of_measured_bf16_burst": (f_fwd + f_bwd) / ((fm + bm) * 1e-3) / 1e12 / burst,
+           "bwd_tflops": f_bwd / (bm * 1e-3) / 1e12, "peak_mem_bytes": int(c.step_bytes()),
+           "kernels_warmup": kernel_table(warm, 2, fm + bm)}
+    del c
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, wl):
     rank, world, local = rdist.init_from_env(backend="nccl")
     torch.cuda.set_device(local)
@@ -558,6 +576,10 @@ def run_ours(args, wl):
     # ---- end to end through the public API: pinned host in, host out ----
     e2e = run_e2e(args, wl, c, dev, stream, world, mode)
 
+    lean = None
+    if (world == 1 and path_name == "auto" and not args.no_side_workloads
+            and bd.relpos_attn_workspace_size(P, 2) < bd.relpos_attn_workspace_size(P, 1)):
+        lean = lean_backward(wl, dev, flush, stream, peaks, min(args.steps, 50))
     side = []
     if not args.no_side_workloads and world == 1 and path_name == "auto":
         for name in SIDE_WORKLOADS:
@@ -605,6 +627,7 @@ def run_ours(args, wl):
         "gpu_launches_expected": (fl + bl) * args.steps,
         "clocks": clk,
         "workloads": side,
+        "smallest_workspace": lean,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
