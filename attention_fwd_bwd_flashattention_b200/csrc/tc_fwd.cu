@@ -449,13 +449,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (MECH != M_TXL) named_bar_sync(1, NSOFT);
       good = good && warp_wait(BAR(B_SFULL), n & 1, abort_flag, status);
       float x[NC];
+      uint32_t rs[32];  // S row segment; its registers are valid only after tcgen05.wait::ld
       if (good) {
         tc_fence_after();
-        uint32_t r[32];
-        tmem_ld32(tl + TM_S + cb, r);
-        tmem_wait_ld();
+        tmem_ld32(tl + TM_S + cb, rs);
+        // Transformer-XL: the relation block's load (in the skew below) is issued before this
+        // one is waited for, so that the two TMEM latencies overlap
+        if (MECH != M_TXL) {
+          tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < NC; ++t) x[t] = u2f(r[t]);
+          for (int t = 0; t < NC; ++t) x[t] = u2f(rs[t]);
+        }
       } else {
 #pragma unroll
         for (int t = 0; t < NC; ++t) x[t] = 0.f;
@@ -464,9 +468,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (MECH == M_TXL) {
         if (good) {
           const bool hasB = !(p.causal && Delta == 0);
-          // relation terms in key order, already c1 (T + v.r)
+          // relation terms in key order, already c1 (T + v.r); its tcgen05.wait::ld also
+          // completes the S load above
           txl_skew<ROT_LD, SK_PACKED>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane,
                                       c1, vrA, vrB, rot);
+          tmem_wait_ld();  // when the skew had no load to wait for (no block Delta - 1 for this warp)
+#pragma unroll
+          for (int t = 0; t < NC; ++t) x[t] = u2f(rs[t]);
           tc_fence_before();
           mbar_arrive(BAR(B_SFREE));
         }
