@@ -772,10 +772,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       float x[NC];
       if (good) {
         tc_fence_after();
-        // S is loaded first: the skew's tcgen05.wait::ld completes it too, so the two TMEM
-        // latencies overlap (its registers are read only after a wait)
-        uint32_t r[32];
-        tmem_ld32(tl + T_S + cb, r);
         if (hasA) {
           txl_skew<ROT_LD>(tl, T_REL + 128 * (D & 1), T_REL + 128 * ((D - 1) & 1), hasB, g, qt, lane, c1, tu[128 + il],
                            tu[256 + il], rot);
@@ -783,6 +779,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
 #pragma unroll
           for (int c = 0; c < NC; ++c) rrow[(il - cb - c) & 127] = 0.f;
         }
+        uint32_t r[32];
+        tmem_ld32(tl + T_S + cb, r);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < NC; ++e) x[e] = u2f(r[e]);

@@ -38,7 +38,7 @@ namespace tcbias {
 using namespace tc;
 using namespace tcb;
 
-constexpr int MAX_BAND = 8;                      // band tiles per query tile (T5), else CUDA-core path
+constexpr int MAX_BAND = 64;                     // band tiles per query tile (T5), else CUDA-core path
 constexpr int GMAX = 128 * (MAX_BAND - 1) + 256;  // per-offset sums of the band tiles of one query tile
 
 struct BiasArgs {

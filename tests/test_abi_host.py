@@ -236,7 +236,10 @@ def test_resolved_paths(lib):
     with pytest.raises(bd.RelposError):
         bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, shaw_clip=65,
                                                kernel_path=bd.PATH_TC), 1)
+    # T5: the band of tiles with more than one bias value, up to 64 tiles, on the tensor cores
     wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
-    assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == SIMT
+    assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == TC
     assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC
+    wider = dict(mech=bd.T5, B=1, H=2, t5_max_distance=20000)
+    assert bd.relpos_attn_resolved_path(bd.Params(L=32768, **wider), 1) == SIMT
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, t5_bidirectional=False, **wide), 1) == TC  # one side flat

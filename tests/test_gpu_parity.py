@@ -220,6 +220,11 @@ def test_parity_bias_family_tensor_core_backward(causal):
         assert bd.relpos_attn_resolved_path(P, 1) == bd.PATH_TC, (nb, md, bidir)
         inp = make_inputs(wl, nb)
         compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+    # a band of distinct-bias tiles far wider than eight (max_distance 3000: about 47 tiles)
+    wl = Workload("t5_wide", T5, torch.bfloat16, causal, 1, 2, 3500, t5_num_buckets=32, t5_max_distance=3000)
+    assert bd.relpos_attn_resolved_path(params_of(wl, bd.PATH_AUTO), 1) == bd.PATH_TC
+    inp = make_inputs(wl, 11)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
     wl = Workload("alibi_x", ALIBI, torch.bfloat16, causal, 2, 4, 1100)
     inp = make_inputs(wl, 3)
     inp["rel"] = [torch.tensor([1e-4, 0.02, 1.0, 8.0])]
