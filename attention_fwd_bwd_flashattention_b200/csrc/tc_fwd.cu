@@ -64,8 +64,12 @@ constexpr int SMEM_BYTES = SMEM_USED + 1024;
 // B_V0 / B_V1: V of the even / odd key tiles (loaded on their own schedule)
 enum {
   B_Q = 0, B_K0 = 1, B_K1 = 2, B_SFULL = 3, B_SFREE = 4, B_PFULL = 5, B_PV = 6, B_PLOAD = 7, B_PFULLPRO = 8,
-  B_PFREEPRO = 9, B_RLOAD = 10, B_RFREE = 11, B_GFULL = 12, B_DRAIN = 13, B_V0 = 14, B_V1 = 15, NBARS = 16
+  B_PFREEPRO = 9, B_RLOAD = 10, B_RFREE = 11, B_GFULL = 12, B_DRAIN = 13, B_V0 = 14, B_V1 = 15, B_RLOAD2 = 16,
+  NBARS = 17
 };
+// DeBERTa: P (bf16 pairs) in TMEM columns [448, 512) as the PV MMA's A operand, so that the
+// P smem tile holds the p2c table window while OFF_R holds the c2p one (B_RLOAD / B_RLOAD2)
+constexpr uint32_t TM_PD = 448;
 
 constexpr uint32_t TM_S = 0, TM_REL = 128, TM_O = 384, TM_COLS = 512;
 constexpr uint32_t TM_P = 128;  // Shaw with the value table: P (bf16 pairs, 64 columns) as the PV MMA's A operand
@@ -140,6 +144,8 @@ __device__ __forceinline__ bool shaw_band(int clip, int m, int n) {
 template <int MECH, bool VAL = false>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ FwdArgs A) {
   constexpr bool SV = MECH == M_SHAW && VAL;
+  constexpr bool PTM = SV || MECH == M_DEB;  // P in TMEM (the PV MMA's A operand)
+  constexpr uint32_t TMP = MECH == M_DEB ? TM_PD : TM_P;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
@@ -183,6 +189,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     mbar_init(BAR(B_PFULLPRO), 1);
     mbar_init(BAR(B_PFREEPRO), NSOFT);
     mbar_init(BAR(B_RLOAD), 1);
+    mbar_init(BAR(B_RLOAD2), 1);
     mbar_init(BAR(B_RFREE), NSOFT);
     mbar_init(BAR(B_GFULL), 1);
     mbar_init(BAR(B_DRAIN), 1);
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 
       expect(B_Q, 0, 16384);
       tma_load_3d(sbase + OFF_Q, &A.mq, BAR(B_Q), 0, i0, bh);
-      int rl_phase = 0, band_cnt = 0;
+      int band_cnt = 0;
       bool ok = true;
       if (MECH == M_SHAW) {
         expect(B_PLOAD, 0, (uint32_t)A.shaw_n * 128u);
@@ -257,6 +264,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         expect(B_PLOAD, 0, 16384);
         tma_load_3d(sbase + OFF_P, &A.mt0, BAR(B_PLOAD), 0, 128 * m + p.off, h);
       }
+      // DeBERTa band tile: some offsets of tile (m, n) are inside the span
+      auto deb_band = [&](int n) {
+        const int D = m - n;
+        return 128 * (D < 0 ? -D : D) - 127 < p.span;
+      };
+      // both table windows of band tile n (c2p: Kr rows into OFF_R; p2c: Qr rows into the P
+      // smem tile, free because P lives in TMEM), phase = the band tile's index & 1
+      auto issue_win = [&](int n) {
+        const int D = m - n;
+        const uint32_t ph = (uint32_t)(band_cnt & 1);
+        expect(B_RLOAD, ph, 32768);
+        tma_load_3d(sbase + OFF_R, &A.mt0, BAR(B_RLOAD), 0, p.span + 128 * D - 127, h);
+        expect(B_RLOAD2, ph, 32768);
+        tma_load_3d(sbase + OFF_P, &A.mt1, BAR(B_RLOAD2), 0, p.span - 128 * D - 127, h);
+      };
       auto needs_new_block = [&](int n) {  // TXL: block (m - n - 1), unless it is entirely masked
         return !(p.causal && m - n - 1 < 0);
       };
@@ -279,12 +301,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       };
       auto issue_pv = [&](int n) {  // O (+)= P(n) V(n)
         const int ps = n & 1;
-        if constexpr (SV) {  // P from TMEM; on band tiles also O += Pe aV (Pe in the P smem tile)
+        if constexpr (PTM) {  // P from TMEM; Shaw's value side on band tiles also O += Pe aV (Pe in the P smem tile)
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            umma_bf16_ts(tbase + TM_O, tbase + TM_P + 8 * k, sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024),
+            umma_bf16_ts(tbase + TM_O, tbase + TMP + 8 * k, sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024),
                          idPV, (n > 0 || k > 0) ? 1u : 0u);
-          if (shaw_band(p.clip, m, n)) {
+          if (SV && shaw_band(p.clip, m, n)) {
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
@@ -307,6 +329,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
       }
       if (SV && ok) ok = wait_load(B_PLOAD, 1);  // aV staged before the first PV
+      if (MECH == M_DEB && ok && deb_band(0)) issue_win(0);
       for (int n = 0; ok && n < nTiles; ++n) {
         const int st = n & 1;
         const int Delta = m - n;
@@ -325,12 +348,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           if (needs_new_block(n))
             umma_k64(tbase + TM_REL + 128 * ((Delta - 1) & 1), sbase + OFF_R + 16384 * st, sbase + OFF_Q, idS, false);
         }
-        const bool band = (MECH == M_DEB) && (128 * (Delta < 0 ? -Delta : Delta) - 127 < p.span);
-        if (band) {
-          expect(B_RLOAD, (uint32_t)rl_phase, 32768);
-          tma_load_3d(sbase + OFF_R, &A.mt0, BAR(B_RLOAD), 0, p.span + 128 * Delta - 127, h);
-          if (!wait_load(B_RLOAD, rl_phase)) break;
-          rl_phase ^= 1;
+        const bool band = (MECH == M_DEB) && deb_band(n);
+        if (band) {  // c2p window, prefetched (issue_win)
+          if (!wait_load(B_RLOAD, (uint32_t)(band_cnt & 1))) break;
           umma_k64(tbase + TM_REL, sbase + OFF_Q, sbase + OFF_R, idW, false);
         }
         umma_commit(BAR(B_SFULL));
@@ -338,16 +358,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         // S(n - 1) and every MMA committed with it (and DeBERTa's p2c product of tile n - 1,
         // which the rows read before that release) are complete
         if (n >= 1 && n + 1 < nTiles) issue_k(n + 1);
-        if (band) {
+        if (band) {  // p2c once the rows have read c2p; its window was prefetched with c2p's
           if (!wait_bar(B_RFREE, band_cnt & 1)) break;
+          if (!wait_load(B_RLOAD2, (uint32_t)(band_cnt & 1))) break;
           tc_fence_after();
-          expect(B_RLOAD, (uint32_t)rl_phase, 32768);
-          tma_load_3d(sbase + OFF_R, &A.mt1, BAR(B_RLOAD), 0, p.span - 128 * Delta - 127, h);
-          if (!wait_load(B_RLOAD, rl_phase)) break;
-          rl_phase ^= 1;
-          umma_k64(tbase + TM_REL, sbase + OFF_K + 16384 * st, sbase + OFF_R, idW, false);
+          umma_k64(tbase + TM_REL, sbase + OFF_K + 16384 * st, sbase + OFF_P, idW, false);
           umma_commit(BAR(B_GFULL));
           ++band_cnt;
+        }
+        // the next band tile's two table windows, as soon as this tile's relation MMAs (the
+        // windows' last readers, committed to B_GFULL) are done
+        if (MECH == M_DEB && n + 1 < nTiles && deb_band(n + 1)) {
+          if (band && !wait_bar(B_GFULL, (band_cnt - 1) & 1)) break;
+          issue_win(n + 1);
         }
         // V(n) into the stage of tile n - 2 once PV(n - 2) is complete (committed one tile ago)
         if (n >= 2) {
@@ -663,6 +686,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           tc_fence_before();
           mbar_arrive(BAR(B_PFULL));
         }
+      } else if (MECH == M_DEB && good) {  // P (bf16 pairs) into TMEM for the PV MMA
+        uint32_t pk[NC / 2];
+#pragma unroll
+        for (int k = 0; k < NC / 2; ++k) pk[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
+        tmem_st16(tl + TM_PD + 16 * qt, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFULL));
       } else if (good) {
         // P quarter-row -> smem sub-tile qt / 2, K-major 128B swizzle: chunk c of row r at chunk c ^ (r & 7)
 #pragma unroll
