@@ -8,12 +8,12 @@
 //              They read S = Q K^T and the relation products from TMEM, add the
 //              relative term gathered by offset, run the online softmax (row max
 //              exchanged through smem; lazy rescale of O only when the running max
-//              grows by more than 2^8), and write P (bf16) into shared memory in the
-//              128-byte-swizzled layout the tensor core reads.
+//              grows by more than 2^8), and write P (bf16 pairs) into TMEM, where the
+//              PV MMA reads it as its A operand.
 //   warp 16    lane 0 issues every TMA load (Q, K, V, relation-table windows,
-//              2-stage K/V ring) and every tcgen05.mma, and signals through
-//              mbarriers and tcgen05.commit.
-// TMEM (512 columns): S [0,128), relation products [128,384), O [384,448).
+//              2-stage K and V rings on separate barriers) and every tcgen05.mma, and
+//              signals through mbarriers and tcgen05.commit.
+// TMEM (512 columns): S [0,128), relation products [128,384), O [384,448), P [448,512).
 //
 // Relation stage per mechanism ("Fast and Exact Relative-Position Attention via
 // Structure-Aware Kernels", Abstract, techniques (1) and (2)):
@@ -67,12 +67,13 @@ enum {
   B_PFREEPRO = 9, B_RLOAD = 10, B_RFREE = 11, B_GFULL = 12, B_DRAIN = 13, B_V0 = 14, B_V1 = 15, B_RLOAD2 = 16,
   NBARS = 17
 };
-// DeBERTa: P (bf16 pairs) in TMEM columns [448, 512) as the PV MMA's A operand, so that the
-// P smem tile holds the p2c table window while OFF_R holds the c2p one (B_RLOAD / B_RLOAD2)
+// P (bf16 pairs) lives in TMEM columns [448, 512) as the PV MMA's A operand (no P smem
+// traffic).  The P smem tile then holds: DeBERTa's p2c table window (OFF_R holds the c2p
+// one; B_RLOAD / B_RLOAD2), Shaw's value side's offset-ordered P (Pe), Transformer-XL's
+// first relation block.
 constexpr uint32_t TM_PD = 448;
 
 constexpr uint32_t TM_S = 0, TM_REL = 128, TM_O = 384, TM_COLS = 512;
-constexpr uint32_t TM_P = 128;  // Shaw with the value table: P (bf16 pairs, 64 columns) as the PV MMA's A operand
 
 struct FwdArgs {
   CUtensorMap mq, mk, mv, mt0, mt1;
@@ -144,8 +145,7 @@ __device__ __forceinline__ bool shaw_band(int clip, int m, int n) {
 template <int MECH, bool VAL = false>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ FwdArgs A) {
   constexpr bool SV = MECH == M_SHAW && VAL;
-  constexpr bool PTM = SV || MECH == M_DEB;  // P in TMEM (the PV MMA's A operand)
-  constexpr uint32_t TMP = MECH == M_DEB ? TM_PD : TM_P;
+  constexpr uint32_t TMP = TM_PD;  // P in TMEM (the PV MMA's A operand)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
@@ -301,22 +301,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       };
       auto issue_pv = [&](int n) {  // O (+)= P(n) V(n)
         const int ps = n & 1;
-        if constexpr (PTM) {  // P from TMEM; Shaw's value side on band tiles also O += Pe aV (Pe in the P smem tile)
+        // P from TMEM; Shaw's value side on band tiles also O += Pe aV (Pe in the P smem tile)
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_bf16_ts(tbase + TM_O, tbase + TMP + 8 * k, sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024),
-                         idPV, (n > 0 || k > 0) ? 1u : 0u);
-          if (SV && shaw_band(p.clip, m, n)) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
-                        sdesc_sw128(sbase + OFF_R + 2048 * k, 16, 1024), idPV, 1u);
-          }
-        } else {
+        for (int k = 0; k < 8; ++k)
+          umma_bf16_ts(tbase + TM_O, tbase + TMP + 8 * k, sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024),
+                       idPV, (n > 0 || k > 0) ? 1u : 0u);
+        if (SV && shaw_band(p.clip, m, n)) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             umma_bf16(tbase + TM_O, sdesc_sw128(sbase + OFF_P + 16384 * (k >> 2) + 32 * (k & 3), 16, 1024),
-                      sdesc_sw128(sbase + OFF_V + 16384 * ps + 2048 * k, 16, 1024), idPV, (n > 0 || k > 0) ? 1u : 0u);
+                      sdesc_sw128(sbase + OFF_R + 2048 * k, 16, 1024), idPV, 1u);
         }
         umma_commit(BAR(B_PV));
       };
@@ -671,7 +665,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           uint32_t pk[NC / 2];
 #pragma unroll
           for (int k = 0; k < NC / 2; ++k) pk[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
-          tmem_st16(tl + TM_P + 16 * qt, pk);
+          tmem_st16(tl + TM_PD + 16 * qt, pk);
           if (shaw_band(p.clip, m, n)) {
 #pragma unroll
             for (int k = 0; k < NC / 2; ++k) {
@@ -686,27 +680,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           tc_fence_before();
           mbar_arrive(BAR(B_PFULL));
         }
-      } else if (MECH == M_DEB && good) {  // P (bf16 pairs) into TMEM for the PV MMA
-        uint32_t pk[NC / 2];
+      } else if (good) {  // P (bf16 pairs) into TMEM for the PV MMA, eight columns at a time
 #pragma unroll
-        for (int k = 0; k < NC / 2; ++k) pk[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
-        tmem_st16(tl + TM_PD + 16 * qt, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(BAR(B_PFULL));
-      } else if (good) {
-        // P quarter-row -> smem sub-tile qt / 2, K-major 128B swizzle: chunk c of row r at chunk c ^ (r & 7)
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[8];
 #pragma unroll
-        for (int cc = 0; cc < NC / 8; ++cc) {
-          const int ch = (NC / 8) * (qt & 1) + cc;
-          uint4 v;
-          v.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
-          v.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
-          v.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
-          v.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
-          *reinterpret_cast<uint4 *>(smem + OFF_P + 16384 * (qt >> 1) + 128 * il + ((ch ^ (il & 7)) << 4)) = v;
+          for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(x[16 * hh + 2 * k], x[16 * hh + 2 * k + 1]);
+          tmem_st8(tl + TM_PD + 16 * qt + 8 * hh, pk);
         }
-        fence_async_smem();
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(B_PFULL));
       }
