@@ -59,6 +59,7 @@ struct BwdArgs {
   CUtensorMap mpd;       // stored P / dS tiles: [planes][128][64] bf16, four 16 KB planes per tile
   __nv_bfloat16 *pd;     // (P keys 0-63, P keys 64-127, dS likewise) and their base
   int pd_stored;         // 1: the query-tile kernel stores P and dS; dK / dV and dr come from them
+  int n_kvs;             // streaming launch: CTAs of the key-tile role (the rest run the diagonal role)
 };
 
 // First of the four 16 KB planes of tile (m, n) of (batch, head) bh in the stored-tile
@@ -446,20 +447,20 @@ enum { B_LD0 = 0, B_LD1, B_FR0, B_FR1, B_DONE, B_DRAIN, NB };
 constexpr uint32_t T_DV = 0, T_DK = 64;  // dK | c: 80 columns
 }  // namespace kvs
 
-__global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_constant__ BwdArgs A) {
+// Body of the key-tile role for CTA index `cta` of its role.  Warps 0-3 (epilogue) and 4
+// (control) work; any further warps of the block only pass its two block barriers.
+__device__ __forceinline__ void kvs_body(const BwdArgs &A, uint8_t *smem, int cta) {
   using namespace kvs;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nth = (int)blockDim.x;
   const int BH = p.B * p.H;
-  const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH, h = bh % p.H;
+  const int bh = cta % BH, n = cta / BH, h = bh % p.H;
   const int L = p.L, j0 = n * 128;
   // query tiles holding only Transformer-XL memory placeholders (rows < mem_len) are skipped
   const int mStart = max(p.causal ? n : 0, p.mem_len / 128), iters = p.nT - mStart;
   const int klen = key_len(p, bh / p.H);
   if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0, no du contribution (whole CTA, no barrier yet)
-    for (int x = tid; x < 128 * (HD / 8); x += NTH) {
+    for (int x = tid; x < 128 * (HD / 8); x += nth) {
       const int r = x / (HD / 8), c8 = x % (HD / 8);
       if (j0 + r < L) {
         const size_t off = ((size_t)bh * L + j0 + r) * HD + 8 * c8;
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_co
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int x = tid; x < 16384 / 16; x += NTH) {
+  for (int x = tid; x < 16384 / 16; x += nth) {
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
@@ -535,7 +536,7 @@ __global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_co
       ctl.drain(BAR(B_DRAIN));
     }
     __syncwarp();
-  } else {  // epilogue: lane il is key j0 + il; this thread takes all 64 columns
+  } else if (warp < 4) {  // epilogue: lane il is key j0 + il; this thread takes all 64 columns
     const int il = 32 * warp + lane, j = j0 + il;
     const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
     float csum = 0.f;
@@ -591,6 +592,11 @@ __global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_co
     tc_fence_after();
     tmem_dealloc(tbase, 256);
   }
+}
+
+__global__ void __launch_bounds__(kvs::NTH, 1) tc_bwd_kvs_kernel(const __grid_constant__ BwdArgs A) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  kvs_body(A, (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023), (int)blockIdx.x);
 }
 
 // ============================================================================
@@ -1189,14 +1195,13 @@ enum { B_LD0 = 0, B_LD1, B_EFULL, B_EFREE, B_DRAIN, NB };
 constexpr uint32_t T_GLO = 0, T_GHI = 128;  // G | g: 80 columns each
 }  // namespace dgs
 
-__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_dgs_kernel(const __grid_constant__ BwdArgs A) {
+// Body of the diagonal role for CTA index `cta` of its role (NTHREADS threads).
+__device__ __forceinline__ void dgs_body(const BwdArgs &A, uint8_t *smem, int cta) {
   using namespace dgs;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const Prm &p = A.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BH = p.B * p.H;
-  const int bh = (int)blockIdx.x % BH, rr0 = (int)blockIdx.x / BH;
+  const int bh = cta % BH, rr0 = cta / BH;
   const int chunk = rr0 % A.dg_nchunk, rank = rr0 / A.dg_nchunk;
   const int D = p.causal ? rank : ((rank & 1) ? (rank + 1) / 2 : -(rank / 2));
   const int band = p.causal ? D : D + (p.nT - 1);
@@ -1326,6 +1331,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_dgs_kernel(const __grid_co
     tc_fence_after();
     tmem_dealloc(tbase, 256);
   }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_dgs_kernel(const __grid_constant__ BwdArgs A) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  dgs_body(A, (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023), (int)blockIdx.x);
+}
+
+// Both streaming roles in one launch.  They are independent (each only reads the stored
+// tiles and Q / dO) and bound differently -- the key-tile role by DRAM bandwidth, the
+// diagonal role by latency -- so their CTAs are interleaved in the grid (the k-th
+// key-tile CTA at index ~ k * gridDim / n_kvs, each role keeping its own heaviest-first
+// order) and the scheduler runs them side by side.
+constexpr int STREAM_SMEM = kvs::SMEM > dgs::SMEM ? kvs::SMEM : dgs::SMEM;
+
+__global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_stream_kernel(const __grid_constant__ BwdArgs A) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint64_t c = blockIdx.x, total = gridDim.x, nk = (uint64_t)A.n_kvs;
+  const int before = (int)(c * nk / total), upto = (int)((c + 1) * nk / total);  // key-tile CTAs in [0, c) / [0, c]
+  if (upto > before)
+    kvs_body(A, smem, before);
+  else
+    dgs_body(A, smem, (int)c - before);
 }
 
 // dr[h][rho][e] = s (sum G + (sum g) v[e]) over the batch, the bands holding
@@ -1504,25 +1532,22 @@ cudaError_t tc_bwd(const Prm &p0, const TcWork &w, cudaStream_t st) {
     return e;
   const unsigned tiles = (unsigned)(nT * p0.H * p0.B);
   const unsigned qtiles = (unsigned)((nT - p0.mem_len / 128) * p0.H * p0.B);  // no memory-placeholder query tiles
-  if (a.pd_stored) {  // the query-tile kernel first: the key-tile pass streams its P / dS tiles
-    if ((e = cudaFuncSetAttribute(tc_bwd_kvs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::SMEM)) != cudaSuccess)
+  const unsigned diag_ctas = (unsigned)(nbands * nchunk * p0.B * p0.H);
+  if (a.pd_stored) {  // the query-tile kernel first; then both roles streaming its P / dS tiles
+    if ((e = cudaFuncSetAttribute(tc_bwd_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, STREAM_SMEM)) !=
+        cudaSuccess)
       return e;
     RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<qtiles, NTHREADS, qk::SMEM, st>>>(a));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    RP_TRACED("tc_bwd_kvs_kernel", st, tc_bwd_kvs_kernel<<<tiles, kvs::NTH, kvs::SMEM, st>>>(a));
+    a.n_kvs = (int)tiles;
+    RP_TRACED("tc_bwd_stream_kernel", st, tc_bwd_stream_kernel<<<tiles + diag_ctas, NTHREADS, STREAM_SMEM, st>>>(a));
   } else {
     RP_TRACED("tc_bwd_kv_kernel", st, tc_bwd_kv_kernel<<<tiles, NTHREADS, kv::SMEM, st>>>(a));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     RP_TRACED("tc_bwd_q_kernel", st, tc_bwd_q_kernel<<<qtiles, NTHREADS, qk::SMEM, st>>>(a));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (a.pd_stored) {
-    if ((e = cudaFuncSetAttribute(tc_bwd_dgs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dgs::SMEM)) != cudaSuccess)
-      return e;
-    RP_TRACED("tc_bwd_dgs_kernel", st, tc_bwd_dgs_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dgs::SMEM, st>>>(a));
-  } else {
-    RP_TRACED("tc_bwd_diag_kernel", st, tc_bwd_diag_kernel<<<(unsigned)(nbands * nchunk * p0.B * p0.H), NTHREADS, dg::SMEM, st>>>(a));
-  }
+  if (!a.pd_stored) RP_TRACED("tc_bwd_diag_kernel", st, tc_bwd_diag_kernel<<<diag_ctas, NTHREADS, dg::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   RP_TRACED("reduce_dr_kernel", st, reduce_dr_kernel<<<(unsigned)(p0.H * ((p0.nrows + 31) / 32)), 256, 0, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -95,8 +95,12 @@ def kernel_launches(wl, path):
         fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
     else:
         fwd = 1 + t5
-    if tc_bwd and wl.mech == TXL:  # D, relation prep, key-tile, query-tile, diagonal, dr and u/v reductions
-        bwd = 7
+    if tc_bwd and wl.mech == TXL:
+        nt = (wl.L + wl.mem_len + 127) // 128
+        tiles = wl.B * wl.H * (nt * (nt + 1) // 2 if wl.causal else nt * nt)
+        # stored P / dS tiles (up to 16 GiB): D, relation prep, query-tile, one launch of both
+        # streaming roles, dr and u/v reductions; else key-tile, query-tile and diagonal kernels
+        bwd = 6 if tiles * 65536 <= 16 << 30 else 7
     elif tc_bwd and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction; the value
         bwd = 7 if wl.shaw_value else 5  # side adds the dO.aV products and the daV reduction
     elif tc_bwd and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
@@ -327,9 +331,8 @@ def run_reference(args, wl):
 # not credited): the Transformer-XL backward's 8U split over its kernels.
 KERNEL_CREDIT_U = {
     (TXL, "tc_bwd_q_kernel"): 5,     # S = Q K^T, the relation products, dP, dS K and E r (dQ)
-    (TXL, "tc_bwd_kvs_kernel"): 2,   # dV = P^T dO, dK = dS^T Q
-    (TXL, "tc_bwd_kv_kernel"): 2,    # the same (it recomputes S, P, dS: not credited)
-    (TXL, "tc_bwd_dgs_kernel"): 1,   # G = E^T Q (dr)
+    (TXL, "tc_bwd_stream_kernel"): 3,  # dV = P^T dO, dK = dS^T Q and G = E^T Q (dr) from the stored tiles
+    (TXL, "tc_bwd_kv_kernel"): 2,    # dV, dK (it recomputes S, P, dS: not credited)
     (TXL, "tc_bwd_diag_kernel"): 1,  # the same (recomputing)
 }
 # DRAM traffic per launch of a kernel (dram__bytes_read.sum + dram__bytes_write.sum) from

@@ -68,17 +68,20 @@ def test_median_iqr(xs):
 
 
 def test_kernel_launch_counts_of_the_default_workload():
-    """Transformer-XL bf16: relation prep + forward; D, relation prep, query-tile, the two
-    tile-streaming kernels, dr and u / v reductions (the ncu launch list's kernels)."""
-    assert bench.kernel_launches(WORKLOADS["txl_causal_L8192_bf16"], "auto") == (2, 7)
+    """Transformer-XL bf16: relation prep + forward; D, relation prep, query-tile, the
+    streaming launch, dr and u / v reductions; past 16 GiB of stored tiles the three
+    recomputing kernels instead."""
+    assert bench.kernel_launches(WORKLOADS["txl_causal_L8192_bf16"], "auto") == (2, 6)
+    assert bench.kernel_launches(WORKLOADS["txl_L32768_bf16"], "auto") == (2, 7)
 
 
 def test_txl_backward_credit_splits_8U():
     """The Transformer-XL backward's algorithmic 8U, split over the kernels of each
-    variant: query-tile 5U with the streaming (2U + 1U) or recomputing (2U + 1U) kernels."""
+    variant: query-tile 5U with the streaming launch (3U) or the recomputing key-tile and
+    diagonal kernels (2U + 1U)."""
     c = bench.KERNEL_CREDIT_U
     T = bench.TXL
-    assert c[(T, "tc_bwd_q_kernel")] + c[(T, "tc_bwd_kvs_kernel")] + c[(T, "tc_bwd_dgs_kernel")] == 8
+    assert c[(T, "tc_bwd_q_kernel")] + c[(T, "tc_bwd_stream_kernel")] == 8
     assert c[(T, "tc_bwd_q_kernel")] + c[(T, "tc_bwd_kv_kernel")] + c[(T, "tc_bwd_diag_kernel")] == 8
 
 
