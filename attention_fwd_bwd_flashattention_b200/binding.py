@@ -78,6 +78,18 @@ def lib_path() -> str:
     return _LIB_PATH
 
 
+RELEASE_LIB = _LIB_PATH
+DEBUG_LIB = os.path.join(os.path.dirname(_LIB_PATH), "librelpos_attn_debug.so")
+
+
+def use_library(path: str) -> None:
+    """Bind every wrapper to the library at `path` from now on (e.g. the RELPOS_DEBUG
+    build, _lib/librelpos_attn_debug.so, in tests)."""
+    global _lib, _LIB_PATH
+    _LIB_PATH = path
+    _lib = None
+
+
 def load() -> ctypes.CDLL:
     """Load the compiled library (raises if it was not built)."""
     global _lib

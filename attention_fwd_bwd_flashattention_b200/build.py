@@ -18,6 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "_lib")
 LIBNAME = "librelpos_attn.so"
+DEBUG_LIBNAME = "librelpos_attn_debug.so"  # RELPOS_DEBUG: index checks of the kernels' stores
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -32,12 +33,12 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def lib_path() -> str:
-    return os.path.join(LIBDIR, LIBNAME)
+def lib_path(debug: bool = False) -> str:
+    return os.path.join(LIBDIR, DEBUG_LIBNAME if debug else LIBNAME)
 
 
-def up_to_date() -> bool:
-    out = lib_path()
+def up_to_date(debug: bool = False) -> bool:
+    out = lib_path(debug)
     if not os.path.exists(out):
         return False
     t = os.path.getmtime(out)
@@ -45,16 +46,17 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    """Compile (if stale) and return the path of the shared library.  Each source is
+def build(force: bool = False, verbose: bool = False, extra=None, debug: bool = False) -> str:
+    """Compile (if stale) and return the path of the shared library (debug: the
+    RELPOS_DEBUG build, whose kernels check the indices of their stores).  Each source is
     compiled by its own nvcc process (in parallel), then the objects are linked."""
-    if not force and up_to_date():
-        return lib_path()
+    if not force and up_to_date(debug):
+        return lib_path(debug)
     os.makedirs(LIBDIR, exist_ok=True)
-    objdir = os.path.join(LIBDIR, "obj")
+    objdir = os.path.join(LIBDIR, "obj_debug" if debug else "obj")
     os.makedirs(objdir, exist_ok=True)
     flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "--expt-relaxed-constexpr",
-             "-I", INCLUDE, "-I", CSRC, *(extra or [])]
+             "-I", INCLUDE, "-I", CSRC, *(["-DRELPOS_DEBUG"] if debug else []), *(extra or [])]
 
     def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
@@ -75,14 +77,15 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
             failed = True
     if failed:
         raise subprocess.CalledProcessError(1, "nvcc")
-    tmp = lib_path() + ".tmp"
+    tmp = lib_path(debug) + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *[o for _, o, _ in results]]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, lib_path())
-    return lib_path()
+    os.replace(tmp, lib_path(debug))
+    return lib_path(debug)
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True, extra=["-Xptxas", "-v"] if "--ptxas" in sys.argv else None))
+    print(build(force="--force" in sys.argv, verbose=True, extra=["-Xptxas", "-v"] if "--ptxas" in sys.argv else None,
+                debug="--debug" in sys.argv))

@@ -16,7 +16,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10600;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len; 1.5.0: relpos_selftest_wait; 1.6.0: relpos_trace_begin / _end
+constexpr int kVersion = 10700;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len; 1.5.0: relpos_selftest_wait; 1.6.0: relpos_trace_begin / _end; 1.7.0: relpos_last_cuda_error, RELPOS_ERR_BOUNDS
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -529,6 +529,7 @@ extern "C" const char *relpos_strerror(int status) {
     case RELPOS_ERR_LAUNCH: return "kernel launch failed";
     case RELPOS_ERR_TIMEOUT: return "a bounded device wait ran out";
     case RELPOS_ERR_CUDA: return "CUDA runtime error";
+    case RELPOS_ERR_BOUNDS: return "an index check of the debug build failed (the access was skipped)";
     default: return "unknown status";
   }
 }

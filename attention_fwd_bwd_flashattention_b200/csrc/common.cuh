@@ -19,6 +19,22 @@ namespace rp {
 
 constexpr int HD = 64;  // head dimension supported by every kernel
 constexpr int RELPOS_ERR_TIMEOUT_DEV = -5;  // value of RELPOS_ERR_TIMEOUT written to the device status word
+constexpr int RELPOS_ERR_BOUNDS_DEV = -7;   // value of RELPOS_ERR_BOUNDS (debug build)
+
+// Index check of the debug build (RELPOS_DEBUG): true when the access may go ahead.  A
+// failed check writes RELPOS_ERR_BOUNDS to the status word and the caller skips the
+// access; control flow is otherwise unchanged, so every barrier stays balanced.  In the
+// release build it is the constant true and the check disappears.
+__device__ __forceinline__ bool dcheck(bool ok, int32_t *status) {
+#ifdef RELPOS_DEBUG
+  if (!ok && status) *status = RELPOS_ERR_BOUNDS_DEV;
+  return ok;
+#else
+  (void)status;
+  (void)ok;
+  return true;
+#endif
+}
 
 enum { M_T5 = 0, M_SHAW = 1, M_TXL = 2, M_DEB = 3 };
 

@@ -404,8 +404,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_kv_kernel(const __grid_con
           wk.y = pack_bf16x2(kv[2], kv[3]);
           wk.z = pack_bf16x2(kv[4], kv[5]);
           wk.w = pack_bf16x2(kv[6], kv[7]);
-          *reinterpret_cast<uint4 *>(dvp + 8 * c8) = wv;
-          *reinterpret_cast<uint4 *>(dkp + 8 * c8) = wk;
+          if (dcheck((size_t)(dvp + 8 * c8 - (__nv_bfloat16 *)p.dv) + 8 <= (size_t)BH * L * HD, status)) {
+            *reinterpret_cast<uint4 *>(dvp + 8 * c8) = wv;
+            *reinterpret_cast<uint4 *>(dkp + 8 * c8) = wk;
+          }
         }
       } else {
         csum = 0.f;
@@ -570,8 +572,10 @@ __device__ __forceinline__ void kvs_body(const BwdArgs &A, uint8_t *smem, int ct
             wk.y = pack_bf16x2(kv[2], kv[3]);
             wk.z = pack_bf16x2(kv[4], kv[5]);
             wk.w = pack_bf16x2(kv[6], kv[7]);
-            *reinterpret_cast<uint4 *>(dvp + 8 * c8) = wv;
-            *reinterpret_cast<uint4 *>(dkp + 8 * c8) = wk;
+            if (dcheck((size_t)(dvp + 8 * c8 - (__nv_bfloat16 *)p.dv) + 8 <= (size_t)BH * L * HD, status)) {
+              *reinterpret_cast<uint4 *>(dvp + 8 * c8) = wv;
+              *reinterpret_cast<uint4 *>(dkp + 8 * c8) = wk;
+            }
           }
         }
       }
@@ -822,7 +826,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
       // row-major bf16 P / dS planes of this tile for the key-tile kernel: row il, keys cb .. cb + 31
       __nv_bfloat16 *pdrow = A.pd_stored ? A.pd + (size_t)(tile_plane(p, bh, m, n) + (qt >> 1)) * 8192 + il * 64 + 32 * (qt & 1)
                                          : nullptr;
-      if (A.pd_stored && good) {
+      // elements of the stored-tile buffer: four 8192-element planes per stored tile
+      const size_t pd_elems = (size_t)BH * (p.causal ? p.nT * (p.nT + 1) / 2 : p.nT * p.nT) * 4 * 8192;
+      if (A.pd_stored && good && dcheck((size_t)(pdrow - A.pd) + 2 * 8192 + NC <= pd_elems, status)) {
 #pragma unroll
         for (int c8 = 0; c8 < NC / 8; ++c8)
           *reinterpret_cast<uint4 *>(pdrow + 8 * c8) =
@@ -854,7 +860,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-        if (A.pd_stored) {
+        if (A.pd_stored && dcheck((size_t)(pdrow - A.pd) + 2 * 8192 + NC <= pd_elems, status)) {
 #pragma unroll
           for (int c8 = 0; c8 < NC / 8; ++c8)
             *reinterpret_cast<uint4 *>(pdrow + 2 * 8192 + 8 * c8) = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
@@ -886,7 +892,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
           w.y = pack_bf16x2(p.scale * u2f(r[8 * c8 + 2]), p.scale * u2f(r[8 * c8 + 3]));
           w.z = pack_bf16x2(p.scale * u2f(r[8 * c8 + 4]), p.scale * u2f(r[8 * c8 + 5]));
           w.w = pack_bf16x2(p.scale * u2f(r[8 * c8 + 6]), p.scale * u2f(r[8 * c8 + 7]));
-          *reinterpret_cast<uint4 *>(dqp + 8 * c8) = w;
+          if (dcheck((size_t)(dqp + 8 * c8 - (__nv_bfloat16 *)p.dq) + 8 <= (size_t)BH * L * HD, status))
+            *reinterpret_cast<uint4 *>(dqp + 8 * c8) = w;
         }
       }
     }
@@ -1161,12 +1168,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_diag_kernel(const __grid_c
       tmem_wait_ld();
       // partial layout [block lo / hi][65][128 offsets]: G columns 0..63, then g
       float *part = A.part_dg + (((size_t)bh * A.nbands + band) * A.dg_nchunk + chunk) * DG_STRIDE;
+      const bool part_ok = dcheck(
+          (size_t)(part - A.part_dg) + DG_STRIDE <= (size_t)BH * A.nbands * A.dg_nchunk * DG_STRIDE, status);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
+      for (int e = 0; e < 16 && part_ok; ++e) {
         part[(size_t)(16 * qt + e) * 128 + il] = u2f(rlo[e]);
         part[(size_t)(65 + 16 * qt + e) * 128 + il] = u2f(rhi[e]);
       }
-      if (qt == 0) {
+      if (qt == 0 && part_ok) {
         part[(size_t)64 * 128 + il] = u2f(glo[0]);
         part[(size_t)(65 + 64) * 128 + il] = u2f(ghi[0]);
       }
@@ -1314,12 +1323,14 @@ __device__ __forceinline__ void dgs_body(const BwdArgs &A, uint8_t *smem, int ct
       tmem_ld16(tl + T_GLO + 64, glo);
       tmem_ld16(tl + T_GHI + 64, ghi);
       tmem_wait_ld();
+      const bool part_ok = dcheck(
+          (size_t)(part - A.part_dg) + DG_STRIDE <= (size_t)BH * A.nbands * A.dg_nchunk * DG_STRIDE, status);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
+      for (int e = 0; e < 16 && part_ok; ++e) {
         part[(size_t)(16 * qt + e) * 128 + il] = u2f(rlo[e]);
         part[(size_t)(65 + 16 * qt + e) * 128 + il] = u2f(rhi[e]);
       }
-      if (qt == 0) {
+      if (qt == 0 && part_ok) {
         part[(size_t)64 * 128 + il] = u2f(glo[0]);
         part[(size_t)(65 + 64) * 128 + il] = u2f(ghi[0]);
       }

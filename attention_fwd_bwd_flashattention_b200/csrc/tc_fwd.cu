@@ -734,9 +734,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           v.y = pack_bf16x2(u2f(r[8 * c8 + 2]) * inv, u2f(r[8 * c8 + 3]) * inv);
           v.z = pack_bf16x2(u2f(r[8 * c8 + 4]) * inv, u2f(r[8 * c8 + 5]) * inv);
           v.w = pack_bf16x2(u2f(r[8 * c8 + 6]) * inv, u2f(r[8 * c8 + 7]) * inv);
-          *reinterpret_cast<uint4 *>(orow + 8 * c8) = v;
+          if (dcheck((size_t)(orow + 8 * c8 - (__nv_bfloat16 *)p.out) + 8 <= (size_t)BH * L * HD, status))
+            *reinterpret_cast<uint4 *>(orow + 8 * c8) = v;
         }
-        if (qt == 0) p.lse[(size_t)bh * L + i] = ltot > 0.f ? (m2 + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+        if (qt == 0 && dcheck((size_t)bh * L + i < (size_t)BH * L, status))
+          p.lse[(size_t)bh * L + i] = ltot > 0.f ? (m2 + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
       }
     }
     tc_fence_before();

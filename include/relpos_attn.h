@@ -68,6 +68,11 @@
  * enqueued before it may still run, and the outputs are undefined.
  * Nothing aborts, traps or throws across this boundary.
  *
+ * Debug build: the library built with RELPOS_DEBUG (librelpos_attn_debug.so) checks
+ * the indices of its kernels' global stores and skew / offset-order shared-memory
+ * stores; a failed check skips that access and writes RELPOS_ERR_BOUNDS to the
+ * status word (no thread leaves a kernel early: the barriers stay balanced).
+ *
  * Determinism: the backward pass uses no atomic operations; the relative-table
  * gradients are reduced from per-shard partials in a fixed order, so repeated
  * calls give bitwise identical results.
@@ -104,7 +109,9 @@ enum relpos_status {
   RELPOS_ERR_UNSUPPORTED = -3,      /* valid but not implemented (e.g. path/dtype)  */
   RELPOS_ERR_LAUNCH = -4,           /* a kernel launch was rejected by the driver  */
   RELPOS_ERR_TIMEOUT = -5,          /* (device status only) a bounded wait ran out  */
-  RELPOS_ERR_CUDA = -6              /* a CUDA runtime call failed                    */
+  RELPOS_ERR_CUDA = -6,             /* a CUDA runtime call failed                    */
+  RELPOS_ERR_BOUNDS = -7            /* (device status only, debug build) an index
+                                       check failed; the access was skipped          */
 };
 
 typedef struct relpos_params {

@@ -86,8 +86,8 @@ def test_trace_registration_is_validated(lib):
 
 
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10600
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    assert lib.relpos_attn_version() == 10700
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"
 
@@ -243,3 +243,14 @@ def test_resolved_paths(lib):
     wider = dict(mech=bd.T5, B=1, H=2, t5_max_distance=20000)
     assert bd.relpos_attn_resolved_path(bd.Params(L=32768, **wider), 1) == SIMT
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, t5_bidirectional=False, **wide), 1) == TC  # one side flat
+
+
+def test_debug_build_exports_the_same_abi():
+    """The RELPOS_DEBUG build (index-checked stores) is a complete library with the same
+    exported C ABI."""
+    path = bld.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert {s for s in exported if s.startswith("relpos")} == set(declared_symbols())
+    dlib = ctypes.CDLL(path)
+    assert dlib.relpos_attn_version() == 10700
