@@ -16,7 +16,7 @@ namespace {
 
 using rp::Prm;
 
-constexpr int kVersion = 10700;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len; 1.5.0: relpos_selftest_wait; 1.6.0: relpos_trace_begin / _end; 1.7.0: relpos_last_cuda_error, RELPOS_ERR_BOUNDS
+constexpr int kVersion = 10800;  // 1.1.0: seqlens_k; 1.2.0: RELPOS_ALIBI; 1.3.0: shaw_value; 1.4.0: mem_len; 1.5.0: relpos_selftest_wait; 1.6.0: relpos_trace_begin / _end; 1.7.0: relpos_last_cuda_error, RELPOS_ERR_BOUNDS; 1.8.0: Shaw c > 64 on the tensor cores
 constexpr int kTile = 64;        // query/key tile of the CUDA-core kernels
 constexpr int kMaxL = 1 << 20;
 
@@ -77,6 +77,16 @@ static int fill_t5(const relpos_params_t *P, Prm &p) {
   return RELPOS_OK;
 }
 
+// Transformer-XL diagonal bands of tiles and their chunking for the relation-gradient partials
+static void set_bands(Prm &p) {
+  p.nbands = p.causal ? p.nT : 2 * p.nT - 1;
+  long long cap = 4000 / ((long long)p.B * p.H * p.nbands);
+  int nch = (int)((p.nT + 7) / 8);
+  if (cap < nch) nch = (int)(cap < 1 ? 1 : cap);
+  p.diag_ch = (p.nT + nch - 1) / nch;
+  p.diag_nchunk = (p.nT + p.diag_ch - 1) / p.diag_ch;
+}
+
 static int validate_and_fill(const relpos_params_t *P, Prm &p) {
   if (!P) return RELPOS_ERR_INVALID_ARG;
   memset(&p, 0, sizeof(p));
@@ -131,20 +141,30 @@ static int validate_and_fill(const relpos_params_t *P, Prm &p) {
       p.nrows = 2 * p.span;
       break;
   }
-  if (p.mech == rp::M_TXL) {
-    p.nbands = p.causal ? p.nT : 2 * p.nT - 1;
-    long long cap = 4000 / ((long long)p.B * p.H * p.nbands);
-    int nch = (int)((p.nT + 7) / 8);
-    if (cap < nch) nch = (int)(cap < 1 ? 1 : cap);
-    p.diag_ch = (p.nT + nch - 1) / nch;
-    p.diag_nchunk = (p.nT + p.diag_ch - 1) / p.diag_ch;
-  }
+  if (p.mech == rp::M_TXL) set_bands(p);
   return RELPOS_OK;
+}
+
+// Shaw with a clip over 64 (and no value-side table): the relative term s q_i . a[clip(j - i)]
+// is the Transformer-XL relation term s q_i . r_{i-j} of the table expanded to one row per
+// offset, r_rho = a[clip(-(rho - off)) + c], with u = v = 0; the gradient of a is the
+// expanded table's gradient summed over the offsets each row of a stands for.  It runs on
+// the relation-block kernels, whose tiles need no per-clip layout.
+static bool shaw_wide(const Prm &p) { return p.mech == rp::M_SHAW && !p.shaw_v && p.clip > 64; }
+
+static Prm txl_view(const Prm &p) {
+  Prm t = p;
+  t.mech = rp::M_TXL;
+  t.nrows = p.causal ? p.L : 2 * p.L - 1;
+  t.off = p.causal ? 0 : p.L - 1;
+  set_bands(t);
+  return t;
 }
 
 // Which kernel family runs pass `pass` (0 forward, 1 backward) of a call.
 static bool use_tc(const relpos_params_t *P, const Prm &p, int pass) {
   if (P->dtype != RELPOS_BF16 || P->kernel_path == RELPOS_PATH_SIMT) return false;
+  if (shaw_wide(p)) return true;
   if (pass == 1)
     return p.mech == rp::M_TXL || (p.mech == rp::M_SHAW && rp::tc_bwd_shaw_supported(p)) ||
            (p.mech == rp::M_T5 && rp::tc_bwd_bias_supported(p)) || (p.mech == rp::M_DEB && rp::tc_bwd_deb_supported(p));
@@ -156,15 +176,42 @@ struct Layout {
   size_t t5_bias, t5_bkt, dvec, part_row, part_col, part_small, part_diag, gtot, part_val;
   size_t uk, vr, c2pE, p2cE;  // tensor-core products
   size_t part_kv, part_dg, part_uv, qa, da;  // tensor-core backward partials / products
-  size_t qkr, kqr, dM, dN, dqc, dkc, dpart;  // DeBERTa tensor-core backward
+  size_t qkr, kqr, dM, dN, dqc, dkc, dpart, dpad;  // DeBERTa tensor-core backward
   size_t pdtiles;                            // Transformer-XL tensor-core backward: stored P / dS tiles (0: none)
   size_t mq, mo, mlse, mdo, mdq;             // Transformer-XL memory: query-side tensors padded to M + L rows
+  size_t xtab, xzero, xdr, xduv;             // wide-clip Shaw: expanded table, zero u / v, its gradients
   size_t total;
 };
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // lean: the smallest backward workspace (no stored P / dS tiles)
-static Layout layout_of(const Prm &p, int pass, bool tc, bool lean = false) {
+static Layout layout_of(const Prm &p, int pass, bool tc, bool lean = false);
+
+// wide-clip Shaw: the Transformer-XL layout of the same shape, then the expanded table
+// (bf16 [H][rows][d]), the zero u / v vector (bf16 [H][d]) and, for the backward, the
+// expanded table's gradient and the u / v gradients (fp32, discarded)
+static Layout wide_layout(const Prm &p, int pass, bool lean) {
+  const Prm t = txl_view(p);
+  Layout l = layout_of(t, pass, true, lean);
+  size_t off = l.total;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  const size_t tab = (size_t)p.H * t.nrows * rp::HD;
+  l.xtab = take(2 * tab);
+  l.xzero = take(2 * (size_t)p.H * rp::HD);
+  if (pass == 1) {
+    l.xdr = take(sizeof(float) * tab);
+    l.xduv = take(sizeof(float) * 2 * (size_t)p.H * rp::HD);
+  }
+  l.total = off;
+  return l;
+}
+
+static Layout layout_of(const Prm &p, int pass, bool tc, bool lean) {
+  if (tc && shaw_wide(p)) return wide_layout(p, pass, lean);
   Layout l;
   memset(&l, 0, sizeof(l));
   size_t off = 0;
@@ -189,8 +236,8 @@ static Layout layout_of(const Prm &p, int pass, bool tc, bool lean = false) {
     }
   }
   if (pass == 1 && tc && p.mech == rp::M_DEB) {  // tensor-core backward (DeBERTa)
-    size_t tab = 0, partf = 0;
-    rp::tc_bwd_deb_sizes(p, tab, partf);
+    size_t tab = 0, partf = 0, padn = 0;
+    rp::tc_bwd_deb_sizes(p, tab, partf, padn);
     l.dvec = take(sizeof(float) * BH * p.L);
     l.qkr = take(sizeof(float) * tab);
     l.kqr = take(sizeof(float) * tab);
@@ -199,6 +246,7 @@ static Layout layout_of(const Prm &p, int pass, bool tc, bool lean = false) {
     l.dqc = take(sizeof(float) * BH * p.L * rp::HD);
     l.dkc = take(sizeof(float) * BH * p.L * rp::HD);
     l.dpart = take(sizeof(float) * partf);
+    l.dpad = take(2 * padn);
   } else if (pass == 1 && tc && p.mech == rp::M_T5) {  // tensor-core backward (T5, ALiBi): per-query-tile partials
     l.dvec = take(sizeof(float) * BH * p.L);
     l.part_small = take(sizeof(float) * BH * (size_t)((p.L + 127) / 128) * p.nb);
@@ -289,6 +337,7 @@ static rp::TcWork tc_work(const Layout &l, void *ws) {
   w.dpart = (float *)(b + l.dpart);
   w.dM = b + l.dM;
   w.dN = b + l.dN;
+  w.dpad = b + l.dpad;
   w.pdtiles = l.pdtiles ? b + l.pdtiles : nullptr;
   return w;
 }
@@ -357,6 +406,18 @@ static cudaError_t unpad_rows(void *dst, const void *src, size_t rb, const Prm &
                            cudaMemcpyDeviceToDevice, st);
 }
 
+// wide-clip Shaw: the expanded table of the Transformer-XL view t (rel0 of t) from a (rel0
+// of p), the zero u / v vector (rel1 = rel2 of t)
+static cudaError_t wide_tables(const Prm &p, Prm &t, void *xtab, void *xzero, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(xzero, 0, 2 * (size_t)p.H * rp::HD, st);
+  if (e != cudaSuccess) return e;
+  if ((e = rp::launch_shaw_expand(p, t, xtab, st)) != cudaSuccess) return e;
+  t.rel0 = xtab;
+  t.rel1 = xzero;
+  t.rel2 = xzero;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" int relpos_attn_workspace_size(const relpos_params_t *params, int pass, size_t *bytes) {
@@ -422,6 +483,11 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
     p.lse = (float *)(wb + l.mlse);
   }
   const bool bf16 = params->dtype == RELPOS_BF16;
+  if (tc && shaw_wide(p)) {
+    Prm t = txl_view(p);
+    if ((e = to_status(wide_tables(p, t, wb + l.xtab, wb + l.xzero, st)))) return e;
+    return to_status(rp::tc_fwd(t, tc_work(l, workspace), st));
+  }
   if (p.mech == rp::M_T5 && (e = to_status(rp::launch_t5_prep(p, st)))) return e;
   e = tc ? to_status(rp::tc_fwd(p, tc_work(l, workspace), st)) : to_status(rp::simt_fwd(p, bf16, st));
   if (e || p.mem_len == 0) return e;
@@ -489,6 +555,16 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
     p.dout = wb + l.mdo;
     p.lse = (float *)(wb + l.mlse);
     p.dq = wb + l.mdq;
+  }
+  if (tc && shaw_wide(p)) {
+    Prm t = txl_view(p);
+    if ((e = to_status(wide_tables(p, t, wb + l.xtab, wb + l.xzero, st)))) return e;
+    t.drel0 = (float *)(wb + l.xdr);
+    t.drel1 = (float *)(wb + l.xduv);
+    t.drel2 = t.drel1 + (size_t)p.H * rp::HD;
+    if ((e = to_status(rp::launch_dvec(t, bf16, st)))) return e;
+    if ((e = to_status(rp::tc_bwd(t, tc_work(l, workspace), st)))) return e;
+    return to_status(rp::launch_shaw_collapse(p, t, t.drel0, p.drel0, st));
   }
   if (tc) {
     if ((e = to_status(rp::launch_dvec(p, bf16, st)))) return e;

@@ -31,7 +31,7 @@ struct TcWork {
   // DeBERTa backward: relation products QKr, KQr and dS K, dS^T Q (fp32), the
   // offset-ordered dS copies M, N (bf16, [B,H,L][2k]) and the table-gradient partials
   float *qkr, *kqr, *dqc, *dkc, *dpart;
-  void *dM, *dN;
+  void *dM, *dN, *dpad;  // dpad: Kr, Qr padded with zero rows to a multiple of 64 (bf16)
 };
 bool tc_supported(const Prm &p);
 cudaError_t tc_prep(const Prm &p, const TcWork &w, cudaStream_t st);
@@ -43,9 +43,13 @@ bool tc_bwd_shaw_supported(const Prm &p);
 size_t tc_bwd_shaw_qa_floats(const Prm &p);
 cudaError_t tc_bwd_shaw(const Prm &p, const TcWork &w, cudaStream_t st);
 bool tc_bwd_deb_supported(const Prm &p);
-void tc_bwd_deb_sizes(const Prm &p, size_t &table_elems, size_t &part_floats);
+void tc_bwd_deb_sizes(const Prm &p, size_t &table_elems, size_t &part_floats, size_t &pad_elems);
 cudaError_t tc_bwd_deb(const Prm &p, const TcWork &w, cudaStream_t st);
 bool tc_bwd_bias_supported(const Prm &p);
 cudaError_t tc_bwd_bias(const Prm &p, cudaStream_t st);
 cudaError_t launch_dvec(const Prm &p, bool bf16, cudaStream_t st);
+// wide-clip Shaw on the Transformer-XL kernels (view t): the table expanded to one row per
+// offset, and its gradient summed back into the 2c + 1 rows
+cudaError_t launch_shaw_expand(const Prm &p, const Prm &t, void *xtab, cudaStream_t st);
+cudaError_t launch_shaw_collapse(const Prm &p, const Prm &t, const float *xdr, float *da, cudaStream_t st);
 }  // namespace rp

@@ -1,5 +1,5 @@
 // Tensor-core (tcgen05 / TMEM / TMA) backward pass of DeBERTa disentangled
-// attention, bf16, d = 64, span k a multiple of 32 up to 256, sm_100a.  No atomics.
+// attention, bf16, d = 64, any span k, sm_100a.  No atomics.
 //
 // S_ij = s (q_i.k_j + q_i.Kr[rho] + k_j.Qr[rho']) with rho = clip(i - j + k, 0, W - 1)
 // and rho' = clip(j - i + k, 0, W - 1), W = 2k table rows (DeBERTa's content-to-
@@ -17,8 +17,11 @@
 // (128 |m - n| - 127 >= k); only the band of tiles around the diagonal touches interior
 // entries (offset-aware tiling, technique (1)).
 //
-//   tables kernel    QKr = Q Kr^T and KQr = K Qr^T, fp32 [B,H,L][W] (one MMA per 256
-//                    table rows).
+//   tables kernel    QKr = Q Kr^T and KQr = K Qr^T, fp32 [B,H,L][Wp] (one MMA per 256
+//                    table rows, 512 per CTA).
+// Rows of QKr, KQr, M and N are Wp = W rounded up to 64 entries long (the K steps of the
+// rows kernel); the tables are read from copies padded with zero rows to Wp, so the
+// entries past W are zero in M and N and never reach a gradient.
 //   key-tile kernel  recomputes P and dS (band tiles gather both relation products by
 //                    offset, far tiles add the clipped end products), dV += P^T dO,
 //                    dK += dS^T Q, the clipped column sums of dS (far tiles: dS^T 1 on
@@ -49,13 +52,13 @@ struct DebArgs {
   CUtensorMap mq, mk, mv, mdo;  // [B,H,L,64], 128-row boxes
   CUtensorMap mkr256, mqr256;   // tables, 256-row boxes (tables kernel)
   CUtensorMap mkr64, mqr64;     // tables, 64-row boxes (rows kernel)
-  CUtensorMap mM, mN;           // [B,H,L][W] bf16, 64 x 128 boxes
+  CUtensorMap mM, mN;           // [B,H,L][Wp] bf16, 64 x 128 boxes
   Prm p;                        // nT counts 128-row tiles
-  const float *qkr, *kqr;       // [B,H,L][W] relation products
-  __nv_bfloat16 *M, *N;         // [B,H,L][W] offset-ordered dS
+  const float *qkr, *kqr;       // [B,H,L][Wp] relation products
+  __nv_bfloat16 *M, *N;         // [B,H,L][Wp] offset-ordered dS
   float *dqc, *dkc;             // [B,H,L,64] dS K and dS^T Q
   float *part;                  // [2][H][W/128][B*nch][128][64] table-gradient partials
-  int W, nbs, nch;              // table rows, band tiles per side, chunks per plane
+  int W, Wp, nbs, nch;          // table rows, row length of QKr / KQr / M / N, band tiles per side, chunks per plane
 };
 
 __device__ __forceinline__ bool far_left(int m, int n, int k) { return 128 * (m - n) - 127 >= k; }
@@ -69,12 +72,12 @@ constexpr int RLD = 129;  // fp32 stride of the band tile's relation terms in sm
 // a warp's 32 loads of a phase are independent.  Ends with R complete for every row thread.
 __device__ __forceinline__ void band_fill(const DebArgs &A, int bh, int i0, int j0, float *R, int warp, int lane) {
   const Prm &p = A.p;
-  const int L = p.L, W = A.W, k = p.span;
+  const int L = p.L, W = A.W, Wp = A.Wp, k = p.span;
   float v[32];
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int i = i0 + 8 * warp + rr;
-    const float *row = A.qkr + ((size_t)bh * L + (i < L ? i : 0)) * W;
+    const float *row = A.qkr + ((size_t)bh * L + (i < L ? i : 0)) * Wp;
 #pragma unroll
     for (int q = 0; q < 4; ++q) v[4 * rr + q] = (i < L) ? row[iclamp(i - j0 - (lane + 32 * q) + k, 0, W - 1)] : 0.f;
   }
@@ -86,7 +89,7 @@ __device__ __forceinline__ void band_fill(const DebArgs &A, int bh, int i0, int 
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int j = j0 + 8 * warp + rr;
-    const float *row = A.kqr + ((size_t)bh * L + (j < L ? j : 0)) * W;
+    const float *row = A.kqr + ((size_t)bh * L + (j < L ? j : 0)) * Wp;
 #pragma unroll
     for (int q = 0; q < 4; ++q) v[4 * rr + q] = (j < L) ? row[iclamp(j - (i0 + lane + 32 * q) + k, 0, W - 1)] : 0.f;
   }
@@ -138,7 +141,9 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
   const int tid = threadIdx.x, warp = tid >> 5;
   const int BH = p.B * p.H, side = blockIdx.y;
   const int bh = (int)blockIdx.x % BH, m = (int)blockIdx.x / BH, h = bh % p.H;
-  const int L = p.L, W = A.W, i0 = m * 128, nchunk = (W + 255) / 256;
+  // this CTA's 512 (or fewer) columns of the Wp
+  const int L = p.L, Wp = A.Wp, col0 = 512 * (int)blockIdx.z, ncol = min(512, Wp - col0), i0 = m * 128;
+  const int nchunk = (ncol + 255) / 256;
   const uint32_t sbase = smem_u32(smem), bar = sbase + OFF_BAR;
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 32);
   uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 16);
@@ -155,14 +160,14 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
   const uint32_t tbase = *tmem_slot;
   if (tid == 0) {
     const CUtensorMap *mx = side ? &A.mk : &A.mq, *mt = side ? &A.mqr256 : &A.mkr256;
-    const int box = W < 256 ? W : 256;  // table rows per load (the map's box)
+    const int box = Wp < 256 ? Wp : 256;  // table rows per load (the map's box)
     mbar_expect_tx(bar, 16384u + 128u * (uint32_t)box * (uint32_t)nchunk);
     tma_load_3d(sbase + OFF_X, mx, bar, 0, i0, bh);
-    for (int c = 0; c < nchunk; ++c) tma_load_3d(sbase + OFF_T + 32768 * c, mt, bar, 0, 256 * c, h);
+    for (int c = 0; c < nchunk; ++c) tma_load_3d(sbase + OFF_T + 32768 * c, mt, bar, 0, col0 + 256 * c, h);
     if (mbar_wait(bar, 0, abort_flag, p.status, RELPOS_ERR_TIMEOUT_DEV)) {
       tc_fence_after();
       for (int c = 0; c < nchunk; ++c) {
-        const int nc = W - 256 * c < 256 ? W - 256 * c : 256;  // a multiple of 64
+        const int nc = ncol - 256 * c < 256 ? ncol - 256 * c : 256;  // a multiple of 64
         umma_k64(tbase + 256 * c, sbase + OFF_X, sbase + OFF_T + 32768 * c, idesc_bf16(128, nc, false), false);
       }
     } else {  // give the copies still in flight a bounded time to land before the CTA exits
@@ -174,11 +179,11 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
   __syncwarp();
   const bool good = warp_wait(bar + 8, 0, abort_flag, p.status);
   const int i = i0 + tid;
-  float *out = (side ? (float *)A.kqr : (float *)A.qkr) + ((size_t)bh * L + i) * W;
+  float *out = (side ? (float *)A.kqr : (float *)A.qkr) + ((size_t)bh * L + i) * Wp + col0;
   if (good) {
     tc_fence_after();
     const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
-    for (int c0 = 0; c0 < W; c0 += 32) {
+    for (int c0 = 0; c0 < ncol; c0 += 32) {
       uint32_t r[32];
       tmem_ld32(tl + c0, r);
       tmem_wait_ld();
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BH = p.B * p.H;
   const int bh = (int)blockIdx.x % BH, n = (int)blockIdx.x / BH;
-  const int L = p.L, W = A.W, k = p.span, j0 = n * 128;
+  const int L = p.L, W = A.W, Wp = A.Wp, k = p.span, j0 = n * 128;
   const int mStart = p.causal ? n : 0, iters = p.nT - mStart;
   const int klen = key_len(p, bh / p.H);
   if (j0 >= klen) {  // a key tile of padding only: dK = dV = 0, N rows zero (whole CTA, no barrier yet)
@@ -235,9 +240,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
         *reinterpret_cast<float4 *>(A.dkc + off + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    for (int x = tid; x < 128 * (W / 8); x += NTHREADS) {
-      const int r = x / (W / 8), c8 = x % (W / 8);
-      if (j0 + r < L) *reinterpret_cast<uint4 *>(A.N + ((size_t)bh * L + j0 + r) * W + 8 * c8) = make_uint4(0, 0, 0, 0);
+    for (int x = tid; x < 128 * (Wp / 8); x += NTHREADS) {
+      const int r = x / (Wp / 8), c8 = x % (Wp / 8);
+      if (j0 + r < L) *reinterpret_cast<uint4 *>(A.N + ((size_t)bh * L + j0 + r) * Wp + 8 * c8) = make_uint4(0, 0, 0, 0);
     }
     return;
   }
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
   for (int x = tid; x < 1024; x += NTHREADS) red[x] = 0.f;
   if (tid < 256) {  // k_j . Qr_0 (far tiles left of the diagonal) and k_j . Qr_{W-1} (right)
     const int s = tid >> 7, j = j0 + (tid & 127);
-    ek[tid] = (j < L) ? A.kqr[((size_t)bh * L + j) * W + (s ? W - 1 : 0)] : 0.f;
+    ek[tid] = (j < L) ? A.kqr[((size_t)bh * L + j) * Wp + (s ? W - 1 : 0)] : 0.f;
   }
   fence_async_smem();
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -361,8 +366,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
       if (tid < 128) return lse2_of(p, bh, i);
       if (i >= L) return 0.f;
       if (tid < 256) return p.Dvec[(size_t)bh * L + i];
-      if (far_left(m, n, k)) return A.qkr[((size_t)bh * L + i) * W + W - 1];
-      if (far_right(m, n, k)) return A.qkr[((size_t)bh * L + i) * W];
+      if (far_left(m, n, k)) return A.qkr[((size_t)bh * L + i) * Wp + W - 1];
+      if (far_right(m, n, k)) return A.qkr[((size_t)bh * L + i) * Wp];
       return 0.f;
     };
     if (tid < 384) vec[tid] = fetch1(0);
@@ -451,7 +456,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
           const int r = r0 + x, j = j0 + cb + x;
           if (r >= 1 && r <= W - 2 && j < L) {
             const uint32_t v = dk[x >> 1];
-            *reinterpret_cast<uint16_t *>(A.N + ((size_t)bh * L + j) * W + r) = (uint16_t)((x & 1) ? (v >> 16) : (v & 0xFFFFu));
+            *reinterpret_cast<uint16_t *>(A.N + ((size_t)bh * L + j) * Wp + r) = (uint16_t)((x & 1) ? (v >> 16) : (v & 0xFFFFu));
           }
         }
         // clipped column sums of the band tile: class 0 (i - j >= k), class W - 1 (j - i >= k - 1)
@@ -488,7 +493,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
 #pragma unroll 4
       for (int x = 0; x < NC; ++x) {
         const int r = r0 + x, j = j0 + cb + x;
-        if (r >= 1 && r <= W - 2 && j < L) *reinterpret_cast<uint16_t *>(A.N + ((size_t)bh * L + j) * W + r) = 0;
+        if (r >= 1 && r <= W - 2 && j < L) *reinterpret_cast<uint16_t *>(A.N + ((size_t)bh * L + j) * Wp + r) = 0;
       }
     }
     // ---- epilogue: lanes are keys; this thread takes 16 of the 64 columns ----
@@ -520,7 +525,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
           *reinterpret_cast<float4 *>(dkp + 4 * q) = make_float4(u2f(rk[4 * q]), u2f(rk[4 * q + 1]), u2f(rk[4 * q + 2]), u2f(rk[4 * q + 3]));
         if (qt == 0) {  // N end columns: clipped column sums (far tiles from TMEM, band tiles from the butterflies)
           const float c0 = (anyL ? u2f(rc0[0]) : 0.f) + bandC0, cw = (anyR ? u2f(rcw[0]) : 0.f) + bandCW;
-          __nv_bfloat16 *np = A.N + ((size_t)bh * L + j) * W;
+          __nv_bfloat16 *np = A.N + ((size_t)bh * L + j) * Wp;
           np[0] = __float2bfloat16_rn(c0);
           np[W - 1] = __float2bfloat16_rn(cw);
         }
@@ -558,7 +563,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BH = p.B * p.H;
   const int bh = (int)blockIdx.x % BH, m = p.nT - 1 - (int)blockIdx.x / BH;
-  const int L = p.L, W = A.W, k = p.span, i0 = m * 128;
+  const int L = p.L, W = A.W, Wp = A.Wp, k = p.span, i0 = m * 128;
   const int klen = key_len(p, bh / p.H);
   const int nTiles = min(p.causal ? m + 1 : p.nT, (klen + 127) / 128);
   if (nTiles == 0) {  // no key at all: dQ = 0, M rows zero (whole CTA, before any barrier)
@@ -566,9 +571,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
       const int r = x / (HD / 4), c4 = x % (HD / 4);
       if (i0 + r < L) *reinterpret_cast<float4 *>(A.dqc + ((size_t)bh * L + i0 + r) * HD + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int x = tid; x < 128 * (W / 8); x += NTHREADS) {
-      const int r = x / (W / 8), c8 = x % (W / 8);
-      if (i0 + r < L) *reinterpret_cast<uint4 *>(A.M + ((size_t)bh * L + i0 + r) * W + 8 * c8) = make_uint4(0, 0, 0, 0);
+    for (int x = tid; x < 128 * (Wp / 8); x += NTHREADS) {
+      const int r = x / (Wp / 8), c8 = x % (Wp / 8);
+      if (i0 + r < L) *reinterpret_cast<uint4 *>(A.M + ((size_t)bh * L + i0 + r) * Wp + 8 * c8) = make_uint4(0, 0, 0, 0);
     }
     return;
   }
@@ -655,18 +660,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
     const uint32_t tl = tbase + ((uint32_t)(g * 32) << 16);
     const float lse2 = lse2_of(p, bh, i);
     const float Dv = (i < L) ? p.Dvec[(size_t)bh * L + i] : 0.f;
-    const float cE0 = (i < L) ? A.qkr[((size_t)bh * L + i) * W] : 0.f;         // q_i . Kr_0
-    const float cEW = (i < L) ? A.qkr[((size_t)bh * L + i) * W + W - 1] : 0.f;  // q_i . Kr_{W-1}
+    const float cE0 = (i < L) ? A.qkr[((size_t)bh * L + i) * Wp] : 0.f;          // q_i . Kr_0
+    const float cEW = (i < L) ? A.qkr[((size_t)bh * L + i) * Wp + W - 1] : 0.f;  // q_i . Kr_{W-1}
     const uint64_t c12 = f2(c1, c1), nlse = f2(-lse2, -lse2), nDv = f2(-Dv, -Dv);
-    __nv_bfloat16 *mrow = A.M + ((size_t)bh * L + i) * W;
+    __nv_bfloat16 *mrow = A.M + ((size_t)bh * L + i) * Wp;
     bool good = true;
     float rs0 = 0.f, rsW = 0.f;  // clipped row sums: rho = 0 (j - i >= k), rho = W - 1 (i - j >= k - 1)
     // p2c end product of key tile n's keys for the tile's side, one tile ahead
     auto fetch_ek = [&](int n) {
       const int j = n * 128 + tid;
       if (tid >= 128 || j >= L) return 0.f;
-      if (far_left(m, n, k)) return A.kqr[((size_t)bh * L + j) * W];
-      if (far_right(m, n, k)) return A.kqr[((size_t)bh * L + j) * W + W - 1];
+      if (far_left(m, n, k)) return A.kqr[((size_t)bh * L + j) * Wp];
+      if (far_right(m, n, k)) return A.kqr[((size_t)bh * L + j) * Wp + W - 1];
       return 0.f;
     };
     float nva = fetch_ek(0);
@@ -748,7 +753,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
         for (int rr = 0; rr < 8; ++rr) {
           const int ir = i0 + 8 * warp + rr;
           if (ir >= L) continue;
-          __nv_bfloat16 *mr = A.M + ((size_t)bh * L + ir) * W;
+          __nv_bfloat16 *mr = A.M + ((size_t)bh * L + ir) * Wp;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int jl = lane + 32 * q, r = ir - j0 - jl + k;
@@ -819,10 +824,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
 // ============================================================================
 // rows kernel: dq = s (dQ + M Kr) (side 0), dk = s (dK + N Qr) (side 1)
 // ============================================================================
+// The Wp / 64 K steps are staged eight at a time; a group's loads are issued once the
+// previous group's MMAs are done with the staging buffers.
 namespace rw {
-constexpr int OFF_X = 0;                // W / 64 chunks of 128 rows x 64 columns (16 KB each)
-constexpr int OFF_T = 8 * 16384;        // W / 64 chunks of 64 table rows x 64 (8 KB each)
-constexpr int OFF_BAR = OFF_T + 8 * 8192;
+constexpr int GK = 8;                   // K steps per group
+constexpr int OFF_X = 0;                // GK chunks of 128 rows x 64 columns (16 KB each)
+constexpr int OFF_T = GK * 16384;       // GK chunks of 64 table rows x 64 (8 KB each)
+constexpr int OFF_BAR = OFF_T + GK * 8192;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 }  // namespace rw
 
@@ -834,13 +842,15 @@ __global__ void __launch_bounds__(128, 1) deb_rows_kernel(const __grid_constant_
   const int tid = threadIdx.x, warp = tid >> 5;
   const int BH = p.B * p.H, side = blockIdx.y;
   const int bh = (int)blockIdx.x % BH, m = (int)blockIdx.x / BH, h = bh % p.H;
-  const int L = p.L, W = A.W, i0 = m * 128, nk = W / 64;
+  const int L = p.L, i0 = m * 128, nk = A.Wp / 64, ng = (nk + GK - 1) / GK;
+  // bar: a group's loads landed; bar + 8: a group's MMAs done (staging free); bar + 24: all MMAs done
   const uint32_t sbase = smem_u32(smem), bar = sbase + OFF_BAR;
-  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 32);
-  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 16);
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 36);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 32);
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(bar + 8, 1);
+    mbar_init(bar + 24, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -851,28 +861,35 @@ __global__ void __launch_bounds__(128, 1) deb_rows_kernel(const __grid_constant_
   const uint32_t tbase = *tmem_slot;
   if (tid == 0) {
     const CUtensorMap *mx = side ? &A.mN : &A.mM, *mt = side ? &A.mqr64 : &A.mkr64;
-    mbar_expect_tx(bar, (uint32_t)nk * (16384u + 8192u));
-    for (int c = 0; c < nk; ++c) {
-      tma_load_3d(sbase + OFF_X + 16384 * c, mx, bar, 64 * c, i0, bh);
-      tma_load_3d(sbase + OFF_T + 8192 * c, mt, bar, 0, 64 * c, h);
-    }
-    const bool landed = mbar_wait(bar, 0, abort_flag, p.status, RELPOS_ERR_TIMEOUT_DEV);
-    if (!landed) {  // give the copies still in flight a bounded time to land before the CTA exits
-      volatile int none = 0;
-      mbar_wait(bar, 0, &none, p.status, RELPOS_ERR_TIMEOUT_DEV);
-    } else {
+    const uint32_t id = idesc_bf16(128, 64, true);
+    for (int gi = 0; gi < ng; ++gi) {
+      const int c0 = GK * gi, nc = min(GK, nk - c0);
+      const uint32_t ph = (uint32_t)(gi & 1);
+      // the previous group's MMAs read the staging buffers: wait for them first
+      if (gi > 0 && !mbar_wait(bar + 8, ph ^ 1u, abort_flag, p.status, RELPOS_ERR_TIMEOUT_DEV)) break;
+      mbar_expect_tx(bar, (uint32_t)nc * (16384u + 8192u));
+      for (int c = 0; c < nc; ++c) {
+        tma_load_3d(sbase + OFF_X + 16384 * c, mx, bar, 64 * (c0 + c), i0, bh);
+        tma_load_3d(sbase + OFF_T + 8192 * c, mt, bar, 0, 64 * (c0 + c), h);
+      }
+      if (!mbar_wait(bar, ph, abort_flag, p.status, RELPOS_ERR_TIMEOUT_DEV)) {
+        // give the copies still in flight a bounded time to land before the CTA exits
+        volatile int none = 0;
+        mbar_wait(bar, ph, &none, p.status, RELPOS_ERR_TIMEOUT_DEV);
+        break;
+      }
       tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 64, true);
-      for (int c = 0; c < nk; ++c)
+      for (int c = 0; c < nc; ++c)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           umma_bf16(tbase, sdesc_sw128(sbase + OFF_X + 16384 * c + 32 * q, 16, 1024),
-                    sdesc_sw128(sbase + OFF_T + 8192 * c + 2048 * q, 16, 1024), id, (c > 0 || q > 0) ? 1u : 0u);
+                    sdesc_sw128(sbase + OFF_T + 8192 * c + 2048 * q, 16, 1024), id, (c0 + c > 0 || q > 0) ? 1u : 0u);
+      umma_commit(bar + 8);
     }
-    umma_commit(bar + 8);
+    umma_commit(bar + 24);
   }
   __syncwarp();
-  const bool good = warp_wait(bar + 8, 0, abort_flag, p.status);
+  const bool good = warp_wait(bar + 24, 0, abort_flag, p.status) && !*abort_flag;
   const int i = i0 + tid;
   if (good) {
     tc_fence_after();
@@ -1024,13 +1041,16 @@ bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t plane
 bool tc_make_map_bf16_wide(CUtensorMap *m, const void *base, uint32_t row_len, uint64_t rows, uint64_t planes,
                            uint32_t box_rows);
 
-bool tc_bwd_deb_supported(const Prm &p) { return p.mech == M_DEB && p.span % 32 == 0 && p.span <= 256 && p.span >= 32; }
+bool tc_bwd_deb_supported(const Prm &p) { return p.mech == M_DEB && p.span >= 1; }
 
-void tc_bwd_deb_sizes(const Prm &p, size_t &table_elems, size_t &part_floats) {
-  const size_t W = 2 * (size_t)p.span, BH = (size_t)p.B * p.H;
+static int deb_wp(const Prm &p) { return (2 * p.span + 63) / 64 * 64; }
+
+void tc_bwd_deb_sizes(const Prm &p, size_t &table_elems, size_t &part_floats, size_t &pad_elems) {
+  const size_t W = 2 * (size_t)p.span, Wp = (size_t)deb_wp(p), BH = (size_t)p.B * p.H;
   const size_t nch = ((size_t)p.L + tcdeb::CH - 1) / tcdeb::CH;
-  table_elems = BH * p.L * W;
+  table_elems = BH * p.L * Wp;
   part_floats = 2 * (size_t)p.H * ((W + 127) / 128) * p.B * nch * 128 * HD;
+  pad_elems = 2 * (size_t)p.H * Wp * HD;  // Kr and Qr, zero rows W .. Wp - 1
 }
 
 cudaError_t tc_bwd_deb(const Prm &p0, const TcWork &w, cudaStream_t st) {
@@ -1040,6 +1060,7 @@ cudaError_t tc_bwd_deb(const Prm &p0, const TcWork &w, cudaStream_t st) {
   a.p = p0;
   a.p.nT = (p0.L + 127) / 128;
   a.W = 2 * p0.span;
+  a.Wp = deb_wp(p0);
   a.nbs = (p0.span + 254) / 128 - 1;  // band tiles per side (also past the sequence ends: their M / N entries are zeroed)
   a.nch = (p0.L + CH - 1) / CH;
   a.qkr = w.qkr;
@@ -1050,21 +1071,32 @@ cudaError_t tc_bwd_deb(const Prm &p0, const TcWork &w, cudaStream_t st) {
   a.dkc = w.dkc;
   a.part = w.dpart;
   const uint64_t BH = (uint64_t)p0.B * p0.H;
+  // Kr and Qr copied into [H][Wp][64] tables whose rows W .. Wp - 1 are zero
+  __nv_bfloat16 *kp = (__nv_bfloat16 *)w.dpad, *qp = kp + (size_t)p0.H * a.Wp * HD;
+  cudaError_t e;
+  const size_t rowb = (size_t)HD * 2, tabb = (size_t)a.W * rowb, padb = (size_t)a.Wp * rowb;
+  if ((e = cudaMemsetAsync(w.dpad, 0, 2 * (size_t)p0.H * padb, st)) != cudaSuccess) return e;
+  if ((e = cudaMemcpy2DAsync(kp, padb, p0.rel0, tabb, tabb, p0.H, cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
+  if ((e = cudaMemcpy2DAsync(qp, padb, p0.rel1, tabb, tabb, p0.H, cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
+  if (a.Wp != a.W) {  // M and N columns W .. Wp - 1 (no kernel writes them) are zero: the rows kernel's K steps read them
+    const size_t rows = (size_t)BH * p0.L, pitch = (size_t)a.Wp * 2, wb = (size_t)(a.Wp - a.W) * 2;
+    if ((e = cudaMemset2DAsync(a.M + a.W, pitch, 0, wb, rows, st)) != cudaSuccess) return e;
+    if ((e = cudaMemset2DAsync(a.N + a.W, pitch, 0, wb, rows, st)) != cudaSuccess) return e;
+  }
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
         tc_make_map(&a.mv, p0.v, p0.L, BH, 128) && tc_make_map(&a.mdo, p0.dout, p0.L, BH, 128) &&
-        tc_make_map(&a.mkr256, p0.rel0, a.W, p0.H, std::min(a.W, 256)) &&
-        tc_make_map(&a.mqr256, p0.rel1, a.W, p0.H, std::min(a.W, 256)) &&
-        tc_make_map(&a.mkr64, p0.rel0, a.W, p0.H, 64) && tc_make_map(&a.mqr64, p0.rel1, a.W, p0.H, 64) &&
-        tc_make_map_bf16_wide(&a.mM, a.M, a.W, p0.L, BH, 128) && tc_make_map_bf16_wide(&a.mN, a.N, a.W, p0.L, BH, 128)))
+        tc_make_map(&a.mkr256, kp, a.Wp, p0.H, std::min(a.Wp, 256)) &&
+        tc_make_map(&a.mqr256, qp, a.Wp, p0.H, std::min(a.Wp, 256)) &&
+        tc_make_map(&a.mkr64, kp, a.Wp, p0.H, 64) && tc_make_map(&a.mqr64, qp, a.Wp, p0.H, 64) &&
+        tc_make_map_bf16_wide(&a.mM, a.M, a.Wp, p0.L, BH, 128) && tc_make_map_bf16_wide(&a.mN, a.N, a.Wp, p0.L, BH, 128)))
     return cudaErrorInvalidValue;
-  cudaError_t e;
   if ((e = cudaFuncSetAttribute(deb_tables_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tb::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(deb_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kvd::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(deb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qd::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(deb_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rw::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(deb_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tk::SMEM)) != cudaSuccess) return e;
   const unsigned tiles = (unsigned)(a.p.nT * BH);
-  RP_TRACED("deb_tables_kernel", st, deb_tables_kernel<<<dim3(tiles, 2), 128, tb::SMEM, st>>>(a));
+  RP_TRACED("deb_tables_kernel", st, deb_tables_kernel<<<dim3(tiles, 2, (unsigned)((a.Wp + 511) / 512)), 128, tb::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   RP_TRACED("deb_kv_kernel", st, deb_kv_kernel<<<tiles, NTHREADS, kvd::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

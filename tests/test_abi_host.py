@@ -86,7 +86,7 @@ def test_trace_registration_is_validated(lib):
 
 
 def test_version_and_strerror(lib):
-    assert lib.relpos_attn_version() == 10700
+    assert lib.relpos_attn_version() == 10800
     for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert bd.strerror(code) and bd.strerror(code) != "unknown status"
     assert bd.strerror(-99) == "unknown status"
@@ -202,16 +202,17 @@ def test_t5_thresholds_match_oracle_buckets(lib):
 
 def test_resolved_paths(lib):
     """Which kernel family each pass runs (host-side dispatch, no device work): bf16
-    runs on the tensor cores except the backward of DeBERTa with a span that is not a
-    multiple of 32 up to 256, of Shaw with c > 64 and of T5 whose buckets stay distinct
-    over more than 8 tiles;
-    float32 and an explicit CUDA-core request always run the CUDA-core kernels."""
+    runs on the tensor cores except Shaw's value-side table with c > 64 and the backward of T5
+    whose buckets stay distinct over more than 64 tiles (Shaw with c > 64 and no value
+    table runs on the Transformer-XL tensor-core kernels); float32 and an explicit
+    CUDA-core request always run the CUDA-core kernels."""
     TC, SIMT = bd.PATH_TC, bd.PATH_SIMT
     want = {  # (mech, clip) -> (forward, backward) for bf16, automatic choice
         (bd.T5, 64): (TC, TC),
         (bd.SHAW, 64): (TC, TC),
-        (bd.SHAW, 65): (TC, SIMT),
-        (bd.SHAW, 100): (SIMT, SIMT),
+        (bd.SHAW, 65): (TC, TC),
+        (bd.SHAW, 100): (TC, TC),
+        (bd.SHAW, 4096): (TC, TC),
         (bd.TXL, 64): (TC, TC),
         (bd.DEBERTA, 64): (TC, TC),
         (bd.ALIBI, 64): (TC, TC),
@@ -225,8 +226,8 @@ def test_resolved_paths(lib):
         assert bd.relpos_attn_resolved_path(Ps, 0) == SIMT and bd.relpos_attn_resolved_path(Ps, 1) == SIMT
     # T5 buckets distinct out to distance 547 (max_distance 1000) span 11 tiles at L = 4096
     # (CUDA-core backward); at L = 300 all three tiles are band tiles (tensor cores)
-    # DeBERTa: spans that are multiples of 32 up to 256 take the tensor-core backward
-    for span, want_b in ((256, TC), (32, TC), (96, TC), (24, SIMT), (288, SIMT)):
+    # DeBERTa: every span takes the tensor-core backward
+    for span, want_b in ((256, TC), (32, TC), (96, TC), (24, TC), (288, TC), (1, TC), (4096, TC)):
         assert bd.relpos_attn_resolved_path(bd.Params(mech=bd.DEBERTA, B=1, H=2, L=300, deberta_span=span), 1) == want_b, span
     # Shaw's value-side term: tensor cores in both passes for c <= 64
     Pv = bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True)
@@ -253,4 +254,4 @@ def test_debug_build_exports_the_same_abi():
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
     assert {s for s in exported if s.startswith("relpos")} == set(declared_symbols())
     dlib = ctypes.CDLL(path)
-    assert dlib.relpos_attn_version() == 10700
+    assert dlib.relpos_attn_version() == 10800

@@ -150,11 +150,11 @@ def test_parity_deberta_tensor_core_key_lengths(causal):
 def test_parity_shaw_clip(clip, causal, L):
     """Shaw's clip decides which tiles hold unclipped offsets (the tensor-core backward's
     band tiles: only the diagonal one for small c) and where each row's clipped pairs
-    start; c > 64 runs the CUDA-core backward."""
+    start; c > 64 runs on the Transformer-XL kernels over the table expanded by offset."""
     wl = small_wl("shaw", torch.bfloat16, causal, L, shaw_clip=clip)
     P = bd.Params(mech=SHAW, B=wl.B, H=wl.H, L=L, causal=causal, shaw_clip=clip)
-    want_bwd = bd.PATH_TC if clip <= 64 else bd.PATH_SIMT
-    assert bd.relpos_attn_resolved_path(P, 1) == want_bwd
+    assert bd.relpos_attn_resolved_path(P, 0) == bd.PATH_TC
+    assert bd.relpos_attn_resolved_path(P, 1) == bd.PATH_TC
     inp = make_inputs(wl, seed=clip + L)
     compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
 
@@ -377,11 +377,47 @@ def test_parity_shaw_value_o1_tables(clip, L, causal):
     compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
 
 
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("clip,L", [(65, 300), (100, 1100), (257, 700), (1000, 700), (4096, 130)])
+def test_parity_shaw_wide_clip(clip, L, causal):
+    """Shaw with c > 64 on the Transformer-XL tensor-core kernels: the table expanded to
+    one row per offset, its gradient summed back into the 2c + 1 rows.  Tables at std
+    1.0; interior rows, both end rows (the clipped offsets) and c >= L (no offset
+    clipped, the end rows' gradients zero)."""
+    wl = Workload("shaw_wide", SHAW, torch.bfloat16, causal, 2, 2, L, shaw_clip=clip, rel_std=1.0)
+    inp = make_inputs(wl, seed=clip + L)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_TC))
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_parity_shaw_wide_clip_key_lengths_smallest_workspace(causal):
+    """The wide-clip route with per-batch key lengths (an empty key set among them) and
+    with the smallest backward workspace (the recomputing Transformer-XL kernels)."""
+    wl = Workload("shaw_wide_len", SHAW, torch.bfloat16, causal, 3, 2, 700, shaw_clip=150, rel_std=1.0)
+    lens = (700, 0, 257)
+    inp = make_inputs(wl, 11)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO, seqlens_k=lens, bwd_pass=2), seqlens_k=lens)
+
+
 def test_parity_shaw_L2048_o1_tables():
     """The Shaw workload's shape (B2 H8 L2048, clip 64), tables at std 1.0: every output."""
     wl = WORKLOADS["shaw_L2048_bf16"].with_(rel_std=1.0)
     inp = make_inputs(wl, 0)
     compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("span,L", [(1, 300), (24, 700), (100, 1100), (300, 700), (700, 1100), (2000, 300)])
+def test_parity_deberta_any_span(span, L, causal):
+    """DeBERTa's tensor-core backward at spans whose 2k table rows are not a multiple of
+    64 (rows kept Wp = 2k rounded up to 64 long, the tables read from zero-padded copies)
+    or exceed 512 (the relation products in 512-column pieces, the rows kernel's K steps
+    in groups); k = 1 (no interior offset) and k >= L.  Tables at std 1.0."""
+    wl = Workload("deb_span", DEBERTA, torch.bfloat16, causal, 2, 2, L, deberta_span=span, rel_std=1.0)
+    P = params_of(wl, bd.PATH_AUTO)
+    assert bd.relpos_attn_resolved_path(P, 1) == bd.PATH_TC
+    inp = make_inputs(wl, seed=span + L)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_TC))
 
 
 def test_parity_deberta_L8192_o1_tables_one_head():
