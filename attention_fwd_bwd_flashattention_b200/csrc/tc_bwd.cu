@@ -828,12 +828,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
                                          : nullptr;
       // elements of the stored-tile buffer: four 8192-element planes per stored tile
       const size_t pd_elems = (size_t)BH * (p.causal ? p.nT * (p.nT + 1) / 2 : p.nT * p.nT) * 4 * 8192;
+      // (pdrow is 64-byte aligned: 16 KB planes, 128-byte rows, 64-byte halves of a row)
       if (A.pd_stored && good && dcheck((size_t)(pdrow - A.pd) + 2 * 8192 + NC <= pd_elems, status)) {
 #pragma unroll
-        for (int c8 = 0; c8 < NC / 8; ++c8)
-          *reinterpret_cast<uint4 *>(pdrow + 8 * c8) =
-              make_uint4(pack_bf16x2(x[8 * c8], x[8 * c8 + 1]), pack_bf16x2(x[8 * c8 + 2], x[8 * c8 + 3]),
-                         pack_bf16x2(x[8 * c8 + 4], x[8 * c8 + 5]), pack_bf16x2(x[8 * c8 + 6], x[8 * c8 + 7]));
+        for (int c16 = 0; c16 < NC / 16; ++c16) {
+          uint32_t w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(x[16 * c16 + 2 * e], x[16 * c16 + 2 * e + 1]);
+          st_global_32B(pdrow + 16 * c16, w);
+        }
       }
       good = good && warp_wait(BAR(B_DPF), n & 1, abort_flag, status);
       if (good) {
@@ -862,8 +865,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_q_kernel(const __grid_cons
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
         if (A.pd_stored && dcheck((size_t)(pdrow - A.pd) + 2 * 8192 + NC <= pd_elems, status)) {
 #pragma unroll
-          for (int c8 = 0; c8 < NC / 8; ++c8)
-            *reinterpret_cast<uint4 *>(pdrow + 2 * 8192 + 8 * c8) = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+          for (int c16 = 0; c16 < NC / 16; ++c16) st_global_32B(pdrow + 2 * 8192 + 16 * c16, pk + 8 * c16);
         }
         // the previous tile's dS K MMAs read T_DS: wait for them (long done in practice)
         if (n >= 1 && !warp_wait(BAR(B_DSFREE), (n - 1) & 1, abort_flag, status)) good = false;

@@ -339,7 +339,6 @@ KERNEL_CREDIT_U = {
 # one ncu capture of the same build and workload (profiles/tc_kernels_txl_causal_L8192.md);
 # removed whenever that kernel changes.
 KERNEL_TRAFFIC = {
-    ("txl_causal_L8192_bf16", "tc_bwd_q_kernel"): 1131.53e6,
     ("txl_causal_L8192_bf16", "tc_fwd_kernel"): 34.58e6,
     ("txl_causal_L8192_bf16", "tc_bwd_stream_kernel"): 1810.86e6,
 }
