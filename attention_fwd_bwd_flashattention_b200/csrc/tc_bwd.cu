@@ -80,11 +80,13 @@ constexpr int DG_STRIDE = 2 * 128 * 65;
 // partner c' ^ 128 in the other tile gets 0, so both tiles are fully rewritten.
 // x[e] sits at c' = C0 - e, C0 = il - cb + 128: values go out as aligned bf16 pairs;
 // when C0 is even the first and last value pair with a neighbouring thread's and
-// are written alone.
+// are written alone.  The positions of values and zeros are the same for every tile, so
+// a kernel whose E tiles hold nothing else zeroes them once and passes ZERO = false.
 __device__ __forceinline__ uint32_t E_off(uint32_t t, uint32_t rowb, uint32_t r7) {  // t = 2 c', c' even
   return (((t << 7) & 0xC000u) ^ 0x8000u) + rowb + ((t & 126u) ^ r7);
 }
 // pk[k] = bf16 pair (x[2k+1] low, x[2k] high) of the thread's values
+template <bool ZERO = true>
 __device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const uint32_t (&pk)[NC / 2]) {
   const uint32_t C0 = (uint32_t)(il - cb + 128);
   const bool ev = (C0 & 1u) == 0;
@@ -98,18 +100,18 @@ __device__ __forceinline__ void store_E(uint8_t *E, int il, int cb, const uint32
   for (int k = 0; k < NC / 2 - 1; ++k) {
     const uint32_t off = E_off(T0 - 4u * k, rowb, r7);
     *reinterpret_cast<uint32_t *>(E + off) = prmt(pk[k], pk[k + 1], sel);
-    *reinterpret_cast<uint32_t *>(E + (off ^ 0x8000u)) = 0u;
+    if (ZERO) *reinterpret_cast<uint32_t *>(E + (off ^ 0x8000u)) = 0u;
   }
   if (!ev) {
     const uint32_t off = E_off(T0 - 4u * (NC / 2 - 1), rowb, r7);
     *reinterpret_cast<uint32_t *>(E + off) = pk[NC / 2 - 1];
-    *reinterpret_cast<uint32_t *>(E + (off ^ 0x8000u)) = 0u;
+    if (ZERO) *reinterpret_cast<uint32_t *>(E + (off ^ 0x8000u)) = 0u;
   } else {
     const uint32_t o0 = E_off(2u * C0, rowb, r7), o1 = E_off(2u * (C0 - NC), rowb, r7) + 2u;
     *reinterpret_cast<uint16_t *>(E + o0) = (uint16_t)(pk[0] >> 16);
-    *reinterpret_cast<uint16_t *>(E + (o0 ^ 0x8000u)) = 0;
+    if (ZERO) *reinterpret_cast<uint16_t *>(E + (o0 ^ 0x8000u)) = 0;
     *reinterpret_cast<uint16_t *>(E + o1) = (uint16_t)(pk[NC / 2 - 1] & 0xFFFFu);
-    *reinterpret_cast<uint16_t *>(E + (o1 ^ 0x8000u)) = 0;
+    if (ZERO) *reinterpret_cast<uint16_t *>(E + (o1 ^ 0x8000u)) = 0;
   }
 }
 
@@ -1242,6 +1244,9 @@ __device__ __forceinline__ void dgs_body(const BwdArgs &A, uint8_t *smem, int ct
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4 *>(smem + OFF_ONES + 16 * x) = make_uint4(one2, one2, one2, one2);
   }
+  // E's zero entries sit at the same places in every tile: written once here, the rows
+  // then write only the values (store_E<false>)
+  for (int x = tid; x < 65536 / 16; x += NTHREADS) *reinterpret_cast<uint4 *>(smem + OFF_E + 16 * x) = make_uint4(0, 0, 0, 0);
   fence_async_smem();
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
   tc_fence_before();
@@ -1309,7 +1314,7 @@ __device__ __forceinline__ void dgs_body(const BwdArgs &A, uint8_t *smem, int ct
           ds[4 * c + 2] = prmt(v.z, v.z, 0x1032u);
           ds[4 * c + 3] = prmt(v.w, v.w, 0x1032u);
         }
-        store_E(smem + OFF_E, il, cb, ds);
+        store_E<false>(smem + OFF_E, il, cb, ds);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_EFULL));
