@@ -757,10 +757,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 // and the partial dot products are combined by a fixed shuffle tree.
 //   TXL      uk[b,h,j] = u_h . k_j  and  vr[h,rho] = v_h . r_rho
 //   DeBERTa  c2pE[b,h,i] = (q_i . Kr_0, q_i . Kr_last), p2cE[b,h,j] = (k_j . Qr_0, k_j . Qr_last)
+// a . b over eight bf16: a is 16-byte aligned (a row of q, k or a table, which the tensor-core
+// path requires aligned) and read in one load; b (a per-head vector or a table row) may be
+// read element by element
+template <bool B_ALIGNED = false>
 __device__ __forceinline__ float dot8(const __nv_bfloat16 *a, const __nv_bfloat16 *b) {
+  const uint4 av = __ldg(reinterpret_cast<const uint4 *>(a));
+  const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+  uint32_t bw[4];
+  if constexpr (B_ALIGNED) {
+    const uint4 bv = __ldg(reinterpret_cast<const uint4 *>(b));
+    bw[0] = bv.x;
+    bw[1] = bv.y;
+    bw[2] = bv.z;
+    bw[3] = bv.w;
+  }
   float s = 0.f;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) s = fmaf(__bfloat162float(a[c]), __bfloat162float(b[c]), s);
+  for (int c = 0; c < 4; ++c) {
+    const float alo = __uint_as_float(aw[c] << 16), ahi = __uint_as_float(aw[c] & 0xFFFF0000u);
+    float blo, bhi;
+    if constexpr (B_ALIGNED) {
+      blo = __uint_as_float(bw[c] << 16);
+      bhi = __uint_as_float(bw[c] & 0xFFFF0000u);
+    } else {
+      blo = __bfloat162float(b[2 * c]);
+      bhi = __bfloat162float(b[2 * c + 1]);
+    }
+    s = fmaf(alo, blo, s);
+    s = fmaf(ahi, bhi, s);
+  }
   return s;
 }
 __device__ __forceinline__ float sum8(float x) {  // over the eight threads of a row
@@ -798,10 +824,10 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(Prm p, float *uk, float *v
       const bf *Kr = (const bf *)p.rel0 + (size_t)h * p.nrows * HD + 8 * sub;
       const bf *Qr = (const bf *)p.rel1 + (size_t)h * p.nrows * HD + 8 * sub;
       const size_t last = (size_t)(p.nrows - 1) * HD;
-      a0 = dot8(q, Kr);
-      a1 = dot8(q, Kr + last);
-      b0 = dot8(k, Qr);
-      b1 = dot8(k, Qr + last);
+      a0 = dot8<true>(q, Kr);
+      a1 = dot8<true>(q, Kr + last);
+      b0 = dot8<true>(k, Qr);
+      b1 = dot8<true>(k, Qr + last);
     }
     a0 = sum8(a0);
     a1 = sum8(a1);
