@@ -28,7 +28,7 @@
 // A fixed-order reduction turns the partials into dr = s (G + g v), dv = s sum g r
 // and du = s sum_j c_j k_j.
 //
-// Stored tiles (whenever the buffer fits in 16 GiB): the query-tile kernel runs first and
+// Stored tiles (whenever the buffer fits in 32 GiB): the query-tile kernel runs first and
 // its row threads also write every tile's P and dS (bf16, 64 KB per tile) to a workspace
 // buffer; the key-tile and diagonal work then stream those tiles instead of recomputing
 // S, P and dS (tc_bwd_kvs_kernel: dV, [dK | c] MMAs only; tc_bwd_dgs_kernel: E rebuilt in
@@ -1500,12 +1500,12 @@ void tc_bwd_shape(const Prm &p, int &nT, int &nbands, int &ch, int &nchunk) {
 }
 
 // Bytes of the stored P / dS tile buffer: 64 KB per tile of the backward, or 0 when over
-// 16 GiB (the key-tile and diagonal kernels then recompute S, P and dS).
+// 32 GiB (the key-tile and diagonal kernels then recompute S, P and dS).
 size_t tc_bwd_tile_bytes(const Prm &p) {
   const size_t nT = ((size_t)p.L + 127) / 128;
   const size_t ntiles = p.causal ? nT * (nT + 1) / 2 : nT * nT;
   const size_t bytes = (size_t)p.B * p.H * ntiles * 65536;
-  return bytes <= ((size_t)16 << 30) ? bytes : 0;
+  return bytes <= ((size_t)32 << 30) ? bytes : 0;
 }
 
 size_t tc_bwd_part_floats(const Prm &p, size_t &kv_floats) {

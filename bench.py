@@ -98,9 +98,9 @@ def kernel_launches(wl, path):
     if tc_bwd and wl.mech == TXL:
         nt = (wl.L + wl.mem_len + 127) // 128
         tiles = wl.B * wl.H * (nt * (nt + 1) // 2 if wl.causal else nt * nt)
-        # stored P / dS tiles (up to 16 GiB): D, relation prep, query-tile, one launch of both
+        # stored P / dS tiles (up to 32 GiB): D, relation prep, query-tile, one launch of both
         # streaming roles, dr and u/v reductions; else key-tile, query-tile and diagonal kernels
-        bwd = 6 if tiles * 65536 <= 16 << 30 else 7
+        bwd = 6 if tiles * 65536 <= 32 << 30 else 7
     elif tc_bwd and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction; the value
         bwd = 7 if wl.shaw_value else 5  # side adds the dO.aV products and the daV reduction
     elif tc_bwd and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction

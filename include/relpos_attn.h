@@ -167,7 +167,8 @@ typedef struct relpos_params {
  * tensor-core backward recomputes S, P and dS in its key-tile and diagonal kernels.
  * With the pass-1 size or more, the query-tile kernel writes every tile's P and dS
  * (64 KB per 128 x 128 tile, e.g. 1.1 GB at B = 1, H = 8, L = 8192 causal) and those
- * kernels stream them back: faster, but the memory grows with L^2.  Other calls
+ * kernels stream them back: faster, but the memory grows with L^2.  Past 32 GiB of tiles
+ * the pass-1 size leaves them out as well (the recomputing kernels run).  Other calls
  * need the same size for passes 1 and 2.  The split trades memory for time and is
  * no part of the method.
  * Returns RELPOS_OK and sets *bytes, or RELPOS_ERR_INVALID_ARG. */

@@ -157,13 +157,15 @@ def test_smallest_backward_workspace(lib):
 
 def test_backward_workspace_holds_the_stored_tiles(lib):
     """The Transformer-XL tensor-core backward keeps each 128 x 128 tile's P and dS (64 KB)
-    in the workspace while they fit in 16 GiB, and recomputes them past that."""
+    in the workspace while they fit in 32 GiB, and recomputes them past that."""
     tile = 64 * 1024
     P = bd.Params(mech=bd.TXL, B=1, H=8, L=8192, causal=True)
     n_t = 8192 // 128
     assert bd.relpos_attn_workspace_size(P, 1) >= 8 * (n_t * (n_t + 1) // 2) * tile
-    big = bd.Params(mech=bd.TXL, B=1, H=8, L=32768, causal=False)  # 8 x 256^2 tiles = 32 GiB: not stored
-    assert bd.relpos_attn_workspace_size(big, 1) < 8 * 256 * 256 * tile // 4
+    at_limit = bd.Params(mech=bd.TXL, B=1, H=8, L=32768, causal=False)  # 8 x 256^2 tiles = 32 GiB: stored
+    assert bd.relpos_attn_workspace_size(at_limit, 1) >= 8 * 256 * 256 * tile
+    big = bd.Params(mech=bd.TXL, B=1, H=9, L=32768, causal=False)  # 9 x 256^2 tiles = 36 GiB: not stored
+    assert bd.relpos_attn_workspace_size(big, 1) < 9 * 256 * 256 * tile // 4
     f32 = bd.Params(mech=bd.TXL, B=1, H=8, L=8192, causal=True, dtype=bd.F32)  # CUDA-core path: none
     assert bd.relpos_attn_workspace_size(f32, 1) < 8 * (n_t * (n_t + 1) // 2) * tile
 
