@@ -1429,10 +1429,21 @@ __global__ void __launch_bounds__(256) reduce_dr_kernel(BwdArgs A) {
   float pv[8];
   if (ok) {
     float *out = p.drel0 + ((size_t)h * p.nrows + rho) * HD + 8 * eg;
+    // the r row (16-byte aligned: the boundary checks the table's alignment) in one load
+    const uint4 rw4 = __ldg(reinterpret_cast<const uint4 *>(rr));
+    const uint32_t rw[4] = {rw4.x, rw4.y, rw4.z, rw4.w};
+    uint32_t ob[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      out[k] = p.scale * (acc[k] + gs * __bfloat162float(vv[k]));
-      pv[k] = gs * __bfloat162float(rr[k]);
+      ob[k] = __float_as_uint(p.scale * (acc[k] + gs * __bfloat162float(vv[k])));
+      pv[k] = gs * ((k & 1) ? __uint_as_float(rw[k >> 1] & 0xFFFF0000u) : __uint_as_float(rw[k >> 1] << 16));
+    }
+    // a warp's 32 lanes write 32 rows: one 32-byte store each when the gradient buffer allows
+    if ((reinterpret_cast<uintptr_t>(out) & 31u) == 0) {
+      st_global_32B(out, ob);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) out[k] = __uint_as_float(ob[k]);
     }
   } else {
 #pragma unroll

@@ -187,10 +187,9 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
       uint32_t r[32];
       tmem_ld32(tl + c0, r);
       tmem_wait_ld();
-      if (i < L) {
+      if (i < L) {  // rows of Wp floats (Wp a multiple of 64) in the workspace: 32-byte stores
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<float4 *>(out + c0 + 4 * q) = make_float4(u2f(r[4 * q]), u2f(r[4 * q + 1]), u2f(r[4 * q + 2]), u2f(r[4 * q + 3]));
+        for (int q = 0; q < 4; ++q) st_global_32B(out + c0 + 8 * q, r + 8 * q);
       }
     }
   }
