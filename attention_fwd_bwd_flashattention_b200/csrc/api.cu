@@ -457,7 +457,7 @@ extern "C" int relpos_attn_fwd(const relpos_params_t *params, const void *q, con
   if (params->kernel_path == RELPOS_PATH_TC && !tc) return RELPOS_ERR_UNSUPPORTED;
   if (tc) {  // TMA needs 16-byte aligned tensors
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(rel[0]) ||
-        (p.mech == rp::M_DEB && !aligned16(rel[1])))
+        ((p.mech == rp::M_DEB || p.shaw_v) && !aligned16(rel[1])))
       return RELPOS_ERR_INVALID_ARG;
   }
   const Layout l = layout_of(p, 0, tc);
@@ -534,7 +534,7 @@ extern "C" int relpos_attn_bwd(const relpos_params_t *params, const void *q, con
   if (tc) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(rel[0]))
       return RELPOS_ERR_INVALID_ARG;
-    if (p.mech == rp::M_DEB && !aligned16(rel[1])) return RELPOS_ERR_INVALID_ARG;
+    if ((p.mech == rp::M_DEB || p.shaw_v) && !aligned16(rel[1])) return RELPOS_ERR_INVALID_ARG;
   }
   if ((e = ensure_context())) return e;  // argument errors are all found above
   const size_t rb = (size_t)p.esize * rp::HD;

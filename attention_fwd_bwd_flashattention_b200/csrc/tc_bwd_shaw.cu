@@ -62,65 +62,86 @@ __device__ __forceinline__ bool band_tile(int c, int m, int n) {
 // ---------------------------------------------------------------------------
 // QA[b,h,i][rho] = q_i . a_rho (and, for the value side, DA[b,h,i][rho] = dO_i . aV_rho):
 // X[b,h,i][rho] = x_i . T_rho for rows x [B,H,L,64] and a table T [H,rows,64], rho < 132
-// (rows past the table give 0).  One CTA per 64 rows of one (b,h), both operands staged
-// transposed (d-major) in smem; each thread accumulates a 4-row x 8-column register
-// tile of rho < 128 (one f32 FMA per product, fixed order over d) and one of the 256
-// products of rho = 128..131.
+// (rows past the table give 0).  One CTA per 128 rows of one (b,h): TMA brings the x tile
+// and the table (n = 2c + 1 rows rounded up to 16, rows past the table read as zeros), one
+// tcgen05 MMA (M = 128, N = n, K = 64) leaves the products in TMEM (the same products the
+// forward computes for its QA tile), and each of the four warps writes its 32 rows.
 // ---------------------------------------------------------------------------
-constexpr int QA_ROWS = 64;
-constexpr int QA_XS = QA_ROWS + 4;  // padded smem row of x^T (floats)
-constexpr int QA_TS = QA_LD + 4;    // padded smem row of T^T (floats)
-constexpr int QA_SMEM = (HD * QA_XS + HD * QA_TS) * 4;
-__global__ void __launch_bounds__(256) shaw_qa_kernel(Prm p, const __nv_bfloat16 *xrows, const __nv_bfloat16 *table,
-                                                      float *qa) {
-  extern __shared__ __align__(16) float qsm[];
-  float *Xs = qsm;               // [64 d][QA_XS]: x^T
-  float *Ts = qsm + HD * QA_XS;  // [64 d][QA_TS]: T^T
-  const int tid = threadIdx.x;
-  const int tiles = (p.L + QA_ROWS - 1) / QA_ROWS;
-  const int bh = (int)blockIdx.x / tiles, i0 = ((int)blockIdx.x % tiles) * QA_ROWS, h = bh % p.H;
-  const __nv_bfloat16 *a = table + (size_t)h * p.nrows * HD;
-  const __nv_bfloat16 *q = xrows + ((size_t)bh * p.L) * HD;
-  for (int x = tid; x < QA_LD * HD; x += 256) {
-    const int r = x / HD, d = x % HD;
-    Ts[d * QA_TS + r] = r < p.nrows ? __bfloat162float(a[(size_t)r * HD + d]) : 0.f;
+struct QaArgs {
+  CUtensorMap mx, mt;  // rows x (128-row boxes), table T (n-row box)
+  Prm p;               // nT counts 128-row tiles
+  float *out;          // [B,H,L][QA_LD]
+  int n;               // table rows multiplied (a multiple of 16, <= 144)
+};
+namespace qat {
+constexpr int OFF_X = 0, OFF_T = 16384;   // x tile 16 KB, table up to 144 x 128 B
+constexpr int OFF_BAR = OFF_T + 144 * 128;
+constexpr int SMEM = OFF_BAR + 64 + 1024;
+}  // namespace qat
+__global__ void __launch_bounds__(128, 1) shaw_qa_kernel(const __grid_constant__ QaArgs A) {
+  using namespace qat;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const Prm &p = A.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int BH = p.B * p.H;
+  const int bh = (int)blockIdx.x % BH, m = (int)blockIdx.x / BH, h = bh % p.H, i0 = m * 128;
+  const uint32_t sbase = smem_u32(smem), bar = sbase + OFF_BAR;
+  volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 20);
+  uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 16);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 8, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
   }
-  for (int x = tid; x < QA_ROWS * HD; x += 256) {
-    const int r = x / HD, d = x % HD;
-    Xs[d * QA_XS + r] = (i0 + r < p.L) ? __bfloat162float(q[(size_t)(i0 + r) * HD + d]) : 0.f;
-  }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
+  tc_fence_before();
   __syncthreads();
-  const int r4 = tid >> 4, c8 = tid & 15;  // rows 4 r4 .. +3, columns 8 c8 .. +7
-  float acc[4][8];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-  const int tr = tid >> 2, tc = 128 + (tid & 3);  // the tail product of this thread
-  float tail = 0.f;
-#pragma unroll 4
-  for (int d = 0; d < HD; ++d) {
-    const float4 xv = *reinterpret_cast<const float4 *>(Xs + d * QA_XS + 4 * r4);
-    const float4 t0 = *reinterpret_cast<const float4 *>(Ts + d * QA_TS + 8 * c8);
-    const float4 t1 = *reinterpret_cast<const float4 *>(Ts + d * QA_TS + 8 * c8 + 4);
-    const float xr[4] = {xv.x, xv.y, xv.z, xv.w};
-    const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(xr[r], tv[c], acc[r][c]);
-    tail = fmaf(Xs[d * QA_XS + tr], Ts[d * QA_TS + tc], tail);
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  if (tid == 0) {
+    mbar_expect_tx(bar, 16384u + 128u * (uint32_t)A.n);
+    tma_load_3d(sbase + OFF_X, &A.mx, bar, 0, i0, bh);
+    tma_load_3d(sbase + OFF_T, &A.mt, bar, 0, 0, h);
+    if (mbar_wait(bar, 0, abort_flag, p.status, RELPOS_ERR_TIMEOUT_DEV)) {
+      tc_fence_after();
+      umma_k64(tbase, sbase + OFF_X, sbase + OFF_T, idesc_bf16(128, A.n, false), false);
+    } else {  // give the copies still in flight a bounded time to land before the CTA exits
+      volatile int none = 0;
+      mbar_wait(bar, 0, &none, p.status, RELPOS_ERR_TIMEOUT_DEV);
+    }
+    umma_commit(bar + 8);
   }
+  __syncwarp();
+  const bool good = warp_wait(bar + 8, 0, abort_flag, p.status) && !*abort_flag;
+  const int i = i0 + 32 * warp + lane;
+  if (good) {
+    tc_fence_after();
+    const uint32_t tl = tbase + ((uint32_t)(warp * 32) << 16);
+    float *out = A.out + ((size_t)bh * p.L + (i < p.L ? i : 0)) * QA_LD;
+    for (int c0 = 0; c0 < QA_LD; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tl + c0, r);
+      tmem_wait_ld();
+      if (i < p.L) {
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int i = i0 + 4 * r4 + r;
-    if (i < p.L) {
-      float *out = qa + ((size_t)bh * p.L + i) * QA_LD + 8 * c8;
-      *reinterpret_cast<float4 *>(out) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-      *reinterpret_cast<float4 *>(out + 4) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+        for (int q = 0; q < 8; ++q) {
+          const int c = c0 + 4 * q;
+          if (c < QA_LD)  // columns past the n multiplied (0 .. 3 of the last chunk) are zero
+            *reinterpret_cast<float4 *>(out + c) =
+                make_float4(c < A.n ? u2f(r[4 * q]) : 0.f, c + 1 < A.n ? u2f(r[4 * q + 1]) : 0.f,
+                            c + 2 < A.n ? u2f(r[4 * q + 2]) : 0.f, c + 3 < A.n ? u2f(r[4 * q + 3]) : 0.f);
+        }
+      }
     }
   }
-  if (i0 + tr < p.L) qa[((size_t)bh * p.L + i0 + tr) * QA_LD + tc] = tail;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
 }
 
 // log2-domain scores of four keys, y = (s + R) c1 - lse2, with the relation terms R
@@ -868,15 +889,23 @@ cudaError_t tc_bwd_shaw(const Prm &p0, const TcWork &w, cudaStream_t st) {
         tc_make_map_f32_rows(&a.mqa, w.qa, QA_LD, p0.L, BH, 128)))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  const unsigned qa_blocks = (unsigned)(BH * ((p0.L + QA_ROWS - 1) / QA_ROWS));
-  if ((e = cudaFuncSetAttribute(shaw_qa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QA_SMEM)) != cudaSuccess)
+  const unsigned qa_blocks = (unsigned)(BH * a.p.nT);
+  QaArgs qa;
+  memset(&qa, 0, sizeof(qa));
+  qa.p = a.p;
+  qa.n = (2 * p0.clip + 1 + 15) / 16 * 16;
+  qa.out = w.qa;
+  qa.mx = a.mq;
+  if (!tc_make_map(&qa.mt, p0.rel0, p0.nrows, p0.H, (uint32_t)qa.n)) return cudaErrorInvalidValue;
+  if ((e = cudaFuncSetAttribute(shaw_qa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qat::SMEM)) != cudaSuccess)
     return e;
-  RP_TRACED("shaw_qa_kernel", st,
-            shaw_qa_kernel<<<qa_blocks, 256, QA_SMEM, st>>>(a.p, (const bf *)p0.q, (const bf *)p0.rel0, w.qa));
+  RP_TRACED("shaw_qa_kernel", st, shaw_qa_kernel<<<qa_blocks, 128, qat::SMEM, st>>>(qa));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (p0.shaw_v) {  // DA = dO aV^T by row, for the value side
-    RP_TRACED("shaw_qa_kernel", st,
-              shaw_qa_kernel<<<qa_blocks, 256, QA_SMEM, st>>>(a.p, (const bf *)p0.dout, (const bf *)p0.rel1, w.da));
+    qa.out = w.da;
+    qa.mx = a.mdo;
+    if (!tc_make_map(&qa.mt, p0.rel1, p0.nrows, p0.H, (uint32_t)qa.n)) return cudaErrorInvalidValue;
+    RP_TRACED("shaw_qa_kernel", st, shaw_qa_kernel<<<qa_blocks, 128, qat::SMEM, st>>>(qa));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = p0.shaw_v ? run_shaw_bwd<true>(a, st) : run_shaw_bwd<false>(a, st)) != cudaSuccess) return e;

@@ -45,6 +45,9 @@
  *       DeBERTa  rel[0] = Kr [H, 2k, d], rel[1] = Qr [H, 2k, d]
  *       ALiBi    rel[0] = m  [H]  per-head slopes            float32 always
  *     Unused entries may be NULL.
+ *     On the tensor-core path (bfloat16) Q, K, V, dO and the bf16 tables rel[0] (and
+ *     rel[1] for DeBERTa and for Shaw's value table) must start on a 16-byte boundary;
+ *     RELPOS_ERR_INVALID_ARG otherwise.
  *   - LSE: float32 [B, H, L], natural log.
  *   - drel[0..2]: float32 gradients with the shapes of rel[0..2], summed over the
  *     batch; they are overwritten (not accumulated into).

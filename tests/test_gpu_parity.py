@@ -182,6 +182,37 @@ def test_key_lengths_on_the_host_are_rejected():
     assert ei.value.code == -1
 
 
+@pytest.mark.parametrize("which", ["q", "a", "aV"])
+def test_misaligned_tensor_core_operands_are_rejected(which):
+    """The tensor-core path reads Q, K, V, dO and the bf16 tables with 16-byte loads (TMA
+    and vector loads): a tensor that starts 2 bytes off a 16-byte boundary is refused on
+    the host with RELPOS_ERR_INVALID_ARG, before anything is launched."""
+    P = bd.Params(mech=SHAW, B=1, H=2, L=64, shaw_clip=8, shaw_value=True)
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16, device="cuda")
+    a = torch.zeros(2, 17, 64, dtype=torch.bfloat16, device="cuda")
+    aV = torch.zeros(2, 17, 64, dtype=torch.bfloat16, device="cuda")
+
+    def off(t):  # same shape, one element further on: 2 bytes past the 16-byte boundary
+        return torch.zeros(t.numel() + 1, dtype=t.dtype, device=t.device)[1:].view(t.shape)
+
+    if which == "q":
+        q = off(q)
+    elif which == "a":
+        a = off(a)
+    else:
+        aV = off(aV)
+    o, lse = torch.empty_like(q), torch.empty(1, 2, 64, dtype=torch.float32, device="cuda")
+    with pytest.raises(bd.RelposError) as ei:
+        bd.relpos_attn_fwd(P, q, q, q, [a, aV], o, lse, bd.workspace(P, 0, q.device))
+    assert ei.value.code == -1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    drel = [torch.empty(2, 17, 64, dtype=torch.float32, device="cuda") for _ in range(2)]
+    with pytest.raises(bd.RelposError) as ei:
+        bd.relpos_attn_bwd(P, q, q, q, [a, aV], o, lse, q, dq, dk, dv, drel, bd.workspace(P, 1, q.device))
+    assert ei.value.code == -1
+    torch.cuda.synchronize()
+
+
 def test_key_lengths_match_truncated_keys():
     """A batch whose keys stop at Lk gives the same O and LSE as the same keys with
     everything after Lk replaced (T5 and Shaw depend only on j - i)."""
