@@ -401,8 +401,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_kv_kernel(const __grid_consta
             for (int c4 = 0; c4 < 4; ++c4) {
               const int x0 = 16 * hq + 4 * c4;
               float R[4], y[4], pr[4], dd[4];
+              if constexpr (decltype(banded)::value) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) R[e] = decltype(banded)::value ? Rrow[x0 + e] : cE + ekr[x0 + e];
+                for (int e = 0; e < 4; ++e) R[e] = Rrow[x0 + e];
+              } else {  // four keys' end products in one 16-byte load (aligned: cb, x0 multiples of 4)
+                const float4 ev = *reinterpret_cast<const float4 *>(ekr + x0);
+                R[0] = cE + ev.x;
+                R[1] = cE + ev.y;
+                R[2] = cE + ev.z;
+                R[3] = cE + ev.w;
+              }
               score_rel4(rs + 4 * c4, R, c12, nlse, y);
               if constexpr (decltype(masked)::value) {
 #pragma unroll
@@ -702,8 +710,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
             for (int c4 = 0; c4 < 4; ++c4) {
               const int x0 = 16 * hq + 4 * c4;
               float R[4], y[4], pr[4], dd[4];
+              if constexpr (decltype(banded)::value) {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) R[e] = decltype(banded)::value ? Rrow[x0 + e] : cE + ekr[x0 + e];
+                for (int e = 0; e < 4; ++e) R[e] = Rrow[x0 + e];
+              } else {  // four keys' end products in one 16-byte load (aligned: cb, x0 multiples of 4)
+                const float4 ev = *reinterpret_cast<const float4 *>(ekr + x0);
+                R[0] = cE + ev.x;
+                R[1] = cE + ev.y;
+                R[2] = cE + ev.z;
+                R[3] = cE + ev.w;
+              }
               score_rel4(rs + 4 * c4, R, c12, nlse, y);
               if constexpr (decltype(masked)::value) {
 #pragma unroll
