@@ -128,9 +128,12 @@ __device__ __forceinline__ float warp_colsum32(float (&v)[32], int lane) {
 // ============================================================================
 // tables kernel: QKr = Q Kr^T (side 0), KQr = K Qr^T (side 1)
 // ============================================================================
+// One CTA per 128 rows, side and 256 columns of the Wp: 256 TMEM columns each, and shared
+// memory sized so that two CTAs share an SM (one writes its rows out while the other's
+// loads and MMA run).
 namespace tb {
-constexpr int OFF_X = 0, OFF_T = 16384, OFF_BAR = OFF_T + 2 * 32768;
-constexpr int SMEM = 120 * 1024;  // one CTA per SM (512 TMEM columns each)
+constexpr int OFF_X = 0, OFF_T = 16384, OFF_BAR = OFF_T + 32768;
+constexpr int SMEM = 100 * 1024;  // two CTAs per SM (256 TMEM columns each), never three
 }  // namespace tb
 
 __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constant__ DebArgs A) {
@@ -141,9 +144,9 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
   const int tid = threadIdx.x, warp = tid >> 5;
   const int BH = p.B * p.H, side = blockIdx.y;
   const int bh = (int)blockIdx.x % BH, m = (int)blockIdx.x / BH, h = bh % p.H;
-  // this CTA's 512 (or fewer) columns of the Wp
-  const int L = p.L, Wp = A.Wp, col0 = 512 * (int)blockIdx.z, ncol = min(512, Wp - col0), i0 = m * 128;
-  const int nchunk = (ncol + 255) / 256;
+  // this CTA's 256 (or fewer) columns of the Wp
+  const int L = p.L, Wp = A.Wp, col0 = 256 * (int)blockIdx.z, ncol = min(256, Wp - col0), i0 = m * 128;
+  const int nchunk = 1;
   const uint32_t sbase = smem_u32(smem), bar = sbase + OFF_BAR;
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 32);
   uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 16);
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
     umma_commit(bar + 8);
   }
   __syncwarp();
-  const bool good = warp_wait(bar + 8, 0, abort_flag, p.status);
+  const bool good = warp_wait(bar + 8, 0, abort_flag, p.status) && !*abort_flag;
   const int i = i0 + tid;
   float *out = (side ? (float *)A.kqr : (float *)A.qkr) + ((size_t)bh * L + i) * Wp + col0;
   if (good) {
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(128, 1) deb_tables_kernel(const __grid_constan
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tbase, 512);
+    tmem_dealloc(tbase, 256);
   }
 }
 
@@ -839,10 +842,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) deb_q_kernel(const __grid_constan
 // ============================================================================
 // rows kernel: dq = s (dQ + M Kr) (side 0), dk = s (dK + N Qr) (side 1)
 // ============================================================================
-// The Wp / 64 K steps are staged eight at a time; a group's loads are issued once the
+// The Wp / 64 K steps are staged four at a time; a group's loads are issued once the
 // previous group's MMAs are done with the staging buffers.
 namespace rw {
-constexpr int GK = 8;                   // K steps per group
+constexpr int GK = 4;                   // K steps per group (96 KB: two CTAs per SM)
 constexpr int OFF_X = 0;                // GK chunks of 128 rows x 64 columns (16 KB each)
 constexpr int OFF_T = GK * 16384;       // GK chunks of 64 table rows x 64 (8 KB each)
 constexpr int OFF_BAR = OFF_T + GK * 8192;
@@ -1111,7 +1114,7 @@ cudaError_t tc_bwd_deb(const Prm &p0, const TcWork &w, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(deb_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rw::SMEM)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(deb_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tk::SMEM)) != cudaSuccess) return e;
   const unsigned tiles = (unsigned)(a.p.nT * BH);
-  RP_TRACED("deb_tables_kernel", st, deb_tables_kernel<<<dim3(tiles, 2, (unsigned)((a.Wp + 511) / 512)), 128, tb::SMEM, st>>>(a));
+  RP_TRACED("deb_tables_kernel", st, deb_tables_kernel<<<dim3(tiles, 2, (unsigned)((a.Wp + 255) / 256)), 128, tb::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   RP_TRACED("deb_kv_kernel", st, deb_kv_kernel<<<tiles, NTHREADS, kvd::SMEM, st>>>(a));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
