@@ -645,7 +645,8 @@ def run_e2e(args, wl, c, dev, stream, world, mode="single"):
     from pinned host memory and its results (O, LSE, dQ, dK, dV, drel) copied back.  Steps are
     pipelined over two buffer sets: step k's host-to-device copies (one stream) and
     step k - 1's device-to-host copies (another) overlap step k - 1's / k's kernels (the
-    compute stream); events order every reuse of a buffer.  The timed region runs from
+    compute stream); within a step dO's copy overlaps the forward and O / LSE go back
+    under the backward; events order every reuse of a buffer.  The timed region runs from
     the first input copy to the last result copy."""
     P, inp = c.P, c.inp
     host_in = {n: inp[n].pin_memory() for n in ("q", "k", "v", "do")}
@@ -670,32 +671,42 @@ def run_e2e(args, wl, c, dev, stream, world, mode="single"):
     h2d = sum(t.numel() * t.element_size() for t in list(host_in.values()) + host_rel)
     d2h = sum(t.numel() * t.element_size() for t in bufs[0]["out"])
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # q, k, v and the tables landed
+    ev_in_do = [torch.cuda.Event() for _ in range(2)]  # dO landed (the backward's only extra input)
+    ev_fwd = [torch.cuda.Event() for _ in range(2)]    # O, LSE written
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def step(kk):
         i = kk & 1
         B = bufs[i]
+        res = results(B)
         with torch.cuda.stream(s_in):
             s_in.wait_event(ev_done[i])  # the kernels of step kk - 2 are done with these inputs
-            for n in ("q", "k", "v", "do"):
+            for n in ("q", "k", "v"):
                 B[n].copy_(host_in[n], non_blocking=True)
             for dst, src in zip(B["rel"], host_rel):
                 dst.copy_(src, non_blocking=True)
             ev_in[i].record(s_in)
+            B["do"].copy_(host_in["do"], non_blocking=True)  # under the forward
+            ev_in_do[i].record(s_in)
         with torch.cuda.stream(stream):
             stream.wait_event(ev_in[i])
             stream.wait_event(ev_out[i])  # step kk - 2's results have left these buffers
             bd.relpos_attn_fwd(P, B["q"], B["k"], B["v"], B["rel"], B["o"], B["lse"], ws_f, stream=stream)
+            ev_fwd[i].record(stream)
+            stream.wait_event(ev_in_do[i])
             bd.relpos_attn_bwd(P, B["q"], B["k"], B["v"], B["rel"], B["o"], B["lse"], B["do"], B["dq"], B["dk"], B["dv"],
                                B["drel"], ws_b, stream=stream)
             if mode == "batch":
                 rdist.allreduce_table_grads(B["drel"])
             ev_done[i].record(stream)
         with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_fwd[i])  # O and LSE go out under the backward (which only reads them)
+            for dst, src in zip(B["out"][:2], res[:2]):
+                dst.copy_(src, non_blocking=True)
             s_out.wait_event(ev_done[i])
-            for dst, src in zip(B["out"], results(B)):
+            for dst, src in zip(B["out"][2:], res[2:]):
                 dst.copy_(src, non_blocking=True)
             ev_out[i].record(s_out)
 
