@@ -98,6 +98,21 @@ def test_noalloc_at_the_scratch_limit_twice():
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_noalloc_wide_clip_shaw_twice(causal):
+    """Shaw with c > 64 runs on the Transformer-XL kernels: its expanded table and zero
+    u / v vector also live in the built-in array."""
+    dev = torch.device("cuda", 0)
+    wl = Workload("shaw_wide_noalloc", SHAW, torch.bfloat16, causal, 2, 2, 300, shaw_clip=150, rel_std=1.0)
+    inp = make_inputs(wl, seed=13)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    rel = [r.to(dev) for r in inp["rel"]]
+    P = bd.Params(mech=SHAW, B=2, H=2, L=300, dtype=bd.BF16, causal=causal, scale=wl.scale, shaw_clip=150)
+    assert bd.relpos_attn_resolved_path(P, 0) == bd.PATH_TC
+    _check_twice(P, q, k, v, rel, TOL[torch.bfloat16])
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("wl", CASES, ids=[w.name for w in CASES])
 def test_noalloc_matches_regular_entry_point_twice(wl):
     dev = torch.device("cuda", 0)
