@@ -441,26 +441,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       }
       return va;
     };
-    // TXL: this thread's v.r (pre-scaled by c1), offset il of blocks Delta and Delta - 1,
-    // one key tile ahead
-    auto fetch_vr = [&](int n, float &va, float &vb) {
-      if (MECH == M_TXL) {
-        const int ra = 128 * (m - n) + il + p.off, rb = ra - 128;
-        va = (ra >= 0 && ra < p.nrows) ? A.vr[(size_t)h * p.nrows + ra] * c1 : 0.f;
-        vb = (rb >= 0 && rb < p.nrows) ? A.vr[(size_t)h * p.nrows + rb] * c1 : 0.f;
-      }
+    // TXL: v.r of the tile's two offset blocks, one value per thread tid < 256, staged in
+    // smem one tile ahead (slots 128 .. 383 of the tile's vector buffer)
+    auto fetch_vr1 = [&](int n) {
+      if (MECH != M_TXL || tid >= 256) return 0.f;
+      const int ro = 128 * (tid < 128 ? m - n : m - n - 1) + (tid & 127) + p.off;
+      return (ro >= 0 && ro < p.nrows) ? A.vr[(size_t)h * p.nrows + ro] * c1 : 0.f;
     };
-    float nva = fetch_vec(0), nvrA = 0.f, nvrB = 0.f;
-    fetch_vr(0, nvrA, nvrB);
+    float nva = fetch_vec(0);
+    if (MECH == M_TXL) {
+      if (tid < 256) vec[128 + tid] = fetch_vr1(0);
+      named_bar_sync(1, NSOFT);
+    }
     for (int n = 0; n < nTiles; ++n) {
       const int j0 = n * BN, Delta = m - n;
       float *tv = vec + 512 * (n & 1);
       if ((MECH == M_TXL && tid < 128) || (MECH == M_T5 && tid < 255) || (MECH == M_DEB && tid < 256)) tv[tid] = nva;
-      const float vrA = nvrA, vrB = nvrB;
-      if (n + 1 < nTiles) {
-        nva = fetch_vec(n + 1);
-        fetch_vr(n + 1, nvrA, nvrB);
-      }
+      const float nvr = (n + 1 < nTiles) ? fetch_vr1(n + 1) : 0.f;
+      if (n + 1 < nTiles) nva = fetch_vec(n + 1);
       // the per-tile vectors written above are read only after a later barrier of this tile
       // (Transformer-XL: the one after the skew; the other mechanisms: this one)
       if (MECH != M_TXL) named_bar_sync(1, NSOFT);
@@ -488,7 +486,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           // relation terms in key order, already c1 (T + v.r); its tcgen05.wait::ld also
           // completes the S load above
           txl_skew<ROT_LD, SK_PACKED>(tl, TM_REL + 128 * (Delta & 1), TM_REL + 128 * ((Delta - 1) & 1), hasB, g, qt, lane,
-                                      c1, vrA, vrB, rot);
+                                      c1, tv[128 + il], tv[256 + il], rot);
           tmem_wait_ld();  // when the skew had no load to wait for (no block Delta - 1 for this warp)
 #pragma unroll
           for (int t = 0; t < NC; ++t) x[t] = u2f(rs[t]);
@@ -605,6 +603,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       for (int t = 0; t < NC; t += 2) mt = fmax3(mt, x[t], x[t + 1]);
       float *rd = red + TPR * 128 * (n & 1);
       rd[128 * qt + il] = mt;
+      // the next tile's v.r into the other buffer (read last by tile n - 1's skew)
+      if (MECH == M_TXL && tid < 256 && n + 1 < nTiles) vec[512 * ((n + 1) & 1) + 128 + tid] = nvr;
       named_bar_sync(1, NSOFT);
       mt = rd[il];
 #pragma unroll
