@@ -340,7 +340,6 @@ KERNEL_CREDIT_U = {
 # removed whenever that kernel changes.
 KERNEL_TRAFFIC = {
     ("txl_causal_L8192_bf16", "tc_bwd_q_kernel"): 1133.79e6,
-    ("txl_causal_L8192_bf16", "tc_fwd_kernel"): 34.57e6,
     ("txl_causal_L8192_bf16", "tc_bwd_stream_kernel"): 1801.05e6,
 }
 # Further workloads timed by the default run (one line, sub-record "workloads"): the other
