@@ -20,9 +20,12 @@
 //                     gradient (offset-sharded, technique (3)): T5 sums dS per row on
 //                     flat tiles (one bucket per side) and per offset on band tiles
 //                     (the fp32 dS tile goes to smem and 255 threads add its diagonals
-//                     in a fixed order), then folds offsets into buckets; ALiBi sums
-//                     dS_ij |j - i| per thread.  A fixed-order reduction over batches and
-//                     query tiles finishes dt / dm.
+//                     in a fixed order), folding each band tile's 255 offset sums into
+//                     its buckets at once (a bucket's offsets are consecutive: a
+//                     segmented scan per warp, then the warps' carries), so a band of
+//                     any width needs no per-offset storage; ALiBi sums dS_ij |j - i|
+//                     per thread.  A fixed-order reduction over batches and query tiles
+//                     finishes dt / dm.
 #include <algorithm>
 #include <climits>
 #include <cstring>
@@ -38,15 +41,13 @@ namespace tcbias {
 using namespace tc;
 using namespace tcb;
 
-constexpr int MAX_BAND = 64;                     // band tiles per query tile (T5), else CUDA-core path
-constexpr int GMAX = 128 * (MAX_BAND - 1) + 256;  // per-offset sums of the band tiles of one query tile
+constexpr int NB_MAX = 64;  // T5 buckets (the boundary's limit)
 
 struct BiasArgs {
   CUtensorMap mq, mk, mv, mdo;
   Prm p;                   // nT counts 128-row tiles
   float *part;             // [B,H,nT][nb] per-query-tile partial of dt (ALiBi: dm, nb = 1)
   int flat_pos, flat_neg;  // offsets >= flat_pos (<= -flat_neg) all have one bias value
-  int bandL, bandR;        // T5: band tiles left / right of the diagonal tile
 };
 
 __device__ __forceinline__ bool flat_tile(const BiasArgs &A, int m, int n) {
@@ -314,8 +315,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_bias_kv_kernel(const __gri
 namespace qb {
 constexpr int OFF_Q = 0, OFF_DO = 16384, OFF_K = 32768, OFF_V = OFF_K + 32768;
 constexpr int OFF_T = OFF_V + 32768;     // band tiles: fp32 dS, 128 rows x 132 (also the epilogue's scratch)
-constexpr int OFF_G = OFF_T + 128 * ROT_LD * 4;  // per-offset dS sums of the band tiles (GMAX floats)
-constexpr int OFF_VEC = OFF_G + 4 * GMAX;        // bias window, double-buffered (2 x 256)
+// T5 band tiles: per-bucket dS sums of this query tile (NB_MAX floats), then each warp's
+// carry (the sum of its last run of equal buckets, that bucket, and its first bucket)
+constexpr int OFF_G = OFF_T + 128 * ROT_LD * 4;
+constexpr int OFF_GC = OFF_G + 4 * NB_MAX;
+constexpr int OFF_VEC = OFF_GC + 3 * 4 * 8;      // bias window, double-buffered (2 x 256)
 constexpr int OFF_BAR = OFF_VEC + 2048;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 enum { B_QD = 0, B_ST0, B_ST1, B_SDP, B_SDPCONS, B_PDS, B_DSFREE, B_DRAIN, NB };
@@ -348,18 +352,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_bias_q_kernel(const __grid
   volatile int *abort_flag = (volatile int *)(smem + OFF_BAR + 8 * NB + 4);
   uint32_t *tmem_slot = (uint32_t *)(smem + OFF_BAR + 8 * NB);
   float *T = (float *)(smem + OFF_T);
-  float *G = (float *)(smem + OFF_G);
+  float *G = (float *)(smem + OFF_G);  // dt partial per bucket
+  float *gc = (float *)(smem + OFF_GC);
+  int *gcb = (int *)(smem + OFF_GC + 32), *gfb = (int *)(smem + OFF_GC + 64);
   float *vec = (float *)(smem + OFF_VEC);
   int32_t *status = p.status;
   const float c1 = p.scale * LOG2E;
-  const int nG = 128 * (A.bandL + A.bandR) + 255;  // band offsets 128 (n - m) - 127 + k, n - m in [-bandL, bandR]
 
   if (tid == 0) {
     for (int k = 0; k < NB; ++k) mbar_init(BAR(k), (k == B_SDPCONS || k == B_PDS) ? NSOFT : 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  for (int x = tid; x < GMAX; x += NTHREADS) G[x] = 0.f;
+  for (int x = tid; x < NB_MAX; x += NTHREADS) G[x] = 0.f;
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
   tc_fence_before();
   __syncthreads();
@@ -522,15 +527,43 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_bias_q_kernel(const __grid
           *reinterpret_cast<float4 *>(T + il * ROT_LD + cb + 4 * c4) =
               make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
         named_bar_sync(2, NSOFT);
-        if (tid < 255) {  // local offset k - 127 = jl - il
-          float s = 0.f;
-          for (int r = 0; r < 128; ++r) {
-            const int c = r + tid - 127;
-            if (c >= 0 && c < 128) s += T[r * ROT_LD + c];
+        // warps 0-7: thread tid takes the offset j - i = 128 (n - m) - 127 + tid (tid 255: none)
+        float s = 0.f;
+        int b = -1;
+        bool last = false;  // this thread ends its bucket's run of offsets
+        if (tid < 256) {
+          const int delta = 128 * (n - m) - 127 + tid;
+          if (tid < 255 && delta > -L && delta < L) b = p.t5_bkt[delta + L - 1];
+          if (tid < 255) {
+            for (int r = 0; r < 128; ++r) {
+              const int c = r + tid - 127;
+              if (c >= 0 && c < 128) s += T[r * ROT_LD + c];
+            }
           }
-          G[128 * (n - m + A.bandL) + tid] += s;  // this offset's slot: one thread per offset per tile
+          // inclusive scan within runs of equal buckets over the warp's 32 offsets (the
+          // bucket is monotone in |j - i| on each side, so a bucket's offsets are consecutive)
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, s, o);
+            const int bb = __shfl_up_sync(0xffffffffu, b, o);
+            if (lane >= o && bb == b) s += y;
+          }
+          const int bn = __shfl_down_sync(0xffffffffu, b, 1);
+          last = lane != 31 && bn != b;
+          if (lane == 31) {
+            gc[warp] = s;
+            gcb[warp] = b;
+          }
+          if (lane == 0) gfb[warp] = b;
         }
         named_bar_sync(2, NSOFT);
+        if (tid < 256 && b >= 0) {
+          if (lane == 31) last = warp == 7 || gfb[warp + 1] != b;
+          if (last) {  // the run's parts in the warps before this one, nearest first
+            for (int w = warp - 1; w >= 0 && gfb[w + 1] == b && gcb[w] == b; --w) s += gc[w];
+            G[b] += s;  // one thread per bucket per tile
+          }
+        }
       }
     }
     // ---- epilogue: dQ ----
@@ -572,16 +605,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_bwd_bias_q_kernel(const __grid
     } else {
       const float SL = T[2 * NSOFT], SR = T[2 * NSOFT + 1];
       const int bL = p.t5_bkt[0], bR = p.t5_bkt[2 * L - 2];  // buckets of the far offsets -(L - 1), L - 1
-      for (int b = warp; b < p.nb; b += NSOFT / 32) {
-        float s = 0.f;
-        for (int k = lane; k < nG; k += 32) {
-          const int delta = k - 128 * A.bandL - 127;
-          if (delta > -L && delta < L && p.t5_bkt[delta + L - 1] == b) s += G[k];
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) part[b] = s + (b == bL ? SL : 0.f) + (b == bR ? SR : 0.f);
-      }
+      if (tid < p.nb) part[tid] = G[tid] + (tid == bL ? SL : 0.f) + (tid == bR ? SR : 0.f);
     }
     tc_fence_before();
   }
@@ -621,29 +645,20 @@ static int flat_from(const Prm &p, int sign) {
   return lo;
 }
 
-static void band_setup(const Prm &p, int nT, BiasArgs &a) {
+static void band_setup(const Prm &p, BiasArgs &a) {
   if (p.alibi) {  // ALiBi: no two offsets share a bias value, no flat tile
     a.flat_pos = a.flat_neg = INT_MAX / 4;
-    a.bandL = a.bandR = 0;
     return;
   }
   a.flat_pos = flat_from(p, 1);
   a.flat_neg = flat_from(p, -1);
-  // band tiles on a side: distances d >= 1 with 128 d - 127 < flat
-  a.bandL = std::min(nT - 1, (a.flat_neg + 254) / 128 - 1);
-  a.bandR = std::min(nT - 1, (a.flat_pos + 254) / 128 - 1);
 }
 
 }  // namespace tcbias
 
 bool tc_make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t planes, uint32_t box_rows);
 
-bool tc_bwd_bias_supported(const Prm &p) {
-  if (p.mech != M_T5) return false;
-  tcbias::BiasArgs a;
-  tcbias::band_setup(p, (p.L + 127) / 128, a);
-  return p.alibi || a.bandL + a.bandR + 1 <= tcbias::MAX_BAND;
-}
+bool tc_bwd_bias_supported(const Prm &p) { return p.mech == M_T5 && p.nb <= tcbias::NB_MAX; }
 
 cudaError_t tc_bwd_bias(const Prm &p0, cudaStream_t st) {
   using namespace tcbias;
@@ -652,7 +667,7 @@ cudaError_t tc_bwd_bias(const Prm &p0, cudaStream_t st) {
   a.p = p0;
   a.p.nT = (p0.L + 127) / 128;
   a.part = p0.part_small;
-  band_setup(p0, a.p.nT, a);
+  band_setup(p0, a);
   const uint64_t BH = (uint64_t)p0.B * p0.H;
   if (!(tc_make_map(&a.mq, p0.q, p0.L, BH, 128) && tc_make_map(&a.mk, p0.k, p0.L, BH, 128) &&
         tc_make_map(&a.mv, p0.v, p0.L, BH, 128) && tc_make_map(&a.mdo, p0.dout, p0.L, BH, 128)))

@@ -105,9 +105,8 @@ enum relpos_dtype { RELPOS_F32 = 0, RELPOS_BF16 = 1 };
  * any dtype).  Both are GPU paths; there is no CPU path.
  * bfloat16 cases that the tensor-core kernels do not cover, and that therefore run on the
  * CUDA-core kernels under RELPOS_PATH_AUTO (RELPOS_ERR_UNSUPPORTED under RELPOS_PATH_TC):
- * Shaw with the value-side table and c > 64 (both passes); the T5 backward when the tiles
- * whose buckets differ by offset span more than 64 diagonals of 128 x 128 tiles.  (DeBERTa
- * runs on the tensor cores at every span.)
+ * Shaw with the value-side table and c > 64 (both passes).  (DeBERTa runs on the tensor
+ * cores at every span, T5 at every bucket layout.)
  * Shaw without the value-side table and c > 64 runs on the Transformer-XL kernels: its
  * table is expanded to one row per offset (row i - j + off = a[clip(j - i) + c]) with
  * u = v = 0, and the expanded table's gradient is summed back into the 2c + 1 rows; the

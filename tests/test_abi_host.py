@@ -204,10 +204,9 @@ def test_t5_thresholds_match_oracle_buckets(lib):
 
 def test_resolved_paths(lib):
     """Which kernel family each pass runs (host-side dispatch, no device work): bf16
-    runs on the tensor cores except Shaw's value-side table with c > 64 and the backward of T5
-    whose buckets stay distinct over more than 64 tiles (Shaw with c > 64 and no value
-    table runs on the Transformer-XL tensor-core kernels); float32 and an explicit
-    CUDA-core request always run the CUDA-core kernels."""
+    runs on the tensor cores except Shaw's value-side table with c > 64 (Shaw with c > 64
+    and no value table runs on the Transformer-XL tensor-core kernels); float32 and an
+    explicit CUDA-core request always run the CUDA-core kernels."""
     TC, SIMT = bd.PATH_TC, bd.PATH_SIMT
     want = {  # (mech, clip) -> (forward, backward) for bf16, automatic choice
         (bd.T5, 64): (TC, TC),
@@ -226,8 +225,6 @@ def test_resolved_paths(lib):
         assert bd.relpos_attn_resolved_path(P32, 0) == SIMT and bd.relpos_attn_resolved_path(P32, 1) == SIMT
         Ps = bd.Params(mech=mech, B=1, H=2, L=300, shaw_clip=clip, kernel_path=bd.PATH_SIMT)
         assert bd.relpos_attn_resolved_path(Ps, 0) == SIMT and bd.relpos_attn_resolved_path(Ps, 1) == SIMT
-    # T5 buckets distinct out to distance 547 (max_distance 1000) span 11 tiles at L = 4096
-    # (CUDA-core backward); at L = 300 all three tiles are band tiles (tensor cores)
     # DeBERTa: every span takes the tensor-core backward
     for span, want_b in ((256, TC), (32, TC), (96, TC), (24, TC), (288, TC), (1, TC), (4096, TC)):
         assert bd.relpos_attn_resolved_path(bd.Params(mech=bd.DEBERTA, B=1, H=2, L=300, deberta_span=span), 1) == want_b, span
@@ -239,12 +236,14 @@ def test_resolved_paths(lib):
     with pytest.raises(bd.RelposError):
         bd.relpos_attn_resolved_path(bd.Params(mech=bd.SHAW, B=1, H=2, L=300, shaw_value=True, shaw_clip=65,
                                                kernel_path=bd.PATH_TC), 1)
-    # T5: the band of tiles with more than one bias value, up to 64 tiles, on the tensor cores
+    # T5: a band of tiles with more than one bias value of any width on the tensor cores
+    # (all three tiles at L = 300; about 250 band tiles at L = 32768, max_distance 20000)
     wide = dict(mech=bd.T5, B=1, H=2, t5_max_distance=1000)
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, **wide), 1) == TC
     assert bd.relpos_attn_resolved_path(bd.Params(L=300, **wide), 1) == TC
     wider = dict(mech=bd.T5, B=1, H=2, t5_max_distance=20000)
-    assert bd.relpos_attn_resolved_path(bd.Params(L=32768, **wider), 1) == SIMT
+    assert bd.relpos_attn_resolved_path(bd.Params(L=32768, **wider), 1) == TC
+    assert bd.relpos_attn_resolved_path(bd.Params(L=32768, t5_num_buckets=64, **wider), 1) == TC
     assert bd.relpos_attn_resolved_path(bd.Params(L=4096, t5_bidirectional=False, **wide), 1) == TC  # one side flat
 
 

@@ -256,9 +256,8 @@ def test_parity_t5_unidirectional_and_odd_buckets(causal):
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_parity_bias_family_tensor_core_backward(causal):
-    """T5 bucket layouts whose band of distinct-bias tiles is narrow, wide (up to the
-    eight-tile limit) or one-sided, and ALiBi slopes from nearly flat to sharply local,
-    on the bf16 tensor-core backward."""
+    """T5 bucket layouts whose band of distinct-bias tiles is narrow, wide or one-sided,
+    and ALiBi slopes from nearly flat to sharply local, on the bf16 tensor-core backward."""
     for nb, md, bidir in ((32, 128, True), (10, 40, True), (7, 20, False), (32, 600, True), (64, 900, False)):
         wl = Workload("t5x", T5, torch.bfloat16, causal, 1, 2, 1100, t5_num_buckets=nb, t5_max_distance=md,
                       t5_bidirectional=bidir)
@@ -266,7 +265,7 @@ def test_parity_bias_family_tensor_core_backward(causal):
         assert bd.relpos_attn_resolved_path(P, 1) == bd.PATH_TC, (nb, md, bidir)
         inp = make_inputs(wl, nb)
         compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
-    # a band of distinct-bias tiles far wider than eight (max_distance 3000: about 47 tiles)
+    # a wide band of distinct-bias tiles (max_distance 3000: about 47 tiles)
     wl = Workload("t5_wide", T5, torch.bfloat16, causal, 1, 2, 3500, t5_num_buckets=32, t5_max_distance=3000)
     assert bd.relpos_attn_resolved_path(params_of(wl, bd.PATH_AUTO), 1) == bd.PATH_TC
     inp = make_inputs(wl, 11)
@@ -275,6 +274,19 @@ def test_parity_bias_family_tensor_core_backward(causal):
     inp = make_inputs(wl, 3)
     inp["rel"] = [torch.tensor([1e-4, 0.02, 1.0, 8.0])]
     compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_parity_t5_band_of_89_tiles_L8192(causal):
+    """T5 buckets that stay distinct across most of an 8K sequence (64 buckets,
+    max_distance 8192: 63 buckets in use, a band of 89 distinct-bias tiles around each
+    query tile) on the tensor-core backward, which folds each band tile's offset sums
+    into buckets as it goes; every output of head 0 (its table gradient is exact with one
+    batch) against the oracle."""
+    wl = Workload("t5_band89", T5, torch.bfloat16, causal, 1, 2, 8192, t5_num_buckets=64, t5_max_distance=8192)
+    assert bd.relpos_attn_resolved_path(params_of(wl, bd.PATH_AUTO), 1) == bd.PATH_TC
+    inp = make_inputs(wl, 13)
+    compare_full(wl, inp, run_gpu(wl, inp, bd.PATH_AUTO), heads=slice(0, 1))
 
 
 def test_t5_small_buckets_and_fp32_config():
