@@ -89,27 +89,32 @@ def fa_flops(wl):
 def kernel_launches(wl, path):
     """Kernels this library launches per forward and per backward call (the dispatch of csrc/api.cu)."""
     t5 = 1 if wl.mech in (T5, ALIBI) else 0  # per-call per-offset bias preparation
-    tc = path != "simt" and wl.dtype == torch.bfloat16
-    tc_bwd = tc and not (wl.mech == SHAW and wl.shaw_clip > 64)  # wider Shaw clips: CUDA-core backward
-    if tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
+    # bf16 runs on the tensor cores except Shaw's value-side table with c > 64
+    tc = path != "simt" and wl.dtype == torch.bfloat16 and not (wl.mech == SHAW and wl.shaw_value and wl.shaw_clip > 64)
+    wide = tc and wl.mech == SHAW and wl.shaw_clip > 64  # the Transformer-XL kernels over the clip-expanded table
+    if wide:  # table expansion, relation prep, the forward kernel
+        fwd = 3
+    elif tc:  # tensor-core forward: relation prep (TXL, DeBERTa) + the forward kernel
         fwd = 1 + t5 + (1 if wl.mech in (TXL, DEBERTA) else 0)
     else:
         fwd = 1 + t5
-    if tc_bwd and wl.mech == TXL:
+    if tc and (wl.mech == TXL or wide):
         nt = (wl.L + wl.mem_len + 127) // 128
         tiles = wl.B * wl.H * (nt * (nt + 1) // 2 if wl.causal else nt * nt)
         # stored P / dS tiles (up to 32 GiB): D, relation prep, query-tile, one launch of both
-        # streaming roles, dr and u/v reductions; else key-tile, query-tile and diagonal kernels
-        bwd = 6 if tiles * 65536 <= 32 << 30 else 7
-    elif tc_bwd and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction; the value
+        # streaming roles, dr and u/v reductions; else key-tile, query-tile and diagonal kernels;
+        # the wide Shaw route adds the table expansion and the collapse of its gradient
+        bwd = (6 if tiles * 65536 <= 32 << 30 else 7) + (2 if wide else 0)
+    elif tc and wl.mech == SHAW:  # D, per-row q.a products, key-tile, query-tile, da reduction; the value
         bwd = 7 if wl.shaw_value else 5  # side adds the dO.aV products and the daV reduction
-    elif tc_bwd and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
+    elif tc and wl.mech in (T5, ALIBI):  # bias vector, D, key-tile, query-tile, bucket / slope reduction
         bwd = 5
-    elif tc_bwd and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction
+    elif tc and wl.mech == DEBERTA:  # D, relation products, key-tile, query-tile, rows GEMM, table GEMM, reduction
         bwd = 7
     else:  # D, key-tile, query-tile, then the table-gradient reductions (Shaw's value side: one more)
         bwd = 3 + t5 + {T5: 1, SHAW: 1, TXL: 3, DEBERTA: 2, ALIBI: 1}[wl.mech] + (1 if wl.shaw_value else 0)
-    return fwd, bwd
+    # Transformer-XL memory: the backward fills the placeholder rows' LSE (+inf)
+    return fwd, bwd + (1 if wl.mem_len > 0 else 0)
 
 
 def median_iqr(xs):

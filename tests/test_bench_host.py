@@ -76,6 +76,21 @@ def test_kernel_launch_counts_of_the_default_workload():
     assert bench.kernel_launches(WORKLOADS["txl_L32768_bf16"].with_(H=9), "auto") == (2, 7)
 
 
+def test_kernel_launch_counts_of_the_other_routes():
+    """Transformer-XL memory adds the backward's LSE fill of the placeholder rows; Shaw
+    with c > 64 runs the Transformer-XL kernels with the table expansion (both passes)
+    and the gradient's collapse; with its value-side table and c > 64 it runs the CUDA-core
+    kernels; T5 takes the tensor cores at any band width."""
+    assert bench.kernel_launches(WORKLOADS["txl_mem_M4096_L4096_bf16"], "auto") == (2, 7)
+    shaw = WORKLOADS["shaw_L2048_bf16"]
+    assert bench.kernel_launches(shaw, "auto") == (1, 5)
+    assert bench.kernel_launches(shaw.with_(shaw_clip=100), "auto") == (3, 8)
+    assert bench.kernel_launches(shaw.with_(shaw_clip=100, shaw_value=True), "auto") == (1, 5)
+    assert bench.kernel_launches(shaw.with_(shaw_value=True), "auto") == (1, 7)
+    t5 = WORKLOADS["t5_causal_L8192_bf16"]
+    assert bench.kernel_launches(t5.with_(t5_max_distance=8192, t5_num_buckets=64), "auto") == (2, 5)
+
+
 def test_txl_backward_credit_splits_8U():
     """The Transformer-XL backward's algorithmic 8U, split over the kernels of each
     variant: query-tile 5U with the streaming launch (3U) or the recomputing key-tile and
