@@ -1,7 +1,7 @@
 // Inline-PTX wrappers for the sm_100a tensor-core path: mbarriers with bounded
 // waits, TMA tile loads, TMEM allocation, tcgen05.mma / commit / ld / st and the
-// shared-memory matrix descriptors.  Only per-CTA TMA loads are used (no
-// cluster multicast anywhere).
+// shared-memory matrix descriptors.  Every TMA load is issued by one CTA for its
+// own shared memory, from this GPU's memory.
 #pragma once
 
 #include <cuda.h>
