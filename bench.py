@@ -346,7 +346,6 @@ KERNEL_CREDIT_U = {
 KERNEL_TRAFFIC = {
     ("txl_causal_L8192_bf16", "tc_fwd_kernel"): 34.50e6,
     ("txl_causal_L8192_bf16", "tc_bwd_q_kernel"): 1137.51e6,
-    ("txl_causal_L8192_bf16", "tc_bwd_stream_kernel"): 1803.87e6,
 }
 # Further workloads timed by the default run (one line, sub-record "workloads"): the other
 # configuration quoted at L = 8192 (DeBERTa), the Shaw configuration, and one point of the
